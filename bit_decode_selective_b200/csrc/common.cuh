@@ -1,0 +1,76 @@
+// common.cuh -- host-side error plumbing and small device helpers shared by the
+// CUDA translation units of the library.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "../../include/sf.h"
+
+namespace sf {
+
+// ---- host: thread-local error message -------------------------------------
+
+void set_error(const char* fmt, ...);
+void clear_error();
+
+#define SF_REQUIRE(cond, ...)                  \
+  do {                                         \
+    if (!(cond)) {                             \
+      ::sf::set_error(__VA_ARGS__);            \
+      return SF_ERR_INVALID_ARG;               \
+    }                                          \
+  } while (0)
+
+#define SF_UNSUPPORTED(cond, ...)              \
+  do {                                         \
+    if (!(cond)) {                             \
+      ::sf::set_error(__VA_ARGS__);            \
+      return SF_ERR_UNSUPPORTED;               \
+    }                                          \
+  } while (0)
+
+// Check the last launch (or a runtime call) and turn a failure into SF_ERR_CUDA.
+#define SF_CUDA(call)                                                           \
+  do {                                                                          \
+    cudaError_t e_ = (call);                                                    \
+    if (e_ != cudaSuccess) {                                                    \
+      ::sf::set_error("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),   \
+                      __FILE__, __LINE__);                                      \
+      return SF_ERR_CUDA;                                                       \
+    }                                                                           \
+  } while (0)
+
+#define SF_LAUNCHED() SF_CUDA(cudaGetLastError())
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(sf_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int num_sms();  // multiprocessors of the current device (cached per device)
+
+// Host-side validation of the descriptor structs (pack.cu).
+sf_status check_kv(const sf_kv* kv);
+sf_status check_wq_public(const sf_wq* w, bool need_refine);
+
+// ---- device helpers ---------------------------------------------------------
+
+__device__ __forceinline__ double h2d(uint16_t h) {
+  return (double)__half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue now / wait until the previous kernel's results are visible.  Both
+// are no-ops when the launch carried no programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+}  // namespace sf

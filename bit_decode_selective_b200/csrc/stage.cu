@@ -1,0 +1,98 @@
+// stage.cu -- staging of selected refinement rows from pinned host memory.
+//
+// "StrataFlux -- Selective precision streaming -- What does it mean?": on a
+// machine with a dedicated GPU the refinement bits live in host RAM; only the
+// rows of the selected channels cross the link, and fetch lead starts that
+// transfer one or more layers early, from an earlier activation, so it
+// overlaps the projections in between.
+//
+// sf_stage_refinements gathers the rows named by a DEVICE index array straight
+// from mapped pinned host memory (the GPU issues the PCIe reads itself), so a
+// selection made on the GPU needs no round trip through the host and the copy
+// can be captured in a CUDA graph.  sf_stage_refinements_host is the plain
+// variant for indices known on the host: one cudaMemcpyAsync per run of
+// consecutive rows.
+#include "common.cuh"
+
+namespace sf {
+namespace {
+
+constexpr int kVec = 4;  // 16-byte words in flight per thread
+
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
+                                                          size_t row_vecs,
+                                                          const int32_t* __restrict__ sel,
+                                                          int n_sel, uint4* __restrict__ dst) {
+  const size_t total = (size_t)n_sel * row_vecs;
+  const size_t stride = (size_t)gridDim.x * blockDim.x * kVec;
+  for (size_t base = ((size_t)blockIdx.x * blockDim.x) * kVec + threadIdx.x; base < total;
+       base += stride) {
+    uint4 v[kVec];
+#pragma unroll
+    for (int u = 0; u < kVec; u++) {
+      size_t i = base + (size_t)u * blockDim.x;
+      if (i < total) {
+        size_t j = i / row_vecs, c = i % row_vecs;
+        v[u] = src[(size_t)sel[j] * row_vecs + c];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kVec; u++) {
+      size_t i = base + (size_t)u * blockDim.x;
+      if (i < total) dst[i] = v[u];
+    }
+  }
+}
+
+}  // namespace
+}  // namespace sf
+
+using namespace sf;
+
+extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes,
+                                          const int32_t* sel, int n_sel, void* dst,
+                                          sf_stream_t stream, sf_event_t done) {
+  SF_REQUIRE(host_rows && dst && sel, "host_rows, sel and dst must be non-null");
+  SF_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "row_bytes=%zu must be a multiple of 16",
+             row_bytes);
+  SF_REQUIRE(aligned16(host_rows) && aligned16(dst) && aligned16(sel),
+             "host_rows, sel and dst must be 16-byte aligned");
+  SF_REQUIRE(n_sel >= 0, "n_sel=%d < 0", n_sel);
+  cudaPointerAttributes attr;
+  SF_CUDA(cudaPointerGetAttributes(&attr, host_rows));
+  SF_REQUIRE(attr.type == cudaMemoryTypeHost && attr.devicePointer != nullptr,
+             "host_rows must be page-locked host memory mapped into the device address space");
+  cudaStream_t s = as_stream(stream);
+  if (n_sel > 0) {
+    size_t vecs = (size_t)n_sel * (row_bytes / 16);
+    long blocks = (long)((vecs + 256 * kVec - 1) / (256 * kVec));
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4*)attr.devicePointer,
+                                                        row_bytes / 16, sel, n_sel, (uint4*)dst);
+    SF_LAUNCHED();
+  }
+  if (done) SF_CUDA(cudaEventRecord((cudaEvent_t)done, s));
+  return SF_OK;
+}
+
+extern "C" sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes,
+                                               const int32_t* sel_host, int n_sel, void* dst,
+                                               sf_stream_t stream, sf_event_t done) {
+  SF_REQUIRE(host_rows && dst && (sel_host || n_sel == 0), "null argument");
+  SF_REQUIRE(row_bytes > 0, "row_bytes must be positive");
+  SF_REQUIRE(n_sel >= 0, "n_sel=%d < 0", n_sel);
+  cudaStream_t s = as_stream(stream);
+  const char* src = (const char*)host_rows;
+  char* out = (char*)dst;
+  int j = 0;
+  while (j < n_sel) {
+    int run = 1;
+    while (j + run < n_sel && sel_host[j + run] == sel_host[j] + run) run++;
+    SF_REQUIRE(sel_host[j] >= 0, "negative row index %d", sel_host[j]);
+    SF_CUDA(cudaMemcpyAsync(out + (size_t)j * row_bytes, src + (size_t)sel_host[j] * row_bytes,
+                            (size_t)run * row_bytes, cudaMemcpyHostToDevice, s));
+    j += run;
+  }
+  if (done) SF_CUDA(cudaEventRecord((cudaEvent_t)done, s));
+  return SF_OK;
+}

@@ -1,0 +1,251 @@
+/*
+ * sf.h -- C ABI of the selective-precision (nested refinement) decode path.
+ *
+ * The operations follow the StrataFlux pages, cited by title and paragraph:
+ *   [EXPL] "StrataFlux -- Selective precision streaming -- What does it mean?"
+ *          - "nested quantization": fetched bits subdivide the bin the resident
+ *            code already names (a 2-bit code + 2 fetched bits = 4-bit
+ *            resolution);
+ *          - "which tiles count": weights refine the k input channels with the
+ *            largest |activation| in each chunk of 1,024 channels; the KV cache
+ *            scores every cached token by the attention it receives from the
+ *            resident low-bit keys and refines the highest-scoring tokens per
+ *            KV head; everything not selected still takes part at low
+ *            precision;
+ *          - "the map app also loads tiles": refinements are fetched early
+ *            (fetch lead) and applied late (fetch lag), overlapping transfers
+ *            with compute;
+ *          - "where it earns its keep": KV refinement is a step that cannot
+ *            overlap the attention around it, because the selection depends on
+ *            the attention scores.
+ *   [ABS]  "StrataFlux: Memory-Hierarchy-Native Low-Bit LLM Inference",
+ *          abstract: 2-4-bit weights and 2-3-bit KV caches.
+ *
+ * Conventions
+ *   - Every pointer is a DEVICE pointer unless its comment says "host".
+ *   - All memory is owned and allocated by the caller.  No entry point
+ *     allocates device memory.  Scratch space is passed as (ws, ws_bytes); the
+ *     matching *_workspace_bytes() function gives the size needed.
+ *   - Every entry point that takes a stream only enqueues work on it and
+ *     returns without waiting for the device.  Arguments are validated on the
+ *     host before anything is enqueued; on a validation error nothing is
+ *     enqueued.
+ *   - fp16 values are IEEE binary16 bit patterns in uint16_t.
+ *   - Errors are returned as sf_status; sf_last_error() gives a message for
+ *     the calling thread's most recent failure.  The library never aborts,
+ *     prints, traps or asserts on the device.
+ *   - Device pointers must be 16-byte aligned.
+ *
+ * Quantisation (shared by weights and KV), for one group of values w:
+ *   s = fp16((max w - min w) / (2^b - 1)),  m = fp16(min w)   (one rounding each)
+ *   u = (w - m) / s,  Q = clamp(floor((u + 1/2) * 2^r), 0, 2^(b+r) - 1)
+ *   base code q = Q >> r,  refinement code rho = Q & (2^r - 1)
+ *   base value    = m + s * q
+ *   refined value = m + s * (q + (2*rho + 1 - 2^r) / 2^(r+1))
+ * (all in fp64, one rounding per operation; a group whose s is 0 gets all
+ * codes 0).  q alone is the ordinary b-bit round-to-nearest code; q and rho
+ * together are the (b+r)-bit round-to-nearest code on the grid with step
+ * s/2^r and offset m + s(1 - 2^r)/2^(r+1).
+ *
+ * "Natural w-bit stream": element e sits at bit w*e of a little-endian byte
+ * string (byte (w*e)/8, bit offset (w*e)%8).
+ */
+#ifndef SF_H_
+#define SF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SF_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SF_API __attribute__((visibility("default")))
+#else
+#define SF_API
+#endif
+
+typedef struct CUstream_st* sf_stream_t; /* same type as cudaStream_t */
+typedef struct CUevent_st* sf_event_t;   /* same type as cudaEvent_t */
+
+typedef enum {
+  SF_OK = 0,
+  SF_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or range      */
+  SF_ERR_UNSUPPORTED = 2, /* valid request this build does not implement     */
+  SF_ERR_CUDA = 3,        /* a CUDA call or launch failed (see sf_last_error) */
+  SF_ERR_TIMEOUT = 4,     /* a bounded host-side wait ran out                */
+  SF_ERR_WORKSPACE = 5    /* ws too small (or NULL with ws_bytes needed > 0) */
+} sf_status;
+
+SF_API int sf_abi_version(void);
+SF_API const char* sf_status_string(sf_status st);
+/* Message of the calling thread's last failure ("" if none).  The pointer
+ * stays valid until the thread's next failing call. */
+SF_API const char* sf_last_error(void);
+
+/* ======================================================================== */
+/* Weights                                                                   */
+/* ======================================================================== */
+
+/* A quantised weight matrix W[n][k] (n output rows, k input channels), in
+ * groups of `group` consecutive input channels of one row.
+ *   b in {2,3,4}, r in {1,2}, group in {32,64,128,256}, k % 1024 == 0 and
+ *   k % group == 0, n % 128 == 0.
+ * base (n*k*b/8 bytes):
+ *   b = 2, 4 : one natural b-bit stream of the k codes per row, rows in order.
+ *   b = 3    : plane L = the low 2 bits of every code, a natural 2-bit stream
+ *              per row (n*k/4 bytes), then plane H = the high bit (n*k/8
+ *              bytes): per row, per block of 32 channels, one little-endian
+ *              32-bit word in which channel c (0..31 within the block) sits at
+ *              bit 8*(c/4) + c%4 for c < 16 and at bit 8*((c-16)/4) + 4 +
+ *              (c-16)%4 for c >= 16.
+ * refine (k*n*r/8 bytes): channel-major, one natural r-bit stream of the n
+ *   refinement codes of each input channel ("one contiguous run per channel",
+ *   so a selected channel's refinement is one row); may be NULL when
+ *   refinements only ever arrive as staged rows.
+ * sz (n * k/group * 2 fp16): (s, m) of row i's group j at sz[(i*(k/group)+j)*2]. */
+typedef struct {
+  int32_t n, k, b, r, group;
+  void* base;
+  void* refine;
+  uint16_t* sz;
+} sf_wq;
+
+/* Byte sizes of the three buffers of an sf_wq; any out pointer may be NULL. */
+SF_API sf_status sf_wq_bytes(int n, int k, int b, int r, int group, size_t* base_bytes,
+                      size_t* refine_bytes, size_t* sz_bytes);
+
+/* Quantise w[n][k] (fp32, device) into the buffers of *out (nested
+ * quantisation above, [EXPL] "nested quantization").  Bit-exact with the
+ * definition: the fp64 decisions are made with IEEE operations and no
+ * contraction.  out->refine must be non-NULL. */
+SF_API sf_status sf_pack_nested(const float* w, const sf_wq* out, sf_stream_t stream);
+
+/* Inverse of the packing, for checking: qb[n][k] and rho[n][k] (one code per
+ * byte).  rho may be NULL (or out->refine NULL: rho is then not written). */
+SF_API sf_status sf_unpack_codes(const sf_wq* w, uint8_t* qb, uint8_t* rho, sf_stream_t stream);
+
+/* Chunked channel selection ([EXPL] "which tiles count"): for every batch row
+ * and every chunk of `chunk` input channels, the kch channels with the
+ * largest fp16 magnitude |x| (bits & 0x7fff; +0 == -0), equal magnitudes to
+ * the lower index, written as absolute channel indices in ascending order.
+ *   x   [batch][k] fp16;  sel [batch][k/chunk][kch] int32.
+ *   1 <= batch <= 64, k % chunk == 0, chunk in {256, 512, 1024, 2048},
+ *   1 <= kch <= chunk. */
+SF_API sf_status sf_select_channels(const uint16_t* x, int batch, int k, int chunk, int kch,
+                             int32_t* sel, sf_stream_t stream);
+
+/* Refined GEMV ([EXPL] "which tiles count"):
+ *   y[b][i] = sum_c x[b][c] * w~[i][c],
+ * where w~ is the refined value for the channels selected for batch row b and
+ * the base value for every other channel.  Accumulation is fp32.
+ *   x [batch][k] fp16, y [batch][n] fp32, 1 <= batch <= 8.
+ *   kch = 0: base only (sel_in, sel_out, refine_rows ignored).
+ *   sel_in (nullable): a selection made earlier ([batch][k/chunk][kch],
+ *     ascending per chunk), e.g. from the previous layer's activation (fetch
+ *     lead).  NULL: the call selects from x itself and writes sel_out.
+ *   sel_out (nullable when sel_in is given): receives the selection used.
+ *   refine_rows (nullable): staged refinement rows [batch][k/chunk*kch][n*r/8];
+ *     row j of batch row b holds the refinement of channel sel[b][j]
+ *     (flattened over chunks).  NULL: rows are read from w->refine.
+ *   ws/ws_bytes: sf_gemv_workspace_bytes(); currently 0 (ws may be NULL). */
+SF_API sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
+                          const int32_t* sel_in, int32_t* sel_out, const void* refine_rows,
+                          float* y, void* ws, size_t ws_bytes, sf_stream_t stream);
+SF_API size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch);
+
+/* ======================================================================== */
+/* KV cache                                                                  */
+/* ======================================================================== */
+
+/* `batch` independent caches of h_kv heads with room for t_max tokens of d
+ * elements, quantised per token in groups of `group` consecutive elements.
+ *   d == 128, group == 32, b in {2,4}, r in {1,2}, t_max % 16 == 0.
+ * kb, vb: [batch][h_kv][t_max] tokens, each a natural b-bit stream of its d
+ *   codes (d*b/8 bytes).
+ * kr, vr: same with the r-bit refinement codes (d*r/8 bytes per token).
+ * ksz, vsz: [batch][h_kv][t_max][d/group][2] fp16 (s, m). */
+typedef struct {
+  int32_t batch, h_kv, d, t_max, b, r, group;
+  void *kb, *kr, *vb, *vr;
+  uint16_t *ksz, *vsz;
+} sf_kv;
+
+SF_API sf_status sf_kv_bytes(int batch, int h_kv, int d, int t_max, int b, int r, int group,
+                      size_t* code_bytes, size_t* refine_bytes, size_t* sz_bytes);
+
+/* Quantise and store tokens t0 .. t0+nt-1 of every head (nested quantisation
+ * applied to the KV cache, [EXPL] "nested quantization").
+ *   k, v: [batch][h_kv][nt][d] fp16 (either may be NULL to skip it). */
+SF_API sf_status sf_kv_pack_tokens(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0,
+                            int nt, sf_stream_t stream);
+
+/* Codes of tokens 0..t-1, for checking: which = 0 keys, 1 values;
+ * qb, rho: [batch][h_kv][t][d] (rho nullable). */
+SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* qb, uint8_t* rho,
+                             sf_stream_t stream);
+
+/* Token scoring and selection ([EXPL] "which tiles count"):
+ *   logit[h][t] = q[h] . k^_base[h / (h_q/h_kv)][t] / sqrt(d)
+ *   score[g][t] = sum over the query heads h of KV head g of
+ *                 exp(logit[h][t] - max_t logit[h]) / sum_t exp(...)
+ *   sel[g] = the k_tok tokens with the highest score (equal scores: lower
+ *            token first), ascending.
+ *   q [batch][h_q][d] fp16;  sel [batch][h_kv][k_tok] int32.
+ *   logits (nullable): receives the base logits [batch][h_q][t] fp32; pass the
+ *     same buffer to sf_kv_attn_refined so it need not re-read the keys.
+ *   scores (nullable): receives score [batch][h_kv][t] fp32.
+ *   1 <= t <= t_max, 1 <= k_tok <= min(t, 4096), h_q % h_kv == 0,
+ *   h_q / h_kv <= 8. */
+SF_API sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok,
+                             int32_t* sel, float* logits, float* scores, void* ws,
+                             size_t ws_bytes, sf_stream_t stream);
+SF_API size_t sf_kv_score_select_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
+                                          int logits_given);
+
+/* Refined attention ([EXPL] "which tiles count", "nested quantization"):
+ *   out[h] = sum_t softmax_t(q[h] . k~[t] / sqrt(d)) v~[t]
+ * over all t tokens, where k~, v~ are the refined values for the tokens in
+ * sel[g] (g the KV head of h) and the base values for every other token.
+ * The context is split into n_splits parts (0: automatic) whose partial
+ * (max, sum, weighted values) are merged by log-sum-exp; the result does not
+ * depend on the split count beyond fp32 rounding.
+ *   sel [batch][h_kv][k_tok] ascending (k_tok may be 0: base attention);
+ *   base_logits (nullable): the logits written by sf_kv_score_select for the
+ *     same q, cache and t; unselected tokens then use them instead of
+ *     re-reading their keys;
+ *   out [batch][h_q][d] fp32. */
+SF_API sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                             const int32_t* sel, int k_tok, const float* base_logits,
+                             int n_splits, float* out, void* ws, size_t ws_bytes,
+                             sf_stream_t stream);
+SF_API size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int n_splits);
+
+/* ======================================================================== */
+/* Refinement staging ([EXPL] "the map app also loads tiles": fetch lead)    */
+/* ======================================================================== */
+
+/* Copy the rows host_rows[sel[j]] (j < n_sel, each row_bytes long) into
+ * dst[j] on `stream`, reading pinned host memory directly from the GPU, and
+ * record `done` (nullable) on `stream` after the copy.  sel is a DEVICE array
+ * (a selection made on the GPU, e.g. by sf_select_channels one layer early),
+ * so no host round trip is needed.  host_rows must be page-locked host memory
+ * mapped into the device address space (cudaHostAlloc with
+ * cudaHostAllocMapped, or cudaHostRegister with cudaHostRegisterMapped);
+ * row_bytes % 16 == 0. */
+SF_API sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, const int32_t* sel,
+                               int n_sel, void* dst, sf_stream_t stream, sf_event_t done);
+
+/* Same copy with a HOST index array: one cudaMemcpyAsync per run of
+ * consecutive indices.  host_rows must be pinned. */
+SF_API sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes,
+                                    const int32_t* sel_host, int n_sel, void* dst,
+                                    sf_stream_t stream, sf_event_t done);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SF_H_ */

@@ -1,0 +1,76 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/sf.h declares, and rejects bad arguments on the host
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_decode_selective_b200 import abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sf.h")).read()
+    return set(re.findall(r"^SF_API\s+[\w\s\*]+?\b(sf_\w+)\s*\(", text, flags=re.M))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_decode_selective_b200.build import build_library
+
+    build_library()
+    return abi.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert len(names) >= 18
+    for name in names:
+        assert hasattr(L, name), name
+    assert names == set(abi.EXPORTED)
+
+
+def test_version_and_status_strings(L):
+    assert abi.sf_abi_version() == 1
+    assert abi.sf_status_string(0) == b"ok"
+    assert abi.sf_status_string(abi.SF_ERR_WORKSPACE) == b"workspace too small"
+
+
+def test_byte_sizes(L):
+    s = [ctypes.c_size_t() for _ in range(3)]
+    assert abi.sf_wq_bytes(4096, 4096, 2, 2, 128, *[ctypes.byref(x) for x in s]) == 0
+    assert [x.value for x in s] == [4096 * 4096 // 4, 4096 * 4096 // 4, 4096 * 32 * 4]
+    assert abi.sf_wq_bytes(4096, 4096, 5, 2, 128, *[ctypes.byref(x) for x in s]) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_kv_bytes(1, 8, 128, 8192, 2, 2, 32, *[ctypes.byref(x) for x in s]) == 0
+    assert [x.value for x in s] == [8 * 8192 * 32, 8 * 8192 * 32, 8 * 8192 * 16]
+
+
+def test_validation_rejects_before_launch(L):
+    # null pointers / unsupported shapes are refused on the host
+    wq = abi.sf_wq(4096, 4096, 2, 2, 128, None, None, None)
+    assert abi.sf_pack_nested(None, ctypes.byref(wq), None) == abi.SF_ERR_INVALID_ARG
+    assert b"base" in abi.sf_last_error()
+    wq = abi.sf_wq(4096, 4000, 2, 2, 128, 16, 16, 16)
+    assert abi.sf_pack_nested(ctypes.c_void_p(16), ctypes.byref(wq), None) == abi.SF_ERR_UNSUPPORTED
+    wq = abi.sf_wq(4096, 4096, 2, 2, 128, 17, 16, 16)  # misaligned
+    assert abi.sf_pack_nested(ctypes.c_void_p(16), ctypes.byref(wq), None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_select_channels(None, 1, 4096, 1024, 32, None, None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_select_channels(ctypes.c_void_p(16), 1, 4096, 1000, 32, ctypes.c_void_p(16), None) \
+        == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_select_channels(ctypes.c_void_p(16), 1, 4096, 1024, 0, ctypes.c_void_p(16), None) \
+        == abi.SF_ERR_INVALID_ARG
+    kv = abi.sf_kv(1, 8, 128, 8192, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    # k_tok > t
+    assert abi.sf_kv_score_select(ctypes.byref(kv), 10, ctypes.c_void_p(16), 32, 11, ctypes.c_void_p(16),
+                                  None, None, None, 0, None) == abi.SF_ERR_INVALID_ARG
+    # 3-bit KV is not built
+    kv3 = abi.sf_kv(1, 8, 128, 8192, 3, 2, 32, 16, 16, 16, 16, 16, 16)
+    assert abi.sf_kv_pack_tokens(ctypes.byref(kv3), ctypes.c_void_p(16), None, 0, 1, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    # too little workspace is reported, not overrun
+    assert abi.sf_kv_attn_refined(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, None, 0, None, 4,
+                                  ctypes.c_void_p(16), ctypes.c_void_p(16), 8, None) == abi.SF_ERR_WORKSPACE
+    assert abi.sf_stage_refinements_host(None, 16, None, 1, None, None, None) == abi.SF_ERR_INVALID_ARG

@@ -1,0 +1,275 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bar (from the method's pass criteria): packed bytes, codes and channel indices
+bit-exact; KV token sets equal except tokens whose oracle score is within 1e-5
+(relative) of the k-th score; outputs within relative L2 1e-3, attention also
+within max-abs 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_decode_selective_b200 import inputs
+from bit_decode_selective_b200.ops import KVCache, QuantWeights, select_channels
+
+pytestmark = pytest.mark.gpu
+
+RTOL_L2 = 1e-3
+ATTN_MAX_ABS = 2e-3
+SEL_RTOL = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def dev():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    oracle.set_threads(0)
+    return torch.device("cuda")
+
+
+def cu(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def f16bits(x):
+    return np.ascontiguousarray(x).view(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# weight packing
+
+
+def special_weights(rng, n, k):
+    w = inputs.weight(rng, n, k)
+    w[0, :128] = 0.25                      # constant group: step 0
+    w[1, :64] = 0.0
+    w[1, 64:128] = -0.0                    # signed zeros
+    w[2, 128:256] = rng.normal(0, 30, 128)  # wide range
+    w[3, :128] = np.linspace(-1, 1, 128)   # many exact bin edges
+    return w
+
+
+def check_packed(qw, w, b, r, G):
+    qb, rho, sz = oracle.quant_weights(w, b, r, G)
+    base, refine = oracle.pack_weights(qb, rho, b, r)
+    gq, grho = qw.unpack()
+    torch.cuda.synchronize()
+    assert np.array_equal(host(qw.sz).view(np.uint16).reshape(sz.shape), sz)
+    assert np.array_equal(host(gq), qb)
+    assert np.array_equal(host(grho), rho)
+    assert np.array_equal(host(qw.base), base)
+    assert np.array_equal(host(qw.refine), refine)
+    return qb, rho, sz
+
+
+@pytest.mark.parametrize("b,r,G", [(2, 2, 128), (2, 1, 64), (3, 1, 128), (3, 2, 32), (4, 2, 128), (4, 1, 256)])
+def test_pack_weights_bit_exact(b, r, G):
+    rng = np.random.default_rng(100 + 10 * b + r)
+    w = special_weights(rng, 256, 2048)
+    qw = QuantWeights.pack(cu(w), b, r, G)
+    check_packed(qw, w, b, r, G)
+
+
+def test_pack_weights_gemv_workload_full_size():
+    w, _ = inputs.gemv_case(seed=0)
+    qw = QuantWeights.pack(cu(w), 2, 2, 128)
+    check_packed(qw, w, 2, 2, 128)
+
+
+# ---------------------------------------------------------------------------
+# channel selection
+
+
+@pytest.mark.parametrize("chunk,kch", [(1024, 32), (1024, 1), (1024, 1024), (256, 7), (2048, 100), (512, 512)])
+def test_select_channels_bit_exact(chunk, kch):
+    rng = np.random.default_rng(chunk + kch)
+    x = inputs.activation(rng, 4096, batch=3)
+    x[0, ::9] = np.float16(1.5)      # ties of both signs
+    x[0, 1::13] = np.float16(-1.5)
+    x[1, :50] = np.float16(0.0)
+    x[1, 50:80] = np.float16(-0.0)
+    x[2, :] = np.float16(2.0)        # a row of equal magnitudes
+    sel = select_channels(cu(f16bits(x)), chunk, kch)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(sel), oracle.select_chunks(x, chunk, kch))
+
+
+# ---------------------------------------------------------------------------
+# refined GEMV
+
+
+def gemv_check(w, x, b, r, G, chunk, kch, staged=False, give_sel=False):
+    qb, rho, sz = oracle.quant_weights(w, b, r, G)
+    qw = QuantWeights.pack(cu(w), b, r, G)
+    xd = cu(f16bits(x))
+    sel_o = oracle.select_chunks(x, chunk, kch) if kch else None
+    if staged or give_sel:
+        sel_d = cu(sel_o)
+        rows = qw.refine_rows()[sel_d.view(x.shape[0], -1).long()].contiguous() if staged else None
+        y, sel = qw.gemv(xd, chunk, kch, sel_in=sel_d, refine_rows=rows)
+    else:
+        y, sel = qw.gemv(xd, chunk, kch)
+    torch.cuda.synchronize()
+    if kch:
+        assert np.array_equal(host(sel), sel_o)
+    yo = oracle.gemv_refined(qb, rho, sz, r, G, x, sel_o, chunk, kch)
+    err = rel_l2(host(y), yo)
+    assert err <= RTOL_L2, err
+    return err
+
+
+@pytest.mark.parametrize("b,r", [(2, 2), (2, 1), (3, 1), (3, 2), (4, 2)])
+@pytest.mark.parametrize("kch", [0, 32, 1024])
+def test_gemv_parity(b, r, kch):
+    rng = np.random.default_rng(7 * b + r + kch)
+    # k = 3072: one full 2048-channel segment plus a half one (ragged lane tail)
+    w = inputs.weight(rng, 384, 3072)
+    x = inputs.activation(rng, 3072, batch=1)
+    err = gemv_check(w, x, b, r, 128, 1024, kch)
+    assert err < 1e-5  # fp32 accumulation of exact fixed-point partial sums
+
+
+@pytest.mark.parametrize("batch", [2, 5])
+def test_gemv_batch_and_staged_rows(batch):
+    rng = np.random.default_rng(50 + batch)
+    w = inputs.weight(rng, 256, 4096)
+    x = inputs.activation(rng, 4096, batch=batch)
+    gemv_check(w, x, 2, 2, 128, 1024, 32)
+    gemv_check(w, x, 2, 2, 128, 1024, 32, give_sel=True)
+    gemv_check(w, x, 2, 2, 128, 1024, 32, staged=True)
+
+
+@pytest.mark.parametrize("G", [32, 64, 256])
+def test_gemv_group_sizes(G):
+    rng = np.random.default_rng(G)
+    w = inputs.weight(rng, 128, 1024)
+    x = inputs.activation(rng, 1024)
+    gemv_check(w, x, 3, 2, G, 1024, 16)
+    gemv_check(w, x, 2, 2, G, 256, 5)
+
+
+def test_gemv_single_workload_full_size():
+    """4096 x 4096, 2-bit base + 2 refinement bits, k = 32 per 1,024 (seed 0)."""
+    w, x = inputs.gemv_case(seed=0)
+    gemv_check(w, x, 2, 2, 128, 1024, 32)
+
+
+def test_gemv_layer_workload_full_size():
+    """One Llama-3.1-8B-shaped layer's projections, 3-bit base + 1 refinement bit."""
+    for name, (w, x) in inputs.layer_case(seed=1).items():
+        gemv_check(w, x, 3, 1, 128, 1024, 32)
+
+
+# ---------------------------------------------------------------------------
+# KV cache
+
+
+def kv_setup(T, b=2, r=2, t_max=None, seed=2, batch=1, h_kv=8, h_q=32, split_pack=False):
+    k, v, q = inputs.kv_case(seed=seed, t=T, h_kv=h_kv, h_q=h_q, batch=batch)
+    t_max = t_max or ((T + 15) // 16) * 16
+    cache = KVCache(batch, h_kv, t_max, b, r)
+    if split_pack and T > 1:
+        h = T // 2
+        cache.pack_tokens(cu(f16bits(k[:, :, :h])), cu(f16bits(v[:, :, :h])), 0)
+        cache.pack_tokens(cu(f16bits(k[:, :, h:])), cu(f16bits(v[:, :, h:])), h)
+    else:
+        cache.pack_tokens(cu(f16bits(k)), cu(f16bits(v)), 0)
+    kc = oracle.quant_kv(k, b, r)
+    vc = oracle.quant_kv(v, b, r)
+    return cache, kc, vc, q
+
+
+def check_selection(sel, score, k_tok):
+    B, H, T = score.shape
+    for bb in range(B):
+        for g in range(H):
+            s = sel[bb, g]
+            assert len(s) == k_tok and np.all(np.diff(s) > 0) and s[0] >= 0 and s[-1] < T
+            order = np.lexsort((np.arange(T), -score[bb, g]))
+            kth = score[bb, g, order[k_tok - 1]]
+            diff = set(s.tolist()) ^ set(order[:k_tok].tolist())
+            for t in diff:
+                assert abs(score[bb, g, t] - kth) <= SEL_RTOL * kth, (bb, g, t, score[bb, g, t], kth)
+
+
+@pytest.mark.parametrize("b,r", [(2, 2), (2, 1), (4, 2), (4, 1)])
+def test_kv_pack_bit_exact(b, r):
+    cache, kc, vc, q = kv_setup(37, b, r, t_max=48, split_pack=True, batch=2, h_kv=2, h_q=8)
+    torch.cuda.synchronize()
+    for which, (qb, rho, sz) in ((0, kc), (1, vc)):
+        gq, grho = cache.unpack(which, 37)
+        assert np.array_equal(host(gq), qb) and np.array_equal(host(grho), rho)
+        gsz = host(cache.ksz if which == 0 else cache.vsz).view(np.uint16).reshape(2, 2, 48, 4, 2)[:, :, :37]
+        assert np.array_equal(gsz, sz)
+        base, refine = oracle.pack_kv(qb, rho, b, r, t_max=48)
+        gb = host(cache.kb if which == 0 else cache.vb)
+        gr = host(cache.kr if which == 0 else cache.vr)
+        tok_b, tok_r = 128 * b // 8, 128 * r // 8
+        for bh in range(4):  # compare the written token slots only
+            sl_b = slice(bh * 48 * tok_b, (bh * 48 + 37) * tok_b)
+            sl_r = slice(bh * 48 * tok_r, (bh * 48 + 37) * tok_r)
+            assert np.array_equal(gb[sl_b], base[sl_b]) and np.array_equal(gr[sl_r], refine[sl_r])
+
+
+def kv_parity(T, k_tok, splits=(0,), use_logits=True, b=2, r=2, batch=1, h_kv=8, h_q=32, seed=2):
+    cache, kc, vc, q = kv_setup(T, b, r, batch=batch, h_kv=h_kv, h_q=h_q, seed=seed)
+    qd = cu(f16bits(q))
+    sel, logits, scores = cache.score_select(qd, T, k_tok, want_scores=True)
+    torch.cuda.synchronize()
+    lo = oracle.kv_logits(kc[0], kc[2], q)
+    assert rel_l2(host(logits), lo) < 1e-5
+    so = oracle.kv_scores(lo, h_kv)
+    assert rel_l2(host(scores), so) < 1e-5
+    gsel = host(sel)
+    check_selection(gsel, so, k_tok)
+    ref = oracle.kv_attention(kc, vc, q, gsel, k_tok, r)
+    for ns in splits:
+        out = cache.attn_refined(qd, T, sel, k_tok, base_logits=logits if use_logits else None, n_splits=ns)
+        torch.cuda.synchronize()
+        o = host(out)
+        assert rel_l2(o, ref) <= RTOL_L2
+        assert np.abs(o - ref).max() <= ATTN_MAX_ABS
+    return cache, kc, vc, q, qd
+
+
+@pytest.mark.parametrize("T,k_tok", [(1, 1), (37, 1), (37, 37), (100, 10), (1000, 64), (2049, 300)])
+def test_kv_parity_small(T, k_tok):
+    kv_parity(T, k_tok, splits=(0, 1, 7), use_logits=True)
+
+
+def test_kv_parity_without_stored_logits_and_batch():
+    kv_parity(777, 50, splits=(0, 3), use_logits=False, batch=2, h_kv=4, h_q=32, seed=9)
+    kv_parity(500, 20, splits=(0,), use_logits=True, b=4, r=1, h_kv=2, h_q=4, seed=10)
+
+
+def test_kv_base_only_and_all_selected():
+    cache, kc, vc, q = kv_setup(300, batch=1, h_kv=8, h_q=32, seed=11)
+    qd = cu(f16bits(q))
+    out0 = cache.attn_refined(qd, 300, None, 0)
+    all_sel = torch.arange(300, dtype=torch.int32, device="cuda").repeat(1, 8, 1).contiguous()
+    outT = cache.attn_refined(qd, 300, all_sel, 300)
+    torch.cuda.synchronize()
+    ref0 = oracle.kv_attention(kc, vc, q, None, 0, 2)
+    refT = oracle.kv_attention(kc, vc, q, host(all_sel), 300, 2)
+    assert np.abs(host(out0) - ref0).max() <= ATTN_MAX_ABS and rel_l2(host(out0), ref0) <= RTOL_L2
+    assert np.abs(host(outT) - refT).max() <= ATTN_MAX_ABS and rel_l2(host(outT), refT) <= RTOL_L2
+
+
+def test_kv_attention_8k_workload():
+    """32 query / 8 KV heads, d 128, T = 8,192, 2+2 bits, top-256 tokens per KV head."""
+    kv_parity(8192, 256, splits=(0, 1, 7), seed=2)
+
+
+def test_kv_attention_128k_workload():
+    """T = 131,072, top-1,024 tokens per KV head, split-K merged by log-sum-exp."""
+    kv_parity(131072, 1024, splits=(0,), seed=3)
