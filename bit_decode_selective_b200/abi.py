@@ -45,15 +45,28 @@ _SIGNATURES = {
     "sf_gemv_refined": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_gemv_workspace_bytes": ([POINTER(sf_wq), c_int, c_int, c_int], c_size_t),
+    "sf_gemv_correction": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                            c_void_p, c_void_p], c_int),
     "sf_kv_bytes": ([c_int] * 7 + [POINTER(c_size_t)] * 3, c_int),
     "sf_kv_pack_tokens": ([POINTER(sf_kv), c_void_p, c_void_p, c_int, c_int, c_void_p], c_int),
     "sf_kv_unpack_codes": ([POINTER(sf_kv), c_int, c_int, c_void_p, c_void_p, c_void_p], c_int),
     "sf_kv_score_select": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_kv_score_select_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
-    "sf_kv_attn_refined": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_void_p, c_int, c_void_p,
-                            c_int, c_void_p, c_void_p, c_size_t, c_void_p], c_int),
-    "sf_kv_attn_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int], c_size_t),
+    "sf_kv_attn_refined": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_void_p, c_int, c_int,
+                            c_void_p, c_void_p, c_size_t, c_void_p], c_int),
+    "sf_kv_attn_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
+    "sf_kv_attend_selective": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_size_t, c_void_p], c_int),
+    "sf_kv_attend_selective_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
+    "sf_rmsnorm_residual": ([c_void_p, c_void_p, c_void_p, c_int, c_int, ctypes.c_float, c_void_p,
+                             c_void_p], c_int),
+    "sf_rope_split": ([c_void_p, c_int, c_int, c_int, c_int, c_int, ctypes.c_float, c_void_p, c_void_p,
+                       c_void_p, c_void_p], c_int),
+    "sf_silu_mul": ([c_void_p, c_int, c_int, c_void_p, c_void_p], c_int),
+    "sf_cast_f16": ([c_void_p, c_size_t, c_void_p, c_void_p], c_int),
+    "sf_widen_f16": ([c_void_p, c_size_t, c_void_p, c_void_p], c_int),
+    "sf_gemv_f16": ([c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p], c_int),
     "sf_stage_refinements": ([c_void_p, c_size_t, c_void_p, c_int, c_void_p, c_void_p, c_void_p],
                              c_int),
     "sf_stage_refinements_host": ([c_void_p, c_size_t, c_void_p, c_int, c_void_p, c_void_p,
@@ -106,6 +119,7 @@ sf_unpack_codes = _call("sf_unpack_codes")
 sf_select_channels = _call("sf_select_channels")
 sf_gemv_refined = _call("sf_gemv_refined")
 sf_gemv_workspace_bytes = _call("sf_gemv_workspace_bytes")
+sf_gemv_correction = _call("sf_gemv_correction")
 sf_kv_bytes = _call("sf_kv_bytes")
 sf_kv_pack_tokens = _call("sf_kv_pack_tokens")
 sf_kv_unpack_codes = _call("sf_kv_unpack_codes")
@@ -113,5 +127,13 @@ sf_kv_score_select = _call("sf_kv_score_select")
 sf_kv_score_select_workspace_bytes = _call("sf_kv_score_select_workspace_bytes")
 sf_kv_attn_refined = _call("sf_kv_attn_refined")
 sf_kv_attn_workspace_bytes = _call("sf_kv_attn_workspace_bytes")
+sf_kv_attend_selective = _call("sf_kv_attend_selective")
+sf_kv_attend_selective_workspace_bytes = _call("sf_kv_attend_selective_workspace_bytes")
+sf_rmsnorm_residual = _call("sf_rmsnorm_residual")
+sf_rope_split = _call("sf_rope_split")
+sf_silu_mul = _call("sf_silu_mul")
+sf_cast_f16 = _call("sf_cast_f16")
+sf_widen_f16 = _call("sf_widen_f16")
+sf_gemv_f16 = _call("sf_gemv_f16")
 sf_stage_refinements = _call("sf_stage_refinements")
 sf_stage_refinements_host = _call("sf_stage_refinements_host")

@@ -8,32 +8,39 @@
 //   nested-quantization paragraph -- the refined value is the centre of the
 //     refinement's sub-bin inside the base bin:
 //       w~ = w^ + s * (2*rho + 1 - 2^r) / 2^(r+1).
+//   the-map-app-also-loads-tiles paragraph -- with fetch lag the correction
+//     of a projection is applied later than its base product; the
+//     correction-only mode below computes it on its own.
 //
 // Decomposition, per output row i (fp32 accumulation):
 //   y_i = sum_groups [ s_ig * sum_{c in g} x_c q_ic + m_ig * sum_{c in g} x_c ]
 //       + sum_{c selected} x_c * s_i,g(c) * (2 rho_ic + 1 - 2^r) / 2^(r+1)
 //
-// Base pass (HBM-bound; every resident code is read once): each CTA owns a
+// Base pass (HBM-bound: every resident code is read once).  Each CTA owns a
 // contiguous range of rows; each warp owns one 2,048-channel segment of K and
-// keeps that segment's activations in registers as exact fixed point (per
-// 32-channel block, x = x_fix * 2^e with |x_fix| < 2^23, split into three
-// bytes).  A lane reads 64 channels of a row (16 B of 2-bit codes) per step,
-// expands them to byte vectors with shifts and masks and takes the integer
-// dot products with dp4a (4 code x byte products per instruction); the three
-// byte planes are recombined, scaled by 2^e, s and m in fp32.
+// keeps that segment's activations in registers as exact fixed point: per
+// 64-channel lane group x = x_fix * 2^e with |x_fix| < 2^23, split into three
+// byte planes.  A lane streams 64 channels of a row per step (16 B of 2-bit
+// codes), expands them to byte vectors with shifts and masks and takes the
+// integer dot products with dp4a (4 code x byte products per instruction).
+// Rows are prefetched one step ahead in registers; partial sums of four rows
+// are reduced across the warp with a transposed butterfly.
 //
 // Correction pass: after griddepcontrol.wait (the selection kernel may still
-// be running while the base pass streams), one warp per row sums the
-// selected channels' corrections from the channel-major refinement rows.
+// be running while the base pass streams), the CTA stages the selected
+// channels' activations and the refinement words covering its rows in shared
+// memory with independent loads, then one warp per row sums the corrections.
 #include "common.cuh"
 #include "internal.cuh"
 
 namespace sf {
 namespace {
 
-constexpr int kSegChannels = 2048;  // 32 lanes x 2 blocks x 32 channels
-constexpr int kMaxWarps = 16;
-constexpr int kUnroll = 4;          // rows in flight per warp
+constexpr int kSegChannels = 2048;  // 32 lanes x 64 channels
+constexpr int kWarps = 8;
+constexpr int kCtasPerSm = 2;
+constexpr int kXWords = 52;         // per 64-channel group: 16 vectors x 3 planes, sum, 2^e, pad
+constexpr int kCorrSmemWords = 12 * 1024;
 
 struct GemvParams {
   const uint32_t* base;
@@ -45,9 +52,9 @@ struct GemvParams {
   int N, K, G, r, batch, n_sel, segs, row_warps;
   int refine_row_words;  // N * r / 32
   int staged;            // refine holds [batch][n_sel] staged rows
+  int mode;              // 0: base + correction, 1: correction only, added into y
 };
 
-// ---- dp4a wrappers (inline PTX: unsigned codes times unsigned/signed bytes)
 __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -59,79 +66,52 @@ __device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c) {
   return d;
 }
 
-// Words of packed codes per lane per row (two 32-channel blocks).
+// Words of packed codes per lane per row (64 channels).
 template <int BITS>
-struct Lane;
-template <>
-struct Lane<2> {
-  static constexpr int W = 4;
-};
-template <>
-struct Lane<3> {
-  static constexpr int W = 6;
-};
-template <>
-struct Lane<4> {
-  static constexpr int W = 8;
+struct Lane {
+  static constexpr int W = BITS == 2 ? 4 : BITS == 3 ? 6 : 8;
+  static constexpr int U = BITS == 4 ? 2 : 4;  // rows per step
 };
 
 template <int BITS>
-__device__ __forceinline__ void load_codes(const GemvParams& p, int row, int blk0,
+__device__ __forceinline__ void load_codes(const GemvParams& p, int row, int lg,
                                            uint32_t (&w)[Lane<BITS>::W]) {
+  // lg: the lane's 64-channel group index within the row
   if constexpr (BITS == 2) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16) + blk0 * 2));
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16)) + lg);
     w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
   } else if constexpr (BITS == 3) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16) + blk0 * 2));
-    uint2 h = __ldg(reinterpret_cast<const uint2*>(p.base + (size_t)p.N * p.K / 16 +
-                                                   (size_t)row * (p.K / 32) + blk0));
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16)) + lg);
+    uint2 h = __ldg(reinterpret_cast<const uint2*>(p.base + (size_t)p.N * p.K / 16 + (size_t)row * (p.K / 32)) + lg);
     w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w, w[4] = h.x, w[5] = h.y;
   } else {
-    const uint4* src = reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 8) + blk0 * 4);
+    const uint4* src = reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 8)) + 2 * lg;
     uint4 a = __ldg(src), b = __ldg(src + 1);
     w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
   }
 }
 
-// Code byte-vector v (0..7) of block k (0,1) of the lane's words.  Byte L of
-// vector v holds the code of channel chan_of(v, L) (see prep_x).
+// Code byte-vector v (0..15) of the lane's 64 channels; byte L holds the code
+// of channel chan_of(v, L) (0..63).
 template <int BITS>
-__device__ __forceinline__ uint32_t code_vec(const uint32_t (&w)[Lane<BITS>::W], int k, int v) {
+__device__ __forceinline__ uint32_t code_vec(const uint32_t (&w)[Lane<BITS>::W], int v) {
   if constexpr (BITS == 4) {
-    int wi = v >> 1, j = v & 1;
-    return (w[k * 4 + wi] >> (4 * j)) & 0x0F0F0F0Fu;
+    return (w[v >> 1] >> (4 * (v & 1))) & 0x0F0F0F0Fu;  // word v/2: 8 channels
   } else {
-    int wi = v >> 2, j = v & 3;  // wi: channels 0-15 (A) or 16-31 (B) of the block
-    uint32_t c = (w[k * 2 + wi] >> (2 * j)) & 0x03030303u;
+    const int wi = v >> 2, j = v & 3;  // word wi: 16 channels
+    uint32_t c = (w[wi] >> (2 * j)) & 0x03030303u;
     if constexpr (BITS == 3) {
-      uint32_t h = w[4 + k];
-      c |= ((h >> (4 * wi + j)) << 2) & 0x04040404u;
+      const int sh = 4 * (wi & 1) + j;  // high bits of the 32-channel block wi/2
+      c |= ((w[4 + (wi >> 1)] >> sh) << 2) & 0x04040404u;
     }
     return c;
   }
 }
 
-// Channel (0..31 within the block) held in byte L of vector v.
 template <int BITS>
 __host__ __device__ __forceinline__ int chan_of(int v, int L) {
   if (BITS == 4) return 8 * (v >> 1) + (v & 1) + 2 * L;
   return 16 * (v >> 2) + (v & 3) + 4 * L;
-}
-
-// Integer dot product of one block's codes with the x byte planes, as fp32.
-template <int BITS>
-__device__ __forceinline__ float block_dot(const uint32_t (&w)[Lane<BITS>::W], int k,
-                                           const uint32_t* xv) {
-  uint32_t lo = 0, mid = 0;
-  int32_t hi = 0;
-#pragma unroll
-  for (int v = 0; v < 8; v++) {
-    uint32_t c = code_vec<BITS>(w, k, v);
-    lo = dp4a_uu(c, xv[v * 3 + 0], lo);
-    mid = dp4a_uu(c, xv[v * 3 + 1], mid);
-    hi = dp4a_us(c, xv[v * 3 + 2], hi);
-  }
-  return fmaf((float)hi, 65536.0f, (float)((mid << 8) + lo));
 }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -140,170 +120,295 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Shared-memory image of x for one batch row: per 32-channel block, 8 vectors
-// x 3 byte planes (lo, mid, hi), two floats (sum of x, 2^e) and two words of
-// padding so that every block starts on a 16-byte boundary.
-constexpr int kXWords = 28;
+// Sum each of U per-lane values over the warp; lane (u * 32 / U) .. holds row u.
+// Returns the full sum of row (lane >> (5 - log2 U)) in every lane.
+template <int U>
+__device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
+  if constexpr (U == 4) {
+    // xor 16: lanes < 16 keep rows 0,1; lanes >= 16 keep rows 2,3
+    const bool up = lane & 16;
+    float k0 = up ? a[2] : a[0], k1 = up ? a[3] : a[1];
+    float s0 = up ? a[0] : a[2], s1 = up ? a[1] : a[3];
+    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    // xor 8: keep one row
+    const bool up8 = lane & 8;
+    float k = up8 ? k1 : k0, s = up8 ? k0 : k1;
+    k += __shfl_xor_sync(0xffffffffu, s, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;  // row 2*(lane>>4) + ((lane>>3)&1) = lane >> 3
+  } else {
+    const bool up = lane & 16;
+    float k = up ? a[1] : a[0], s = up ? a[0] : a[1];
+    k += __shfl_xor_sync(0xffffffffu, s, 16);
+    k += __shfl_xor_sync(0xffffffffu, k, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;  // row lane >> 4
+  }
+}
 
+// x of one batch row -> fixed-point byte planes per 64-channel group.
 template <int BITS>
-__device__ void prep_x(const uint16_t* __restrict__ x, int K, uint32_t* xs) {
+__device__ void prep_x(const uint16_t* __restrict__ x, int K, uint16_t* xraw, uint32_t* xs) {
+  // all loads first (16 B per thread per step), then the per-group work
+  for (int i = threadIdx.x; i < K / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(xraw)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   uint8_t* xb = reinterpret_cast<uint8_t*>(xs);
-  for (int blk = warp; blk < K / 32; blk += nwarps) {
-    float xv = h2f(x[blk * 32 + lane]);
-    float mx = fabsf(xv);
+  for (int grp = warp; grp < K / 64; grp += nwarps) {
+    // lane handles channels 2*lane, 2*lane + 1 of the group
+    __half2 hv = reinterpret_cast<const __half2*>(xraw + grp * 64)[lane];
+    float2 xv = __half22float2(hv);
+    float mx = fmaxf(fabsf(xv.x), fabsf(xv.y));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    // scale so that |x_fix| < 2^23: e = floor(log2 max|x|) - 22
-    int e = mx > 0.f ? ilogbf(mx) - 22 : 0;
-    int xf = mx > 0.f ? __float2int_rn(ldexpf(xv, -e)) : 0;  // exact power-of-2 scaling
-    // lane = channel c; find its (vector, byte) slot
-    int v, L;
-    if (BITS == 4) {
-      v = 2 * (lane >> 3) + (lane & 1);
-      L = (lane & 7) >> 1;
-    } else {
-      v = 4 * (lane >> 4) + (lane & 3);
-      L = (lane & 15) >> 2;
+    const int e = mx > 0.f ? ilogbf(mx) - 22 : 0;  // |x| * 2^-e < 2^23
+    uint8_t* base = xb + (size_t)grp * kXWords * 4;
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int c = 2 * lane + h;
+      const float xc = h ? xv.y : xv.x;
+      const int xf = mx > 0.f ? __float2int_rn(ldexpf(xc, -e)) : 0;
+      int v, L;
+      if (BITS == 4) {
+        v = 2 * (c >> 3) + (c & 1);
+        L = (c & 7) >> 1;
+      } else {
+        v = 4 * (c >> 4) + (c & 3);
+        L = (c & 15) >> 2;
+      }
+      uint8_t* dst = base + v * 12 + L;
+      dst[0] = (uint8_t)(xf & 0xff);
+      dst[4] = (uint8_t)((xf >> 8) & 0xff);
+      dst[8] = (uint8_t)((xf >> 16) & 0xff);
     }
-    uint8_t* dst = xb + (size_t)blk * kXWords * 4 + v * 12 + L;
-    dst[0] = (uint8_t)(xf & 0xff);
-    dst[4] = (uint8_t)((xf >> 8) & 0xff);
-    dst[8] = (uint8_t)((xf >> 16) & 0xff);
-    float s = warp_sum(xv);
+    float s = warp_sum(xv.x + xv.y);
     if (lane == 0) {
-      reinterpret_cast<float*>(xs)[blk * kXWords + 24] = s;
-      reinterpret_cast<float*>(xs)[blk * kXWords + 25] = ldexpf(1.0f, e);
+      reinterpret_cast<float*>(base)[48] = s;
+      reinterpret_cast<float*>(base)[49] = ldexpf(1.0f, e);
     }
   }
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(GemvParams p) {
-  extern __shared__ __align__(16) uint32_t smem[];
-  const int nblk = p.K / 32;
-  uint32_t* xs = smem;                                        // nblk * kXWords
-  float* part = reinterpret_cast<float*>(smem + nblk * kXWords);  // rows x segs
+__device__ __forceinline__ float group_dot(const uint32_t (&w)[Lane<BITS>::W], const uint32_t (&xr)[48]) {
+  uint32_t lo = 0, mid = 0;
+  int32_t hi = 0;
+#pragma unroll
+  for (int v = 0; v < 16; v++) {
+    uint32_t c = code_vec<BITS>(w, v);
+    lo = dp4a_uu(c, xr[3 * v + 0], lo);
+    mid = dp4a_uu(c, xr[3 * v + 1], mid);
+    hi = dp4a_us(c, xr[3 * v + 2], hi);
+  }
+  return fmaf((float)hi, 65536.0f, (float)mid * 256.0f + (float)lo);
+}
 
+// Same, split into the two 32-channel halves (groups of 32 channels).
+template <int BITS>
+__device__ __forceinline__ float2 group_dot_halves(const uint32_t (&w)[Lane<BITS>::W],
+                                                   const uint32_t (&xr)[48]) {
+  uint32_t lo[2] = {0, 0}, mid[2] = {0, 0};
+  int32_t hi[2] = {0, 0};
+#pragma unroll
+  for (int v = 0; v < 16; v++) {
+    const int h = chan_of<BITS>(v, 0) >= 32;
+    uint32_t c = code_vec<BITS>(w, v);
+    lo[h] = dp4a_uu(c, xr[3 * v + 0], lo[h]);
+    mid[h] = dp4a_uu(c, xr[3 * v + 1], mid[h]);
+    hi[h] = dp4a_us(c, xr[3 * v + 2], hi[h]);
+  }
+  return make_float2(fmaf((float)hi[0], 65536.0f, (float)mid[0] * 256.0f + (float)lo[0]),
+                     fmaf((float)hi[1], 65536.0f, (float)mid[1] * 256.0f + (float)lo[1]));
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kWarps * 32, BITS == 2 ? kCtasPerSm : 1) gemv_kernel(GemvParams p) {
+  constexpr int W = Lane<BITS>::W, U = Lane<BITS>::U;
+  extern __shared__ __align__(16) uint32_t smem[];
+  const int ngrp = p.K / 64;
+  uint32_t* xs = smem;                                       // ngrp * kXWords
+  float* part = reinterpret_cast<float*>(xs + ngrp * kXWords);  // rows x segs
   const int n0 = (int)((long)blockIdx.x * p.N / gridDim.x);
   const int n1 = (int)((long)(blockIdx.x + 1) * p.N / gridDim.x);
+  const int rows = n1 - n0;
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(part + ((rows * p.segs + 3) & ~3));  // x staging, then correction
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = warp % p.segs, rw = warp / p.segs;
-  const bool warp_active = rw < p.row_warps;
-  const int blk0 = seg * (kSegChannels / 32) + 2 * lane;  // first of the lane's two blocks
-  const bool lane_active = warp_active && blk0 < nblk;
-  const int gpb = p.G / 32;  // blocks per group
+  const bool warp_active = p.mode == 0 && rw < p.row_warps;
+  const int lg = seg * 32 + lane;  // lane's 64-channel group
+  const bool lane_active = warp_active && lg < ngrp;
+  const int G = p.G;
+  const bool split = G == 32;
 
   for (int b = 0; b < p.batch; b++) {
-    prep_x<BITS>(p.x + (size_t)b * p.K, p.K, xs);
-    __syncthreads();
-    uint32_t xr[2][24];
-    float xsum[2] = {0.f, 0.f}, xscale[2] = {0.f, 0.f};
-    if (lane_active) {
-#pragma unroll
-      for (int k = 0; k < 2; k++) {
-        const uint4* src = reinterpret_cast<const uint4*>(xs + (blk0 + k) * kXWords);
-#pragma unroll
-        for (int i = 0; i < 6; i++) {
-          uint4 v = src[i];
-          xr[k][4 * i + 0] = v.x, xr[k][4 * i + 1] = v.y, xr[k][4 * i + 2] = v.z,
-          xr[k][4 * i + 3] = v.w;
-        }
-        xsum[k] = __uint_as_float(xs[(blk0 + k) * kXWords + 24]);
-        xscale[k] = __uint_as_float(xs[(blk0 + k) * kXWords + 25]);
-      }
+    const uint16_t* xrow = p.x + (size_t)b * p.K;
+    if (p.mode == 0) {
+      // every (row, segment) partial is written by exactly one warp below
+      prep_x<BITS>(xrow, p.K, reinterpret_cast<uint16_t*>(scratch), xs);
+    } else {
+      for (int i = threadIdx.x; i < rows * p.segs; i += blockDim.x) part[i] = 0.f;
     }
+    __syncthreads();
     if (warp_active) {
-      for (int i0 = n0 + rw * kUnroll; i0 < n1; i0 += p.row_warps * kUnroll) {
-        uint32_t w[kUnroll][Lane<BITS>::W];
-        uint32_t zs[kUnroll][2];
+      uint32_t xr[48];
+      float xsum = 0.f, xscale = 0.f;
+      if (lane_active) {
+        const uint4* src = reinterpret_cast<const uint4*>(xs + lg * kXWords);
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
-          int row = i0 + u;
+        for (int i = 0; i < 12; i++) {
+          uint4 v = src[i];
+          xr[4 * i + 0] = v.x, xr[4 * i + 1] = v.y, xr[4 * i + 2] = v.z, xr[4 * i + 3] = v.w;
+        }
+        xsum = __uint_as_float(xs[lg * kXWords + 48]);
+        xscale = __uint_as_float(xs[lg * kXWords + 49]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 48; i++) xr[i] = 0;
+      }
+      // sums of x over the two 32-channel halves (groups of 32 only)
+      float xs0 = 0.f, xs1 = 0.f;
+      if (split && lane_active) {
+        const __half2* xh = reinterpret_cast<const __half2*>(xrow + lg * 64);
+        for (int i = 0; i < 16; i++) {
+          float2 a = __half22float2(xh[i]), c = __half22float2(xh[16 + i]);
+          xs0 += a.x + a.y;
+          xs1 += c.x + c.y;
+        }
+      }
+      const uint32_t* szrow = reinterpret_cast<const uint32_t*>(p.sz);
+      const int gpr = p.K / G;
+      const int g0 = (lg * 64) / G, g1 = (lg * 64 + 32) / G;
+      const int step = p.row_warps * U;
+      uint32_t wa[U][W], wb[U][W], za[U][2], zb[U][2];
+      auto load = [&](int i0, uint32_t (&w)[U][W], uint32_t (&z)[U][2]) {
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+          const int row = i0 + u;
           if (lane_active && row < n1) {
-            load_codes<BITS>(p, row, blk0, w[u]);
-            const uint32_t* szw = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)row * (p.K / p.G);
-            zs[u][0] = __ldg(szw + blk0 / gpb);
-            zs[u][1] = __ldg(szw + (blk0 + 1) / gpb);
+            load_codes<BITS>(p, row, lg, w[u]);
+            z[u][0] = __ldg(szrow + (size_t)row * gpr + g0);
+            z[u][1] = split ? __ldg(szrow + (size_t)row * gpr + g1) : z[u][0];
+          } else {
+#pragma unroll
+            for (int i = 0; i < W; i++) w[u][i] = 0;
+            z[u][0] = z[u][1] = 0;
           }
         }
+      };
+      auto compute = [&](int i0, const uint32_t (&w)[U][W], const uint32_t (&z)[U][2]) {
+        float acc[U];
 #pragma unroll
-        for (int u = 0; u < kUnroll; u++) {
-          int row = i0 + u;
-          float acc = 0.f;
-          if (lane_active && row < n1) {
-#pragma unroll
-            for (int k = 0; k < 2; k++) {
-              float2 sm = __half22float2(*reinterpret_cast<const __half2*>(&zs[u][k]));
-              float d = block_dot<BITS>(w[u], k, xr[k]) * xscale[k];
-              acc = fmaf(sm.x, d, acc);
-              acc = fmaf(sm.y, xsum[k], acc);
-            }
+        for (int u = 0; u < U; u++) {
+          float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&z[u][0]));
+          if (!split) {
+            float d = group_dot<BITS>(w[u], xr) * xscale;
+            acc[u] = fmaf(s0.x, d, s0.y * xsum);
+          } else {
+            float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&z[u][1]));
+            float2 d = group_dot_halves<BITS>(w[u], xr);
+            acc[u] = fmaf(s0.x, d.x * xscale, fmaf(s1.x, d.y * xscale, fmaf(s0.y, xs0, s1.y * xs1)));
           }
-          acc = warp_sum(acc);
-          if (lane == 0 && row < n1) part[(row - n0) * p.segs + seg] = acc;
         }
+        const float tot = warp_sum_rows<U>(acc, lane);
+        const int u = U == 4 ? (lane >> 3) : (lane >> 4);
+        const int row = i0 + u;
+        if ((lane & (32 / U - 1)) == 0 && row < n1) part[(row - n0) * p.segs + seg] = tot;
+      };
+      int i0 = n0 + rw * U;
+      if (i0 < n1) load(i0, wa, za);
+      for (; i0 < n1; i0 += 2 * step) {
+        if (i0 + step < n1) load(i0 + step, wb, zb);
+        compute(i0, wa, za);
+        if (i0 + step >= n1) break;
+        if (i0 + 2 * step < n1) load(i0 + 2 * step, wa, za);
+        compute(i0 + step, wb, zb);
       }
     }
     __syncthreads();
 
-    // correction for the selected channels of batch row b
+    // ---- correction of the selected channels of batch row b
     if (p.n_sel > 0) {
       pdl_wait();  // selection (and staged rows) complete and visible
       const int32_t* sel = p.sel + (size_t)b * p.n_sel;
-      const uint16_t* xb = p.x + (size_t)b * p.K;
-      const int nwarps = blockDim.x >> 5;
-      // (2 rho + 1 - 2^r) / 2^(r+1) = (rho + 1/2 - 2^(r-1)) / 2^r
-      const float half = 0.5f * (float)(1 << p.r);
-      const float inv = 1.0f / (float)(1 << p.r);
-      for (int row = n0 + warp; row < n1; row += nwarps) {
-        float corr = 0.f;
-        const int rbit = row * p.r;
-        for (int j = lane; j < p.n_sel; j += 32) {
-          int c = __ldg(sel + j);
-          const uint32_t* rrow = p.staged ? p.refine + ((size_t)b * p.n_sel + j) * p.refine_row_words
-                                          : p.refine + (size_t)c * p.refine_row_words;
-          uint32_t rho = (__ldg(rrow + (rbit >> 5)) >> (rbit & 31)) & ((1u << p.r) - 1);
-          float s = h2f(__ldg(p.sz + ((size_t)row * (p.K / p.G) + c / p.G) * 2));
-          float cf = ((float)rho + 0.5f - half) * inv;
-          corr = fmaf(h2f(__ldg(xb + c)) * s, cf, corr);
+      const int w0 = (n0 * p.r) >> 5;
+      const int nw = (((n1 * p.r) + 31) >> 5) - w0;
+      const float half = 0.5f * (float)(1 << p.r), inv = 1.0f / (float)(1 << p.r);
+      const int per_sel = 2 + nw;
+      const bool staged_smem = (long)p.n_sel * per_sel <= kCorrSmemWords;
+      if (staged_smem) {
+        // [n_sel] x * 2^-r, [n_sel] group, [n_sel][nw] refinement words
+        float* cx = reinterpret_cast<float*>(scratch);
+        int* cg = reinterpret_cast<int*>(cx + p.n_sel);
+        uint32_t* cw = reinterpret_cast<uint32_t*>(cg + p.n_sel);
+        for (int j = threadIdx.x; j < p.n_sel; j += blockDim.x) {
+          const int c = __ldg(sel + j);
+          cx[j] = h2f(__ldg(xrow + c)) * inv;
+          cg[j] = c / G;
         }
-        corr = warp_sum(corr);
-        if (lane == 0) part[(row - n0) * p.segs] += corr;
+        for (int i = threadIdx.x; i < p.n_sel * nw; i += blockDim.x) {
+          const int j = i / nw, k = i % nw;
+          const uint32_t* rrow = p.staged ? p.refine + ((size_t)b * p.n_sel + j) * p.refine_row_words
+                                          : p.refine + (size_t)__ldg(sel + j) * p.refine_row_words;
+          cw[j * nw + k] = __ldg(rrow + w0 + k);
+        }
+        __syncthreads();
+        const int nwarps = blockDim.x >> 5;
+        for (int row = n0 + warp; row < n1; row += nwarps) {
+          const int bit = row * p.r - w0 * 32;
+          const uint16_t* zr = p.sz + (size_t)row * (p.K / G) * 2;
+          float corr = 0.f;
+          for (int j = lane; j < p.n_sel; j += 32) {
+            const uint32_t rho = (cw[j * nw + (bit >> 5)] >> (bit & 31)) & ((1u << p.r) - 1);
+            const float s = h2f(__ldg(zr + 2 * cg[j]));
+            corr = fmaf(cx[j] * s, (float)rho + 0.5f - half, corr);
+          }
+          corr = warp_sum(corr);
+          if (lane == 0) part[(row - n0) * p.segs] += corr;
+        }
+      } else {
+        const int nwarps = blockDim.x >> 5;
+        for (int row = n0 + warp; row < n1; row += nwarps) {
+          float corr = 0.f;
+          const int rbit = row * p.r;
+          for (int j = lane; j < p.n_sel; j += 32) {
+            const int c = __ldg(sel + j);
+            const uint32_t* rrow = p.staged ? p.refine + ((size_t)b * p.n_sel + j) * p.refine_row_words
+                                            : p.refine + (size_t)c * p.refine_row_words;
+            const uint32_t rho = (__ldg(rrow + (rbit >> 5)) >> (rbit & 31)) & ((1u << p.r) - 1);
+            const float s = h2f(__ldg(p.sz + ((size_t)row * (p.K / G) + c / G) * 2));
+            corr = fmaf(h2f(__ldg(xrow + c)) * inv * s, (float)rho + 0.5f - half, corr);
+          }
+          corr = warp_sum(corr);
+          if (lane == 0) part[(row - n0) * p.segs] += corr;
+        }
       }
       __syncthreads();
     }
     for (int row = n0 + threadIdx.x; row < n1; row += blockDim.x) {
       float acc = 0.f;
       for (int s = 0; s < p.segs; s++) acc += part[(row - n0) * p.segs + s];
-      p.y[(size_t)b * p.N + row] = acc;
+      float* dst = p.y + (size_t)b * p.N + row;
+      *dst = p.mode == 1 ? *dst + acc : acc;
     }
     __syncthreads();
   }
 }
 
-}  // namespace
-}  // namespace sf
-
-using namespace sf;
-
-extern "C" size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch) {
-  (void)w, (void)batch, (void)chunk, (void)kch;
-  return 0;
-}
-
-extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk,
-                                     int kch, const int32_t* sel_in, int32_t* sel_out,
-                                     const void* refine_rows, float* y, void* ws, size_t ws_bytes,
-                                     sf_stream_t stream) {
-  (void)ws, (void)ws_bytes;
+sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
+                      const int32_t* sel_in, int32_t* sel_out, const void* refine_rows, float* y,
+                      int mode, cudaStream_t s) {
   sf_status st = check_wq_public(w, false);
   if (st != SF_OK) return st;
   SF_REQUIRE(x && aligned16(x), "x must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(y && aligned16(y), "y must be a non-null 16-byte aligned device pointer");
   SF_UNSUPPORTED(batch >= 1 && batch <= 8, "batch=%d outside [1, 8]", batch);
   SF_REQUIRE(kch >= 0, "kch=%d < 0", kch);
-  cudaStream_t s = as_stream(stream);
   const int32_t* sel = nullptr;
   int n_sel = 0;
   if (kch > 0) {
@@ -321,6 +426,8 @@ extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batc
       if (st != SF_OK) return st;
       sel = sel_out;
     }
+  } else if (mode == 1) {
+    return SF_OK;  // nothing to correct
   }
   GemvParams p;
   p.base = (const uint32_t*)w->base;
@@ -330,24 +437,30 @@ extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batc
   p.sel = sel;
   p.y = y;
   p.N = w->n, p.K = w->k, p.G = w->group, p.r = w->r, p.batch = batch, p.n_sel = n_sel;
+  p.mode = mode;
   p.segs = (w->k + kSegChannels - 1) / kSegChannels;
-  SF_UNSUPPORTED(p.segs <= kMaxWarps, "k=%d too large", w->k);
+  SF_UNSUPPORTED(p.segs <= kWarps, "k=%d above %d", w->k, kWarps * kSegChannels);
   p.refine_row_words = w->n * w->r / 32;
   p.staged = refine_rows != nullptr;
-  int grid = num_sms();
-  if (grid > w->n / 8) grid = w->n / 8;
-  int rows_per_cta = (w->n + grid - 1) / grid;
-  p.row_warps = kMaxWarps / p.segs;
-  int needed = (rows_per_cta + kUnroll - 1) / kUnroll;
+  // 2-bit codes fit two CTAs of 8 warps per SM in registers; wider codes one
+  int grid = (w->b == 2 ? kCtasPerSm : 1) * num_sms();
+  if (grid > w->n / 4) grid = w->n / 4;
+  const int rows_per_cta = (w->n + grid - 1) / grid;
+  const int U = w->b == 4 ? 2 : 4;
+  p.row_warps = kWarps / p.segs;
+  const int needed = (rows_per_cta + U - 1) / U;
   if (p.row_warps > needed) p.row_warps = needed;
-  int threads = p.segs * p.row_warps * 32;
-  if (threads < 128) threads = 128;  // the correction pass uses every warp
-  size_t smem = (size_t)(w->k / 32) * kXWords * 4 + (size_t)rows_per_cta * p.segs * 4;
-  SF_UNSUPPORTED(smem <= 200 * 1024, "k=%d needs too much shared memory", w->k);
+  if (p.row_warps < 1) p.row_warps = 1;
+  const size_t xs_words = (size_t)(w->k / 64) * kXWords;
+  const size_t part_words = ((size_t)rows_per_cta * p.segs + 3) & ~(size_t)3;
+  size_t scratch_words = (size_t)w->k / 2;  // raw x (fp16)
+  if (scratch_words < (size_t)kCorrSmemWords) scratch_words = kCorrSmemWords;
+  const size_t smem = (xs_words + part_words + scratch_words) * 4;
+  SF_UNSUPPORTED(smem <= 110 * 1024, "k=%d needs too much shared memory", w->k);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
+  cfg.blockDim = dim3(kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -356,7 +469,32 @@ extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batc
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void (*kern)(GemvParams) = w->b == 2 ? gemv_kernel<2> : w->b == 3 ? gemv_kernel<3> : gemv_kernel<4>;
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024));
   SF_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
   return SF_OK;
+}
+
+}  // namespace
+}  // namespace sf
+
+using namespace sf;
+
+extern "C" size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch) {
+  (void)w, (void)batch, (void)chunk, (void)kch;
+  return 0;
+}
+
+extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk,
+                                     int kch, const int32_t* sel_in, int32_t* sel_out,
+                                     const void* refine_rows, float* y, void* ws, size_t ws_bytes,
+                                     sf_stream_t stream) {
+  (void)ws, (void)ws_bytes;
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, 0, as_stream(stream));
+}
+
+extern "C" sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch, int chunk,
+                                        int kch, const int32_t* sel, const void* refine_rows,
+                                        float* y, sf_stream_t stream) {
+  SF_REQUIRE(kch == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
+  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, 1, as_stream(stream));
 }

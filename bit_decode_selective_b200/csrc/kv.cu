@@ -10,117 +10,416 @@
 //   nested-quantization paragraph -- refinement bits subdivide the base bin;
 //   where-it-earns-its-keep paragraph -- KV refinement is a step that cannot
 //     overlap the attention around it, since the selection depends on the
-//     attention scores.  Hence the order: logits -> softmax stats -> scores ->
-//     selection -> refined attention.
+//     attention scores.
 //
-// Kernels:
-//   kv_logits_kernel   base logits of a span of tokens for the query heads of
-//                      one KV head, plus the span's (max, sum exp) per head;
-//   kv_stats_kernel    merge the spans' (max, sum) into the softmax stats;
-//   kv_local_kernel    per span, score every token and keep the span's
-//                      k_tok best (a token in the global top-k is in the top-k
-//                      of its own span), in token order;
+// Schedule (one pass over the resident cache, then work on the selected
+// tokens only):
+//   kv_base_kernel     per 16-token tile, logits of the group's query heads
+//                      from the base keys and the base attention (online
+//                      softmax, split-K partials) from the base values; the
+//                      logits are stored for scoring.  Codes are turned into
+//                      exact fp16 integers in registers and contracted on the
+//                      tensor cores (mma.sync m16n8k16, fp32 accumulation);
+//                      the per-token fp16 steps/offsets are applied in fp32.
+//   kv_stats_kernel    softmax max/sum of every query head from the partials;
+//   kv_local_kernel    per context span, score every token and keep the
+//                      span's k_tok best (a token in the global top-k is in
+//                      the top-k of its own span), in token order;
 //   kv_final_kernel    per KV head, the k_tok best of the candidates;
-//   kv_attn_kernel     per context split, online-softmax attention with the
-//                      selected tokens dequantised at b+r bits;
-//   kv_merge_kernel    log-sum-exp merge of the splits.
+//   kv_correct_kernel  for the selected tokens only: swap each token's base
+//                      contribution for its refined one (refined logit, refined
+//                      value), relative to the head's softmax max;
+//   kv_merge_kernel    log-sum-exp merge of the partials plus the correction.
+// The result equals softmax(q.k~) v~ with refined k~, v~ on the selected
+// tokens, up to fp32 rounding.
 #include <cfloat>
 
 #include "common.cuh"
+#include "kvlayout.cuh"
 
 namespace sf {
 namespace {
 
-constexpr int kD = 128;          // head dim (validated)
-constexpr int kGroups = kD / 32; // quantisation groups per token
-constexpr int kTile = 64;        // tokens per shared-memory tile (logits)
-constexpr int kATile = 32;       // tokens per shared-memory tile (attention)
+constexpr int kD = kHeadDim;
+constexpr int kRec = kD + 2;     // partial record: acc[kD], m, l
+constexpr int kWarps = 4;        // warps per base-pass CTA (independent splits)
+constexpr int kStages = 4;       // cp.async ring depth per warp
 constexpr int kMaxCand = 16384;  // candidates per KV head in the final select
 constexpr int kMaxSpan = 8192;   // tokens per local-select CTA
+constexpr int kCorrTok = 16;     // selected tokens per correction CTA
 
-struct KvView {
-  const uint32_t *kb, *kr, *vb, *vr;
-  const uint16_t *ksz, *vsz;
-  int h_kv, t_max, b, r;
-};
+// ---- small PTX helpers -------------------------------------------------------
 
-__device__ __forceinline__ long slot_of(const KvView& kv, int bat, int g, int t) {
-  return ((long)bat * kv.h_kv + g) * kv.t_max + t;
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Dequantise element d of token `slot` (base, or refined when `refined`).
-__device__ __forceinline__ float kv_value(const uint32_t* codes, const uint32_t* refine,
-                                          const uint16_t* sz, long slot, int d, int b, int r,
-                                          bool refined) {
-  long e = slot * kD + d;
-  uint32_t q = (codes[(e * b) >> 5] >> ((e * b) & 31)) & ((1u << b) - 1);
-  const uint16_t* z = sz + (slot * kGroups + d / 32) * 2;
-  float s = h2f(z[0]), m = h2f(z[1]);
-  float v = (float)q;
-  if (refined) {
-    uint32_t rho = (refine[(e * r) >> 5] >> ((e * r) & 31)) & ((1u << r) - 1);
-    v += ((float)rho + 0.5f - 0.5f * (float)(1 << r)) / (float)(1 << r);
-  }
-  return fmaf(s, v, m);
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+}
+
+// Pair slot `slot` (compile-time after unrolling) of a w-bit pair-slot word as
+// an exact half2; see kvlayout.cuh.
+template <int W>
+__device__ __forceinline__ uint32_t pair_at(uint32_t w, uint32_t w_hi8, int slot) {
+  const int bit = W * slot;
+  const bool shift = bit + W > 10;
+  const int b2 = shift ? bit - 8 : bit;
+  const uint32_t mask = (((1u << W) - 1u) << b2) * 0x00010001u;
+  uint32_t v = ((shift ? w_hi8 : w) & mask) | 0x64006400u;  // 1024 + c * 2^b2 per half
+  const uint32_t sc = (uint32_t)((15 - b2) << 10) * 0x00010001u;              // 2^-b2
+  const uint32_t off = (uint32_t)(0x8000u | ((25 - b2) << 10)) * 0x00010001u;  // -1024 * 2^-b2
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&v), *reinterpret_cast<const __half2*>(&sc),
+                      *reinterpret_cast<const __half2*>(&off));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+template <int W>
+__device__ __forceinline__ uint32_t pair_of(const uint32_t* words, const uint32_t* words8, int p) {
+  constexpr int per = 16 / W;
+  return pair_at<W>(words[p / per], words8[p / per], p % per);
 }
 
 // ---------------------------------------------------------------------------
-// logits
+// base pass
 
-__global__ void __launch_bounds__(256) kv_logits_kernel(KvView kv, int T, int span,
-                                                        const uint16_t* __restrict__ q, int h_q,
-                                                        float* __restrict__ logits,
-                                                        float2* __restrict__ part) {
-  const int gq = h_q / kv.h_kv;
-  const int sp = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
-  const int t0 = sp * span, t1 = min(T, t0 + span);
-  __shared__ float qs[8][kD + 1];
-  __shared__ float kd[kTile][kD + 1];
-  __shared__ float red[8][kTile];
-  const float scale = rsqrtf((float)kD);
-  for (int i = threadIdx.x; i < gq * kD; i += blockDim.x)
-    qs[i / kD][i % kD] = h2f(q[((long)bat * h_q + g * gq + i / kD) * kD + i % kD]) * scale;
-  float run_m[8], run_s[8];  // used by threads 0..gq-1
-  for (int h = 0; h < 8; h++) run_m[h] = -FLT_MAX, run_s[h] = 0.f;
-  __syncthreads();
-  for (int tt = t0; tt < t1; tt += kTile) {
-    const int nt = min(kTile, t1 - tt);
-    for (int i = threadIdx.x; i < nt * kD; i += blockDim.x) {
-      int t = i / kD, d = i % kD;
-      kd[t][d] = kv_value(kv.kb, kv.kr, kv.ksz, slot_of(kv, bat, g, tt + t), d, kv.b, kv.r, false);
+struct BaseArgs {
+  const uint8_t* kb;
+  const uint8_t* vb;
+  const uint16_t* ksz;
+  const uint16_t* vsz;
+  int h_kv, t_max, T;
+  const uint16_t* q;
+  int h_q, gq;
+  float* logits;  // [batch][h_q][T]
+  float* part;    // [batch][h_q][nsplit][rec]  (rec = kRec with values, 2 without)
+  int span, nsplit;
+  float scale;
+};
+
+template <int B, bool PV>
+struct Stage {
+  static constexpr int kBytes = 256 * B;           // key codes of 16 tokens
+  static constexpr int vBytes = PV ? 256 * B : 0;  // value tile
+  static constexpr int szBytes = PV ? 512 : 256;   // key (+ value) step/offset
+  static constexpr int bytes = kBytes + vBytes + szBytes;
+};
+
+// GQP: query heads per KV head padded to 4 or 8.  B: base bits (2 or 4).
+template <int GQP, int B, bool PV>
+__global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
+  using St = Stage<B, PV>;
+  constexpr int NT = GQP / 4;  // value-side n-tiles (4 heads x hi/lo each)
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int g = blockIdx.y, bat = blockIdx.z;
+  const int split = blockIdx.x * kWarps + warp;
+  if (split >= a.nsplit) return;  // warp-private from here on: no block barriers
+  uint8_t* wsm = smem + warp * (kStages * St::bytes + 16 * 9 * 4 + 8 * 4);
+  float* Ps = reinterpret_cast<float*>(wsm + kStages * St::bytes);  // [16][9]
+  float* As = Ps + 16 * 9;                                           // [8]
+
+  const int tw0 = split * a.span;
+  const int tw1 = min(a.T, tw0 + a.span);
+  const int ntile = tw1 > tw0 ? (tw1 - tw0 + 15) / 16 : 0;
+  const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;  // first token slot of this head
+  const int gq = a.gq;
+
+  // ---- query fragments (B operand of the key contraction): head gid
+  const uint16_t* qg = a.q + ((long)bat * a.h_q + (long)g * gq) * kD;
+  uint32_t qf[8][2];
+  float qsum[4];  // per group j: sum of q over the lane's 8 dims of head gid
+#pragma unroll
+  for (int j = 0; j < 4; j++) qsum[j] = 0.f;
+#pragma unroll
+  for (int s = 0; s < 8; s++) {
+    uint32_t lo = 0, hi = 0;
+    if (gid < gq) {
+      lo = *reinterpret_cast<const uint32_t*>(qg + gid * kD + 16 * s + 2 * tig);
+      hi = *reinterpret_cast<const uint32_t*>(qg + gid * kD + 16 * s + 2 * tig + 8);
     }
-    __syncthreads();
-    for (int pr = threadIdx.x; pr < nt * gq; pr += blockDim.x) {
-      int t = pr / gq, h = pr % gq;
-      float acc = 0.f;
-      for (int d = 0; d < kD; d++) acc = fmaf(qs[h][d], kd[t][d], acc);
-      logits[((long)bat * h_q + g * gq + h) * T + tt + t] = acc;
-      red[h][t] = acc;
-    }
-    __syncthreads();
-    if (threadIdx.x < gq) {
-      int h = threadIdx.x;
-      float m = run_m[h];
-      for (int t = 0; t < nt; t++) m = fmaxf(m, red[h][t]);
-      float s = run_s[h] * expf(run_m[h] - m);
-      for (int t = 0; t < nt; t++) s += expf(red[h][t] - m);
-      run_m[h] = m, run_s[h] = s;
-    }
-    __syncthreads();
+    qf[s][0] = lo, qf[s][1] = hi;
+    float2 f0 = __half22float2(*reinterpret_cast<__half2*>(&lo));
+    float2 f1 = __half22float2(*reinterpret_cast<__half2*>(&hi));
+    qsum[s >> 1] += (f0.x + f0.y) + (f1.x + f1.y);
   }
-  if (threadIdx.x < gq) {
-    int h = g * gq + threadIdx.x;
-    part[((long)bat * h_q + h) * gridDim.x + sp] = make_float2(run_m[threadIdx.x], run_s[threadIdx.x]);
+  // full per-group sums of head gid, then fetch heads 2tig, 2tig+1 for the epilogue
+  float Q0[4], Q1[4];
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    float v = qsum[j];
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    Q0[j] = __shfl_sync(0xffffffffu, v, 8 * tig);      // head 2tig   (gid = 2tig)
+    Q1[j] = __shfl_sync(0xffffffffu, v, 8 * tig + 4);  // head 2tig+1 (gid = 2tig+1)
+  }
+
+  float mrun0 = -FLT_MAX, mrun1 = -FLT_MAX, lsum0 = 0.f, lsum1 = 0.f;
+  float accv[NT][8][4];
+  float mt[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+    for (int m = 0; m < 8; m++)
+#pragma unroll
+      for (int i = 0; i < 4; i++) accv[nt][m][i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) mt[nt][j] = 0.f;
+  }
+
+  auto issue = [&](int it) {
+    if (it < ntile) {
+      uint8_t* st = wsm + (it % kStages) * St::bytes;
+      const long slot = slot0 + tw0 + 16 * it;
+#pragma unroll
+      for (int c = 0; c < B / 2; c++) {
+        int ci = lane + 32 * c;
+        cp_async16(st + 16 * ci, a.kb + slot * 16 * B + 16 * ci);
+        if (PV) cp_async16(st + St::kBytes + 16 * ci, a.vb + (slot / 16) * 256 * B + 16 * ci);
+      }
+      if (lane < 16)
+        cp_async16(st + St::kBytes + St::vBytes + 16 * lane, reinterpret_cast<const uint8_t*>(a.ksz) + slot * 16 + 16 * lane);
+      else if (PV)
+        cp_async16(st + St::kBytes + St::vBytes + 16 * lane,
+                   reinterpret_cast<const uint8_t*>(a.vsz) + slot * 16 + 16 * (lane - 16));
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int i = 0; i < kStages - 1; i++) issue(i);
+
+  const float NEG = -INFINITY;
+  for (int it = 0; it < ntile; it++) {
+    issue(it + kStages - 1);
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const uint8_t* st = wsm + (it % kStages) * St::bytes;
+    const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
+    const uint16_t* ks = reinterpret_cast<const uint16_t*>(st + St::kBytes + St::vBytes);
+    const int t0 = tw0 + 16 * it;
+
+    // ---- logits: tokens on M (gid, gid+8), heads on N, k-steps of 16 dims
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+#pragma unroll
+      for (int i = 0; i < 4; i++) acc[j][i] = 0.f;
+    {
+      uint32_t w0[B], w8[B], w0s[B], w8s[B];
+#pragma unroll
+      for (int i = 0; i < B; i++) {
+        w0[i] = kc[gid * 4 * B + tig * B + i];
+        w8[i] = kc[(gid + 8) * 4 * B + tig * B + i];
+        w0s[i] = w0[i] >> 8;
+        w8s[i] = w8[i] >> 8;
+      }
+#pragma unroll
+      for (int s = 0; s < 8; s++) {
+        uint32_t a0 = pair_of<B>(w0, w0s, 2 * s), a1 = pair_of<B>(w8, w8s, 2 * s);
+        uint32_t a2 = pair_of<B>(w0, w0s, 2 * s + 1), a3 = pair_of<B>(w8, w8s, 2 * s + 1);
+        mma16816(acc[s >> 1], a0, a1, a2, a3, qf[s][0], qf[s][1]);
+      }
+    }
+    float l[4];  // (tok gid, head 2tig), (gid, 2tig+1), (gid+8, 2tig), (gid+8, 2tig+1)
+#pragma unroll
+    for (int r = 0; r < 2; r++) {
+      const int tok = gid + 8 * r;
+      const uint32_t* zw = reinterpret_cast<const uint32_t*>(ks + tok * 8);
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        uint32_t z = zw[j];
+        float2 sm = __half22float2(*reinterpret_cast<__half2*>(&z));
+        x0 = fmaf(sm.x, acc[j][2 * r + 0], fmaf(sm.y, Q0[j], x0));
+        x1 = fmaf(sm.x, acc[j][2 * r + 1], fmaf(sm.y, Q1[j], x1));
+      }
+      const bool valid = t0 + tok < tw1;
+      l[2 * r + 0] = valid ? x0 * a.scale : NEG;
+      l[2 * r + 1] = valid ? x1 * a.scale : NEG;
+    }
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
+    {
+      float* lg = a.logits + ((long)bat * a.h_q + (long)g * gq) * a.T;
+#pragma unroll
+      for (int r = 0; r < 2; r++) {
+        const int t = t0 + gid + 8 * r;
+        if (t < tw1) {
+          if (h0 < gq) lg[(long)h0 * a.T + t] = l[2 * r];
+          if (h1 < gq) lg[(long)h1 * a.T + t] = l[2 * r + 1];
+        }
+      }
+    }
+    // ---- online softmax over this warp's tokens (heads 2tig, 2tig+1)
+    float mx0 = fmaxf(l[0], l[2]), mx1 = fmaxf(l[1], l[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(mrun0, mx0), mn1 = fmaxf(mrun1, mx1);
+    const float al0 = __expf(mrun0 - mn0), al1 = __expf(mrun1 - mn1);
+    float p[4];
+    p[0] = (h0 < gq && l[0] != NEG) ? __expf(l[0] - mn0) : 0.f;
+    p[1] = (h1 < gq && l[1] != NEG) ? __expf(l[1] - mn1) : 0.f;
+    p[2] = (h0 < gq && l[2] != NEG) ? __expf(l[2] - mn0) : 0.f;
+    p[3] = (h1 < gq && l[3] != NEG) ? __expf(l[3] - mn1) : 0.f;
+    lsum0 = fmaf(lsum0, al0, p[0] + p[2]);
+    lsum1 = fmaf(lsum1, al1, p[1] + p[3]);
+    mrun0 = mn0, mrun1 = mn1;
+
+    if constexpr (PV) {
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + St::kBytes);
+      const uint16_t* vs = ks + 128;
+      Ps[gid * 9 + h0] = p[0];
+      Ps[gid * 9 + h1] = p[1];
+      Ps[(gid + 8) * 9 + h0] = p[2];
+      Ps[(gid + 8) * 9 + h1] = p[3];
+      if (gid == 0) As[h0] = al0, As[h1] = al1;
+      __syncwarp();
+      // value step/offset of the lane's four tokens 2tig, 2tig+1, 2tig+8, 2tig+9
+      float vsv[4][4], vmv[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const int tk = 2 * tig + (i & 1) + 8 * (i >> 1);
+        const bool valid = t0 + tk < tw1;
+        const uint32_t* zw = reinterpret_cast<const uint32_t*>(vs + tk * 8);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          uint32_t z = zw[j];
+          float2 sm = __half22float2(*reinterpret_cast<__half2*>(&z));
+          vsv[i][j] = valid ? sm.x : 0.f;
+          vmv[i][j] = valid ? sm.y : 0.f;
+        }
+      }
+      uint32_t bf[NT][4][2];
+      float av[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; nt++) {
+        av[nt] = As[4 * nt + tig];
+        const int hb = 4 * nt + (gid >> 1);
+        const bool hi_part = (gid & 1) == 0;
+        float pv[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) pv[i] = Ps[(2 * tig + (i & 1) + 8 * (i >> 1)) * 9 + hb];
+        const float ab = As[hb];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          __half hv[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            float v = pv[i] * vsv[i][j];
+            __half h = __float2half_rn(v);
+            hv[i] = hi_part ? h : __float2half_rn(v - __half2float(h));
+          }
+          bf[nt][j][0] = pack_h2(hv[0], hv[1]);
+          bf[nt][j][1] = pack_h2(hv[2], hv[3]);
+          if (hi_part) {
+            float s = mt[nt][j] * ab;
+#pragma unroll
+            for (int i = 0; i < 4; i++) s = fmaf(pv[i], vmv[i][j], s);
+            mt[nt][j] = s;
+          }
+        }
+      }
+      uint32_t vw[2 * B], vws[2 * B];
+#pragma unroll
+      for (int i = 0; i < 2 * B; i++) {
+        vw[i] = vc[lane * 2 * B + i];
+        vws[i] = vw[i] >> 8;
+      }
+      // Each tile's product starts from zero and is folded into the running
+      // sum with one fp32 FMA that also applies the softmax rescale: long
+      // accumulation chains inside the tensor-core accumulator would drift.
+#pragma unroll
+      for (int m = 0; m < 8; m++) {
+        uint32_t a0 = pair_of<B>(vw, vws, 2 * m), a1 = pair_of<B>(vw, vws, 2 * m + 1);
+        uint32_t a2 = pair_of<B>(vw, vws, 16 + 2 * m), a3 = pair_of<B>(vw, vws, 17 + 2 * m);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+          float t4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma16816(t4, a0, a1, a2, a3, bf[nt][m >> 1][0], bf[nt][m >> 1][1]);
+#pragma unroll
+          for (int i = 0; i < 4; i++) accv[nt][m][i] = fmaf(accv[nt][m][i], av[nt], t4[i]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+  // ---- partial record of this split
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    lsum0 += __shfl_xor_sync(0xffffffffu, lsum0, o);
+    lsum1 += __shfl_xor_sync(0xffffffffu, lsum1, o);
+  }
+  const long hq0 = (long)bat * a.h_q + (long)g * gq;
+  if constexpr (!PV) {
+    if (gid == 0) {
+      if (2 * tig < gq) {
+        float* rec = a.part + ((hq0 + 2 * tig) * a.nsplit + split) * 2;
+        rec[0] = mrun0, rec[1] = lsum0;
+      }
+      if (2 * tig + 1 < gq) {
+        float* rec = a.part + ((hq0 + 2 * tig + 1) * a.nsplit + split) * 2;
+        rec[0] = mrun1, rec[1] = lsum1;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NT; nt++) {
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        float v = mt[nt][j];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        mt[nt][j] = __shfl_sync(0xffffffffu, v, 8 * tig);  // head 4nt + tig (gid = 2tig, hi part)
+      }
+      const int h = 4 * nt + tig;
+      const float ma = __shfl_sync(0xffffffffu, mrun0, h >> 1), mb = __shfl_sync(0xffffffffu, mrun1, h >> 1);
+      const float la = __shfl_sync(0xffffffffu, lsum0, h >> 1), lb = __shfl_sync(0xffffffffu, lsum1, h >> 1);
+      if (h < gq) {
+        float* rec = a.part + ((hq0 + h) * a.nsplit + split) * kRec;
+#pragma unroll
+        for (int m = 0; m < 8; m++) {
+          rec[16 * m + gid] = accv[nt][m][0] + accv[nt][m][1] + mt[nt][m >> 1];
+          rec[16 * m + gid + 8] = accv[nt][m][2] + accv[nt][m][3] + mt[nt][m >> 1];
+        }
+        if (gid == 0) {
+          rec[kD] = (h & 1) ? mb : ma;
+          rec[kD + 1] = (h & 1) ? lb : la;
+        }
+      }
+    }
   }
 }
 
-// (max, sum exp) of every query head from the spans' partials.
-__global__ void kv_stats_kernel(const float2* __restrict__ part, int nspan, float2* __restrict__ stats) {
-  const long bh = blockIdx.x;  // bat * h_q + h
-  const float2* p = part + bh * nspan;
+// Softmax max and sum of every query head: M = max_s m_s, Z = sum_s l_s e^(m_s - M).
+__global__ void kv_stats_kernel(const float* __restrict__ part, int nsplit, int rec,
+                                float2* __restrict__ stats) {
+  const long bh = blockIdx.x;
+  const float* p = part + bh * nsplit * rec;
+  const int mo = rec == 2 ? 0 : kD;
   __shared__ float sm[256];
   float m = -FLT_MAX;
-  for (int i = threadIdx.x; i < nspan; i += blockDim.x) m = fmaxf(m, p[i].x);
+  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) m = fmaxf(m, p[(long)i * rec + mo]);
   sm[threadIdx.x] = m;
   __syncthreads();
   for (int o = blockDim.x / 2; o > 0; o >>= 1) {
@@ -130,7 +429,10 @@ __global__ void kv_stats_kernel(const float2* __restrict__ part, int nspan, floa
   const float M = sm[0];
   __syncthreads();
   float s = 0.f;
-  for (int i = threadIdx.x; i < nspan; i += blockDim.x) s += p[i].y * expf(p[i].x - M);
+  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) {
+    float mi = p[(long)i * rec + mo];
+    if (mi > -FLT_MAX) s += p[(long)i * rec + mo + 1] * expf(mi - M);
+  }
   sm[threadIdx.x] = s;
   __syncthreads();
   for (int o = blockDim.x / 2; o > 0; o >>= 1) {
@@ -153,7 +455,6 @@ __device__ __forceinline__ int key_token(uint64_t key) {
 }
 
 // k-th largest of n unique keys (1 <= k <= n), 8 bits per pass from the top.
-// keys in shared memory; hist: 256 ints of shared scratch.
 __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int k, int* hist) {
   __shared__ int s_digit, s_k;
   uint64_t prefix = 0, mask = 0;
@@ -166,8 +467,7 @@ __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int k, int* h
     }
     __syncthreads();
     if (threadIdx.x < 32) {
-      // lane l owns digits 255-8l .. 248-8l (descending)
-      const int lane = threadIdx.x;
+      const int lane = threadIdx.x;  // owns digits 255-8*lane .. 248-8*lane
       int c[8], tot = 0;
 #pragma unroll
       for (int j = 0; j < 8; j++) tot += (c[j] = hist[255 - 8 * lane - j]);
@@ -177,7 +477,7 @@ __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int k, int* h
         int v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      int above = incl - tot;  // keys with a larger digit
+      int above = incl - tot;
       if (above < k && incl >= k) {
         int run = above;
         for (int j = 0; j < 8; j++) {
@@ -199,8 +499,7 @@ __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int k, int* h
   return prefix;
 }
 
-// Write the keys >= tau in index order: out[pos] for pos = rank among them.
-// Thread i handles a contiguous range of indices, so order is preserved.
+// Emit the keys >= tau in index order (each thread owns a contiguous range).
 template <class Emit>
 __device__ void block_compact(const uint64_t* keys, int n, uint64_t tau, Emit emit) {
   __shared__ int warp_tot[32];
@@ -271,7 +570,7 @@ __global__ void __launch_bounds__(1024) kv_final_kernel(const uint64_t* __restri
   const int per = min(k_tok, span);
   const uint64_t* src = cand + ((long)bat * h_kv + g) * nspan * (long)per;
   int n = 0;
-  for (int sp = 0; sp < nspan; sp++) {  // spans hold min(k_tok, their length) keys
+  for (int sp = 0; sp < nspan; sp++) {
     int len = min(T, (sp + 1) * span) - sp * span;
     int cnt = min(k_tok, len);
     for (int i = threadIdx.x; i < cnt; i += blockDim.x) keys[n + i] = src[(long)sp * per + i];
@@ -284,173 +583,163 @@ __global__ void __launch_bounds__(1024) kv_final_kernel(const uint64_t* __restri
 }
 
 // ---------------------------------------------------------------------------
-// refined attention (split over the context, partials merged by log-sum-exp)
+// correction on the selected tokens
 
-__global__ void __launch_bounds__(256) kv_attn_kernel(KvView kv, int T, int span,
-                                                      const uint16_t* __restrict__ q, int h_q,
-                                                      const int32_t* __restrict__ sel, int k_tok,
-                                                      const float* __restrict__ base_logits,
-                                                      float* __restrict__ part) {
-  const int gq = h_q / kv.h_kv;
-  const int sp = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
-  const int t0 = sp * span, t1 = min(T, t0 + span);
-  __shared__ float qs[8][kD + 1];
-  __shared__ float kd[kATile][kD + 1];
-  __shared__ float vd[kATile][kD + 1];
-  __shared__ float pl[8][kATile];
-  __shared__ float s_m[8], s_l[8], s_alpha[8];
-  extern __shared__ uint32_t selmask[];  // one bit per token of the span
-  const float scale = rsqrtf((float)kD);
-  for (int i = threadIdx.x; i < gq * kD; i += blockDim.x)
-    qs[i / kD][i % kD] = h2f(q[((long)bat * h_q + g * gq + i / kD) * kD + i % kD]) * scale;
-  for (int i = threadIdx.x; i < (span + 31) / 32; i += blockDim.x) selmask[i] = 0;
-  if (threadIdx.x < 8) s_m[threadIdx.x] = -FLT_MAX, s_l[threadIdx.x] = 0.f;
-  __syncthreads();
-  const int32_t* sg = sel + ((long)bat * kv.h_kv + g) * k_tok;
-  for (int j = threadIdx.x; j < k_tok; j += blockDim.x) {
-    int t = sg[j];
-    if (t >= t0 && t < t1) atomicOr(&selmask[(t - t0) >> 5], 1u << ((t - t0) & 31));
-  }
-  // accumulators: thread owns (head, dim) pairs idx, idx + 256, ...
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  __syncthreads();
-  for (int tt = t0; tt < t1; tt += kATile) {
-    const int nt = min(kATile, t1 - tt);
-    for (int i = threadIdx.x; i < nt * kD; i += blockDim.x) {
-      int t = i / kD, d = i % kD;
-      int lt = tt + t - t0;
-      bool rf = (selmask[lt >> 5] >> (lt & 31)) & 1;
-      long slot = slot_of(kv, bat, g, tt + t);
-      if (rf || !base_logits) kd[t][d] = kv_value(kv.kb, kv.kr, kv.ksz, slot, d, kv.b, kv.r, rf);
-      vd[t][d] = kv_value(kv.vb, kv.vr, kv.vsz, slot, d, kv.b, kv.r, rf);
-    }
-    __syncthreads();
-    for (int pr = threadIdx.x; pr < nt * gq; pr += blockDim.x) {
-      int t = pr / gq, h = pr % gq;
-      int lt = tt + t - t0;
-      bool rf = (selmask[lt >> 5] >> (lt & 31)) & 1;
-      float l;
-      if (rf || !base_logits) {
-        l = 0.f;
-        for (int d = 0; d < kD; d++) l = fmaf(qs[h][d], kd[t][d], l);
-      } else {
-        l = base_logits[((long)bat * h_q + g * gq + h) * T + tt + t];
-      }
-      pl[h][t] = l;
-    }
-    __syncthreads();
-    if (threadIdx.x < gq) {  // online softmax update of head h
-      int h = threadIdx.x;
-      float m = s_m[h];
-      for (int t = 0; t < nt; t++) m = fmaxf(m, pl[h][t]);
-      float alpha = expf(s_m[h] - m);
-      float l = s_l[h] * alpha;
-      for (int t = 0; t < nt; t++) {
-        float p = expf(pl[h][t] - m);
-        pl[h][t] = p;
-        l += p;
-      }
-      s_m[h] = m, s_l[h] = l, s_alpha[h] = alpha;
-    }
-    __syncthreads();
-    for (int k = 0; k < 4; k++) {
-      int idx = threadIdx.x + 256 * k;
-      if (idx < gq * kD) {
-        int h = idx / kD, d = idx % kD;
-        float a = acc[k] * s_alpha[h];
-        for (int t = 0; t < nt; t++) a = fmaf(pl[h][t], vd[t][d], a);
-        acc[k] = a;
-      }
-    }
-    __syncthreads();
-  }
-  // partial layout: [bat][h_q][nsplit][kD + 2] = (acc[kD], m, l)
-  for (int k = 0; k < 4; k++) {
-    int idx = threadIdx.x + 256 * k;
-    if (idx < gq * kD) {
-      int h = idx / kD, d = idx % kD;
-      part[(((long)bat * h_q + g * gq + h) * gridDim.x + sp) * (kD + 2) + d] = acc[k];
-    }
-  }
-  if (threadIdx.x < gq) {
-    float* p = part + (((long)bat * h_q + g * gq + threadIdx.x) * gridDim.x + sp) * (kD + 2);
-    p[kD] = s_m[threadIdx.x];
-    p[kD + 1] = s_l[threadIdx.x];
-  }
-}
-
-__global__ void kv_merge_kernel(const float* __restrict__ part, int nsplit, float* __restrict__ out) {
-  const long bh = blockIdx.x;
-  const float* p = part + bh * nsplit * (kD + 2);
-  float M = -FLT_MAX;
-  for (int s = 0; s < nsplit; s++) M = fmaxf(M, p[s * (kD + 2) + kD]);
-  float L = 0.f, a = 0.f;
-  const int d = threadIdx.x;
-  for (int s = 0; s < nsplit; s++) {
-    float w = expf(p[s * (kD + 2) + kD] - M);
-    L += w * p[s * (kD + 2) + kD + 1];
-    a += w * p[s * (kD + 2) + d];
-  }
-  out[bh * kD + d] = a / L;
-}
-
-KvView view_of(const sf_kv* kv) {
-  KvView v;
-  v.kb = (const uint32_t*)kv->kb, v.kr = (const uint32_t*)kv->kr;
-  v.vb = (const uint32_t*)kv->vb, v.vr = (const uint32_t*)kv->vr;
-  v.ksz = kv->ksz, v.vsz = kv->vsz;
-  v.h_kv = kv->h_kv, v.t_max = kv->t_max, v.b = kv->b, v.r = kv->r;
-  return v;
-}
-
-// ---- launch geometry --------------------------------------------------------
-
-struct ScorePlan {
-  int lspan, nl;       // logits spans
-  int sspan, ns;       // selection spans
-  size_t off_logits, off_part, off_stats, off_cand, total;
+struct CorrArgs {
+  const uint8_t *kb, *kr, *vb, *vr;
+  const uint16_t *ksz, *vsz;
+  int h_kv, t_max, b, r, T;
+  const uint16_t* q;
+  int h_q, gq;
+  const int32_t* sel;
+  int k_tok;
+  const float* logits;  // base logits [batch][h_q][T]
+  const float2* stats;  // [batch][h_q] (max, sum)
+  float* corr;          // [batch][h_q][ncorr][kRec]: d-acc[kD], d-sum, unused
+  int ncorr;
+  float scale;
 };
 
-ScorePlan score_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool logits_given) {
-  ScorePlan P;
+__device__ __forceinline__ uint32_t read_bits(const uint8_t* base, int word, int bit, int w) {
+  return (reinterpret_cast<const uint32_t*>(base)[word] >> bit) & ((1u << w) - 1u);
+}
+
+// block = kD threads (thread = head-dim element)
+__global__ void __launch_bounds__(kD) kv_correct_kernel(CorrArgs a) {
+  __shared__ float kf[kCorrTok][kD + 4];
+  __shared__ float vbs[kCorrTok][kD];
+  __shared__ float vfs[kCorrTok][kD];
+  __shared__ float qs[8][kD + 4];
+  __shared__ float wf[kCorrTok][8], wb[kCorrTok][8];
+  const int d = threadIdx.x;
+  const int chunk = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
+  const int gq = a.gq;
+  const long hq0 = (long)bat * a.h_q + (long)g * gq;
+  for (int h = 0; h < gq; h++) qs[h][d] = h2f(a.q[(hq0 + h) * kD + d]);
+  const int j0 = chunk * kCorrTok;
+  const int nsel = min(kCorrTok, a.k_tok - j0);
+  const int32_t* sg = a.sel + ((long)bat * a.h_kv + g) * a.k_tok + j0;
+  const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
+  const float half = 0.5f * (float)(1 << a.r), inv = 1.0f / (float)(1 << a.r);
+  for (int i = 0; i < nsel; i++) {
+    const int t = sg[i];
+    const long slot = slot0 + t;
+    int word, bit;
+    // key, refined
+    key_pos(d, a.b, word, bit);
+    uint32_t qk = read_bits(a.kb + slot * 16 * a.b, word, bit, a.b);
+    key_pos(d, a.r, word, bit);
+    uint32_t rk = read_bits(a.kr + slot * 16 * a.r, word, bit, a.r);
+    const uint16_t* zk = a.ksz + (slot * 4 + d / 32) * 2;
+    kf[i][d] = fmaf(h2f(zk[0]), (float)qk + ((float)rk + 0.5f - half) * inv, h2f(zk[1]));
+    // value, base and refined
+    const long tile = slot / 16;
+    value_pos(t & 15, d, a.b, word, bit);
+    uint32_t qv = read_bits(a.vb + tile * 256 * a.b, word, bit, a.b);
+    value_pos(t & 15, d, a.r, word, bit);
+    uint32_t rv = read_bits(a.vr + tile * 256 * a.r, word, bit, a.r);
+    const uint16_t* zv = a.vsz + (slot * 4 + d / 32) * 2;
+    const float sv = h2f(zv[0]), mv = h2f(zv[1]);
+    vbs[i][d] = fmaf(sv, (float)qv, mv);
+    vfs[i][d] = fmaf(sv, (float)qv + ((float)rv + 0.5f - half) * inv, mv);
+  }
+  __syncthreads();
+  // refined logits of (token, head) pairs; base logits as the base pass stored them
+  for (int pr = d; pr < nsel * gq; pr += kD) {
+    const int i = pr / gq, h = pr % gq;
+    float acc = 0.f;
+    for (int e = 0; e < kD; e++) acc = fmaf(qs[h][e], kf[i][e], acc);
+    const float M = a.stats[hq0 + h].x;
+    const float lb = a.logits[(hq0 + h) * a.T + sg[i]];
+    wf[i][h] = __expf(acc * a.scale - M);
+    wb[i][h] = __expf(lb - M);
+  }
+  __syncthreads();
+  for (int h = 0; h < gq; h++) {
+    float da = 0.f, dz = 0.f;
+    for (int i = 0; i < nsel; i++) {
+      da = fmaf(wf[i][h], vfs[i][d], fmaf(-wb[i][h], vbs[i][d], da));
+      dz += wf[i][h] - wb[i][h];
+    }
+    float* rec = a.corr + ((hq0 + h) * a.ncorr + chunk) * kRec;
+    rec[d] = da;
+    if (d == 0) rec[kD] = dz;
+  }
+}
+
+// out = (sum_s e^(m_s - M) acc_s + sum_c dA_c) / (Z + sum_c dZ_c)
+__global__ void __launch_bounds__(kD) kv_merge_kernel(const float* __restrict__ part, int nsplit,
+                                                      const float* __restrict__ corr, int ncorr,
+                                                      const float2* __restrict__ stats,
+                                                      float* __restrict__ out) {
+  const long bh = blockIdx.x;
+  const int d = threadIdx.x;
+  const float2 st = stats[bh];
+  const float* p = part + bh * nsplit * kRec;
+  float num = 0.f;
+  for (int s = 0; s < nsplit; s++) {
+    float ms = p[(long)s * kRec + kD];
+    if (ms > -FLT_MAX) num = fmaf(expf(ms - st.x), p[(long)s * kRec + d], num);
+  }
+  float den = st.y;
+  if (corr) {
+    const float* c = corr + bh * ncorr * kRec;
+    for (int i = 0; i < ncorr; i++) {
+      num += c[(long)i * kRec + d];
+      den += c[(long)i * kRec + kD];
+    }
+  }
+  out[bh * kD + d] = num / den;
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+struct Plan {
+  int nsplit, span;       // base pass (warp splits)
+  int sspan, ns;          // selection spans
+  int ncorr;              // correction chunks per KV head
+  size_t off_logits, off_part, off_stats, off_cand, off_corr, total;
+};
+
+Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, bool with_pv,
+               bool select, int n_splits) {
+  Plan P;
   const int sms = num_sms();
   const int heads = kv->batch * kv->h_kv;
-  P.lspan = 256;
-  P.nl = (t + P.lspan - 1) / P.lspan;
-  int ns = (sms + heads - 1) / heads;
+  int ns = n_splits > 0 ? n_splits : (16 * sms + heads - 1) / heads;
+  int maxs = (t + 15) / 16;
+  if (ns > maxs) ns = maxs;
   if (ns < 1) ns = 1;
-  int span = (t + ns - 1) / ns;
+  P.span = ((t + ns - 1) / ns + 15) / 16 * 16;
+  P.nsplit = (t + P.span - 1) / P.span;
+  // selection spans
+  int ss = (sms + heads - 1) / heads;
+  if (ss < 1) ss = 1;
+  int span = (t + ss - 1) / ss;
   if (span > kMaxSpan) span = kMaxSpan;
   if (span < 32) span = 32;
-  ns = (t + span - 1) / span;
-  while (ns > 1 && (long)ns * (k_tok < span ? k_tok : span) > kMaxCand) {
-    span = (span * 2 > kMaxSpan) ? kMaxSpan : span * 2;
-    int ns2 = (t + span - 1) / span;
-    if (ns2 == ns) break;
-    ns = ns2;
+  ss = (t + span - 1) / span;
+  while (ss > 1 && (long)ss * (k_tok < span ? k_tok : span) > kMaxCand && span < kMaxSpan) {
+    span = span * 2 > kMaxSpan ? kMaxSpan : span * 2;
+    ss = (t + span - 1) / span;
   }
-  P.sspan = span, P.ns = ns;
+  P.sspan = span, P.ns = ss;
+  P.ncorr = k_tok > 0 ? (k_tok + kCorrTok - 1) / kCorrTok : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
     off += (bytes + 255) & ~(size_t)255;
     return o;
   };
-  P.off_logits = logits_given ? 0 : take((size_t)kv->batch * h_q * t * 4);
-  P.off_part = take((size_t)kv->batch * h_q * P.nl * 8);
+  const int rec = with_pv ? kRec : 2;
+  P.off_logits = need_logits ? take((size_t)kv->batch * h_q * t * 4) : 0;
+  P.off_part = take((size_t)kv->batch * h_q * P.nsplit * rec * 4);
   P.off_stats = take((size_t)kv->batch * h_q * 8);
-  P.off_cand = take((size_t)heads * ns * (k_tok < span ? k_tok : span) * 8);
+  P.off_cand = select ? take((size_t)heads * P.ns * (k_tok < span ? k_tok : span) * 8) : 0;
+  P.off_corr = (with_pv && P.ncorr) ? take((size_t)kv->batch * h_q * P.ncorr * kRec * 4) : 0;
   P.total = off;
   return P;
-}
-
-int attn_splits(const sf_kv* kv, int t, int n_splits) {
-  if (n_splits > 0) return n_splits < t ? n_splits : t;
-  const int heads = kv->batch * kv->h_kv;
-  int s = (2 * num_sms() + heads - 1) / heads;
-  int maxs = (t + kATile - 1) / kATile;
-  if (s > maxs) s = maxs;
-  return s < 1 ? 1 : s;
 }
 
 sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
@@ -462,6 +751,90 @@ sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
   return SF_OK;
 }
 
+template <int GQP, int B, bool PV>
+sf_status launch_base_t(const BaseArgs& a, int batch, cudaStream_t s) {
+  const size_t per_warp = kStages * Stage<B, PV>::bytes + 16 * 9 * 4 + 8 * 4;
+  const size_t smem = kWarps * per_warp;
+  auto kern = kv_base_kernel<GQP, B, PV>;
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch);
+  kern<<<grid, kWarps * 32, smem, s>>>(a);
+  SF_LAUNCHED();
+  return SF_OK;
+}
+
+sf_status launch_base(const sf_kv* kv, const BaseArgs& a, bool pv, cudaStream_t s) {
+  const int gqp = a.gq <= 4 ? 4 : 8;
+  if (kv->b == 2) {
+    if (gqp == 4) return pv ? launch_base_t<4, 2, true>(a, kv->batch, s) : launch_base_t<4, 2, false>(a, kv->batch, s);
+    return pv ? launch_base_t<8, 2, true>(a, kv->batch, s) : launch_base_t<8, 2, false>(a, kv->batch, s);
+  }
+  if (gqp == 4) return pv ? launch_base_t<4, 4, true>(a, kv->batch, s) : launch_base_t<4, 4, false>(a, kv->batch, s);
+  return pv ? launch_base_t<8, 4, true>(a, kv->batch, s) : launch_base_t<8, 4, false>(a, kv->batch, s);
+}
+
+BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* logits, float* part,
+                   const Plan& P) {
+  BaseArgs a;
+  a.kb = (const uint8_t*)kv->kb, a.vb = (const uint8_t*)kv->vb;
+  a.ksz = kv->ksz, a.vsz = kv->vsz;
+  a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.T = t;
+  a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
+  a.logits = logits, a.part = part;
+  a.span = P.span, a.nsplit = P.nsplit;
+  a.scale = 1.0f / sqrtf((float)kD);
+  return a;
+}
+
+sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& P,
+                        const float* logits, const float2* stats, float* scores, uint64_t* cand,
+                        int32_t* sel, cudaStream_t s) {
+  long ncand = (long)P.ns * (k_tok < P.sspan ? k_tok : P.sspan);
+  SF_UNSUPPORTED(ncand <= kMaxCand, "t=%d with k_tok=%d needs %ld candidates (max %d)", t, k_tok,
+                 ncand, kMaxCand);
+  SF_CUDA(cudaFuncSetAttribute(kv_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSpan * 8));
+  kv_local_kernel<<<dim3(P.ns, kv->h_kv, kv->batch), 1024, (size_t)P.sspan * 8, s>>>(
+      logits, stats, t, P.sspan, h_q, kv->h_kv, k_tok, scores, cand);
+  SF_LAUNCHED();
+  SF_CUDA(cudaFuncSetAttribute(kv_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCand * 8));
+  kv_final_kernel<<<dim3(kv->h_kv, kv->batch), 1024, (size_t)ncand * 8, s>>>(cand, P.ns, P.sspan, t,
+                                                                           kv->h_kv, k_tok, sel);
+  SF_LAUNCHED();
+  return SF_OK;
+}
+
+sf_status launch_correct_merge(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                               const int32_t* sel, int k_tok, const Plan& P, const float* logits,
+                               const float* part, const float2* stats, float* corr, float* out,
+                               cudaStream_t s) {
+  if (k_tok > 0) {
+    CorrArgs c;
+    c.kb = (const uint8_t*)kv->kb, c.kr = (const uint8_t*)kv->kr;
+    c.vb = (const uint8_t*)kv->vb, c.vr = (const uint8_t*)kv->vr;
+    c.ksz = kv->ksz, c.vsz = kv->vsz;
+    c.h_kv = kv->h_kv, c.t_max = kv->t_max, c.b = kv->b, c.r = kv->r, c.T = t;
+    c.q = q, c.h_q = h_q, c.gq = h_q / kv->h_kv;
+    c.sel = sel, c.k_tok = k_tok, c.logits = logits, c.stats = stats;
+    c.corr = corr, c.ncorr = P.ncorr;
+    c.scale = 1.0f / sqrtf((float)kD);
+    kv_correct_kernel<<<dim3(P.ncorr, kv->h_kv, kv->batch), kD, 0, s>>>(c);
+    SF_LAUNCHED();
+  }
+  kv_merge_kernel<<<kv->batch * h_q, kD, 0, s>>>(part, P.nsplit, k_tok > 0 ? corr : nullptr,
+                                                 P.ncorr, stats, out);
+  SF_LAUNCHED();
+  return SF_OK;
+}
+
+sf_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (ws_bytes < need || (need > 0 && !ws)) {
+    set_error("workspace: need %zu bytes, got %zu", need, ws_bytes);
+    return SF_ERR_WORKSPACE;
+  }
+  SF_REQUIRE(!ws || aligned16(ws), "ws must be 16-byte aligned");
+  return SF_OK;
+}
+
 }  // namespace
 }  // namespace sf
 
@@ -470,7 +843,7 @@ using namespace sf;
 extern "C" size_t sf_kv_score_select_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                                      int logits_given) {
   if (!kv || t <= 0 || h_q <= 0 || k_tok <= 0) return 0;
-  return score_plan(kv, t, h_q, k_tok, logits_given != 0).total;
+  return make_plan(kv, t, h_q, k_tok, !logits_given, false, true, 0).total;
 }
 
 extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q,
@@ -485,50 +858,30 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(!scores || aligned16(scores), "scores must be 16-byte aligned");
-  ScorePlan P = score_plan(kv, t, h_q, k_tok, logits != nullptr);
-  long ncand = (long)P.ns * (k_tok < P.sspan ? k_tok : P.sspan);
-  SF_UNSUPPORTED(ncand <= kMaxCand, "t=%d with k_tok=%d needs %ld candidates (max %d)", t, k_tok,
-                 ncand, kMaxCand);
-  if (ws_bytes < P.total || (P.total > 0 && !ws)) {
-    set_error("workspace: need %zu bytes, got %zu", P.total, ws_bytes);
-    return SF_ERR_WORKSPACE;
-  }
-  SF_REQUIRE(!ws || aligned16(ws), "ws must be 16-byte aligned");
+  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, false, true, 0);
+  st = check_ws(ws, ws_bytes, P.total);
+  if (st != SF_OK) return st;
   char* w = (char*)ws;
   float* lg = logits ? logits : (float*)(w + P.off_logits);
-  float2* part = (float2*)(w + P.off_part);
-  float2* stats = (float2*)(w + P.off_stats);
-  uint64_t* cand = (uint64_t*)(w + P.off_cand);
   cudaStream_t s = as_stream(stream);
-  KvView v = view_of(kv);
-  kv_logits_kernel<<<dim3(P.nl, kv->h_kv, kv->batch), 256, 0, s>>>(v, t, P.lspan, q, h_q, lg, part);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, (float*)(w + P.off_part), P);
+  st = launch_base(kv, a, false, s);
+  if (st != SF_OK) return st;
+  float2* stats = (float2*)(w + P.off_stats);
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>((const float*)(w + P.off_part), P.nsplit, 2, stats);
   SF_LAUNCHED();
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nl, stats);
-  SF_LAUNCHED();
-  size_t smem_l = (size_t)P.sspan * 8;
-  SF_CUDA(cudaFuncSetAttribute(kv_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kMaxSpan * 8));
-  kv_local_kernel<<<dim3(P.ns, kv->h_kv, kv->batch), 1024, smem_l, s>>>(
-      lg, stats, t, P.sspan, h_q, kv->h_kv, k_tok, scores, cand);
-  SF_LAUNCHED();
-  SF_CUDA(cudaFuncSetAttribute(kv_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kMaxCand * 8));
-  kv_final_kernel<<<dim3(kv->h_kv, kv->batch), 1024, (size_t)ncand * 8, s>>>(
-      cand, P.ns, P.sspan, t, kv->h_kv, k_tok, sel);
-  SF_LAUNCHED();
-  return SF_OK;
+  return launch_select(kv, t, h_q, k_tok, P, lg, stats, scores, (uint64_t*)(w + P.off_cand), sel, s);
 }
 
-extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int n_splits) {
+extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
+                                             int n_splits) {
   if (!kv || t <= 0 || h_q <= 0) return 0;
-  int ns = attn_splits(kv, t, n_splits);
-  return (size_t)kv->batch * h_q * ns * (kD + 2) * 4;
+  return make_plan(kv, t, h_q, k_tok, true, true, false, n_splits).total;
 }
 
 extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* q, int h_q,
-                                        const int32_t* sel, int k_tok, const float* base_logits,
-                                        int n_splits, float* out, void* ws, size_t ws_bytes,
-                                        sf_stream_t stream) {
+                                        const int32_t* sel, int k_tok, int n_splits, float* out,
+                                        void* ws, size_t ws_bytes, sf_stream_t stream) {
   sf_status st = check_kv(kv);
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
@@ -537,24 +890,56 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(k_tok == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
   SF_REQUIRE(n_splits >= 0, "n_splits=%d < 0", n_splits);
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
-  SF_REQUIRE(!base_logits || aligned16(base_logits), "base_logits must be 16-byte aligned");
-  int ns = attn_splits(kv, t, n_splits);
-  size_t need = (size_t)kv->batch * h_q * ns * (kD + 2) * 4;
-  if (ws_bytes < need || !ws) {
-    set_error("workspace: need %zu bytes, got %zu", need, ws_bytes);
-    return SF_ERR_WORKSPACE;
-  }
-  SF_REQUIRE(aligned16(ws), "ws must be 16-byte aligned");
-  int span = (t + ns - 1) / ns;
-  ns = (t + span - 1) / span;
+  Plan P = make_plan(kv, t, h_q, k_tok, true, true, false, n_splits);
+  st = check_ws(ws, ws_bytes, P.total);
+  if (st != SF_OK) return st;
+  char* w = (char*)ws;
   cudaStream_t s = as_stream(stream);
-  size_t smem = (size_t)((span + 31) / 32) * 4;
-  SF_UNSUPPORTED(smem <= 64 * 1024, "split of %d tokens too long", span);
-  SF_CUDA(cudaFuncSetAttribute(kv_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
-  kv_attn_kernel<<<dim3(ns, kv->h_kv, kv->batch), 256, smem, s>>>(
-      view_of(kv), t, span, q, h_q, k_tok ? sel : nullptr, k_tok, base_logits, (float*)ws);
+  float* lg = (float*)(w + P.off_logits);
+  float* part = (float*)(w + P.off_part);
+  float2* stats = (float2*)(w + P.off_stats);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
+  st = launch_base(kv, a, true, s);
+  if (st != SF_OK) return st;
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nsplit, kRec, stats);
   SF_LAUNCHED();
-  kv_merge_kernel<<<kv->batch * h_q, kD, 0, s>>>((const float*)ws, ns, out);
+  return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
+                              (float*)(w + P.off_corr), out, s);
+}
+
+extern "C" size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q,
+                                                         int k_tok, int logits_given) {
+  if (!kv || t <= 0 || h_q <= 0 || k_tok <= 0) return 0;
+  return make_plan(kv, t, h_q, k_tok, !logits_given, true, true, 0).total;
+}
+
+extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                            int k_tok, int32_t* sel, float* logits, float* out,
+                                            void* ws, size_t ws_bytes, sf_stream_t stream) {
+  sf_status st = check_kv(kv);
+  if (st != SF_OK) return st;
+  st = check_q(kv, t, q, h_q);
+  if (st != SF_OK) return st;
+  SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
+  SF_UNSUPPORTED(k_tok <= 4096, "k_tok=%d above 4096", k_tok);
+  SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
+  SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
+  SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
+  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0);
+  st = check_ws(ws, ws_bytes, P.total);
+  if (st != SF_OK) return st;
+  char* w = (char*)ws;
+  cudaStream_t s = as_stream(stream);
+  float* lg = logits ? logits : (float*)(w + P.off_logits);
+  float* part = (float*)(w + P.off_part);
+  float2* stats = (float2*)(w + P.off_stats);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
+  st = launch_base(kv, a, true, s);
+  if (st != SF_OK) return st;
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nsplit, kRec, stats);
   SF_LAUNCHED();
-  return SF_OK;
+  st = launch_select(kv, t, h_q, k_tok, P, lg, stats, nullptr, (uint64_t*)(w + P.off_cand), sel, s);
+  if (st != SF_OK) return st;
+  return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
+                              (float*)(w + P.off_corr), out, s);
 }

@@ -9,34 +9,11 @@
 // explicitly rounded operations (no contraction) so that they are bit-exact
 // with the definition in sf.h.
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace sf {
+
 namespace {
-
-struct Grid16 {
-  uint16_t s16, m16;
-  double S, M;
-};
-
-__device__ __forceinline__ Grid16 group_grid(double lo, double hi, int b) {
-  Grid16 g;
-  double step = __ddiv_rn(__dsub_rn(hi, lo), (double)((1 << b) - 1));
-  g.s16 = __half_as_ushort(__double2half(step));  // one rounding, nearest-even
-  g.m16 = __half_as_ushort(__double2half(lo));
-  g.S = h2d(g.s16);
-  g.M = h2d(g.m16);
-  return g;
-}
-
-// (b+r)-bit nested code Q of one value: floor((u + 1/2) * 2^r), clamped.
-__device__ __forceinline__ int nested_code(double w, const Grid16& g, int r, int qmax) {
-  if (g.S == 0.0) return 0;
-  double u = __ddiv_rn(__dsub_rn(w, g.M), g.S);
-  double t = __dadd_rn(u, 0.5);
-  double f = floor(__dmul_rn(t, (double)(1 << r)));
-  f = fmin(fmax(f, 0.0), (double)qmax);
-  return (int)f;
-}
 
 // Bit position of channel c (0..31) in the high-bit word of a 3-bit base block.
 __device__ __forceinline__ int hi_plane_bit(int c) {
@@ -118,58 +95,6 @@ __global__ void unpack_weights_kernel(const uint32_t* __restrict__ base,
   }
 }
 
-// One thread per (batch, head, token, group of 32 elements).  A group's codes
-// fill whole 32-bit words in both streams, so no two threads share a word.
-__global__ void pack_kv_kernel(const uint16_t* __restrict__ x, int BH, int nt, int t_max, int t0,
-                               int D, int b, int r, uint32_t* __restrict__ codes,
-                               uint32_t* __restrict__ refine, uint16_t* __restrict__ sz) {
-  long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  int gpt = D / 32;
-  if (idx >= (long)BH * nt * gpt) return;
-  int j = (int)(idx % gpt);
-  long tok = idx / gpt;
-  int t = (int)(tok % nt);
-  long bh = tok / nt;
-  const uint16_t* src = x + (bh * nt + t) * D + j * 32;
-  double lo = h2d(src[0]), hi = lo;
-  for (int c = 1; c < 32; c++) {
-    double v = h2d(src[c]);
-    if (v < lo) lo = v;
-    if (v > hi) hi = v;
-  }
-  Grid16 g = group_grid(lo, hi, b);
-  long slot = bh * t_max + t0 + t;  // cache token index
-  sz[(slot * gpt + j) * 2 + 0] = g.s16;
-  sz[(slot * gpt + j) * 2 + 1] = g.m16;
-  const int qmax = (1 << (b + r)) - 1;
-  uint32_t cw[4] = {0, 0, 0, 0}, rw[2] = {0, 0};
-  for (int c = 0; c < 32; c++) {
-    int Q = nested_code(h2d(src[c]), g, r, qmax);
-    int q = Q >> r, rho = Q & ((1 << r) - 1);
-    int cb = c * b, rb = c * r;
-    cw[cb >> 5] |= (uint32_t)q << (cb & 31);
-    rw[rb >> 5] |= (uint32_t)rho << (rb & 31);
-  }
-  uint32_t* cdst = codes + (slot * D + j * 32) * b / 32;
-  for (int i = 0; i < b; i++) cdst[i] = cw[i];
-  uint32_t* rdst = refine + (slot * D + j * 32) * r / 32;
-  for (int i = 0; i < r; i++) rdst[i] = rw[i];
-}
-
-__global__ void unpack_kv_kernel(const uint32_t* __restrict__ codes,
-                                 const uint32_t* __restrict__ refine, int BH, int t, int t_max,
-                                 int D, int b, int r, uint8_t* __restrict__ qb,
-                                 uint8_t* __restrict__ rho) {
-  long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long)BH * t * D) return;
-  int d = (int)(idx % D);
-  long tok = idx / D;
-  long slot = (tok / t) * t_max + tok % t;
-  long e = slot * D + d;
-  qb[idx] = (uint8_t)((codes[e * b / 32] >> ((e * b) & 31)) & ((1u << b) - 1));
-  if (rho) rho[idx] = (uint8_t)((refine[e * r / 32] >> ((e * r) & 31)) & ((1u << r) - 1));
-}
-
 sf_status check_wq(const sf_wq* w, bool need_refine) {
   SF_REQUIRE(w != nullptr, "null sf_wq");
   SF_REQUIRE(w->n > 0 && w->k > 0, "bad shape n=%d k=%d", w->n, w->k);
@@ -237,48 +162,6 @@ sf_status sf_unpack_codes(const sf_wq* w, uint8_t* qb, uint8_t* rho, sf_stream_t
                           as_stream(stream)>>>((const uint32_t*)w->base,
                                                (const uint32_t*)w->refine, w->n, w->k, w->b, w->r,
                                                qb, w->refine ? rho : nullptr);
-  SF_LAUNCHED();
-  return SF_OK;
-}
-
-sf_status sf_kv_pack_tokens(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0,
-                            int nt, sf_stream_t stream) {
-  sf_status st = check_kv(kv);
-  if (st != SF_OK) return st;
-  SF_REQUIRE(nt >= 0 && t0 >= 0 && t0 + nt <= kv->t_max, "tokens [%d, %d) outside t_max=%d", t0,
-             t0 + nt, kv->t_max);
-  if (nt == 0) return SF_OK;
-  int BH = kv->batch * kv->h_kv;
-  long total = (long)BH * nt * (kv->d / 32);
-  int threads = 128;
-  unsigned blocks = (unsigned)((total + threads - 1) / threads);
-  cudaStream_t s = as_stream(stream);
-  if (k) {
-    pack_kv_kernel<<<blocks, threads, 0, s>>>(k, BH, nt, kv->t_max, t0, kv->d, kv->b, kv->r,
-                                              (uint32_t*)kv->kb, (uint32_t*)kv->kr, kv->ksz);
-    SF_LAUNCHED();
-  }
-  if (v) {
-    pack_kv_kernel<<<blocks, threads, 0, s>>>(v, BH, nt, kv->t_max, t0, kv->d, kv->b, kv->r,
-                                              (uint32_t*)kv->vb, (uint32_t*)kv->vr, kv->vsz);
-    SF_LAUNCHED();
-  }
-  return SF_OK;
-}
-
-sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* qb, uint8_t* rho,
-                             sf_stream_t stream) {
-  sf_status st = check_kv(kv);
-  if (st != SF_OK) return st;
-  SF_REQUIRE(which == 0 || which == 1, "which must be 0 (keys) or 1 (values)");
-  SF_REQUIRE(t > 0 && t <= kv->t_max, "t=%d outside (0, t_max]", t);
-  SF_REQUIRE(qb != nullptr, "qb must be non-null");
-  int BH = kv->batch * kv->h_kv;
-  long total = (long)BH * t * kv->d;
-  int threads = 256;
-  unpack_kv_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, as_stream(stream)>>>(
-      (const uint32_t*)(which ? kv->vb : kv->kb), (const uint32_t*)(which ? kv->vr : kv->kr), BH, t,
-      kv->t_max, kv->d, kv->b, kv->r, qb, rho);
   SF_LAUNCHED();
   return SF_OK;
 }

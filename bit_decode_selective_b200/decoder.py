@@ -1,0 +1,273 @@
+"""A Llama-shaped decode step built from the refined kernels.
+
+Every step of the computation runs in the CUDA library (include/sf.h); this
+module only owns the buffers (allocated with PyTorch), the streams and events,
+and the order of the calls.  The call order implements the schedule of
+"StrataFlux -- Selective precision streaming -- What does it mean?":
+  which-tiles-count paragraph -- every projection refines the k channels with
+    the largest |x| per 1,024-channel chunk; attention refines the
+    highest-scoring tokens per KV head;
+  the-map-app-also-loads-tiles paragraph -- refinement rows live in host RAM;
+    fetch lead (1 layer) selects a projection's channels from the previous
+    layer's activation and starts the row transfer on a side stream while the
+    layers in between compute; fetch lag (1 layer) applies the residual-writing
+    projections' (o, down) corrections at the start of the next layer.
+Readings as in the oracle (oracle/decoder.py): layer 0 selects from its own
+activations; q/k/v and gate/up correct in place; the new token is appended at
+position T and attention runs over T + 1 tokens.
+
+step() only enqueues work on the current stream (plus the side stream), so it
+can be captured in a CUDA graph and replayed.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import abi
+from .abi import check
+from .ops import KVCache, QuantWeights, _p
+
+
+@dataclass
+class DecoderConfig:
+    n_layers: int = 32
+    hidden: int = 4096
+    inter: int = 14336
+    h_q: int = 32
+    h_kv: int = 8
+    d: int = 128
+    vocab: int = 128256
+    w_bits: int = 2
+    w_refine: int = 2
+    group: int = 128
+    chunk: int = 1024
+    kch: int = 32
+    kv_bits: int = 2
+    kv_refine: int = 2
+    k_tok: int = 512
+    lead: int = 1
+    lag: int = 1
+    host_refine: bool = True  # refinement rows in pinned host memory, staged per layer
+    eps: float = 1e-5
+    theta: float = 500000.0
+
+    def shapes(self):
+        """(name, n, k) of the four fused projections of a layer."""
+        qkv = (self.h_q + 2 * self.h_kv) * self.d
+        return (("qkv", qkv, self.hidden), ("o", self.hidden, self.h_q * self.d),
+                ("gate_up", 2 * self.inter, self.hidden), ("down", self.hidden, self.inter))
+
+
+PROJ = ("qkv", "o", "gate_up", "down")
+
+
+def _s(stream):
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Decoder:
+    def __init__(self, cfg: DecoderConfig, batch: int, t: int, device="cuda"):
+        self.cfg, self.B, self.T = cfg, batch, t
+        self.dev = torch.device(device)
+        dev = self.dev
+        self.t_max = (t + 1 + 15) // 16 * 16
+        self.layers = []
+        self.host_rows = []   # per layer: name -> pinned [k][n*r/8] uint8
+        f32 = lambda *s: torch.zeros(*s, dtype=torch.float32, device=dev)
+        f16 = lambda *s: torch.zeros(*s, dtype=torch.float16, device=dev)
+        i32 = lambda *s: torch.zeros(*s, dtype=torch.int32, device=dev)
+        shp = {n: (nn, kk) for n, nn, kk in cfg.shapes()}
+        self.shp = shp
+        self.n_sel = {n: (shp[n][1] // cfg.chunk) * cfg.kch for n in PROJ}
+        self.row_bytes = {n: shp[n][0] * cfg.w_refine // 8 for n in PROJ}
+        B = batch
+        # activations
+        self.h = f32(B, cfg.hidden)
+        self.x_attn = f16(B, cfg.hidden)
+        self.qkv_out = f32(B, shp["qkv"][0])
+        self.q = f16(B, cfg.h_q, cfg.d)
+        self.k_new = f16(B, cfg.h_kv, 1, cfg.d)
+        self.v_new = f16(B, cfg.h_kv, 1, cfg.d)
+        self.attn = f32(B, cfg.h_q, cfg.d)
+        self.x_o = [f16(B, cfg.h_q * cfg.d) for _ in range(2)]
+        self.o_out = f32(B, cfg.hidden)
+        self.x_mlp = f16(B, cfg.hidden)
+        self.gu_out = f32(B, 2 * cfg.inter)
+        self.x_down = [f16(B, cfg.inter) for _ in range(2)]
+        self.down_out = f32(B, cfg.hidden)
+        self.x_final = f16(B, cfg.hidden)
+        self.logits = f32(B, cfg.vocab)
+        self.tok_sel = i32(B, cfg.h_kv, cfg.k_tok)
+        # selections (two slots: this layer / next layer) and staged rows
+        self.sel = {n: [i32(B, self.n_sel[n]) for _ in range(2)] for n in PROJ}
+        if cfg.kch and cfg.host_refine:
+            self.slots = {n: [torch.empty(B * self.n_sel[n] * self.row_bytes[n], dtype=torch.uint8, device=dev)
+                              for _ in range(2)] for n in PROJ}
+        else:
+            self.slots = None
+        self.side = torch.cuda.Stream(device=dev)
+        self.ev_sel = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
+        self.ev_stage = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
+        self.lm_head = None
+        self.ws = None
+
+    # ---- model state -----------------------------------------------------
+
+    def load_layer(self, weights: dict, k_cache: torch.Tensor, v_cache: torch.Tensor):
+        """weights: name -> fp32 [n][k] on the device; k/v_cache fp16
+        [B][h_kv][T][d] on the device (the T cached tokens)."""
+        cfg = self.cfg
+        L = {}
+        host = {}
+        for n in PROJ:
+            w = weights[n]
+            qw = QuantWeights.pack(w.contiguous(), cfg.w_bits, cfg.w_refine, cfg.group)
+            if cfg.host_refine:
+                rows = torch.empty(qw.refine.numel(), dtype=torch.uint8, pin_memory=True)
+                rows.copy_(qw.refine)
+                host[n] = rows
+                qw.refine = None
+                qw.desc.refine = None
+            L[n] = qw
+        kv = KVCache(self.B, cfg.h_kv, self.t_max, cfg.kv_bits, cfg.kv_refine, cfg.d, device=self.dev)
+        kv.pack_tokens(k_cache.contiguous(), v_cache.contiguous(), 0)
+        L["kv"] = kv
+        self.layers.append(L)
+        self.host_rows.append(host)
+        torch.cuda.synchronize(self.dev)
+
+    def set_lm_head(self, lm_fp16: torch.Tensor):
+        self.lm_head = lm_fp16.contiguous()
+        kv = self.layers[0]["kv"]
+        need = kv.attend_workspace(self.T + 1, self.cfg.h_q, self.cfg.k_tok, False)
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=self.dev)
+
+    # ---- the step ----------------------------------------------------------
+
+    def _select(self, name, x, slot, stream):
+        cfg = self.cfg
+        check(abi.sf_select_channels(_p(x), self.B, self.shp[name][1], cfg.chunk, cfg.kch,
+                                     _p(self.sel[name][slot]), _s(stream)), "sf_select_channels")
+
+    def _stage(self, layer, name, slot, main):
+        """Copy layer `layer`'s rows of the selection in `slot` into staging
+        slot `slot` on the side stream, after the selection is done."""
+        ev = self.ev_sel[name][slot]
+        ev.record(main)
+        self.side.wait_event(ev)
+        check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
+                                       _p(self.sel[name][slot]), self.B * self.n_sel[name],
+                                       _p(self.slots[name][slot]), _s(self.side), None),
+              "sf_stage_refinements")
+        self.ev_stage[name][slot].record(self.side)
+
+    def _rows(self, name, slot, main):
+        if self.slots is None:
+            return None
+        main.wait_event(self.ev_stage[name][slot])
+        return self.slots[name][slot]
+
+    def _proj(self, layer, name, x, y, slot, main, base_only=False):
+        """y = W~ x for layer `layer` with the selection in `slot` (lead) or
+        selected here (no lead / layer 0)."""
+        cfg = self.cfg
+        qw = self.layers[layer][name]
+        if cfg.kch == 0 or base_only:
+            check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, 0, None, None, None,
+                                      _p(y), None, 0, _s(main)), "sf_gemv_refined")
+            return
+        rows = self._rows(name, slot, main)
+        check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
+                                  _p(self.sel[name][slot]), None, _p(rows), _p(y), None, 0, _s(main)),
+              "sf_gemv_refined")
+
+    def _prepare(self, layer, name, x, main):
+        """Make sure the selection and staged rows of (layer, name) exist in
+        slot layer % 2 before the projection runs."""
+        cfg = self.cfg
+        if cfg.kch == 0:
+            return
+        slot = layer % 2
+        if not cfg.lead or layer == 0:
+            self._select(name, x, slot, main)
+            if self.slots is not None:
+                self._stage(layer, name, slot, main)
+
+    def _lead(self, layer, name, x, main):
+        """Fetch lead: select (layer + 1)'s channels from this activation and
+        start their transfer."""
+        cfg = self.cfg
+        if cfg.kch == 0 or not cfg.lead or layer + 1 >= cfg.n_layers:
+            return
+        slot = (layer + 1) % 2
+        self._select(name, x, slot, main)
+        if self.slots is not None:
+            self._stage(layer + 1, name, slot, main)
+
+    def _lagged(self, layer, main):
+        """Fetch lag: layer `layer`'s o and down corrections into the residual."""
+        cfg = self.cfg
+        if cfg.kch == 0 or not cfg.lag:
+            return
+        slot = layer % 2
+        for name, x in (("o", self.x_o[slot]), ("down", self.x_down[slot])):
+            qw = self.layers[layer][name]
+            rows = self._rows(name, slot, main)
+            check(abi.sf_gemv_correction(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
+                                         _p(self.sel[name][slot]), _p(rows), _p(self.h), _s(main)),
+                  "sf_gemv_correction")
+
+    def step(self, hidden: torch.Tensor):
+        """Enqueue one decode step: hidden fp16 [B][hidden] -> self.logits."""
+        cfg = self.cfg
+        main = torch.cuda.current_stream(self.dev)
+        self.side.wait_stream(main)
+        B, T = self.B, self.T
+        check(abi.sf_widen_f16(_p(hidden), B * cfg.hidden, _p(self.h), _s(main)), "sf_widen_f16")
+        add = None
+        for l in range(cfg.n_layers):
+            slot = l % 2
+            L = self.layers[l]
+            if l > 0:
+                self._lagged(l - 1, main)
+            check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), None, B, cfg.hidden, cfg.eps, _p(self.x_attn),
+                                          _s(main)), "sf_rmsnorm_residual")
+            # attention block
+            self._prepare(l, "qkv", self.x_attn, main)
+            self._proj(l, "qkv", self.x_attn, self.qkv_out, slot, main)
+            self._lead(l, "qkv", self.x_attn, main)
+            check(abi.sf_rope_split(_p(self.qkv_out), B, cfg.h_q, cfg.h_kv, cfg.d, T, cfg.theta, _p(self.q),
+                                    _p(self.k_new), _p(self.v_new), _s(main)), "sf_rope_split")
+            kv = L["kv"]
+            check(abi.sf_kv_pack_tokens(ctypes.byref(kv.desc), _p(self.k_new), _p(self.v_new), T, 1, _s(main)),
+                  "sf_kv_pack_tokens")
+            check(abi.sf_kv_attend_selective(ctypes.byref(kv.desc), T + 1, _p(self.q), cfg.h_q, cfg.k_tok,
+                                             _p(self.tok_sel), None, _p(self.attn), _p(self.ws), self.ws.numel(),
+                                             _s(main)), "sf_kv_attend_selective")
+            x_o = self.x_o[slot]
+            check(abi.sf_cast_f16(_p(self.attn), B * cfg.h_q * cfg.d, _p(x_o), _s(main)), "sf_cast_f16")
+            self._prepare(l, "o", x_o, main)
+            self._proj(l, "o", x_o, self.o_out, slot, main, base_only=bool(cfg.lag))
+            self._lead(l, "o", x_o, main)
+            check(abi.sf_rmsnorm_residual(_p(self.h), _p(self.o_out), None, B, cfg.hidden, cfg.eps,
+                                          _p(self.x_mlp), _s(main)), "sf_rmsnorm_residual")
+            # MLP block
+            self._prepare(l, "gate_up", self.x_mlp, main)
+            self._proj(l, "gate_up", self.x_mlp, self.gu_out, slot, main)
+            self._lead(l, "gate_up", self.x_mlp, main)
+            x_down = self.x_down[slot]
+            check(abi.sf_silu_mul(_p(self.gu_out), B, cfg.inter, _p(x_down), _s(main)), "sf_silu_mul")
+            self._prepare(l, "down", x_down, main)
+            self._proj(l, "down", x_down, self.down_out, slot, main, base_only=bool(cfg.lag))
+            self._lead(l, "down", x_down, main)
+            add = self.down_out
+        self._lagged(cfg.n_layers - 1, main)
+        check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), None, B, cfg.hidden, cfg.eps, _p(self.x_final),
+                                      _s(main)), "sf_rmsnorm_residual")
+        check(abi.sf_gemv_f16(_p(self.lm_head), _p(self.x_final), B, cfg.vocab, cfg.hidden, _p(self.logits),
+                              _s(main)), "sf_gemv_f16")
+        main.wait_stream(self.side)
+        return self.logits

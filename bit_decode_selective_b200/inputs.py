@@ -124,3 +124,48 @@ def kv_case(seed: int = 2, t: int = 8192, h_kv: int = N_KV_HEADS, h_q: int = N_H
     k, v = kv_values(rng, h_kv, t, d, batch)
     q = query(rng, h_q, d, batch)
     return k, v, q
+
+
+# ---------------------------------------------------------------------------
+# a Llama-shaped decoder (the full decode-step workload)
+
+def decoder_layer_weights(seed: int, layer: int, hidden: int = HIDDEN, inter: int = INTER,
+                          h_q: int = N_HEADS, h_kv: int = N_KV_HEADS, d: int = HEAD_DIM):
+    """fp32 weights of one layer, projections sharing an input concatenated:
+    qkv [(h_q + 2 h_kv) d][hidden], o [hidden][h_q d], gate_up [2 inter][hidden],
+    down [hidden][inter].  Seed: seed * 1000 + layer."""
+    rng = np.random.default_rng(seed * 1000 + layer)
+    return {
+        "qkv": weight(rng, (h_q + 2 * h_kv) * d, hidden),
+        "o": weight(rng, hidden, h_q * d),
+        "gate_up": weight(rng, 2 * inter, hidden),
+        "down": weight(rng, hidden, inter),
+    }
+
+
+def decoder_layer_kv(seed: int, layer: int, t: int, batch: int = 1, h_kv: int = N_KV_HEADS,
+                     d: int = HEAD_DIM):
+    """The layer's cached keys and values (fp16 [batch][h_kv][t][d]), drawn as
+    for the KV workloads.  Seed: seed * 1000 + 500 + layer."""
+    rng = np.random.default_rng(seed * 1000 + 500 + layer)
+    return kv_values(rng, h_kv, t, d, batch)
+
+
+def decoder_io(seed: int, batch: int = 1, hidden: int = HIDDEN, vocab: int = VOCAB):
+    """(input hidden state fp16 [batch][hidden], LM head fp16 [vocab][hidden])."""
+    rng = np.random.default_rng(seed * 1000 + 999)
+    h = rng.normal(0.0, 1.0, size=(batch, hidden)).astype(np.float16)
+    lm = rng.normal(0.0, 0.02, size=(vocab, hidden)).astype(np.float16)
+    return h, lm
+
+
+def torch_normal(shape, std: float, seed: int, device="cuda", dtype=None):
+    """Seeded N(0, std) drawn on the device with torch's Philox generator (used
+    where a workload is too large to draw on the host in reasonable time)."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    t.mul_(std)
+    return t if dtype is None else t.to(dtype)

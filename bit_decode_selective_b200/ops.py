@@ -71,6 +71,15 @@ class QuantWeights:
               "sf_gemv_refined")
         return y, (sel_in if sel_in is not None else sel_out)
 
+    def correction(self, x: torch.Tensor, sel, y, chunk: int = 1024, kch: int = 32,
+                   refine_rows=None, stream=None):
+        """y += (W~ - W^) x over the selected channels (sf_gemv_correction)."""
+        x = _f16(x if x.dim() == 2 else x.view(1, -1))
+        check(abi.sf_gemv_correction(ctypes.byref(self.desc), _p(x), x.shape[0], chunk, kch, _p(sel),
+                                     _p(refine_rows), _p(y), _stream(stream)),
+              "sf_gemv_correction")
+        return y
+
 
 def select_channels(x: torch.Tensor, chunk: int = 1024, kch: int = 32, sel=None, stream=None):
     x = _f16(x if x.dim() == 2 else x.view(1, -1))
@@ -90,11 +99,11 @@ class KVCache:
         sizes = [ctypes.c_size_t() for _ in range(3)]
         check(abi.sf_kv_bytes(batch, h_kv, d, t_max, b, r, group, *[ctypes.byref(s) for s in sizes]),
               "sf_kv_bytes")
-        mk = lambda nbytes: torch.empty(nbytes, dtype=torch.uint8, device=device)
+        mk = lambda nbytes: torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.batch, self.h_kv, self.t_max, self.b, self.r, self.d, self.group = batch, h_kv, t_max, b, r, d, group
         self.kb, self.kr, self.vb, self.vr = mk(sizes[0].value), mk(sizes[1].value), mk(sizes[0].value), mk(sizes[1].value)
-        self.ksz = torch.empty(sizes[2].value // 2, dtype=torch.int16, device=device)
-        self.vsz = torch.empty(sizes[2].value // 2, dtype=torch.int16, device=device)
+        self.ksz = torch.zeros(sizes[2].value // 2, dtype=torch.int16, device=device)
+        self.vsz = torch.zeros(sizes[2].value // 2, dtype=torch.int16, device=device)
         self.desc = abi.sf_kv(batch, h_kv, d, t_max, b, r, group, self.kb.data_ptr(), self.kr.data_ptr(),
                               self.vb.data_ptr(), self.vr.data_ptr(), self.ksz.data_ptr(), self.vsz.data_ptr())
 
@@ -136,20 +145,41 @@ class KVCache:
               "sf_kv_score_select")
         return sel, logits, scores
 
-    def attn_workspace(self, t: int, h_q: int, n_splits: int = 0) -> int:
-        return abi.sf_kv_attn_workspace_bytes(ctypes.byref(self.desc), t, h_q, n_splits)
+    def attn_workspace(self, t: int, h_q: int, k_tok: int, n_splits: int = 0) -> int:
+        return abi.sf_kv_attn_workspace_bytes(ctypes.byref(self.desc), t, h_q, k_tok, n_splits)
 
-    def attn_refined(self, q: torch.Tensor, t: int, sel, k_tok: int, base_logits=None,
-                     n_splits: int = 0, out=None, ws=None, stream=None):
+    def attn_refined(self, q: torch.Tensor, t: int, sel, k_tok: int, n_splits: int = 0, out=None,
+                     ws=None, stream=None):
         q = _f16(q)
         h_q = q.shape[1]
         if out is None:
             out = torch.empty((self.batch, h_q, self.d), dtype=torch.float32, device=q.device)
-        need = self.attn_workspace(t, h_q, n_splits)
+        need = self.attn_workspace(t, h_q, k_tok, n_splits)
         if ws is None:
             ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-        check(abi.sf_kv_attn_refined(ctypes.byref(self.desc), t, _p(q), h_q, _p(sel), k_tok,
-                                     _p(base_logits), n_splits, _p(out), _p(ws), ws.numel(),
-                                     _stream(stream)),
+        check(abi.sf_kv_attn_refined(ctypes.byref(self.desc), t, _p(q), h_q, _p(sel), k_tok, n_splits,
+                                     _p(out), _p(ws), ws.numel(), _stream(stream)),
               "sf_kv_attn_refined")
         return out
+
+    def attend_workspace(self, t: int, h_q: int, k_tok: int, logits_given: bool) -> int:
+        return abi.sf_kv_attend_selective_workspace_bytes(ctypes.byref(self.desc), t, h_q, k_tok,
+                                                          int(logits_given))
+
+    def attend_selective(self, q: torch.Tensor, t: int, k_tok: int, sel=None, logits=None,
+                         out=None, ws=None, stream=None):
+        """Score, select and attend in one call.  Returns (out, sel)."""
+        q = _f16(q)
+        h_q = q.shape[1]
+        dev = q.device
+        if out is None:
+            out = torch.empty((self.batch, h_q, self.d), dtype=torch.float32, device=dev)
+        if sel is None:
+            sel = torch.empty((self.batch, self.h_kv, k_tok), dtype=torch.int32, device=dev)
+        need = self.attend_workspace(t, h_q, k_tok, logits is not None)
+        if ws is None:
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        check(abi.sf_kv_attend_selective(ctypes.byref(self.desc), t, _p(q), h_q, k_tok, _p(sel),
+                                         _p(logits), _p(out), _p(ws), ws.numel(), _stream(stream)),
+              "sf_kv_attend_selective")
+        return out, sel

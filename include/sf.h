@@ -157,6 +157,17 @@ SF_API sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, i
                           float* y, void* ws, size_t ws_bytes, sf_stream_t stream);
 SF_API size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch);
 
+/* The refinement correction of a GEMV on its own, ADDED into y:
+ *   y[b][i] += sum_{c in sel[b]} x[b][c] * (w~[i][c] - w^[i][c]).
+ * This is the fetch-lag form ([EXPL] "the map app also loads tiles": the
+ * correction is applied one or more layers later than the base product, so
+ * the refinement transfer has longer to land): run sf_gemv_refined with
+ * kch = 0 for the base product, and this call once the rows are resident.
+ * Arguments as sf_gemv_refined; sel is required (kch = 0: no-op). */
+SF_API sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch, int chunk,
+                                    int kch, const int32_t* sel, const void* refine_rows,
+                                    float* y, sf_stream_t stream);
+
 /* ======================================================================== */
 /* KV cache                                                                  */
 /* ======================================================================== */
@@ -164,10 +175,20 @@ SF_API size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int 
 /* `batch` independent caches of h_kv heads with room for t_max tokens of d
  * elements, quantised per token in groups of `group` consecutive elements.
  *   d == 128, group == 32, b in {2,4}, r in {1,2}, t_max % 16 == 0.
- * kb, vb: [batch][h_kv][t_max] tokens, each a natural b-bit stream of its d
- *   codes (d*b/8 bytes).
- * kr, vr: same with the r-bit refinement codes (d*r/8 bytes per token).
- * ksz, vsz: [batch][h_kv][t_max][d/group][2] fp16 (s, m). */
+ * Codes (w = b bits) and refinements (w = r bits) use a pair-slot layout laid
+ * out for the tensor-core fragments that consume them: a little-endian 32-bit
+ * word holds 16/w pairs of w-bit codes; pair slot j keeps its first code at
+ * bits [w*j, w*j + w) and its second at bits [16 + w*j, 16 + w*j + w).
+ *   kb, kr: per token (16*w bytes), 4 chunks c = 0..3 of w words each; pair
+ *     p = 2*s + e (s = 0..7, e = 0..1) of chunk c (word p/(16/w) of the chunk,
+ *     slot p%(16/w)) holds dims 16*s + 2*c + 8*e (first) and 16*s + 2*c + 8*e + 1
+ *     (second).  Tokens are consecutive: [batch][h_kv][t_max][16*w bytes].
+ *   vb, vr: per tile of 16 consecutive tokens 16*u .. 16*u + 15 (256*w bytes),
+ *     32 chunks l = 4*g + c (g = 0..7, c = 0..3) of 2*w words each; pair
+ *     p = 16*h + 2*m + e (h, e = 0..1, m = 0..7) of chunk l holds dim
+ *     16*m + g + 8*e of tokens 16*u + 2*c + 8*h (first) and 16*u + 2*c + 8*h + 1
+ *     (second).  [batch][h_kv][t_max/16][256*w bytes].
+ * ksz, vsz: [batch][h_kv][t_max][d/group][2] fp16 (s, m) per token and group. */
 typedef struct {
   int32_t batch, h_kv, d, t_max, b, r, group;
   void *kb, *kr, *vb, *vr;
@@ -195,8 +216,7 @@ SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* 
  *   sel[g] = the k_tok tokens with the highest score (equal scores: lower
  *            token first), ascending.
  *   q [batch][h_q][d] fp16;  sel [batch][h_kv][k_tok] int32.
- *   logits (nullable): receives the base logits [batch][h_q][t] fp32; pass the
- *     same buffer to sf_kv_attn_refined so it need not re-read the keys.
+ *   logits (nullable): receives the base logits [batch][h_q][t] fp32.
  *   scores (nullable): receives score [batch][h_kv][t] fp32.
  *   1 <= t <= t_max, 1 <= k_tok <= min(t, 4096), h_q % h_kv == 0,
  *   h_q / h_kv <= 8. */
@@ -206,23 +226,35 @@ SF_API sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, i
 SF_API size_t sf_kv_score_select_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                           int logits_given);
 
-/* Refined attention ([EXPL] "which tiles count", "nested quantization"):
+/* Refined attention for a given selection ([EXPL] "which tiles count",
+ * "nested quantization"):
  *   out[h] = sum_t softmax_t(q[h] . k~[t] / sqrt(d)) v~[t]
  * over all t tokens, where k~, v~ are the refined values for the tokens in
  * sel[g] (g the KV head of h) and the base values for every other token.
- * The context is split into n_splits parts (0: automatic) whose partial
- * (max, sum, weighted values) are merged by log-sum-exp; the result does not
- * depend on the split count beyond fp32 rounding.
- *   sel [batch][h_kv][k_tok] ascending (k_tok may be 0: base attention);
- *   base_logits (nullable): the logits written by sf_kv_score_select for the
- *     same q, cache and t; unselected tokens then use them instead of
- *     re-reading their keys;
+ * One pass over the cache computes the base attention split over the
+ * context (n_splits parts, 0 = automatic); the selected tokens' base
+ * contributions are then replaced by their refined ones and the parts are
+ * merged by log-sum-exp.  The result does not depend on n_splits beyond fp32
+ * rounding.
+ *   sel [batch][h_kv][k_tok] (k_tok may be 0: base attention);
  *   out [batch][h_q][d] fp32. */
 SF_API sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* q, int h_q,
-                             const int32_t* sel, int k_tok, const float* base_logits,
-                             int n_splits, float* out, void* ws, size_t ws_bytes,
-                             sf_stream_t stream);
-SF_API size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int n_splits);
+                                    const int32_t* sel, int k_tok, int n_splits, float* out,
+                                    void* ws, size_t ws_bytes, sf_stream_t stream);
+SF_API size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
+                                         int n_splits);
+
+/* Score, select and attend in one call (the decode-step form of the two calls
+ * above): the base pass over the cache yields the base logits, the softmax
+ * statistics and the base attention at once; the tokens are then scored and
+ * selected exactly as sf_kv_score_select does, and the selected tokens'
+ * contributions are swapped for their refined ones as in sf_kv_attn_refined.
+ * The cache is read once.  sel, logits (nullable) and out as above. */
+SF_API sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                        int k_tok, int32_t* sel, float* logits, float* out,
+                                        void* ws, size_t ws_bytes, sf_stream_t stream);
+SF_API size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
+                                                     int logits_given);
 
 /* ======================================================================== */
 /* Refinement staging ([EXPL] "the map app also loads tiles": fetch lead)    */
@@ -244,6 +276,36 @@ SF_API sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, c
 SF_API sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes,
                                     const int32_t* sel_host, int n_sel, void* dst,
                                     sf_stream_t stream, sf_event_t done);
+
+/* ======================================================================== */
+/* Decoder-step glue (standard Llama operations around the refined ones)     */
+/* ======================================================================== */
+
+/* h[b] += add0[b] + add1[b] (each nullable), then x[b] = fp16(h[b] /
+ * sqrt(mean(h[b]^2) + eps)) (RMSNorm with unit weights).  h [batch][n] fp32,
+ * x [batch][n] fp16. */
+SF_API sf_status sf_rmsnorm_residual(float* h, const float* add0, const float* add1, int batch,
+                                     int n, float eps, uint16_t* x, sf_stream_t stream);
+
+/* qkv [batch][(h_q + 2 h_kv) d] fp32 -> q [batch][h_q][d], k, v [batch][h_kv][d]
+ * fp16; q and k turned by the rotary embedding (pairs (i, i + d/2), angle
+ * pos * theta^(-2i/d), computed in fp64). */
+SF_API sf_status sf_rope_split(const float* qkv, int batch, int h_q, int h_kv, int d, int pos,
+                               float theta, uint16_t* q, uint16_t* k, uint16_t* v,
+                               sf_stream_t stream);
+
+/* out[b][i] = fp16(silu(gu[b][i]) * gu[b][inter + i]). */
+SF_API sf_status sf_silu_mul(const float* gu, int batch, int inter, uint16_t* out,
+                             sf_stream_t stream);
+
+/* y = fp16(x) and y = fp32(x) element-wise. */
+SF_API sf_status sf_cast_f16(const float* x, size_t n, uint16_t* y, sf_stream_t stream);
+SF_API sf_status sf_widen_f16(const uint16_t* x, size_t n, float* y, sf_stream_t stream);
+
+/* y[b][i] = sum_c w[i][c] x[b][c] with fp16 w [n][k] and x [batch][k], fp32
+ * accumulation (the LM head).  1 <= batch <= 8, k % 8 == 0. */
+SF_API sf_status sf_gemv_f16(const uint16_t* w, const uint16_t* x, int batch, int n, int k,
+                             float* y, sf_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -46,13 +46,18 @@ def _declare(L):
         "or_quant_weights": ([vp, i, i, i, i, i, vp, vp, vp], None),
         "or_quant_kv": ([vp, i, i, i, i, i, i, i, vp, vp, vp], None),
         "or_pack_weights": ([vp, vp, i, i, i, i, vp, vp], None),
-        "or_pack_kv": ([vp, vp, i, i, i, i, i, i, i, vp, vp], None),
+        "or_pack_kv": ([vp, vp, i, i, i, i, i, i, i, i, vp, vp], None),
         "or_select_chunks": ([vp, i, i, i, i, vp], None),
         "or_gemv_refined": ([vp, vp, vp, i, i, i, i, vp, i, vp, i, i, vp], None),
         "or_kv_logits": ([vp, vp, i, i, i, i, i, vp, i, vp], None),
         "or_kv_scores": ([vp, i, i, i, i, vp], None),
         "or_kv_select": ([vp, i, i, i, i, vp], None),
         "or_kv_attention": ([vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i, vp, i, vp], None),
+        "or_rmsnorm_f16": ([vp, i, d, vp], None),
+        "or_rope": ([vp, i, i, i, d], None),
+        "or_silu_mul_f16": ([vp, i, vp], None),
+        "or_gemv_f16": ([vp, vp, i, i, vp], None),
+        "or_gemv_correction": ([vp, vp, vp, i, i, i, i, vp, vp, i, vp], None),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -155,14 +160,16 @@ def pack_weights(qb, rho, b: int, r: int):
     return base, refine
 
 
-def pack_kv(qb, rho, b: int, r: int, t_max: int | None = None):
+def pack_kv(qb, rho, which: int, b: int, r: int, t_max: int | None = None):
+    """Packed bytes of keys (which=0) or values (which=1) in the pair-slot layout."""
     B, H, T, D = qb.shape
     t_max = T if t_max is None else t_max
+    assert D == 128 and t_max % 16 == 0
     qb = np.ascontiguousarray(qb, np.uint8)
     rho = np.ascontiguousarray(rho, np.uint8)
     base = np.empty(B * H * t_max * D * b // 8, np.uint8)
     refine = np.empty(B * H * t_max * D * r // 8, np.uint8)
-    lib().or_pack_kv(_p(qb), _p(rho), B, H, T, t_max, D, b, r, _p(base), _p(refine))
+    lib().or_pack_kv(_p(qb), _p(rho), which, B, H, T, t_max, D, b, r, _p(base), _p(refine))
     return base, refine
 
 
@@ -237,3 +244,48 @@ def kv_attention(k_codes, v_codes, q, sel, k_tok: int, r: int, G: int = 32) -> n
     lib().or_kv_attention(_p(kqb), _p(krho), _p(ksz), _p(vqb), _p(vrho), _p(vsz), B, H, T, D, G, r,
                           _p(qb16), Hq, _p(sel), k_tok, _p(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# decoder-step glue (standard Llama operations; readings in sf_oracle.c)
+
+
+def rmsnorm_f16(h, eps: float = 1e-5) -> np.ndarray:
+    h = np.ascontiguousarray(h, np.float64)
+    x = np.empty(h.size, np.uint16)
+    lib().or_rmsnorm_f16(_p(h), h.size, eps, _p(x))
+    return x
+
+
+def rope(v, pos: int, theta: float = 500000.0) -> np.ndarray:
+    """v[heads][d] (fp64), rotated in a copy."""
+    v = np.array(v, np.float64, copy=True, order="C")
+    lib().or_rope(_p(v), v.shape[0], v.shape[1], pos, theta)
+    return v
+
+
+def silu_mul_f16(gu) -> np.ndarray:
+    gu = np.ascontiguousarray(gu, np.float64)
+    out = np.empty(gu.size // 2, np.uint16)
+    lib().or_silu_mul_f16(_p(gu), gu.size // 2, _p(out))
+    return out
+
+
+def gemv_f16(w, x) -> np.ndarray:
+    w16 = _as_f16_bits(w)
+    x16 = _as_f16_bits(x).ravel()
+    N, K = w16.shape
+    y = np.empty(N, np.float64)
+    lib().or_gemv_f16(_p(w16), _p(x16), N, K, _p(y))
+    return y
+
+
+def gemv_correction(qb, rho, sz, r: int, G: int, x, sel) -> np.ndarray:
+    """y = sum over sel of x_c (w~ - w^)[:, c] for one activation row x."""
+    x16 = _as_f16_bits(x).ravel()
+    sel = np.ascontiguousarray(np.asarray(sel, np.int32).ravel())
+    N, K = qb.shape
+    y = np.empty(N, np.float64)
+    lib().or_gemv_correction(_p(np.ascontiguousarray(qb)), _p(np.ascontiguousarray(rho)),
+                             _p(np.ascontiguousarray(sz)), N, K, r, G, _p(x16), _p(sel), sel.size, _p(y))
+    return y

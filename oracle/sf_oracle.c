@@ -240,22 +240,79 @@ OR_API void or_pack_weights(const uint8_t* qb, const uint8_t* rho, int N, int K,
   }
 }
 
-/* KV codes: per (batch, head, token) a natural b-bit stream of the D codes
- * (D*b/8 B), tokens consecutive inside a head, heads inside a batch row, with a
- * token capacity Tmax per head; refinements likewise with r bits.  Only the
- * first T tokens of each head are written. */
-OR_API void or_pack_kv(const uint8_t* qb, const uint8_t* rho, int B, int H, int T,
-                       int Tmax, int D, int b, int r, uint8_t* base, uint8_t* refine) {
-  memset(base, 0, (size_t)B * H * Tmax * D * b / 8);
-  memset(refine, 0, (size_t)B * H * Tmax * D * r / 8);
+/* KV codes and refinements: pair-slot layout.  A little-endian 32-bit word
+ * holds 16/w pairs of w-bit codes; pair slot j keeps its first code at bits
+ * [w*j, w*j+w) and its second at bits [16+w*j, 16+w*j+w).
+ * Keys: per token, 4 chunks c of w words; pair p = 2s+e of chunk c holds dims
+ * 16s+2c+8e (first) and 16s+2c+8e+1 (second).
+ * Values: per tile of 16 tokens, 32 chunks l = 4g+c of 2w words; pair
+ * p = 16h+2m+e of chunk l holds dim 16m+g+8e of tile tokens 2c+8h (first) and
+ * 2c+8h+1 (second).  D must be 128. */
+static void put_pair(uint8_t* chunk, int w, int p, int second, int v) {
+  int per_word = 16 / w;
+  int word = p / per_word, slot = p % per_word;
+  int bit = 32 * word + 16 * second + w * slot;
+  chunk[bit >> 3] |= (uint8_t)((v & ((1 << w) - 1)) << (bit & 7));
+}
+
+/* (chunk, pair, second) of head-dim element d of a key token */
+static void key_place(int d, int* c, int* p, int* second) {
+  int s = d / 16, within = d % 16;
+  int e = within / 8;
+  *c = (within % 8) / 2;
+  *second = within % 2;
+  *p = 2 * s + e;
+}
+
+/* (chunk, pair, second) of element (token tt of its 16-token tile, dim d) of
+ * a value tile */
+static void value_place(int tt, int d, int* l, int* p, int* second) {
+  int m = d / 16, within = d % 16;
+  int e = within / 8, g = within % 8;
+  int h = tt / 8, c = (tt % 8) / 2;
+  *second = tt % 2;
+  *l = 4 * g + c;
+  *p = 16 * h + 2 * m + e;
+}
+
+static void pack_keys(const uint8_t* x, int w, int B, int H, int T, int Tmax, int D, uint8_t* out) {
+  size_t tok_bytes = (size_t)16 * w;
+  memset(out, 0, (size_t)B * H * Tmax * tok_bytes);
   for (long bh = 0; bh < (long)B * H; bh++)
     for (long t = 0; t < T; t++)
-      for (long d = 0; d < D; d++) {
-        long src = (bh * T + t) * D + d;
-        long dst = (bh * Tmax + t) * D + d;
-        put_bits(base, dst, b, qb[src]);
-        put_bits(refine, dst, r, rho[src]);
+      for (int d = 0; d < D; d++) {
+        int c, p, second;
+        key_place(d, &c, &p, &second);
+        uint8_t* chunk = out + ((size_t)bh * Tmax + t) * tok_bytes + (size_t)c * 4 * w;
+        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d]);
       }
+}
+
+static void pack_values(const uint8_t* x, int w, int B, int H, int T, int Tmax, int D, uint8_t* out) {
+  size_t tile_bytes = (size_t)256 * w;
+  memset(out, 0, (size_t)B * H * (Tmax / 16) * tile_bytes);
+  for (long bh = 0; bh < (long)B * H; bh++)
+    for (long t = 0; t < T; t++)
+      for (int d = 0; d < D; d++) {
+        int l, p, second;
+        value_place((int)(t % 16), d, &l, &p, &second);
+        uint8_t* chunk = out + ((size_t)bh * (Tmax / 16) + t / 16) * tile_bytes + (size_t)l * 8 * w;
+        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d]);
+      }
+}
+
+/* which = 0: keys, 1: values.  Writes base (b bits) and refinement (r bits)
+ * buffers of a cache with token capacity Tmax; only the first T tokens of each
+ * head are written, everything else is zero. */
+OR_API void or_pack_kv(const uint8_t* qb, const uint8_t* rho, int which, int B, int H, int T,
+                       int Tmax, int D, int b, int r, uint8_t* base, uint8_t* refine) {
+  if (which == 0) {
+    pack_keys(qb, b, B, H, T, Tmax, D, base);
+    pack_keys(rho, r, B, H, T, Tmax, D, refine);
+  } else {
+    pack_values(qb, b, B, H, T, Tmax, D, base);
+    pack_values(rho, r, B, H, T, Tmax, D, refine);
+  }
 }
 
 /* ------------------------------------------------------------------------- */
@@ -452,4 +509,75 @@ OR_API void or_kv_attention(const uint8_t* kqb, const uint8_t* krho, const uint1
       free(l);
       free(selected);
     }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Decoder-step glue.  The pages run StrataFlux inside llama.cpp on
+ * Llama-3.1-8B and leave the rest of the decoder as it is; these are the
+ * standard Llama operations, in fp64, with activations rounded to fp16
+ * where the decode step hands them from one operation to the next.
+ * Readings: RMSNorm weights are 1 and eps = 1e-5; rotary embedding pairs
+ * element i with i + d/2 and turns it by pos * theta^(-2i/d), theta = 500000,
+ * no frequency rescaling; the MLP is SiLU(gate) * up. */
+
+OR_API void or_rmsnorm_f16(const double* h, int n, double eps, uint16_t* x) {
+  double ss = 0.0;
+  for (int i = 0; i < n; i++) ss += h[i] * h[i];
+  double inv = 1.0 / sqrt(ss / (double)n + eps);
+  for (int i = 0; i < n; i++) x[i] = or_f16_from_f64(h[i] * inv);
+}
+
+OR_API void or_rope(double* v, int heads, int d, int pos, double theta) {
+  int half = d / 2;
+  for (int h = 0; h < heads; h++) {
+    double* x = v + (size_t)h * d;
+    for (int i = 0; i < half; i++) {
+      double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)d);
+      double c = cos(ang), s = sin(ang);
+      double x0 = x[i], x1 = x[i + half];
+      x[i] = x0 * c - x1 * s;
+      x[i + half] = x0 * s + x1 * c;
+    }
+  }
+}
+
+OR_API void or_silu_mul_f16(const double* gu, int inter, uint16_t* out) {
+  for (int i = 0; i < inter; i++) {
+    double g = gu[i], u = gu[inter + i];
+    out[i] = or_f16_from_f64(g / (1.0 + exp(-g)) * u);
+  }
+}
+
+/* y[n] = sum_c w[n][c] x[c], fp16 weights and activations (the LM head). */
+OR_API void or_gemv_f16(const uint16_t* w, const uint16_t* x, int N, int K, double* y) {
+  double* xv = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int c = 0; c < K; c++) xv[c] = or_f16_to_f64(x[c]);
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; n++) {
+    double acc = 0.0;
+    for (int c = 0; c < K; c++) acc += or_f16_to_f64(w[(size_t)n * K + c]) * xv[c];
+    y[n] = acc;
+  }
+  free(xv);
+}
+
+/* The refinement correction alone ([EXPL] "the map app also loads tiles":
+ * with fetch lag it is applied after the base product):
+ * y[n] = sum over the n_sel selected channels c of x[c] * (w~[n][c] - w^[n][c]). */
+OR_API void or_gemv_correction(const uint8_t* qb, const uint8_t* rho, const uint16_t* sz, int N,
+                               int K, int r, int G, const uint16_t* x, const int32_t* sel,
+                               int n_sel, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; n++) {
+    double acc = 0.0;
+    for (int j = 0; j < n_sel; j++) {
+      int c = sel[j];
+      size_t e = (size_t)n * K + c;
+      size_t zo = ((size_t)n * (K / G) + c / G) * 2;
+      double d = or_dequant_refined(sz[zo], sz[zo + 1], qb[e], rho[e], r) -
+                 or_dequant_base(sz[zo], sz[zo + 1], qb[e]);
+      acc += or_f16_to_f64(x[c]) * d;
+    }
+    y[n] = acc;
+  }
 }

@@ -71,6 +71,8 @@ def test_validation_rejects_before_launch(L):
     assert abi.sf_kv_pack_tokens(ctypes.byref(kv3), ctypes.c_void_p(16), None, 0, 1, None) \
         == abi.SF_ERR_UNSUPPORTED
     # too little workspace is reported, not overrun
-    assert abi.sf_kv_attn_refined(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, None, 0, None, 4,
+    assert abi.sf_kv_attn_refined(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, None, 0, 4,
                                   ctypes.c_void_p(16), ctypes.c_void_p(16), 8, None) == abi.SF_ERR_WORKSPACE
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, 0, ctypes.c_void_p(16),
+                                      None, ctypes.c_void_p(16), None, 0, None) == abi.SF_ERR_INVALID_ARG
     assert abi.sf_stage_refinements_host(None, 16, None, 1, None, None, None) == abi.SF_ERR_INVALID_ARG

@@ -149,6 +149,25 @@ def test_gemv_batch_and_staged_rows(batch):
     gemv_check(w, x, 2, 2, 128, 1024, 32, staged=True)
 
 
+@pytest.mark.parametrize("b,r,staged", [(2, 2, False), (3, 1, True), (4, 2, False)])
+def test_gemv_correction_only_equals_fused(b, r, staged):
+    """Fetch-lag form: base product (kch = 0) plus the correction on its own."""
+    rng = np.random.default_rng(70 + b)
+    w = inputs.weight(rng, 512, 4096)
+    x = inputs.activation(rng, 4096, batch=2)
+    qb, rho, sz = oracle.quant_weights(w, b, r, 128)
+    qw = QuantWeights.pack(cu(w), b, r, 128)
+    xd = cu(f16bits(x))
+    sel_o = oracle.select_chunks(x, 1024, 32)
+    sel_d = cu(sel_o)
+    rows = qw.refine_rows()[sel_d.view(2, -1).long()].contiguous() if staged else None
+    y, _ = qw.gemv(xd, 1024, 0)
+    qw.correction(xd, sel_d, y, 1024, 32, refine_rows=rows)
+    torch.cuda.synchronize()
+    yo = oracle.gemv_refined(qb, rho, sz, r, 128, x, sel_o, 1024, 32)
+    assert rel_l2(host(y), yo) < 1e-5
+
+
 @pytest.mark.parametrize("G", [32, 64, 256])
 def test_gemv_group_sizes(G):
     rng = np.random.default_rng(G)
@@ -211,17 +230,13 @@ def test_kv_pack_bit_exact(b, r):
         assert np.array_equal(host(gq), qb) and np.array_equal(host(grho), rho)
         gsz = host(cache.ksz if which == 0 else cache.vsz).view(np.uint16).reshape(2, 2, 48, 4, 2)[:, :, :37]
         assert np.array_equal(gsz, sz)
-        base, refine = oracle.pack_kv(qb, rho, b, r, t_max=48)
-        gb = host(cache.kb if which == 0 else cache.vb)
-        gr = host(cache.kr if which == 0 else cache.vr)
-        tok_b, tok_r = 128 * b // 8, 128 * r // 8
-        for bh in range(4):  # compare the written token slots only
-            sl_b = slice(bh * 48 * tok_b, (bh * 48 + 37) * tok_b)
-            sl_r = slice(bh * 48 * tok_r, (bh * 48 + 37) * tok_r)
-            assert np.array_equal(gb[sl_b], base[sl_b]) and np.array_equal(gr[sl_r], refine[sl_r])
+        base, refine = oracle.pack_kv(qb, rho, which, b, r, t_max=48)
+        # the cache buffers start zeroed, so unwritten slots compare equal too
+        assert np.array_equal(host(cache.kb if which == 0 else cache.vb), base)
+        assert np.array_equal(host(cache.kr if which == 0 else cache.vr), refine)
 
 
-def kv_parity(T, k_tok, splits=(0,), use_logits=True, b=2, r=2, batch=1, h_kv=8, h_q=32, seed=2):
+def kv_parity(T, k_tok, splits=(0,), b=2, r=2, batch=1, h_kv=8, h_q=32, seed=2):
     cache, kc, vc, q = kv_setup(T, b, r, batch=batch, h_kv=h_kv, h_q=h_q, seed=seed)
     qd = cu(f16bits(q))
     sel, logits, scores = cache.score_select(qd, T, k_tok, want_scores=True)
@@ -234,22 +249,31 @@ def kv_parity(T, k_tok, splits=(0,), use_logits=True, b=2, r=2, batch=1, h_kv=8,
     check_selection(gsel, so, k_tok)
     ref = oracle.kv_attention(kc, vc, q, gsel, k_tok, r)
     for ns in splits:
-        out = cache.attn_refined(qd, T, sel, k_tok, base_logits=logits if use_logits else None, n_splits=ns)
+        out = cache.attn_refined(qd, T, sel, k_tok, n_splits=ns)
         torch.cuda.synchronize()
         o = host(out)
         assert rel_l2(o, ref) <= RTOL_L2
         assert np.abs(o - ref).max() <= ATTN_MAX_ABS
+    # the fused score-select-attend call: same selection, same output
+    lg2 = torch.empty_like(logits)
+    out2, sel2 = cache.attend_selective(qd, T, k_tok, logits=lg2)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(sel2), gsel)
+    assert np.array_equal(host(lg2), host(logits))
+    o2 = host(out2)
+    assert rel_l2(o2, ref) <= RTOL_L2 and np.abs(o2 - ref).max() <= ATTN_MAX_ABS
     return cache, kc, vc, q, qd
 
 
 @pytest.mark.parametrize("T,k_tok", [(1, 1), (37, 1), (37, 37), (100, 10), (1000, 64), (2049, 300)])
 def test_kv_parity_small(T, k_tok):
-    kv_parity(T, k_tok, splits=(0, 1, 7), use_logits=True)
+    kv_parity(T, k_tok, splits=(0, 1, 7))
 
 
-def test_kv_parity_without_stored_logits_and_batch():
-    kv_parity(777, 50, splits=(0, 3), use_logits=False, batch=2, h_kv=4, h_q=32, seed=9)
-    kv_parity(500, 20, splits=(0,), use_logits=True, b=4, r=1, h_kv=2, h_q=4, seed=10)
+def test_kv_parity_batch_and_head_groups():
+    kv_parity(777, 50, splits=(0, 3), batch=2, h_kv=4, h_q=32, seed=9)   # 8 query heads per KV head
+    kv_parity(500, 20, splits=(0,), b=4, r=1, h_kv=2, h_q=4, seed=10)    # 2 per KV head, 4-bit base
+    kv_parity(300, 30, splits=(0, 5), h_kv=4, h_q=4, seed=12)            # 1 per KV head
 
 
 def test_kv_base_only_and_all_selected():

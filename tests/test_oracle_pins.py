@@ -221,14 +221,25 @@ def test_pack_weights_3bit_high_plane_by_hand(orc):
 
 
 def test_pack_kv_by_hand(orc):
-    qb = np.zeros((1, 2, 3, 32), np.uint8)
+    qb = np.zeros((1, 2, 3, 128), np.uint8)
     rho = np.zeros_like(qb)
     qb[0, 1, 2, 3] = 2
     rho[0, 0, 1, 31] = 3
-    base, refine = orc.pack_kv(qb, rho, 2, 2, t_max=4)
-    # token (head 1, t 2) starts at ((1*4)+2)*8 bytes; code 3 at bits 6-7 of byte 0
-    assert base[(4 + 2) * 8] == 2 << 6 and base.sum() == 2 << 6
-    assert refine[(0 * 4 + 1) * 8 + 7] == 3 << 6 and refine.sum() == 3 << 6
+    # keys, 2-bit codes, 32 bytes per token, t_max 16.  Dim 3: s=0, e=0, chunk
+    # c=1 (bytes 8..15 of the token), pair 0, second code -> bit 16 -> byte 2.
+    kb, kr = orc.pack_kv(qb, rho, 0, 2, 2, t_max=16)
+    assert kb[(1 * 16 + 2) * 32 + 8 + 2] == 2 and kb.sum() == 2
+    # dim 31: s=1, e=1, chunk 3, pair 3, second -> bit 22 -> byte 2, bits 6-7
+    assert kr[(0 * 16 + 1) * 32 + 24 + 2] == 3 << 6 and kr.sum() == 3 << 6
+    # values, 512-byte tiles of 16 tokens.  Token 2 of its tile: c=1, h=0,
+    # first code; dim 3: g=3, m=0, e=0 -> chunk 4*3+1 = 13 (16 bytes each),
+    # pair 0 -> bit 0.
+    vb, vr = orc.pack_kv(qb, rho, 1, 2, 2, t_max=16)
+    assert vb[1 * 512 + 13 * 16] == 2 and vb.sum() == 2
+    # 1-bit refinements: 16 pairs per word; token 1, dim 31: c=0, h=0,
+    # second; g=7, m=1, e=1 -> chunk 28 (8 bytes), pair 16*0+2+1 = 3 -> bit 16+3
+    vb1, vr1 = orc.pack_kv(qb, np.minimum(rho, 1), 1, 2, 1, t_max=16)
+    assert vr1[28 * 8 + 2] == 1 << 3 and vr1.sum() == 1 << 3
 
 
 # ---------------------------------------------------------------------------
@@ -442,3 +453,149 @@ def test_byte_model_configs():
     assert bytemodel.gemv_bytes(4096, 4096, 2, 2, 128, 32, 1024) == 4_874_752
     assert bytemodel.kv_attention_bytes(8192, 8, 32, 128, 2, 2, 32, 256) == 6_447_104
     assert bytemodel.kv_attention_bytes(131072, 8, 32, 128, 2, 2, 32, 1024) == 101_212_160
+
+
+# ---------------------------------------------------------------------------
+# decoder-step glue: closed forms and library routines
+
+
+def test_rmsnorm_closed_form(orc):
+    rng = np.random.default_rng(51)
+    h = rng.normal(0, 3, 4096)
+    x = f16(orc.rmsnorm_f16(h))
+    ref = h / np.sqrt(np.mean(h * h) + 1e-5)
+    assert np.array_equal(orc.rmsnorm_f16(h), ref.astype(np.float16).view(np.uint16))
+    assert abs(np.mean(x * x) - 1.0) < 1e-3
+    # scale invariance (eps aside)
+    assert np.abs(f16(orc.rmsnorm_f16(h * 7.0)) - x).max() <= 2 ** -9
+
+
+def test_rope_is_a_rotation_by_the_stated_angle(orc):
+    rng = np.random.default_rng(52)
+    v = rng.normal(0, 1, (3, 128))
+    assert np.allclose(orc.rope(v, 0), v)
+    pos, theta = 32768, 500000.0
+    out = orc.rope(v, pos, theta)
+    # complex multiplication of (x_i + i x_{i+64}) by e^{i pos theta^(-2i/128)}
+    z = v[:, :64] + 1j * v[:, 64:]
+    ang = pos * theta ** (-2.0 * np.arange(64) / 128)
+    w = z * np.exp(1j * ang)
+    assert np.allclose(out[:, :64], w.real, atol=1e-9) and np.allclose(out[:, 64:], w.imag, atol=1e-9)
+    assert np.allclose(np.linalg.norm(out, axis=1), np.linalg.norm(v, axis=1))
+
+
+def test_silu_mul_and_f16_gemv(orc):
+    rng = np.random.default_rng(53)
+    gu = rng.normal(0, 2, 2 * 300)
+    g, u = gu[:300], gu[300:]
+    ref = (g / (1 + np.exp(-g)) * u).astype(np.float16).view(np.uint16)
+    assert np.array_equal(orc.silu_mul_f16(gu), ref)
+    w = rng.normal(0, 0.02, (70, 256)).astype(np.float16)
+    x = rng.normal(0, 1, 256).astype(np.float16)
+    assert np.allclose(orc.gemv_f16(w, x), w.astype(np.float64) @ x.astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def test_correction_is_the_difference_of_refined_and_base(orc, small_gemv):
+    W, x, N, K, G, C = small_gemv
+    qb, rho, sz = orc.quant_weights(W, 2, 2, G)
+    sel = orc.select_chunks(x, C, 9)
+    y0 = orc.gemv_refined(qb, rho, sz, 2, G, x, None, C, 0)
+    yk = orc.gemv_refined(qb, rho, sz, 2, G, x, sel, C, 9)
+    for b in range(x.shape[0]):
+        corr = orc.gemv_correction(qb, rho, sz, 2, G, x[b], sel[b])
+        assert np.allclose(y0[b] + corr, yk[b], rtol=1e-12, atol=1e-12)
+
+
+def _dense_decoder(h16, layers, lm16, pos, h_q, h_kv, d, theta=500000.0, eps=1e-5):
+    """Textbook fp64 Llama step with dense weights/KV (every value refined)."""
+    f = lambda a: np.asarray(a, np.float16).astype(np.float64)
+    h = f(h16)[0].copy()
+
+    def norm(v):
+        return (v / np.sqrt(np.mean(v * v) + eps)).astype(np.float16).astype(np.float64)
+
+    def rot(v):
+        z = v[:, : d // 2] + 1j * v[:, d // 2:]
+        z = z * np.exp(1j * pos * theta ** (-2.0 * np.arange(d // 2) / d))
+        return np.concatenate([z.real, z.imag], axis=1)
+
+    for L in layers:
+        x = norm(h)
+        qkv = L["qkv"] @ x
+        q = rot(qkv[: h_q * d].reshape(h_q, d)).astype(np.float16).astype(np.float64)
+        k = rot(qkv[h_q * d:(h_q + h_kv) * d].reshape(h_kv, d)).astype(np.float16)
+        v = qkv[(h_q + h_kv) * d:].reshape(h_kv, d).astype(np.float16)
+        K = L["K"](k)  # dense refined keys [h_kv][T+1][d]
+        V = L["V"](v)
+        att = np.zeros((h_q, d))
+        for hh in range(h_q):
+            g = hh // (h_q // h_kv)
+            lg = K[g] @ q[hh] / math.sqrt(d)
+            p = np.exp(lg - lg.max())
+            att[hh] = (p / p.sum()) @ V[g]
+        h = h + L["o"] @ att.reshape(-1).astype(np.float16).astype(np.float64)
+        x = norm(h)
+        gu = L["gate_up"] @ x
+        I = gu.size // 2
+        xd = (gu[:I] / (1 + np.exp(-gu[:I])) * gu[I:]).astype(np.float16).astype(np.float64)
+        h = h + L["down"] @ xd
+    return f(lm16) @ norm(h)
+
+
+def test_oracle_decoder_all_refined_equals_dense_decoder(orc):
+    """lead = lag = 0, every channel and token refined: the step is a plain
+    decoder with (b+r)-bit weights and KV (textbook fp64 reference)."""
+    from oracle.decoder import OracleDecoder
+
+    rng = np.random.default_rng(61)
+    H, I, h_q, h_kv, d, T, C = 512, 1024, 4, 2, 128, 20, 256
+    h16 = rng.normal(0, 1, (1, H)).astype(np.float16)
+    dec = OracleDecoder(h16, h_q=h_q, h_kv=h_kv, d=d, r=2, G=128, chunk=C, kch=C, kv_b=2, kv_r=2,
+                        k_tok=T + 1, lead=0, lag=0)
+    dense_layers = []
+    for layer in range(2):
+        Ws = {"qkv": rng.normal(0, 0.02, ((h_q + 2 * h_kv) * d, H)), "o": rng.normal(0, 0.02, (H, h_q * d)),
+              "gate_up": rng.normal(0, 0.02, (2 * I, H)), "down": rng.normal(0, 0.02, (H, I))}
+        Q, D = {}, {}
+        for n, w in Ws.items():
+            qb, rho, sz = orc.quant_weights(w.astype(np.float32), 2, 2, 128)
+            Q[n] = (qb, rho, sz)
+            D[n] = orc.dequant_weights(qb, rho, sz, 2, 128, refined_mask=np.ones(qb.shape, bool))
+        kc = rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16)
+        vc = rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16)
+
+        def dense_kv(new, cache):
+            full = np.concatenate([cache[0], np.asarray(new)[:, None, :]], axis=1)[None]
+            qb, rho, sz = orc.quant_kv(full, 2, 2)
+            Sv = np.repeat(f16(sz[..., 0]), 32, -1)
+            Mv = np.repeat(f16(sz[..., 1]), 32, -1)
+            return (Mv + Sv * (qb + (2.0 * rho + 1 - 4) / 8))[0]
+
+        D["K"] = lambda new, cache=kc: dense_kv(new, cache)
+        D["V"] = lambda new, cache=vc: dense_kv(new, cache)
+        dense_layers.append(D)
+        dec.layer(Q, kc, vc, T)
+    lm = rng.normal(0, 0.02, (300, H)).astype(np.float16)
+    got = dec.finish(lm)[0]
+    ref = _dense_decoder(h16, dense_layers, lm, T, h_q, h_kv, d)
+    assert np.allclose(got, ref, rtol=1e-9, atol=1e-9), np.abs(got - ref).max()
+
+
+def test_oracle_decoder_lag_without_refinement_is_a_no_op(orc):
+    from oracle.decoder import OracleDecoder
+
+    rng = np.random.default_rng(62)
+    H, I, h_q, h_kv, d, T = 512, 1024, 4, 2, 128, 9
+    h16 = rng.normal(0, 1, (1, H)).astype(np.float16)
+    W = {n: orc.quant_weights(rng.normal(0, 0.02, s).astype(np.float32), 2, 2, 128)
+         for n, s in {"qkv": ((h_q + 2 * h_kv) * d, H), "o": (H, h_q * d), "gate_up": (2 * I, H),
+                      "down": (H, I)}.items()}
+    kc = rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16)
+    vc = rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16)
+    lm = rng.normal(0, 0.02, (50, H)).astype(np.float16)
+    outs = []
+    for lag in (0, 1):
+        dec = OracleDecoder(h16, h_q=h_q, h_kv=h_kv, d=d, chunk=256, kch=0, k_tok=3, lead=1, lag=lag)
+        dec.layer(W, kc, vc, T)
+        outs.append(dec.finish(lm))
+    assert np.array_equal(outs[0], outs[1])
