@@ -55,6 +55,24 @@ struct GemvParams {
   int mode;              // 0: base + correction, 1: correction only, added into y
 };
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
   asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -73,22 +91,56 @@ struct Lane {
   static constexpr int U = BITS == 4 ? 2 : 4;  // rows per step
 };
 
+// Ring slot layout (per warp, words): codes [U][W/4 chunks][32 lanes][4 words]
+// (b = 3: then [U][32 lanes][2 words] of high bits), then sz [U][2][32 lanes].
+// Consecutive lanes read consecutive 16-byte chunks, so reads are conflict-free.
 template <int BITS>
-__device__ __forceinline__ void load_codes(const GemvParams& p, int row, int lg,
-                                           uint32_t (&w)[Lane<BITS>::W]) {
-  // lg: the lane's 64-channel group index within the row
-  if constexpr (BITS == 2) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16)) + lg);
-    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
-  } else if constexpr (BITS == 3) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 16)) + lg);
-    uint2 h = __ldg(reinterpret_cast<const uint2*>(p.base + (size_t)p.N * p.K / 16 + (size_t)row * (p.K / 32)) + lg);
-    w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w, w[4] = h.x, w[5] = h.y;
+struct Ring {
+  static constexpr int W = Lane<BITS>::W, U = Lane<BITS>::U;
+  static constexpr int CW = BITS == 3 ? 4 : W;           // words in 16-byte chunks
+  static constexpr int slot_words = U * 32 * (W + 2);   // one item of U rows
+};
+
+template <int BITS>
+__device__ __forceinline__ void issue_row(const GemvParams& p, int row, int lg, int gpr, int g0,
+                                          int g1, uint32_t* slot, int u, int lane) {
+  using R = Ring<BITS>;
+  const uint8_t* rowbase;
+  if constexpr (BITS == 4) {
+    rowbase = reinterpret_cast<const uint8_t*>(p.base + (size_t)row * (p.K / 8)) + 32 * lg;
   } else {
-    const uint4* src = reinterpret_cast<const uint4*>(p.base + (size_t)row * (p.K / 8)) + 2 * lg;
-    uint4 a = __ldg(src), b = __ldg(src + 1);
-    w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
+    rowbase = reinterpret_cast<const uint8_t*>(p.base + (size_t)row * (p.K / 16)) + 16 * lg;
   }
+#pragma unroll
+  for (int c = 0; c < R::CW / 4; c++)
+    cp_async16(slot + ((u * (R::CW / 4) + c) * 32 + lane) * 4, rowbase + 16 * c);
+  if constexpr (BITS == 3) {
+    const uint8_t* hb = reinterpret_cast<const uint8_t*>(p.base + (size_t)p.N * p.K / 16 +
+                                                         (size_t)row * (p.K / 32)) + 8 * lg;
+    cp_async8(slot + R::U * R::CW * 32 + (u * 32 + lane) * 2, hb);
+  }
+  uint32_t* zs = slot + R::U * 32 * R::W;
+  const uint32_t* szrow = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)row * gpr;
+  cp_async4(zs + (u * 2 + 0) * 32 + lane, szrow + g0);
+  if (g1 != g0) cp_async4(zs + (u * 2 + 1) * 32 + lane, szrow + g1);
+}
+
+template <int BITS>
+__device__ __forceinline__ void read_row(const uint32_t* slot, int u, int lane,
+                                         uint32_t (&w)[Lane<BITS>::W], uint32_t (&z)[2], bool split) {
+  using R = Ring<BITS>;
+#pragma unroll
+  for (int c = 0; c < R::CW / 4; c++) {
+    const uint4 v = *reinterpret_cast<const uint4*>(slot + ((u * (R::CW / 4) + c) * 32 + lane) * 4);
+    w[4 * c + 0] = v.x, w[4 * c + 1] = v.y, w[4 * c + 2] = v.z, w[4 * c + 3] = v.w;
+  }
+  if constexpr (BITS == 3) {
+    const uint2 h = *reinterpret_cast<const uint2*>(slot + R::U * R::CW * 32 + (u * 32 + lane) * 2);
+    w[4] = h.x, w[5] = h.y;
+  }
+  const uint32_t* zs = slot + R::U * 32 * R::W;
+  z[0] = zs[(u * 2 + 0) * 32 + lane];
+  z[1] = split ? zs[(u * 2 + 1) * 32 + lane] : z[0];
 }
 
 // Code byte-vector v (0..15) of the lane's 64 channels; byte L holds the code
@@ -227,8 +279,8 @@ __device__ __forceinline__ float2 group_dot_halves(const uint32_t (&w)[Lane<BITS
                      fmaf((float)hi[1], 65536.0f, (float)mid[1] * 256.0f + (float)lo[1]));
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(kWarps * 32, BITS == 2 ? kCtasPerSm : 1) gemv_kernel(GemvParams p) {
+template <int BITS, int PD>
+__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_kernel(GemvParams p) {
   constexpr int W = Lane<BITS>::W, U = Lane<BITS>::U;
   extern __shared__ __align__(16) uint32_t smem[];
   const int ngrp = p.K / 64;
@@ -237,7 +289,9 @@ __global__ void __launch_bounds__(kWarps * 32, BITS == 2 ? kCtasPerSm : 1) gemv_
   const int n0 = (int)((long)blockIdx.x * p.N / gridDim.x);
   const int n1 = (int)((long)(blockIdx.x + 1) * p.N / gridDim.x);
   const int rows = n1 - n0;
-  uint32_t* scratch = reinterpret_cast<uint32_t*>(part + ((rows * p.segs + 3) & ~3));  // x staging, then correction
+  // scratch: x staging (prologue), then the per-warp copy rings (base pass),
+  // then the correction staging
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(part + ((rows * p.segs + 3) & ~3));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = warp % p.segs, rw = warp / p.segs;
   const bool warp_active = p.mode == 0 && rw < p.row_warps;
@@ -281,54 +335,54 @@ __global__ void __launch_bounds__(kWarps * 32, BITS == 2 ? kCtasPerSm : 1) gemv_
           xs1 += c.x + c.y;
         }
       }
-      const uint32_t* szrow = reinterpret_cast<const uint32_t*>(p.sz);
       const int gpr = p.K / G;
       const int g0 = (lg * 64) / G, g1 = (lg * 64 + 32) / G;
       const int step = p.row_warps * U;
-      uint32_t wa[U][W], wb[U][W], za[U][2], zb[U][2];
-      auto load = [&](int i0, uint32_t (&w)[U][W], uint32_t (&z)[U][2]) {
+      const int first = n0 + rw * U;
+      const int nitems = first < n1 ? (n1 - first + step - 1) / step : 0;
+      uint32_t* ring = scratch + warp * PD * Ring<BITS>::slot_words;
+      auto issue = [&](int k) {
+        if (k < nitems && lane_active) {
+          uint32_t* slot = ring + (k % PD) * Ring<BITS>::slot_words;
 #pragma unroll
-        for (int u = 0; u < U; u++) {
-          const int row = i0 + u;
-          if (lane_active && row < n1) {
-            load_codes<BITS>(p, row, lg, w[u]);
-            z[u][0] = __ldg(szrow + (size_t)row * gpr + g0);
-            z[u][1] = split ? __ldg(szrow + (size_t)row * gpr + g1) : z[u][0];
-          } else {
-#pragma unroll
-            for (int i = 0; i < W; i++) w[u][i] = 0;
-            z[u][0] = z[u][1] = 0;
+          for (int u = 0; u < U; u++) {
+            const int row = first + k * step + u;
+            if (row < n1) issue_row<BITS>(p, row, lg, gpr, g0, g1, slot, u, lane);
           }
         }
+        cp_async_commit();
       };
-      auto compute = [&](int i0, const uint32_t (&w)[U][W], const uint32_t (&z)[U][2]) {
+#pragma unroll
+      for (int k = 0; k < PD - 1; k++) issue(k);
+      for (int k = 0; k < nitems; k++) {
+        issue(k + PD - 1);
+        cp_async_wait<PD - 1>();
+        const uint32_t* slot = ring + (k % PD) * Ring<BITS>::slot_words;
+        const int i0 = first + k * step;
         float acc[U];
 #pragma unroll
         for (int u = 0; u < U; u++) {
-          float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&z[u][0]));
-          if (!split) {
-            float d = group_dot<BITS>(w[u], xr) * xscale;
-            acc[u] = fmaf(s0.x, d, s0.y * xsum);
-          } else {
-            float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&z[u][1]));
-            float2 d = group_dot_halves<BITS>(w[u], xr);
-            acc[u] = fmaf(s0.x, d.x * xscale, fmaf(s1.x, d.y * xscale, fmaf(s0.y, xs0, s1.y * xs1)));
+          acc[u] = 0.f;
+          if (lane_active && i0 + u < n1) {
+            uint32_t w[W], z[2];
+            read_row<BITS>(slot, u, lane, w, z, split);
+            float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&z[0]));
+            if (!split) {
+              const float d = group_dot<BITS>(w, xr) * xscale;
+              acc[u] = fmaf(s0.x, d, s0.y * xsum);
+            } else {
+              float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&z[1]));
+              const float2 d = group_dot_halves<BITS>(w, xr);
+              acc[u] = fmaf(s0.x, d.x * xscale, fmaf(s1.x, d.y * xscale, fmaf(s0.y, xs0, s1.y * xs1)));
+            }
           }
         }
         const float tot = warp_sum_rows<U>(acc, lane);
         const int u = U == 4 ? (lane >> 3) : (lane >> 4);
         const int row = i0 + u;
         if ((lane & (32 / U - 1)) == 0 && row < n1) part[(row - n0) * p.segs + seg] = tot;
-      };
-      int i0 = n0 + rw * U;
-      if (i0 < n1) load(i0, wa, za);
-      for (; i0 < n1; i0 += 2 * step) {
-        if (i0 + step < n1) load(i0 + step, wb, zb);
-        compute(i0, wa, za);
-        if (i0 + step >= n1) break;
-        if (i0 + 2 * step < n1) load(i0 + 2 * step, wa, za);
-        compute(i0 + step, wb, zb);
       }
+      cp_async_wait<0>();
     }
     __syncthreads();
 
@@ -442,21 +496,36 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   SF_UNSUPPORTED(p.segs <= kWarps, "k=%d above %d", w->k, kWarps * kSegChannels);
   p.refine_row_words = w->n * w->r / 32;
   p.staged = refine_rows != nullptr;
-  // 2-bit codes fit two CTAs of 8 warps per SM in registers; wider codes one
-  int grid = (w->b == 2 ? kCtasPerSm : 1) * num_sms();
+  const int U = w->b == 4 ? 2 : 4;
+  const int W = w->b == 2 ? 4 : w->b == 3 ? 6 : 8;
+  const size_t slot_bytes = (size_t)U * 32 * (W + 2) * 4;
+  const size_t xs_bytes = (size_t)(w->k / 64) * kXWords * 4;
+  const size_t xraw_bytes = (size_t)w->k * 2;
+  const size_t corr_bytes = (size_t)kCorrSmemWords * 4;
+  auto smem_for = [&](int ctas_per_sm, int pd) {
+    int grid = ctas_per_sm * num_sms();
+    if (grid > w->n / 4) grid = w->n / 4;
+    const size_t rows = (w->n + grid - 1) / grid;
+    const size_t segs = (w->k + kSegChannels - 1) / kSegChannels;
+    const size_t part = ((rows * segs + 3) & ~(size_t)3) * 4;
+    size_t scratch = (size_t)kWarps * pd * slot_bytes;
+    if (scratch < xraw_bytes) scratch = xraw_bytes;
+    if (scratch < corr_bytes) scratch = corr_bytes;
+    return xs_bytes + part + scratch;
+  };
+  const size_t per_sm = 227 * 1024;
+  int ctas = kCtasPerSm, pd = 3;
+  if (smem_for(ctas, 3) * ctas > per_sm - ctas * 1024) pd = 2;
+  if (smem_for(ctas, pd) * ctas > per_sm - ctas * 1024) ctas = 1, pd = 3;
+  int grid = ctas * num_sms();
   if (grid > w->n / 4) grid = w->n / 4;
   const int rows_per_cta = (w->n + grid - 1) / grid;
-  const int U = w->b == 4 ? 2 : 4;
   p.row_warps = kWarps / p.segs;
   const int needed = (rows_per_cta + U - 1) / U;
   if (p.row_warps > needed) p.row_warps = needed;
   if (p.row_warps < 1) p.row_warps = 1;
-  const size_t xs_words = (size_t)(w->k / 64) * kXWords;
-  const size_t part_words = ((size_t)rows_per_cta * p.segs + 3) & ~(size_t)3;
-  size_t scratch_words = (size_t)w->k / 2;  // raw x (fp16)
-  if (scratch_words < (size_t)kCorrSmemWords) scratch_words = kCorrSmemWords;
-  const size_t smem = (xs_words + part_words + scratch_words) * 4;
-  SF_UNSUPPORTED(smem <= 110 * 1024, "k=%d needs too much shared memory", w->k);
+  const size_t smem = smem_for(ctas, pd);
+  SF_UNSUPPORTED(smem <= 200 * 1024, "k=%d needs too much shared memory", w->k);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -468,8 +537,12 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   attr[0].val.programmaticStreamSerializationAllowed = (kch > 0 && !sel_in) ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void (*kern)(GemvParams) = w->b == 2 ? gemv_kernel<2> : w->b == 3 ? gemv_kernel<3> : gemv_kernel<4>;
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 110 * 1024));
+  void (*kern)(GemvParams);
+  if (pd == 3)
+    kern = w->b == 2 ? gemv_kernel<2, 3> : w->b == 3 ? gemv_kernel<3, 3> : gemv_kernel<4, 3>;
+  else
+    kern = w->b == 2 ? gemv_kernel<2, 2> : w->b == 3 ? gemv_kernel<3, 2> : gemv_kernel<4, 2>;
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
   SF_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
   return SF_OK;
 }

@@ -36,6 +36,7 @@
 
 #include "common.cuh"
 #include "kvlayout.cuh"
+#include "radix.cuh"
 
 namespace sf {
 namespace {
@@ -69,30 +70,47 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
-  return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-}
-
 // Pair slot `slot` (compile-time after unrolling) of a w-bit pair-slot word as
-// an exact half2; see kvlayout.cuh.
+// an exact half2 of CENTRED codes c - (2^W - 1)/2 (for 2-bit codes
+// -1.5, -0.5, 0.5, 1.5).  The code is masked in place, OR-ed into the
+// mantissa of 1024.0 and rescaled with one fused multiply-add; the word is
+// shifted first so that the code sits at a bit offset b2 in [2, 10 - W], which
+// keeps the fma constant exactly representable.  w_l2 = w << 2, w_r = w >> 8
+// (W = 2) or w >> 6 (W = 4).
 template <int W>
-__device__ __forceinline__ uint32_t pair_at(uint32_t w, uint32_t w_hi8, int slot) {
+__device__ __forceinline__ uint32_t pair_at(uint32_t w, uint32_t w_l2, uint32_t w_r, int slot) {
   const int bit = W * slot;
-  const bool shift = bit + W > 10;
-  const int b2 = shift ? bit - 8 : bit;
+  const int rsh = W == 2 ? 8 : 6;
+  const bool left = bit < 2;
+  const bool right = !left && bit + W > 10;
+  const int b2 = left ? bit + 2 : right ? bit - rsh : bit;
+  const uint32_t src = left ? w_l2 : right ? w_r : w;
   const uint32_t mask = (((1u << W) - 1u) << b2) * 0x00010001u;
-  uint32_t v = ((shift ? w_hi8 : w) & mask) | 0x64006400u;  // 1024 + c * 2^b2 per half
-  const uint32_t sc = (uint32_t)((15 - b2) << 10) * 0x00010001u;              // 2^-b2
-  const uint32_t off = (uint32_t)(0x8000u | ((25 - b2) << 10)) * 0x00010001u;  // -1024 * 2^-b2
+  uint32_t v = (src & mask) | 0x64006400u;  // 1024 + c * 2^b2 per half
+  // fp16 bit patterns: 2^-b2, and -(2^(10-b2) + centre) whose mantissa is
+  // centre * 2^b2 = (2^W - 1) * 2^(b2-1)
+  const uint32_t sc = (uint32_t)((15 - b2) << 10) * 0x00010001u;
+  const uint32_t off = (0x8000u | ((uint32_t)(25 - b2) << 10) | (((1u << W) - 1u) << (b2 - 1))) * 0x00010001u;
   __half2 r = __hfma2(*reinterpret_cast<__half2*>(&v), *reinterpret_cast<const __half2*>(&sc),
                       *reinterpret_cast<const __half2*>(&off));
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
 template <int W>
-__device__ __forceinline__ uint32_t pair_of(const uint32_t* words, const uint32_t* words8, int p) {
+struct Words {
+  uint32_t w, l2, r;
+  __device__ __forceinline__ void set(uint32_t x) {
+    w = x;
+    l2 = x << 2;
+    r = x >> (W == 2 ? 8 : 6);
+  }
+};
+
+template <int W, int N>
+__device__ __forceinline__ uint32_t pair_of(const Words<W> (&ws)[N], int p) {
   constexpr int per = 16 / W;
-  return pair_at<W>(words[p / per], words8[p / per], p % per);
+  const Words<W>& x = ws[p / per];
+  return pair_at<W>(x.w, x.l2, x.r, p % per);
 }
 
 // ---------------------------------------------------------------------------
@@ -107,8 +125,8 @@ struct BaseArgs {
   const uint16_t* q;
   int h_q, gq;
   float* logits;  // [batch][h_q][T]
-  float* part;    // [batch][h_q][nsplit][rec]  (rec = kRec with values, 2 without)
-  int span, nsplit;
+  float* part;    // [batch][h_q][nrec][rec]  (rec = kRec with values, 2 without)
+  int span, nsplit, nrec;
   float scale;
 };
 
@@ -116,37 +134,44 @@ template <int B, bool PV>
 struct Stage {
   static constexpr int kBytes = 256 * B;           // key codes of 16 tokens
   static constexpr int vBytes = PV ? 256 * B : 0;  // value tile
-  static constexpr int szBytes = PV ? 512 : 256;   // key (+ value) step/offset
+  static constexpr int szBytes = PV ? 512 : 256;   // key (+ value) step/offset (fp16)
   static constexpr int bytes = kBytes + vBytes + szBytes;
+};
+
+template <int B, bool PV>
+struct WarpSmem {
+  static constexpr int ring = kStages * Stage<B, PV>::bytes;
+  static constexpr int zf = 16 * 4 * 2 * 4 * (PV ? 2 : 1);  // fp32 (s, m') of 16 tokens x 4 groups
+  static constexpr int ps = 16 * 9 * 4;                      // transposed probabilities
+  static constexpr int bytes = ring + zf + ps;
 };
 
 // GQP: query heads per KV head padded to 4 or 8.  B: base bits (2 or 4).
 template <int GQP, int B, bool PV>
-__global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
   using St = Stage<B, PV>;
-  constexpr int NT = GQP / 4;  // value-side n-tiles (4 heads x hi/lo each)
+  using WS = WarpSmem<B, PV>;
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int g = blockIdx.y, bat = blockIdx.z;
   const int split = blockIdx.x * kWarps + warp;
-  if (split >= a.nsplit) return;  // warp-private from here on: no block barriers
-  uint8_t* wsm = smem + warp * (kStages * St::bytes + 16 * 9 * 4 + 8 * 4);
-  float* Ps = reinterpret_cast<float*>(wsm + kStages * St::bytes);  // [16][9]
-  float* As = Ps + 16 * 9;                                           // [8]
+  uint8_t* wsm = smem + warp * WS::bytes;
+  float* Zs = reinterpret_cast<float*>(wsm + WS::ring);        // [PV+1][16][4][2]
+  float* Ps = reinterpret_cast<float*>(wsm + WS::ring + WS::zf);  // [16][9]
+  const float centre = 0.5f * (float)((1 << B) - 1);
 
   const int tw0 = split * a.span;
   const int tw1 = min(a.T, tw0 + a.span);
-  const int ntile = tw1 > tw0 ? (tw1 - tw0 + 15) / 16 : 0;
+  const int ntile = (split < a.nsplit && tw1 > tw0) ? (tw1 - tw0 + 15) / 16 : 0;
   const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;  // first token slot of this head
   const int gq = a.gq;
+  const int h0 = 2 * tig, h1 = 2 * tig + 1;  // the lane's logit / output head columns
 
   // ---- query fragments (B operand of the key contraction): head gid
   const uint16_t* qg = a.q + ((long)bat * a.h_q + (long)g * gq) * kD;
   uint32_t qf[8][2];
-  float qsum[4];  // per group j: sum of q over the lane's 8 dims of head gid
-#pragma unroll
-  for (int j = 0; j < 4; j++) qsum[j] = 0.f;
+  float qsum[4] = {0.f, 0.f, 0.f, 0.f};  // per group j: the lane's 8 dims of head gid
 #pragma unroll
   for (int s = 0; s < 8; s++) {
     uint32_t lo = 0, hi = 0;
@@ -159,29 +184,24 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
     float2 f1 = __half22float2(*reinterpret_cast<__half2*>(&hi));
     qsum[s >> 1] += (f0.x + f0.y) + (f1.x + f1.y);
   }
-  // full per-group sums of head gid, then fetch heads 2tig, 2tig+1 for the epilogue
-  float Q0[4], Q1[4];
+  float Q0[4], Q1[4];  // per-group sums of q for heads 2tig, 2tig+1
 #pragma unroll
   for (int j = 0; j < 4; j++) {
     float v = qsum[j];
     v += __shfl_xor_sync(0xffffffffu, v, 1);
     v += __shfl_xor_sync(0xffffffffu, v, 2);
-    Q0[j] = __shfl_sync(0xffffffffu, v, 8 * tig);      // head 2tig   (gid = 2tig)
-    Q1[j] = __shfl_sync(0xffffffffu, v, 8 * tig + 4);  // head 2tig+1 (gid = 2tig+1)
+    Q0[j] = __shfl_sync(0xffffffffu, v, 8 * tig);
+    Q1[j] = __shfl_sync(0xffffffffu, v, 8 * tig + 4);
   }
 
-  float mrun0 = -FLT_MAX, mrun1 = -FLT_MAX, lsum0 = 0.f, lsum1 = 0.f;
-  float accv[NT][8][4];
-  float mt[NT][4];
+  // softmax state of heads 2tig, 2tig+1 (the lane's logit and output columns)
+  float mrun0 = -INFINITY, mrun1 = -INFINITY, lsum0 = 0.f, lsum1 = 0.f;
+  float accv[8][4];
+  float mt[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p m'_t,j of head gid
 #pragma unroll
-  for (int nt = 0; nt < NT; nt++) {
+  for (int m = 0; m < 8; m++)
 #pragma unroll
-    for (int m = 0; m < 8; m++)
-#pragma unroll
-      for (int i = 0; i < 4; i++) accv[nt][m][i] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; j++) mt[nt][j] = 0.f;
-  }
+    for (int i = 0; i < 4; i++) accv[m][i] = 0.f;
 
   auto issue = [&](int it) {
     if (it < ntile) {
@@ -189,12 +209,13 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
       const long slot = slot0 + tw0 + 16 * it;
 #pragma unroll
       for (int c = 0; c < B / 2; c++) {
-        int ci = lane + 32 * c;
+        const int ci = lane + 32 * c;
         cp_async16(st + 16 * ci, a.kb + slot * 16 * B + 16 * ci);
         if (PV) cp_async16(st + St::kBytes + 16 * ci, a.vb + (slot / 16) * 256 * B + 16 * ci);
       }
       if (lane < 16)
-        cp_async16(st + St::kBytes + St::vBytes + 16 * lane, reinterpret_cast<const uint8_t*>(a.ksz) + slot * 16 + 16 * lane);
+        cp_async16(st + St::kBytes + St::vBytes + 16 * lane,
+                   reinterpret_cast<const uint8_t*>(a.ksz) + slot * 16 + 16 * lane);
       else if (PV)
         cp_async16(st + St::kBytes + St::vBytes + 16 * lane,
                    reinterpret_cast<const uint8_t*>(a.vsz) + slot * 16 + 16 * (lane - 16));
@@ -205,15 +226,26 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
 #pragma unroll
   for (int i = 0; i < kStages - 1; i++) issue(i);
 
-  const float NEG = -INFINITY;
   for (int it = 0; it < ntile; it++) {
     issue(it + kStages - 1);
     cp_async_wait<kStages - 1>();
     __syncwarp();
     const uint8_t* st = wsm + (it % kStages) * St::bytes;
-    const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
-    const uint16_t* ks = reinterpret_cast<const uint16_t*>(st + St::kBytes + St::vBytes);
     const int t0 = tw0 + 16 * it;
+    // (s, m') = (s, m + centre * s) in fp32 for the tile's tokens; tokens past
+    // the end of the span get (0, 0) so they contribute nothing
+    {
+      const uint32_t* zh = reinterpret_cast<const uint32_t*>(st + St::kBytes + St::vBytes);
+#pragma unroll
+      for (int i = 0; i < (PV ? 4 : 2); i++) {
+        const int e = lane + 32 * i;  // (which, token, group) = (e / 64, (e / 4) % 16, e % 4)
+        uint32_t z = zh[e];
+        float2 sm = __half22float2(*reinterpret_cast<__half2*>(&z));
+        const bool valid = t0 + ((e >> 2) & 15) < tw1;
+        reinterpret_cast<float2*>(Zs)[e] = valid ? make_float2(sm.x, fmaf(centre, sm.x, sm.y)) : make_float2(0.f, 0.f);
+      }
+    }
+    __syncwarp();
 
     // ---- logits: tokens on M (gid, gid+8), heads on N, k-steps of 16 dims
     float acc[4][4];
@@ -222,18 +254,17 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; i++) acc[j][i] = 0.f;
     {
-      uint32_t w0[B], w8[B], w0s[B], w8s[B];
+      const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
+      Words<B> w0[B], w8[B];
 #pragma unroll
       for (int i = 0; i < B; i++) {
-        w0[i] = kc[gid * 4 * B + tig * B + i];
-        w8[i] = kc[(gid + 8) * 4 * B + tig * B + i];
-        w0s[i] = w0[i] >> 8;
-        w8s[i] = w8[i] >> 8;
+        w0[i].set(kc[gid * 4 * B + tig * B + i]);
+        w8[i].set(kc[(gid + 8) * 4 * B + tig * B + i]);
       }
 #pragma unroll
       for (int s = 0; s < 8; s++) {
-        uint32_t a0 = pair_of<B>(w0, w0s, 2 * s), a1 = pair_of<B>(w8, w8s, 2 * s);
-        uint32_t a2 = pair_of<B>(w0, w0s, 2 * s + 1), a3 = pair_of<B>(w8, w8s, 2 * s + 1);
+        uint32_t a0 = pair_of<B>(w0, 2 * s), a1 = pair_of<B>(w8, 2 * s);
+        uint32_t a2 = pair_of<B>(w0, 2 * s + 1), a3 = pair_of<B>(w8, 2 * s + 1);
         mma16816(acc[s >> 1], a0, a1, a2, a3, qf[s][0], qf[s][1]);
       }
     }
@@ -241,20 +272,20 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
 #pragma unroll
     for (int r = 0; r < 2; r++) {
       const int tok = gid + 8 * r;
-      const uint32_t* zw = reinterpret_cast<const uint32_t*>(ks + tok * 8);
+      const float4* zk = reinterpret_cast<const float4*>(Zs + tok * 8);
       float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; j++) {
-        uint32_t z = zw[j];
-        float2 sm = __half22float2(*reinterpret_cast<__half2*>(&z));
-        x0 = fmaf(sm.x, acc[j][2 * r + 0], fmaf(sm.y, Q0[j], x0));
-        x1 = fmaf(sm.x, acc[j][2 * r + 1], fmaf(sm.y, Q1[j], x1));
+      for (int jj = 0; jj < 2; jj++) {
+        const float4 z = zk[jj];  // groups 2jj, 2jj+1: (s, m')
+        x0 = fmaf(z.x, acc[2 * jj][2 * r], fmaf(z.y, Q0[2 * jj], x0));
+        x1 = fmaf(z.x, acc[2 * jj][2 * r + 1], fmaf(z.y, Q1[2 * jj], x1));
+        x0 = fmaf(z.z, acc[2 * jj + 1][2 * r], fmaf(z.w, Q0[2 * jj + 1], x0));
+        x1 = fmaf(z.z, acc[2 * jj + 1][2 * r + 1], fmaf(z.w, Q1[2 * jj + 1], x1));
       }
       const bool valid = t0 + tok < tw1;
-      l[2 * r + 0] = valid ? x0 * a.scale : NEG;
-      l[2 * r + 1] = valid ? x1 * a.scale : NEG;
+      l[2 * r + 0] = valid ? x0 * a.scale : -INFINITY;
+      l[2 * r + 1] = valid ? x1 * a.scale : -INFINITY;
     }
-    const int h0 = 2 * tig, h1 = 2 * tig + 1;
     {
       float* lg = a.logits + ((long)bat * a.h_q + (long)g * gq) * a.T;
 #pragma unroll
@@ -273,141 +304,135 @@ __global__ void __launch_bounds__(kWarps * 32) kv_base_kernel(BaseArgs a) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
-    const float mn0 = fmaxf(mrun0, mx0), mn1 = fmaxf(mrun1, mx1);
+    const float mn0 = fmaxf(mrun0, mx0), mn1 = fmaxf(mrun1, mx1);  // finite: the tile has a token
     const float al0 = __expf(mrun0 - mn0), al1 = __expf(mrun1 - mn1);
     float p[4];
-    p[0] = (h0 < gq && l[0] != NEG) ? __expf(l[0] - mn0) : 0.f;
-    p[1] = (h1 < gq && l[1] != NEG) ? __expf(l[1] - mn1) : 0.f;
-    p[2] = (h0 < gq && l[2] != NEG) ? __expf(l[2] - mn0) : 0.f;
-    p[3] = (h1 < gq && l[3] != NEG) ? __expf(l[3] - mn1) : 0.f;
+    p[0] = h0 < gq ? __expf(l[0] - mn0) : 0.f;
+    p[1] = h1 < gq ? __expf(l[1] - mn1) : 0.f;
+    p[2] = h0 < gq ? __expf(l[2] - mn0) : 0.f;
+    p[3] = h1 < gq ? __expf(l[3] - mn1) : 0.f;
     lsum0 = fmaf(lsum0, al0, p[0] + p[2]);
     lsum1 = fmaf(lsum1, al1, p[1] + p[3]);
     mrun0 = mn0, mrun1 = mn1;
 
     if constexpr (PV) {
-      const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + St::kBytes);
-      const uint16_t* vs = ks + 128;
       Ps[gid * 9 + h0] = p[0];
       Ps[gid * 9 + h1] = p[1];
       Ps[(gid + 8) * 9 + h0] = p[2];
       Ps[(gid + 8) * 9 + h1] = p[3];
-      if (gid == 0) As[h0] = al0, As[h1] = al1;
+      // rescale factor of head gid (held by the lanes with tig = gid / 2)
+      const float ala = __shfl_sync(0xffffffffu, al0, gid >> 1);
+      const float alb = __shfl_sync(0xffffffffu, al1, gid >> 1);
+      const float alg = (gid & 1) ? alb : ala;
       __syncwarp();
-      // value step/offset of the lane's four tokens 2tig, 2tig+1, 2tig+8, 2tig+9
-      float vsv[4][4], vmv[4][4];
+      // B operand: fp16(p * s) of head gid for the lane's tokens 2tig, 2tig+1,
+      // 2tig+8, 2tig+9; the offsets m' go to the fp32 m-term
+      const float* zv = Zs + 16 * 8;
+      float pv[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const int tk = 2 * tig + (i & 1) + 8 * (i >> 1);
-        const bool valid = t0 + tk < tw1;
-        const uint32_t* zw = reinterpret_cast<const uint32_t*>(vs + tk * 8);
+      for (int i = 0; i < 4; i++) pv[i] = Ps[(2 * tig + (i & 1) + 8 * (i >> 1)) * 9 + gid];
+      uint32_t bf[4][2];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-          uint32_t z = zw[j];
-          float2 sm = __half22float2(*reinterpret_cast<__half2*>(&z));
-          vsv[i][j] = valid ? sm.x : 0.f;
-          vmv[i][j] = valid ? sm.y : 0.f;
+      for (int jj = 0; jj < 2; jj++) {
+        float4 z[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+          z[i] = reinterpret_cast<const float4*>(zv + (2 * tig + (i & 1) + 8 * (i >> 1)) * 8)[jj];
+        // group 2jj: (z.x, z.y); group 2jj+1: (z.z, z.w)
+        __half2 b00 = __floats2half2_rn(pv[0] * z[0].x, pv[1] * z[1].x);
+        __half2 b01 = __floats2half2_rn(pv[2] * z[2].x, pv[3] * z[3].x);
+        __half2 b10 = __floats2half2_rn(pv[0] * z[0].z, pv[1] * z[1].z);
+        __half2 b11 = __floats2half2_rn(pv[2] * z[2].z, pv[3] * z[3].z);
+        bf[2 * jj][0] = *reinterpret_cast<uint32_t*>(&b00);
+        bf[2 * jj][1] = *reinterpret_cast<uint32_t*>(&b01);
+        bf[2 * jj + 1][0] = *reinterpret_cast<uint32_t*>(&b10);
+        bf[2 * jj + 1][1] = *reinterpret_cast<uint32_t*>(&b11);
+        float s0 = mt[2 * jj] * alg, s1 = mt[2 * jj + 1] * alg;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+          s0 = fmaf(pv[i], z[i].y, s0);
+          s1 = fmaf(pv[i], z[i].w, s1);
         }
+        mt[2 * jj] = s0, mt[2 * jj + 1] = s1;
       }
-      uint32_t bf[NT][4][2];
-      float av[NT];
+      const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + St::kBytes);
+      Words<B> vw[2 * B];
 #pragma unroll
-      for (int nt = 0; nt < NT; nt++) {
-        av[nt] = As[4 * nt + tig];
-        const int hb = 4 * nt + (gid >> 1);
-        const bool hi_part = (gid & 1) == 0;
-        float pv[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++) pv[i] = Ps[(2 * tig + (i & 1) + 8 * (i >> 1)) * 9 + hb];
-        const float ab = As[hb];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-          __half hv[4];
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            float v = pv[i] * vsv[i][j];
-            __half h = __float2half_rn(v);
-            hv[i] = hi_part ? h : __float2half_rn(v - __half2float(h));
-          }
-          bf[nt][j][0] = pack_h2(hv[0], hv[1]);
-          bf[nt][j][1] = pack_h2(hv[2], hv[3]);
-          if (hi_part) {
-            float s = mt[nt][j] * ab;
-#pragma unroll
-            for (int i = 0; i < 4; i++) s = fmaf(pv[i], vmv[i][j], s);
-            mt[nt][j] = s;
-          }
-        }
-      }
-      uint32_t vw[2 * B], vws[2 * B];
-#pragma unroll
-      for (int i = 0; i < 2 * B; i++) {
-        vw[i] = vc[lane * 2 * B + i];
-        vws[i] = vw[i] >> 8;
-      }
+      for (int i = 0; i < 2 * B; i++) vw[i].set(vc[lane * 2 * B + i]);
       // Each tile's product starts from zero and is folded into the running
       // sum with one fp32 FMA that also applies the softmax rescale: long
       // accumulation chains inside the tensor-core accumulator would drift.
 #pragma unroll
       for (int m = 0; m < 8; m++) {
-        uint32_t a0 = pair_of<B>(vw, vws, 2 * m), a1 = pair_of<B>(vw, vws, 2 * m + 1);
-        uint32_t a2 = pair_of<B>(vw, vws, 16 + 2 * m), a3 = pair_of<B>(vw, vws, 17 + 2 * m);
-#pragma unroll
-        for (int nt = 0; nt < NT; nt++) {
-          float t4[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(t4, a0, a1, a2, a3, bf[nt][m >> 1][0], bf[nt][m >> 1][1]);
-#pragma unroll
-          for (int i = 0; i < 4; i++) accv[nt][m][i] = fmaf(accv[nt][m][i], av[nt], t4[i]);
-        }
+        uint32_t a0 = pair_of<B>(vw, 2 * m), a1 = pair_of<B>(vw, 2 * m + 1);
+        uint32_t a2 = pair_of<B>(vw, 16 + 2 * m), a3 = pair_of<B>(vw, 17 + 2 * m);
+        float t4[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16816(t4, a0, a1, a2, a3, bf[m >> 1][0], bf[m >> 1][1]);
+        accv[m][0] = fmaf(accv[m][0], al0, t4[0]);
+        accv[m][1] = fmaf(accv[m][1], al1, t4[1]);
+        accv[m][2] = fmaf(accv[m][2], al0, t4[2]);
+        accv[m][3] = fmaf(accv[m][3], al1, t4[3]);
       }
     }
     __syncwarp();
   }
   cp_async_wait<0>();
 
-  // ---- partial record of this split
+  // ---- per-warp state of heads 2tig, 2tig+1, then merge the CTA's warps
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     lsum0 += __shfl_xor_sync(0xffffffffu, lsum0, o);
     lsum1 += __shfl_xor_sync(0xffffffffu, lsum1, o);
   }
+  __syncwarp();
+  // warp record in its own smem: [GQP][kRec] (the stage ring is free now)
+  float* wrec = reinterpret_cast<float*>(wsm);
+  const int rec = PV ? kRec : 2;
+  if constexpr (PV) {
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      float v = mt[j];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      mt[j] = v;  // head gid
+    }
+    float m0[4], m1[4];  // m-terms of heads 2tig, 2tig+1
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      m0[j] = __shfl_sync(0xffffffffu, mt[j], 8 * tig);
+      m1[j] = __shfl_sync(0xffffffffu, mt[j], 8 * tig + 4);
+    }
+#pragma unroll
+    for (int m = 0; m < 8; m++) {
+      wrec[h0 * kRec + 16 * m + gid] = accv[m][0] + m0[m >> 1];
+      wrec[h1 * kRec + 16 * m + gid] = accv[m][1] + m1[m >> 1];
+      wrec[h0 * kRec + 16 * m + gid + 8] = accv[m][2] + m0[m >> 1];
+      wrec[h1 * kRec + 16 * m + gid + 8] = accv[m][3] + m1[m >> 1];
+    }
+  }
+  if (gid == 0) {
+    wrec[h0 * rec + rec - 2] = mrun0, wrec[h0 * rec + rec - 1] = lsum0;
+    wrec[h1 * rec + rec - 2] = mrun1, wrec[h1 * rec + rec - 1] = lsum1;
+  }
+  __syncthreads();
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
-  if constexpr (!PV) {
-    if (gid == 0) {
-      if (2 * tig < gq) {
-        float* rec = a.part + ((hq0 + 2 * tig) * a.nsplit + split) * 2;
-        rec[0] = mrun0, rec[1] = lsum0;
-      }
-      if (2 * tig + 1 < gq) {
-        float* rec = a.part + ((hq0 + 2 * tig + 1) * a.nsplit + split) * 2;
-        rec[0] = mrun1, rec[1] = lsum1;
+  for (int e = threadIdx.x; e < gq * rec; e += blockDim.x) {
+    const int h = e / rec, d = e % rec;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++)
+      M = fmaxf(M, reinterpret_cast<const float*>(smem + w * WS::bytes)[h * rec + rec - 2]);
+    float v = 0.f;
+    if (M > -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; w++) {
+        const float* r = reinterpret_cast<const float*>(smem + w * WS::bytes) + h * rec;
+        const float mw = r[rec - 2];
+        if (mw > -INFINITY) v = fmaf(__expf(mw - M), d == rec - 2 ? 0.f : r[d], v);
       }
     }
-  } else {
-#pragma unroll
-    for (int nt = 0; nt < NT; nt++) {
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        float v = mt[nt][j];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        mt[nt][j] = __shfl_sync(0xffffffffu, v, 8 * tig);  // head 4nt + tig (gid = 2tig, hi part)
-      }
-      const int h = 4 * nt + tig;
-      const float ma = __shfl_sync(0xffffffffu, mrun0, h >> 1), mb = __shfl_sync(0xffffffffu, mrun1, h >> 1);
-      const float la = __shfl_sync(0xffffffffu, lsum0, h >> 1), lb = __shfl_sync(0xffffffffu, lsum1, h >> 1);
-      if (h < gq) {
-        float* rec = a.part + ((hq0 + h) * a.nsplit + split) * kRec;
-#pragma unroll
-        for (int m = 0; m < 8; m++) {
-          rec[16 * m + gid] = accv[nt][m][0] + accv[nt][m][1] + mt[nt][m >> 1];
-          rec[16 * m + gid + 8] = accv[nt][m][2] + accv[nt][m][3] + mt[nt][m >> 1];
-        }
-        if (gid == 0) {
-          rec[kD] = (h & 1) ? mb : ma;
-          rec[kD + 1] = (h & 1) ? lb : la;
-        }
-      }
-    }
+    if (d == rec - 2) v = M;
+    a.part[((hq0 + h) * a.nrec + blockIdx.x) * rec + d] = v;
   }
 }
 
@@ -416,9 +441,9 @@ __global__ void kv_stats_kernel(const float* __restrict__ part, int nsplit, int 
                                 float2* __restrict__ stats) {
   const long bh = blockIdx.x;
   const float* p = part + bh * nsplit * rec;
-  const int mo = rec == 2 ? 0 : kD;
+  const int mo = rec - 2;
   __shared__ float sm[256];
-  float m = -FLT_MAX;
+  float m = -INFINITY;
   for (int i = threadIdx.x; i < nsplit; i += blockDim.x) m = fmaxf(m, p[(long)i * rec + mo]);
   sm[threadIdx.x] = m;
   __syncthreads();
@@ -431,7 +456,7 @@ __global__ void kv_stats_kernel(const float* __restrict__ part, int nsplit, int 
   float s = 0.f;
   for (int i = threadIdx.x; i < nsplit; i += blockDim.x) {
     float mi = p[(long)i * rec + mo];
-    if (mi > -FLT_MAX) s += p[(long)i * rec + mo + 1] * expf(mi - M);
+    if (mi > -INFINITY) s += p[(long)i * rec + mo + 1] * expf(mi - M);
   }
   sm[threadIdx.x] = s;
   __syncthreads();
@@ -454,132 +479,54 @@ __device__ __forceinline__ int key_token(uint64_t key) {
   return (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu));
 }
 
-// k-th largest of n unique keys (1 <= k <= n), 8 bits per pass from the top.
-__device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int k, int* hist) {
-  __shared__ int s_digit, s_k;
-  uint64_t prefix = 0, mask = 0;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      uint64_t key = keys[i];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      const int lane = threadIdx.x;  // owns digits 255-8*lane .. 248-8*lane
-      int c[8], tot = 0;
-#pragma unroll
-      for (int j = 0; j < 8; j++) tot += (c[j] = hist[255 - 8 * lane - j]);
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      int above = incl - tot;
-      if (above < k && incl >= k) {
-        int run = above;
-        for (int j = 0; j < 8; j++) {
-          if (run + c[j] >= k) {
-            s_digit = 255 - 8 * lane - j;
-            s_k = k - run;
-            break;
-          }
-          run += c[j];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= (uint64_t)s_digit << shift;
-    mask |= (uint64_t)255 << shift;
-    k = s_k;
-    __syncthreads();
-  }
-  return prefix;
-}
-
-// Emit the keys >= tau in index order (each thread owns a contiguous range).
-template <class Emit>
-__device__ void block_compact(const uint64_t* keys, int n, uint64_t tau, Emit emit) {
-  __shared__ int warp_tot[32];
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
-  int mine = 0;
-  for (int i = i0; i < i1; i++) mine += keys[i] >= tau;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = mine;
-  for (int o = 1; o < 32; o <<= 1) {
-    int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int nw = blockDim.x >> 5;
-    int v = lane < nw ? warp_tot[lane] : 0;
-    int x = v;
-    for (int o = 1; o < 32; o <<= 1) {
-      int u = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += u;
-    }
-    if (lane < nw) warp_tot[lane] = x - v;
-  }
-  __syncthreads();
-  int pos = warp_tot[warp] + incl - mine;
-  for (int i = i0; i < i1; i++)
-    if (keys[i] >= tau) emit(pos++, keys[i]);
-  __syncthreads();
-}
-
 __global__ void __launch_bounds__(1024) kv_local_kernel(const float* __restrict__ logits,
                                                         const float2* __restrict__ stats, int T,
                                                         int span, int h_q, int h_kv, int k_tok,
                                                         float* __restrict__ scores,
                                                         uint64_t* __restrict__ cand) {
   extern __shared__ uint64_t keys[];  // span entries
-  __shared__ int hist[256];
+  __shared__ RadixShared sh;
+  __shared__ float Ms[8], invZ[8];
   const int gq = h_q / h_kv;
   const int sp = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
   const int t0 = sp * span, n = min(T, t0 + span) - t0;
-  float M[8], invZ[8];
-  for (int h = 0; h < gq; h++) {
-    float2 st = stats[(long)bat * h_q + g * gq + h];
-    M[h] = st.x, invZ[h] = 1.0f / st.y;
+  if (threadIdx.x < gq) {
+    const float2 st = stats[(long)bat * h_q + g * gq + threadIdx.x];
+    Ms[threadIdx.x] = st.x, invZ[threadIdx.x] = 1.0f / st.y;
   }
+  __syncthreads();
+  const float* lg = logits + ((long)bat * h_q + g * gq) * T + t0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     float s = 0.f;
-    for (int h = 0; h < gq; h++)
-      s += expf(logits[((long)bat * h_q + g * gq + h) * T + t0 + i] - M[h]) * invZ[h];
+    for (int h = 0; h < gq; h++) s += expf(lg[(long)h * T + i] - Ms[h]) * invZ[h];
     if (scores) scores[((long)bat * h_kv + g) * T + t0 + i] = s;
     keys[i] = score_key(s, t0 + i);
   }
   __syncthreads();
   const int kl = min(k_tok, n);
-  uint64_t tau = block_kth_largest(keys, n, kl, hist);
+  auto key_at = [&](int i) { return keys[i]; };
+  const uint64_t tau = block_kth_largest<64>(key_at, n, kl, sh);
   uint64_t* out = cand + (((long)bat * h_kv + g) * gridDim.x + sp) * (long)min(k_tok, span);
-  block_compact(keys, n, tau, [&](int pos, uint64_t key) { out[pos] = key; });
+  block_compact(key_at, n, tau, sh, [&](int pos, int, uint64_t key) { out[pos] = key; });
 }
 
 __global__ void __launch_bounds__(1024) kv_final_kernel(const uint64_t* __restrict__ cand, int nspan,
                                                         int span, int T, int h_kv, int k_tok,
                                                         int32_t* __restrict__ sel) {
   extern __shared__ uint64_t keys[];  // all candidates of this KV head
-  __shared__ int hist[256];
+  __shared__ RadixShared sh;
   const int g = blockIdx.x, bat = blockIdx.y;
   const int per = min(k_tok, span);
   const uint64_t* src = cand + ((long)bat * h_kv + g) * nspan * (long)per;
-  int n = 0;
-  for (int sp = 0; sp < nspan; sp++) {
-    int len = min(T, (sp + 1) * span) - sp * span;
-    int cnt = min(k_tok, len);
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) keys[n + i] = src[(long)sp * per + i];
-    n += cnt;
-  }
+  // every span but the last holds `per` keys, so the candidates are one run
+  const int last = min(k_tok, T - (nspan - 1) * span);
+  const int n = (nspan - 1) * per + last;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = src[i];
   __syncthreads();
-  uint64_t tau = block_kth_largest(keys, n, k_tok, hist);
+  auto key_at = [&](int i) { return keys[i]; };
+  const uint64_t tau = block_kth_largest<64>(key_at, n, k_tok, sh);
   int32_t* out = sel + ((long)bat * h_kv + g) * k_tok;
-  block_compact(keys, n, tau, [&](int pos, uint64_t key) { out[pos] = key_token(key); });
+  block_compact(key_at, n, tau, sh, [&](int pos, int, uint64_t key) { out[pos] = key_token(key); });
 }
 
 // ---------------------------------------------------------------------------
@@ -600,17 +547,16 @@ struct CorrArgs {
   float scale;
 };
 
-__device__ __forceinline__ uint32_t read_bits(const uint8_t* base, int word, int bit, int w) {
-  return (reinterpret_cast<const uint32_t*>(base)[word] >> bit) & ((1u << w) - 1u);
-}
 
-// block = kD threads (thread = head-dim element)
+// block = kD threads (thread = head-dim element); every token of the chunk is
+// loaded with independent loads before anything is computed
 __global__ void __launch_bounds__(kD) kv_correct_kernel(CorrArgs a) {
   __shared__ float kf[kCorrTok][kD + 4];
   __shared__ float vbs[kCorrTok][kD];
   __shared__ float vfs[kCorrTok][kD];
   __shared__ float qs[8][kD + 4];
   __shared__ float wf[kCorrTok][8], wb[kCorrTok][8];
+  __shared__ int ts[kCorrTok];
   const int d = threadIdx.x;
   const int chunk = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
   const int gq = a.gq;
@@ -619,38 +565,57 @@ __global__ void __launch_bounds__(kD) kv_correct_kernel(CorrArgs a) {
   const int j0 = chunk * kCorrTok;
   const int nsel = min(kCorrTok, a.k_tok - j0);
   const int32_t* sg = a.sel + ((long)bat * a.h_kv + g) * a.k_tok + j0;
+  if (d < nsel) ts[d] = sg[d];
+  __syncthreads();
   const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
   const float half = 0.5f * (float)(1 << a.r), inv = 1.0f / (float)(1 << a.r);
-  for (int i = 0; i < nsel; i++) {
-    const int t = sg[i];
-    const long slot = slot0 + t;
-    int word, bit;
-    // key, refined
-    key_pos(d, a.b, word, bit);
-    uint32_t qk = read_bits(a.kb + slot * 16 * a.b, word, bit, a.b);
-    key_pos(d, a.r, word, bit);
-    uint32_t rk = read_bits(a.kr + slot * 16 * a.r, word, bit, a.r);
-    const uint16_t* zk = a.ksz + (slot * 4 + d / 32) * 2;
-    kf[i][d] = fmaf(h2f(zk[0]), (float)qk + ((float)rk + 0.5f - half) * inv, h2f(zk[1]));
-    // value, base and refined
-    const long tile = slot / 16;
-    value_pos(t & 15, d, a.b, word, bit);
-    uint32_t qv = read_bits(a.vb + tile * 256 * a.b, word, bit, a.b);
-    value_pos(t & 15, d, a.r, word, bit);
-    uint32_t rv = read_bits(a.vr + tile * 256 * a.r, word, bit, a.r);
-    const uint16_t* zv = a.vsz + (slot * 4 + d / 32) * 2;
-    const float sv = h2f(zv[0]), mv = h2f(zv[1]);
-    vbs[i][d] = fmaf(sv, (float)qv, mv);
-    vfs[i][d] = fmaf(sv, (float)qv + ((float)rv + 0.5f - half) * inv, mv);
+  int kw, kbit, krw, krbit;
+  key_pos(d, a.b, kw, kbit);
+  key_pos(d, a.r, krw, krbit);
+  // all loads first (independent), then the arithmetic
+  uint32_t rqk[kCorrTok], rrk[kCorrTok], rzk[kCorrTok], rqv[kCorrTok], rrv[kCorrTok], rzv[kCorrTok];
+  int rvb[kCorrTok], rvr[kCorrTok];
+#pragma unroll
+  for (int i = 0; i < kCorrTok; i++) {
+    if (i < nsel) {
+      const int t = ts[i];
+      const long slot = slot0 + t;
+      const long tile = slot / 16;
+      int vw, vbit, vrw, vrbit;
+      value_pos(t & 15, d, a.b, vw, vbit);
+      value_pos(t & 15, d, a.r, vrw, vrbit);
+      rqk[i] = reinterpret_cast<const uint32_t*>(a.kb + slot * 16 * a.b)[kw];
+      rrk[i] = reinterpret_cast<const uint32_t*>(a.kr + slot * 16 * a.r)[krw];
+      rzk[i] = *reinterpret_cast<const uint32_t*>(a.ksz + (slot * 4 + d / 32) * 2);
+      rqv[i] = reinterpret_cast<const uint32_t*>(a.vb + tile * 256 * a.b)[vw];
+      rrv[i] = reinterpret_cast<const uint32_t*>(a.vr + tile * 256 * a.r)[vrw];
+      rzv[i] = *reinterpret_cast<const uint32_t*>(a.vsz + (slot * 4 + d / 32) * 2);
+      rvb[i] = vbit, rvr[i] = vrbit;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kCorrTok; i++) {
+    if (i < nsel) {
+      const uint32_t qk = (rqk[i] >> kbit) & ((1u << a.b) - 1);
+      const uint32_t rk = (rrk[i] >> krbit) & ((1u << a.r) - 1);
+      const uint32_t qv = (rqv[i] >> rvb[i]) & ((1u << a.b) - 1);
+      const uint32_t rv = (rrv[i] >> rvr[i]) & ((1u << a.r) - 1);
+      const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&rzk[i]));
+      const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&rzv[i]));
+      kf[i][d] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
+      vbs[i][d] = fmaf(v2.x, (float)qv, v2.y);
+      vfs[i][d] = fmaf(v2.x, (float)qv + ((float)rv + 0.5f - half) * inv, v2.y);
+    }
   }
   __syncthreads();
   // refined logits of (token, head) pairs; base logits as the base pass stored them
   for (int pr = d; pr < nsel * gq; pr += kD) {
     const int i = pr / gq, h = pr % gq;
     float acc = 0.f;
+#pragma unroll 8
     for (int e = 0; e < kD; e++) acc = fmaf(qs[h][e], kf[i][e], acc);
     const float M = a.stats[hq0 + h].x;
-    const float lb = a.logits[(hq0 + h) * a.T + sg[i]];
+    const float lb = a.logits[(hq0 + h) * a.T + ts[i]];
     wf[i][h] = __expf(acc * a.scale - M);
     wb[i][h] = __expf(lb - M);
   }
@@ -667,36 +632,62 @@ __global__ void __launch_bounds__(kD) kv_correct_kernel(CorrArgs a) {
   }
 }
 
-// out = (sum_s e^(m_s - M) acc_s + sum_c dA_c) / (Z + sum_c dZ_c)
-__global__ void __launch_bounds__(kD) kv_merge_kernel(const float* __restrict__ part, int nsplit,
-                                                      const float* __restrict__ corr, int ncorr,
-                                                      const float2* __restrict__ stats,
-                                                      float* __restrict__ out) {
+// out = (sum_s e^(m_s - M) acc_s + sum_c dA_c) / (Z + sum_c dZ_c).
+// 4 x kD threads: thread group r sums every 4th record.
+constexpr int kMergeGroups = 4;
+constexpr int kMaxRec = 4096;
+
+__global__ void __launch_bounds__(kMergeGroups * kD) kv_merge_kernel(
+    const float* __restrict__ part, int nrec, const float* __restrict__ corr, int ncorr,
+    const float2* __restrict__ stats, float* __restrict__ out) {
+  __shared__ float wts[kMaxRec];
+  __shared__ float red[kMergeGroups][kD + 1];
   const long bh = blockIdx.x;
-  const int d = threadIdx.x;
   const float2 st = stats[bh];
-  const float* p = part + bh * nsplit * kRec;
-  float num = 0.f;
-  for (int s = 0; s < nsplit; s++) {
-    float ms = p[(long)s * kRec + kD];
-    if (ms > -FLT_MAX) num = fmaf(expf(ms - st.x), p[(long)s * kRec + d], num);
+  const float* p = part + bh * nrec * kRec;
+  for (int s = threadIdx.x; s < nrec; s += blockDim.x) {
+    const float ms = p[(long)s * kRec + kD];
+    wts[s] = ms > -INFINITY ? expf(ms - st.x) : 0.f;
   }
-  float den = st.y;
+  __syncthreads();
+  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
+  float num = 0.f, dz = 0.f;
+  int s = grp;
+  for (; s + 3 * kMergeGroups < nrec; s += 4 * kMergeGroups) {
+    const float v0 = p[(long)s * kRec + d], v1 = p[(long)(s + kMergeGroups) * kRec + d];
+    const float v2 = p[(long)(s + 2 * kMergeGroups) * kRec + d], v3 = p[(long)(s + 3 * kMergeGroups) * kRec + d];
+    num = fmaf(wts[s], v0, num);
+    num = fmaf(wts[s + kMergeGroups], v1, num);
+    num = fmaf(wts[s + 2 * kMergeGroups], v2, num);
+    num = fmaf(wts[s + 3 * kMergeGroups], v3, num);
+  }
+  for (; s < nrec; s += kMergeGroups) num = fmaf(wts[s], p[(long)s * kRec + d], num);
   if (corr) {
     const float* c = corr + bh * ncorr * kRec;
-    for (int i = 0; i < ncorr; i++) {
+    for (int i = grp; i < ncorr; i += kMergeGroups) {
       num += c[(long)i * kRec + d];
-      den += c[(long)i * kRec + kD];
+      dz += c[(long)i * kRec + kD];
     }
   }
-  out[bh * kD + d] = num / den;
+  red[grp][d] = num;
+  if (d == 0) red[grp][kD] = dz;
+  __syncthreads();
+  if (grp == 0) {
+    float n = 0.f, z = st.y;
+#pragma unroll
+    for (int r = 0; r < kMergeGroups; r++) {
+      n += red[r][d];
+      z += red[r][kD];
+    }
+    out[bh * kD + d] = n / z;
+  }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 
 struct Plan {
-  int nsplit, span;       // base pass (warp splits)
+  int nsplit, span, nrec; // base pass (warp splits; one record per CTA of kWarps splits)
   int sspan, ns;          // selection spans
   int ncorr;              // correction chunks per KV head
   size_t off_logits, off_part, off_stats, off_cand, off_corr, total;
@@ -713,6 +704,7 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   if (ns < 1) ns = 1;
   P.span = ((t + ns - 1) / ns + 15) / 16 * 16;
   P.nsplit = (t + P.span - 1) / P.span;
+  P.nrec = (P.nsplit + kWarps - 1) / kWarps;  // <= kMaxRec is checked by the callers
   // selection spans
   int ss = (sms + heads - 1) / heads;
   if (ss < 1) ss = 1;
@@ -734,7 +726,7 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   };
   const int rec = with_pv ? kRec : 2;
   P.off_logits = need_logits ? take((size_t)kv->batch * h_q * t * 4) : 0;
-  P.off_part = take((size_t)kv->batch * h_q * P.nsplit * rec * 4);
+  P.off_part = take((size_t)kv->batch * h_q * P.nrec * rec * 4);
   P.off_stats = take((size_t)kv->batch * h_q * 8);
   P.off_cand = select ? take((size_t)heads * P.ns * (k_tok < span ? k_tok : span) * 8) : 0;
   P.off_corr = (with_pv && P.ncorr) ? take((size_t)kv->batch * h_q * P.ncorr * kRec * 4) : 0;
@@ -753,8 +745,7 @@ sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
 
 template <int GQP, int B, bool PV>
 sf_status launch_base_t(const BaseArgs& a, int batch, cudaStream_t s) {
-  const size_t per_warp = kStages * Stage<B, PV>::bytes + 16 * 9 * 4 + 8 * 4;
-  const size_t smem = kWarps * per_warp;
+  const size_t smem = kWarps * WarpSmem<B, PV>::bytes;
   auto kern = kv_base_kernel<GQP, B, PV>;
   SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   dim3 grid((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch);
@@ -781,7 +772,7 @@ BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* lo
   a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.T = t;
   a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
   a.logits = logits, a.part = part;
-  a.span = P.span, a.nsplit = P.nsplit;
+  a.span = P.span, a.nsplit = P.nsplit, a.nrec = P.nrec;
   a.scale = 1.0f / sqrtf((float)kD);
   return a;
 }
@@ -820,8 +811,8 @@ sf_status launch_correct_merge(const sf_kv* kv, int t, const uint16_t* q, int h_
     kv_correct_kernel<<<dim3(P.ncorr, kv->h_kv, kv->batch), kD, 0, s>>>(c);
     SF_LAUNCHED();
   }
-  kv_merge_kernel<<<kv->batch * h_q, kD, 0, s>>>(part, P.nsplit, k_tok > 0 ? corr : nullptr,
-                                                 P.ncorr, stats, out);
+  kv_merge_kernel<<<kv->batch * h_q, kMergeGroups * kD, 0, s>>>(part, P.nrec, k_tok > 0 ? corr : nullptr,
+                                                                P.ncorr, stats, out);
   SF_LAUNCHED();
   return SF_OK;
 }
@@ -859,6 +850,7 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(!scores || aligned16(scores), "scores must be 16-byte aligned");
   Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, false, true, 0);
+  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
@@ -868,7 +860,7 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   st = launch_base(kv, a, false, s);
   if (st != SF_OK) return st;
   float2* stats = (float2*)(w + P.off_stats);
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>((const float*)(w + P.off_part), P.nsplit, 2, stats);
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>((const float*)(w + P.off_part), P.nrec, 2, stats);
   SF_LAUNCHED();
   return launch_select(kv, t, h_q, k_tok, P, lg, stats, scores, (uint64_t*)(w + P.off_cand), sel, s);
 }
@@ -891,6 +883,7 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(n_splits >= 0, "n_splits=%d < 0", n_splits);
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
   Plan P = make_plan(kv, t, h_q, k_tok, true, true, false, n_splits);
+  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
@@ -901,7 +894,7 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nsplit, kRec, stats);
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nrec, kRec, stats);
   SF_LAUNCHED();
   return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
                               (float*)(w + P.off_corr), out, s);
@@ -926,6 +919,7 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
   Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0);
+  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
@@ -936,7 +930,7 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nsplit, kRec, stats);
+  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nrec, kRec, stats);
   SF_LAUNCHED();
   st = launch_select(kv, t, h_q, k_tok, P, lg, stats, nullptr, (uint64_t*)(w + P.off_cand), sel, s);
   if (st != SF_OK) return st;

@@ -6,69 +6,35 @@
 // each chunk are refined at this step (the error of a projection is the sum of
 // activation times weight error, so a large |x| magnifies its channel's error).
 //
-// One CTA per (batch row, chunk).  Every channel gets the unique key
-// (|x| as the 15-bit fp16 magnitude) << 11 | (2047 - index in chunk), so equal
-// magnitudes rank the lower index first.  The k-th largest key is found bit by
-// bit from the top with block-wide counts; the selected channels are then
-// written in ascending index order with a block prefix sum.
+// Every channel gets the unique key (|x| as the 15-bit fp16 magnitude) << 11 |
+// (2047 - index in chunk), so equal magnitudes rank the lower index first.
+// The k-th largest key is found by a block-wide radix select (radix.cuh); the
+// selected channels are then written in ascending index order.
 #include "common.cuh"
 #include "internal.cuh"
+#include "radix.cuh"
 
 namespace sf {
 namespace {
 
-template <int E>
-__global__ void __launch_bounds__(1024) select_chunks_kernel(const uint16_t* __restrict__ x, int K,
-                                                             int chunk, int kch,
-                                                             int32_t* __restrict__ sel) {
+constexpr int kSelThreads = 256;
+
+// One CTA per (batch row, chunk of up to 2,048 channels).
+__global__ void __launch_bounds__(kSelThreads) select_chunks_kernel(const uint16_t* __restrict__ x,
+                                                                   int K, int chunk, int kch,
+                                                                   int32_t* __restrict__ sel) {
   pdl_trigger();  // a dependent GEMV may start streaming its base codes now
-  __shared__ int warp_sums[32];
+  __shared__ uint32_t keys[2048];
+  __shared__ RadixShared sh;
   const int b = blockIdx.y, c = blockIdx.x;
   const uint16_t* xc = x + (size_t)b * K + (size_t)c * chunk;
-  uint32_t key[E];
-#pragma unroll
-  for (int e = 0; e < E; e++) {
-    int i = threadIdx.x * E + e;
-    key[e] = ((uint32_t)(xc[i] & 0x7fff) << 11) | (uint32_t)(2047 - i);
-  }
-  uint32_t tau = 0;  // largest value with count(key >= tau) >= kch
-  for (int bit = 25; bit >= 0; --bit) {
-    uint32_t cand = tau | (1u << bit);
-    int cnt = 0;
-#pragma unroll
-    for (int e = 0; e < E; e++) cnt += __syncthreads_count(key[e] >= cand);
-    if (cnt >= kch) tau = cand;
-  }
-  // exclusive prefix sum of the per-thread selected counts, in index order
-  int mine = 0;
-#pragma unroll
-  for (int e = 0; e < E; e++) mine += key[e] >= tau;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
+  for (int i = threadIdx.x; i < chunk; i += blockDim.x)
+    keys[i] = ((uint32_t)(xc[i] & 0x7fff) << 11) | (uint32_t)(2047 - i);
   __syncthreads();
-  if (warp == 0) {
-    int nw = blockDim.x >> 5;
-    int v = lane < nw ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int u = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += u;
-    }
-    if (lane < nw) warp_sums[lane] = v - (lane < nw ? warp_sums[lane] : 0);  // exclusive
-  }
-  __syncthreads();
-  int pos = warp_sums[warp] + incl - mine;
+  auto key_at = [&](int i) { return (uint64_t)keys[i]; };
+  const uint64_t tau = block_kth_largest<26>(key_at, chunk, kch, sh);
   int32_t* out = sel + ((size_t)b * (K / chunk) + c) * kch;
-#pragma unroll
-  for (int e = 0; e < E; e++) {
-    if (key[e] >= tau) out[pos++] = c * chunk + threadIdx.x * E + e;
-  }
+  block_compact(key_at, chunk, tau, sh, [&](int pos, int i, uint64_t) { out[pos] = c * chunk + i; });
 }
 
 }  // namespace
@@ -86,10 +52,7 @@ sf_status check_select_args(const uint16_t* x, int batch, int k, int chunk, int 
 sf_status launch_select(const uint16_t* x, int batch, int k, int chunk, int kch, int32_t* sel,
                         cudaStream_t s) {
   dim3 grid(k / chunk, batch);
-  if (chunk <= 1024)
-    select_chunks_kernel<1><<<grid, chunk, 0, s>>>(x, k, chunk, kch, sel);
-  else
-    select_chunks_kernel<2><<<grid, chunk / 2, 0, s>>>(x, k, chunk, kch, sel);
+  select_chunks_kernel<<<grid, kSelThreads, 0, s>>>(x, k, chunk, kch, sel);
   SF_LAUNCHED();
   return SF_OK;
 }

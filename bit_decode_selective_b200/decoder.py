@@ -86,7 +86,7 @@ class Decoder:
         B = batch
         # activations
         self.h = f32(B, cfg.hidden)
-        self.x_attn = f16(B, cfg.hidden)
+        self.x_attn = [f16(B, cfg.hidden) for _ in range(2)]
         self.qkv_out = f32(B, shp["qkv"][0])
         self.q = f16(B, cfg.h_q, cfg.d)
         self.k_new = f16(B, cfg.h_kv, 1, cfg.d)
@@ -94,7 +94,7 @@ class Decoder:
         self.attn = f32(B, cfg.h_q, cfg.d)
         self.x_o = [f16(B, cfg.h_q * cfg.d) for _ in range(2)]
         self.o_out = f32(B, cfg.hidden)
-        self.x_mlp = f16(B, cfg.hidden)
+        self.x_mlp = [f16(B, cfg.hidden) for _ in range(2)]
         self.gu_out = f32(B, 2 * cfg.inter)
         self.x_down = [f16(B, cfg.inter) for _ in range(2)]
         self.down_out = f32(B, cfg.hidden)
@@ -152,60 +152,59 @@ class Decoder:
         check(abi.sf_select_channels(_p(x), self.B, self.shp[name][1], cfg.chunk, cfg.kch,
                                      _p(self.sel[name][slot]), _s(stream)), "sf_select_channels")
 
-    def _stage(self, layer, name, slot, main):
+    def _stage(self, layer, name, slot):
         """Copy layer `layer`'s rows of the selection in `slot` into staging
-        slot `slot` on the side stream, after the selection is done."""
-        ev = self.ev_sel[name][slot]
-        ev.record(main)
-        self.side.wait_event(ev)
+        slot `slot` on the side stream (enqueued after the selection)."""
         check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
                                        _p(self.sel[name][slot]), self.B * self.n_sel[name],
                                        _p(self.slots[name][slot]), _s(self.side), None),
               "sf_stage_refinements")
+
+    def _side_select_stage(self, layer, name, x, slot, main):
+        """Selection from x and the row transfer, both on the side stream; the
+        event ev_stage[name][slot] marks both done."""
+        ev = self.ev_sel[name][slot]
+        ev.record(main)
+        self.side.wait_event(ev)
+        self._select(name, x, slot, self.side)
+        if self.slots is not None:
+            self._stage(layer, name, slot)
         self.ev_stage[name][slot].record(self.side)
 
-    def _rows(self, name, slot, main):
-        if self.slots is None:
-            return None
+    def _ready(self, name, slot, main):
+        """Wait (on the main stream) for the selection and rows in `slot`."""
         main.wait_event(self.ev_stage[name][slot])
-        return self.slots[name][slot]
+        return self.slots[name][slot] if self.slots is not None else None
 
     def _proj(self, layer, name, x, y, slot, main, base_only=False):
-        """y = W~ x for layer `layer` with the selection in `slot` (lead) or
-        selected here (no lead / layer 0)."""
+        """y = W~ x for layer `layer` with the selection in `slot`."""
         cfg = self.cfg
         qw = self.layers[layer][name]
         if cfg.kch == 0 or base_only:
             check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, 0, None, None, None,
                                       _p(y), None, 0, _s(main)), "sf_gemv_refined")
             return
-        rows = self._rows(name, slot, main)
+        rows = self._ready(name, slot, main)
         check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
                                   _p(self.sel[name][slot]), None, _p(rows), _p(y), None, 0, _s(main)),
               "sf_gemv_refined")
 
     def _prepare(self, layer, name, x, main):
-        """Make sure the selection and staged rows of (layer, name) exist in
-        slot layer % 2 before the projection runs."""
+        """Without lead (or at layer 0) the projection selects from its own
+        input: selection and transfer now, the projection waits for them."""
         cfg = self.cfg
         if cfg.kch == 0:
             return
-        slot = layer % 2
         if not cfg.lead or layer == 0:
-            self._select(name, x, slot, main)
-            if self.slots is not None:
-                self._stage(layer, name, slot, main)
+            self._side_select_stage(layer, name, x, layer % 2, main)
 
     def _lead(self, layer, name, x, main):
         """Fetch lead: select (layer + 1)'s channels from this activation and
-        start their transfer."""
+        start their transfer on the side stream."""
         cfg = self.cfg
         if cfg.kch == 0 or not cfg.lead or layer + 1 >= cfg.n_layers:
             return
-        slot = (layer + 1) % 2
-        self._select(name, x, slot, main)
-        if self.slots is not None:
-            self._stage(layer + 1, name, slot, main)
+        self._side_select_stage(layer + 1, name, x, (layer + 1) % 2, main)
 
     def _lagged(self, layer, main):
         """Fetch lag: layer `layer`'s o and down corrections into the residual."""
@@ -215,7 +214,7 @@ class Decoder:
         slot = layer % 2
         for name, x in (("o", self.x_o[slot]), ("down", self.x_down[slot])):
             qw = self.layers[layer][name]
-            rows = self._rows(name, slot, main)
+            rows = self._ready(name, slot, main)
             check(abi.sf_gemv_correction(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
                                          _p(self.sel[name][slot]), _p(rows), _p(self.h), _s(main)),
                   "sf_gemv_correction")
@@ -233,12 +232,13 @@ class Decoder:
             L = self.layers[l]
             if l > 0:
                 self._lagged(l - 1, main)
-            check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), None, B, cfg.hidden, cfg.eps, _p(self.x_attn),
+            x_attn, x_o, x_mlp, x_down = self.x_attn[slot], self.x_o[slot], self.x_mlp[slot], self.x_down[slot]
+            check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), None, B, cfg.hidden, cfg.eps, _p(x_attn),
                                           _s(main)), "sf_rmsnorm_residual")
             # attention block
-            self._prepare(l, "qkv", self.x_attn, main)
-            self._proj(l, "qkv", self.x_attn, self.qkv_out, slot, main)
-            self._lead(l, "qkv", self.x_attn, main)
+            self._prepare(l, "qkv", x_attn, main)
+            self._lead(l, "qkv", x_attn, main)
+            self._proj(l, "qkv", x_attn, self.qkv_out, slot, main)
             check(abi.sf_rope_split(_p(self.qkv_out), B, cfg.h_q, cfg.h_kv, cfg.d, T, cfg.theta, _p(self.q),
                                     _p(self.k_new), _p(self.v_new), _s(main)), "sf_rope_split")
             kv = L["kv"]
@@ -247,22 +247,20 @@ class Decoder:
             check(abi.sf_kv_attend_selective(ctypes.byref(kv.desc), T + 1, _p(self.q), cfg.h_q, cfg.k_tok,
                                              _p(self.tok_sel), None, _p(self.attn), _p(self.ws), self.ws.numel(),
                                              _s(main)), "sf_kv_attend_selective")
-            x_o = self.x_o[slot]
             check(abi.sf_cast_f16(_p(self.attn), B * cfg.h_q * cfg.d, _p(x_o), _s(main)), "sf_cast_f16")
             self._prepare(l, "o", x_o, main)
-            self._proj(l, "o", x_o, self.o_out, slot, main, base_only=bool(cfg.lag))
             self._lead(l, "o", x_o, main)
+            self._proj(l, "o", x_o, self.o_out, slot, main, base_only=bool(cfg.lag))
             check(abi.sf_rmsnorm_residual(_p(self.h), _p(self.o_out), None, B, cfg.hidden, cfg.eps,
-                                          _p(self.x_mlp), _s(main)), "sf_rmsnorm_residual")
+                                          _p(x_mlp), _s(main)), "sf_rmsnorm_residual")
             # MLP block
-            self._prepare(l, "gate_up", self.x_mlp, main)
-            self._proj(l, "gate_up", self.x_mlp, self.gu_out, slot, main)
-            self._lead(l, "gate_up", self.x_mlp, main)
-            x_down = self.x_down[slot]
+            self._prepare(l, "gate_up", x_mlp, main)
+            self._lead(l, "gate_up", x_mlp, main)
+            self._proj(l, "gate_up", x_mlp, self.gu_out, slot, main)
             check(abi.sf_silu_mul(_p(self.gu_out), B, cfg.inter, _p(x_down), _s(main)), "sf_silu_mul")
             self._prepare(l, "down", x_down, main)
-            self._proj(l, "down", x_down, self.down_out, slot, main, base_only=bool(cfg.lag))
             self._lead(l, "down", x_down, main)
+            self._proj(l, "down", x_down, self.down_out, slot, main, base_only=bool(cfg.lag))
             add = self.down_out
         self._lagged(cfg.n_layers - 1, main)
         check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), None, B, cfg.hidden, cfg.eps, _p(self.x_final),
