@@ -173,7 +173,6 @@ def gemv_roofline(dec, steps, warmup, hbm_peak):
     from bit_decode_selective_b200.ops import _p
 
     cfg = dec.cfg
-    s = torch.cuda.current_stream()
     xs = {"qkv": dec.x_attn[0], "o": dec.x_o[0], "gate_up": dec.x_mlp[0], "down": dec.x_down[0]}
     ys = {"qkv": dec.qkv_out, "o": dec.o_out, "gate_up": dec.gu_out, "down": dec.down_out}
     # selections and staged rows as the step leaves them (slot 0)
@@ -186,9 +185,11 @@ def gemv_roofline(dec, steps, warmup, hbm_peak):
             nbytes += bytemodel.gemv_bytes(n, k, cfg.w_bits, cfg.w_refine, cfg.group, cfg.kch, cfg.chunk, dec.B)
 
     def run():
+        s = torch.cuda.current_stream()  # the capture stream inside torch.cuda.graph
         for qw, x, y, sel, rows in calls:
             abi.check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), dec.B, cfg.chunk, cfg.kch, _p(sel), None,
-                                          _p(rows), _p(y), None, 0, ctypes.c_void_p(s.cuda_stream)),
+                                          _p(rows), _p(y), _p(dec.gemv_ws), dec.gemv_ws.numel(),
+                                          ctypes.c_void_p(s.cuda_stream)),
                       "sf_gemv_refined")
 
     run()

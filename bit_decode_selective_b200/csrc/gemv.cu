@@ -14,45 +14,71 @@
 //
 // Decomposition, per output row i (fp32 accumulation):
 //   y_i = sum_groups [ s_ig * sum_{c in g} x_c q_ic + m_ig * sum_{c in g} x_c ]
-//       + sum_{c selected} x_c * s_i,g(c) * (2 rho_ic + 1 - 2^r) / 2^(r+1)
+//       + sum_{c selected} x_c * s_i,g(c) * (rho_ic + 1/2 - 2^(r-1)) / 2^r
 //
-// Base pass (HBM-bound: every resident code is read once).  Each CTA owns a
-// contiguous range of rows; each warp owns one 2,048-channel segment of K and
-// keeps that segment's activations in registers as exact fixed point: per
-// 64-channel lane group x = x_fix * 2^e with |x_fix| < 2^23, split into three
-// byte planes.  A lane streams 64 channels of a row per step (16 B of 2-bit
-// codes), expands them to byte vectors with shifts and masks and takes the
-// integer dot products with dp4a (4 code x byte products per instruction).
-// Rows are prefetched one step ahead in registers; partial sums of four rows
-// are reduced across the warp with a transposed butterfly.
+// Activation prologue (gemv_prep_kernel, once per call): every 64-channel
+// lane group of x becomes exact fixed point x = x_fix * 2^e with
+// |x_fix| < 2^21, split into three byte planes laid out in the order of the
+// code byte vectors below, plus the group's sums.
 //
-// Correction pass: after griddepcontrol.wait (the selection kernel may still
-// be running while the base pass streams), the CTA stages the selected
-// channels' activations and the refinement words covering its rows in shared
-// memory with independent loads, then one warp per row sums the corrections.
+// Base pass (HBM-bound: every resident code is read once).  One CTA of 16
+// warps per SM owns a contiguous, 4-aligned range of rows.  Its work is a list
+// of (2,048-channel segment, 4-row step) tasks split evenly over the warps; a
+// warp keeps the byte planes of its current segment in registers (a lane owns
+// 64 channels) and streams the codes of its rows through a per-lane cp.async
+// ring.  A lane turns 16 B of 2-bit codes into byte vectors with one AND per
+// four codes (codes at bit offsets 2 and 6 keep a factor 4 that is removed
+// once per row), takes integer dot products with dp4a (four code x byte
+// products per instruction) and combines the planes in 32-bit integers, so the
+// lane's partial dot product is exact.  Partial sums of four rows are reduced
+// across the warp with a transposed butterfly.
+//
+// Correction pass: the prologue writes a table of the selected channels
+// (x_c, group, refinement row); the GEMV copies it and the refinement words
+// covering its rows into shared memory while the base pass streams (the base
+// pass also keeps the rows' (s, m) words), then each lane owns 1, 2 or 4 rows
+// and every warp walks a range of the table, summing x_c (rho_ic + 1/2 -
+// 2^(r-1)) / 2^r over each run of channels that share a scale group and
+// scaling each run once.
 #include "common.cuh"
 #include "internal.cuh"
 
 namespace sf {
 namespace {
 
-constexpr int kSegChannels = 2048;  // 32 lanes x 64 channels
-constexpr int kWarps = 8;
-constexpr int kCtasPerSm = 2;
-constexpr int kXWords = 52;         // per 64-channel group: 16 vectors x 3 planes, sum, 2^e, pad
-constexpr int kCorrSmemWords = 12 * 1024;
+constexpr int kLaneCh = 64;                 // input channels per lane
+constexpr int kSegChannels = 32 * kLaneCh;  // 2,048 channels per warp segment
+constexpr int kWarps = 16;                  // one CTA of 16 warps per SM
+constexpr int kThreads = kWarps * 32;
+#ifndef SF_GEMV_XPLANES
+#define SF_GEMV_XPLANES 3
+#endif
+constexpr int kXP = SF_GEMV_XPLANES;        // byte planes of the fixed-point activations
+constexpr int kXShift = 8 * kXP - 4;        // x_fix = x * 2^-(ilogb(max|x|) - kXShift), |x_fix| < 2^(8 kXP - 3)
+constexpr int kXR = 16 * kXP;               // plane words per lane group
+constexpr int kXWords = kXR + 4;            // then sum0, sum1, 2^e, sum
+constexpr int kRowUnit = 4;                 // CTA row ranges start at multiples of 4
+constexpr int kPrepWarps = 8;
+constexpr size_t kSmemLimit = 227 * 1024;
 
 struct GemvParams {
   const uint32_t* base;
-  const uint32_t* refine;  // channel-major rows, or staged rows
+  const uint32_t* refine;  // channel-major rows, or staged rows [batch][n_sel]
   const uint16_t* sz;
-  const uint16_t* x;
-  const int32_t* sel;
+  const uint16_t* x;       // [batch][K] fp16
+  const uint32_t* xp;      // [batch][K/64][kXWords] prepared activations (mode 0)
+  const uint4* jdg;        // [batch][n_sel] correction table written by the prologue (mode 0)
+  const int32_t* sel;      // [batch][n_sel]
   float* y;
-  int N, K, G, r, batch, n_sel, segs, row_warps;
+  int N, K, G, gshift, r, batch, n_sel, segs;
   int refine_row_words;  // N * r / 32
   int staged;            // refine holds [batch][n_sel] staged rows
   int mode;              // 0: base + correction, 1: correction only, added into y
+  int rows_max;          // most rows a CTA owns
+  int area_words;        // shared words of the copy rings (reused by the slow correction path)
+  int fast;              // correction tables in their own shared region, filled before the base pass
+  int w_span;            // stride of the refinement-word table (words a CTA's rows can span)
+  int corr_rows;         // rows per lane in the correction (1, 2 or 4)
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -84,113 +110,129 @@ __device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c) {
   return d;
 }
 
-// Words of packed codes per lane per row (64 channels).
+// Per lane and row: CW words of codes (64 channels), U rows per task.
 template <int BITS>
 struct Lane {
-  static constexpr int W = BITS == 2 ? 4 : BITS == 3 ? 6 : 8;
-  static constexpr int U = BITS == 4 ? 2 : 4;  // rows per step
+  static constexpr int CW = BITS == 2 ? 4 : BITS == 3 ? 6 : 8;
+  static constexpr int U = BITS == 4 ? 2 : 4;
 };
 
-// Ring slot layout (per warp, words): codes [U][W/4 chunks][32 lanes][4 words]
-// (b = 3: then [U][32 lanes][2 words] of high bits), then sz [U][2][32 lanes].
-// Consecutive lanes read consecutive 16-byte chunks, so reads are conflict-free.
-template <int BITS>
+// Ring slot of one task (words): codes [U][C16][32 lanes][4] in 16-byte chunks,
+// for b = 3 then the high-bit words [U][32][2], then (s, m) [U][ZW][32].
+// Consecutive lanes read consecutive chunks, so reads are conflict-free.
+template <int BITS, int ZW>
 struct Ring {
-  static constexpr int W = Lane<BITS>::W, U = Lane<BITS>::U;
-  static constexpr int CW = BITS == 3 ? 4 : W;           // words in 16-byte chunks
-  static constexpr int slot_words = U * 32 * (W + 2);   // one item of U rows
+  static constexpr int CW = Lane<BITS>::CW, U = Lane<BITS>::U;
+  static constexpr int C16 = BITS == 3 ? 1 : CW / 4;
+  static constexpr int hi_off() { return U * C16 * 32 * 4; }
+  static constexpr int z_off = U * 32 * CW;
+  static constexpr int words = U * 32 * (CW + ZW);
 };
 
-template <int BITS>
-__device__ __forceinline__ void issue_row(const GemvParams& p, int row, int lg, int gpr, int g0,
-                                          int g1, uint32_t* slot, int u, int lane) {
-  using R = Ring<BITS>;
-  const uint8_t* rowbase;
-  if constexpr (BITS == 4) {
-    rowbase = reinterpret_cast<const uint8_t*>(p.base + (size_t)row * (p.K / 8)) + 32 * lg;
-  } else {
-    rowbase = reinterpret_cast<const uint8_t*>(p.base + (size_t)row * (p.K / 16)) + 16 * lg;
-  }
+// Copies of one row into ring slot position u: the lane's codes (lane_base:
+// the row-0 address of the lane's 16-byte chunks, row_bytes apart) and its
+// (s, m) word(s) (lane_z: row 0's, gpr words apart).
+template <int BITS, int ZW>
+__device__ __forceinline__ void issue_row(const uint8_t* lane_base, const uint8_t* lane_hi, size_t row_bytes,
+                                          const uint32_t* lane_z, int gpr, int row, uint32_t* slot, int u,
+                                          int lane) {
+  using R = Ring<BITS, ZW>;
+  const uint8_t* rb = lane_base + (size_t)row * row_bytes;
 #pragma unroll
-  for (int c = 0; c < R::CW / 4; c++)
-    cp_async16(slot + ((u * (R::CW / 4) + c) * 32 + lane) * 4, rowbase + 16 * c);
-  if constexpr (BITS == 3) {
-    const uint8_t* hb = reinterpret_cast<const uint8_t*>(p.base + (size_t)p.N * p.K / 16 +
-                                                         (size_t)row * (p.K / 32)) + 8 * lg;
-    cp_async8(slot + R::U * R::CW * 32 + (u * 32 + lane) * 2, hb);
-  }
-  uint32_t* zs = slot + R::U * 32 * R::W;
-  const uint32_t* szrow = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)row * gpr;
-  cp_async4(zs + (u * 2 + 0) * 32 + lane, szrow + g0);
-  if (g1 != g0) cp_async4(zs + (u * 2 + 1) * 32 + lane, szrow + g1);
-}
-
-template <int BITS>
-__device__ __forceinline__ void read_row(const uint32_t* slot, int u, int lane,
-                                         uint32_t (&w)[Lane<BITS>::W], uint32_t (&z)[2], bool split) {
-  using R = Ring<BITS>;
+  for (int c = 0; c < R::C16; c++) cp_async16(slot + ((u * R::C16 + c) * 32 + lane) * 4, rb + 16 * c);
+  if constexpr (BITS == 3) cp_async8(slot + R::hi_off() + (u * 32 + lane) * 2, lane_hi + (size_t)row * (row_bytes / 2));
+  const uint32_t* zr = lane_z + (size_t)row * gpr;
 #pragma unroll
-  for (int c = 0; c < R::CW / 4; c++) {
-    const uint4 v = *reinterpret_cast<const uint4*>(slot + ((u * (R::CW / 4) + c) * 32 + lane) * 4);
-    w[4 * c + 0] = v.x, w[4 * c + 1] = v.y, w[4 * c + 2] = v.z, w[4 * c + 3] = v.w;
-  }
-  if constexpr (BITS == 3) {
-    const uint2 h = *reinterpret_cast<const uint2*>(slot + R::U * R::CW * 32 + (u * 32 + lane) * 2);
-    w[4] = h.x, w[5] = h.y;
-  }
-  const uint32_t* zs = slot + R::U * 32 * R::W;
-  z[0] = zs[(u * 2 + 0) * 32 + lane];
-  z[1] = split ? zs[(u * 2 + 1) * 32 + lane] : z[0];
+  for (int h = 0; h < ZW; h++) cp_async4(slot + R::z_off + (u * ZW + h) * 32 + lane, zr + h);
 }
 
-// Code byte-vector v (0..15) of the lane's 64 channels; byte L holds the code
-// of channel chan_of(v, L) (0..63).
-template <int BITS>
-__device__ __forceinline__ uint32_t code_vec(const uint32_t (&w)[Lane<BITS>::W], int v) {
-  if constexpr (BITS == 4) {
-    return (w[v >> 1] >> (4 * (v & 1))) & 0x0F0F0F0Fu;  // word v/2: 8 channels
-  } else {
-    const int wi = v >> 2, j = v & 3;  // word wi: 16 channels
-    uint32_t c = (w[wi] >> (2 * j)) & 0x03030303u;
-    if constexpr (BITS == 3) {
-      const int sh = 4 * (wi & 1) + j;  // high bits of the 32-channel block wi/2
-      c |= ((w[4 + (wi >> 1)] >> sh) << 2) & 0x04040404u;
-    }
-    return c;
-  }
-}
-
+// Code byte vector v (0..15) of a lane's 64 channels; byte L holds the code of
+// channel chan_of(v, L).
 template <int BITS>
 __host__ __device__ __forceinline__ int chan_of(int v, int L) {
   if (BITS == 4) return 8 * (v >> 1) + (v & 1) + 2 * L;
   return 16 * (v >> 2) + (v & 3) + 4 * L;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+template <int BITS>
+__device__ __forceinline__ uint32_t code_vec(const uint32_t (&w)[Lane<BITS>::CW], int v) {
+  if constexpr (BITS == 4) {
+    return (w[v >> 1] >> (4 * (v & 1))) & 0x0F0F0F0Fu;
+  } else {
+    const int wi = v >> 2, j = v & 3;
+    uint32_t c = (w[wi] >> (2 * j)) & 0x03030303u;
+    if constexpr (BITS == 3) c |= ((w[4 + (wi >> 1)] >> (4 * (wi & 1) + j)) << 2) & 0x04040404u;
+    return c;
+  }
 }
 
-// Sum each of U per-lane values over the warp; lane (u * 32 / U) .. holds row u.
-// Returns the full sum of row (lane >> (5 - log2 U)) in every lane.
+// sum_c code_c * x_fix_c over the lane's 64 channels (ZW = 1) or over each
+// 32-channel half (ZW = 2), exact in 32-bit integers: |x_fix| < 2^(8 kXP - 3)
+// and codes < 16 keep every partial below 2^31 (intermediate wrap-around
+// cancels).  Plane p of vector v is xr[kXP v + p]; the top plane is signed.
+template <int BITS, int ZW>
+__device__ __forceinline__ void lane_dot(const uint32_t (&w)[Lane<BITS>::CW], const uint32_t (&xr)[kXR],
+                                         int32_t (&d)[ZW]) {
+  auto mac = [&](uint32_t c, int v, uint32_t (&acc)[kXP]) {
+#pragma unroll
+    for (int q = 0; q < kXP; q++)
+      acc[q] = q == kXP - 1 ? (uint32_t)dp4a_us(c, xr[kXP * v + q], (int32_t)acc[q]) : dp4a_uu(c, xr[kXP * v + q], acc[q]);
+  };
+  auto combine = [&](const uint32_t (&acc)[kXP]) {
+    uint32_t t = acc[0];
+#pragma unroll
+    for (int q = 1; q < kXP; q++) t += acc[q] << (8 * q);
+    return (int32_t)t;
+  };
+  if constexpr (BITS == 2) {
+    // c0 = w & 0x03.. (channels 4L), c1 = w & 0x0C.. = 4 x (channels 4L+1),
+    // the same on w >> 4 for 4L+2 and 4L+3: set A has factor 1, set B factor 4
+    uint32_t A[ZW][kXP], B[ZW][kXP];
+#pragma unroll
+    for (int h = 0; h < ZW; h++)
+#pragma unroll
+      for (int q = 0; q < kXP; q++) A[h][q] = B[h][q] = 0;
+#pragma unroll
+    for (int wi = 0; wi < 4; wi++) {
+      const int h = ZW == 2 ? (wi >> 1) : 0;
+      const uint32_t w0 = w[wi], w4 = w0 >> 4;
+      mac(w0 & 0x03030303u, 4 * wi + 0, A[h]);
+      mac(w0 & 0x0C0C0C0Cu, 4 * wi + 1, B[h]);
+      mac(w4 & 0x03030303u, 4 * wi + 2, A[h]);
+      mac(w4 & 0x0C0C0C0Cu, 4 * wi + 3, B[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < ZW; h++) d[h] = combine(A[h]) + (combine(B[h]) >> 2);
+  } else {
+    uint32_t A[ZW][kXP];
+#pragma unroll
+    for (int h = 0; h < ZW; h++)
+#pragma unroll
+      for (int q = 0; q < kXP; q++) A[h][q] = 0;
+#pragma unroll
+    for (int v = 0; v < 16; v++) mac(code_vec<BITS>(w, v), v, A[ZW == 2 ? (chan_of<BITS>(v, 0) >= 32) : 0]);
+#pragma unroll
+    for (int h = 0; h < ZW; h++) d[h] = combine(A[h]);
+  }
+}
+
+// Sum each of U per-lane values over the warp.  Returns the full sum of row
+// lane >> 3 (U = 4) or lane >> 4 (U = 2) in every lane.
 template <int U>
 __device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
   if constexpr (U == 4) {
-    // xor 16: lanes < 16 keep rows 0,1; lanes >= 16 keep rows 2,3
     const bool up = lane & 16;
     float k0 = up ? a[2] : a[0], k1 = up ? a[3] : a[1];
     float s0 = up ? a[0] : a[2], s1 = up ? a[1] : a[3];
     k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
     k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    // xor 8: keep one row
     const bool up8 = lane & 8;
     float k = up8 ? k1 : k0, s = up8 ? k0 : k1;
     k += __shfl_xor_sync(0xffffffffu, s, 8);
     k += __shfl_xor_sync(0xffffffffu, k, 4);
     k += __shfl_xor_sync(0xffffffffu, k, 2);
     k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;  // row 2*(lane>>4) + ((lane>>3)&1) = lane >> 3
+    return k;
   } else {
     const bool up = lane & 16;
     float k = up ? a[1] : a[0], s = up ? a[0] : a[1];
@@ -199,252 +241,332 @@ __device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
     k += __shfl_xor_sync(0xffffffffu, k, 4);
     k += __shfl_xor_sync(0xffffffffu, k, 2);
     k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;  // row lane >> 4
+    return k;
   }
 }
 
-// x of one batch row -> fixed-point byte planes per 64-channel group.
+// ---------------------------------------------------------------------------
+// correction table entries: (x_c, x_c (1 - off/2^r), group of c, word offset of
+// the refinement row of c), off = 1/2 - 2^(r-1)
+
+__device__ __forceinline__ uint4 make_jd(const GemvParams& p, int b, int j) {
+  const int c = __ldg(p.sel + (size_t)b * p.n_sel + j);
+  const float xc = h2f(__ldg(p.x + (size_t)b * p.K + c));
+  const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << p.r)) / (float)(1 << p.r);
+  const uint32_t off = p.staged ? (uint32_t)(((size_t)b * p.n_sel + j) * p.refine_row_words)
+                                : (uint32_t)((size_t)c * p.refine_row_words);
+  return make_uint4(__float_as_uint(xc), __float_as_uint(xc * cfac), (uint32_t)(c >> p.gshift), off);
+}
+
+// ---------------------------------------------------------------------------
+// activation prologue: one warp per (batch row, 64-channel lane group), then
+// (blocks past the plane blocks) the correction table of every batch row
+
 template <int BITS>
-__device__ void prep_x(const uint16_t* __restrict__ x, int K, uint16_t* xraw, uint32_t* xs) {
-  // all loads first (16 B per thread per step), then the per-group work
-  for (int i = threadIdx.x; i < K / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(xraw)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  uint8_t* xb = reinterpret_cast<uint8_t*>(xs);
-  for (int grp = warp; grp < K / 64; grp += nwarps) {
-    // lane handles channels 2*lane, 2*lane + 1 of the group
-    __half2 hv = reinterpret_cast<const __half2*>(xraw + grp * 64)[lane];
-    float2 xv = __half22float2(hv);
+__global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(GemvParams p, uint32_t* __restrict__ xp,
+                                                                   uint4* __restrict__ jdg, int plane_blocks) {
+  pdl_trigger();  // the GEMV may start streaming codes now
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ngrp = p.K / kLaneCh;
+  const int b = blockIdx.y;
+  if ((int)blockIdx.x >= plane_blocks) {
+    pdl_wait();  // the selection launched before this kernel (if any) is complete
+    const int j = (blockIdx.x - plane_blocks) * blockDim.x + threadIdx.x;
+    if (j < p.n_sel) jdg[(size_t)b * p.n_sel + j] = make_jd(p, b, j);
+    return;
+  }
+  const int grp = blockIdx.x * kPrepWarps + warp;
+  if (grp < ngrp) {
+    const float2 xv = __half22float2(
+        reinterpret_cast<const __half2*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh)[lane]);
     float mx = fmaxf(fabsf(xv.x), fabsf(xv.y));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const int e = mx > 0.f ? ilogbf(mx) - 22 : 0;  // |x| * 2^-e < 2^23
-    uint8_t* base = xb + (size_t)grp * kXWords * 4;
+    const int e = mx > 0.f ? ilogbf(mx) - kXShift : 0;
+    const int xf0 = __float2int_rn(ldexpf(xv.x, -e)), xf1 = __float2int_rn(ldexpf(xv.y, -e));
+    // lane v < 16 assembles the three plane words of code byte vector v
+    const int v = lane & 15;
+    uint32_t pl[kXP];
 #pragma unroll
-    for (int h = 0; h < 2; h++) {
-      const int c = 2 * lane + h;
-      const float xc = h ? xv.y : xv.x;
-      const int xf = mx > 0.f ? __float2int_rn(ldexpf(xc, -e)) : 0;
-      int v, L;
-      if (BITS == 4) {
-        v = 2 * (c >> 3) + (c & 1);
-        L = (c & 7) >> 1;
-      } else {
-        v = 4 * (c >> 4) + (c & 3);
-        L = (c & 15) >> 2;
-      }
-      uint8_t* dst = base + v * 12 + L;
-      dst[0] = (uint8_t)(xf & 0xff);
-      dst[4] = (uint8_t)((xf >> 8) & 0xff);
-      dst[8] = (uint8_t)((xf >> 16) & 0xff);
+    for (int q = 0; q < kXP; q++) pl[q] = 0;
+#pragma unroll
+    for (int L = 0; L < 4; L++) {
+      const int c = chan_of<BITS>(v, L);
+      const int a0 = __shfl_sync(0xffffffffu, xf0, c >> 1), a1 = __shfl_sync(0xffffffffu, xf1, c >> 1);
+      const uint32_t f = (uint32_t)((c & 1) ? a1 : a0);
+#pragma unroll
+      for (int q = 0; q < kXP; q++) pl[q] |= ((f >> (8 * q)) & 0xffu) << (8 * L);
     }
-    float s = warp_sum(xv.x + xv.y);
+    uint32_t* dst = xp + ((size_t)b * ngrp + grp) * kXWords;
+    if (lane < 16) {
+#pragma unroll
+      for (int q = 0; q < kXP; q++) dst[kXP * v + q] = pl[q];
+    }
+    float s = xv.x + xv.y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float s1 = __shfl_sync(0xffffffffu, s, 16);
     if (lane == 0) {
-      reinterpret_cast<float*>(base)[48] = s;
-      reinterpret_cast<float*>(base)[49] = ldexpf(1.0f, e);
+      reinterpret_cast<float*>(dst)[kXR + 0] = s;
+      reinterpret_cast<float*>(dst)[kXR + 1] = s1;
+      reinterpret_cast<float*>(dst)[kXR + 2] = ldexpf(1.0f, e);
+      reinterpret_cast<float*>(dst)[kXR + 3] = s + s1;
+    }
+  }
+  pdl_wait();  // the grid completes only after the selection launched before it
+}
+
+// ---------------------------------------------------------------------------
+// correction
+
+// Table entries [j0, j0 + jn) of batch row b into jd, and the refinement words
+// [w_lo, w_lo + nwr) of each entry's row into wt (stride nwr), by cp.async.
+__device__ void corr_fill(const GemvParams& p, int b, int j0, int jn, int w_lo, int nwr, uint4* jd,
+                          uint32_t* wt) {
+  for (int i = threadIdx.x; i < jn; i += kThreads) {
+    const uint4 d = p.mode == 0 ? __ldg(p.jdg + (size_t)b * p.n_sel + j0 + i) : make_jd(p, b, j0 + i);
+    jd[i] = d;
+    for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + d.w + w_lo + k);
+  }
+  cp_async_commit();
+}
+
+// Adds the correction of table entries [0, jn) into part[row][0].  Lanes own
+// RL consecutive rows (inside one refinement word); warps split the entries.
+// Entries come in ascending channel order, so channels of one scale group are
+// consecutive: each run is summed unscaled and multiplied by s once.  szt:
+// the CTA's (s, m) words [rows][gpr], or NULL (scales read from global).
+template <int RL>
+__device__ void corr_process(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
+                             const uint4* __restrict__ jd, const uint32_t* __restrict__ wt,
+                             const uint32_t* __restrict__ szt, float* part) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gpr = p.K >> p.gshift;
+  const int units = rows / RL;
+  const int nblk = (units + 31) / 32;
+  const int js_n = nblk >= kWarps ? 1 : kWarps / nblk;
+  const int ntasks = nblk * js_n;
+  const int r = p.r;
+  const uint32_t fmask = ((1u << r) - 1u) << (23 - r);
+  for (int task = warp; task < ntasks; task += kWarps) {
+    const int blk = task % nblk, js = task / nblk;
+    const int qu = blk * 32 + lane;
+    const bool ok = qu < units;
+    const int rl0 = RL * qu;
+    const int bit0 = (n0 + rl0) * r;
+    const int wr = (bit0 >> 5) - w_lo;
+    int rot[RL];
+#pragma unroll
+    for (int t = 0; t < RL; t++) rot[t] = (23 - r - ((bit0 & 31) + r * t)) & 31;
+    const int ia = (int)((long)js * jn / js_n), ib = (int)((long)(js + 1) * jn / js_n);
+    float acc[RL], run[RL];
+#pragma unroll
+    for (int t = 0; t < RL; t++) acc[t] = run[t] = 0.f;
+    float C = 0.f;
+    int gcur = -1;
+    auto flush = [&]() {
+      if (gcur >= 0 && ok) {
+#pragma unroll
+        for (int t = 0; t < RL; t++) {
+          const uint32_t zw = szt ? szt[(rl0 + t) * gpr + gcur]
+                                  : __ldg(reinterpret_cast<const uint32_t*>(p.sz) + (size_t)(n0 + rl0 + t) * gpr + gcur);
+          const float sc = __low2float(*reinterpret_cast<const __half2*>(&zw));
+          acc[t] = fmaf(sc, run[t] - C, acc[t]);
+        }
+      }
+    };
+    for (int i = ia; i < ib; i++) {
+      const uint4 d = jd[i];
+      if ((int)d.z != gcur) {
+        flush();
+        gcur = (int)d.z;
+        C = 0.f;
+#pragma unroll
+        for (int t = 0; t < RL; t++) run[t] = 0.f;
+      }
+      const uint32_t w = ok ? wt[(size_t)i * nwr + wr] : 0u;
+      const float xc = __uint_as_float(d.x);
+      // f = 1 + rho / 2^r; sum x f - sum x (1 - off/2^r) = sum x (rho + off) / 2^r
+#pragma unroll
+      for (int t = 0; t < RL; t++)
+        run[t] = fmaf(__uint_as_float(0x3F800000u | (__funnelshift_l(w, w, rot[t]) & fmask)), xc, run[t]);
+      C += __uint_as_float(d.y);
+    }
+    flush();
+    if (ok && ib > ia) {
+#pragma unroll
+      for (int t = 0; t < RL; t++) atomicAdd(&part[(rl0 + t) * p.segs], acc[t]);
     }
   }
 }
 
-template <int BITS>
-__device__ __forceinline__ float group_dot(const uint32_t (&w)[Lane<BITS>::W], const uint32_t (&xr)[48]) {
-  uint32_t lo = 0, mid = 0;
-  int32_t hi = 0;
-#pragma unroll
-  for (int v = 0; v < 16; v++) {
-    uint32_t c = code_vec<BITS>(w, v);
-    lo = dp4a_uu(c, xr[3 * v + 0], lo);
-    mid = dp4a_uu(c, xr[3 * v + 1], mid);
-    hi = dp4a_us(c, xr[3 * v + 2], hi);
-  }
-  return fmaf((float)hi, 65536.0f, (float)mid * 256.0f + (float)lo);
+__device__ __forceinline__ void corr_dispatch(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
+                                              const uint4* jd, const uint32_t* wt, const uint32_t* szt,
+                                              float* part) {
+  if (p.corr_rows == 4)
+    corr_process<4>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
+  else if (p.corr_rows == 2)
+    corr_process<2>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
+  else
+    corr_process<1>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
 }
 
-// Same, split into the two 32-channel halves (groups of 32 channels).
-template <int BITS>
-__device__ __forceinline__ float2 group_dot_halves(const uint32_t (&w)[Lane<BITS>::W],
-                                                   const uint32_t (&xr)[48]) {
-  uint32_t lo[2] = {0, 0}, mid[2] = {0, 0};
-  int32_t hi[2] = {0, 0};
-#pragma unroll
-  for (int v = 0; v < 16; v++) {
-    const int h = chan_of<BITS>(v, 0) >= 32;
-    uint32_t c = code_vec<BITS>(w, v);
-    lo[h] = dp4a_uu(c, xr[3 * v + 0], lo[h]);
-    mid[h] = dp4a_uu(c, xr[3 * v + 1], mid[h]);
-    hi[h] = dp4a_us(c, xr[3 * v + 2], hi[h]);
-  }
-  return make_float2(fmaf((float)hi[0], 65536.0f, (float)mid[0] * 256.0f + (float)lo[0]),
-                     fmaf((float)hi[1], 65536.0f, (float)mid[1] * 256.0f + (float)lo[1]));
-}
+// ---------------------------------------------------------------------------
+// the GEMV
 
-template <int BITS, int PD>
-__global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_kernel(GemvParams p) {
-  constexpr int W = Lane<BITS>::W, U = Lane<BITS>::U;
+template <int BITS, int ZW, int PD>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
+  using R = Ring<BITS, ZW>;
+  constexpr int U = Lane<BITS>::U, CW = Lane<BITS>::CW;
   extern __shared__ __align__(16) uint32_t smem[];
-  const int ngrp = p.K / 64;
-  uint32_t* xs = smem;                                       // ngrp * kXWords
-  float* part = reinterpret_cast<float*>(xs + ngrp * kXWords);  // rows x segs
-  const int n0 = (int)((long)blockIdx.x * p.N / gridDim.x);
-  const int n1 = (int)((long)(blockIdx.x + 1) * p.N / gridDim.x);
-  const int rows = n1 - n0;
-  // scratch: x staging (prologue), then the per-warp copy rings (base pass),
-  // then the correction staging
-  uint32_t* scratch = reinterpret_cast<uint32_t*>(part + ((rows * p.segs + 3) & ~3));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = warp % p.segs, rw = warp / p.segs;
-  const bool warp_active = p.mode == 0 && rw < p.row_warps;
-  const int lg = seg * 32 + lane;  // lane's 64-channel group
-  const bool lane_active = warp_active && lg < ngrp;
-  const int G = p.G;
-  const bool split = G == 32;
+  const int units = p.N / kRowUnit;
+  const int n0 = (int)((long)blockIdx.x * units / gridDim.x) * kRowUnit;
+  const int n1 = (int)((long)(blockIdx.x + 1) * units / gridDim.x) * kRowUnit;
+  const int rows = n1 - n0;
+  const int ngrp = p.K / kLaneCh, gpr = p.K >> p.gshift;
+  // shared memory: partial sums [rows][segs] | rings | (fast) table, words, scales
+  float* part = reinterpret_cast<float*>(smem);
+  uint32_t* area = smem + ((p.rows_max * p.segs + 3) & ~3);
+  uint4* jd_fast = reinterpret_cast<uint4*>(area + p.area_words);
+  uint32_t* wt_fast = reinterpret_cast<uint32_t*>(jd_fast + p.n_sel);
+  uint32_t* szt = wt_fast + (((size_t)p.n_sel * p.w_span + 3) & ~(size_t)3);
+  const int w_lo = (n0 * p.r) >> 5;
+  const int nwr = (((n1 * p.r) + 31) >> 5) - w_lo;
+  const int steps = (rows + U - 1) / U, ntask = p.segs * steps;
+  const int ta = (int)((long)warp * ntask / kWarps), tb = (int)((long)(warp + 1) * ntask / kWarps);
+  const size_t row_bytes = (size_t)p.K * (BITS == 3 ? 2 : BITS) / 8;
+  const bool fill_szt = p.fast && p.mode == 0 && p.n_sel > 0;
 
   for (int b = 0; b < p.batch; b++) {
-    const uint16_t* xrow = p.x + (size_t)b * p.K;
     if (p.mode == 0) {
-      // every (row, segment) partial is written by exactly one warp below
-      prep_x<BITS>(xrow, p.K, reinterpret_cast<uint16_t*>(scratch), xs);
-    } else {
-      for (int i = threadIdx.x; i < rows * p.segs; i += blockDim.x) part[i] = 0.f;
-    }
-    __syncthreads();
-    if (warp_active) {
-      uint32_t xr[48];
-      float xsum = 0.f, xscale = 0.f;
-      if (lane_active) {
-        const uint4* src = reinterpret_cast<const uint4*>(xs + lg * kXWords);
+      // ---- base pass of batch row b: every (row, segment) partial is written once
+      uint32_t* ring = area + warp * PD * R::words;
+      const uint32_t* xpb = p.xp + (size_t)b * ngrp * kXWords;
+      int iseg = ta / steps, ist = ta - iseg * steps, islot = 0, left = tb - ta;
+      auto issue = [&]() {
+        if (left > 0) {
+          const int lg = iseg * 32 + lane;
+          if (lg < ngrp) {
+            const uint8_t* lb = reinterpret_cast<const uint8_t*>(p.base) + 16 * R::C16 * lg;
+            const uint8_t* lh = reinterpret_cast<const uint8_t*>(p.base) + (size_t)p.N * p.K / 4 + 8 * lg;
+            const uint32_t* lz = reinterpret_cast<const uint32_t*>(p.sz) + ((lg * kLaneCh) >> p.gshift);
+            uint32_t* slot = ring + islot * R::words;
+            const int r0 = n0 + ist * U;
 #pragma unroll
-        for (int i = 0; i < 12; i++) {
-          uint4 v = src[i];
-          xr[4 * i + 0] = v.x, xr[4 * i + 1] = v.y, xr[4 * i + 2] = v.z, xr[4 * i + 3] = v.w;
-        }
-        xsum = __uint_as_float(xs[lg * kXWords + 48]);
-        xscale = __uint_as_float(xs[lg * kXWords + 49]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 48; i++) xr[i] = 0;
-      }
-      // sums of x over the two 32-channel halves (groups of 32 only)
-      float xs0 = 0.f, xs1 = 0.f;
-      if (split && lane_active) {
-        const __half2* xh = reinterpret_cast<const __half2*>(xrow + lg * 64);
-        for (int i = 0; i < 16; i++) {
-          float2 a = __half22float2(xh[i]), c = __half22float2(xh[16 + i]);
-          xs0 += a.x + a.y;
-          xs1 += c.x + c.y;
-        }
-      }
-      const int gpr = p.K / G;
-      const int g0 = (lg * 64) / G, g1 = (lg * 64 + 32) / G;
-      const int step = p.row_warps * U;
-      const int first = n0 + rw * U;
-      const int nitems = first < n1 ? (n1 - first + step - 1) / step : 0;
-      uint32_t* ring = scratch + warp * PD * Ring<BITS>::slot_words;
-      auto issue = [&](int k) {
-        if (k < nitems && lane_active) {
-          uint32_t* slot = ring + (k % PD) * Ring<BITS>::slot_words;
-#pragma unroll
-          for (int u = 0; u < U; u++) {
-            const int row = first + k * step + u;
-            if (row < n1) issue_row<BITS>(p, row, lg, gpr, g0, g1, slot, u, lane);
+            for (int u = 0; u < U; u++) issue_row<BITS, ZW>(lb, lh, row_bytes, lz, gpr, r0 + u, slot, u, lane);
           }
+          if (++ist == steps) ist = 0, ++iseg;
+          --left;
         }
+        islot = islot + 1 == PD ? 0 : islot + 1;
         cp_async_commit();
       };
 #pragma unroll
-      for (int k = 0; k < PD - 1; k++) issue(k);
-      for (int k = 0; k < nitems; k++) {
-        issue(k + PD - 1);
+      for (int i = 0; i < PD - 1; i++) issue();
+      if (b == 0) pdl_wait();  // prepared activations, selection and staged rows are complete
+      if (p.fast && p.n_sel > 0) corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
+      uint32_t xr[kXR];
+      float xsum0 = 0.f, xsum1 = 0.f, xscale = 0.f;
+      int cseg = ta / steps, cst = ta - cseg * steps, cslot = 0, cur = -1;
+      for (int t = ta; t < tb; t++) {
+        issue();
+        const int lg = cseg * 32 + lane;
+        const bool la = lg < ngrp;
+        if (cseg != cur) {
+          cur = cseg;
+          if (la) {
+            const uint4* src = reinterpret_cast<const uint4*>(xpb + (size_t)lg * kXWords);
+#pragma unroll
+            for (int k = 0; k < kXR / 4; k++) {
+              const uint4 q = __ldg(src + k);
+              xr[4 * k + 0] = q.x, xr[4 * k + 1] = q.y, xr[4 * k + 2] = q.z, xr[4 * k + 3] = q.w;
+            }
+            const float4 f = __ldg(reinterpret_cast<const float4*>(src + kXR / 4));
+            xsum0 = ZW == 2 ? f.x : f.w, xsum1 = f.y, xscale = f.z;
+          } else {
+#pragma unroll
+            for (int k = 0; k < kXR; k++) xr[k] = 0;
+            xsum0 = xsum1 = xscale = 0.f;
+          }
+        }
         cp_async_wait<PD - 1>();
-        const uint32_t* slot = ring + (k % PD) * Ring<BITS>::slot_words;
-        const int i0 = first + k * step;
+        const uint32_t* slot = ring + cslot * R::words;
+        const int r0 = n0 + cst * U;
+        const int zg = (lg * kLaneCh) >> p.gshift;
+        const bool zown = fill_szt && la && ((lg * kLaneCh) & (p.G - 1)) == 0;
         float acc[U];
 #pragma unroll
         for (int u = 0; u < U; u++) {
           acc[u] = 0.f;
-          if (lane_active && i0 + u < n1) {
-            uint32_t w[W], z[2];
-            read_row<BITS>(slot, u, lane, w, z, split);
-            float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&z[0]));
-            if (!split) {
-              const float d = group_dot<BITS>(w, xr) * xscale;
-              acc[u] = fmaf(s0.x, d, s0.y * xsum);
+          if (la) {
+            uint32_t w[CW];
+#pragma unroll
+            for (int c = 0; c < R::C16; c++) {
+              const uint4 q = *reinterpret_cast<const uint4*>(slot + ((u * R::C16 + c) * 32 + lane) * 4);
+              w[4 * c + 0] = q.x, w[4 * c + 1] = q.y, w[4 * c + 2] = q.z, w[4 * c + 3] = q.w;
+            }
+            if constexpr (BITS == 3) {
+              const uint2 h = *reinterpret_cast<const uint2*>(slot + R::hi_off() + (u * 32 + lane) * 2);
+              w[4] = h.x, w[5] = h.y;
+            }
+            int32_t d[ZW];
+            lane_dot<BITS, ZW>(w, xr, d);
+            const uint32_t z0 = slot[R::z_off + (u * ZW) * 32 + lane];
+            const float2 sm0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
+            if constexpr (ZW == 1) {
+              acc[u] = fmaf(sm0.x * xscale, (float)d[0], sm0.y * xsum0);
+              if (zown) szt[(r0 + u - n0) * gpr + zg] = z0;
             } else {
-              float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&z[1]));
-              const float2 d = group_dot_halves<BITS>(w, xr);
-              acc[u] = fmaf(s0.x, d.x * xscale, fmaf(s1.x, d.y * xscale, fmaf(s0.y, xs0, s1.y * xs1)));
+              const uint32_t z1 = slot[R::z_off + (u * ZW + 1) * 32 + lane];
+              const float2 sm1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
+              acc[u] = fmaf(sm0.x * xscale, (float)d[0],
+                            fmaf(sm1.x * xscale, (float)d[1], fmaf(sm0.y, xsum0, sm1.y * xsum1)));
+              if (fill_szt && la) szt[(r0 + u - n0) * gpr + zg] = z0, szt[(r0 + u - n0) * gpr + zg + 1] = z1;
             }
           }
         }
         const float tot = warp_sum_rows<U>(acc, lane);
         const int u = U == 4 ? (lane >> 3) : (lane >> 4);
-        const int row = i0 + u;
-        if ((lane & (32 / U - 1)) == 0 && row < n1) part[(row - n0) * p.segs + seg] = tot;
+        if ((lane & (32 / U - 1)) == 0) part[(r0 + u - n0) * p.segs + cseg] = tot;
+        if (++cst == steps) cst = 0, ++cseg;
+        cslot = cslot + 1 == PD ? 0 : cslot + 1;
       }
       cp_async_wait<0>();
+    } else {
+      for (int i = threadIdx.x; i < rows * p.segs; i += kThreads) part[i] = 0.f;
+      if (p.fast) {
+        // the CTA's (s, m) words are one contiguous block of sz
+        const uint32_t* zsrc = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)n0 * gpr;
+        for (int i = threadIdx.x; i < rows * gpr / 4; i += kThreads) cp_async16(szt + 4 * i, zsrc + 4 * i);
+        corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
+        cp_async_wait<0>();
+      }
     }
     __syncthreads();
 
     // ---- correction of the selected channels of batch row b
     if (p.n_sel > 0) {
-      pdl_wait();  // selection (and staged rows) complete and visible
-      const int32_t* sel = p.sel + (size_t)b * p.n_sel;
-      const int w0 = (n0 * p.r) >> 5;
-      const int nw = (((n1 * p.r) + 31) >> 5) - w0;
-      const float half = 0.5f * (float)(1 << p.r), inv = 1.0f / (float)(1 << p.r);
-      const int per_sel = 2 + nw;
-      const bool staged_smem = (long)p.n_sel * per_sel <= kCorrSmemWords;
-      if (staged_smem) {
-        // [n_sel] x * 2^-r, [n_sel] group, [n_sel][nw] refinement words
-        float* cx = reinterpret_cast<float*>(scratch);
-        int* cg = reinterpret_cast<int*>(cx + p.n_sel);
-        uint32_t* cw = reinterpret_cast<uint32_t*>(cg + p.n_sel);
-        for (int j = threadIdx.x; j < p.n_sel; j += blockDim.x) {
-          const int c = __ldg(sel + j);
-          cx[j] = h2f(__ldg(xrow + c)) * inv;
-          cg[j] = c / G;
-        }
-        for (int i = threadIdx.x; i < p.n_sel * nw; i += blockDim.x) {
-          const int j = i / nw, k = i % nw;
-          const uint32_t* rrow = p.staged ? p.refine + ((size_t)b * p.n_sel + j) * p.refine_row_words
-                                          : p.refine + (size_t)__ldg(sel + j) * p.refine_row_words;
-          cw[j * nw + k] = __ldg(rrow + w0 + k);
-        }
-        __syncthreads();
-        const int nwarps = blockDim.x >> 5;
-        for (int row = n0 + warp; row < n1; row += nwarps) {
-          const int bit = row * p.r - w0 * 32;
-          const uint16_t* zr = p.sz + (size_t)row * (p.K / G) * 2;
-          float corr = 0.f;
-          for (int j = lane; j < p.n_sel; j += 32) {
-            const uint32_t rho = (cw[j * nw + (bit >> 5)] >> (bit & 31)) & ((1u << p.r) - 1);
-            const float s = h2f(__ldg(zr + 2 * cg[j]));
-            corr = fmaf(cx[j] * s, (float)rho + 0.5f - half, corr);
-          }
-          corr = warp_sum(corr);
-          if (lane == 0) part[(row - n0) * p.segs] += corr;
-        }
+      if (p.fast) {
+        corr_dispatch(p, n0, rows, w_lo, nwr, p.n_sel, jd_fast, wt_fast, szt, part);
       } else {
-        const int nwarps = blockDim.x >> 5;
-        for (int row = n0 + warp; row < n1; row += nwarps) {
-          float corr = 0.f;
-          const int rbit = row * p.r;
-          for (int j = lane; j < p.n_sel; j += 32) {
-            const int c = __ldg(sel + j);
-            const uint32_t* rrow = p.staged ? p.refine + ((size_t)b * p.n_sel + j) * p.refine_row_words
-                                            : p.refine + (size_t)c * p.refine_row_words;
-            const uint32_t rho = (__ldg(rrow + (rbit >> 5)) >> (rbit & 31)) & ((1u << p.r) - 1);
-            const float s = h2f(__ldg(p.sz + ((size_t)row * (p.K / G) + c / G) * 2));
-            corr = fmaf(h2f(__ldg(xrow + c)) * inv * s, (float)rho + 0.5f - half, corr);
-          }
-          corr = warp_sum(corr);
-          if (lane == 0) part[(row - n0) * p.segs] += corr;
+        // tables in chunks in the ring area; scales from global memory
+        const int jcap = p.area_words / (4 + nwr);
+        uint4* jd = reinterpret_cast<uint4*>(area);
+        for (int j0 = 0; j0 < p.n_sel; j0 += jcap) {
+          const int jn = min(jcap, p.n_sel - j0);
+          uint32_t* wt = reinterpret_cast<uint32_t*>(jd + jn);
+          corr_fill(p, b, j0, jn, w_lo, nwr, jd, wt);
+          cp_async_wait<0>();
+          __syncthreads();
+          corr_dispatch(p, n0, rows, w_lo, nwr, jn, jd, wt, nullptr, part);
+          __syncthreads();
         }
       }
-      __syncthreads();
     }
-    for (int row = n0 + threadIdx.x; row < n1; row += blockDim.x) {
+    __syncthreads();
+
+    for (int row = n0 + threadIdx.x; row < n1; row += kThreads) {
       float acc = 0.f;
       for (int s = 0; s < p.segs; s++) acc += part[(row - n0) * p.segs + s];
       float* dst = p.y + (size_t)b * p.N + row;
@@ -454,16 +576,47 @@ __global__ void __launch_bounds__(kWarps * 32, kCtasPerSm) gemv_kernel(GemvParam
   }
 }
 
+// ---------------------------------------------------------------------------
+// host side
+
+size_t prep_bytes(const sf_wq* w, int batch, int n_sel) {
+  return (size_t)batch * (w->k / kLaneCh) * kXWords * 4 + (size_t)batch * n_sel * 16;
+}
+
+size_t slot_words(int bits, int zw) {
+  if (bits == 2) return zw == 1 ? Ring<2, 1>::words : Ring<2, 2>::words;
+  if (bits == 3) return zw == 1 ? Ring<3, 1>::words : Ring<3, 2>::words;
+  return zw == 1 ? Ring<4, 1>::words : Ring<4, 2>::words;
+}
+
+// Ring depth: 4 stages (3 for b = 3, whose stages are larger).
+template <int BITS, int ZW>
+void* kernel_for() {
+  return (void*)gemv_kernel<BITS, ZW, BITS == 3 ? 3 : 4>;
+}
+
+// Rows per lane in the correction: the fewest warp steps, counting ~6 + 3 RL
+// instructions per step of RL rows.
+int pick_corr_rows(int rows) {
+  int best = 1;
+  long best_cost = -1;
+  for (int rl = 1; rl <= 4; rl *= 2) {
+    const long blocks = (rows / rl + 31) / 32;
+    const long cost = blocks * (6 + 3 * rl);
+    if (best_cost < 0 || cost < best_cost) best = rl, best_cost = cost;
+  }
+  return best;
+}
+
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                       const int32_t* sel_in, int32_t* sel_out, const void* refine_rows, float* y,
-                      int mode, cudaStream_t s) {
+                      void* ws, size_t ws_bytes, int mode, cudaStream_t s) {
   sf_status st = check_wq_public(w, false);
   if (st != SF_OK) return st;
   SF_REQUIRE(x && aligned16(x), "x must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(y && aligned16(y), "y must be a non-null 16-byte aligned device pointer");
   SF_UNSUPPORTED(batch >= 1 && batch <= 8, "batch=%d outside [1, 8]", batch);
   SF_REQUIRE(kch >= 0, "kch=%d < 0", kch);
-  const int32_t* sel = nullptr;
   int n_sel = 0;
   if (kch > 0) {
     st = check_select_args(x, batch, w->k, chunk, kch);
@@ -473,77 +626,115 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
     SF_REQUIRE(!refine_rows || aligned16(refine_rows), "refine_rows must be 16-byte aligned");
     if (sel_in) {
       SF_REQUIRE(aligned16(sel_in), "sel_in must be 16-byte aligned");
-      sel = sel_in;
     } else {
+      SF_REQUIRE(mode == 0, "the correction-only call needs a selection");
       SF_REQUIRE(sel_out && aligned16(sel_out), "sel_out is needed when sel_in is NULL");
-      st = launch_select(x, batch, w->k, chunk, kch, sel_out, s);
-      if (st != SF_OK) return st;
-      sel = sel_out;
     }
   } else if (mode == 1) {
     return SF_OK;  // nothing to correct
   }
-  GemvParams p;
+  if (mode == 0) {
+    const size_t need = prep_bytes(w, batch, n_sel);
+    if (ws_bytes < need || !ws) {
+      set_error("workspace: need %zu bytes, got %zu", need, ws_bytes);
+      return SF_ERR_WORKSPACE;
+    }
+    SF_REQUIRE(aligned16(ws), "ws must be 16-byte aligned");
+  }
+
+  GemvParams p = {};
   p.base = (const uint32_t*)w->base;
   p.refine = (const uint32_t*)(refine_rows ? refine_rows : w->refine);
   p.sz = w->sz;
   p.x = x;
-  p.sel = sel;
   p.y = y;
   p.N = w->n, p.K = w->k, p.G = w->group, p.r = w->r, p.batch = batch, p.n_sel = n_sel;
+  p.gshift = 0;
+  while ((1 << p.gshift) < w->group) p.gshift++;
   p.mode = mode;
   p.segs = (w->k + kSegChannels - 1) / kSegChannels;
-  SF_UNSUPPORTED(p.segs <= kWarps, "k=%d above %d", w->k, kWarps * kSegChannels);
   p.refine_row_words = w->n * w->r / 32;
   p.staged = refine_rows != nullptr;
-  const int U = w->b == 4 ? 2 : 4;
-  const int W = w->b == 2 ? 4 : w->b == 3 ? 6 : 8;
-  const size_t slot_bytes = (size_t)U * 32 * (W + 2) * 4;
-  const size_t xs_bytes = (size_t)(w->k / 64) * kXWords * 4;
-  const size_t xraw_bytes = (size_t)w->k * 2;
-  const size_t corr_bytes = (size_t)kCorrSmemWords * 4;
-  auto smem_for = [&](int ctas_per_sm, int pd) {
-    int grid = ctas_per_sm * num_sms();
-    if (grid > w->n / 4) grid = w->n / 4;
-    const size_t rows = (w->n + grid - 1) / grid;
-    const size_t segs = (w->k + kSegChannels - 1) / kSegChannels;
-    const size_t part = ((rows * segs + 3) & ~(size_t)3) * 4;
-    size_t scratch = (size_t)kWarps * pd * slot_bytes;
-    if (scratch < xraw_bytes) scratch = xraw_bytes;
-    if (scratch < corr_bytes) scratch = corr_bytes;
-    return xs_bytes + part + scratch;
-  };
-  const size_t per_sm = 227 * 1024;
-  int ctas = kCtasPerSm, pd = 3;
-  if (smem_for(ctas, 3) * ctas > per_sm - ctas * 1024) pd = 2;
-  if (smem_for(ctas, pd) * ctas > per_sm - ctas * 1024) ctas = 1, pd = 3;
-  int grid = ctas * num_sms();
-  if (grid > w->n / 4) grid = w->n / 4;
-  const int rows_per_cta = (w->n + grid - 1) / grid;
-  p.row_warps = kWarps / p.segs;
-  const int needed = (rows_per_cta + U - 1) / U;
-  if (p.row_warps > needed) p.row_warps = needed;
-  if (p.row_warps < 1) p.row_warps = 1;
-  const size_t smem = smem_for(ctas, pd);
-  SF_UNSUPPORTED(smem <= 200 * 1024, "k=%d needs too much shared memory", w->k);
+  if (mode == 0) {
+    p.xp = (const uint32_t*)ws;
+    p.jdg = reinterpret_cast<const uint4*>((const char*)ws + (size_t)batch * (w->k / kLaneCh) * kXWords * 4);
+  }
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
+  const int zw = w->group == 32 ? 2 : 1;
+  const int pd = w->b == 3 ? 3 : 4;
+  int grid = num_sms();
+  const int units = w->n / kRowUnit;
+  if (grid > units) grid = units;
+  p.rows_max = ((units + grid - 1) / grid) * kRowUnit;
+  p.w_span = p.rows_max * w->r / 32 + 2;
+  p.corr_rows = pick_corr_rows(p.rows_max);
+  const size_t gpr = (size_t)(w->k / w->group);
+  const size_t part_words = ((size_t)p.rows_max * p.segs + 3) & ~(size_t)3;
+  size_t area = mode == 0 ? (size_t)kWarps * pd * slot_words(w->b, zw) : 0;
+  const size_t table_words = (size_t)n_sel * 4 + (((size_t)n_sel * p.w_span + 3) & ~(size_t)3) +
+                             (size_t)p.rows_max * gpr;
+  const size_t limit_words = kSmemLimit / 4;
+  p.fast = n_sel > 0 && part_words + area + table_words <= limit_words;
+  if (!p.fast && n_sel > 0) {
+    // slow path: chunks of the table in the ring area (grown for the correction-only call)
+    const size_t min_area = (size_t)(4 + p.w_span) * 64;
+    if (area < min_area) area = min_area;
+    if (mode == 1) area = limit_words - part_words;
+  }
+  if (area < 4) area = 4;
+  const size_t smem = (part_words + area + (p.fast ? table_words : 0)) * 4;
+  SF_UNSUPPORTED(smem <= kSmemLimit, "n=%d, k=%d needs %zu bytes of shared memory", w->n, w->k, smem);
+  p.area_words = (int)area;
+
+  // 1. the selection (when not given), 2. the activation prologue, 3. the GEMV
+  bool chained = false;
+  if (kch > 0 && !sel_in) {
+    st = launch_select(x, batch, w->k, chunk, kch, sel_out, s);
+    if (st != SF_OK) return st;
+    p.sel = sel_out;
+    chained = true;
+  } else {
+    p.sel = sel_in;
+  }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = (kch > 0 && !sel_in) ? 1 : 0;
+  if (mode == 0) {
+    const int plane_blocks = (w->k / kLaneCh + kPrepWarps - 1) / kPrepWarps;
+    const int jd_blocks = (n_sel + kPrepWarps * 32 - 1) / (kPrepWarps * 32);
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(plane_blocks + jd_blocks, batch);
+    pc.blockDim = dim3(kPrepWarps * 32);
+    pc.stream = s;
+    attr[0].val.programmaticStreamSerializationAllowed = chained ? 1 : 0;
+    pc.attrs = attr;
+    pc.numAttrs = 1;
+    uint32_t* xp = (uint32_t*)ws;
+    uint4* jdg = const_cast<uint4*>(p.jdg);
+    if (w->b == 4)
+      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<4>, p, xp, jdg, plane_blocks));
+    else if (w->b == 3)
+      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<3>, p, xp, jdg, plane_blocks));
+    else
+      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<2>, p, xp, jdg, plane_blocks));
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].val.programmaticStreamSerializationAllowed = mode == 0 ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void (*kern)(GemvParams);
-  if (pd == 3)
-    kern = w->b == 2 ? gemv_kernel<2, 3> : w->b == 3 ? gemv_kernel<3, 3> : gemv_kernel<4, 3>;
+  void* kern;
+  if (w->b == 2)
+    kern = zw == 1 ? kernel_for<2, 1>() : kernel_for<2, 2>();
+  else if (w->b == 3)
+    kern = zw == 1 ? kernel_for<3, 1>() : kernel_for<3, 2>();
   else
-    kern = w->b == 2 ? gemv_kernel<2, 2> : w->b == 3 ? gemv_kernel<3, 2> : gemv_kernel<4, 2>;
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-  SF_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
+    kern = zw == 1 ? kernel_for<4, 1>() : kernel_for<4, 2>();
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit));
+  void* args[] = {&p};
+  SF_CUDA(cudaLaunchKernelExC(&cfg, kern, args));
   return SF_OK;
 }
 
@@ -553,21 +744,23 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
 using namespace sf;
 
 extern "C" size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch) {
-  (void)w, (void)batch, (void)chunk, (void)kch;
-  return 0;
+  if (!w || w->k <= 0 || batch <= 0) return 0;
+  const int n_sel = (kch > 0 && chunk > 0) ? (w->k / chunk) * kch : 0;
+  return prep_bytes(w, batch, n_sel);
 }
 
 extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk,
                                      int kch, const int32_t* sel_in, int32_t* sel_out,
                                      const void* refine_rows, float* y, void* ws, size_t ws_bytes,
                                      sf_stream_t stream) {
-  (void)ws, (void)ws_bytes;
-  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, 0, as_stream(stream));
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, ws, ws_bytes, 0,
+                     as_stream(stream));
 }
 
 extern "C" sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch, int chunk,
                                         int kch, const int32_t* sel, const void* refine_rows,
                                         float* y, sf_stream_t stream) {
   SF_REQUIRE(kch == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
-  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, 1, as_stream(stream));
+  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, nullptr, 0, 1,
+                     as_stream(stream));
 }

@@ -148,7 +148,7 @@ struct WarpSmem {
 
 // GQP: query heads per KV head padded to 4 or 8.  B: base bits (2 or 4).
 template <int GQP, int B, bool PV>
-__global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
+__global__ void __launch_bounds__(kWarps * 32, GQP == 4 ? 4 : 2) kv_base_kernel(BaseArgs a) {
   using St = Stage<B, PV>;
   using WS = WarpSmem<B, PV>;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -196,12 +196,15 @@ __global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
 
   // softmax state of heads 2tig, 2tig+1 (the lane's logit and output columns)
   float mrun0 = -INFINITY, mrun1 = -INFINITY, lsum0 = 0.f, lsum1 = 0.f;
-  float accv[8][4];
-  float mt[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p m'_t,j of head gid
+  constexpr int NT = GQP == 4 ? 1 : 2;  // value-side n-tiles (hi/lo of 8 heads: two)
+  float accv[NT][8][4];
+  float mt[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t p m'_t,j of the B-operand head
 #pragma unroll
-  for (int m = 0; m < 8; m++)
+  for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-    for (int i = 0; i < 4; i++) accv[m][i] = 0.f;
+    for (int m = 0; m < 8; m++)
+#pragma unroll
+      for (int i = 0; i < 4; i++) accv[nt][m][i] = 0.f;
 
   auto issue = [&](int it) {
     if (it < ntile) {
@@ -320,33 +323,56 @@ __global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
       Ps[gid * 9 + h1] = p[1];
       Ps[(gid + 8) * 9 + h0] = p[2];
       Ps[(gid + 8) * 9 + h1] = p[3];
-      // rescale factor of head gid (held by the lanes with tig = gid / 2)
-      const float ala = __shfl_sync(0xffffffffu, al0, gid >> 1);
-      const float alb = __shfl_sync(0xffffffffu, al1, gid >> 1);
-      const float alg = (gid & 1) ? alb : ala;
+      // rescale factors of the heads of the lane's output columns; with four
+      // heads the columns are (head, hi/lo part): tig < 2 hi, tig >= 2 lo of
+      // heads 2(tig&1), 2(tig&1)+1, held by lane tig ^ 2 in the logit layout
+      float ac0 = al0, ac1 = al1;
+      if constexpr (GQP == 4) {
+        const float x0 = __shfl_xor_sync(0xffffffffu, al0, 2), x1 = __shfl_xor_sync(0xffffffffu, al1, 2);
+        if (tig >= 2) ac0 = x0, ac1 = x1;
+      }
+      // rescale factor of the B-operand head (held by the lanes with tig = hb / 2)
+      const int hb = GQP == 4 ? (gid & 3) : gid;
+      const float ala = __shfl_sync(0xffffffffu, al0, hb >> 1);
+      const float alb = __shfl_sync(0xffffffffu, al1, hb >> 1);
+      const float alg = (hb & 1) ? alb : ala;
       __syncwarp();
-      // B operand: fp16(p * s) of head gid for the lane's tokens 2tig, 2tig+1,
-      // 2tig+8, 2tig+9; the offsets m' go to the fp32 m-term
+      // B operand: p * s of head hb for the lane's tokens 2tig, 2tig+1,
+      // 2tig+8, 2tig+9, split into an fp16 high part and an fp16 low part
+      // (v - hi) so the product keeps ~22 bits; the offsets m' go to the fp32
+      // m-term.  Four heads: lanes gid < 4 carry hi, gid >= 4 lo (one n-tile).
+      // Eight heads: n-tile 0 hi, n-tile 1 lo.
       const float* zv = Zs + 16 * 8;
       float pv[4];
 #pragma unroll
-      for (int i = 0; i < 4; i++) pv[i] = Ps[(2 * tig + (i & 1) + 8 * (i >> 1)) * 9 + gid];
-      uint32_t bf[4][2];
+      for (int i = 0; i < 4; i++) pv[i] = Ps[(2 * tig + (i & 1) + 8 * (i >> 1)) * 9 + hb];
+      uint32_t bf[NT][4][2];
 #pragma unroll
       for (int jj = 0; jj < 2; jj++) {
         float4 z[4];
 #pragma unroll
         for (int i = 0; i < 4; i++)
           z[i] = reinterpret_cast<const float4*>(zv + (2 * tig + (i & 1) + 8 * (i >> 1)) * 8)[jj];
-        // group 2jj: (z.x, z.y); group 2jj+1: (z.z, z.w)
-        __half2 b00 = __floats2half2_rn(pv[0] * z[0].x, pv[1] * z[1].x);
-        __half2 b01 = __floats2half2_rn(pv[2] * z[2].x, pv[3] * z[3].x);
-        __half2 b10 = __floats2half2_rn(pv[0] * z[0].z, pv[1] * z[1].z);
-        __half2 b11 = __floats2half2_rn(pv[2] * z[2].z, pv[3] * z[3].z);
-        bf[2 * jj][0] = *reinterpret_cast<uint32_t*>(&b00);
-        bf[2 * jj][1] = *reinterpret_cast<uint32_t*>(&b01);
-        bf[2 * jj + 1][0] = *reinterpret_cast<uint32_t*>(&b10);
-        bf[2 * jj + 1][1] = *reinterpret_cast<uint32_t*>(&b11);
+#pragma unroll
+        for (int e = 0; e < 2; e++) {  // group 2jj + e
+          float v[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++) v[i] = pv[i] * (e ? z[i].z : z[i].x);
+          const __half2 h01 = __floats2half2_rn(v[0], v[1]), h23 = __floats2half2_rn(v[2], v[3]);
+          const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+          const __half2 l01 = __floats2half2_rn(v[0] - f01.x, v[1] - f01.y);
+          const __half2 l23 = __floats2half2_rn(v[2] - f23.x, v[3] - f23.y);
+          if constexpr (GQP == 4) {
+            const bool lo = gid >= 4;
+            bf[0][2 * jj + e][0] = *reinterpret_cast<const uint32_t*>(lo ? &l01 : &h01);
+            bf[0][2 * jj + e][1] = *reinterpret_cast<const uint32_t*>(lo ? &l23 : &h23);
+          } else {
+            bf[0][2 * jj + e][0] = *reinterpret_cast<const uint32_t*>(&h01);
+            bf[0][2 * jj + e][1] = *reinterpret_cast<const uint32_t*>(&h23);
+            bf[NT - 1][2 * jj + e][0] = *reinterpret_cast<const uint32_t*>(&l01);
+            bf[NT - 1][2 * jj + e][1] = *reinterpret_cast<const uint32_t*>(&l23);
+          }
+        }
         float s0 = mt[2 * jj] * alg, s1 = mt[2 * jj + 1] * alg;
 #pragma unroll
         for (int i = 0; i < 4; i++) {
@@ -366,12 +392,15 @@ __global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
       for (int m = 0; m < 8; m++) {
         uint32_t a0 = pair_of<B>(vw, 2 * m), a1 = pair_of<B>(vw, 2 * m + 1);
         uint32_t a2 = pair_of<B>(vw, 16 + 2 * m), a3 = pair_of<B>(vw, 17 + 2 * m);
-        float t4[4] = {0.f, 0.f, 0.f, 0.f};
-        mma16816(t4, a0, a1, a2, a3, bf[m >> 1][0], bf[m >> 1][1]);
-        accv[m][0] = fmaf(accv[m][0], al0, t4[0]);
-        accv[m][1] = fmaf(accv[m][1], al1, t4[1]);
-        accv[m][2] = fmaf(accv[m][2], al0, t4[2]);
-        accv[m][3] = fmaf(accv[m][3], al1, t4[3]);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++) {
+          float t4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma16816(t4, a0, a1, a2, a3, bf[nt][m >> 1][0], bf[nt][m >> 1][1]);
+          accv[nt][m][0] = fmaf(accv[nt][m][0], ac0, t4[0]);
+          accv[nt][m][1] = fmaf(accv[nt][m][1], ac1, t4[1]);
+          accv[nt][m][2] = fmaf(accv[nt][m][2], ac0, t4[2]);
+          accv[nt][m][3] = fmaf(accv[nt][m][3], ac1, t4[3]);
+        }
       }
     }
     __syncwarp();
@@ -396,7 +425,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
       v += __shfl_xor_sync(0xffffffffu, v, 2);
       mt[j] = v;  // head gid
     }
-    float m0[4], m1[4];  // m-terms of heads 2tig, 2tig+1
+    float m0[4], m1[4];  // m-terms of heads 2tig, 2tig+1 (held by the hi lanes gid = head)
 #pragma unroll
     for (int j = 0; j < 4; j++) {
       m0[j] = __shfl_sync(0xffffffffu, mt[j], 8 * tig);
@@ -404,10 +433,21 @@ __global__ void __launch_bounds__(kWarps * 32, 4) kv_base_kernel(BaseArgs a) {
     }
 #pragma unroll
     for (int m = 0; m < 8; m++) {
-      wrec[h0 * kRec + 16 * m + gid] = accv[m][0] + m0[m >> 1];
-      wrec[h1 * kRec + 16 * m + gid] = accv[m][1] + m1[m >> 1];
-      wrec[h0 * kRec + 16 * m + gid + 8] = accv[m][2] + m0[m >> 1];
-      wrec[h1 * kRec + 16 * m + gid + 8] = accv[m][3] + m1[m >> 1];
+      float o[4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        if constexpr (GQP == 4) {
+          o[i] = accv[0][m][i] + __shfl_xor_sync(0xffffffffu, accv[0][m][i], 2);  // hi + lo
+        } else {
+          o[i] = accv[0][m][i] + accv[NT - 1][m][i];
+        }
+      }
+      if (GQP == 8 || tig < 2) {
+        wrec[h0 * kRec + 16 * m + gid] = o[0] + m0[m >> 1];
+        wrec[h1 * kRec + 16 * m + gid] = o[1] + m1[m >> 1];
+        wrec[h0 * kRec + 16 * m + gid + 8] = o[2] + m0[m >> 1];
+        wrec[h1 * kRec + 16 * m + gid + 8] = o[3] + m1[m >> 1];
+      }
     }
   }
   if (gid == 0) {
@@ -937,3 +977,4 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
   return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
                               (float*)(w + P.off_corr), out, s);
 }
+

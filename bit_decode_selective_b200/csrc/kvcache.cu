@@ -5,9 +5,9 @@
 // nested-quantization paragraph: the same nesting as for weights is applied
 // to the KV cache, per token in groups of 32 head-dim elements.
 //
-// One thread per (batch, head, token).  A key token's words belong to that
+// One warp per (batch, head, token).  A key token's words belong to that
 // token alone; in a value tile each token owns whole 16-bit halves of the
-// words it touches, so tokens packed by different threads never share a store.
+// words it touches, so tokens packed by different warps never share a store.
 #include "common.cuh"
 #include "kvlayout.cuh"
 #include "quant.cuh"
@@ -15,86 +15,94 @@
 namespace sf {
 namespace {
 
-// Value halves of one token: chunk lane l = 4g + c (c from the token) owns, per
-// w-bit stream, w halves: word l*2w + h*w + k, half `second` (h, c, second from
-// the token; k = (2m+e) / (16/w)).
-template <int W>
-struct ValueHalves {
-  uint16_t v[8][W];
-  __device__ void clear() {
-    for (int g = 0; g < 8; g++)
-      for (int k = 0; k < W; k++) v[g][k] = 0;
-  }
-  __device__ void put(int d, uint32_t code) {
-    int m = d >> 4, within = d & 15, e = within >> 3, g = within & 7;
-    constexpr int per = 16 / W;
-    int k = (2 * m + e) / per, slot = (2 * m + e) % per;
-    v[g][k] |= (uint16_t)(code << (W * slot));
-  }
-  __device__ void store(uint16_t* tile_halves, int tt) {
-    int h = tt >> 3, c = (tt & 7) >> 1, second = tt & 1;
-    for (int g = 0; g < 8; g++)
-      for (int k = 0; k < W; k++) {
-        int word = (4 * g + c) * 2 * W + h * W + k;
-        tile_halves[word * 2 + second] = v[g][k];
-      }
-  }
-};
+constexpr int kPackWarps = 4;  // tokens per CTA of the pack kernel
 
+// Min and max of the 32 elements of a group held by 8 lanes (4 each), with
+// the first occurrence winning among equal values (so -0 and +0 keep the
+// order-dependent choice of a sequential scan).
+__device__ __forceinline__ void group_minmax(const double (&v)[4], int d0, double& lo, double& hi) {
+  lo = v[0], hi = v[0];
+  int ilo = d0, ihi = d0;
+#pragma unroll
+  for (int i = 1; i < 4; i++) {
+    if (v[i] < lo) lo = v[i], ilo = d0 + i;
+    if (v[i] > hi) hi = v[i], ihi = d0 + i;
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const double olo = __shfl_xor_sync(0xffffffffu, lo, o), ohi = __shfl_xor_sync(0xffffffffu, hi, o);
+    const int oilo = __shfl_xor_sync(0xffffffffu, ilo, o), oihi = __shfl_xor_sync(0xffffffffu, ihi, o);
+    if (olo < lo || (olo == lo && oilo < ilo)) lo = olo, ilo = oilo;
+    if (ohi > hi || (ohi == hi && oihi < ihi)) hi = ohi, ihi = oihi;
+  }
+}
+
+// One warp per (batch, head, token); lane l quantises head-dim elements
+// 4l .. 4l+3 (group l / 8).  The token's code words (keys) or 16-bit word
+// halves (values) are assembled in shared memory and stored by the first
+// lanes; a token owns all of them, so tokens never share a store.
 template <int B, int R>
-__global__ void pack_kv_kernel(const uint16_t* __restrict__ x, int BH, int nt, int t_max, int t0,
-                               int is_value, uint32_t* __restrict__ codes,
-                               uint32_t* __restrict__ refine, uint16_t* __restrict__ sz) {
-  long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long)BH * nt) return;
+__global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(
+    const uint16_t* __restrict__ x, int BH, int nt, int t_max, int t0, int is_value,
+    uint32_t* __restrict__ codes, uint32_t* __restrict__ refine, uint16_t* __restrict__ sz) {
+  // keys: 4B code words + 4R refinement words; values: 8B + 8R halves
+  __shared__ uint32_t acc[kPackWarps][8 * (B + R)];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long idx = (long)blockIdx.x * kPackWarps + warp;
+  if (idx >= (long)BH * nt) return;  // whole warps only
   const int t = (int)(idx % nt);
   const long bh = idx / nt;
-  const uint16_t* src = x + (bh * nt + t) * kHeadDim;
   const long slot = bh * t_max + t0 + t;
-  const int qmax = (1 << (B + R)) - 1;
-  uint32_t kw[4 * B] = {}, kr[4 * R] = {};
-  ValueHalves<B> vb;
-  ValueHalves<R> vr;
-  vb.clear();
-  vr.clear();
-  for (int j = 0; j < kHeadDim / 32; j++) {
-    double lo = h2d(src[j * 32]), hi = lo;
-    for (int c = 1; c < 32; c++) {
-      double v = h2d(src[j * 32 + c]);
-      if (v < lo) lo = v;
-      if (v > hi) hi = v;
-    }
-    Grid16 g = group_grid(lo, hi, B);
+  uint32_t* a = acc[warp];
+  for (int i = lane; i < 8 * (B + R); i += 32) a[i] = 0;
+  const int d0 = 4 * lane;
+  const uint2 raw = *reinterpret_cast<const uint2*>(x + (bh * nt + t) * kHeadDim + d0);
+  double v[4] = {h2d((uint16_t)(raw.x & 0xffff)), h2d((uint16_t)(raw.x >> 16)),
+                 h2d((uint16_t)(raw.y & 0xffff)), h2d((uint16_t)(raw.y >> 16))};
+  double lo, hi;
+  group_minmax(v, d0, lo, hi);
+  const Grid16 g = group_grid(lo, hi, B);
+  const int j = lane >> 3;
+  if ((lane & 7) == 0) {
     sz[(slot * 4 + j) * 2 + 0] = g.s16;
     sz[(slot * 4 + j) * 2 + 1] = g.m16;
-    for (int c = 0; c < 32; c++) {
-      int d = j * 32 + c;
-      int Q = nested_code(h2d(src[d]), g, R, qmax);
-      uint32_t q = (uint32_t)(Q >> R), rho = (uint32_t)(Q & ((1 << R) - 1));
-      if (!is_value) {
-        int word, bit;
-        key_pos(d, B, word, bit);
-        kw[word] |= q << bit;
-        key_pos(d, R, word, bit);
-        kr[word] |= rho << bit;
-      } else {
-        vb.put(d, q);
-        vr.put(d, rho);
-      }
+  }
+  __syncwarp();
+  const int qmax = (1 << (B + R)) - 1;
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const int d = d0 + i;
+    const int Q = nested_code(v[i], g, R, qmax);
+    const uint32_t q = (uint32_t)(Q >> R), rho = (uint32_t)(Q & ((1 << R) - 1));
+    if (!is_value) {
+      int word, bit;
+      key_pos(d, B, word, bit);
+      atomicOr(&a[word], q << bit);
+      key_pos(d, R, word, bit);
+      atomicOr(&a[4 * B + word], rho << bit);
+    } else {
+      // half (gg, k) of the token's value words, slot `sl` of 16/w codes
+      const int m = d >> 4, within = d & 15, e = within >> 3, gg = within & 7;
+      atomicOr(&a[gg * B + (2 * m + e) / (16 / B)], q << (B * ((2 * m + e) % (16 / B))));
+      atomicOr(&a[8 * B + gg * R + (2 * m + e) / (16 / R)], rho << (R * ((2 * m + e) % (16 / R))));
     }
   }
+  __syncwarp();
   if (!is_value) {
-    uint32_t* kd = codes + slot * 4 * B;
-#pragma unroll
-    for (int i = 0; i < 4 * B; i++) kd[i] = kw[i];
-    uint32_t* rd = refine + slot * 4 * R;
-#pragma unroll
-    for (int i = 0; i < 4 * R; i++) rd[i] = kr[i];
+    if (lane < 4 * B) codes[slot * 4 * B + lane] = a[lane];
+    else if (lane < 4 * (B + R)) refine[slot * 4 * R + lane - 4 * B] = a[lane];
   } else {
     const long tile = bh * (t_max / 16) + (t0 + t) / 16;
     const int tt = (t0 + t) & 15;
-    vb.store(reinterpret_cast<uint16_t*>(codes + tile * 64 * B), tt);
-    vr.store(reinterpret_cast<uint16_t*>(refine + tile * 64 * R), tt);
+    const int h = tt >> 3, c = (tt & 7) >> 1, second = tt & 1;
+    for (int i = lane; i < 8 * (B + R); i += 32) {
+      const bool base = i < 8 * B;
+      const int W = base ? B : R, ii = base ? i : i - 8 * B;
+      const int gg = ii / W, k = ii % W;
+      const int word = (4 * gg + c) * 2 * W + h * W + k;
+      uint16_t* halves = reinterpret_cast<uint16_t*>((base ? codes + tile * 64 * B : refine + tile * 64 * R));
+      halves[word * 2 + second] = (uint16_t)a[i];
+    }
   }
 }
 
@@ -131,9 +139,8 @@ __global__ void unpack_kv_kernel(const uint32_t* __restrict__ codes,
 template <int B, int R>
 sf_status launch_pack(const uint16_t* x, int BH, int nt, int t_max, int t0, int is_value,
                       void* codes, void* refine, uint16_t* sz, cudaStream_t s) {
-  long total = (long)BH * nt;
-  int threads = 128;
-  pack_kv_kernel<B, R><<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(
+  const long total = (long)BH * nt;
+  pack_kv_kernel<B, R><<<(unsigned)((total + kPackWarps - 1) / kPackWarps), kPackWarps * 32, 0, s>>>(
       x, BH, nt, t_max, t0, is_value, (uint32_t*)codes, (uint32_t*)refine, sz);
   SF_LAUNCHED();
   return SF_OK;

@@ -108,6 +108,11 @@ class Decoder:
                               for _ in range(2)] for n in PROJ}
         else:
             self.slots = None
+        # prepared activations of the GEMV in flight (sized for the widest input)
+        kmax = max(kk for _, _, kk in cfg.shapes())
+        wq = abi.sf_wq(128, kmax, cfg.w_bits, cfg.w_refine, cfg.group, None, None, None)
+        self.gemv_ws = torch.empty(max(abi.sf_gemv_workspace_bytes(ctypes.byref(wq), B, cfg.chunk, cfg.kch), 16),
+                                   dtype=torch.uint8, device=dev)
         self.side = torch.cuda.Stream(device=dev)
         self.ev_sel = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
         self.ev_stage = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
@@ -182,11 +187,12 @@ class Decoder:
         qw = self.layers[layer][name]
         if cfg.kch == 0 or base_only:
             check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, 0, None, None, None,
-                                      _p(y), None, 0, _s(main)), "sf_gemv_refined")
+                                      _p(y), _p(self.gemv_ws), self.gemv_ws.numel(), _s(main)), "sf_gemv_refined")
             return
         rows = self._ready(name, slot, main)
         check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
-                                  _p(self.sel[name][slot]), None, _p(rows), _p(y), None, 0, _s(main)),
+                                  _p(self.sel[name][slot]), None, _p(rows), _p(y), _p(self.gemv_ws),
+                                  self.gemv_ws.numel(), _s(main)),
               "sf_gemv_refined")
 
     def _prepare(self, layer, name, x, main):

@@ -58,7 +58,7 @@ class QuantWeights:
         return qb, rho
 
     def gemv(self, x: torch.Tensor, chunk: int = 1024, kch: int = 32, sel_in=None,
-             refine_rows=None, y=None, sel_out=None, stream=None):
+             refine_rows=None, y=None, sel_out=None, ws=None, stream=None):
         """y = W~ x (sf_gemv_refined).  Returns (y [batch][n] fp32, selection)."""
         x = _f16(x if x.dim() == 2 else x.view(1, -1))
         batch = x.shape[0]
@@ -66,8 +66,11 @@ class QuantWeights:
             y = torch.empty((batch, self.n), dtype=torch.float32, device=x.device)
         if kch > 0 and sel_in is None and sel_out is None:
             sel_out = torch.empty((batch, self.k // chunk, kch), dtype=torch.int32, device=x.device)
+        if ws is None:
+            need = abi.sf_gemv_workspace_bytes(ctypes.byref(self.desc), batch, chunk, kch)
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
         check(abi.sf_gemv_refined(ctypes.byref(self.desc), _p(x), batch, chunk, kch, _p(sel_in),
-                                  _p(sel_out), _p(refine_rows), _p(y), None, 0, _stream(stream)),
+                                  _p(sel_out), _p(refine_rows), _p(y), _p(ws), ws.numel(), _stream(stream)),
               "sf_gemv_refined")
         return y, (sel_in if sel_in is not None else sel_out)
 
