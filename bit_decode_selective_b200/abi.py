@@ -13,6 +13,8 @@ from ctypes import POINTER, c_char_p, c_int, c_int32, c_size_t, c_void_p
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libsf.so")
 
+SF_KV_STATIC_WS_BYTES = 32 << 20  # include/sf.h
+
 SF_OK, SF_ERR_INVALID_ARG, SF_ERR_UNSUPPORTED, SF_ERR_CUDA, SF_ERR_TIMEOUT, SF_ERR_WORKSPACE = range(6)
 
 
@@ -59,6 +61,8 @@ _SIGNATURES = {
     "sf_kv_attend_selective": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_kv_attend_selective_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
+    "sf_kv_attend_selective_static": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                       c_void_p, c_void_p], c_int),
     "sf_rmsnorm_residual": ([c_void_p, c_void_p, c_void_p, c_int, c_int, ctypes.c_float, c_void_p,
                              c_void_p], c_int),
     "sf_rope_split": ([c_void_p, c_int, c_int, c_int, c_int, c_int, ctypes.c_float, c_void_p, c_void_p,
@@ -129,6 +133,7 @@ sf_kv_attn_refined = _call("sf_kv_attn_refined")
 sf_kv_attn_workspace_bytes = _call("sf_kv_attn_workspace_bytes")
 sf_kv_attend_selective = _call("sf_kv_attend_selective")
 sf_kv_attend_selective_workspace_bytes = _call("sf_kv_attend_selective_workspace_bytes")
+sf_kv_attend_selective_static = _call("sf_kv_attend_selective_static")
 sf_rmsnorm_residual = _call("sf_rmsnorm_residual")
 sf_rope_split = _call("sf_rope_split")
 sf_silu_mul = _call("sf_silu_mul")

@@ -33,6 +33,7 @@
 // The result equals softmax(q.k~) v~ with refined k~, v~ on the selected
 // tokens, up to fp32 rounding.
 #include <cfloat>
+#include <mutex>
 
 #include "common.cuh"
 #include "kvlayout.cuh"
@@ -978,3 +979,73 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
                               (float*)(w + P.off_corr), out, s);
 }
 
+// ---------------------------------------------------------------------------
+// sf_kv_attend_selective with library-owned scratch.
+//
+// Some callers cannot allocate device memory for the workspace.  A plain C
+// host program or an embedding runtime has no caching allocator to draw from,
+// so every call would need cudaMalloc + cudaFree, and cudaFree synchronises the
+// whole device.  A latency-critical decode loop must not stall on that
+// synchronisation.  For those callers the workspace is this file-scope device
+// array: it is part of the library's module image, so using it allocates
+// nothing at call time.  All calls on one device share it, so two such calls
+// that overlap on the GPU (different streams or threads with no ordering
+// between them) race on it.  None of the scratch needs to start at zero:
+// every kernel of the pass writes each scratch word it later reads.
+
+namespace sf {
+namespace {
+
+constexpr size_t kStaticWsBytes = (size_t)SF_KV_STATIC_WS_BYTES;
+constexpr int kStaticWsDevices = 64;
+
+__device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
+
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[kStaticWsDevices] = {};
+
+// Device address of g_static_ws on the current device, looked up once per
+// device (the first lookup loads the module on that device).
+sf_status static_ws(void** ptr) {
+  int dev = -1;
+  SF_CUDA(cudaGetDevice(&dev));
+  SF_UNSUPPORTED(dev >= 0 && dev < kStaticWsDevices, "device %d outside [0, %d)", dev,
+                 kStaticWsDevices);
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_ws);
+    if (e != cudaSuccess || !p) {
+      set_error("cudaGetSymbolAddress(static KV workspace) on device %d failed: %s", dev,
+                cudaGetErrorString(e));
+      return SF_ERR_CUDA;
+    }
+    g_static_ws_ptr[dev] = p;
+  }
+  *ptr = g_static_ws_ptr[dev];
+  return SF_OK;
+}
+
+}  // namespace
+}  // namespace sf
+
+extern "C" sf_status sf_kv_attend_selective_static(const sf_kv* kv, int t, const uint16_t* q,
+                                                   int h_q, int k_tok, int32_t* sel, float* logits,
+                                                   float* out, sf_stream_t stream) {
+  sf_status st = check_kv(kv);
+  if (st != SF_OK) return st;
+  st = check_q(kv, t, q, h_q);
+  if (st != SF_OK) return st;
+  SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
+  const size_t need = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0).total;
+  if (need > kStaticWsBytes) {
+    set_error("workspace of %zu bytes needed (batch=%d, h_q=%d, t=%d, k_tok=%d, logits %s) is above "
+              "the static scratch of %zu bytes; use sf_kv_attend_selective with a caller workspace",
+              need, kv->batch, h_q, t, k_tok, logits ? "given" : "in scratch", kStaticWsBytes);
+    return SF_ERR_WORKSPACE;
+  }
+  void* ws = nullptr;
+  st = static_ws(&ws);
+  if (st != SF_OK) return st;
+  return sf_kv_attend_selective(kv, t, q, h_q, k_tok, sel, logits, out, ws, kStaticWsBytes, stream);
+}

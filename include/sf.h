@@ -261,6 +261,32 @@ SF_API sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* 
 SF_API size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                                      int logits_given);
 
+/* Largest workspace sf_kv_attend_selective_static can serve (32 MiB). */
+#define SF_KV_STATIC_WS_BYTES (32u << 20)
+
+/* sf_kv_attend_selective with a library-owned workspace: the same kernels and
+ * results, but the scratch is a file-scope device array of
+ * SF_KV_STATIC_WS_BYTES inside the library instead of (ws, ws_bytes).  The
+ * pages have no counterpart of this entry point; it serves callers that cannot
+ * allocate device memory per call: a plain C program or an embedding runtime
+ * without a caching allocator would need cudaMalloc/cudaFree around every call,
+ * and cudaFree synchronises the device, which a latency-bound decode loop
+ * cannot afford.  This call allocates nothing.
+ *   - The first call on each device does set-up (looks up the array's device
+ *     address, which loads the library's module on that device); make it before
+ *     any stream capture.
+ *   - The workspace sf_kv_attend_selective_workspace_bytes(kv, t, h_q, k_tok,
+ *     logits != NULL) gives must not exceed SF_KV_STATIC_WS_BYTES; a larger
+ *     request returns SF_ERR_WORKSPACE (with a message) and enqueues nothing.
+ *     Passing logits lowers the need by batch*h_q*t*4 bytes.
+ *   - All calls on one device share the one array: calls that overlap on the
+ *     GPU (streams or threads with no ordering between them) race and give
+ *     wrong results.  Order them on one stream or with events.
+ * Arguments, layouts and the other errors as sf_kv_attend_selective. */
+SF_API sf_status sf_kv_attend_selective_static(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                               int k_tok, int32_t* sel, float* logits, float* out,
+                                               sf_stream_t stream);
+
 /* ======================================================================== */
 /* Refinement staging ([EXPL] "the map app also loads tiles": fetch lead)    */
 /* ======================================================================== */
