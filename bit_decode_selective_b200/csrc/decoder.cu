@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(1024) rmsnorm_residual_kernel(float* __restric
                                                                 const float* __restrict__ add1,
                                                                 int n, float eps,
                                                                 uint16_t* __restrict__ x) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float red[32];
   const long row = blockIdx.x;
   float* hr = h + row * n;
@@ -54,6 +56,8 @@ __global__ void __launch_bounds__(1024) rmsnorm_residual_kernel(float* __restric
 __global__ void rope_split_kernel(const float* __restrict__ qkv, int h_q, int h_kv, int d, int pos,
                                   double theta, uint16_t* __restrict__ q, uint16_t* __restrict__ k,
                                   uint16_t* __restrict__ v) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.y;
   const int head = blockIdx.x;  // 0..h_q+2*h_kv-1
   const int half = d / 2;
@@ -82,6 +86,8 @@ __global__ void rope_split_kernel(const float* __restrict__ qkv, int h_q, int h_
 
 // out[b][i] = fp16(silu(gu[b][i]) * gu[b][inter + i])
 __global__ void silu_mul_kernel(const float* __restrict__ gu, int inter, uint16_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const long b = blockIdx.y;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < inter; i += gridDim.x * blockDim.x) {
     float g = gu[b * 2 * inter + i], u = gu[b * 2 * inter + inter + i];
@@ -91,11 +97,15 @@ __global__ void silu_mul_kernel(const float* __restrict__ gu, int inter, uint16_
 }
 
 __global__ void widen_f16_kernel(const uint16_t* __restrict__ x, long n, float* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
     y[i] = h2f(x[i]);
 }
 
 __global__ void cast_f16_kernel(const float* __restrict__ x, long n, uint16_t* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
     y[i] = __half_as_ushort(__float2half_rn(x[i]));
 }
@@ -107,6 +117,8 @@ template <int BATCH>
 __global__ void __launch_bounds__(256) gemv_f16_kernel(const uint16_t* __restrict__ w,
                                                        const uint16_t* __restrict__ x, int n,
                                                        int k, float* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float xs[];  // BATCH * k
   for (int i = threadIdx.x; i < BATCH * k; i += blockDim.x) xs[i] = h2f(x[i]);
   __syncthreads();
@@ -145,8 +157,7 @@ sf_status launch_gemv_f16(const uint16_t* w, const uint16_t* x, int n, int k, fl
   size_t smem = (size_t)BATCH * k * 4;
   SF_CUDA(cudaFuncSetAttribute(gemv_f16_kernel<BATCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int blocks = 4 * num_sms();
-  gemv_f16_kernel<BATCH><<<blocks, 256, smem, s>>>(w, x, n, k, y);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(gemv_f16_kernel<BATCH>, dim3(blocks), dim3(256), smem, s, w, x, n, k, y));
   return SF_OK;
 }
 
@@ -160,8 +171,8 @@ extern "C" sf_status sf_rmsnorm_residual(float* h, const float* add0, const floa
   SF_REQUIRE(h && x && batch > 0 && n > 0, "bad rmsnorm arguments");
   SF_REQUIRE(aligned16(h) && aligned16(x) && (!add0 || aligned16(add0)) && (!add1 || aligned16(add1)),
              "rmsnorm pointers must be 16-byte aligned");
-  rmsnorm_residual_kernel<<<batch, 1024, 0, as_stream(stream)>>>(h, add0, add1, n, eps, x);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(rmsnorm_residual_kernel, dim3(batch), dim3(1024), 0, as_stream(stream), h, add0, add1, n,
+                     eps, x));
   return SF_OK;
 }
 
@@ -170,17 +181,16 @@ extern "C" sf_status sf_rope_split(const float* qkv, int batch, int h_q, int h_k
                                    sf_stream_t stream) {
   SF_REQUIRE(qkv && q && k && v && batch > 0 && h_q > 0 && h_kv > 0 && d > 0 && d % 2 == 0 && pos >= 0,
              "bad rope arguments");
-  rope_split_kernel<<<dim3(h_q + 2 * h_kv, batch), 64, 0, as_stream(stream)>>>(qkv, h_q, h_kv, d, pos,
-                                                                           (double)theta, q, k, v);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(rope_split_kernel, dim3(h_q + 2 * h_kv, batch), dim3(64), 0, as_stream(stream), qkv, h_q,
+                     h_kv, d, pos, (double)theta, q, k, v));
   return SF_OK;
 }
 
 extern "C" sf_status sf_silu_mul(const float* gu, int batch, int inter, uint16_t* out,
                                  sf_stream_t stream) {
   SF_REQUIRE(gu && out && batch > 0 && inter > 0, "bad silu_mul arguments");
-  silu_mul_kernel<<<dim3((inter + 255) / 256, batch), 256, 0, as_stream(stream)>>>(gu, inter, out);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(silu_mul_kernel, dim3((inter + 255) / 256, batch), dim3(256), 0, as_stream(stream), gu, inter,
+                     out));
   return SF_OK;
 }
 
@@ -189,8 +199,7 @@ extern "C" sf_status sf_cast_f16(const float* x, size_t n, uint16_t* y, sf_strea
   if (n == 0) return SF_OK;
   long blocks = (long)((n + 255) / 256);
   if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
-  cast_f16_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(x, (long)n, y);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(cast_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, as_stream(stream), x, (long)n, y));
   return SF_OK;
 }
 
@@ -199,8 +208,7 @@ extern "C" sf_status sf_widen_f16(const uint16_t* x, size_t n, float* y, sf_stre
   if (n == 0) return SF_OK;
   long blocks = (long)((n + 255) / 256);
   if (blocks > 8 * num_sms()) blocks = 8 * num_sms();
-  widen_f16_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(x, (long)n, y);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(widen_f16_kernel, dim3((unsigned)blocks), dim3(256), 0, as_stream(stream), x, (long)n, y));
   return SF_OK;
 }
 

@@ -16,11 +16,11 @@
 //   y_i = sum_groups [ s_ig * sum_{c in g} x_c q_ic + m_ig * sum_{c in g} x_c ]
 //       + sum_{c selected} x_c * s_i,g(c) * (rho_ic + 1/2 - 2^(r-1)) / 2^r
 //
-// Activation prologue (gemv_prep_kernel, once per call): every 64-channel
-// lane group of x becomes exact fixed point x = x_fix * 2^e with
+// Activation prologue (in every CTA, after griddepcontrol.wait): each
+// 64-channel lane group of x becomes exact fixed point x = x_fix * 2^e with
 // |x_fix| < 2^21, split into three byte planes laid out in the order of the
-// code byte vectors below, plus the group's sums.
-//
+// code byte vectors below, plus the group's sums, in shared memory.
+
 // Base pass (HBM-bound: every resident code is read once).  One CTA of 16
 // warps per SM owns a contiguous, 4-aligned range of rows.  Its work is a list
 // of (2,048-channel segment, 4-row step) tasks split evenly over the warps; a
@@ -33,10 +33,10 @@
 // lane's partial dot product is exact.  Partial sums of four rows are reduced
 // across the warp with a transposed butterfly.
 //
-// Correction pass: the prologue writes a table of the selected channels
-// (x_c, group, refinement row); the GEMV copies it and the refinement words
-// covering its rows into shared memory while the base pass streams (the base
-// pass also keeps the rows' (s, m) words), then each lane owns 1, 2 or 4 rows
+// Correction pass: a table of the selected channels (x_c, group, refinement
+// row) and the refinement words covering the CTA's rows are copied into shared
+// memory while the base pass streams (the base pass also keeps the rows'
+// (s, m) words), then each lane owns 1, 2 or 4 rows
 // and every warp walks a range of the table, summing x_c (rho_ic + 1/2 -
 // 2^(r-1)) / 2^r over each run of channels that share a scale group and
 // scaling each run once.
@@ -58,7 +58,6 @@ constexpr int kXShift = 8 * kXP - 4;        // x_fix = x * 2^-(ilogb(max|x|) - k
 constexpr int kXR = 16 * kXP;               // plane words per lane group
 constexpr int kXWords = kXR + 4;            // then sum0, sum1, 2^e, sum
 constexpr int kRowUnit = 4;                 // CTA row ranges start at multiples of 4
-constexpr int kPrepWarps = 8;
 constexpr size_t kSmemLimit = 227 * 1024;
 
 struct GemvParams {
@@ -66,8 +65,6 @@ struct GemvParams {
   const uint32_t* refine;  // channel-major rows, or staged rows [batch][n_sel]
   const uint16_t* sz;
   const uint16_t* x;       // [batch][K] fp16
-  const uint32_t* xp;      // [batch][K/64][kXWords] prepared activations (mode 0)
-  const uint4* jdg;        // [batch][n_sel] correction table written by the prologue (mode 0)
   const int32_t* sel;      // [batch][n_sel]
   float* y;
   int N, K, G, gshift, r, batch, n_sel, segs;
@@ -75,6 +72,7 @@ struct GemvParams {
   int staged;            // refine holds [batch][n_sel] staged rows
   int mode;              // 0: base + correction, 1: correction only, added into y
   int rows_max;          // most rows a CTA owns
+  int plane_words;       // shared words of the activation planes (mode 0)
   int area_words;        // shared words of the copy rings (reused by the slow correction path)
   int fast;              // correction tables in their own shared region, filled before the base pass
   int w_span;            // stride of the refinement-word table (words a CTA's rows can span)
@@ -259,24 +257,14 @@ __device__ __forceinline__ uint4 make_jd(const GemvParams& p, int b, int j) {
 }
 
 // ---------------------------------------------------------------------------
-// activation prologue: one warp per (batch row, 64-channel lane group), then
-// (blocks past the plane blocks) the correction table of every batch row
+// activation prologue: every CTA turns batch row b of x into the fixed-point
+// byte planes of all K/64 lane groups in shared memory, one warp per group
 
 template <int BITS>
-__global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(GemvParams p, uint32_t* __restrict__ xp,
-                                                                   uint4* __restrict__ jdg, int plane_blocks) {
-  pdl_trigger();  // the GEMV may start streaming codes now
+__device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ xs) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ngrp = p.K / kLaneCh;
-  const int b = blockIdx.y;
-  if ((int)blockIdx.x >= plane_blocks) {
-    pdl_wait();  // the selection launched before this kernel (if any) is complete
-    const int j = (blockIdx.x - plane_blocks) * blockDim.x + threadIdx.x;
-    if (j < p.n_sel) jdg[(size_t)b * p.n_sel + j] = make_jd(p, b, j);
-    return;
-  }
-  const int grp = blockIdx.x * kPrepWarps + warp;
-  if (grp < ngrp) {
+  for (int grp = warp; grp < ngrp; grp += kWarps) {
     const float2 xv = __half22float2(
         reinterpret_cast<const __half2*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh)[lane]);
     float mx = fmaxf(fabsf(xv.x), fabsf(xv.y));
@@ -284,7 +272,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(GemvParams p
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     const int e = mx > 0.f ? ilogbf(mx) - kXShift : 0;
     const int xf0 = __float2int_rn(ldexpf(xv.x, -e)), xf1 = __float2int_rn(ldexpf(xv.y, -e));
-    // lane v < 16 assembles the three plane words of code byte vector v
+    // lane v < 16 assembles the plane words of code byte vector v
     const int v = lane & 15;
     uint32_t pl[kXP];
 #pragma unroll
@@ -297,23 +285,22 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(GemvParams p
 #pragma unroll
       for (int q = 0; q < kXP; q++) pl[q] |= ((f >> (8 * q)) & 0xffu) << (8 * L);
     }
-    uint32_t* dst = xp + ((size_t)b * ngrp + grp) * kXWords;
+    uint32_t* dst = xs + grp * kXWords;
     if (lane < 16) {
 #pragma unroll
       for (int q = 0; q < kXP; q++) dst[kXP * v + q] = pl[q];
     }
-    float s = xv.x + xv.y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
+    float sm = xv.x + xv.y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float s1 = __shfl_sync(0xffffffffu, s, 16);
+    for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+    const float s1 = __shfl_sync(0xffffffffu, sm, 16);
     if (lane == 0) {
-      reinterpret_cast<float*>(dst)[kXR + 0] = s;
+      reinterpret_cast<float*>(dst)[kXR + 0] = sm;
       reinterpret_cast<float*>(dst)[kXR + 1] = s1;
       reinterpret_cast<float*>(dst)[kXR + 2] = ldexpf(1.0f, e);
-      reinterpret_cast<float*>(dst)[kXR + 3] = s + s1;
+      reinterpret_cast<float*>(dst)[kXR + 3] = sm + s1;
     }
   }
-  pdl_wait();  // the grid completes only after the selection launched before it
 }
 
 // ---------------------------------------------------------------------------
@@ -324,7 +311,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(GemvParams p
 __device__ void corr_fill(const GemvParams& p, int b, int j0, int jn, int w_lo, int nwr, uint4* jd,
                           uint32_t* wt) {
   for (int i = threadIdx.x; i < jn; i += kThreads) {
-    const uint4 d = p.mode == 0 ? __ldg(p.jdg + (size_t)b * p.n_sel + j0 + i) : make_jd(p, b, j0 + i);
+    const uint4 d = make_jd(p, b, j0 + i);
     jd[i] = d;
     for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + d.w + w_lo + k);
   }
@@ -419,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   using R = Ring<BITS, ZW>;
   constexpr int U = Lane<BITS>::U, CW = Lane<BITS>::CW;
   extern __shared__ __align__(16) uint32_t smem[];
+  pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this grid
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int units = p.N / kRowUnit;
   const int n0 = (int)((long)blockIdx.x * units / gridDim.x) * kRowUnit;
@@ -427,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   const int ngrp = p.K / kLaneCh, gpr = p.K >> p.gshift;
   // shared memory: partial sums [rows][segs] | rings | (fast) table, words, scales
   float* part = reinterpret_cast<float*>(smem);
-  uint32_t* area = smem + ((p.rows_max * p.segs + 3) & ~3);
+  uint32_t* xs = smem + ((p.rows_max * p.segs + 3) & ~3);  // activation planes [K/64][kXWords]
+  uint32_t* area = xs + p.plane_words;
   uint4* jd_fast = reinterpret_cast<uint4*>(area + p.area_words);
   uint32_t* wt_fast = reinterpret_cast<uint32_t*>(jd_fast + p.n_sel);
   uint32_t* szt = wt_fast + (((size_t)p.n_sel * p.w_span + 3) & ~(size_t)3);
@@ -442,7 +431,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
     if (p.mode == 0) {
       // ---- base pass of batch row b: every (row, segment) partial is written once
       uint32_t* ring = area + warp * PD * R::words;
-      const uint32_t* xpb = p.xp + (size_t)b * ngrp * kXWords;
       int iseg = ta / steps, ist = ta - iseg * steps, islot = 0, left = tb - ta;
       auto issue = [&]() {
         if (left > 0) {
@@ -464,8 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
       };
 #pragma unroll
       for (int i = 0; i < PD - 1; i++) issue();
-      if (b == 0) pdl_wait();  // prepared activations, selection and staged rows are complete
+      if (b == 0) pdl_wait();  // x, the selection and the staged rows are complete
+      prep_planes<BITS>(p, b, xs);
       if (p.fast && p.n_sel > 0) corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
+      __syncthreads();  // planes complete
       uint32_t xr[kXR];
       float xsum0 = 0.f, xsum1 = 0.f, xscale = 0.f;
       int cseg = ta / steps, cst = ta - cseg * steps, cslot = 0, cur = -1;
@@ -476,13 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
         if (cseg != cur) {
           cur = cseg;
           if (la) {
-            const uint4* src = reinterpret_cast<const uint4*>(xpb + (size_t)lg * kXWords);
+            const uint4* src = reinterpret_cast<const uint4*>(xs + lg * kXWords);
 #pragma unroll
             for (int k = 0; k < kXR / 4; k++) {
-              const uint4 q = __ldg(src + k);
+              const uint4 q = src[k];
               xr[4 * k + 0] = q.x, xr[4 * k + 1] = q.y, xr[4 * k + 2] = q.z, xr[4 * k + 3] = q.w;
             }
-            const float4 f = __ldg(reinterpret_cast<const float4*>(src + kXR / 4));
+            const float4 f = reinterpret_cast<const float4*>(src)[kXR / 4];
             xsum0 = ZW == 2 ? f.x : f.w, xsum1 = f.y, xscale = f.z;
           } else {
 #pragma unroll
@@ -535,6 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
       cp_async_wait<0>();
     } else {
       for (int i = threadIdx.x; i < rows * p.segs; i += kThreads) part[i] = 0.f;
+      if (b == 0) pdl_wait();  // x, the selection, the staged rows and y are complete
       if (p.fast) {
         // the CTA's (s, m) words are one contiguous block of sz
         const uint32_t* zsrc = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)n0 * gpr;
@@ -579,20 +570,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
 // ---------------------------------------------------------------------------
 // host side
 
-size_t prep_bytes(const sf_wq* w, int batch, int n_sel) {
-  return (size_t)batch * (w->k / kLaneCh) * kXWords * 4 + (size_t)batch * n_sel * 16;
-}
-
 size_t slot_words(int bits, int zw) {
   if (bits == 2) return zw == 1 ? Ring<2, 1>::words : Ring<2, 2>::words;
   if (bits == 3) return zw == 1 ? Ring<3, 1>::words : Ring<3, 2>::words;
   return zw == 1 ? Ring<4, 1>::words : Ring<4, 2>::words;
 }
 
-// Ring depth: 4 stages (3 for b = 3, whose stages are larger).
 template <int BITS, int ZW>
-void* kernel_for() {
-  return (void*)gemv_kernel<BITS, ZW, BITS == 3 ? 3 : 4>;
+void* kernel_for(int pd) {
+  if (pd == 4) return (void*)gemv_kernel<BITS, ZW, 4>;
+  if (pd == 3) return (void*)gemv_kernel<BITS, ZW, 3>;
+  return (void*)gemv_kernel<BITS, ZW, 2>;
 }
 
 // Rows per lane in the correction: the fewest warp steps, counting ~6 + 3 RL
@@ -610,7 +598,7 @@ int pick_corr_rows(int rows) {
 
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                       const int32_t* sel_in, int32_t* sel_out, const void* refine_rows, float* y,
-                      void* ws, size_t ws_bytes, int mode, cudaStream_t s) {
+                      int mode, cudaStream_t s) {
   sf_status st = check_wq_public(w, false);
   if (st != SF_OK) return st;
   SF_REQUIRE(x && aligned16(x), "x must be a non-null 16-byte aligned device pointer");
@@ -633,14 +621,6 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   } else if (mode == 1) {
     return SF_OK;  // nothing to correct
   }
-  if (mode == 0) {
-    const size_t need = prep_bytes(w, batch, n_sel);
-    if (ws_bytes < need || !ws) {
-      set_error("workspace: need %zu bytes, got %zu", need, ws_bytes);
-      return SF_ERR_WORKSPACE;
-    }
-    SF_REQUIRE(aligned16(ws), "ws must be 16-byte aligned");
-  }
 
   GemvParams p = {};
   p.base = (const uint32_t*)w->base;
@@ -655,83 +635,72 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.segs = (w->k + kSegChannels - 1) / kSegChannels;
   p.refine_row_words = w->n * w->r / 32;
   p.staged = refine_rows != nullptr;
-  if (mode == 0) {
-    p.xp = (const uint32_t*)ws;
-    p.jdg = reinterpret_cast<const uint4*>((const char*)ws + (size_t)batch * (w->k / kLaneCh) * kXWords * 4);
-  }
 
   const int zw = w->group == 32 ? 2 : 1;
-  const int pd = w->b == 3 ? 3 : 4;
   int grid = num_sms();
   const int units = w->n / kRowUnit;
   if (grid > units) grid = units;
   p.rows_max = ((units + grid - 1) / grid) * kRowUnit;
   p.w_span = p.rows_max * w->r / 32 + 2;
   p.corr_rows = pick_corr_rows(p.rows_max);
+  p.plane_words = mode == 0 ? (w->k / kLaneCh) * kXWords : 0;
   const size_t gpr = (size_t)(w->k / w->group);
   const size_t part_words = ((size_t)p.rows_max * p.segs + 3) & ~(size_t)3;
-  size_t area = mode == 0 ? (size_t)kWarps * pd * slot_words(w->b, zw) : 0;
   const size_t table_words = (size_t)n_sel * 4 + (((size_t)n_sel * p.w_span + 3) & ~(size_t)3) +
                              (size_t)p.rows_max * gpr;
   const size_t limit_words = kSmemLimit / 4;
-  p.fast = n_sel > 0 && part_words + area + table_words <= limit_words;
-  if (!p.fast && n_sel > 0) {
-    // slow path: chunks of the table in the ring area (grown for the correction-only call)
-    const size_t min_area = (size_t)(4 + p.w_span) * 64;
-    if (area < min_area) area = min_area;
-    if (mode == 1) area = limit_words - part_words;
+  const size_t fixed = part_words + p.plane_words;
+  // ring depth: the deepest that leaves room for the correction tables, else
+  // the deepest that fits (the tables then go through the ring area in chunks)
+  int pd = 0;
+  size_t area = 0;
+  if (mode == 0) {
+    for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
+      const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
+      if (fixed + ring + (n_sel > 0 ? table_words : 0) <= limit_words) pd = d, area = ring, p.fast = n_sel > 0;
+    }
+    for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
+      const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
+      if (fixed + ring <= limit_words) pd = d, area = ring, p.fast = 0;
+    }
+    SF_UNSUPPORTED(pd > 0, "n=%d, k=%d does not fit in shared memory", w->n, w->k);
+  } else {
+    p.fast = fixed + 4 + table_words <= limit_words;
+    area = p.fast ? 4 : limit_words - fixed;
+    pd = 2;
   }
-  if (area < 4) area = 4;
-  const size_t smem = (part_words + area + (p.fast ? table_words : 0)) * 4;
+  if (!p.fast && n_sel > 0)
+    SF_UNSUPPORTED(area >= (size_t)(4 + p.w_span) * 16, "n=%d, k=%d: no room for the correction", w->n, w->k);
+  const size_t smem = (fixed + area + (p.fast ? table_words : 0)) * 4;
   SF_UNSUPPORTED(smem <= kSmemLimit, "n=%d, k=%d needs %zu bytes of shared memory", w->n, w->k, smem);
   p.area_words = (int)area;
 
-  // 1. the selection (when not given), 2. the activation prologue, 3. the GEMV
-  bool chained = false;
+  // the selection (when not given), then the GEMV, which waits for it (and for
+  // x) through programmatic dependent launch while its first code copies fly
   if (kch > 0 && !sel_in) {
     st = launch_select(x, batch, w->k, chunk, kch, sel_out, s);
     if (st != SF_OK) return st;
     p.sel = sel_out;
-    chained = true;
   } else {
     p.sel = sel_in;
   }
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  if (mode == 0) {
-    const int plane_blocks = (w->k / kLaneCh + kPrepWarps - 1) / kPrepWarps;
-    const int jd_blocks = (n_sel + kPrepWarps * 32 - 1) / (kPrepWarps * 32);
-    cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3(plane_blocks + jd_blocks, batch);
-    pc.blockDim = dim3(kPrepWarps * 32);
-    pc.stream = s;
-    attr[0].val.programmaticStreamSerializationAllowed = chained ? 1 : 0;
-    pc.attrs = attr;
-    pc.numAttrs = 1;
-    uint32_t* xp = (uint32_t*)ws;
-    uint4* jdg = const_cast<uint4*>(p.jdg);
-    if (w->b == 4)
-      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<4>, p, xp, jdg, plane_blocks));
-    else if (w->b == 3)
-      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<3>, p, xp, jdg, plane_blocks));
-    else
-      SF_CUDA(cudaLaunchKernelEx(&pc, gemv_prep_kernel<2>, p, xp, jdg, plane_blocks));
-  }
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  attr[0].val.programmaticStreamSerializationAllowed = mode == 0 ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   void* kern;
   if (w->b == 2)
-    kern = zw == 1 ? kernel_for<2, 1>() : kernel_for<2, 2>();
+    kern = zw == 1 ? kernel_for<2, 1>(pd) : kernel_for<2, 2>(pd);
   else if (w->b == 3)
-    kern = zw == 1 ? kernel_for<3, 1>() : kernel_for<3, 2>();
+    kern = zw == 1 ? kernel_for<3, 1>(pd) : kernel_for<3, 2>(pd);
   else
-    kern = zw == 1 ? kernel_for<4, 1>() : kernel_for<4, 2>();
+    kern = zw == 1 ? kernel_for<4, 1>(pd) : kernel_for<4, 2>(pd);
   SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit));
   void* args[] = {&p};
   SF_CUDA(cudaLaunchKernelExC(&cfg, kern, args));
@@ -744,23 +713,21 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
 using namespace sf;
 
 extern "C" size_t sf_gemv_workspace_bytes(const sf_wq* w, int batch, int chunk, int kch) {
-  if (!w || w->k <= 0 || batch <= 0) return 0;
-  const int n_sel = (kch > 0 && chunk > 0) ? (w->k / chunk) * kch : 0;
-  return prep_bytes(w, batch, n_sel);
+  (void)w, (void)batch, (void)chunk, (void)kch;
+  return 0;
 }
 
 extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk,
                                      int kch, const int32_t* sel_in, int32_t* sel_out,
                                      const void* refine_rows, float* y, void* ws, size_t ws_bytes,
                                      sf_stream_t stream) {
-  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, ws, ws_bytes, 0,
-                     as_stream(stream));
+  (void)ws, (void)ws_bytes;
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, 0, as_stream(stream));
 }
 
 extern "C" sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch, int chunk,
                                         int kch, const int32_t* sel, const void* refine_rows,
                                         float* y, sf_stream_t stream) {
   SF_REQUIRE(kch == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
-  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, nullptr, 0, 1,
-                     as_stream(stream));
+  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, 1, as_stream(stream));
 }

@@ -14,30 +14,29 @@
 //
 // Schedule (one pass over the resident cache, then work on the selected
 // tokens only):
-//   kv_base_kernel     per 16-token tile, logits of the group's query heads
-//                      from the base keys and the base attention (online
-//                      softmax, split-K partials) from the base values; the
-//                      logits are stored for scoring.  Codes are turned into
-//                      exact fp16 integers in registers and contracted on the
-//                      tensor cores (mma.sync m16n8k16, fp32 accumulation);
-//                      the per-token fp16 steps/offsets are applied in fp32.
-//   kv_stats_kernel    softmax max/sum of every query head from the partials;
-//   kv_local_kernel    per context span, score every token and keep the
-//                      span's k_tok best (a token in the global top-k is in
-//                      the top-k of its own span), in token order;
-//   kv_final_kernel    per KV head, the k_tok best of the candidates;
-//   kv_correct_kernel  for the selected tokens only: swap each token's base
-//                      contribution for its refined one (refined logit, refined
-//                      value), relative to the head's softmax max;
-//   kv_merge_kernel    log-sum-exp merge of the partials plus the correction.
+//   kv_base_kernel  per 16-token tile, logits of the group's query heads from
+//                   the base keys and the base attention (online softmax,
+//                   split-K partials) from the base values; the logits are
+//                   stored for scoring.  Codes are turned into exact fp16
+//                   integers in registers and contracted on the tensor cores
+//                   (mma.sync m16n8k16, fp32 accumulation); the per-token fp16
+//                   steps/offsets are applied in fp32.
+//   kv_post_kernel  one thread-block cluster per KV head: softmax statistics
+//                   from the partials, token scores, a cluster-wide radix
+//                   select of the top k_tok (histograms exchanged through
+//                   distributed shared memory), then the correction of the
+//                   selected tokens (each token's base contribution swapped
+//                   for its refined one, relative to the head's softmax
+//                   maximum) and the log-sum-exp merge of the partials.
 // The result equals softmax(q.k~) v~ with refined k~, v~ on the selected
 // tokens, up to fp32 rounding.
+#include <cooperative_groups.h>
+
 #include <cfloat>
 #include <mutex>
 
 #include "common.cuh"
 #include "kvlayout.cuh"
-#include "radix.cuh"
 
 namespace sf {
 namespace {
@@ -46,15 +45,16 @@ constexpr int kD = kHeadDim;
 constexpr int kRec = kD + 2;     // partial record: acc[kD], m, l
 constexpr int kWarps = 4;        // warps per base-pass CTA (independent splits)
 constexpr int kStages = 4;       // cp.async ring depth per warp
-constexpr int kMaxCand = 16384;  // candidates per KV head in the final select
-constexpr int kMaxSpan = 8192;   // tokens per local-select CTA
-constexpr int kCorrTok = 16;     // selected tokens per correction CTA
 
 // ---- small PTX helpers -------------------------------------------------------
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -153,6 +153,8 @@ __global__ void __launch_bounds__(kWarps * 32, GQP == 4 ? 4 : 2) kv_base_kernel(
   using St = Stage<B, PV>;
   using WS = WarpSmem<B, PV>;
   extern __shared__ __align__(16) uint8_t smem[];
+  pdl_trigger();  // the kernel after the base pass may be scheduled now; it waits for this grid
+  pdl_wait();     // q and the cache (including a token appended just before) are complete
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int g = blockIdx.y, bat = blockIdx.z;
@@ -477,250 +479,453 @@ __global__ void __launch_bounds__(kWarps * 32, GQP == 4 ? 4 : 2) kv_base_kernel(
   }
 }
 
-// Softmax max and sum of every query head: M = max_s m_s, Z = sum_s l_s e^(m_s - M).
-__global__ void kv_stats_kernel(const float* __restrict__ part, int nsplit, int rec,
-                                float2* __restrict__ stats) {
-  const long bh = blockIdx.x;
-  const float* p = part + bh * nsplit * rec;
-  const int mo = rec - 2;
-  __shared__ float sm[256];
-  float m = -INFINITY;
-  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) m = fmaxf(m, p[(long)i * rec + mo]);
-  sm[threadIdx.x] = m;
-  __syncthreads();
-  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) sm[threadIdx.x] = fmaxf(sm[threadIdx.x], sm[threadIdx.x + o]);
-    __syncthreads();
-  }
-  const float M = sm[0];
-  __syncthreads();
-  float s = 0.f;
-  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) {
-    float mi = p[(long)i * rec + mo];
-    if (mi > -INFINITY) s += p[(long)i * rec + mo + 1] * expf(mi - M);
-  }
-  sm[threadIdx.x] = s;
-  __syncthreads();
-  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) sm[threadIdx.x] += sm[threadIdx.x + o];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) stats[bh] = make_float2(M, sm[0]);
-}
-
 // ---------------------------------------------------------------------------
-// selection
+// after the base pass: one thread-block cluster per (batch, KV head)
+//
+// The cluster's CTAs split the context: each scores its tokens (sum over the
+// group's query heads of the softmax probability, from the stored base
+// logits) into shared memory.  The k_tok-th largest score is found by a radix
+// select over the score bits (non-negative floats order like their bits),
+// 9 bits per pass from bit 30: every CTA histograms its keys, stores the
+// histogram into every peer's shared memory (distributed shared memory) and,
+// after the cluster barrier, all CTAs take the same decision from their local
+// copies.  Equal scores rank the lower token first; the selected tokens are
+// written in ascending order and also handed, by position, to the CTA that
+// refines them.  Each CTA then copies its share of the selected tokens' codes
+// and scales into shared memory with cp.async in one go, refines them one warp
+// per token (swapping each token's base contribution for its refined one,
+// relative to the head's softmax maximum), sums an interleaved share of the
+// base partial records, and CTA h merges query head h.
 
-// Unique ranking key: score bits (positive floats order like their bits) above
-// the complement of the token index, so equal scores rank the lower token first.
-__device__ __forceinline__ uint64_t score_key(float score, int t) {
-  return ((uint64_t)__float_as_uint(score) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)t);
-}
-__device__ __forceinline__ int key_token(uint64_t key) {
-  return (int)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu));
-}
+constexpr int kPostThreads = 512;
+constexpr int kPostMaxTok = 16640;  // tokens per CTA scored in shared memory (cluster of 8)
+constexpr int kPostCl = 8;
+constexpr int kPostStage = 64;      // selected tokens staged in shared memory at a time
+constexpr int kPostMaxSel = 512;    // selected tokens per CTA (k_tok <= 4096)
+constexpr int kHistBins = 512;
 
-__global__ void __launch_bounds__(1024) kv_local_kernel(const float* __restrict__ logits,
-                                                        const float2* __restrict__ stats, int T,
-                                                        int span, int h_q, int h_kv, int k_tok,
-                                                        float* __restrict__ scores,
-                                                        uint64_t* __restrict__ cand) {
-  extern __shared__ uint64_t keys[];  // span entries
-  __shared__ RadixShared sh;
-  __shared__ float Ms[8], invZ[8];
-  const int gq = h_q / h_kv;
-  const int sp = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
-  const int t0 = sp * span, n = min(T, t0 + span) - t0;
-  if (threadIdx.x < gq) {
-    const float2 st = stats[(long)bat * h_q + g * gq + threadIdx.x];
-    Ms[threadIdx.x] = st.x, invZ[threadIdx.x] = 1.0f / st.y;
-  }
-  __syncthreads();
-  const float* lg = logits + ((long)bat * h_q + g * gq) * T + t0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    float s = 0.f;
-    for (int h = 0; h < gq; h++) s += expf(lg[(long)h * T + i] - Ms[h]) * invZ[h];
-    if (scores) scores[((long)bat * h_kv + g) * T + t0 + i] = s;
-    keys[i] = score_key(s, t0 + i);
-  }
-  __syncthreads();
-  const int kl = min(k_tok, n);
-  auto key_at = [&](int i) { return keys[i]; };
-  const uint64_t tau = block_kth_largest<64>(key_at, n, kl, sh);
-  uint64_t* out = cand + (((long)bat * h_kv + g) * gridDim.x + sp) * (long)min(k_tok, span);
-  block_compact(key_at, n, tau, sh, [&](int pos, int, uint64_t key) { out[pos] = key; });
-}
-
-__global__ void __launch_bounds__(1024) kv_final_kernel(const uint64_t* __restrict__ cand, int nspan,
-                                                        int span, int T, int h_kv, int k_tok,
-                                                        int32_t* __restrict__ sel) {
-  extern __shared__ uint64_t keys[];  // all candidates of this KV head
-  __shared__ RadixShared sh;
-  const int g = blockIdx.x, bat = blockIdx.y;
-  const int per = min(k_tok, span);
-  const uint64_t* src = cand + ((long)bat * h_kv + g) * nspan * (long)per;
-  // every span but the last holds `per` keys, so the candidates are one run
-  const int last = min(k_tok, T - (nspan - 1) * span);
-  const int n = (nspan - 1) * per + last;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = src[i];
-  __syncthreads();
-  auto key_at = [&](int i) { return keys[i]; };
-  const uint64_t tau = block_kth_largest<64>(key_at, n, k_tok, sh);
-  int32_t* out = sel + ((long)bat * h_kv + g) * k_tok;
-  block_compact(key_at, n, tau, sh, [&](int pos, int, uint64_t key) { out[pos] = key_token(key); });
-}
-
-// ---------------------------------------------------------------------------
-// correction on the selected tokens
-
-struct CorrArgs {
+struct PostArgs {
   const uint8_t *kb, *kr, *vb, *vr;
   const uint16_t *ksz, *vsz;
   int h_kv, t_max, b, r, T;
   const uint16_t* q;
   int h_q, gq;
-  const int32_t* sel;
-  int k_tok;
   const float* logits;  // base logits [batch][h_q][T]
-  const float2* stats;  // [batch][h_q] (max, sum)
-  float* corr;          // [batch][h_q][ncorr][kRec]: d-acc[kD], d-sum, unused
-  int ncorr;
+  const float* part;    // base partial records [batch][h_q][nrec][rec]
+  int nrec, rec;        // rec = kRec (with values) or 2 (scores only)
+  int k_tok;
+  int32_t* sel;         // [batch][h_kv][k_tok]: written when select, else read
+  int select;
+  float* scores;        // nullable [batch][h_kv][T]
+  float* out;           // nullable [batch][h_q][kD]
+  int chunk;            // tokens per CTA
   float scale;
 };
 
+struct PostShared {
+  int hist[kHistBins];  // this CTA's histogram of the current pass
+  int tot[kHistBins];
+  int warp_tot[32];
+  int cnt;
+  int digit, kleft, done;
+  float M[8], Z[8];
+  float dnum[8][kD];  // this CTA's correction of the numerators, then its partial numerators
+  float dden[8];      // this CTA's correction of the denominators
+};
 
-// block = kD threads (thread = head-dim element); every token of the chunk is
-// loaded with independent loads before anything is computed
-__global__ void __launch_bounds__(kD) kv_correct_kernel(CorrArgs a) {
-  __shared__ float kf[kCorrTok][kD + 4];
-  __shared__ float vbs[kCorrTok][kD];
-  __shared__ float vfs[kCorrTok][kD];
-  __shared__ float qs[8][kD + 4];
-  __shared__ float wf[kCorrTok][8], wb[kCorrTok][8];
-  __shared__ int ts[kCorrTok];
-  const int d = threadIdx.x;
-  const int chunk = blockIdx.x, g = blockIdx.y, bat = blockIdx.z;
+// Filled by the peers (distributed shared memory stores, which do not stall the
+// writer); read locally after a cluster barrier.
+struct PostMail {
+  int hist[2][kPostCl][kHistBins];  // per pass (alternating): every CTA's histogram
+  int cnt[kPostCl];                 // every CTA's packed (above, equal) counts
+  int tok[kPostMaxSel];             // the selected tokens this CTA refines, by position
+  float num[kPostCl][kD];           // this CTA's query head: every CTA's partial numerator
+  float den[kPostCl];
+};
+
+// Words of one staged token: K codes (4b), K refinement (4r), K and V (s, m)
+// (4 + 4), the token's 8 value chunks of codes (8 x 2b) and refinement (8 x 2r).
+__host__ __device__ constexpr int tok_words(int b, int r) { return 20 * (b + r) + 8; }
+
+// GQP: query heads per KV head, padded to 4 or 8 (register arrays); B, R:
+// the cache's base and refinement bits.
+template <int GQP, int B, int R>
+__global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cr = (int)cluster.block_rank(), CL = (int)cluster.num_blocks();
+  extern __shared__ __align__(16) uint8_t dyn[];
+  PostMail& mail = *reinterpret_cast<PostMail*>(dyn);
+  uint32_t* stage = reinterpret_cast<uint32_t*>(dyn + sizeof(PostMail));  // staged selected tokens
+  uint32_t* keys = stage + kPostStage * tok_words(B, R);               // this CTA's score keys
+  __shared__ PostShared sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = kPostThreads / 32;
+  const int g = blockIdx.y, bat = blockIdx.z;
   const int gq = a.gq;
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
-  for (int h = 0; h < gq; h++) qs[h][d] = h2f(a.q[(hq0 + h) * kD + d]);
-  const int j0 = chunk * kCorrTok;
-  const int nsel = min(kCorrTok, a.k_tok - j0);
-  const int32_t* sg = a.sel + ((long)bat * a.h_kv + g) * a.k_tok + j0;
-  if (d < nsel) ts[d] = sg[d];
-  __syncthreads();
-  const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
-  const float half = 0.5f * (float)(1 << a.r), inv = 1.0f / (float)(1 << a.r);
-  int kw, kbit, krw, krbit;
-  key_pos(d, a.b, kw, kbit);
-  key_pos(d, a.r, krw, krbit);
-  // all loads first (independent), then the arithmetic
-  uint32_t rqk[kCorrTok], rrk[kCorrTok], rzk[kCorrTok], rqv[kCorrTok], rrv[kCorrTok], rzv[kCorrTok];
-  int rvb[kCorrTok], rvr[kCorrTok];
-#pragma unroll
-  for (int i = 0; i < kCorrTok; i++) {
-    if (i < nsel) {
-      const int t = ts[i];
-      const long slot = slot0 + t;
-      const long tile = slot / 16;
-      int vw, vbit, vrw, vrbit;
-      value_pos(t & 15, d, a.b, vw, vbit);
-      value_pos(t & 15, d, a.r, vrw, vrbit);
-      rqk[i] = reinterpret_cast<const uint32_t*>(a.kb + slot * 16 * a.b)[kw];
-      rrk[i] = reinterpret_cast<const uint32_t*>(a.kr + slot * 16 * a.r)[krw];
-      rzk[i] = *reinterpret_cast<const uint32_t*>(a.ksz + (slot * 4 + d / 32) * 2);
-      rqv[i] = reinterpret_cast<const uint32_t*>(a.vb + tile * 256 * a.b)[vw];
-      rrv[i] = reinterpret_cast<const uint32_t*>(a.vr + tile * 256 * a.r)[vrw];
-      rzv[i] = *reinterpret_cast<const uint32_t*>(a.vsz + (slot * 4 + d / 32) * 2);
-      rvb[i] = vbit, rvr[i] = vrbit;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kCorrTok; i++) {
-    if (i < nsel) {
-      const uint32_t qk = (rqk[i] >> kbit) & ((1u << a.b) - 1);
-      const uint32_t rk = (rrk[i] >> krbit) & ((1u << a.r) - 1);
-      const uint32_t qv = (rqv[i] >> rvb[i]) & ((1u << a.b) - 1);
-      const uint32_t rv = (rrv[i] >> rvr[i]) & ((1u << a.r) - 1);
-      const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&rzk[i]));
-      const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&rzv[i]));
-      kf[i][d] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
-      vbs[i][d] = fmaf(v2.x, (float)qv, v2.y);
-      vfs[i][d] = fmaf(v2.x, (float)qv + ((float)rv + 0.5f - half) * inv, v2.y);
-    }
-  }
-  __syncthreads();
-  // refined logits of (token, head) pairs; base logits as the base pass stored them
-  for (int pr = d; pr < nsel * gq; pr += kD) {
-    const int i = pr / gq, h = pr % gq;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int e = 0; e < kD; e++) acc = fmaf(qs[h][e], kf[i][e], acc);
-    const float M = a.stats[hq0 + h].x;
-    const float lb = a.logits[(hq0 + h) * a.T + ts[i]];
-    wf[i][h] = __expf(acc * a.scale - M);
-    wb[i][h] = __expf(lb - M);
-  }
-  __syncthreads();
-  for (int h = 0; h < gq; h++) {
-    float da = 0.f, dz = 0.f;
-    for (int i = 0; i < nsel; i++) {
-      da = fmaf(wf[i][h], vfs[i][d], fmaf(-wb[i][h], vbs[i][d], da));
-      dz += wf[i][h] - wb[i][h];
-    }
-    float* rec = a.corr + ((hq0 + h) * a.ncorr + chunk) * kRec;
-    rec[d] = da;
-    if (d == 0) rec[kD] = dz;
-  }
-}
+  pdl_trigger();
+  for (int i = tid; i < 8 * kD; i += kPostThreads) (&sh.dnum[0][0])[i] = 0.f;
+  if (tid < 8) sh.dden[tid] = 0.f;
+  // every CTA of the cluster must have started before peers touch its shared
+  // memory: arrive now, wait right before the first distributed access
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  pdl_wait();  // the base pass is complete
 
-// out = (sum_s e^(m_s - M) acc_s + sum_c dA_c) / (Z + sum_c dZ_c).
-// 4 x kD threads: thread group r sums every 4th record.
-constexpr int kMergeGroups = 4;
-constexpr int kMaxRec = 4096;
-
-__global__ void __launch_bounds__(kMergeGroups * kD) kv_merge_kernel(
-    const float* __restrict__ part, int nrec, const float* __restrict__ corr, int ncorr,
-    const float2* __restrict__ stats, float* __restrict__ out) {
-  __shared__ float wts[kMaxRec];
-  __shared__ float red[kMergeGroups][kD + 1];
-  const long bh = blockIdx.x;
-  const float2 st = stats[bh];
-  const float* p = part + bh * nrec * kRec;
-  for (int s = threadIdx.x; s < nrec; s += blockDim.x) {
-    const float ms = p[(long)s * kRec + kD];
-    wts[s] = ms > -INFINITY ? expf(ms - st.x) : 0.f;
-  }
-  __syncthreads();
-  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
-  float num = 0.f, dz = 0.f;
-  int s = grp;
-  for (; s + 3 * kMergeGroups < nrec; s += 4 * kMergeGroups) {
-    const float v0 = p[(long)s * kRec + d], v1 = p[(long)(s + kMergeGroups) * kRec + d];
-    const float v2 = p[(long)(s + 2 * kMergeGroups) * kRec + d], v3 = p[(long)(s + 3 * kMergeGroups) * kRec + d];
-    num = fmaf(wts[s], v0, num);
-    num = fmaf(wts[s + kMergeGroups], v1, num);
-    num = fmaf(wts[s + 2 * kMergeGroups], v2, num);
-    num = fmaf(wts[s + 3 * kMergeGroups], v3, num);
-  }
-  for (; s < nrec; s += kMergeGroups) num = fmaf(wts[s], p[(long)s * kRec + d], num);
-  if (corr) {
-    const float* c = corr + bh * ncorr * kRec;
-    for (int i = grp; i < ncorr; i += kMergeGroups) {
-      num += c[(long)i * kRec + d];
-      dz += c[(long)i * kRec + kD];
-    }
-  }
-  red[grp][d] = num;
-  if (d == 0) red[grp][kD] = dz;
-  __syncthreads();
-  if (grp == 0) {
-    float n = 0.f, z = st.y;
+  // softmax statistics of the group's query heads: every record's (m, l)
+  // loaded in one batch per lane
+  if (warp < gq) {
+    const float* pr = a.part + (hq0 + warp) * a.nrec * a.rec;
+    constexpr int PER = 8;
+    float ms[PER], ls[PER];
+    float m = -INFINITY, z = 0.f;
+    for (int s0 = 0; s0 < a.nrec; s0 += 32 * PER) {
 #pragma unroll
-    for (int r = 0; r < kMergeGroups; r++) {
-      n += red[r][d];
-      z += red[r][kD];
+      for (int k = 0; k < PER; k++) {
+        const int s = s0 + lane + 32 * k;
+        ms[k] = s < a.nrec ? pr[(long)s * a.rec + a.rec - 2] : -INFINITY;
+        ls[k] = s < a.nrec ? pr[(long)s * a.rec + a.rec - 1] : 0.f;
+      }
+      float mb = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < PER; k++) mb = fmaxf(mb, ms[k]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+      const float mn = fmaxf(m, mb);
+      float zb = 0.f;
+#pragma unroll
+      for (int k = 0; k < PER; k++)
+        if (ms[k] > -INFINITY) zb += ls[k] * expf(ms[k] - mn);
+      z = (m > -INFINITY ? z * expf(m - mn) : 0.f) + zb;
+      m = mn;
     }
-    out[bh * kD + d] = n / z;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) sh.M[warp] = m, sh.Z[warp] = z;
+  }
+  __syncthreads();
+
+  const int ja = (int)((long)cr * a.k_tok / CL), jb = (int)((long)(cr + 1) * a.k_tok / CL);
+  if (a.select) {
+    const int t0 = cr * a.chunk, n = max(0, min(a.T, t0 + a.chunk) - t0);
+    const float* lg = a.logits + hq0 * a.T + t0;
+    float Mh[GQP], invZ[GQP];
+#pragma unroll
+    for (int h = 0; h < GQP; h++) Mh[h] = h < gq ? sh.M[h] : 0.f, invZ[h] = h < gq ? 1.0f / sh.Z[h] : 0.f;
+    // eight tokens per thread per step (token tid + 512 e: coalesced), every load
+    // of the step issued first
+    constexpr int TPT = 8;
+    for (int i0 = tid; i0 < n; i0 += TPT * kPostThreads) {
+      float l[GQP][TPT];
+#pragma unroll
+      for (int h = 0; h < GQP; h++)
+#pragma unroll
+        for (int e = 0; e < TPT; e++) {
+          const int i = i0 + e * kPostThreads;
+          l[h][e] = (h < gq && i < n) ? lg[(long)h * a.T + i] : -INFINITY;
+        }
+#pragma unroll
+      for (int e = 0; e < TPT; e++) {
+        const int i = i0 + e * kPostThreads;
+        if (i < n) {
+          float sc = 0.f;
+#pragma unroll
+          for (int h = 0; h < GQP; h++)
+            if (h < gq) sc += __expf(l[h][e] - Mh[h]) * invZ[h];
+          if (a.scores) a.scores[((long)bat * a.h_kv + g) * a.T + t0 + i] = sc;
+          keys[i] = __float_as_uint(sc);
+        }
+      }
+    }
+    // ---- radix select of the k_tok-th largest key over the cluster: digits of
+    // bits 30..22, 21..13, 12..4, 3..0 (bit 31 is 0 for non-negative scores)
+    uint32_t prefix = 0, mask = 0x80000000u;
+    int kleft = a.k_tok, buf = 0;
+    bool done = false;
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    for (int pass = 0; pass < 4 && !done; pass++) {
+      const int shift = pass < 3 ? 22 - 9 * pass : 0;
+      const int bits = pass < 3 ? 9 : 4, bins = 1 << bits;
+      for (int i = tid; i < bins; i += kPostThreads) sh.hist[i] = 0;
+      __syncthreads();
+      for (int i0 = warp * 32; i0 < n; i0 += kPostThreads) {  // whole warps: lanes with equal bins add once
+        const int i = i0 + lane;
+        const uint32_t key = i < n ? keys[i] : 0u;
+        const bool in = i < n && (key & mask) == prefix;
+        const int bn = in ? (int)((key >> shift) & (bins - 1)) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, bn);
+        if (in && (__ffs(same) - 1) == lane) atomicAdd(&sh.hist[bn], __popc(same));
+      }
+      __syncthreads();
+      for (int i = tid; i < bins * CL; i += kPostThreads)  // my histogram into every peer's mailbox
+        cluster.map_shared_rank(&mail.hist[buf][cr][0], i / bins)[i % bins] = sh.hist[i % bins];
+      cluster.sync();  // every CTA's histogram is in every mailbox
+      for (int bn = tid; bn < bins; bn += kPostThreads) {
+        int t = 0;
+        for (int rk = 0; rk < CL; rk++) t += mail.hist[buf][rk][bn];
+        sh.tot[bn] = t;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane covers the bins below bins - 1 - PL lane, from the top
+        const int PL = bins >= 32 ? bins / 32 : 1;
+        int c[16], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+          const int bn = bins - 1 - PL * lane - j;
+          c[j] = (j < PL && bn >= 0) ? sh.tot[bn] : 0;
+          tot += c[j];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int above = incl - tot;
+        if (above < kleft && incl >= kleft) {
+          int run = above;
+          for (int j = 0; j < PL; j++) {
+            if (run + c[j] >= kleft) {
+              sh.digit = bins - 1 - PL * lane - j;
+              sh.kleft = kleft - run;
+              sh.done = c[j] == kleft - run;  // the whole bucket is needed
+              break;
+            }
+            run += c[j];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sh.digit << shift;
+      mask |= (uint32_t)(bins - 1) << shift;
+      kleft = sh.kleft;
+      done = sh.done;
+      buf ^= 1;  // the next pass fills the other mailbox while this one may still be read
+    }
+    // keys above `prefix` (or, when the last bucket was taken whole, at or above
+    // it) are selected; of the keys equal to it, the first `kleft` in token order
+    const int per = (n + kPostThreads - 1) / kPostThreads;
+    const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
+    int ngt = 0, neq = 0;
+    for (int i = i0; i < i1; i++) {
+      const uint32_t key = keys[i];
+      if (done ? key >= prefix : key > prefix) ngt++;
+      else if (!done && key == prefix) neq++;
+    }
+    // one block scan of the packed counts (above + equal << 16), in token order
+    const int v = ngt + (neq << 16);
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) sh.warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int wv = lane < NW ? sh.warp_tot[lane] : 0;
+      int x = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += u;
+      }
+      if (lane < NW) sh.warp_tot[lane] = x - wv;
+      if (lane == 31) sh.cnt = x;
+    }
+    __syncthreads();
+    const int ex = sh.warp_tot[warp] + incl - v;
+    const int gt_ex = ex & 0xFFFF, eq_ex = ex >> 16;
+    if (tid < CL) cluster.map_shared_rank(&mail.cnt[cr], tid)[0] = sh.cnt;
+    cluster.sync();  // every CTA's counts are in every mailbox
+    int sel_before = 0, eq_before = 0;
+    for (int rk = 0; rk < cr; rk++) {
+      const int c = mail.cnt[rk];
+      sel_before += (c & 0xFFFF) + max(0, min(c >> 16, kleft - eq_before));
+      eq_before += c >> 16;
+    }
+    // my selected tokens: above-threshold ones, and equal ones while the budget lasts
+    const int eq_mine = done ? 0 : max(0, min(neq, kleft - (eq_before + eq_ex)));
+    int pos = sel_before + gt_ex + max(0, min(eq_ex, kleft - eq_before));
+    int eq_seen = 0;
+    int32_t* selw = a.sel + ((long)bat * a.h_kv + g) * a.k_tok;
+    for (int i = i0; i < i1; i++) {
+      const uint32_t key = keys[i];
+      bool take = done ? key >= prefix : key > prefix;
+      if (!done && key == prefix) take = eq_seen++ < eq_mine;
+      if (take && pos < a.k_tok) {
+        selw[pos] = t0 + i;
+        if (a.out) {  // hand the token to the CTA that refines position pos
+          const int dst = (int)(((long)(pos + 1) * CL + a.k_tok - 1) / a.k_tok) - 1;
+          const int dja = (int)((long)dst * a.k_tok / CL);
+          cluster.map_shared_rank(&mail.tok[0], dst)[pos - dja] = t0 + i;
+        }
+      }
+      if (take) pos++;
+    }
+    cluster.sync();  // every selected token is in its refining CTA's mailbox
+  } else {
+    const int32_t* selg = a.sel + ((long)bat * a.h_kv + g) * a.k_tok;
+    for (int j = ja + tid; j < jb; j += kPostThreads) mail.tok[j - ja] = selg[j];
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    __syncthreads();
+  }
+  if (!a.out) return;  // no peer reads or writes this CTA's shared memory any more
+
+  // ---- refined attention on this CTA's share of the selected tokens
+  {
+    const int W = tok_words(B, R);
+    const int oK = 0, oKr = 4 * B, oZk = 4 * (B + R), oZv = oZk + 4, oV = oZv + 4, oVr = oV + 16 * B;
+    const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
+    const float half = 0.5f * (float)(1 << R), inv = 1.0f / (float)(1 << R);
+    const uint32_t bmask = (1u << B) - 1u, rmask = (1u << R) - 1u;
+    // lane owns head dims d_e = lane + 32 e (scale group e)
+    int kw[4], kbit[4], krw[4], krbit[4];
+    float qv[GQP][4];
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      key_pos(lane + 32 * e, B, kw[e], kbit[e]);
+      key_pos(lane + 32 * e, R, krw[e], krbit[e]);
+#pragma unroll
+      for (int h = 0; h < GQP; h++) qv[h][e] = h < gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
+    }
+    float an[GQP][4], ad[GQP];
+#pragma unroll
+    for (int h = 0; h < GQP; h++) {
+      ad[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; e++) an[h][e] = 0.f;
+    }
+    // pieces of one staged token: 16-byte copies (8-byte for 1-bit value refinement chunks)
+    const int pk = B, pkr = R, pv = 8 * (B >= 2 ? B / 2 : 1), pvr = 8 * (R >= 2 ? R / 2 : 1);
+    const int npiece = pk + pkr + 2 + pv + pvr;
+    for (int j0 = ja; j0 < jb; j0 += kPostStage) {
+      const int nt = min(kPostStage, jb - j0);
+      __syncthreads();  // the previous batch is consumed
+      for (int it = tid; it < nt * npiece; it += kPostThreads) {
+        const int i = it / npiece, pc = it % npiece;
+        int t = mail.tok[j0 - ja + i];
+        if (t < 0 || t >= a.T) t = 0;  // out-of-range indices are never produced by the selection
+        const long slot = slot0 + t, tile = slot / 16;
+        const int c = (t & 7) >> 1;  // the token's value chunk column
+        uint32_t* dst = stage + i * W;
+        if (pc < pk) {
+          cp_async16(dst + oK + 4 * pc, a.kb + slot * 16 * B + 16 * pc);
+        } else if (pc < pk + pkr) {
+          const int q4 = pc - pk;
+          cp_async16(dst + oKr + 4 * q4, a.kr + slot * 16 * R + 16 * q4);
+        } else if (pc == pk + pkr) {
+          cp_async16(dst + oZk, reinterpret_cast<const uint8_t*>(a.ksz) + slot * 16);
+        } else if (pc == pk + pkr + 1) {
+          cp_async16(dst + oZv, reinterpret_cast<const uint8_t*>(a.vsz) + slot * 16);
+        } else if (pc < pk + pkr + 2 + pv) {
+          // value codes: chunk l = 4 gg + c holds 2b words; b = 4 takes two 16-byte copies
+          const int q4 = pc - (pk + pkr + 2), gg = B >= 2 ? q4 / (B / 2) : q4, part = B >= 2 ? q4 % (B / 2) : 0;
+          cp_async16(dst + oV + gg * 2 * B + 4 * part,
+                     a.vb + tile * 256 * B + (size_t)(4 * gg + c) * 8 * B + 16 * part);
+        } else {
+          const int q4 = pc - (pk + pkr + 2 + pv);
+          if constexpr (R >= 2) {
+            const int gg = q4 / (R / 2), part = q4 % (R / 2);
+            cp_async16(dst + oVr + gg * 2 * R + 4 * part,
+                       a.vr + tile * 256 * R + (size_t)(4 * gg + c) * 8 * R + 16 * part);
+          } else {
+            cp_async8(dst + oVr + q4 * 2, a.vr + tile * 256 * R + (size_t)(4 * q4 + c) * 8 * R);
+          }
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+      for (int i = warp; i < nt; i += NW) {
+        const uint32_t* st = stage + i * W;
+        const int t = mail.tok[j0 - ja + i];
+        const int tt = t & 15;
+        float kf[4], vbs[4], vfs[4], lg[GQP], lb[GQP];
+#pragma unroll
+        for (int h = 0; h < GQP; h++) lb[h] = h < gq ? a.logits[(hq0 + h) * a.T + t] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int d = lane + 32 * e;
+          int vw, vbit, vrw, vrbit;
+          value_pos(tt, d, B, vw, vbit);
+          value_pos(tt, d, R, vrw, vrbit);
+          // staged chunk gg = d & 7 holds words [l 2w, l 2w + 2w) of the tile
+          const int vwl = vw - (4 * (d & 7) + ((tt & 7) >> 1)) * 2 * B + (d & 7) * 2 * B;
+          const int vrwl = vrw - (4 * (d & 7) + ((tt & 7) >> 1)) * 2 * R + (d & 7) * 2 * R;
+          const uint32_t zk = st[oZk + e], zv = st[oZv + e];
+          const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&zk));
+          const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv));
+          const uint32_t qk = (st[oK + kw[e]] >> kbit[e]) & bmask, rk = (st[oKr + krw[e]] >> krbit[e]) & rmask;
+          const uint32_t qq = (st[oV + vwl] >> vbit) & bmask, rv = (st[oVr + vrwl] >> vrbit) & rmask;
+          kf[e] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
+          vbs[e] = fmaf(v2.x, (float)qq, v2.y);
+          vfs[e] = fmaf(v2.x, (float)qq + ((float)rv + 0.5f - half) * inv, v2.y);
+        }
+#pragma unroll
+        for (int h = 0; h < GQP; h++) {
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[e], acc);
+          lg[h] = acc;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int h = 0; h < GQP; h++)
+            if (h < gq) lg[h] += __shfl_xor_sync(0xffffffffu, lg[h], o);
+#pragma unroll
+        for (int h = 0; h < GQP; h++) {
+          if (h < gq) {
+            const float wf = __expf(lg[h] * a.scale - sh.M[h]), wb = __expf(lb[h] - sh.M[h]);
+#pragma unroll
+            for (int e = 0; e < 4; e++) an[h][e] = fmaf(wf, vfs[e], fmaf(-wb, vbs[e], an[h][e]));
+            ad[h] += wf - wb;
+          }
+        }
+      }
+    }
+    if (ja + warp < jb) {
+#pragma unroll
+      for (int h = 0; h < GQP; h++) {
+        if (h < gq) {
+#pragma unroll
+          for (int e = 0; e < 4; e++) atomicAdd(&sh.dnum[h][lane + 32 * e], an[h][e]);
+          if (lane == 0) atomicAdd(&sh.dden[h], ad[h]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // this CTA's share of the base records: records s = cr, cr + CL, ... (loads batched)
+  for (int e = tid; e < gq * kD; e += kPostThreads) {
+    const int hh = e / kD, d = e % kD;
+    const float* pr = a.part + (hq0 + hh) * a.nrec * a.rec;
+    float num = sh.dnum[hh][d];
+    constexpr int PER = 8;
+    for (int s0 = cr; s0 < a.nrec; s0 += CL * PER) {
+      float mv[PER], av[PER];
+#pragma unroll
+      for (int k = 0; k < PER; k++) {
+        const int s = s0 + CL * k;
+        mv[k] = s < a.nrec ? pr[(long)s * a.rec + kD] : -INFINITY;
+        av[k] = s < a.nrec ? pr[(long)s * a.rec + d] : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < PER; k++)
+        if (mv[k] > -INFINITY) num = fmaf(__expf(mv[k] - sh.M[hh]), av[k], num);
+    }
+    cluster.map_shared_rank(&mail.num[cr][0], hh)[d] = num;  // to the CTA that merges head hh
+  }
+  if (tid < gq) cluster.map_shared_rank(&mail.den[cr], tid)[0] = sh.dden[tid];
+  cluster.sync();  // every partial numerator is in its head's mailbox
+  if (cr < gq) {
+    for (int d = tid; d < kD; d += kPostThreads) {
+      float num = 0.f, den = sh.Z[cr];
+      for (int rk = 0; rk < CL; rk++) num += mail.num[rk][d], den += mail.den[rk];
+      a.out[(hq0 + cr) * kD + d] = num / den;
+    }
   }
 }
 
@@ -728,14 +933,14 @@ __global__ void __launch_bounds__(kMergeGroups * kD) kv_merge_kernel(
 // host side
 
 struct Plan {
-  int nsplit, span, nrec; // base pass (warp splits; one record per CTA of kWarps splits)
-  int sspan, ns;          // selection spans
-  int ncorr;              // correction chunks per KV head
-  size_t off_logits, off_part, off_stats, off_cand, off_corr, total;
+  int nsplit, span, nrec;  // base pass (warp splits; one record per CTA of kWarps splits)
+  int cl, chunk;           // cluster size and tokens per CTA after the base pass
+  size_t off_logits, off_part, total;
 };
 
 Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, bool with_pv,
                bool select, int n_splits) {
+  (void)k_tok, (void)select;
   Plan P;
   const int sms = num_sms();
   const int heads = kv->batch * kv->h_kv;
@@ -745,20 +950,9 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   if (ns < 1) ns = 1;
   P.span = ((t + ns - 1) / ns + 15) / 16 * 16;
   P.nsplit = (t + P.span - 1) / P.span;
-  P.nrec = (P.nsplit + kWarps - 1) / kWarps;  // <= kMaxRec is checked by the callers
-  // selection spans
-  int ss = (sms + heads - 1) / heads;
-  if (ss < 1) ss = 1;
-  int span = (t + ss - 1) / ss;
-  if (span > kMaxSpan) span = kMaxSpan;
-  if (span < 32) span = 32;
-  ss = (t + span - 1) / span;
-  while (ss > 1 && (long)ss * (k_tok < span ? k_tok : span) > kMaxCand && span < kMaxSpan) {
-    span = span * 2 > kMaxSpan ? kMaxSpan : span * 2;
-    ss = (t + span - 1) / span;
-  }
-  P.sspan = span, P.ns = ss;
-  P.ncorr = k_tok > 0 ? (k_tok + kCorrTok - 1) / kCorrTok : 0;
+  P.nrec = (P.nsplit + kWarps - 1) / kWarps;
+  P.cl = kPostCl;
+  P.chunk = (t + P.cl - 1) / P.cl;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -768,9 +962,6 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   const int rec = with_pv ? kRec : 2;
   P.off_logits = need_logits ? take((size_t)kv->batch * h_q * t * 4) : 0;
   P.off_part = take((size_t)kv->batch * h_q * P.nrec * rec * 4);
-  P.off_stats = take((size_t)kv->batch * h_q * 8);
-  P.off_cand = select ? take((size_t)heads * P.ns * (k_tok < span ? k_tok : span) * 8) : 0;
-  P.off_corr = (with_pv && P.ncorr) ? take((size_t)kv->batch * h_q * P.ncorr * kRec * 4) : 0;
   P.total = off;
   return P;
 }
@@ -781,6 +972,7 @@ sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
   SF_UNSUPPORTED(h_q > 0 && h_q % kv->h_kv == 0 && h_q / kv->h_kv <= 8,
                  "h_q=%d must be a multiple of h_kv=%d with at most 8 query heads per KV head", h_q,
                  kv->h_kv);
+  SF_UNSUPPORTED(t <= kPostCl * kPostMaxTok, "t=%d above %d", t, kPostCl * kPostMaxTok);
   return SF_OK;
 }
 
@@ -789,9 +981,17 @@ sf_status launch_base_t(const BaseArgs& a, int batch, cudaStream_t s) {
   const size_t smem = kWarps * WarpSmem<B, PV>::bytes;
   auto kern = kv_base_kernel<GQP, B, PV>;
   SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  dim3 grid((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch);
-  kern<<<grid, kWarps * 32, smem, s>>>(a);
-  SF_LAUNCHED();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;  // launch overlaps the previous kernel's tail
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SF_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
   return SF_OK;
 }
 
@@ -818,43 +1018,44 @@ BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* lo
   return a;
 }
 
-sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& P,
-                        const float* logits, const float2* stats, float* scores, uint64_t* cand,
-                        int32_t* sel, cudaStream_t s) {
-  long ncand = (long)P.ns * (k_tok < P.sspan ? k_tok : P.sspan);
-  SF_UNSUPPORTED(ncand <= kMaxCand, "t=%d with k_tok=%d needs %ld candidates (max %d)", t, k_tok,
-                 ncand, kMaxCand);
-  SF_CUDA(cudaFuncSetAttribute(kv_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSpan * 8));
-  kv_local_kernel<<<dim3(P.ns, kv->h_kv, kv->batch), 1024, (size_t)P.sspan * 8, s>>>(
-      logits, stats, t, P.sspan, h_q, kv->h_kv, k_tok, scores, cand);
-  SF_LAUNCHED();
-  SF_CUDA(cudaFuncSetAttribute(kv_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCand * 8));
-  kv_final_kernel<<<dim3(kv->h_kv, kv->batch), 1024, (size_t)ncand * 8, s>>>(cand, P.ns, P.sspan, t,
-                                                                           kv->h_kv, k_tok, sel);
-  SF_LAUNCHED();
-  return SF_OK;
-}
-
-sf_status launch_correct_merge(const sf_kv* kv, int t, const uint16_t* q, int h_q,
-                               const int32_t* sel, int k_tok, const Plan& P, const float* logits,
-                               const float* part, const float2* stats, float* corr, float* out,
-                               cudaStream_t s) {
-  if (k_tok > 0) {
-    CorrArgs c;
-    c.kb = (const uint8_t*)kv->kb, c.kr = (const uint8_t*)kv->kr;
-    c.vb = (const uint8_t*)kv->vb, c.vr = (const uint8_t*)kv->vr;
-    c.ksz = kv->ksz, c.vsz = kv->vsz;
-    c.h_kv = kv->h_kv, c.t_max = kv->t_max, c.b = kv->b, c.r = kv->r, c.T = t;
-    c.q = q, c.h_q = h_q, c.gq = h_q / kv->h_kv;
-    c.sel = sel, c.k_tok = k_tok, c.logits = logits, c.stats = stats;
-    c.corr = corr, c.ncorr = P.ncorr;
-    c.scale = 1.0f / sqrtf((float)kD);
-    kv_correct_kernel<<<dim3(P.ncorr, kv->h_kv, kv->batch), kD, 0, s>>>(c);
-    SF_LAUNCHED();
-  }
-  kv_merge_kernel<<<kv->batch * h_q, kMergeGroups * kD, 0, s>>>(part, P.nrec, k_tok > 0 ? corr : nullptr,
-                                                                P.ncorr, stats, out);
-  SF_LAUNCHED();
+// The cluster kernel after the base pass (launched with programmatic
+// serialization: its CTAs start while the base pass drains).
+sf_status launch_post(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
+                      const float* logits, const float* part, int rec, int32_t* sel, int select,
+                      float* scores, float* out, cudaStream_t s) {
+  PostArgs a;
+  a.kb = (const uint8_t*)kv->kb, a.kr = (const uint8_t*)kv->kr;
+  a.vb = (const uint8_t*)kv->vb, a.vr = (const uint8_t*)kv->vr;
+  a.ksz = kv->ksz, a.vsz = kv->vsz;
+  a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.b = kv->b, a.r = kv->r, a.T = t;
+  a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
+  a.logits = logits, a.part = part, a.nrec = P.nrec, a.rec = rec;
+  a.k_tok = k_tok, a.sel = sel, a.select = select, a.scores = scores, a.out = out;
+  a.chunk = P.chunk;
+  a.scale = 1.0f / sqrtf((float)kD);
+  const size_t smem = sizeof(PostMail) + ((size_t)kPostStage * tok_words(kv->b, kv->r) + P.chunk) * 4;
+  void (*kern)(PostArgs);
+  if (a.gq <= 4)
+    kern = kv->b == 2 ? (kv->r == 2 ? kv_post_kernel<4, 2, 2> : kv_post_kernel<4, 2, 1>)
+                      : (kv->r == 2 ? kv_post_kernel<4, 4, 2> : kv_post_kernel<4, 4, 1>);
+  else
+    kern = kv->b == 2 ? (kv->r == 2 ? kv_post_kernel<8, 2, 2> : kv_post_kernel<8, 2, 1>)
+                      : (kv->r == 2 ? kv_post_kernel<8, 4, 2> : kv_post_kernel<8, 4, 1>);
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(sizeof(PostMail) + ((size_t)kPostStage * tok_words(4, 2) + kPostMaxTok) * 4)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.cl, kv->h_kv, kv->batch);
+  cfg.blockDim = dim3(kPostThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = P.cl, attr[0].val.clusterDim.y = 1, attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  SF_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
   return SF_OK;
 }
 
@@ -886,24 +1087,20 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
   SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
-  SF_UNSUPPORTED(k_tok <= 4096, "k_tok=%d above 4096", k_tok);
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(!scores || aligned16(scores), "scores must be 16-byte aligned");
   Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, false, true, 0);
-  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   float* lg = logits ? logits : (float*)(w + P.off_logits);
+  float* part = (float*)(w + P.off_part);
   cudaStream_t s = as_stream(stream);
-  BaseArgs a = base_args(kv, t, q, h_q, lg, (float*)(w + P.off_part), P);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, false, s);
   if (st != SF_OK) return st;
-  float2* stats = (float2*)(w + P.off_stats);
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>((const float*)(w + P.off_part), P.nrec, 2, stats);
-  SF_LAUNCHED();
-  return launch_select(kv, t, h_q, k_tok, P, lg, stats, scores, (uint64_t*)(w + P.off_cand), sel, s);
+  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, 2, sel, 1, scores, nullptr, s);
 }
 
 extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
@@ -924,21 +1121,17 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(n_splits >= 0, "n_splits=%d < 0", n_splits);
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
   Plan P = make_plan(kv, t, h_q, k_tok, true, true, false, n_splits);
-  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   cudaStream_t s = as_stream(stream);
   float* lg = (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
-  float2* stats = (float2*)(w + P.off_stats);
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nrec, kRec, stats);
-  SF_LAUNCHED();
-  return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
-                              (float*)(w + P.off_corr), out, s);
+  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, const_cast<int32_t*>(sel), 0, nullptr,
+                     out, s);
 }
 
 extern "C" size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q,
@@ -955,28 +1148,20 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
   SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
-  SF_UNSUPPORTED(k_tok <= 4096, "k_tok=%d above 4096", k_tok);
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
   Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0);
-  SF_UNSUPPORTED(P.nrec <= kMaxRec, "t=%d needs %d partial records (max %d)", t, P.nrec, kMaxRec);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   cudaStream_t s = as_stream(stream);
   float* lg = logits ? logits : (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
-  float2* stats = (float2*)(w + P.off_stats);
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  kv_stats_kernel<<<kv->batch * h_q, 256, 0, s>>>(part, P.nrec, kRec, stats);
-  SF_LAUNCHED();
-  st = launch_select(kv, t, h_q, k_tok, P, lg, stats, nullptr, (uint64_t*)(w + P.off_cand), sel, s);
-  if (st != SF_OK) return st;
-  return launch_correct_merge(kv, t, q, h_q, sel, k_tok, P, lg, part, stats,
-                              (float*)(w + P.off_corr), out, s);
+  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, sel, 1, nullptr, out, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(
     uint32_t* __restrict__ codes, uint32_t* __restrict__ refine, uint16_t* __restrict__ sz) {
   // keys: 4B code words + 4R refinement words; values: 8B + 8R halves
   __shared__ uint32_t acc[kPackWarps][8 * (B + R)];
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long idx = (long)blockIdx.x * kPackWarps + warp;
   if (idx >= (long)BH * nt) return;  // whole warps only
@@ -140,9 +142,9 @@ template <int B, int R>
 sf_status launch_pack(const uint16_t* x, int BH, int nt, int t_max, int t0, int is_value,
                       void* codes, void* refine, uint16_t* sz, cudaStream_t s) {
   const long total = (long)BH * nt;
-  pack_kv_kernel<B, R><<<(unsigned)((total + kPackWarps - 1) / kPackWarps), kPackWarps * 32, 0, s>>>(
-      x, BH, nt, t_max, t0, is_value, (uint32_t*)codes, (uint32_t*)refine, sz);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(pack_kv_kernel<B, R>, dim3((unsigned)((total + kPackWarps - 1) / kPackWarps)),
+                     dim3(kPackWarps * 32), 0, s, x, BH, nt, t_max, t0, is_value, (uint32_t*)codes,
+                     (uint32_t*)refine, sz));
   return SF_OK;
 }
 

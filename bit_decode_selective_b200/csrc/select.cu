@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(kSelThreads) select_chunks_kernel(const uint16
                                                                    int K, int chunk, int kch,
                                                                    int32_t* __restrict__ sel) {
   pdl_trigger();  // a dependent GEMV may start streaming its base codes now
+  pdl_wait();
   __shared__ uint32_t keys[2048];
   __shared__ RadixShared sh;
   const int b = blockIdx.y, c = blockIdx.x;
@@ -52,8 +53,7 @@ sf_status check_select_args(const uint16_t* x, int batch, int k, int chunk, int 
 sf_status launch_select(const uint16_t* x, int batch, int k, int chunk, int kch, int32_t* sel,
                         cudaStream_t s) {
   dim3 grid(k / chunk, batch);
-  select_chunks_kernel<<<grid, kSelThreads, 0, s>>>(x, k, chunk, kch, sel);
-  SF_LAUNCHED();
+  SF_CUDA(launch_pdl(select_chunks_kernel, grid, dim3(kSelThreads), 0, s, x, k, chunk, kch, sel));
   return SF_OK;
 }
 

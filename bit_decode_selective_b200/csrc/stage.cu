@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           size_t row_vecs,
                                                           const int32_t* __restrict__ sel,
                                                           int n_sel, uint4* __restrict__ dst) {
+  pdl_trigger();
+  pdl_wait();
   const size_t total = (size_t)n_sel * row_vecs;
   const size_t stride = (size_t)gridDim.x * blockDim.x * kVec;
   for (size_t base = ((size_t)blockIdx.x * blockDim.x) * kVec + threadIdx.x; base < total;
@@ -67,9 +69,8 @@ extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_byte
     size_t vecs = (size_t)n_sel * (row_bytes / 16);
     long blocks = (long)((vecs + 256 * kVec - 1) / (256 * kVec));
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, s>>>((const uint4*)attr.devicePointer,
-                                                        row_bytes / 16, sel, n_sel, (uint4*)dst);
-    SF_LAUNCHED();
+    SF_CUDA(launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
+                       (const uint4*)attr.devicePointer, (size_t)(row_bytes / 16), sel, n_sel, (uint4*)dst));
   }
   if (done) SF_CUDA(cudaEventRecord((cudaEvent_t)done, s));
   return SF_OK;

@@ -151,12 +151,11 @@ SF_API sf_status sf_select_channels(const uint16_t* x, int batch, int k, int chu
  *   refine_rows (nullable): staged refinement rows [batch][k/chunk*kch][n*r/8];
  *     row j of batch row b holds the refinement of channel sel[b][j]
  *     (flattened over chunks).  NULL: rows are read from w->refine.
- *   ws/ws_bytes: at least sf_gemv_workspace_bytes() bytes of device scratch
- *     (the activations prepared as exact fixed point: batch * k/64 * 208
- *     bytes); a smaller ws returns SF_ERR_WORKSPACE.
- * The call enqueues up to three kernels: the selection (when sel_in is NULL),
- * the activation prologue and the GEMV (the latter two overlapped through
- * programmatic dependent launch). */
+ *   ws/ws_bytes: sf_gemv_workspace_bytes(); currently 0 (ws may be NULL).
+ * The call enqueues the selection (when sel_in is NULL) and the GEMV, which is
+ * launched with programmatic serialization: its CTAs start copying codes
+ * while the previous kernel of the stream drains, and wait for it before
+ * reading x, the selection or the staged rows. */
 SF_API sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                           const int32_t* sel_in, int32_t* sel_out, const void* refine_rows,
                           float* y, void* ws, size_t ws_bytes, sf_stream_t stream);

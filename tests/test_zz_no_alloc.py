@@ -79,13 +79,13 @@ def test_static_scratch_matches_workspace_call(T, k_tok, batch):
 def test_static_scratch_rejects_oversize_request():
     """A request whose workspace exceeds the 32 MiB array fails with
     SF_ERR_WORKSPACE before anything is enqueued."""
-    T = 270000  # 32 query heads x T x 4-byte logits = 34.6 MB > 32 MiB
-    cache = KVCache(1, 8, (T + 15) // 16 * 16)
+    B, T = 2, 133000  # 2 x 32 query heads x T x 4-byte logits = 34.0 MB > 32 MiB
+    cache = KVCache(B, 8, (T + 15) // 16 * 16)
     need = abi.sf_kv_attend_selective_workspace_bytes(ctypes.byref(cache.desc), T, 32, 64, 0)
     assert need > abi.SF_KV_STATIC_WS_BYTES
-    q = torch.zeros((1, 32, 128), dtype=torch.float16, device="cuda")
-    out = torch.zeros((1, 32, 128), dtype=torch.float32, device="cuda")
-    sel = torch.zeros((1, 8, 64), dtype=torch.int32, device="cuda")
+    q = torch.zeros((B, 32, 128), dtype=torch.float16, device="cuda")
+    out = torch.zeros((B, 32, 128), dtype=torch.float32, device="cuda")
+    sel = torch.zeros((B, 8, 64), dtype=torch.int32, device="cuda")
     st = abi.sf_kv_attend_selective_static(ctypes.byref(cache.desc), T, _p(q), 32, 64, _p(sel), None, _p(out),
                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == abi.SF_ERR_WORKSPACE
