@@ -115,7 +115,11 @@ class Decoder:
         wq = abi.sf_wq(128, kmax, cfg.w_bits, cfg.w_refine, cfg.group, None, None, None)
         self.gemv_ws = torch.empty(max(abi.sf_gemv_workspace_bytes(ctypes.byref(wq), B, cfg.chunk, cfg.kch), 16),
                                    dtype=torch.uint8, device=dev)
+        # staging queues: selections and row transfers of qkv and gate_up on one,
+        # of o and down on the other, so that transfers of different projections overlap
         self.side = torch.cuda.Stream(device=dev)
+        self.side2 = torch.cuda.Stream(device=dev)
+        self.stage_stream = {"qkv": self.side, "gate_up": self.side, "o": self.side2, "down": self.side2}
         self.ev_sel = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
         self.ev_stage = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
         # fetch lag: the side stream sums layer l's o and down corrections into
@@ -172,22 +176,23 @@ class Decoder:
         slot `slot` on the side stream (enqueued after the selection)."""
         check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
                                        _p(self.sel[name][slot]), self.B * self.n_sel[name],
-                                       _p(self.slots[name][slot]), _s(self.side), None),
+                                       _p(self.slots[name][slot]), _s(self.stage_stream[name]), None),
               "sf_stage_refinements")
 
     def _side_select_stage(self, layer, name, x, slot, main):
-        """Selection from x and the row transfer, both on the side stream; the
-        event ev_stage[name][slot] marks both done."""
+        """Selection from x and the row transfer, both on the projection's
+        staging stream; the event ev_stage[name][slot] marks both done."""
+        side = self.stage_stream[name]
         ev = self.ev_sel[name][slot]
         ev.record(main)
-        self.side.wait_event(ev)
+        side.wait_event(ev)
         if (name, slot) in self.lag_pending:  # a lag correction still reads this slot
-            self.side.wait_event(self.ev_lag_done[name][slot])
+            side.wait_event(self.ev_lag_done[name][slot])
             self.lag_pending.discard((name, slot))
-        self._select(name, x, slot, self.side)
+        self._select(name, x, slot, side)
         if self.slots is not None:
             self._stage(layer, name, slot)
-        self.ev_stage[name][slot].record(self.side)
+        self.ev_stage[name][slot].record(side)
 
     def _ready(self, name, slot, main):
         """Wait (on the main stream) for the selection and rows in `slot`."""
@@ -263,6 +268,7 @@ class Decoder:
         cfg = self.cfg
         main = torch.cuda.current_stream(self.dev)
         self.side.wait_stream(main)
+        self.side2.wait_stream(main)
         self.lag_stream.wait_stream(main)
         self.lag_pending = set()
         B, T = self.B, self.T
@@ -313,5 +319,6 @@ class Decoder:
         check(abi.sf_gemv_f16(_p(self.lm_head), _p(self.x_final), B, cfg.vocab, cfg.hidden, _p(self.logits),
                               _s(main)), "sf_gemv_f16")
         main.wait_stream(self.side)
+        main.wait_stream(self.side2)
         main.wait_stream(self.lag_stream)
         return self.logits
