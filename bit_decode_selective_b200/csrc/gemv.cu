@@ -264,9 +264,25 @@ template <int BITS>
 __device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ xs) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ngrp = p.K / kLaneCh;
-  for (int grp = warp; grp < ngrp; grp += kWarps) {
-    const float2 xv = __half22float2(
-        reinterpret_cast<const __half2*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh)[lane]);
+  // the activations of all this warp's groups are loaded before any is used
+  constexpr int PRE = 16;
+  uint32_t xpre[PRE];
+#pragma unroll
+  for (int k = 0; k < PRE; k++) {
+    const int grp = warp + k * kWarps;
+    xpre[k] = grp < ngrp ? __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane)
+                         : 0u;
+  }
+  for (int grp = warp, k = 0; grp < ngrp; grp += kWarps, k++) {
+    uint32_t xw;
+    if (k < PRE) {
+#pragma unroll
+      for (int kk = 0; kk < PRE; kk++)
+        if (kk == k) xw = xpre[kk];
+    } else {
+      xw = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane);
+    }
+    const float2 xv = __half22float2(*reinterpret_cast<const __half2*>(&xw));
     float mx = fmaxf(fabsf(xv.x), fabsf(xv.y));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -311,9 +327,15 @@ __device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ x
 __device__ void corr_fill(const GemvParams& p, int b, int j0, int jn, int w_lo, int nwr, uint4* jd,
                           uint32_t* wt) {
   for (int i = threadIdx.x; i < jn; i += kThreads) {
-    const uint4 d = make_jd(p, b, j0 + i);
-    jd[i] = d;
-    for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + d.w + w_lo + k);
+    if (p.staged) {  // the staged row of entry j is known without the selection: copy it first
+      const uint32_t off = (uint32_t)(((size_t)b * p.n_sel + j0 + i) * p.refine_row_words);
+      for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + off + w_lo + k);
+      jd[i] = make_jd(p, b, j0 + i);
+    } else {
+      const uint4 d = make_jd(p, b, j0 + i);
+      jd[i] = d;
+      for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + d.w + w_lo + k);
+    }
   }
   cp_async_commit();
 }
