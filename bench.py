@@ -71,7 +71,7 @@ class ClockSampler:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -161,6 +161,13 @@ def count_kernels(graph) -> int | None:
         return kern
     except Exception:
         return None
+
+
+# DRAM bytes (read + write) of one refined GEMV launch in an ncu capture
+# (`bench.py --case gemv`: the 28,672 x 4,096 launch, 2 + 2 bits, k = 32 per
+# 1,024) over that launch's algorithmic bytes; traffic grows in proportion to
+# the codes a launch streams, so a launch's traffic is its bytes times this.
+GEMV_TRAFFIC_PER_BYTE = 34027264 / 34071040
 
 
 def gemv_roofline(dec, steps, warmup, hbm_peak):
@@ -288,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac_of_measured_copy": step_bytes / (ms / 1e3) / 1e9 / hbm_peak,
                 "frac_of_8tbs": step_bytes / (ms / 1e3) / 1e9 / 8000.0,
                 "pcie_bytes_per_step": staged_bytes(cfg, BATCH)},
-        "roofline": {**roof, "traffic": None},
+        "roofline": {**roof, "traffic": roof["bytes_per_launch"] * GEMV_TRAFFIC_PER_BYTE},
         "e2e": {"value": ms_e2e * 1e3 / tokens, "unit": UNIT,
                 "h2d_bytes_per_step": hidden.numel() * 2, "d2h_bytes_per_step": dec.logits.numel() * 4},
         "gpu_launches": (n_kernels * args.steps) if n_kernels else None,
@@ -373,13 +380,55 @@ def run_reference(args, rank, world):
             "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(name):
+    """A few launches of one hot kernel on a small case, for profiler captures
+    (no timing): `gemv` = the gate/up-shaped refined GEMV (28,672 x 4,096,
+    2 + 2 bits, k = 32 per 1,024), base then refined with a given selection,
+    three times; `kv` = score-select-attend over 8 KV heads x 32,768 tokens,
+    top-512, three times."""
+    import torch
+
+    from bit_decode_selective_b200 import inputs
+    from bit_decode_selective_b200.ops import KVCache, QuantWeights, select_channels
+
+    if name == "gemv":
+        w = inputs.torch_normal((28672, 4096), 0.02, 1)
+        qw = QuantWeights.pack(w, 2, 2, 128)
+        del w
+        x = inputs.torch_normal((1, 4096), 1.0, 2, dtype=torch.float16)
+        y = torch.empty(1, 28672, device="cuda")
+        sel = select_channels(x, 1024, 32)
+        for _ in range(3):
+            qw.gemv(x, 1024, 0, y=y)
+            qw.gemv(x, 1024, 32, y=y, sel_in=sel)
+    else:
+        t = 32768
+        k = inputs.torch_normal((1, 8, t, 128), 1.0, 3, dtype=torch.float16)
+        v = inputs.torch_normal((1, 8, t, 128), 1.0, 4, dtype=torch.float16)
+        c = KVCache(1, 8, t, 2, 2)
+        c.pack_tokens(k, v, 0)
+        del k, v
+        q = inputs.torch_normal((1, 32, 128), 1.0, 5, dtype=torch.float16)
+        out = torch.empty(1, 32, 128, device="cuda")
+        sel = torch.empty(1, 8, 512, dtype=torch.int32, device="cuda")
+        for _ in range(3):
+            c.attend_selective(q, t, 512, sel=sel, out=out)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": name, "ok": True}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", choices=["gemv", "kv"], default=None,
+                    help="run a few launches of one kernel for a profiler capture instead")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -261,61 +261,79 @@ __device__ __forceinline__ uint4 make_jd(const GemvParams& p, int b, int j) {
 // byte planes of all K/64 lane groups in shared memory, one warp per group
 
 template <int BITS>
-__device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ xs) {
+__device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ xs, int* __restrict__ scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ngrp = p.K / kLaneCh;
-  // the activations of all this warp's groups are loaded before any is used
-  constexpr int PRE = 16;
-  uint32_t xpre[PRE];
+  // UNR groups per warp at a time (independent shuffle chains interleave); the
+  // warp's scratch holds their 64 fixed-point values each, by (vector, byte)
+  constexpr int UNR = 4;
+  int* sw = scratch + warp * UNR * kLaneCh;
+  auto slot_of = [](int c) {
+    const int v = BITS == 4 ? 2 * (c >> 3) + (c & 1) : 4 * (c >> 4) + (c & 3);
+    const int L = BITS == 4 ? (c >> 1) & 3 : (c >> 2) & 3;
+    return 4 * v + L;
+  };
+  for (int g0 = warp; g0 < ngrp; g0 += UNR * kWarps) {
+    uint32_t xw[UNR];
 #pragma unroll
-  for (int k = 0; k < PRE; k++) {
-    const int grp = warp + k * kWarps;
-    xpre[k] = grp < ngrp ? __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane)
+    for (int u = 0; u < UNR; u++) {
+      const int grp = g0 + u * kWarps;
+      xw[u] = grp < ngrp ? __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane)
                          : 0u;
-  }
-  for (int grp = warp, k = 0; grp < ngrp; grp += kWarps, k++) {
-    uint32_t xw;
-    if (k < PRE) {
-#pragma unroll
-      for (int kk = 0; kk < PRE; kk++)
-        if (kk == k) xw = xpre[kk];
-    } else {
-      xw = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane);
     }
-    const float2 xv = __half22float2(*reinterpret_cast<const __half2*>(&xw));
-    float mx = fmaxf(fabsf(xv.x), fabsf(xv.y));
+    float2 xv[UNR];
+    float mx[UNR], sm[UNR];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const int e = mx > 0.f ? ilogbf(mx) - kXShift : 0;
-    const int xf0 = __float2int_rn(ldexpf(xv.x, -e)), xf1 = __float2int_rn(ldexpf(xv.y, -e));
-    // lane v < 16 assembles the plane words of code byte vector v
-    const int v = lane & 15;
-    uint32_t pl[kXP];
-#pragma unroll
-    for (int q = 0; q < kXP; q++) pl[q] = 0;
-#pragma unroll
-    for (int L = 0; L < 4; L++) {
-      const int c = chan_of<BITS>(v, L);
-      const int a0 = __shfl_sync(0xffffffffu, xf0, c >> 1), a1 = __shfl_sync(0xffffffffu, xf1, c >> 1);
-      const uint32_t f = (uint32_t)((c & 1) ? a1 : a0);
-#pragma unroll
-      for (int q = 0; q < kXP; q++) pl[q] |= ((f >> (8 * q)) & 0xffu) << (8 * L);
+    for (int u = 0; u < UNR; u++) {
+      xv[u] = __half22float2(*reinterpret_cast<const __half2*>(&xw[u]));
+      mx[u] = fmaxf(fabsf(xv[u].x), fabsf(xv[u].y));
+      sm[u] = xv[u].x + xv[u].y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
     }
-    uint32_t* dst = xs + grp * kXWords;
-    if (lane < 16) {
 #pragma unroll
-      for (int q = 0; q < kXP; q++) dst[kXP * v + q] = pl[q];
-    }
-    float sm = xv.x + xv.y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
+    for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-    const float s1 = __shfl_sync(0xffffffffu, sm, 16);
-    if (lane == 0) {
-      reinterpret_cast<float*>(dst)[kXR + 0] = sm;
-      reinterpret_cast<float*>(dst)[kXR + 1] = s1;
-      reinterpret_cast<float*>(dst)[kXR + 2] = ldexpf(1.0f, e);
-      reinterpret_cast<float*>(dst)[kXR + 3] = sm + s1;
+      for (int u = 0; u < UNR; u++) mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], o));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < UNR; u++) sm[u] += __shfl_xor_sync(0xffffffffu, sm[u], o);
+    int eb[UNR];
+    float s1[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; u++) {
+      // x_fix = x 2^-e with e = ilogb(max |x|) - kXShift; every nonzero fp16 value
+      // is a normal float, so the exponent and 2^-e come from the float bits (exact)
+      eb[u] = (__float_as_int(mx[u]) >> 23) & 0xff;  // biased exponent; 0 only for max 0
+      const float scale = eb[u] ? __int_as_float((254 + kXShift - eb[u]) << 23) : 0.f;
+      sw[u * kLaneCh + slot_of(2 * lane)] = __float2int_rn(xv[u].x * scale);
+      sw[u * kLaneCh + slot_of(2 * lane + 1)] = __float2int_rn(xv[u].y * scale);
+      s1[u] = __shfl_sync(0xffffffffu, sm[u], 16);
     }
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < UNR; u++) {
+      const int grp = g0 + u * kWarps;
+      if (grp < ngrp) {
+        uint32_t* dst = xs + grp * kXWords;
+        if (lane < 16) {  // lane v: plane q of vector v = byte q of its four values
+          const int4 f = reinterpret_cast<const int4*>(sw + u * kLaneCh)[lane];
+#pragma unroll
+          for (int q = 0; q < kXP; q++) {
+            const uint32_t sel = (uint32_t)q | ((uint32_t)(4 + q) << 4);
+            const uint32_t t01 = __byte_perm((uint32_t)f.x, (uint32_t)f.y, sel);
+            const uint32_t t23 = __byte_perm((uint32_t)f.z, (uint32_t)f.w, sel);
+            dst[kXP * lane + q] = __byte_perm(t01, t23, 0x5410);
+          }
+        }
+        if (lane == 0) {  // lane 0 holds the first half's sum, s1 the second's
+          reinterpret_cast<float*>(dst)[kXR + 0] = sm[u];
+          reinterpret_cast<float*>(dst)[kXR + 1] = s1[u];
+          reinterpret_cast<float*>(dst)[kXR + 2] = eb[u] ? __int_as_float((eb[u] - kXShift) << 23) : 1.0f;
+          reinterpret_cast<float*>(dst)[kXR + 3] = sm[u] + s1[u];
+        }
+      }
+    }
+    __syncwarp();  // the scratch is rewritten by the next groups
   }
 }
 
@@ -437,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   const int ngrp = p.K / kLaneCh, gpr = p.K >> p.gshift;
   // shared memory: partial sums [rows][segs] | rings | (fast) table, words, scales
   float* part = reinterpret_cast<float*>(smem);
-  uint32_t* xs = smem + ((p.rows_max * p.segs + 3) & ~3);  // activation planes [K/64][kXWords]
+  uint32_t* xs = smem + ((p.rows_max * p.segs + 3) & ~3);  // activation planes [K/64][kXWords], prologue scratch
   uint32_t* area = xs + p.plane_words;
   uint4* jd_fast = reinterpret_cast<uint4*>(area + p.area_words);
   uint32_t* wt_fast = reinterpret_cast<uint32_t*>(jd_fast + p.n_sel);
@@ -475,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
 #pragma unroll
       for (int i = 0; i < PD - 1; i++) issue();
       if (b == 0) pdl_wait();  // x, the selection and the staged rows are complete
-      prep_planes<BITS>(p, b, xs);
+      prep_planes<BITS>(p, b, xs, reinterpret_cast<int*>(xs + ngrp * kXWords));
       if (p.fast && p.n_sel > 0) corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
       __syncthreads();  // planes complete
       uint32_t xr[kXR];
@@ -665,7 +683,7 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.rows_max = ((units + grid - 1) / grid) * kRowUnit;
   p.w_span = p.rows_max * w->r / 32 + 2;
   p.corr_rows = pick_corr_rows(p.rows_max);
-  p.plane_words = mode == 0 ? (w->k / kLaneCh) * kXWords : 0;
+  p.plane_words = mode == 0 ? (w->k / kLaneCh) * kXWords + kWarps * 4 * kLaneCh : 0;  // planes, then per-warp scratch
   const size_t gpr = (size_t)(w->k / w->group);
   const size_t part_words = ((size_t)p.rows_max * p.segs + 3) & ~(size_t)3;
   const size_t table_words = (size_t)n_sel * 4 + (((size_t)n_sel * p.w_span + 3) & ~(size_t)3) +

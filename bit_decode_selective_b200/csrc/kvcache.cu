@@ -41,14 +41,27 @@ __device__ __forceinline__ void group_minmax(const double (&v)[4], int d0, doubl
 // 4l .. 4l+3 (group l / 8).  The token's code words (keys) or 16-bit word
 // halves (values) are assembled in shared memory and stored by the first
 // lanes; a token owns all of them, so tokens never share a store.
+// Keys and values of the same tokens in one launch: blockIdx.y picks the kind.
+struct PackArgs {
+  const uint16_t* x[2];  // [BH][nt][128] fp16 keys, values (either may be null)
+  uint32_t* codes[2];
+  uint32_t* refine[2];
+  uint16_t* sz[2];
+  int BH, nt, t_max, t0, first_kind;
+};
+
 template <int B, int R>
-__global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(
-    const uint16_t* __restrict__ x, int BH, int nt, int t_max, int t0, int is_value,
-    uint32_t* __restrict__ codes, uint32_t* __restrict__ refine, uint16_t* __restrict__ sz) {
+__global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
   // keys: 4B code words + 4R refinement words; values: 8B + 8R halves
   __shared__ uint32_t acc[kPackWarps][8 * (B + R)];
   pdl_trigger();
   pdl_wait();
+  const int is_value = pa.first_kind + blockIdx.y;
+  const uint16_t* __restrict__ x = pa.x[is_value];
+  uint32_t* __restrict__ codes = pa.codes[is_value];
+  uint32_t* __restrict__ refine = pa.refine[is_value];
+  uint16_t* __restrict__ sz = pa.sz[is_value];
+  const int BH = pa.BH, nt = pa.nt, t_max = pa.t_max, t0 = pa.t0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long idx = (long)blockIdx.x * kPackWarps + warp;
   if (idx >= (long)BH * nt) return;  // whole warps only
@@ -139,25 +152,27 @@ __global__ void unpack_kv_kernel(const uint32_t* __restrict__ codes,
 }
 
 template <int B, int R>
-sf_status launch_pack(const uint16_t* x, int BH, int nt, int t_max, int t0, int is_value,
-                      void* codes, void* refine, uint16_t* sz, cudaStream_t s) {
-  const long total = (long)BH * nt;
-  SF_CUDA(launch_pdl(pack_kv_kernel<B, R>, dim3((unsigned)((total + kPackWarps - 1) / kPackWarps)),
-                     dim3(kPackWarps * 32), 0, s, x, BH, nt, t_max, t0, is_value, (uint32_t*)codes,
-                     (uint32_t*)refine, sz));
+sf_status launch_pack(const PackArgs& pa, int kinds, cudaStream_t s) {
+  const long total = (long)pa.BH * pa.nt;
+  SF_CUDA(launch_pdl(pack_kv_kernel<B, R>, dim3((unsigned)((total + kPackWarps - 1) / kPackWarps), kinds),
+                     dim3(kPackWarps * 32), 0, s, pa));
   return SF_OK;
 }
 
-sf_status pack_one(const sf_kv* kv, const uint16_t* x, int t0, int nt, int is_value,
-                   cudaStream_t s) {
-  int BH = kv->batch * kv->h_kv;
-  void* codes = is_value ? kv->vb : kv->kb;
-  void* refine = is_value ? kv->vr : kv->kr;
-  uint16_t* sz = is_value ? kv->vsz : kv->ksz;
-  if (kv->b == 2 && kv->r == 2) return launch_pack<2, 2>(x, BH, nt, kv->t_max, t0, is_value, codes, refine, sz, s);
-  if (kv->b == 2 && kv->r == 1) return launch_pack<2, 1>(x, BH, nt, kv->t_max, t0, is_value, codes, refine, sz, s);
-  if (kv->b == 4 && kv->r == 2) return launch_pack<4, 2>(x, BH, nt, kv->t_max, t0, is_value, codes, refine, sz, s);
-  return launch_pack<4, 1>(x, BH, nt, kv->t_max, t0, is_value, codes, refine, sz, s);
+sf_status pack_both(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0, int nt, cudaStream_t s) {
+  PackArgs pa;
+  pa.x[0] = k, pa.x[1] = v;
+  pa.codes[0] = (uint32_t*)kv->kb, pa.codes[1] = (uint32_t*)kv->vb;
+  pa.refine[0] = (uint32_t*)kv->kr, pa.refine[1] = (uint32_t*)kv->vr;
+  pa.sz[0] = kv->ksz, pa.sz[1] = kv->vsz;
+  pa.BH = kv->batch * kv->h_kv, pa.nt = nt, pa.t_max = kv->t_max, pa.t0 = t0;
+  pa.first_kind = k ? 0 : 1;
+  const int kinds = (k ? 1 : 0) + (v ? 1 : 0);
+  if (kinds == 0) return SF_OK;
+  if (kv->b == 2 && kv->r == 2) return launch_pack<2, 2>(pa, kinds, s);
+  if (kv->b == 2 && kv->r == 1) return launch_pack<2, 1>(pa, kinds, s);
+  if (kv->b == 4 && kv->r == 2) return launch_pack<4, 2>(pa, kinds, s);
+  return launch_pack<4, 1>(pa, kinds, s);
 }
 
 }  // namespace
@@ -174,16 +189,7 @@ extern "C" sf_status sf_kv_pack_tokens(const sf_kv* kv, const uint16_t* k, const
   SF_REQUIRE(!k || aligned16(k), "k must be 16-byte aligned");
   SF_REQUIRE(!v || aligned16(v), "v must be 16-byte aligned");
   if (nt == 0) return SF_OK;
-  cudaStream_t s = as_stream(stream);
-  if (k) {
-    st = pack_one(kv, k, t0, nt, 0, s);
-    if (st != SF_OK) return st;
-  }
-  if (v) {
-    st = pack_one(kv, v, t0, nt, 1, s);
-    if (st != SF_OK) return st;
-  }
-  return SF_OK;
+  return pack_both(kv, k, v, t0, nt, as_stream(stream));
 }
 
 extern "C" sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* qb,
