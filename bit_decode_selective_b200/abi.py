@@ -49,6 +49,8 @@ _SIGNATURES = {
     "sf_gemv_workspace_bytes": ([POINTER(sf_wq), c_int, c_int, c_int], c_size_t),
     "sf_gemv_correction": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                             c_void_p, c_void_p], c_int),
+    "sf_gemv_refined_split": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p], c_int),
     "sf_kv_bytes": ([c_int] * 7 + [POINTER(c_size_t)] * 3, c_int),
     "sf_kv_pack_tokens": ([POINTER(sf_kv), c_void_p, c_void_p, c_int, c_int, c_void_p], c_int),
     "sf_kv_unpack_codes": ([POINTER(sf_kv), c_int, c_int, c_void_p, c_void_p, c_void_p], c_int),
@@ -124,6 +126,7 @@ sf_select_channels = _call("sf_select_channels")
 sf_gemv_refined = _call("sf_gemv_refined")
 sf_gemv_workspace_bytes = _call("sf_gemv_workspace_bytes")
 sf_gemv_correction = _call("sf_gemv_correction")
+sf_gemv_refined_split = _call("sf_gemv_refined_split")
 sf_kv_bytes = _call("sf_kv_bytes")
 sf_kv_pack_tokens = _call("sf_kv_pack_tokens")
 sf_kv_unpack_codes = _call("sf_kv_unpack_codes")

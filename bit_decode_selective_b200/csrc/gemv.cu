@@ -77,6 +77,9 @@ struct GemvParams {
   int fast;              // correction tables in their own shared region, filled before the base pass
   int w_span;            // stride of the refinement-word table (words a CTA's rows can span)
   int corr_rows;         // rows per lane in the correction (1, 2 or 4)
+  int corr_split;        // fast path: the warps' correction partials go to the free ring area
+  int pstride;           // row stride of the partial sums: segs base columns, then the correction
+  float* y_corr;         // non-null: the correction goes here ([batch][N]) and y gets the base only
 };
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -358,20 +361,31 @@ __device__ void corr_fill(const GemvParams& p, int b, int j0, int jn, int w_lo, 
   cp_async_commit();
 }
 
-// Adds the correction of table entries [0, jn) into part[row][0].  Lanes own
-// RL consecutive rows (inside one refinement word); warps split the entries.
+// Warp tasks of the correction: row blocks of 32 lanes x RL rows, times
+// splits of the table entries.
+__device__ __forceinline__ void corr_tasks(int rows, int RL, int& nblk, int& js_n) {
+  nblk = (rows / RL + 31) / 32;
+  js_n = nblk >= kWarps ? 1 : kWarps / nblk;
+}
+
+// The correction of table entries [0, jn): into cpart[js][row] (entry split
+// js, stride rows_max; every row of every split written), or added into
+// the correction column part[row][segs] when cpart is NULL.  Lanes own RL consecutive rows (inside one
+// refinement word); warps split the entries.
 // Entries come in ascending channel order, so channels of one scale group are
 // consecutive: each run is summed unscaled and multiplied by s once.  szt:
-// the CTA's (s, m) words [rows][gpr], or NULL (scales read from global).
+// the CTA's (s, m) words group-major, [gpr][rows_max], so that the lanes of a
+// warp (consecutive rows) read consecutive words; or NULL (scales read from
+// global memory).
 template <int RL>
 __device__ void corr_process(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
                              const uint4* __restrict__ jd, const uint32_t* __restrict__ wt,
-                             const uint32_t* __restrict__ szt, float* part) {
+                             const uint32_t* __restrict__ szt, float* part, float* cpart) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gpr = p.K >> p.gshift;
   const int units = rows / RL;
-  const int nblk = (units + 31) / 32;
-  const int js_n = nblk >= kWarps ? 1 : kWarps / nblk;
+  int nblk, js_n;
+  corr_tasks(rows, RL, nblk, js_n);
   const int ntasks = nblk * js_n;
   const int r = p.r;
   const uint32_t fmask = ((1u << r) - 1u) << (23 - r);
@@ -393,9 +407,23 @@ __device__ void corr_process(const GemvParams& p, int n0, int rows, int w_lo, in
     int gcur = -1;
     auto flush = [&]() {
       if (gcur >= 0 && ok) {
+        // the lane's RL rows of group gcur are consecutive words of szt
+        uint32_t zt[RL];
+        if (szt) {
+          const uint32_t* zp = szt + gcur * p.rows_max + rl0;
+          if constexpr (RL == 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(zp);
+            zt[0] = v.x, zt[1] = v.y, zt[2] = v.z, zt[3] = v.w;
+          } else if constexpr (RL == 2) {
+            const uint2 v = *reinterpret_cast<const uint2*>(zp);
+            zt[0] = v.x, zt[1] = v.y;
+          } else {
+            zt[0] = zp[0];
+          }
+        }
 #pragma unroll
         for (int t = 0; t < RL; t++) {
-          const uint32_t zw = szt ? szt[(rl0 + t) * gpr + gcur]
+          const uint32_t zw = szt ? zt[t]
                                   : __ldg(reinterpret_cast<const uint32_t*>(p.sz) + (size_t)(n0 + rl0 + t) * gpr + gcur);
           const float sc = __low2float(*reinterpret_cast<const __half2*>(&zw));
           acc[t] = fmaf(sc, run[t] - C, acc[t]);
@@ -420,22 +448,25 @@ __device__ void corr_process(const GemvParams& p, int n0, int rows, int w_lo, in
       C += __uint_as_float(d.y);
     }
     flush();
-    if (ok && ib > ia) {
+    if (ok && cpart) {
 #pragma unroll
-      for (int t = 0; t < RL; t++) atomicAdd(&part[(rl0 + t) * p.segs], acc[t]);
+      for (int t = 0; t < RL; t++) cpart[js * p.rows_max + rl0 + t] = acc[t];
+    } else if (ok && ib > ia) {
+#pragma unroll
+      for (int t = 0; t < RL; t++) atomicAdd(&part[(rl0 + t) * p.pstride + p.segs], acc[t]);
     }
   }
 }
 
 __device__ __forceinline__ void corr_dispatch(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
                                               const uint4* jd, const uint32_t* wt, const uint32_t* szt,
-                                              float* part) {
+                                              float* part, float* cpart) {
   if (p.corr_rows == 4)
-    corr_process<4>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
+    corr_process<4>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
   else if (p.corr_rows == 2)
-    corr_process<2>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
+    corr_process<2>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
   else
-    corr_process<1>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part);
+    corr_process<1>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
 }
 
 // ---------------------------------------------------------------------------
@@ -455,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   const int ngrp = p.K / kLaneCh, gpr = p.K >> p.gshift;
   // shared memory: partial sums [rows][segs] | rings | (fast) table, words, scales
   float* part = reinterpret_cast<float*>(smem);
-  uint32_t* xs = smem + ((p.rows_max * p.segs + 3) & ~3);  // activation planes [K/64][kXWords], prologue scratch
+  uint32_t* xs = smem + ((p.rows_max * p.pstride + 3) & ~3);  // activation planes [K/64][kXWords], prologue scratch
   uint32_t* area = xs + p.plane_words;
   uint4* jd_fast = reinterpret_cast<uint4*>(area + p.area_words);
   uint32_t* wt_fast = reinterpret_cast<uint32_t*>(jd_fast + p.n_sel);
@@ -466,6 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
   const int ta = (int)((long)warp * ntask / kWarps), tb = (int)((long)(warp + 1) * ntask / kWarps);
   const size_t row_bytes = (size_t)p.K * (BITS == 3 ? 2 : BITS) / 8;
   const bool fill_szt = p.fast && p.mode == 0 && p.n_sel > 0;
+  // the fast correction's per-warp partials: in the ring area, free once the base pass is done
+  float* cpart = p.corr_split && p.fast && p.n_sel > 0 ? reinterpret_cast<float*>(area) : nullptr;
 
   for (int b = 0; b < p.batch; b++) {
     if (p.mode == 0) {
@@ -493,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
 #pragma unroll
       for (int i = 0; i < PD - 1; i++) issue();
       if (b == 0) pdl_wait();  // x, the selection and the staged rows are complete
+      for (int i = threadIdx.x; i < rows; i += kThreads) part[i * p.pstride + p.segs] = 0.f;  // correction column
       prep_planes<BITS>(p, b, xs, reinterpret_cast<int*>(xs + ngrp * kXWords));
       if (p.fast && p.n_sel > 0) corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
       __syncthreads();  // planes complete
@@ -546,30 +580,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
             const float2 sm0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
             if constexpr (ZW == 1) {
               acc[u] = fmaf(sm0.x * xscale, (float)d[0], sm0.y * xsum0);
-              if (zown) szt[(r0 + u - n0) * gpr + zg] = z0;
+              if (zown) szt[zg * p.rows_max + (r0 + u - n0)] = z0;
             } else {
               const uint32_t z1 = slot[R::z_off + (u * ZW + 1) * 32 + lane];
               const float2 sm1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
               acc[u] = fmaf(sm0.x * xscale, (float)d[0],
                             fmaf(sm1.x * xscale, (float)d[1], fmaf(sm0.y, xsum0, sm1.y * xsum1)));
-              if (fill_szt && la) szt[(r0 + u - n0) * gpr + zg] = z0, szt[(r0 + u - n0) * gpr + zg + 1] = z1;
+              if (fill_szt && la) szt[zg * p.rows_max + (r0 + u - n0)] = z0, szt[(zg + 1) * p.rows_max + (r0 + u - n0)] = z1;
             }
           }
         }
         const float tot = warp_sum_rows<U>(acc, lane);
         const int u = U == 4 ? (lane >> 3) : (lane >> 4);
-        if ((lane & (32 / U - 1)) == 0) part[(r0 + u - n0) * p.segs + cseg] = tot;
+        if ((lane & (32 / U - 1)) == 0) part[(r0 + u - n0) * p.pstride + cseg] = tot;
         if (++cst == steps) cst = 0, ++cseg;
         cslot = cslot + 1 == PD ? 0 : cslot + 1;
       }
       cp_async_wait<0>();
     } else {
-      for (int i = threadIdx.x; i < rows * p.segs; i += kThreads) part[i] = 0.f;
+      for (int i = threadIdx.x; i < rows * p.pstride; i += kThreads) part[i] = 0.f;
       if (b == 0) pdl_wait();  // x, the selection, the staged rows and y are complete
       if (p.fast) {
-        // the CTA's (s, m) words are one contiguous block of sz
+        // the CTA's (s, m) words are one contiguous block of sz, [rows][gpr];
+        // they are stored transposed
         const uint32_t* zsrc = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)n0 * gpr;
-        for (int i = threadIdx.x; i < rows * gpr / 4; i += kThreads) cp_async16(szt + 4 * i, zsrc + 4 * i);
+        for (int i = threadIdx.x; i < rows * gpr; i += kThreads) {
+          const int row = i / gpr, g = i - row * gpr;
+          cp_async4(szt + g * p.rows_max + row, zsrc + i);
+        }
         corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
         cp_async_wait<0>();
       }
@@ -579,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
     // ---- correction of the selected channels of batch row b
     if (p.n_sel > 0) {
       if (p.fast) {
-        corr_dispatch(p, n0, rows, w_lo, nwr, p.n_sel, jd_fast, wt_fast, szt, part);
+        corr_dispatch(p, n0, rows, w_lo, nwr, p.n_sel, jd_fast, wt_fast, szt, part, cpart);
       } else {
         // tables in chunks in the ring area; scales from global memory
         const int jcap = p.area_words / (4 + nwr);
@@ -590,18 +628,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
           corr_fill(p, b, j0, jn, w_lo, nwr, jd, wt);
           cp_async_wait<0>();
           __syncthreads();
-          corr_dispatch(p, n0, rows, w_lo, nwr, jn, jd, wt, nullptr, part);
+          corr_dispatch(p, n0, rows, w_lo, nwr, jn, jd, wt, nullptr, part, nullptr);
           __syncthreads();
         }
       }
     }
     __syncthreads();
 
+    int cjs = 0;  // entry splits of the correction partials in cpart
+    if (cpart) {
+      int nblk;
+      corr_tasks(rows, p.corr_rows, nblk, cjs);
+    }
     for (int row = n0 + threadIdx.x; row < n1; row += kThreads) {
-      float acc = 0.f;
-      for (int s = 0; s < p.segs; s++) acc += part[(row - n0) * p.segs + s];
+      const float* pr = part + (row - n0) * p.pstride;
+      float base = 0.f, corr = pr[p.segs];
+      for (int s = 0; s < p.segs; s++) base += pr[s];
+      for (int js = 0; js < cjs; js++) corr += cpart[js * p.rows_max + row - n0];
       float* dst = p.y + (size_t)b * p.N + row;
-      *dst = p.mode == 1 ? *dst + acc : acc;
+      if (p.y_corr) {
+        *dst = base;
+        p.y_corr[(size_t)b * p.N + row] = corr;
+      } else {
+        *dst = p.mode == 1 ? *dst + corr : base + corr;
+      }
     }
     __syncthreads();
   }
@@ -638,7 +688,7 @@ int pick_corr_rows(int rows) {
 
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                       const int32_t* sel_in, int32_t* sel_out, const void* refine_rows, float* y,
-                      int mode, cudaStream_t s) {
+                      int mode, cudaStream_t s, float* y_corr = nullptr) {
   sf_status st = check_wq_public(w, false);
   if (st != SF_OK) return st;
   SF_REQUIRE(x && aligned16(x), "x must be a non-null 16-byte aligned device pointer");
@@ -668,6 +718,7 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.sz = w->sz;
   p.x = x;
   p.y = y;
+  p.y_corr = y_corr;
   p.N = w->n, p.K = w->k, p.G = w->group, p.r = w->r, p.batch = batch, p.n_sel = n_sel;
   p.gshift = 0;
   while ((1 << p.gshift) < w->group) p.gshift++;
@@ -685,7 +736,8 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.corr_rows = pick_corr_rows(p.rows_max);
   p.plane_words = mode == 0 ? (w->k / kLaneCh) * kXWords + kWarps * 4 * kLaneCh : 0;  // planes, then per-warp scratch
   const size_t gpr = (size_t)(w->k / w->group);
-  const size_t part_words = ((size_t)p.rows_max * p.segs + 3) & ~(size_t)3;
+  p.pstride = p.segs + 1;
+  const size_t part_words = ((size_t)p.rows_max * p.pstride + 3) & ~(size_t)3;
   const size_t table_words = (size_t)n_sel * 4 + (((size_t)n_sel * p.w_span + 3) & ~(size_t)3) +
                              (size_t)p.rows_max * gpr;
   const size_t limit_words = kSmemLimit / 4;
@@ -705,10 +757,16 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
     }
     SF_UNSUPPORTED(pd > 0, "n=%d, k=%d does not fit in shared memory", w->n, w->k);
   } else {
-    p.fast = fixed + 4 + table_words <= limit_words;
-    area = p.fast ? 4 : limit_words - fixed;
+    const size_t split_words = (size_t)kWarps * p.rows_max;
+    if (fixed + split_words + table_words <= limit_words) {
+      p.fast = 1, area = split_words;
+    } else {
+      p.fast = fixed + 4 + table_words <= limit_words;
+      area = p.fast ? 4 : limit_words - fixed;
+    }
     pd = 2;
   }
+  p.corr_split = p.fast && area >= (size_t)kWarps * p.rows_max;
   if (!p.fast && n_sel > 0)
     SF_UNSUPPORTED(area >= (size_t)(4 + p.w_span) * 16, "n=%d, k=%d: no room for the correction", w->n, w->k);
   const size_t smem = (fixed + area + (p.fast ? table_words : 0)) * 4;
@@ -770,4 +828,17 @@ extern "C" sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int b
                                         float* y, sf_stream_t stream) {
   SF_REQUIRE(kch == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
   return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, 1, as_stream(stream));
+}
+
+extern "C" sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, int batch, int chunk,
+                                           int kch, const int32_t* sel_in, const void* refine_rows,
+                                           float* y_base, float* y_corr, sf_stream_t stream) {
+  SF_REQUIRE(kch >= 1, "kch=%d: the split form needs a correction (kch >= 1)", kch);
+  SF_REQUIRE(sel_in && aligned16(sel_in), "sel_in must be non-null and 16-byte aligned");
+  SF_REQUIRE(y_corr && aligned16(y_corr), "y_corr must be a non-null 16-byte aligned device pointer");
+  SF_REQUIRE(w && batch >= 1, "null weights or batch < 1");
+  const size_t bytes = (size_t)batch * (size_t)w->n * sizeof(float);
+  const char *a0 = (const char*)y_base, *b0 = (const char*)y_corr;
+  SF_REQUIRE(!y_base || a0 + bytes <= b0 || b0 + bytes <= a0, "y_base and y_corr overlap");
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, nullptr, refine_rows, y_base, 0, as_stream(stream), y_corr);
 }

@@ -32,6 +32,7 @@
 // tokens, up to fp32 rounding.
 #include <cooperative_groups.h>
 
+#include <algorithm>
 #include <cfloat>
 #include <mutex>
 
@@ -503,6 +504,10 @@ constexpr int kPostCl = 8;
 constexpr int kPostStage = 64;      // selected tokens staged in shared memory at a time
 constexpr int kPostMaxSel = 512;    // selected tokens per CTA (k_tok <= 4096)
 constexpr int kHistBins = 512;
+// a warp's share of one staging batch, times 8 query heads, fits its 32 lanes
+static_assert(kPostStage / (kPostThreads / 32) * 8 <= 32, "staging batch too large for the lane layout");
+// the per-warp partial numerators reuse the score keys' space
+static_assert((kPostThreads / 32) * 8 * kD <= kPostMaxTok, "key space too small for the partial numerators");
 
 struct PostArgs {
   const uint8_t *kb, *kr, *vb, *vr;
@@ -529,8 +534,8 @@ struct PostShared {
   int cnt;
   int digit, kleft, done;
   float M[8], Z[8];
-  float dnum[8][kD];  // this CTA's correction of the numerators, then its partial numerators
-  float dden[8];      // this CTA's correction of the denominators
+  float wden[kPostThreads / 32][8];      // per warp: its tokens' change of each head's denominator
+  float wtab[kPostThreads / 32][2 * 32];  // per warp: (w_refined, w_base) of its (token, head) slots
 };
 
 // Filled by the peers (distributed shared memory stores, which do not stall the
@@ -546,6 +551,26 @@ struct PostMail {
 // Words of one staged token: K codes (4b), K refinement (4r), K and V (s, m)
 // (4 + 4), the token's 8 value chunks of codes (8 x 2b) and refinement (8 x 2r).
 __host__ __device__ constexpr int tok_words(int b, int r) { return 20 * (b + r) + 8; }
+
+// Sums each of the N (16 or 32) per-lane values v over the warp; returns the
+// sum of value lane % N.  Each round keeps the half of the values that the
+// lane's bit selects and adds the partner's copy of it.
+template <int N>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
+  static_assert(N == 16 || N == 32, "16 or 32 values");
+#pragma unroll
+  for (int n = N, o = N / 2; n > 1; n >>= 1, o >>= 1) {
+    const bool up = lane & o;
+#pragma unroll
+    for (int j = 0; j < n / 2; j++) {
+      const float keep = up ? v[j + n / 2] : v[j], send = up ? v[j] : v[j + n / 2];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float r = v[0];
+  if constexpr (N == 16) r += __shfl_xor_sync(0xffffffffu, r, 16);
+  return r;
+}
 
 // GQP: query heads per KV head, padded to 4 or 8 (register arrays); B, R:
 // the cache's base and refinement bits.
@@ -565,8 +590,6 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
   const int gq = a.gq;
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
   pdl_trigger();
-  for (int i = tid; i < 8 * kD; i += kPostThreads) (&sh.dnum[0][0])[i] = 0.f;
-  if (tid < 8) sh.dden[tid] = 0.f;
   // every CTA of the cluster must have started before peers touch its shared
   // memory: arrive now, wait right before the first distributed access
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -790,13 +813,12 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
 #pragma unroll
       for (int h = 0; h < GQP; h++) qv[h][e] = h < gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
     }
-    float an[GQP][4], ad[GQP];
+    constexpr int TPW = kPostStage / NW;  // tokens of a staging batch per warp
+    float an[GQP][4], ad_own = 0.f;
 #pragma unroll
-    for (int h = 0; h < GQP; h++) {
-      ad[h] = 0.f;
+    for (int h = 0; h < GQP; h++)
 #pragma unroll
       for (int e = 0; e < 4; e++) an[h][e] = 0.f;
-    }
     // pieces of one staged token: 16-byte copies (8-byte for 1-bit value refinement chunks)
     const int pk = B, pkr = R, pv = 8 * (B >= 2 ? B / 2 : 1), pvr = 8 * (R >= 2 ? R / 2 : 1);
     const int npiece = pk + pkr + 2 + pv + pvr;
@@ -836,15 +858,25 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
         }
       }
       cp_async_commit();
+      // while the copies fly: the base weights exp(l_base - M) of the warp's
+      // tokens; lane L holds slot u = L % (TPW GQP), i.e. token i = warp + NW
+      // (u / GQP), head u % GQP (the slot the transposed reduction below
+      // leaves in lane L)
+      float wbl = 0.f;
+      const int u_own = lane % (TPW * GQP), m_own = u_own / GQP, h_own = u_own % GQP;
+      const bool own_ok = h_own < gq && warp + NW * m_own < nt;
+      if (own_ok)
+        wbl = __expf(a.logits[(hq0 + h_own) * a.T + mail.tok[j0 - ja + warp + NW * m_own]] - sh.M[h_own]);
       cp_async_wait<0>();
       __syncthreads();
-      for (int i = warp; i < nt; i += NW) {
-        const uint32_t* st = stage + i * W;
-        const int t = mail.tok[j0 - ja + i];
-        const int tt = t & 15;
-        float kf[4], vbs[4], vfs[4], lg[GQP], lb[GQP];
+      // the warp's TPW tokens together: refined keys, base and refined values
+      float kf[TPW][4], vbs[TPW][4], vfs[TPW][4];
 #pragma unroll
-        for (int h = 0; h < GQP; h++) lb[h] = h < gq ? a.logits[(hq0 + h) * a.T + t] : 0.f;
+      for (int m = 0; m < TPW; m++) {
+        const int i = warp + NW * m;
+        const bool ok = i < nt;
+        const uint32_t* st = stage + (ok ? i : 0) * W;
+        const int tt = ok ? (mail.tok[j0 - ja + i] & 15) : 0;
 #pragma unroll
         for (int e = 0; e < 4; e++) {
           const int d = lane + 32 * e;
@@ -859,50 +891,65 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
           const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv));
           const uint32_t qk = (st[oK + kw[e]] >> kbit[e]) & bmask, rk = (st[oKr + krw[e]] >> krbit[e]) & rmask;
           const uint32_t qq = (st[oV + vwl] >> vbit) & bmask, rv = (st[oVr + vrwl] >> vrbit) & rmask;
-          kf[e] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
-          vbs[e] = fmaf(v2.x, (float)qq, v2.y);
-          vfs[e] = fmaf(v2.x, (float)qq + ((float)rv + 0.5f - half) * inv, v2.y);
+          kf[m][e] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
+          vbs[m][e] = ok ? fmaf(v2.x, (float)qq, v2.y) : 0.f;
+          vfs[m][e] = ok ? fmaf(v2.x, (float)qq + ((float)rv + 0.5f - half) * inv, v2.y) : 0.f;
         }
+      }
+      // refined logits of the TPW x GQP (token, head) slots: per-lane partial
+      // dot products, summed over the warp by a transposed butterfly that
+      // leaves slot lane % (TPW GQP) in each lane
+      float lg[TPW * GQP];
+#pragma unroll
+      for (int m = 0; m < TPW; m++)
 #pragma unroll
         for (int h = 0; h < GQP; h++) {
           float acc = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[e], acc);
-          lg[h] = acc;
+          for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[m][e], acc);
+          lg[m * GQP + h] = acc;
         }
+      const float lg_own = warp_transpose_sum<TPW * GQP>(lg, lane);
+      float wfl = 0.f;
+      if (own_ok) wfl = __expf(lg_own * a.scale - sh.M[h_own]);
+      // every lane needs every slot's (w_refined, w_base): through the warp's table
+      float2* wtab = reinterpret_cast<float2*>(&sh.wtab[warp][0]);
+      if (lane < TPW * GQP) wtab[lane] = make_float2(wfl, wbl);
+      ad_own += wfl - wbl;
+      __syncwarp();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int h = 0; h < GQP; h++)
-            if (h < gq) lg[h] += __shfl_xor_sync(0xffffffffu, lg[h], o);
+      for (int m = 0; m < TPW; m++)
 #pragma unroll
         for (int h = 0; h < GQP; h++) {
-          if (h < gq) {
-            const float wf = __expf(lg[h] * a.scale - sh.M[h]), wb = __expf(lb[h] - sh.M[h]);
+          const float2 w = wtab[m * GQP + h];
 #pragma unroll
-            for (int e = 0; e < 4; e++) an[h][e] = fmaf(wf, vfs[e], fmaf(-wb, vbs[e], an[h][e]));
-            ad[h] += wf - wb;
-          }
+          for (int e = 0; e < 4; e++) an[h][e] = fmaf(w.x, vfs[m][e], fmaf(-w.y, vbs[m][e], an[h][e]));
         }
-      }
+      __syncwarp();
     }
-    if (ja + warp < jb) {
+    // per-warp partial numerators and denominators (the score keys are no
+    // longer needed: their space holds them), summed in the merge below
+    float* wnum = reinterpret_cast<float*>(keys);
 #pragma unroll
-      for (int h = 0; h < GQP; h++) {
-        if (h < gq) {
+    for (int h = 0; h < GQP; h++)
+      if (h < gq) {
 #pragma unroll
-          for (int e = 0; e < 4; e++) atomicAdd(&sh.dnum[h][lane + 32 * e], an[h][e]);
-          if (lane == 0) atomicAdd(&sh.dden[h], ad[h]);
-        }
+        for (int e = 0; e < 4; e++) wnum[(warp * GQP + h) * kD + lane + 32 * e] = an[h][e];
       }
-    }
+    // slot u's denominator change sits in lanes u, u + TPW GQP, ...; sum over
+    // the TPW tokens of each head
+    float dsum = lane < TPW * GQP ? ad_own : 0.f;
+#pragma unroll
+    for (int o = GQP; o < 32; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    if (lane < gq) sh.wden[warp][lane] = dsum;
   }
   __syncthreads();
   // this CTA's share of the base records: records s = cr, cr + CL, ... (loads batched)
   for (int e = tid; e < gq * kD; e += kPostThreads) {
     const int hh = e / kD, d = e % kD;
     const float* pr = a.part + (hq0 + hh) * a.nrec * a.rec;
-    float num = sh.dnum[hh][d];
+    float num = 0.f;  // the correction: every warp's partial
+    for (int w = 0; w < NW; w++) num += reinterpret_cast<const float*>(keys)[(w * GQP + hh) * kD + d];
     constexpr int PER = 8;
     for (int s0 = cr; s0 < a.nrec; s0 += CL * PER) {
       float mv[PER], av[PER];
@@ -918,7 +965,11 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
     }
     cluster.map_shared_rank(&mail.num[cr][0], hh)[d] = num;  // to the CTA that merges head hh
   }
-  if (tid < gq) cluster.map_shared_rank(&mail.den[cr], tid)[0] = sh.dden[tid];
+  if (tid < gq) {
+    float den = 0.f;
+    for (int w = 0; w < NW; w++) den += sh.wden[w][tid];
+    cluster.map_shared_rank(&mail.den[cr], tid)[0] = den;
+  }
   cluster.sync();  // every partial numerator is in its head's mailbox
   if (cr < gq) {
     for (int d = tid; d < kD; d += kPostThreads) {
@@ -1033,7 +1084,11 @@ sf_status launch_post(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_
   a.k_tok = k_tok, a.sel = sel, a.select = select, a.scores = scores, a.out = out;
   a.chunk = P.chunk;
   a.scale = 1.0f / sqrtf((float)kD);
-  const size_t smem = sizeof(PostMail) + ((size_t)kPostStage * tok_words(kv->b, kv->r) + P.chunk) * 4;
+  // the score keys' space, which later holds the per-warp partial numerators
+  // of the refined attention [warps][GQP][kD]
+  const size_t gqp = a.gq <= 4 ? 4 : 8;
+  const size_t key_words = out ? std::max((size_t)P.chunk, (size_t)(kPostThreads / 32) * gqp * kD) : (size_t)P.chunk;
+  const size_t smem = sizeof(PostMail) + ((size_t)kPostStage * tok_words(kv->b, kv->r) + key_words) * 4;
   void (*kern)(PostArgs);
   if (a.gq <= 4)
     kern = kv->b == 2 ? (kv->r == 2 ? kv_post_kernel<4, 2, 2> : kv_post_kernel<4, 2, 1>)

@@ -84,6 +84,22 @@ class QuantWeights:
         return y
 
 
+    def gemv_split(self, x: torch.Tensor, sel, chunk: int = 1024, kch: int = 32, refine_rows=None,
+                   y_base=None, y_corr=None, stream=None):
+        """Base product and correction to separate outputs (sf_gemv_refined_split).
+        Returns (y_base, y_corr), each [batch][n] fp32."""
+        x = _f16(x if x.dim() == 2 else x.view(1, -1))
+        batch = x.shape[0]
+        if y_base is None:
+            y_base = torch.empty((batch, self.n), dtype=torch.float32, device=x.device)
+        if y_corr is None:
+            y_corr = torch.empty((batch, self.n), dtype=torch.float32, device=x.device)
+        check(abi.sf_gemv_refined_split(ctypes.byref(self.desc), _p(x), batch, chunk, kch, _p(sel),
+                                        _p(refine_rows), _p(y_base), _p(y_corr), _stream(stream)),
+              "sf_gemv_refined_split")
+        return y_base, y_corr
+
+
 def select_channels(x: torch.Tensor, chunk: int = 1024, kch: int = 32, sel=None, stream=None):
     x = _f16(x if x.dim() == 2 else x.view(1, -1))
     batch, k = x.shape

@@ -172,6 +172,19 @@ SF_API sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch
                                     int kch, const int32_t* sel, const void* refine_rows,
                                     float* y, sf_stream_t stream);
 
+/* Base product and correction of one refined GEMV in one launch, written to
+ * separate outputs (both overwritten):
+ *   y_base[b][i] = sum_c x[b][c] * w^[i][c],
+ *   y_corr[b][i] = sum_{c in sel[b]} x[b][c] * (w~[i][c] - w^[i][c]).
+ * This serves fetch lag ([EXPL] "the map app also loads tiles") when the rows
+ * are already resident: the base product goes on at once and the correction
+ * is kept aside until the point of the residual stream where the lag applies
+ * it.  Arguments as sf_gemv_refined; kch >= 1, sel_in is required, y_corr is
+ * [batch][n] fp32 (16-byte aligned, not overlapping y_base). */
+SF_API sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
+                                const int32_t* sel_in, const void* refine_rows, float* y_base,
+                                float* y_corr, sf_stream_t stream);
+
 /* ======================================================================== */
 /* KV cache                                                                  */
 /* ======================================================================== */

@@ -168,6 +168,30 @@ def test_gemv_correction_only_equals_fused(b, r, staged):
     assert rel_l2(host(y), yo) < 1e-5
 
 
+@pytest.mark.parametrize("b,r,staged,n", [(2, 2, True, 6144), (3, 1, False, 512), (4, 2, True, 1152)])
+def test_gemv_split_outputs(b, r, staged, n):
+    """Base product and correction to separate outputs in one launch: the base
+    against the oracle's kch = 0 product, the correction against the oracle's
+    correction on its own (6,144 rows: 1,536 four-row units over the 148-CTA
+    grid, ragged; 1,152 rows: 288 units, most CTAs two, some one)."""
+    rng = np.random.default_rng(90 + b + n)
+    w = inputs.weight(rng, n, 4096)
+    x = inputs.activation(rng, 4096, batch=2)
+    qb, rho, sz = oracle.quant_weights(w, b, r, 128)
+    qw = QuantWeights.pack(cu(w), b, r, 128)
+    xd = cu(f16bits(x))
+    sel_o = oracle.select_chunks(x, 1024, 32)
+    sel_d = cu(sel_o)
+    rows = qw.refine_rows()[sel_d.view(2, -1).long()].contiguous() if staged else None
+    yb, yc = qw.gemv_split(xd, sel_d, 1024, 32, refine_rows=rows)
+    torch.cuda.synchronize()
+    base_o = oracle.gemv_refined(qb, rho, sz, r, 128, x, None, 1024, 0)
+    assert rel_l2(host(yb), base_o) < 1e-5
+    for bb in range(2):
+        corr_o = oracle.gemv_correction(qb, rho, sz, r, 128, x[bb], sel_o[bb])
+        assert rel_l2(host(yc)[bb], corr_o) < 1e-5
+
+
 @pytest.mark.parametrize("G", [32, 64, 256])
 def test_gemv_group_sizes(G):
     rng = np.random.default_rng(G)
