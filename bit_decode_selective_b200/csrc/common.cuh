@@ -54,6 +54,14 @@ inline cudaStream_t as_stream(sf_stream_t s) { return reinterpret_cast<cudaStrea
 
 int num_sms();  // multiprocessors of the current device (cached per device)
 
+// Room left on every SM for the small CTAs of the staging kernels (channel
+// selection, row gather), which run on other streams: the kernels that take a
+// whole SM per CTA (the refined GEMV, the KV base pass) keep their registers to
+// kSideRegs fewer than the SM's 65,536 and their shared memory a block's
+// reservation below the SM's, and a staging CTA fits in what is left (at most
+// kSideRegs registers, no shared memory), so staging never delays them.
+constexpr int kSideRegs = 4096;
+
 // Host-side validation of the descriptor structs (pack.cu).
 sf_status check_kv(const sf_kv* kv);
 sf_status check_wq_public(const sf_wq* w, bool need_refine);

@@ -58,7 +58,7 @@ constexpr int kXShift = 8 * kXP - 4;        // x_fix = x * 2^-(ilogb(max|x|) - k
 constexpr int kXR = 16 * kXP;               // plane words per lane group
 constexpr int kXWords = kXR + 4;            // then sum0, sum1, 2^e, sum
 constexpr int kRowUnit = 4;                 // CTA row ranges start at multiples of 4
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemLimit = 226 * 1024;  // one block reservation (1 KB) below the SM's 228 KB
 
 struct GemvParams {
   const uint32_t* base;
@@ -472,8 +472,10 @@ __device__ __forceinline__ void corr_dispatch(const GemvParams& p, int n0, int r
 // ---------------------------------------------------------------------------
 // the GEMV
 
+// 120 registers x 512 threads: kSideRegs of the SM's registers stay free
+static_assert(65536 - 120 * kThreads >= kSideRegs, "GEMV registers leave no room for a staging CTA");
 template <int BITS, int ZW, int PD>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(GemvParams p) {
+__global__ void __maxnreg__(120) gemv_kernel(GemvParams p) {
   using R = Ring<BITS, ZW>;
   constexpr int U = Lane<BITS>::U, CW = Lane<BITS>::CW;
   extern __shared__ __align__(16) uint32_t smem[];
@@ -776,7 +778,7 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   // the selection (when not given), then the GEMV, which waits for it (and for
   // x) through programmatic dependent launch while its first code copies fly
   if (kch > 0 && !sel_in) {
-    st = launch_select(x, batch, w->k, chunk, kch, sel_out, s);
+    st = launch_select(x, batch, w->k, chunk, kch, sel_out, s, true);
     if (st != SF_OK) return st;
     p.sel = sel_out;
   } else {

@@ -149,8 +149,11 @@ struct WarpSmem {
 };
 
 // GQP: query heads per KV head padded to 4 or 8.  B: base bits (2 or 4).
+// four CTAs of 128 threads per SM at 120 registers (GQP = 4) leave kSideRegs
+// of the SM's registers free; GQP = 8 takes two CTAs of up to 255
+static_assert(65536 - 4 * 120 * kWarps * 32 >= kSideRegs, "base pass registers leave no room for a staging CTA");
 template <int GQP, int B, bool PV>
-__global__ void __launch_bounds__(kWarps * 32, GQP == 4 ? 4 : 2) kv_base_kernel(BaseArgs a) {
+__global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
   using St = Stage<B, PV>;
   using WS = WarpSmem<B, PV>;
   extern __shared__ __align__(16) uint8_t smem[];

@@ -17,30 +17,33 @@
 namespace sf {
 namespace {
 
-constexpr int kVec = 4;  // 16-byte words in flight per thread
+constexpr int kVec = 4;                // 16-byte words in flight per thread
+constexpr int kGatherThreads = 128;     // small CTAs: each fits in the room whole-SM kernels leave
+constexpr int kGatherBlocksMax = 64;    // 64 x 8 KB in flight keeps the host link busy
 
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src,
-                                                          size_t row_vecs,
-                                                          const int32_t* __restrict__ sel,
-                                                          int n_sel, uint4* __restrict__ dst) {
-  pdl_trigger();
-  pdl_wait();
+// CTAs walk the n_sel x row_vecs 16-byte words of the selected rows, kVec loads
+// in flight per thread.  The reads cross the host link, so the CTAs live about
+// as long as the transfer; each fits beside a whole-SM kernel's CTA (at most
+// kSideRegs registers, no shared memory), so the transfer never delays one.
+static_assert(kGatherThreads * 32 <= kSideRegs, "a gather CTA must fit in the room left for staging");
+__global__ void __maxnreg__(32) gather_rows_kernel(const uint4* __restrict__ src, size_t row_vecs,
+                                                   const int32_t* __restrict__ sel, int n_sel,
+                                                   uint4* __restrict__ dst) {
   const size_t total = (size_t)n_sel * row_vecs;
-  const size_t stride = (size_t)gridDim.x * blockDim.x * kVec;
-  for (size_t base = ((size_t)blockIdx.x * blockDim.x) * kVec + threadIdx.x; base < total;
-       base += stride) {
+  const size_t step = (size_t)gridDim.x * kGatherThreads * kVec;
+  for (size_t base = (size_t)blockIdx.x * kGatherThreads * kVec + threadIdx.x; base < total; base += step) {
     uint4 v[kVec];
 #pragma unroll
     for (int u = 0; u < kVec; u++) {
-      size_t i = base + (size_t)u * blockDim.x;
+      const size_t i = base + (size_t)u * kGatherThreads;
       if (i < total) {
-        size_t j = i / row_vecs, c = i % row_vecs;
+        const size_t j = i / row_vecs, c = i - j * row_vecs;
         v[u] = src[(size_t)sel[j] * row_vecs + c];
       }
     }
 #pragma unroll
     for (int u = 0; u < kVec; u++) {
-      size_t i = base + (size_t)u * blockDim.x;
+      const size_t i = base + (size_t)u * kGatherThreads;
       if (i < total) dst[i] = v[u];
     }
   }
@@ -66,11 +69,12 @@ extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_byte
              "host_rows must be page-locked host memory mapped into the device address space");
   cudaStream_t s = as_stream(stream);
   if (n_sel > 0) {
-    size_t vecs = (size_t)n_sel * (row_bytes / 16);
-    long blocks = (long)((vecs + 256 * kVec - 1) / (256 * kVec));
-    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
-    SF_CUDA(launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
-                       (const uint4*)attr.devicePointer, (size_t)(row_bytes / 16), sel, n_sel, (uint4*)dst));
+    const size_t vecs = (size_t)n_sel * (row_bytes / 16);
+    size_t blocks = (vecs + kGatherThreads * kVec - 1) / (kGatherThreads * kVec);
+    if (blocks > (size_t)kGatherBlocksMax) blocks = kGatherBlocksMax;
+    gather_rows_kernel<<<(unsigned)blocks, kGatherThreads, 0, s>>>((const uint4*)attr.devicePointer,
+                                                                   (size_t)(row_bytes / 16), sel, n_sel, (uint4*)dst);
+    SF_LAUNCHED();
   }
   if (done) SF_CUDA(cudaEventRecord((cudaEvent_t)done, s));
   return SF_OK;

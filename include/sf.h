@@ -86,6 +86,7 @@ SF_API const char* sf_status_string(sf_status st);
  * stays valid until the thread's next failing call. */
 SF_API const char* sf_last_error(void);
 
+
 /* ======================================================================== */
 /* Weights                                                                   */
 /* ======================================================================== */

@@ -76,3 +76,18 @@ def test_validation_rejects_before_launch(L):
     assert abi.sf_kv_attend_selective(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, 0, ctypes.c_void_p(16),
                                       None, ctypes.c_void_p(16), None, 0, None) == abi.SF_ERR_INVALID_ARG
     assert abi.sf_stage_refinements_host(None, 16, None, 1, None, None, None) == abi.SF_ERR_INVALID_ARG
+
+
+def test_split_gemv_checks(L):
+    wq = abi.sf_wq(4096, 4096, 2, 2, 128, 16, 16, 16)
+    p16 = ctypes.c_void_p(16)
+    # the split form needs a correction, a selection and a separate output
+    assert abi.sf_gemv_refined_split(ctypes.byref(wq), p16, 1, 1024, 0, p16, None, p16, p16, None) \
+        == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_gemv_refined_split(ctypes.byref(wq), p16, 1, 1024, 32, None, None, p16, p16, None) \
+        == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_gemv_refined_split(ctypes.byref(wq), p16, 1, 1024, 32, p16, None, p16, None, None) \
+        == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_gemv_refined_split(ctypes.byref(wq), p16, 1, 1024, 32, p16, None, ctypes.c_void_p(4096),
+                                     ctypes.c_void_p(4096 + 1024), None) == abi.SF_ERR_INVALID_ARG
+    assert b"overlap" in abi.sf_last_error()
