@@ -10,7 +10,7 @@
 //       w~ = w^ + s * (2*rho + 1 - 2^r) / 2^(r+1).
 //   the-map-app-also-loads-tiles paragraph -- with fetch lag the correction
 //     of a projection is applied later than its base product; the
-//     correction-only mode below computes it on its own.
+//     correction-only kernel below computes it on its own.
 //
 // Decomposition, per output row i (fp32 accumulation):
 //   y_i = sum_groups [ s_ig * sum_{c in g} x_c q_ic + m_ig * sum_{c in g} x_c ]
@@ -70,9 +70,8 @@ struct GemvParams {
   int N, K, G, gshift, r, batch, n_sel, segs;
   int refine_row_words;  // N * r / 32
   int staged;            // refine holds [batch][n_sel] staged rows
-  int mode;              // 0: base + correction, 1: correction only, added into y
   int rows_max;          // most rows a CTA owns
-  int plane_words;       // shared words of the activation planes (mode 0)
+  int plane_words;       // shared words of the activation planes
   int area_words;        // shared words of the copy rings (reused by the slow correction path)
   int fast;              // correction tables in their own shared region, filled before the base pass
   int w_span;            // stride of the refinement-word table (words a CTA's rows can span)
@@ -498,12 +497,12 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvParams p) {
   const int steps = (rows + U - 1) / U, ntask = p.segs * steps;
   const int ta = (int)((long)warp * ntask / kWarps), tb = (int)((long)(warp + 1) * ntask / kWarps);
   const size_t row_bytes = (size_t)p.K * (BITS == 3 ? 2 : BITS) / 8;
-  const bool fill_szt = p.fast && p.mode == 0 && p.n_sel > 0;
+  const bool fill_szt = p.fast && p.n_sel > 0;
   // the fast correction's per-warp partials: in the ring area, free once the base pass is done
   float* cpart = p.corr_split && p.fast && p.n_sel > 0 ? reinterpret_cast<float*>(area) : nullptr;
 
   for (int b = 0; b < p.batch; b++) {
-    if (p.mode == 0) {
+    {
       // ---- base pass of batch row b: every (row, segment) partial is written once
       uint32_t* ring = area + warp * PD * R::words;
       int iseg = ta / steps, ist = ta - iseg * steps, islot = 0, left = tb - ta;
@@ -599,20 +598,6 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvParams p) {
         cslot = cslot + 1 == PD ? 0 : cslot + 1;
       }
       cp_async_wait<0>();
-    } else {
-      for (int i = threadIdx.x; i < rows * p.pstride; i += kThreads) part[i] = 0.f;
-      if (b == 0) pdl_wait();  // x, the selection, the staged rows and y are complete
-      if (p.fast) {
-        // the CTA's (s, m) words are one contiguous block of sz, [rows][gpr];
-        // they are stored transposed
-        const uint32_t* zsrc = reinterpret_cast<const uint32_t*>(p.sz) + (size_t)n0 * gpr;
-        for (int i = threadIdx.x; i < rows * gpr; i += kThreads) {
-          const int row = i / gpr, g = i - row * gpr;
-          cp_async4(szt + g * p.rows_max + row, zsrc + i);
-        }
-        corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
-        cp_async_wait<0>();
-      }
     }
     __syncthreads();
 
@@ -652,10 +637,102 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvParams p) {
         *dst = base;
         p.y_corr[(size_t)b * p.N + row] = corr;
       } else {
-        *dst = p.mode == 1 ? *dst + corr : base + corr;
+        *dst = base + corr;
       }
     }
     __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the correction on its own (fetch lag), added into y
+//
+// A thread owns 8 consecutive output rows of one batch row and walks every
+// selected channel in order, so the sum is deterministic: per channel it reads
+// the refinement word that covers its rows (consecutive threads read
+// consecutive words), adds x_c f_t, f_t = 1 + rho_t / 2^r, into a per-row run,
+// and scales each run of channels that share a scale group once,
+// s (run - sum x_c cfac) = s sum x_c (rho + off) / 2^r.  CTAs of 64 threads,
+// at most 64 registers and no shared memory fit in the room every whole-SM
+// kernel of the library leaves free, so on a staging stream the correction
+// neither waits for them nor delays them.
+
+constexpr int kCorrThreads = 64;
+constexpr int kCorrRows = 8;
+static_assert(kCorrThreads * 64 <= kSideRegs, "a correction CTA must fit in the room left for staging");
+
+struct CorrArgs {
+  const uint32_t* refine;  // channel-major rows [K][row_words], or staged rows [batch][n_sel][row_words]
+  const uint16_t* sz;
+  const uint16_t* x;
+  const int32_t* sel;
+  float* y;
+  int N, K, gshift, r, n_sel, row_words, staged, units;  // units = batch * N / kCorrRows
+};
+
+template <int R>
+__global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
+  const int u = blockIdx.x * kCorrThreads + threadIdx.x;
+  if (u >= a.units) return;
+  const int per_b = a.N / kCorrRows;
+  const int b = u / per_b, row0 = (u - b * per_b) * kCorrRows;
+  const int bit0 = row0 * a.r, wi = bit0 >> 5;
+  const int gpr = a.K >> a.gshift;
+  // the rows' bits start at bit sh of the word (a multiple of 8); the word is
+  // shifted down first, so row t's field sits at bit R t
+  const int sh = bit0 & 31;
+  constexpr uint32_t fmask = ((1u << R) - 1u) << (23 - R);
+  const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << R)) / (float)(1 << R);
+  const uint32_t* zrow = reinterpret_cast<const uint32_t*>(a.sz) + (size_t)row0 * gpr;
+  const int32_t* sel = a.sel + (size_t)b * a.n_sel;
+  const uint16_t* xb = a.x + (size_t)b * a.K;
+  float acc[kCorrRows], run[kCorrRows];
+#pragma unroll
+  for (int t = 0; t < kCorrRows; t++) acc[t] = run[t] = 0.f;
+  float C = 0.f;
+  int gcur = -1;
+  auto flush = [&]() {
+    if (gcur >= 0) {
+#pragma unroll
+      for (int t = 0; t < kCorrRows; t++) {
+        const uint32_t zw = __ldg(zrow + (size_t)t * gpr + gcur);
+        acc[t] = fmaf(__low2float(*reinterpret_cast<const __half2*>(&zw)), run[t] - C, acc[t]);
+      }
+    }
+  };
+  auto word_of = [&](int j, int c) {
+    const size_t row = a.staged ? (size_t)b * a.n_sel + j : (size_t)c;
+    return __ldg(a.refine + row * a.row_words + wi) >> sh;
+  };
+  // channel j + 1's index, activation and word are loaded while j is summed
+  int c = a.n_sel > 0 ? __ldg(sel) : 0;
+  float xc = a.n_sel > 0 ? h2f(__ldg(xb + c)) : 0.f;
+  uint32_t w = a.n_sel > 0 ? word_of(0, c) : 0u;
+  for (int j = 0; j < a.n_sel; j++) {
+    const int cn = j + 1 < a.n_sel ? __ldg(sel + j + 1) : 0;
+    const float xn = j + 1 < a.n_sel ? h2f(__ldg(xb + cn)) : 0.f;
+    const uint32_t wn = j + 1 < a.n_sel ? word_of(j + 1, cn) : 0u;
+    const int g = c >> a.gshift;
+    if (g != gcur) {
+      flush();
+      gcur = g, C = 0.f;
+#pragma unroll
+      for (int t = 0; t < kCorrRows; t++) run[t] = 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < kCorrRows; t++)
+      run[t] = fmaf(__uint_as_float(0x3F800000u | (__funnelshift_l(w, w, (23 - R - R * t) & 31) & fmask)), xc,
+                    run[t]);
+    C = fmaf(xc, cfac, C);
+    c = cn, xc = xn, w = wn;
+  }
+  flush();
+  float4* yv = reinterpret_cast<float4*>(a.y + (size_t)b * a.N + row0);
+#pragma unroll
+  for (int q = 0; q < kCorrRows / 4; q++) {
+    float4 v = yv[q];
+    v.x += acc[4 * q], v.y += acc[4 * q + 1], v.z += acc[4 * q + 2], v.w += acc[4 * q + 3];
+    yv[q] = v;
   }
 }
 
@@ -690,7 +767,7 @@ int pick_corr_rows(int rows) {
 
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                       const int32_t* sel_in, int32_t* sel_out, const void* refine_rows, float* y,
-                      int mode, cudaStream_t s, float* y_corr = nullptr) {
+                      cudaStream_t s, float* y_corr = nullptr) {
   sf_status st = check_wq_public(w, false);
   if (st != SF_OK) return st;
   SF_REQUIRE(x && aligned16(x), "x must be a non-null 16-byte aligned device pointer");
@@ -707,11 +784,8 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
     if (sel_in) {
       SF_REQUIRE(aligned16(sel_in), "sel_in must be 16-byte aligned");
     } else {
-      SF_REQUIRE(mode == 0, "the correction-only call needs a selection");
       SF_REQUIRE(sel_out && aligned16(sel_out), "sel_out is needed when sel_in is NULL");
     }
-  } else if (mode == 1) {
-    return SF_OK;  // nothing to correct
   }
 
   GemvParams p = {};
@@ -724,7 +798,6 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.N = w->n, p.K = w->k, p.G = w->group, p.r = w->r, p.batch = batch, p.n_sel = n_sel;
   p.gshift = 0;
   while ((1 << p.gshift) < w->group) p.gshift++;
-  p.mode = mode;
   p.segs = (w->k + kSegChannels - 1) / kSegChannels;
   p.refine_row_words = w->n * w->r / 32;
   p.staged = refine_rows != nullptr;
@@ -736,7 +809,7 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   p.rows_max = ((units + grid - 1) / grid) * kRowUnit;
   p.w_span = p.rows_max * w->r / 32 + 2;
   p.corr_rows = pick_corr_rows(p.rows_max);
-  p.plane_words = mode == 0 ? (w->k / kLaneCh) * kXWords + kWarps * 4 * kLaneCh : 0;  // planes, then per-warp scratch
+  p.plane_words = (w->k / kLaneCh) * kXWords + kWarps * 4 * kLaneCh;  // planes, then per-warp scratch
   const size_t gpr = (size_t)(w->k / w->group);
   p.pstride = p.segs + 1;
   const size_t part_words = ((size_t)p.rows_max * p.pstride + 3) & ~(size_t)3;
@@ -748,26 +821,15 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
   // the deepest that fits (the tables then go through the ring area in chunks)
   int pd = 0;
   size_t area = 0;
-  if (mode == 0) {
-    for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
-      const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
-      if (fixed + ring + (n_sel > 0 ? table_words : 0) <= limit_words) pd = d, area = ring, p.fast = n_sel > 0;
-    }
-    for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
-      const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
-      if (fixed + ring <= limit_words) pd = d, area = ring, p.fast = 0;
-    }
-    SF_UNSUPPORTED(pd > 0, "n=%d, k=%d does not fit in shared memory", w->n, w->k);
-  } else {
-    const size_t split_words = (size_t)kWarps * p.rows_max;
-    if (fixed + split_words + table_words <= limit_words) {
-      p.fast = 1, area = split_words;
-    } else {
-      p.fast = fixed + 4 + table_words <= limit_words;
-      area = p.fast ? 4 : limit_words - fixed;
-    }
-    pd = 2;
+  for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
+    const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
+    if (fixed + ring + (n_sel > 0 ? table_words : 0) <= limit_words) pd = d, area = ring, p.fast = n_sel > 0;
   }
+  for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
+    const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
+    if (fixed + ring <= limit_words) pd = d, area = ring, p.fast = 0;
+  }
+  SF_UNSUPPORTED(pd > 0, "n=%d, k=%d does not fit in shared memory", w->n, w->k);
   p.corr_split = p.fast && area >= (size_t)kWarps * p.rows_max;
   if (!p.fast && n_sel > 0)
     SF_UNSUPPORTED(area >= (size_t)(4 + p.w_span) * 16, "n=%d, k=%d: no room for the correction", w->n, w->k);
@@ -822,14 +884,41 @@ extern "C" sf_status sf_gemv_refined(const sf_wq* w, const uint16_t* x, int batc
                                      const void* refine_rows, float* y, void* ws, size_t ws_bytes,
                                      sf_stream_t stream) {
   (void)ws, (void)ws_bytes;
-  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, 0, as_stream(stream));
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, sel_out, refine_rows, y, as_stream(stream));
 }
 
 extern "C" sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch, int chunk,
                                         int kch, const int32_t* sel, const void* refine_rows,
                                         float* y, sf_stream_t stream) {
-  SF_REQUIRE(kch == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
-  return gemv_launch(w, x, batch, chunk, kch, sel, nullptr, refine_rows, y, 1, as_stream(stream));
+  sf_status st = check_wq_public(w, false);
+  if (st != SF_OK) return st;
+  SF_REQUIRE(kch >= 0, "kch=%d < 0", kch);
+  if (kch == 0) return SF_OK;  // nothing to correct
+  SF_REQUIRE(sel && aligned16(sel), "sel must be non-null and 16-byte aligned");
+  SF_REQUIRE(y && aligned16(y), "y must be a non-null 16-byte aligned device pointer");
+  SF_UNSUPPORTED(batch >= 1 && batch <= 8, "batch=%d outside [1, 8]", batch);
+  st = check_select_args(x, batch, w->k, chunk, kch);
+  if (st != SF_OK) return st;
+  SF_REQUIRE(refine_rows || w->refine, "the correction needs w->refine or staged refine_rows");
+  SF_REQUIRE(!refine_rows || aligned16(refine_rows), "refine_rows must be 16-byte aligned");
+  CorrArgs a;
+  a.refine = (const uint32_t*)(refine_rows ? refine_rows : w->refine);
+  a.sz = w->sz, a.x = x, a.sel = sel, a.y = y;
+  a.N = w->n, a.K = w->k, a.r = w->r;
+  a.gshift = 0;
+  while ((1 << a.gshift) < w->group) a.gshift++;
+  a.n_sel = (w->k / chunk) * kch;
+  a.row_words = w->n * w->r / 32;
+  a.staged = refine_rows != nullptr;
+  a.units = batch * (w->n / kCorrRows);
+  // a plain launch: on a staging stream it follows an event wait
+  const int blocks = (a.units + kCorrThreads - 1) / kCorrThreads;
+  if (a.r == 2)
+    corr_only_kernel<2><<<blocks, kCorrThreads, 0, as_stream(stream)>>>(a);
+  else
+    corr_only_kernel<1><<<blocks, kCorrThreads, 0, as_stream(stream)>>>(a);
+  SF_LAUNCHED();
+  return SF_OK;
 }
 
 extern "C" sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, int batch, int chunk,
@@ -842,5 +931,5 @@ extern "C" sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, in
   const size_t bytes = (size_t)batch * (size_t)w->n * sizeof(float);
   const char *a0 = (const char*)y_base, *b0 = (const char*)y_corr;
   SF_REQUIRE(!y_base || a0 + bytes <= b0 || b0 + bytes <= a0, "y_base and y_corr overlap");
-  return gemv_launch(w, x, batch, chunk, kch, sel_in, nullptr, refine_rows, y_base, 0, as_stream(stream), y_corr);
+  return gemv_launch(w, x, batch, chunk, kch, sel_in, nullptr, refine_rows, y_base, as_stream(stream), y_corr);
 }

@@ -11,15 +11,18 @@ and the order of the calls.  The call order implements the schedule of
     fetch lead (1 layer) selects a projection's channels from the previous
     layer's activation and starts the row transfer on a side stream while the
     layers in between compute; fetch lag (1 layer) applies the residual-writing
-    projections' (o, down) corrections at the start of the next layer (they are
-    computed on the side stream, off the main stream's path, and added with
-    the next residual).
+    projections' (o, down) corrections at the start of the next layer.  With
+    the rows staged a layer ahead, o's projection computes its correction in
+    the same launch and writes it to a separate buffer that the next layer's
+    residual add picks up (so the MLP input does not see it); down's lagged
+    correction enters the residual stream at the same point as down's own
+    output (nothing reads the residual in between), so down refines in place.
 Readings as in the oracle (oracle/decoder.py): layer 0 selects from its own
 activations; q/k/v and gate/up correct in place; the new token is appended at
 position T and attention runs over T + 1 tokens.
 
-step() only enqueues work on the current stream (plus the side stream), so it
-can be captured in a CUDA graph and replayed.
+step() only enqueues work on the current stream (plus the two staging
+streams), so it can be captured in a CUDA graph and replayed.
 """
 from __future__ import annotations
 
@@ -122,14 +125,9 @@ class Decoder:
         self.stage_stream = {"qkv": self.side, "gate_up": self.side, "o": self.side2, "down": self.side2}
         self.ev_sel = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
         self.ev_stage = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
-        # fetch lag: the side stream sums layer l's o and down corrections into
-        # delta[l % 2]; the next layer's residual add picks them up
-        self.delta = [f32(B, cfg.hidden) for _ in range(2)]
-        self.lag_stream = torch.cuda.Stream(device=dev)  # apart from the staging queue
-        self.ev_lag_done = {n: [torch.cuda.Event() for _ in range(2)] for n in ("o", "down")}
-        self.lag_pending = set()  # (name, slot) whose staged rows a lag correction of this step reads
-        self.ev_x = {n: [torch.cuda.Event() for _ in range(2)] for n in ("o", "down")}
-        self.ev_lag = [torch.cuda.Event() for _ in range(2)]
+        # fetch lag: layer l's o correction, written by its projection and added
+        # by the next layer's residual add
+        self.delta = f32(B, cfg.hidden)
         self.lm_head = None
         self.ws = None
 
@@ -186,9 +184,6 @@ class Decoder:
         ev = self.ev_sel[name][slot]
         ev.record(main)
         side.wait_event(ev)
-        if (name, slot) in self.lag_pending:  # a lag correction still reads this slot
-            side.wait_event(self.ev_lag_done[name][slot])
-            self.lag_pending.discard((name, slot))
         self._select(name, x, slot, side)
         if self.slots is not None:
             self._stage(layer, name, slot)
@@ -199,15 +194,21 @@ class Decoder:
         main.wait_event(self.ev_stage[name][slot])
         return self.slots[name][slot] if self.slots is not None else None
 
-    def _proj(self, layer, name, x, y, slot, main, base_only=False):
-        """y = W~ x for layer `layer` with the selection in `slot`."""
+    def _proj(self, layer, name, x, y, slot, main, y_corr=None):
+        """y = W~ x for layer `layer` with the selection in `slot`; with y_corr,
+        y gets the base product and y_corr the correction (fetch lag)."""
         cfg = self.cfg
         qw = self.layers[layer][name]
-        if cfg.kch == 0 or base_only:
+        if cfg.kch == 0:
             check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, 0, None, None, None,
                                       _p(y), _p(self.gemv_ws), self.gemv_ws.numel(), _s(main)), "sf_gemv_refined")
             return
         rows = self._ready(name, slot, main)
+        if y_corr is not None:
+            check(abi.sf_gemv_refined_split(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
+                                            _p(self.sel[name][slot]), _p(rows), _p(y), _p(y_corr), _s(main)),
+                  "sf_gemv_refined_split")
+            return
         check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
                                   _p(self.sel[name][slot]), None, _p(rows), _p(y), _p(self.gemv_ws),
                                   self.gemv_ws.numel(), _s(main)),
@@ -230,55 +231,20 @@ class Decoder:
             return
         self._side_select_stage(layer + 1, name, x, (layer + 1) % 2, main)
 
-    def _lagged(self, layer, name, x, main):
-        """Fetch lag: layer `layer`'s correction of projection `name` (o or
-        down), computed on the side stream once x is ready and summed into
-        delta[layer % 2]; after down the event ev_lag marks the sum complete."""
-        cfg = self.cfg
-        slot = layer % 2
-        lag = self.lag_stream
-        ev = self.ev_x[name][slot]
-        ev.record(main)
-        lag.wait_event(ev)
-        lag.wait_event(self.ev_stage[name][slot])  # the selection and the staged rows
-        qw = self.layers[layer][name]
-        rows = self.slots[name][slot] if self.slots is not None else None
-        if name == "o":
-            with torch.cuda.stream(lag):
-                self.delta[slot].zero_()
-        check(abi.sf_gemv_correction(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
-                                     _p(self.sel[name][slot]), _p(rows), _p(self.delta[slot]), _s(lag)),
-              "sf_gemv_correction")
-        self.ev_lag_done[name][slot].record(lag)
-        self.lag_pending.add((name, slot))
-        if name == "down":
-            self.ev_lag[slot].record(lag)
-
-    def _lag_delta(self, layer, main):
-        """The summed lagged corrections of `layer` for the next residual add
-        (None without fetch lag)."""
-        cfg = self.cfg
-        if cfg.kch == 0 or not cfg.lag or layer < 0:
-            return None
-        main.wait_event(self.ev_lag[layer % 2])
-        return self.delta[layer % 2]
-
     def step(self, hidden: torch.Tensor):
         """Enqueue one decode step: hidden fp16 [B][hidden] -> self.logits."""
         cfg = self.cfg
         main = torch.cuda.current_stream(self.dev)
         self.side.wait_stream(main)
         self.side2.wait_stream(main)
-        self.lag_stream.wait_stream(main)
-        self.lag_pending = set()
         B, T = self.B, self.T
         check(abi.sf_widen_f16(_p(hidden), B * cfg.hidden, _p(self.h), _s(main)), "sf_widen_f16")
         add = None
         lagging = cfg.kch > 0 and bool(cfg.lag)
+        delta = None  # the previous layer's lagged o correction
         for l in range(cfg.n_layers):
             slot = l % 2
             L = self.layers[l]
-            delta = self._lag_delta(l - 1, main)
             x_attn, x_o, x_mlp, x_down = self.x_attn[slot], self.x_o[slot], self.x_mlp[slot], self.x_down[slot]
             check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), _p(delta), B, cfg.hidden, cfg.eps, _p(x_attn),
                                           _s(main)), "sf_rmsnorm_residual")
@@ -296,10 +262,8 @@ class Decoder:
                                              _s(main)), "sf_kv_attend_selective")
             check(abi.sf_cast_f16(_p(self.attn), B * cfg.h_q * cfg.d, _p(x_o), _s(main)), "sf_cast_f16")
             self._prepare(l, "o", x_o, main)
-            if lagging:
-                self._lagged(l, "o", x_o, main)
             self._lead(l, "o", x_o, main)
-            self._proj(l, "o", x_o, self.o_out, slot, main, base_only=bool(cfg.lag))
+            self._proj(l, "o", x_o, self.o_out, slot, main, y_corr=self.delta if lagging else None)
             check(abi.sf_rmsnorm_residual(_p(self.h), _p(self.o_out), None, B, cfg.hidden, cfg.eps,
                                           _p(x_mlp), _s(main)), "sf_rmsnorm_residual")
             # MLP block
@@ -308,17 +272,14 @@ class Decoder:
             self._proj(l, "gate_up", x_mlp, self.gu_out, slot, main)
             check(abi.sf_silu_mul(_p(self.gu_out), B, cfg.inter, _p(x_down), _s(main)), "sf_silu_mul")
             self._prepare(l, "down", x_down, main)
-            if lagging:
-                self._lagged(l, "down", x_down, main)
             self._lead(l, "down", x_down, main)
-            self._proj(l, "down", x_down, self.down_out, slot, main, base_only=bool(cfg.lag))
+            self._proj(l, "down", x_down, self.down_out, slot, main)  # its lagged correction lands with it
             add = self.down_out
-        delta = self._lag_delta(cfg.n_layers - 1, main)
+            delta = self.delta if lagging else None
         check(abi.sf_rmsnorm_residual(_p(self.h), _p(add), _p(delta), B, cfg.hidden, cfg.eps, _p(self.x_final),
                                       _s(main)), "sf_rmsnorm_residual")
         check(abi.sf_gemv_f16(_p(self.lm_head), _p(self.x_final), B, cfg.vocab, cfg.hidden, _p(self.logits),
                               _s(main)), "sf_gemv_f16")
         main.wait_stream(self.side)
         main.wait_stream(self.side2)
-        main.wait_stream(self.lag_stream)
         return self.logits
