@@ -53,6 +53,8 @@ _SIGNATURES = {
                                c_void_p, c_void_p, c_void_p], c_int),
     "sf_kv_bytes": ([c_int] * 7 + [POINTER(c_size_t)] * 3, c_int),
     "sf_kv_pack_tokens": ([POINTER(sf_kv), c_void_p, c_void_p, c_int, c_int, c_void_p], c_int),
+    "sf_kv_append_rope": ([POINTER(sf_kv), c_void_p, c_int, c_int, ctypes.c_float, c_int, c_void_p, c_void_p],
+                          c_int),
     "sf_kv_unpack_codes": ([POINTER(sf_kv), c_int, c_int, c_void_p, c_void_p, c_void_p], c_int),
     "sf_kv_score_select": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_size_t, c_void_p], c_int),
@@ -62,6 +64,8 @@ _SIGNATURES = {
     "sf_kv_attn_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
     "sf_kv_attend_selective": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_size_t, c_void_p], c_int),
+    "sf_kv_attend_selective_f16": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_size_t, c_void_p], c_int),
     "sf_kv_attend_selective_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
     "sf_kv_attend_selective_static": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                                        c_void_p, c_void_p], c_int),
@@ -130,11 +134,13 @@ sf_gemv_refined_split = _call("sf_gemv_refined_split")
 sf_kv_bytes = _call("sf_kv_bytes")
 sf_kv_pack_tokens = _call("sf_kv_pack_tokens")
 sf_kv_unpack_codes = _call("sf_kv_unpack_codes")
+sf_kv_append_rope = _call("sf_kv_append_rope")
 sf_kv_score_select = _call("sf_kv_score_select")
 sf_kv_score_select_workspace_bytes = _call("sf_kv_score_select_workspace_bytes")
 sf_kv_attn_refined = _call("sf_kv_attn_refined")
 sf_kv_attn_workspace_bytes = _call("sf_kv_attn_workspace_bytes")
 sf_kv_attend_selective = _call("sf_kv_attend_selective")
+sf_kv_attend_selective_f16 = _call("sf_kv_attend_selective_f16")
 sf_kv_attend_selective_workspace_bytes = _call("sf_kv_attend_selective_workspace_bytes")
 sf_kv_attend_selective_static = _call("sf_kv_attend_selective_static")
 sf_rmsnorm_residual = _call("sf_rmsnorm_residual")

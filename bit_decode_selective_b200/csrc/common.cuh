@@ -74,6 +74,24 @@ __device__ __forceinline__ double h2d(uint16_t h) {
 
 __device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 
+// Rotary embedding, rotate-half pairing: element i (< d/2) and i + d/2 of a
+// head turn by the angle pos * theta^(-2i/d), computed in fp64 so that long
+// positions keep their precision; the rotation itself is fp32, each product
+// and sum rounded once.
+__device__ __forceinline__ void rope_cos_sin(int pos, double theta, int i, int d, float& c, float& s) {
+  const double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)d);
+  double sn, cs;
+  sincos(ang, &sn, &cs);
+  c = (float)cs, s = (float)sn;
+}
+// first (x0 = element i) and second (x1 = element i + d/2) rotated element
+__device__ __forceinline__ float rope_first(float x0, float x1, float c, float s) {
+  return __fsub_rn(__fmul_rn(x0, c), __fmul_rn(x1, s));
+}
+__device__ __forceinline__ float rope_second(float x0, float x1, float c, float s) {
+  return __fadd_rn(__fmul_rn(x0, s), __fmul_rn(x1, c));
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue now / wait until the previous kernel's results are visible.  Both
 // are no-ops when the launch carried no programmatic-serialization attribute.

@@ -51,8 +51,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_residual_kernel(float* __restric
 }
 
 // qkv[b] = [q (h_q*d) | k (h_kv*d) | v (h_kv*d)] fp32 -> rotated q, k and v in
-// fp16.  Rotate-half pairing (i, i + d/2); angle pos * theta^(-2i/d), computed
-// in fp64 so that long positions keep their precision.
+// fp16 (rope_cos_sin / rope_first / rope_second).
 __global__ void rope_split_kernel(const float* __restrict__ qkv, int h_q, int h_kv, int d, int pos,
                                   double theta, uint16_t* __restrict__ q, uint16_t* __restrict__ k,
                                   uint16_t* __restrict__ v) {
@@ -65,11 +64,9 @@ __global__ void rope_split_kernel(const float* __restrict__ qkv, int h_q, int h_
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     float x0 = src[i], x1 = src[i + half];
     if (head < h_q + h_kv) {
-      double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)d);
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      float c = (float)cs, s = (float)sn;
-      float y0 = x0 * c - x1 * s, y1 = x0 * s + x1 * c;
+      float c, s;
+      rope_cos_sin(pos, theta, i, d, c, s);
+      const float y0 = rope_first(x0, x1, c, s), y1 = rope_second(x0, x1, c, s);
       x0 = y0, x1 = y1;
     }
     uint16_t* dst;

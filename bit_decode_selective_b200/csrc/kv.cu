@@ -526,6 +526,7 @@ struct PostArgs {
   int select;
   float* scores;        // nullable [batch][h_kv][T]
   float* out;           // nullable [batch][h_q][kD]
+  uint16_t* out16;      // nullable [batch][h_q][kD], the same rounded to fp16
   int chunk;            // tokens per CTA
   float scale;
 };
@@ -782,7 +783,7 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
       if (!done && key == prefix) take = eq_seen++ < eq_mine;
       if (take && pos < a.k_tok) {
         selw[pos] = t0 + i;
-        if (a.out) {  // hand the token to the CTA that refines position pos
+        if (a.out || a.out16) {  // hand the token to the CTA that refines position pos
           const int dst = (int)(((long)(pos + 1) * CL + a.k_tok - 1) / a.k_tok) - 1;
           const int dja = (int)((long)dst * a.k_tok / CL);
           cluster.map_shared_rank(&mail.tok[0], dst)[pos - dja] = t0 + i;
@@ -797,7 +798,7 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
     __syncthreads();
   }
-  if (!a.out) return;  // no peer reads or writes this CTA's shared memory any more
+  if (!a.out && !a.out16) return;  // no peer reads or writes this CTA's shared memory any more
 
   // ---- refined attention on this CTA's share of the selected tokens
   {
@@ -978,7 +979,9 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
     for (int d = tid; d < kD; d += kPostThreads) {
       float num = 0.f, den = sh.Z[cr];
       for (int rk = 0; rk < CL; rk++) num += mail.num[rk][d], den += mail.den[rk];
-      a.out[(hq0 + cr) * kD + d] = num / den;
+      const float o = num / den;
+      if (a.out) a.out[(hq0 + cr) * kD + d] = o;
+      if (a.out16) a.out16[(hq0 + cr) * kD + d] = __half_as_ushort(__float2half_rn(o));
     }
   }
 }
@@ -1076,7 +1079,7 @@ BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* lo
 // serialization: its CTAs start while the base pass drains).
 sf_status launch_post(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
                       const float* logits, const float* part, int rec, int32_t* sel, int select,
-                      float* scores, float* out, cudaStream_t s) {
+                      float* scores, float* out, cudaStream_t s, uint16_t* out16 = nullptr) {
   PostArgs a;
   a.kb = (const uint8_t*)kv->kb, a.kr = (const uint8_t*)kv->kr;
   a.vb = (const uint8_t*)kv->vb, a.vr = (const uint8_t*)kv->vr;
@@ -1084,13 +1087,13 @@ sf_status launch_post(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_
   a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.b = kv->b, a.r = kv->r, a.T = t;
   a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
   a.logits = logits, a.part = part, a.nrec = P.nrec, a.rec = rec;
-  a.k_tok = k_tok, a.sel = sel, a.select = select, a.scores = scores, a.out = out;
+  a.k_tok = k_tok, a.sel = sel, a.select = select, a.scores = scores, a.out = out, a.out16 = out16;
   a.chunk = P.chunk;
   a.scale = 1.0f / sqrtf((float)kD);
   // the score keys' space, which later holds the per-warp partial numerators
   // of the refined attention [warps][GQP][kD]
   const size_t gqp = a.gq <= 4 ? 4 : 8;
-  const size_t key_words = out ? std::max((size_t)P.chunk, (size_t)(kPostThreads / 32) * gqp * kD) : (size_t)P.chunk;
+  const size_t key_words = (out || out16) ? std::max((size_t)P.chunk, (size_t)(kPostThreads / 32) * gqp * kD) : (size_t)P.chunk;
   const size_t smem = sizeof(PostMail) + ((size_t)kPostStage * tok_words(kv->b, kv->r) + key_words) * 4;
   void (*kern)(PostArgs);
   if (a.gq <= 4)
@@ -1198,9 +1201,13 @@ extern "C" size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t,
   return make_plan(kv, t, h_q, k_tok, !logits_given, true, true, 0).total;
 }
 
-extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q,
-                                            int k_tok, int32_t* sel, float* logits, float* out,
-                                            void* ws, size_t ws_bytes, sf_stream_t stream) {
+namespace sf {
+namespace {
+
+// Score, select and attend; the output in fp32 (out) and/or fp16 (out16).
+sf_status attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, int32_t* sel,
+                           float* logits, float* out, uint16_t* out16, void* ws, size_t ws_bytes,
+                           cudaStream_t s) {
   sf_status st = check_kv(kv);
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
@@ -1208,18 +1215,35 @@ extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16
   SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
-  SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
+  SF_REQUIRE((out || out16) && (!out || aligned16(out)) && (!out16 || aligned16(out16)),
+             "out must be a non-null 16-byte aligned device pointer");
   Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
-  cudaStream_t s = as_stream(stream);
   float* lg = logits ? logits : (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, sel, 1, nullptr, out, s);
+  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, sel, 1, nullptr, out, s, out16);
+}
+
+}  // namespace
+}  // namespace sf
+
+extern "C" sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                            int k_tok, int32_t* sel, float* logits, float* out,
+                                            void* ws, size_t ws_bytes, sf_stream_t stream) {
+  SF_REQUIRE(out, "out must be a non-null 16-byte aligned device pointer");
+  return attend_selective(kv, t, q, h_q, k_tok, sel, logits, out, nullptr, ws, ws_bytes, as_stream(stream));
+}
+
+extern "C" sf_status sf_kv_attend_selective_f16(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                                int k_tok, int32_t* sel, float* logits, uint16_t* out,
+                                                void* ws, size_t ws_bytes, sf_stream_t stream) {
+  SF_REQUIRE(out, "out must be a non-null 16-byte aligned device pointer");
+  return attend_selective(kv, t, q, h_q, k_tok, sel, logits, nullptr, out, ws, ws_bytes, as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------

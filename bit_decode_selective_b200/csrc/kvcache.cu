@@ -42,13 +42,39 @@ __device__ __forceinline__ void group_minmax(const double (&v)[4], int d0, doubl
 // halves (values) are assembled in shared memory and stored by the first
 // lanes; a token owns all of them, so tokens never share a store.
 // Keys and values of the same tokens in one launch: blockIdx.y picks the kind.
+// With qkv set, the one token comes straight from a qkv projection row: its
+// key is turned by the rotary embedding and rounded to fp16 first, its value
+// rounded to fp16, and a third kind turns the queries into q_out.
 struct PackArgs {
   const uint16_t* x[2];  // [BH][nt][128] fp16 keys, values (either may be null)
   uint32_t* codes[2];
   uint32_t* refine[2];
   uint16_t* sz[2];
   int BH, nt, t_max, t0, first_kind;
+  const float* qkv;      // nullable: [batch][(h_q + 2 h_kv) 128] fp32 (nt = 1)
+  uint16_t* q_out;       // with qkv: [batch][h_q][128] fp16
+  int h_q, h_kv, pos;
+  double theta;
 };
+
+// The lane's 4 consecutive elements (4 lane .. 4 lane + 3) of a 128-element
+// head row, turned by the rotary embedding: element e < 64 pairs with e + 64,
+// held by lane ^ 16.
+__device__ __forceinline__ void rope_lane4(float (&x)[4], int lane, int pos, double theta) {
+  float xp[4];
+#pragma unroll
+  for (int i = 0; i < 4; i++) xp[i] = __shfl_xor_sync(0xffffffffu, x[i], 16);
+  const bool first = lane < 16;
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const int e = 4 * lane + i, k = first ? e : e - kHeadDim / 2;
+    float c, sn;
+    rope_cos_sin(pos, theta, k, kHeadDim, c, sn);
+    x[i] = first ? rope_first(x[i], xp[i], c, sn) : rope_second(xp[i], x[i], c, sn);
+  }
+}
+
+__device__ __forceinline__ float f16_round(float x) { return __half2float(__float2half_rn(x)); }
 
 template <int B, int R>
 __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
@@ -56,13 +82,29 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
   __shared__ uint32_t acc[kPackWarps][8 * (B + R)];
   pdl_trigger();
   pdl_wait();
-  const int is_value = pa.first_kind + blockIdx.y;
+  const int kind = pa.first_kind + blockIdx.y;  // 0 keys, 1 values, 2 queries (with qkv)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (kind == 2) {  // queries: the rotary embedding only
+    const long idx = (long)blockIdx.x * kPackWarps + warp;
+    if (idx >= (long)(pa.BH / pa.h_kv) * pa.h_q) return;  // whole warps only
+    const long b = idx / pa.h_q, h = idx % pa.h_q;
+    const float4 r4 = *reinterpret_cast<const float4*>(pa.qkv + (b * (pa.h_q + 2 * pa.h_kv) + h) * kHeadDim +
+                                                       4 * lane);
+    float y[4] = {r4.x, r4.y, r4.z, r4.w};
+    rope_lane4(y, lane, pa.pos, pa.theta);
+    const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(y[0])) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(y[1])) << 16);
+    const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(y[2])) |
+                        ((uint32_t)__half_as_ushort(__float2half_rn(y[3])) << 16);
+    *reinterpret_cast<uint2*>(pa.q_out + idx * kHeadDim + 4 * lane) = make_uint2(lo, hi);
+    return;
+  }
+  const int is_value = kind;
   const uint16_t* __restrict__ x = pa.x[is_value];
   uint32_t* __restrict__ codes = pa.codes[is_value];
   uint32_t* __restrict__ refine = pa.refine[is_value];
   uint16_t* __restrict__ sz = pa.sz[is_value];
   const int BH = pa.BH, nt = pa.nt, t_max = pa.t_max, t0 = pa.t0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long idx = (long)blockIdx.x * kPackWarps + warp;
   if (idx >= (long)BH * nt) return;  // whole warps only
   const int t = (int)(idx % nt);
@@ -71,9 +113,20 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
   uint32_t* a = acc[warp];
   for (int i = lane; i < 8 * (B + R); i += 32) a[i] = 0;
   const int d0 = 4 * lane;
-  const uint2 raw = *reinterpret_cast<const uint2*>(x + (bh * nt + t) * kHeadDim + d0);
-  double v[4] = {h2d((uint16_t)(raw.x & 0xffff)), h2d((uint16_t)(raw.x >> 16)),
-                 h2d((uint16_t)(raw.y & 0xffff)), h2d((uint16_t)(raw.y >> 16))};
+  double v[4];
+  if (pa.qkv) {  // the one token from its projection row: key turned, both rounded to fp16
+    const long b = bh / pa.h_kv, g = bh % pa.h_kv;
+    const float4 r4 = *reinterpret_cast<const float4*>(
+        pa.qkv + (b * (pa.h_q + 2 * pa.h_kv) + pa.h_q + (long)is_value * pa.h_kv + g) * kHeadDim + d0);
+    float y[4] = {r4.x, r4.y, r4.z, r4.w};
+    if (!is_value) rope_lane4(y, lane, pa.pos, pa.theta);
+#pragma unroll
+    for (int i = 0; i < 4; i++) v[i] = (double)f16_round(y[i]);
+  } else {
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + (bh * nt + t) * kHeadDim + d0);
+    v[0] = h2d((uint16_t)(raw.x & 0xffff)), v[1] = h2d((uint16_t)(raw.x >> 16));
+    v[2] = h2d((uint16_t)(raw.y & 0xffff)), v[3] = h2d((uint16_t)(raw.y >> 16));
+  }
   double lo, hi;
   group_minmax(v, d0, lo, hi);
   const Grid16 g = group_grid(lo, hi, B);
@@ -153,26 +206,37 @@ __global__ void unpack_kv_kernel(const uint32_t* __restrict__ codes,
 
 template <int B, int R>
 sf_status launch_pack(const PackArgs& pa, int kinds, cudaStream_t s) {
-  const long total = (long)pa.BH * pa.nt;
+  long total = (long)pa.BH * pa.nt;
+  if (pa.qkv && (long)(pa.BH / pa.h_kv) * pa.h_q > total) total = (long)(pa.BH / pa.h_kv) * pa.h_q;
   SF_CUDA(launch_pdl(pack_kv_kernel<B, R>, dim3((unsigned)((total + kPackWarps - 1) / kPackWarps), kinds),
                      dim3(kPackWarps * 32), 0, s, pa));
   return SF_OK;
 }
 
-sf_status pack_both(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0, int nt, cudaStream_t s) {
-  PackArgs pa;
-  pa.x[0] = k, pa.x[1] = v;
-  pa.codes[0] = (uint32_t*)kv->kb, pa.codes[1] = (uint32_t*)kv->vb;
-  pa.refine[0] = (uint32_t*)kv->kr, pa.refine[1] = (uint32_t*)kv->vr;
-  pa.sz[0] = kv->ksz, pa.sz[1] = kv->vsz;
-  pa.BH = kv->batch * kv->h_kv, pa.nt = nt, pa.t_max = kv->t_max, pa.t0 = t0;
-  pa.first_kind = k ? 0 : 1;
-  const int kinds = (k ? 1 : 0) + (v ? 1 : 0);
-  if (kinds == 0) return SF_OK;
+sf_status launch_pack_any(const sf_kv* kv, const PackArgs& pa, int kinds, cudaStream_t s) {
   if (kv->b == 2 && kv->r == 2) return launch_pack<2, 2>(pa, kinds, s);
   if (kv->b == 2 && kv->r == 1) return launch_pack<2, 1>(pa, kinds, s);
   if (kv->b == 4 && kv->r == 2) return launch_pack<4, 2>(pa, kinds, s);
   return launch_pack<4, 1>(pa, kinds, s);
+}
+
+PackArgs pack_args(const sf_kv* kv, int t0, int nt) {
+  PackArgs pa = {};
+  pa.codes[0] = (uint32_t*)kv->kb, pa.codes[1] = (uint32_t*)kv->vb;
+  pa.refine[0] = (uint32_t*)kv->kr, pa.refine[1] = (uint32_t*)kv->vr;
+  pa.sz[0] = kv->ksz, pa.sz[1] = kv->vsz;
+  pa.BH = kv->batch * kv->h_kv, pa.nt = nt, pa.t_max = kv->t_max, pa.t0 = t0;
+  pa.h_kv = kv->h_kv;
+  return pa;
+}
+
+sf_status pack_both(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0, int nt, cudaStream_t s) {
+  PackArgs pa = pack_args(kv, t0, nt);
+  pa.x[0] = k, pa.x[1] = v;
+  pa.first_kind = k ? 0 : 1;
+  const int kinds = (k ? 1 : 0) + (v ? 1 : 0);
+  if (kinds == 0) return SF_OK;
+  return launch_pack_any(kv, pa, kinds, s);
 }
 
 }  // namespace
@@ -190,6 +254,21 @@ extern "C" sf_status sf_kv_pack_tokens(const sf_kv* kv, const uint16_t* k, const
   SF_REQUIRE(!v || aligned16(v), "v must be 16-byte aligned");
   if (nt == 0) return SF_OK;
   return pack_both(kv, k, v, t0, nt, as_stream(stream));
+}
+
+extern "C" sf_status sf_kv_append_rope(const sf_kv* kv, const float* qkv, int h_q, int pos, float theta,
+                                       int t, uint16_t* q, sf_stream_t stream) {
+  sf_status st = check_kv(kv);
+  if (st != SF_OK) return st;
+  SF_REQUIRE(t >= 0 && t < kv->t_max, "t=%d outside [0, t_max=%d)", t, kv->t_max);
+  SF_REQUIRE(pos >= 0, "pos=%d < 0", pos);
+  SF_REQUIRE(h_q > 0 && h_q % kv->h_kv == 0, "h_q=%d must be a positive multiple of h_kv=%d", h_q, kv->h_kv);
+  SF_REQUIRE(qkv && aligned16(qkv), "qkv must be a non-null 16-byte aligned device pointer");
+  SF_REQUIRE(q && aligned16(q), "q must be a non-null 16-byte aligned device pointer");
+  PackArgs pa = pack_args(kv, t, 1);
+  pa.qkv = qkv, pa.q_out = q, pa.h_q = h_q, pa.pos = pos, pa.theta = (double)theta;
+  pa.first_kind = 0;
+  return launch_pack_any(kv, pa, 3, as_stream(stream));
 }
 
 extern "C" sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* qb,

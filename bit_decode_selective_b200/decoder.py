@@ -94,9 +94,6 @@ class Decoder:
         self.x_attn = [f16(B, cfg.hidden) for _ in range(2)]
         self.qkv_out = f32(B, shp["qkv"][0])
         self.q = f16(B, cfg.h_q, cfg.d)
-        self.k_new = f16(B, cfg.h_kv, 1, cfg.d)
-        self.v_new = f16(B, cfg.h_kv, 1, cfg.d)
-        self.attn = f32(B, cfg.h_q, cfg.d)
         self.x_o = [f16(B, cfg.h_q * cfg.d) for _ in range(2)]
         self.o_out = f32(B, cfg.hidden)
         self.x_mlp = [f16(B, cfg.hidden) for _ in range(2)]
@@ -252,15 +249,14 @@ class Decoder:
             self._prepare(l, "qkv", x_attn, main)
             self._lead(l, "qkv", x_attn, main)
             self._proj(l, "qkv", x_attn, self.qkv_out, slot, main)
-            check(abi.sf_rope_split(_p(self.qkv_out), B, cfg.h_q, cfg.h_kv, cfg.d, T, cfg.theta, _p(self.q),
-                                    _p(self.k_new), _p(self.v_new), _s(main)), "sf_rope_split")
             kv = L["kv"]
-            check(abi.sf_kv_pack_tokens(ctypes.byref(kv.desc), _p(self.k_new), _p(self.v_new), T, 1, _s(main)),
-                  "sf_kv_pack_tokens")
-            check(abi.sf_kv_attend_selective(ctypes.byref(kv.desc), T + 1, _p(self.q), cfg.h_q, cfg.k_tok,
-                                             _p(self.tok_sel), None, _p(self.attn), _p(self.ws), self.ws.numel(),
-                                             _s(main)), "sf_kv_attend_selective")
-            check(abi.sf_cast_f16(_p(self.attn), B * cfg.h_q * cfg.d, _p(x_o), _s(main)), "sf_cast_f16")
+            # rotary embedding of q and k and the new token's append, in one launch
+            check(abi.sf_kv_append_rope(ctypes.byref(kv.desc), _p(self.qkv_out), cfg.h_q, T, cfg.theta, T,
+                                        _p(self.q), _s(main)), "sf_kv_append_rope")
+            # attention over T + 1 tokens; its fp16 output is o's input
+            check(abi.sf_kv_attend_selective_f16(ctypes.byref(kv.desc), T + 1, _p(self.q), cfg.h_q, cfg.k_tok,
+                                                 _p(self.tok_sel), None, _p(x_o), _p(self.ws), self.ws.numel(),
+                                                 _s(main)), "sf_kv_attend_selective_f16")
             self._prepare(l, "o", x_o, main)
             self._lead(l, "o", x_o, main)
             self._proj(l, "o", x_o, self.o_out, slot, main, y_corr=self.delta if lagging else None)

@@ -222,6 +222,16 @@ SF_API sf_status sf_kv_bytes(int batch, int h_kv, int d, int t_max, int b, int r
 SF_API sf_status sf_kv_pack_tokens(const sf_kv* kv, const uint16_t* k, const uint16_t* v, int t0,
                             int nt, sf_stream_t stream);
 
+/* The decode step's new token from its qkv projection row, in one launch:
+ * the rotary embedding of q and k (as sf_rope_split: pairs (i, i + d/2),
+ * angle pos * theta^(-2i/d) in fp64), q written to q [batch][h_q][d] fp16,
+ * and k and v rounded to fp16 and stored at token t of every head exactly as
+ * sf_kv_pack_tokens stores them.  The same results as sf_rope_split followed
+ * by sf_kv_pack_tokens(kv, k, v, t, 1).
+ *   qkv [batch][(h_q + 2 h_kv) d] fp32; 0 <= t < t_max; h_q % h_kv == 0. */
+SF_API sf_status sf_kv_append_rope(const sf_kv* kv, const float* qkv, int h_q, int pos, float theta, int t,
+                                   uint16_t* q, sf_stream_t stream);
+
 /* Codes of tokens 0..t-1, for checking: which = 0 keys, 1 values;
  * qb, rho: [batch][h_kv][t][d] (rho nullable). */
 SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* qb, uint8_t* rho,
@@ -273,6 +283,13 @@ SF_API sf_status sf_kv_attend_selective(const sf_kv* kv, int t, const uint16_t* 
                                         void* ws, size_t ws_bytes, sf_stream_t stream);
 SF_API size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                                      int logits_given);
+
+/* sf_kv_attend_selective with out [batch][h_q][d] rounded to fp16 (nearest
+ * even) by the attention kernel itself: the decode step hands the attention
+ * output to the next projection in fp16.  Same workspace and errors. */
+SF_API sf_status sf_kv_attend_selective_f16(const sf_kv* kv, int t, const uint16_t* q, int h_q,
+                                            int k_tok, int32_t* sel, float* logits, uint16_t* out,
+                                            void* ws, size_t ws_bytes, sf_stream_t stream);
 
 /* Largest workspace sf_kv_attend_selective_static can serve (32 MiB). */
 #define SF_KV_STATIC_WS_BYTES (32u << 20)

@@ -10,8 +10,10 @@ import pytest
 import torch
 
 import oracle
-from bit_decode_selective_b200 import inputs
-from bit_decode_selective_b200.ops import KVCache, QuantWeights, select_channels
+import ctypes
+
+from bit_decode_selective_b200 import abi, inputs
+from bit_decode_selective_b200.ops import KVCache, QuantWeights, _p, select_channels
 
 pytestmark = pytest.mark.gpu
 
@@ -311,6 +313,53 @@ def test_kv_base_only_and_all_selected():
     refT = oracle.kv_attention(kc, vc, q, host(all_sel), 300, 2)
     assert np.abs(host(out0) - ref0).max() <= ATTN_MAX_ABS and rel_l2(host(out0), ref0) <= RTOL_L2
     assert np.abs(host(outT) - refT).max() <= ATTN_MAX_ABS and rel_l2(host(outT), refT) <= RTOL_L2
+
+
+@pytest.mark.parametrize("b,r,batch,t", [(2, 2, 1, 37), (4, 1, 2, 0), (2, 1, 3, 47)])
+def test_kv_append_rope_equals_rope_then_pack(b, r, batch, t):
+    """The fused rotary embedding + append of the decode step's token stores
+    the same codes, refinements and steps/offsets, and the same rotated q, as
+    the rotary embedding followed by the token pack (bit-exact)."""
+    h_q, h_kv, theta, pos = 32, 8, 500000.0, 32768 + t
+    rng = np.random.default_rng(300 + 10 * b + batch)
+    qkv = cu((rng.standard_normal((batch, (h_q + 2 * h_kv) * 128)) * 3).astype(np.float32))
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    c1, c2 = KVCache(batch, h_kv, 48, b, r), KVCache(batch, h_kv, 48, b, r)
+    q1 = torch.empty((batch, h_q, 128), dtype=torch.float16, device="cuda")
+    k1 = torch.empty((batch, h_kv, 1, 128), dtype=torch.float16, device="cuda")
+    v1 = torch.empty_like(k1)
+    abi.check(abi.sf_rope_split(_p(qkv), batch, h_q, h_kv, 128, pos, theta, _p(q1), _p(k1), _p(v1), s),
+              "sf_rope_split")
+    abi.check(abi.sf_kv_pack_tokens(ctypes.byref(c1.desc), _p(k1), _p(v1), t, 1, s), "sf_kv_pack_tokens")
+    q2 = torch.empty_like(q1)
+    abi.check(abi.sf_kv_append_rope(ctypes.byref(c2.desc), _p(qkv), h_q, pos, theta, t, _p(q2), s),
+              "sf_kv_append_rope")
+    torch.cuda.synchronize()
+    assert torch.equal(q1.view(torch.int16), q2.view(torch.int16))
+    for name in ("kb", "kr", "vb", "vr", "ksz", "vsz"):
+        assert torch.equal(getattr(c1, name), getattr(c2, name)), name
+    assert getattr(c2, "ksz").abs().sum().item() > 0  # the token was written
+
+
+def test_kv_attend_selective_f16_output():
+    """The fp16-output form equals the fp32 output rounded to fp16 (same kernels)."""
+    T, k_tok = 3000, 128
+    k, v, _ = inputs.kv_case(seed=31, t=T)
+    cache = KVCache(1, 8, (T + 15) // 16 * 16)
+    cache.pack_tokens(cu(f16bits(k)), cu(f16bits(v)), 0)
+    q = cu(f16bits(inputs.query(np.random.default_rng(32), 32, 128, 1)))
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    need = abi.sf_kv_attend_selective_workspace_bytes(ctypes.byref(cache.desc), T, 32, k_tok, 0)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    sel = torch.empty((1, 8, k_tok), dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 32, 128), dtype=torch.float32, device="cuda")
+    out16 = torch.empty((1, 32, 128), dtype=torch.float16, device="cuda")
+    abi.check(abi.sf_kv_attend_selective(ctypes.byref(cache.desc), T, _p(q), 32, k_tok, _p(sel), None, _p(out),
+                                         _p(ws), ws.numel(), s), "sf_kv_attend_selective")
+    abi.check(abi.sf_kv_attend_selective_f16(ctypes.byref(cache.desc), T, _p(q), 32, k_tok, _p(sel), None,
+                                             _p(out16), _p(ws), ws.numel(), s), "sf_kv_attend_selective_f16")
+    torch.cuda.synchronize()
+    assert torch.equal(out.half().view(torch.int16), out16.view(torch.int16))
 
 
 def test_kv_attention_8k_workload():
