@@ -50,6 +50,59 @@ __global__ void __launch_bounds__(1024) rmsnorm_residual_kernel(float* __restric
     x[row * n + i] = __half_as_ushort(__float2half_rn(hr[i] * inv));
 }
 
+// The same with the row held in registers: thread t owns float4 vectors t,
+// t + 1024, ... (VPT of them), all loads of h and the addends issued at once,
+// so the row costs one memory round trip and one block reduction.
+template <int VPT>
+__global__ void __launch_bounds__(1024) rmsnorm_residual_vec_kernel(float* __restrict__ h,
+                                                                    const float* __restrict__ add0,
+                                                                    const float* __restrict__ add1,
+                                                                    int n, float eps,
+                                                                    uint16_t* __restrict__ x) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float red[32];
+  const long row = blockIdx.x;
+  const int nv = n / 4;
+  float4* h4 = reinterpret_cast<float4*>(h + row * n);
+  const float4* a4 = add0 ? reinterpret_cast<const float4*>(add0 + row * n) : nullptr;
+  const float4* b4 = add1 ? reinterpret_cast<const float4*>(add1 + row * n) : nullptr;
+  float4 v[VPT], a[VPT], c[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; k++) {
+    const int i = threadIdx.x + 1024 * k;
+    const bool in = i < nv;
+    v[k] = in ? h4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    a[k] = in && a4 ? a4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    c[k] = in && b4 ? b4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPT; k++) {
+    const int i = threadIdx.x + 1024 * k;
+    v[k].x += a[k].x, v[k].y += a[k].y, v[k].z += a[k].z, v[k].w += a[k].w;
+    v[k].x += c[k].x, v[k].y += c[k].y, v[k].z += c[k].z, v[k].w += c[k].w;
+    if (i < nv) h4[i] = v[k];
+    ss = fmaf(v[k].x, v[k].x, ss);
+    ss = fmaf(v[k].y, v[k].y, ss);
+    ss = fmaf(v[k].z, v[k].z, ss);
+    ss = fmaf(v[k].w, v[k].w, ss);
+  }
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)n + eps);
+#pragma unroll
+  for (int k = 0; k < VPT; k++) {
+    const int i = threadIdx.x + 1024 * k;
+    if (i < nv) {
+      const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(v[k].x * inv)) |
+                          ((uint32_t)__half_as_ushort(__float2half_rn(v[k].y * inv)) << 16);
+      const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(v[k].z * inv)) |
+                          ((uint32_t)__half_as_ushort(__float2half_rn(v[k].w * inv)) << 16);
+      *reinterpret_cast<uint2*>(x + row * n + 4 * i) = make_uint2(lo, hi);
+    }
+  }
+}
+
 // qkv[b] = [q (h_q*d) | k (h_kv*d) | v (h_kv*d)] fp32 -> rotated q, k and v in
 // fp16 (rope_cos_sin / rope_first / rope_second).
 __global__ void rope_split_kernel(const float* __restrict__ qkv, int h_q, int h_kv, int d, int pos,
@@ -168,8 +221,17 @@ extern "C" sf_status sf_rmsnorm_residual(float* h, const float* add0, const floa
   SF_REQUIRE(h && x && batch > 0 && n > 0, "bad rmsnorm arguments");
   SF_REQUIRE(aligned16(h) && aligned16(x) && (!add0 || aligned16(add0)) && (!add1 || aligned16(add1)),
              "rmsnorm pointers must be 16-byte aligned");
-  SF_CUDA(launch_pdl(rmsnorm_residual_kernel, dim3(batch), dim3(1024), 0, as_stream(stream), h, add0, add1, n,
-                     eps, x));
+  cudaStream_t s = as_stream(stream);
+  // rows of up to 16,384 elements, a multiple of 4: held in registers
+  const int vpt = n % 4 == 0 ? (n / 4 + 1023) / 1024 : 0;
+  if (vpt == 1)
+    SF_CUDA(launch_pdl(rmsnorm_residual_vec_kernel<1>, dim3(batch), dim3(1024), 0, s, h, add0, add1, n, eps, x));
+  else if (vpt == 2)
+    SF_CUDA(launch_pdl(rmsnorm_residual_vec_kernel<2>, dim3(batch), dim3(1024), 0, s, h, add0, add1, n, eps, x));
+  else if (vpt >= 3 && vpt <= 4)
+    SF_CUDA(launch_pdl(rmsnorm_residual_vec_kernel<4>, dim3(batch), dim3(1024), 0, s, h, add0, add1, n, eps, x));
+  else
+    SF_CUDA(launch_pdl(rmsnorm_residual_kernel, dim3(batch), dim3(1024), 0, s, h, add0, add1, n, eps, x));
   return SF_OK;
 }
 

@@ -370,3 +370,36 @@ def test_kv_attention_8k_workload():
 def test_kv_attention_128k_workload():
     """T = 131,072, top-1,024 tokens per KV head, split-K merged by log-sum-exp."""
     kv_parity(131072, 1024, splits=(0,), seed=3)
+
+
+# ---------------------------------------------------------------------------
+# decoder glue
+
+
+@pytest.mark.parametrize("n,adds", [(4096, 2), (8192, 1), (14336, 0), (1000, 2), (20000, 1)])
+def test_rmsnorm_residual(n, adds):
+    """h += add0 + add1 in fp32 (bit-exact with the same fp32 sums) and x =
+    fp16(h / rms(h)) within one fp16 step of the oracle's fp64 RMSNorm of the
+    same h (n = 1,000 and 20,000 take the looping kernel, the others the
+    register-resident one)."""
+    batch = 2
+    rng = np.random.default_rng(400 + n + adds)
+    h0 = (rng.standard_normal((batch, n)) * 3).astype(np.float32)
+    a0 = (rng.standard_normal((batch, n))).astype(np.float32)
+    a1 = (rng.standard_normal((batch, n)) * 0.5).astype(np.float32)
+    h = cu(h0)
+    x = torch.empty((batch, n), dtype=torch.float16, device="cuda")
+    d0, d1 = (cu(a0) if adds >= 1 else None), (cu(a1) if adds >= 2 else None)
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    abi.check(abi.sf_rmsnorm_residual(_p(h), _p(d0), _p(d1), batch, n, 1e-5, _p(x), s), "sf_rmsnorm_residual")
+    torch.cuda.synchronize()
+    want_h = h0.copy()
+    if adds >= 1:
+        want_h = want_h + a0
+    if adds >= 2:
+        want_h = want_h + a1
+    assert np.array_equal(host(h), want_h)
+    for b in range(batch):
+        ref = oracle.rmsnorm_f16(want_h[b].astype(np.float64)).view(np.float16).astype(np.float64)
+        got = host(x)[b].astype(np.float64)
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -10 + 2.0 ** -24)
