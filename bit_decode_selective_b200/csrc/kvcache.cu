@@ -59,8 +59,8 @@ struct PackArgs {
 
 // The lane's 4 consecutive elements (4 lane .. 4 lane + 3) of a 128-element
 // head row, turned by the rotary embedding: element e < 64 pairs with e + 64,
-// held by lane ^ 16.
-__device__ __forceinline__ void rope_lane4(float (&x)[4], int lane, int pos, double theta) {
+// held by lane ^ 16; cs[i] = (cos, sin) of pair i (rope_cos_sin).
+__device__ __forceinline__ void rope_lane4(float (&x)[4], int lane, const float2* cs) {
   float xp[4];
 #pragma unroll
   for (int i = 0; i < 4; i++) xp[i] = __shfl_xor_sync(0xffffffffu, x[i], 16);
@@ -68,9 +68,8 @@ __device__ __forceinline__ void rope_lane4(float (&x)[4], int lane, int pos, dou
 #pragma unroll
   for (int i = 0; i < 4; i++) {
     const int e = 4 * lane + i, k = first ? e : e - kHeadDim / 2;
-    float c, sn;
-    rope_cos_sin(pos, theta, k, kHeadDim, c, sn);
-    x[i] = first ? rope_first(x[i], xp[i], c, sn) : rope_second(xp[i], x[i], c, sn);
+    const float2 t = cs[k];
+    x[i] = first ? rope_first(x[i], xp[i], t.x, t.y) : rope_second(xp[i], x[i], t.x, t.y);
   }
 }
 
@@ -84,6 +83,16 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
   pdl_wait();
   const int kind = pa.first_kind + blockIdx.y;  // 0 keys, 1 values, 2 queries (with qkv)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // the rotation of every pair, once per CTA (the same for all heads)
+  __shared__ float2 rope_cs[kHeadDim / 2];
+  if (pa.qkv && kind != 1) {
+    for (int i = threadIdx.x; i < kHeadDim / 2; i += blockDim.x) {
+      float c, sn;
+      rope_cos_sin(pa.pos, pa.theta, i, kHeadDim, c, sn);
+      rope_cs[i] = make_float2(c, sn);
+    }
+    __syncthreads();
+  }
   if (kind == 2) {  // queries: the rotary embedding only
     const long idx = (long)blockIdx.x * kPackWarps + warp;
     if (idx >= (long)(pa.BH / pa.h_kv) * pa.h_q) return;  // whole warps only
@@ -91,7 +100,7 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
     const float4 r4 = *reinterpret_cast<const float4*>(pa.qkv + (b * (pa.h_q + 2 * pa.h_kv) + h) * kHeadDim +
                                                        4 * lane);
     float y[4] = {r4.x, r4.y, r4.z, r4.w};
-    rope_lane4(y, lane, pa.pos, pa.theta);
+    rope_lane4(y, lane, rope_cs);
     const uint32_t lo = (uint32_t)__half_as_ushort(__float2half_rn(y[0])) |
                         ((uint32_t)__half_as_ushort(__float2half_rn(y[1])) << 16);
     const uint32_t hi = (uint32_t)__half_as_ushort(__float2half_rn(y[2])) |
@@ -119,7 +128,7 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
     const float4 r4 = *reinterpret_cast<const float4*>(
         pa.qkv + (b * (pa.h_q + 2 * pa.h_kv) + pa.h_q + (long)is_value * pa.h_kv + g) * kHeadDim + d0);
     float y[4] = {r4.x, r4.y, r4.z, r4.w};
-    if (!is_value) rope_lane4(y, lane, pa.pos, pa.theta);
+    if (!is_value) rope_lane4(y, lane, rope_cs);
 #pragma unroll
     for (int i = 0; i < 4; i++) v[i] = (double)f16_round(y[i]);
   } else {
