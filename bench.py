@@ -8,7 +8,7 @@ intermediate 14336, 32 query / 8 KV heads of 128, vocab 128256 (fp16 LM head);
 channels refined per projection; 2-bit KV cache + 2 refinement bits over
 32,768 cached tokens with the top 512 tokens refined per KV head; weight
 refinement rows in pinned host memory, staged with fetch lead and lag of one
-layer on a side stream.  Batch 1.  Weights, caches and inputs are seeded
+layer on two staging streams.  Batch 1.  Weights, caches and inputs are seeded
 synthetic data of those shapes (N(0, 0.02) weights, N(0, 1) activations and
 keys/values with 4 key outlier channels per head).
 
@@ -224,6 +224,35 @@ def gemv_roofline(dec, steps, warmup, hbm_peak):
             "launches_per_step": launches}
 
 
+def base_only_ms(dec, hidden, s, steps, warmup):
+    """ms per step of the same decoder with channel refinement switched off
+    (kch = 0), captured as its own graph on stream s."""
+    import torch
+
+    kch = dec.cfg.kch
+    dec.cfg.kch = 0
+    try:
+        with torch.cuda.stream(s):
+            dec.step(hidden)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                dec.step(hidden)
+            for _ in range(warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(steps):
+                g.replay()
+            e1.record(s)
+            torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) / steps
+    finally:
+        dec.cfg.kch = kch
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
 
@@ -278,6 +307,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         ms_e2e = f0.elapsed_time(f1) / args.steps
         roof = gemv_roofline(dec, max(3, args.steps // 5), max(3, args.warmup), hbm_peak)
+        ms_base = base_only_ms(dec, hidden, s, max(3, args.steps // 2), args.warmup)
     roof["peak_kind"] = peak_kind
     if world > 1:
         t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
@@ -299,6 +329,9 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": ms_e2e * 1e3 / tokens, "unit": UNIT,
                 "h2d_bytes_per_step": hidden.numel() * 2, "d2h_bytes_per_step": dec.logits.numel() * 4},
         "gpu_launches": (n_kernels * args.steps) if n_kernels else None,
+        "base_only": {"ms_per_step": ms_base, "refined_over_base_throughput": ms_base / ms,
+                      "what": "the same step with no channel refinement (kch = 0: no selection, staging or "
+                              "correction of the weights; the KV path unchanged), its own graph"},
         "clocks": clocks.summary(),
     }
     if rank == 0:

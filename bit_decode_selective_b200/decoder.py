@@ -9,7 +9,7 @@ and the order of the calls.  The call order implements the schedule of
     highest-scoring tokens per KV head;
   the-map-app-also-loads-tiles paragraph -- refinement rows live in host RAM;
     fetch lead (1 layer) selects a projection's channels from the previous
-    layer's activation and starts the row transfer on a side stream while the
+    layer's activation and starts the row transfer on a staging stream while the
     layers in between compute; fetch lag (1 layer) applies the residual-writing
     projections' (o, down) corrections at the start of the next layer.  With
     the rows staged a layer ahead, o's projection computes its correction in
@@ -168,7 +168,7 @@ class Decoder:
 
     def _stage(self, layer, name, slot):
         """Copy layer `layer`'s rows of the selection in `slot` into staging
-        slot `slot` on the side stream (enqueued after the selection)."""
+        slot `slot` on the projection's staging stream (after the selection)."""
         check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
                                        _p(self.sel[name][slot]), self.B * self.n_sel[name],
                                        _p(self.slots[name][slot]), _s(self.stage_stream[name]), None),
@@ -222,7 +222,7 @@ class Decoder:
 
     def _lead(self, layer, name, x, main):
         """Fetch lead: select (layer + 1)'s channels from this activation and
-        start their transfer on the side stream."""
+        start their transfer on the projection's staging stream."""
         cfg = self.cfg
         if cfg.kch == 0 or not cfg.lead or layer + 1 >= cfg.n_layers:
             return
