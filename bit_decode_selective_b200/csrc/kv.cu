@@ -496,10 +496,13 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
 // copies.  Equal scores rank the lower token first; the selected tokens are
 // written in ascending order and also handed, by position, to the CTA that
 // refines them.  Each CTA then copies its share of the selected tokens' codes
-// and scales into shared memory with cp.async in one go, refines them one warp
-// per token (swapping each token's base contribution for its refined one,
-// relative to the head's softmax maximum), sums an interleaved share of the
-// base partial records, and CTA h merges query head h.
+// and scales into shared memory with cp.async in one go and refines them, each
+// warp four tokens together (swapping each token's base contribution for its
+// refined one, relative to the head's softmax maximum; the refined logits of
+// the warp's (token, head) slots summed by one transposed butterfly, each
+// warp's sums kept in its own slot rather than added with shared-memory
+// atomics), sums an interleaved share of the base partial records, and CTA h
+// merges query head h.
 
 constexpr int kPostThreads = 512;
 constexpr int kPostMaxTok = 16640;  // tokens per CTA scored in shared memory (cluster of 8)

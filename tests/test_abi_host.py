@@ -91,3 +91,24 @@ def test_split_gemv_checks(L):
     assert abi.sf_gemv_refined_split(ctypes.byref(wq), p16, 1, 1024, 32, p16, None, ctypes.c_void_p(4096),
                                      ctypes.c_void_p(4096 + 1024), None) == abi.SF_ERR_INVALID_ARG
     assert b"overlap" in abi.sf_last_error()
+
+
+def test_decode_step_forms_reject_before_launch(L):
+    p16 = ctypes.c_void_p(16)
+    kv = abi.sf_kv(1, 8, 128, 8192, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    # the new token's slot must lie inside the cache, h_q a multiple of h_kv, pointers aligned
+    assert abi.sf_kv_append_rope(ctypes.byref(kv), p16, 32, 0, 500000.0, 8192, p16, None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_kv_append_rope(ctypes.byref(kv), p16, 30, 0, 500000.0, 5, p16, None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_kv_append_rope(ctypes.byref(kv), ctypes.c_void_p(20), 32, 0, 500000.0, 5, p16, None) \
+        == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_kv_append_rope(ctypes.byref(kv), p16, 32, -1, 500000.0, 5, p16, None) == abi.SF_ERR_INVALID_ARG
+    # the fp16-output attention needs its output
+    assert abi.sf_kv_attend_selective_f16(ctypes.byref(kv), 100, p16, 32, 8, p16, None, None, p16, 1 << 20,
+                                          None) == abi.SF_ERR_INVALID_ARG
+    # the correction alone: nothing to do without a selection budget, a selection otherwise
+    wq = abi.sf_wq(4096, 4096, 2, 2, 128, 16, 16, 16)
+    assert abi.sf_gemv_correction(ctypes.byref(wq), p16, 1, 1024, 0, None, None, p16, None) == 0
+    assert abi.sf_gemv_correction(ctypes.byref(wq), p16, 1, 1024, 32, None, None, p16, None) \
+        == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_gemv_correction(ctypes.byref(wq), p16, 1, 1024, 32, p16, None, None, None) \
+        == abi.SF_ERR_INVALID_ARG
