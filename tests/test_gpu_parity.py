@@ -403,3 +403,33 @@ def test_rmsnorm_residual(n, adds):
         ref = oracle.rmsnorm_f16(want_h[b].astype(np.float64)).view(np.float16).astype(np.float64)
         got = host(x)[b].astype(np.float64)
         assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -10 + 2.0 ** -24)
+
+
+# ---------------------------------------------------------------------------
+# refinement staging
+
+
+@pytest.mark.parametrize("rows,row_bytes,n_sel", [(4096, 7168, 128), (14336, 1024, 448), (1024, 16, 1000),
+                                                  (512, 1536, 3)])
+def test_stage_refinements_bit_exact(rows, row_bytes, n_sel):
+    """Rows named by a device index array, read from mapped pinned host memory,
+    land in order in the device slot (duplicates and unsorted indices too);
+    the host-index form (one copy per run of consecutive rows) gives the same."""
+    rng = np.random.default_rng(rows + n_sel)
+    host_rows = torch.from_numpy(rng.integers(0, 256, rows * row_bytes, dtype=np.uint8)).pin_memory()
+    sel_h = rng.integers(0, rows, n_sel).astype(np.int32)
+    sel_h[: n_sel // 2] = np.sort(sel_h[: n_sel // 2])  # runs of consecutive rows for the host form
+    sel = cu(sel_h)
+    dst = torch.empty(n_sel * row_bytes, dtype=torch.uint8, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    abi.check(abi.sf_stage_refinements(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, _p(sel), n_sel, _p(dst),
+                                       s, None), "sf_stage_refinements")
+    dst2 = torch.empty_like(dst)
+    sel_c = np.ascontiguousarray(sel_h)
+    abi.check(abi.sf_stage_refinements_host(ctypes.c_void_p(host_rows.data_ptr()), row_bytes,
+                                            sel_c.ctypes.data_as(ctypes.c_void_p), n_sel, _p(dst2), s, None),
+              "sf_stage_refinements_host")
+    torch.cuda.synchronize()
+    want = host_rows.view(rows, row_bytes)[torch.from_numpy(sel_h).long()].reshape(-1)
+    assert torch.equal(dst.cpu(), want)
+    assert torch.equal(dst2.cpu(), want)
