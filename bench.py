@@ -224,6 +224,24 @@ def gemv_roofline(dec, steps, warmup, hbm_peak):
             "launches_per_step": launches}
 
 
+def max_over_ranks(values, world, device):
+    """Each of `values` (per-rank times) maximised over the ranks: the job is
+    as slow as its slowest replica.  world 1: unchanged."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_us_per_token(ms_per_step, world):
+    """Microseconds per token over the tokens of all replicas: every rank
+    decodes BATCH tokens per step."""
+    return ms_per_step * 1e3 / (BATCH * world)
+
+
 def base_only_ms(dec, hidden, s, steps, warmup):
     """ms per step of the same decoder with channel refinement switched off
     (kch = 0), captured as its own graph on stream s."""
@@ -309,14 +327,10 @@ def run_ours(args, rank, world, local_rank):
         roof = gemv_roofline(dec, max(3, args.steps // 5), max(3, args.warmup), hbm_peak)
         ms_base = base_only_ms(dec, hidden, s, max(3, args.steps // 2), args.warmup)
     roof["peak_kind"] = peak_kind
-    if world > 1:
-        t = torch.tensor([ms, ms_e2e], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, ms_e2e = float(t[0]), float(t[1])
-    tokens = BATCH * world
+    ms, ms_e2e, ms_base = max_over_ranks([ms, ms_e2e, ms_base], world, device)
     step_bytes = decode_step_bytes(cfg, BATCH, T_CTX)
     res = {
-        "metric": METRIC, "value": ms * 1e3 / tokens, "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": job_us_per_token(ms, world), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": BATCH, "context_tokens": T_CTX, "parallelism": f"replicas x{world}",
@@ -326,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
                 "frac_of_8tbs": step_bytes / (ms / 1e3) / 1e9 / 8000.0,
                 "pcie_bytes_per_step": staged_bytes(cfg, BATCH)},
         "roofline": {**roof, "traffic": roof["bytes_per_launch"] * GEMV_TRAFFIC_PER_BYTE},
-        "e2e": {"value": ms_e2e * 1e3 / tokens, "unit": UNIT,
+        "e2e": {"value": job_us_per_token(ms_e2e, world), "unit": UNIT,
                 "h2d_bytes_per_step": hidden.numel() * 2, "d2h_bytes_per_step": dec.logits.numel() * 4},
         "gpu_launches": (n_kernels * args.steps) if n_kernels else None,
         "base_only": {"ms_per_step": ms_base, "refined_over_base_throughput": ms_base / ms,
