@@ -599,3 +599,49 @@ def test_oracle_decoder_lag_without_refinement_is_a_no_op(orc):
         dec.layer(W, kc, vc, T)
         outs.append(dec.finish(lm))
     assert np.array_equal(outs[0], outs[1])
+
+
+def _lag_case(orc, seed, zero):
+    """One small model (2 layers) with the projections in `zero` set to zero
+    weights; the final logits at lag 0 and lag 1 (lead 0, channels refined)."""
+    from oracle.decoder import OracleDecoder
+
+    rng = np.random.default_rng(seed)
+    H, I, h_q, h_kv, d, T = 512, 1024, 4, 2, 128, 9
+    h16 = rng.normal(0, 1, (1, H)).astype(np.float16)
+    shapes = {"qkv": ((h_q + 2 * h_kv) * d, H), "o": (H, h_q * d), "gate_up": (2 * I, H), "down": (H, I)}
+    layers = []
+    for _ in range(2):
+        W = {}
+        for n, s in shapes.items():
+            w = np.zeros(s, np.float32) if n in zero else rng.normal(0, 0.05, s).astype(np.float32)
+            W[n] = orc.quant_weights(w, 2, 2, 128)
+        layers.append((W, rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16),
+                       rng.normal(0, 1, (1, h_kv, T, d)).astype(np.float16)))
+    lm = rng.normal(0, 0.02, (50, H)).astype(np.float16)
+    outs = []
+    for lag in (0, 1):
+        dec = OracleDecoder(h16, h_q=h_q, h_kv=h_kv, d=d, chunk=256, kch=16, k_tok=3, lead=0, lag=lag)
+        for W, kc, vc in layers:
+            dec.layer(W, kc, vc, T)
+        outs.append(dec.finish(lm)[0])
+    return outs
+
+
+def test_oracle_decoder_lag_moves_o_correction_past_the_mlp(orc):
+    """Lag 1 holds o's correction back from the MLP input of its layer and adds
+    it to the residual before the next layer: with a zero MLP nothing reads the
+    residual in between, so lag 1 equals lag 0 (up to the order of the sums);
+    with a working MLP it does not (the MLP input differs)."""
+    same = _lag_case(orc, 71, zero=("gate_up", "down"))
+    assert np.allclose(same[0], same[1], rtol=1e-10, atol=1e-12)
+    differ = _lag_case(orc, 71, zero=())
+    assert not np.allclose(differ[0], differ[1], rtol=1e-6, atol=1e-9)
+
+
+def test_oracle_decoder_down_lag_lands_with_down(orc):
+    """Down's lagged correction enters the residual where down's own output
+    does (the next layer's start, or the final norm): with o zero (no o
+    correction to hold back), lag 1 equals lag 0 up to the order of the sums."""
+    outs = _lag_case(orc, 72, zero=("o",))
+    assert np.allclose(outs[0], outs[1], rtol=1e-10, atol=1e-12)
