@@ -110,7 +110,7 @@ class Decoder:
                               for _ in range(2)] for n in PROJ}
         else:
             self.slots = None
-        # prepared activations of the GEMV in flight (sized for the widest input)
+        # the GEMV's workspace (its size query returns 0 today; sized for the widest input)
         kmax = max(kk for _, _, kk in cfg.shapes())
         wq = abi.sf_wq(128, kmax, cfg.w_bits, cfg.w_refine, cfg.group, None, None, None)
         self.gemv_ws = torch.empty(max(abi.sf_gemv_workspace_bytes(ctypes.byref(wq), B, cfg.chunk, cfg.kch), 16),
