@@ -77,9 +77,9 @@ _SIGNATURES = {
     "sf_cast_f16": ([c_void_p, c_size_t, c_void_p, c_void_p], c_int),
     "sf_widen_f16": ([c_void_p, c_size_t, c_void_p, c_void_p], c_int),
     "sf_gemv_f16": ([c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p], c_int),
-    "sf_stage_refinements": ([c_void_p, c_size_t, c_void_p, c_int, c_void_p, c_void_p, c_void_p],
-                             c_int),
-    "sf_stage_refinements_host": ([c_void_p, c_size_t, c_void_p, c_int, c_void_p, c_void_p,
+    "sf_stage_refinements": ([c_void_p, c_size_t, c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                              c_void_p], c_int),
+    "sf_stage_refinements_host": ([c_void_p, c_size_t, c_int, c_void_p, c_int, c_void_p, c_void_p,
                                    c_void_p], c_int),
 }
 

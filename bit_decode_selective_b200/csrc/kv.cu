@@ -509,6 +509,8 @@ constexpr int kPostMaxTok = 16640;  // tokens per CTA scored in shared memory (c
 constexpr int kPostCl = 8;
 constexpr int kPostStage = 64;      // selected tokens staged in shared memory at a time
 constexpr int kPostMaxSel = 512;    // selected tokens per CTA (k_tok <= 4096)
+constexpr int kMaxKTok = 4096;      // the largest k_tok every attention entry point accepts
+static_assert(kPostCl * kPostMaxSel == kMaxKTok, "the cluster's selection buffers must hold k_tok tokens");
 constexpr int kHistBins = 512;
 // a warp's share of one staging batch, times 8 query heads, fits its 32 lanes
 static_assert(kPostStage / (kPostThreads / 32) * 8 <= 32, "staging batch too large for the lane layout");
@@ -661,7 +663,7 @@ __global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
           float sc = 0.f;
 #pragma unroll
           for (int h = 0; h < GQP; h++)
-            if (h < gq) sc += __expf(l[h][e] - Mh[h]) * invZ[h];
+            if (h < gq) sc += expf(l[h][e] - Mh[h]) * invZ[h];  // full-accuracy exp: the score decides the selection
           if (a.scores) a.scores[((long)bat * a.h_kv + g) * a.T + t0 + i] = sc;
           keys[i] = __float_as_uint(sc);
         }
@@ -1026,6 +1028,16 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   return P;
 }
 
+// k_tok of every entry point: at most t, at most kMaxKTok (each of the kPostCl
+// CTAs of a head's cluster holds up to kPostMaxSel of the selected tokens), and
+// at least 1 unless a base-only call (allow_zero) is meant.
+sf_status check_ktok(int k_tok, int t, bool allow_zero) {
+  SF_REQUIRE(k_tok >= (allow_zero ? 0 : 1) && k_tok <= t, "k_tok=%d outside [%d, t=%d]", k_tok,
+             allow_zero ? 0 : 1, t);
+  SF_UNSUPPORTED(k_tok <= kMaxKTok, "k_tok=%d above %d", k_tok, kMaxKTok);
+  return SF_OK;
+}
+
 sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
   SF_REQUIRE(t >= 1 && t <= kv->t_max, "t=%d outside [1, t_max=%d]", t, kv->t_max);
   SF_REQUIRE(q && aligned16(q), "q must be a non-null 16-byte aligned device pointer");
@@ -1150,7 +1162,8 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
-  SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
+  st = check_ktok(k_tok, t, false);
+  if (st != SF_OK) return st;
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(!scores || aligned16(scores), "scores must be 16-byte aligned");
@@ -1180,7 +1193,8 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
-  SF_REQUIRE(k_tok >= 0 && k_tok <= t, "k_tok=%d outside [0, t=%d]", k_tok, t);
+  st = check_ktok(k_tok, t, true);
+  if (st != SF_OK) return st;
   SF_REQUIRE(k_tok == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
   SF_REQUIRE(n_splits >= 0, "n_splits=%d < 0", n_splits);
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
@@ -1215,7 +1229,8 @@ sf_status attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q, i
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
-  SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
+  st = check_ktok(k_tok, t, false);
+  if (st != SF_OK) return st;
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE((out || out16) && (!out || aligned16(out)) && (!out16 || aligned16(out16)),
@@ -1306,7 +1321,8 @@ extern "C" sf_status sf_kv_attend_selective_static(const sf_kv* kv, int t, const
   if (st != SF_OK) return st;
   st = check_q(kv, t, q, h_q);
   if (st != SF_OK) return st;
-  SF_REQUIRE(k_tok >= 1 && k_tok <= t, "k_tok=%d outside [1, t=%d]", k_tok, t);
+  st = check_ktok(k_tok, t, false);
+  if (st != SF_OK) return st;
   const size_t need = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0).total;
   if (need > kStaticWsBytes) {
     set_error("workspace of %zu bytes needed (batch=%d, h_q=%d, t=%d, k_tok=%d, logits %s) is above "

@@ -26,9 +26,11 @@ constexpr int kGatherBlocksMax = 64;    // 64 x 8 KB in flight keeps the host li
 // as long as the transfer; each fits beside a whole-SM kernel's CTA (at most
 // kSideRegs registers, no shared memory), so the transfer never delays one.
 static_assert(kGatherThreads * 32 <= kSideRegs, "a gather CTA must fit in the room left for staging");
+// An index outside [0, n_rows) is never dereferenced: its row is filled with
+// zeros and counted in *bad (when given), which the host can read back.
 __global__ void __maxnreg__(32) gather_rows_kernel(const uint4* __restrict__ src, size_t row_vecs,
-                                                   const int32_t* __restrict__ sel, int n_sel,
-                                                   uint4* __restrict__ dst) {
+                                                   const int32_t* __restrict__ sel, int n_sel, int n_rows,
+                                                   uint4* __restrict__ dst, int32_t* __restrict__ bad) {
   const size_t total = (size_t)n_sel * row_vecs;
   const size_t step = (size_t)gridDim.x * kGatherThreads * kVec;
   for (size_t base = (size_t)blockIdx.x * kGatherThreads * kVec + threadIdx.x; base < total; base += step) {
@@ -36,9 +38,15 @@ __global__ void __maxnreg__(32) gather_rows_kernel(const uint4* __restrict__ src
 #pragma unroll
     for (int u = 0; u < kVec; u++) {
       const size_t i = base + (size_t)u * kGatherThreads;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
       if (i < total) {
         const size_t j = i / row_vecs, c = i - j * row_vecs;
-        v[u] = src[(size_t)sel[j] * row_vecs + c];
+        const int32_t row = sel[j];
+        if (row >= 0 && row < n_rows) {
+          v[u] = src[(size_t)row * row_vecs + c];
+        } else if (bad && c == 0) {
+          atomicAdd(bad, 1);  // once per bad index
+        }
       }
     }
 #pragma unroll
@@ -54,10 +62,12 @@ __global__ void __maxnreg__(32) gather_rows_kernel(const uint4* __restrict__ src
 
 using namespace sf;
 
-extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes,
-                                          const int32_t* sel, int n_sel, void* dst,
+extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, int n_rows,
+                                          const int32_t* sel, int n_sel, void* dst, int32_t* bad,
                                           sf_stream_t stream, sf_event_t done) {
   SF_REQUIRE(host_rows && dst && sel, "host_rows, sel and dst must be non-null");
+  SF_REQUIRE(n_rows >= 1, "n_rows=%d < 1", n_rows);
+  SF_REQUIRE(!bad || (reinterpret_cast<uintptr_t>(bad) & 3u) == 0, "bad must be 4-byte aligned");
   SF_REQUIRE(row_bytes > 0 && row_bytes % 16 == 0, "row_bytes=%zu must be a multiple of 16",
              row_bytes);
   SF_REQUIRE(aligned16(host_rows) && aligned16(dst) && aligned16(sel),
@@ -73,19 +83,24 @@ extern "C" sf_status sf_stage_refinements(const void* host_rows, size_t row_byte
     size_t blocks = (vecs + kGatherThreads * kVec - 1) / (kGatherThreads * kVec);
     if (blocks > (size_t)kGatherBlocksMax) blocks = kGatherBlocksMax;
     gather_rows_kernel<<<(unsigned)blocks, kGatherThreads, 0, s>>>((const uint4*)attr.devicePointer,
-                                                                   (size_t)(row_bytes / 16), sel, n_sel, (uint4*)dst);
+                                                                   (size_t)(row_bytes / 16), sel, n_sel, n_rows,
+                                                                   (uint4*)dst, bad);
     SF_LAUNCHED();
   }
   if (done) SF_CUDA(cudaEventRecord((cudaEvent_t)done, s));
   return SF_OK;
 }
 
-extern "C" sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes,
+extern "C" sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes, int n_rows,
                                                const int32_t* sel_host, int n_sel, void* dst,
                                                sf_stream_t stream, sf_event_t done) {
   SF_REQUIRE(host_rows && dst && (sel_host || n_sel == 0), "null argument");
   SF_REQUIRE(row_bytes > 0, "row_bytes must be positive");
   SF_REQUIRE(n_sel >= 0, "n_sel=%d < 0", n_sel);
+  SF_REQUIRE(n_rows >= 1, "n_rows=%d < 1", n_rows);
+  for (int j = 0; j < n_sel; j++)  // every index is checked before anything is enqueued
+    SF_REQUIRE(sel_host[j] >= 0 && sel_host[j] < n_rows, "row index %d (entry %d) outside [0, %d)",
+               sel_host[j], j, n_rows);
   cudaStream_t s = as_stream(stream);
   const char* src = (const char*)host_rows;
   char* out = (char*)dst;
@@ -93,7 +108,6 @@ extern "C" sf_status sf_stage_refinements_host(const void* host_rows, size_t row
   while (j < n_sel) {
     int run = 1;
     while (j + run < n_sel && sel_host[j + run] == sel_host[j] + run) run++;
-    SF_REQUIRE(sel_host[j] >= 0, "negative row index %d", sel_host[j]);
     SF_CUDA(cudaMemcpyAsync(out + (size_t)j * row_bytes, src + (size_t)sel_host[j] * row_bytes,
                             (size_t)run * row_bytes, cudaMemcpyHostToDevice, s));
     j += run;

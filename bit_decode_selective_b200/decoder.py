@@ -170,8 +170,8 @@ class Decoder:
         """Copy layer `layer`'s rows of the selection in `slot` into staging
         slot `slot` on the projection's staging stream (after the selection)."""
         check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
-                                       _p(self.sel[name][slot]), self.B * self.n_sel[name],
-                                       _p(self.slots[name][slot]), _s(self.stage_stream[name]), None),
+                                       self.shp[name][1], _p(self.sel[name][slot]), self.B * self.n_sel[name],
+                                       _p(self.slots[name][slot]), None, _s(self.stage_stream[name]), None),
               "sf_stage_refinements")
 
     def _side_select_stage(self, layer, name, x, slot, main):

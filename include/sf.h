@@ -246,8 +246,10 @@ SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* 
  *   q [batch][h_q][d] fp16;  sel [batch][h_kv][k_tok] int32.
  *   logits (nullable): receives the base logits [batch][h_q][t] fp32.
  *   scores (nullable): receives score [batch][h_kv][t] fp32.
- *   1 <= t <= t_max, 1 <= k_tok <= min(t, 4096), h_q % h_kv == 0,
- *   h_q / h_kv <= 8. */
+ *   1 <= t <= min(t_max, 133120), 1 <= k_tok <= min(t, 4096),
+ *   h_q % h_kv == 0, h_q / h_kv <= 8 (SF_ERR_UNSUPPORTED above the caps: the
+ *   per-head selection keeps every token's score, and the selected tokens, in
+ *   the shared memory of one 8-CTA cluster). */
 SF_API sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok,
                              int32_t* sel, float* logits, float* scores, void* ws,
                              size_t ws_bytes, sf_stream_t stream);
@@ -265,7 +267,8 @@ SF_API size_t sf_kv_score_select_workspace_bytes(const sf_kv* kv, int t, int h_q
  * merged by log-sum-exp.  The result does not depend on n_splits beyond fp32
  * rounding.
  *   sel [batch][h_kv][k_tok] (k_tok may be 0: base attention);
- *   out [batch][h_q][d] fp32. */
+ *   out [batch][h_q][d] fp32;
+ *   t, k_tok, h_q within the limits of sf_kv_score_select (k_tok >= 0). */
 SF_API sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* q, int h_q,
                                     const int32_t* sel, int k_tok, int n_splits, float* out,
                                     void* ws, size_t ws_bytes, sf_stream_t stream);
@@ -327,16 +330,23 @@ SF_API sf_status sf_kv_attend_selective_static(const sf_kv* kv, int t, const uin
  * (a selection made on the GPU, e.g. by sf_select_channels one layer early),
  * so no host round trip is needed.  host_rows must be page-locked host memory
  * mapped into the device address space (cudaHostAlloc with
- * cudaHostAllocMapped, or cudaHostRegister with cudaHostRegisterMapped);
- * row_bytes % 16 == 0. */
-SF_API sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, const int32_t* sel,
-                               int n_sel, void* dst, sf_stream_t stream, sf_event_t done);
+ * cudaHostAllocMapped, or cudaHostRegister with cudaHostRegisterMapped) that
+ * holds n_rows rows of row_bytes; row_bytes % 16 == 0.
+ * Since the indices are only known on the device, they are checked there: an
+ * index outside [0, n_rows) is not read; its destination row is filled with
+ * zeros and, when `bad` (nullable, a device int32) is given, *bad is
+ * incremented once per such index (the caller zeroes it and reads it back). */
+SF_API sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, int n_rows,
+                                      const int32_t* sel, int n_sel, void* dst, int32_t* bad,
+                                      sf_stream_t stream, sf_event_t done);
 
 /* Same copy with a HOST index array: one cudaMemcpyAsync per run of
- * consecutive indices.  host_rows must be pinned. */
-SF_API sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes,
-                                    const int32_t* sel_host, int n_sel, void* dst,
-                                    sf_stream_t stream, sf_event_t done);
+ * consecutive indices.  host_rows must be pinned and hold n_rows rows; every
+ * index is checked against [0, n_rows) before anything is enqueued
+ * (SF_ERR_INVALID_ARG otherwise). */
+SF_API sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes, int n_rows,
+                                           const int32_t* sel_host, int n_sel, void* dst,
+                                           sf_stream_t stream, sf_event_t done);
 
 /* ======================================================================== */
 /* Decoder-step glue (standard Llama operations around the refined ones)     */

@@ -75,7 +75,50 @@ def test_validation_rejects_before_launch(L):
                                   ctypes.c_void_p(16), ctypes.c_void_p(16), 8, None) == abi.SF_ERR_WORKSPACE
     assert abi.sf_kv_attend_selective(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, 0, ctypes.c_void_p(16),
                                       None, ctypes.c_void_p(16), None, 0, None) == abi.SF_ERR_INVALID_ARG
-    assert abi.sf_stage_refinements_host(None, 16, None, 1, None, None, None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_stage_refinements_host(None, 16, 4, None, 1, None, None, None) == abi.SF_ERR_INVALID_ARG
+
+
+def test_ktok_cap_every_attention_entry_point(L):
+    """k_tok above 4,096 is refused on the host by every attention call (each
+    of a head's 8 cluster CTAs holds at most 512 selected tokens), before any
+    launch or workspace lookup; 4,096 itself passes the k_tok check."""
+    p16 = ctypes.c_void_p(16)
+    kv = abi.sf_kv(1, 8, 128, 8192, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    t = 8000
+    assert abi.sf_kv_score_select(ctypes.byref(kv), t, p16, 32, 4097, p16, None, None, None, 0, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    assert b"4097" in abi.sf_last_error()
+    assert abi.sf_kv_attn_refined(ctypes.byref(kv), t, p16, 32, p16, 4097, 0, p16, None, 0, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), t, p16, 32, 4097, p16, None, p16, None, 0, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_attend_selective_f16(ctypes.byref(kv), t, p16, 32, 4097, p16, None, p16, None, 0, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_attend_selective_static(ctypes.byref(kv), t, p16, 32, 4097, p16, None, p16, None) \
+        == abi.SF_ERR_UNSUPPORTED
+    # at the cap the k_tok check passes and the call stops at the missing workspace instead
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), t, p16, 32, 4096, p16, None, p16, None, 0, None) \
+        == abi.SF_ERR_WORKSPACE
+
+
+def test_context_cap(L):
+    """t above 133,120 tokens is refused (the per-head scores live in one cluster's shared memory)."""
+    p16 = ctypes.c_void_p(16)
+    kv = abi.sf_kv(1, 8, 128, 140000, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), 133121, p16, 32, 64, p16, None, p16, None, 0, None) \
+        == abi.SF_ERR_UNSUPPORTED
+
+
+def test_stage_host_index_out_of_range(L):
+    """The host-index staging checks every index against n_rows before it enqueues a copy."""
+    p16 = ctypes.c_void_p(16)
+    sel = (ctypes.c_int32 * 3)(0, 2, 4)
+    assert abi.sf_stage_refinements_host(p16, 16, 4, sel, 3, p16, None, None) == abi.SF_ERR_INVALID_ARG
+    assert b"outside" in abi.sf_last_error()
+    sel = (ctypes.c_int32 * 2)(-1, 2)
+    assert abi.sf_stage_refinements_host(p16, 16, 4, sel, 2, p16, None, None) == abi.SF_ERR_INVALID_ARG
+    # the device-index form needs a row count
+    assert abi.sf_stage_refinements(p16, 16, 0, p16, 2, p16, None, None, None) == abi.SF_ERR_INVALID_ARG
 
 
 def test_split_gemv_checks(L):

@@ -422,14 +422,39 @@ def test_stage_refinements_bit_exact(rows, row_bytes, n_sel):
     sel = cu(sel_h)
     dst = torch.empty(n_sel * row_bytes, dtype=torch.uint8, device="cuda")
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    abi.check(abi.sf_stage_refinements(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, _p(sel), n_sel, _p(dst),
-                                       s, None), "sf_stage_refinements")
+    bad = torch.zeros(4, dtype=torch.int32, device="cuda")
+    abi.check(abi.sf_stage_refinements(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, rows, _p(sel), n_sel,
+                                       _p(dst), _p(bad), s, None), "sf_stage_refinements")
     dst2 = torch.empty_like(dst)
     sel_c = np.ascontiguousarray(sel_h)
-    abi.check(abi.sf_stage_refinements_host(ctypes.c_void_p(host_rows.data_ptr()), row_bytes,
+    abi.check(abi.sf_stage_refinements_host(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, rows,
                                             sel_c.ctypes.data_as(ctypes.c_void_p), n_sel, _p(dst2), s, None),
               "sf_stage_refinements_host")
     torch.cuda.synchronize()
     want = host_rows.view(rows, row_bytes)[torch.from_numpy(sel_h).long()].reshape(-1)
     assert torch.equal(dst.cpu(), want)
     assert torch.equal(dst2.cpu(), want)
+    assert bad[0].item() == 0
+
+
+def test_stage_refinements_out_of_range_index():
+    """Indices outside [0, n_rows) in the device array are not read: their rows
+    are zero-filled and counted in the error word; the valid ones still land."""
+    rows, row_bytes = 64, 256
+    rng = np.random.default_rng(5)
+    host_rows = torch.from_numpy(rng.integers(1, 256, rows * row_bytes, dtype=np.uint8)).pin_memory()
+    sel_h = np.array([3, 64, 10, -1, 63, 1 << 30], dtype=np.int32)
+    dst = torch.full((len(sel_h) * row_bytes,), 7, dtype=torch.uint8, device="cuda")
+    bad = torch.zeros(4, dtype=torch.int32, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    abi.check(abi.sf_stage_refinements(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, rows, _p(cu(sel_h)),
+                                       len(sel_h), _p(dst), _p(bad), s, None), "sf_stage_refinements")
+    torch.cuda.synchronize()
+    got = dst.cpu().view(len(sel_h), row_bytes)
+    src = host_rows.view(rows, row_bytes)
+    for j, i in enumerate(sel_h):
+        if 0 <= i < rows:
+            assert torch.equal(got[j], src[i])
+        else:
+            assert int(got[j].sum()) == 0
+    assert bad[0].item() == 3

@@ -385,6 +385,34 @@ def test_kv_logits_and_scores(orc, small_kv):
     assert (score > 0).all()
 
 
+def test_kv_scores_head_grouping_closed_form(orc):
+    """Query head h belongs to KV head h // (h_q / h_kv) ("which tiles count":
+    a KV head's score sums the attention of the query heads that share it).
+    Head h puts logit L on token h and 0 on every other token, so its softmax is
+    p_hot = e^L / (e^L + T - 1) on token h and p_cold = 1 / (e^L + T - 1)
+    elsewhere; KV head g's score is then, in closed form,
+    grp * p_cold + (p_hot - p_cold) on each of its own query heads' tokens.
+    A grouping by h % h_kv (or any other) puts the hot tokens elsewhere and fails."""
+    B, Hq, H, T, L = 2, 32, 8, 40, 3.0
+    grp = Hq // H
+    logits = np.zeros((B, Hq, T))
+    for b in range(B):
+        for h in range(Hq):
+            logits[b, h, h] = L
+    score = orc.kv_scores(logits, H)
+    den = np.exp(L) + (T - 1)
+    p_hot, p_cold = np.exp(L) / den, 1.0 / den
+    want = np.full((B, H, T), grp * p_cold)
+    for g in range(H):
+        for h in range(g * grp, (g + 1) * grp):
+            want[:, g, h] += p_hot - p_cold
+    assert np.allclose(score, want, rtol=1e-13, atol=1e-15)
+    # and the selection of each KV head's top grp tokens is exactly its own query heads' hot tokens
+    sel = orc.kv_select(score, grp)
+    for g in range(H):
+        assert list(sel[0, g]) == list(range(g * grp, (g + 1) * grp))
+
+
 def test_kv_select_brute_force(orc):
     rng = np.random.default_rng(41)
     for trial in range(30):
