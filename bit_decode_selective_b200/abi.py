@@ -29,6 +29,12 @@ class sf_wq(ctypes.Structure):
                 ("group", c_int32), ("base", c_void_p), ("refine", c_void_p), ("sz", c_void_p)]
 
 
+class sf_row_cache(ctypes.Structure):
+    _fields_ = [("capacity", c_int32), ("n_channels", c_int32), ("row_bytes", c_int32),
+                ("slot_of", c_void_p), ("channel_of", c_void_p), ("stamp", c_void_p), ("state", c_void_p),
+                ("work", c_void_p), ("max_sel", c_int32), ("rows", c_void_p)]
+
+
 class sf_kv(ctypes.Structure):
     _fields_ = [("batch", c_int32), ("h_kv", c_int32), ("d", c_int32), ("t_max", c_int32),
                 ("b", c_int32), ("r", c_int32), ("group", c_int32),
@@ -51,6 +57,7 @@ _SIGNATURES = {
                             c_void_p, c_void_p], c_int),
     "sf_gemv_refined_split": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                                c_void_p, c_void_p, c_void_p], c_int),
+    "sf_device_wait_timeouts": ([POINTER(ctypes.c_uint), c_int], c_int),
     "sf_kv_bytes": ([c_int] * 7 + [POINTER(c_size_t)] * 3, c_int),
     "sf_kv_pack_tokens": ([POINTER(sf_kv), c_void_p, c_void_p, c_int, c_int, c_void_p], c_int),
     "sf_kv_append_rope": ([POINTER(sf_kv), c_void_p, c_int, c_int, ctypes.c_float, c_int, c_void_p, c_void_p],
@@ -81,6 +88,9 @@ _SIGNATURES = {
                               c_void_p], c_int),
     "sf_stage_refinements_host": ([c_void_p, c_size_t, c_int, c_void_p, c_int, c_void_p, c_void_p,
                                    c_void_p], c_int),
+    "sf_row_cache_reset": ([POINTER(sf_row_cache), c_void_p], c_int),
+    "sf_stage_refinements_cached": ([c_void_p, c_size_t, c_int, c_void_p, c_int, c_int, POINTER(sf_row_cache),
+                                     c_int, c_void_p, c_void_p, c_void_p, c_void_p], c_int),
 }
 
 # Symbols every build must export (the header's declarations).
@@ -131,6 +141,7 @@ sf_gemv_refined = _call("sf_gemv_refined")
 sf_gemv_workspace_bytes = _call("sf_gemv_workspace_bytes")
 sf_gemv_correction = _call("sf_gemv_correction")
 sf_gemv_refined_split = _call("sf_gemv_refined_split")
+sf_device_wait_timeouts = _call("sf_device_wait_timeouts")
 sf_kv_bytes = _call("sf_kv_bytes")
 sf_kv_pack_tokens = _call("sf_kv_pack_tokens")
 sf_kv_unpack_codes = _call("sf_kv_unpack_codes")
@@ -151,3 +162,5 @@ sf_widen_f16 = _call("sf_widen_f16")
 sf_gemv_f16 = _call("sf_gemv_f16")
 sf_stage_refinements = _call("sf_stage_refinements")
 sf_stage_refinements_host = _call("sf_stage_refinements_host")
+sf_row_cache_reset = _call("sf_row_cache_reset")
+sf_stage_refinements_cached = _call("sf_stage_refinements_cached")

@@ -36,10 +36,14 @@ void clear_error();
   } while (0)
 
 // Check the last launch (or a runtime call) and turn a failure into SF_ERR_CUDA.
+// The runtime's record of a non-sticky error (a launch refused for its
+// resources, say) is cleared, so that it is not reported again by a later,
+// unrelated call.
 #define SF_CUDA(call)                                                           \
   do {                                                                          \
     cudaError_t e_ = (call);                                                    \
     if (e_ != cudaSuccess) {                                                    \
+      (void)cudaGetLastError();                                                 \
       ::sf::set_error("%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),   \
                       __FILE__, __LINE__);                                      \
       return SF_ERR_CUDA;                                                       \

@@ -9,94 +9,150 @@
 //     refinement's sub-bin inside the base bin:
 //       w~ = w^ + s * (2*rho + 1 - 2^r) / 2^(r+1).
 //   the-map-app-also-loads-tiles paragraph -- with fetch lag the correction
-//     of a projection is applied later than its base product; the
-//     correction-only kernel below computes it on its own.
+//     of a projection is applied later than its base product; the split form
+//     writes it to its own output and the correction-only kernel computes it
+//     on its own.
 //
 // Decomposition, per output row i (fp32 accumulation):
 //   y_i = sum_groups [ s_ig * sum_{c in g} x_c q_ic + m_ig * sum_{c in g} x_c ]
 //       + sum_{c selected} x_c * s_i,g(c) * (rho_ic + 1/2 - 2^(r-1)) / 2^r
 //
-// Activation prologue (in every CTA, after griddepcontrol.wait): each
-// 64-channel lane group of x becomes exact fixed point x = x_fix * 2^e with
-// |x_fix| < 2^21, split into three byte planes laid out in the order of the
-// code byte vectors below, plus the group's sums, in shared memory.
-
-// Base pass (HBM-bound: every resident code is read once).  One CTA of 16
-// warps per SM owns a contiguous, 4-aligned range of rows.  Its work is a list
-// of (2,048-channel segment, 4-row step) tasks split evenly over the warps; a
-// warp keeps the byte planes of its current segment in registers (a lane owns
-// 64 channels) and streams the codes of its rows through a per-lane cp.async
-// ring.  A lane turns 16 B of 2-bit codes into byte vectors with one AND per
-// four codes (codes at bit offsets 2 and 6 keep a factor 4 that is removed
-// once per row), takes integer dot products with dp4a (four code x byte
-// products per instruction) and combines the planes in 32-bit integers, so the
-// lane's partial dot product is exact.  Partial sums of four rows are reduced
-// across the warp with a transposed butterfly.
+// One CTA per SM owns a contiguous range of rows (a multiple of 4).
 //
-// Correction pass: a table of the selected channels (x_c, group, refinement
-// row) and the refinement words covering the CTA's rows are copied into shared
-// memory while the base pass streams (the base pass also keeps the rows'
-// (s, m) words), then each lane owns 1, 2 or 4 rows
-// and every warp walks a range of the table, summing x_c (rho_ic + 1/2 -
-// 2^(r-1)) / 2^r over each run of channels that share a scale group and
-// scaling each run once.
+// Producer warp: one lane streams the CTA's codes through a ring of shared
+// memory stages with 1-D bulk copies (cp.async.bulk, completion counted on an
+// mbarrier per stage), and copies the rows' (s, m) words once.  The weights do
+// not depend on earlier kernels, so these copies start before the grid
+// dependency wait and overlap the previous kernel's tail.  After the wait the
+// warp builds the correction tables (selected channel, x_c, group) and copies
+// the refinement words of the CTA's rows with cp.async.
+//
+// Compute warps: warp w owns the 2,048-channel segment w % segs (lane L: 64
+// consecutive channels) for every row whose index in its stage is congruent to
+// w / segs.  Its activations are turned once into fixed point
+// x = x_fix * 2^e per 64-channel lane block (e from the block's largest |x|,
+// |x_fix| < 2^20: every value within 2^9 of the block's largest is exact, the
+// rest round to 2^-20 of it) held as three byte planes in registers, in the
+// order of the code byte vectors: a 32-bit word of
+// 2-bit codes gives four byte vectors with one AND each (the codes at bit
+// offsets 2 and 6 of a byte carry a factor 4 that is folded into the scale),
+// dp4a takes four code x byte products per instruction, and the planes are
+// combined in 32-bit integers: the lane's partial dot product over its block is
+// exact for its fixed-point x.  Per row: s * 2^e * dot + m * sum(x), summed over
+// the warp with a transposed butterfly into a per-(row, segment) slot.
+//
+// Correction (after the base pass, all threads): a thread owns 4 consecutive
+// rows (the r bits of 4 rows never straddle a 32-bit word) and a share of the
+// selected channels; per channel it reads one refinement word and adds
+// x_c * (1 + rho/2^r) to a per-row run, and every run of channels in one scale
+// group is scaled once, s * (run - sum x_c (1 - off/2^r)) with
+// off = 1/2 - 2^(r-1).  The base pass leaves the scales group-major for it.
+// Every partial has its own slot, so the sums are deterministic.
 #include "common.cuh"
 #include "internal.cuh"
+
+#include <algorithm>
 
 namespace sf {
 namespace {
 
 constexpr int kLaneCh = 64;                 // input channels per lane
-constexpr int kSegChannels = 32 * kLaneCh;  // 2,048 channels per warp segment
-constexpr int kWarps = 16;                  // one CTA of 16 warps per SM
-constexpr int kThreads = kWarps * 32;
-#ifndef SF_GEMV_XPLANES
-#define SF_GEMV_XPLANES 3
+constexpr int kSegCh = 32 * kLaneCh;        // channels per warp segment
+constexpr int kMaxSegs = 16;                // k <= 32,768
+constexpr int kMaxWarps = 15;               // compute warps per CTA (plus the producer: 16 warps)
+#ifndef SF_GEMV_PLANES
+#define SF_GEMV_PLANES 3
 #endif
-constexpr int kXP = SF_GEMV_XPLANES;        // byte planes of the fixed-point activations
-constexpr int kXShift = 8 * kXP - 4;        // x_fix = x * 2^-(ilogb(max|x|) - kXShift), |x_fix| < 2^(8 kXP - 3)
-constexpr int kXR = 16 * kXP;               // plane words per lane group
-constexpr int kXWords = kXR + 4;            // then sum0, sum1, 2^e, sum
+constexpr int kXP = SF_GEMV_PLANES;         // byte planes of the fixed-point activations (2 or 3)
+constexpr int kXW = 16 * kXP + 4;           // shared words per lane block: planes, sum0, sum1, scale, pad
+// x_fix = x * 2^(kXE - ilogb(max |x| of the block)): |x_fix| < 2^(kXE + 1), so
+// 4 * sum code * x_fix over 64 channels fits an int32 for every base width
+constexpr int kXE = kXP == 2 ? 14 : 19;
 constexpr int kRowUnit = 4;                 // CTA row ranges start at multiples of 4
-constexpr size_t kSmemLimit = 226 * 1024;  // one block reservation (1 KB) below the SM's 228 KB
+constexpr size_t kSmemLimit = 227 * 1024;   // dynamic shared memory of one CTA
+constexpr size_t kStageTarget = 36 * 1024;  // bytes of codes per ring stage, at most
+constexpr int kMaxStages = 6;
+constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
 
-struct GemvParams {
-  const uint32_t* base;
-  const uint32_t* refine;  // channel-major rows, or staged rows [batch][n_sel]
-  const uint16_t* sz;
-  const uint16_t* x;       // [batch][K] fp16
-  const int32_t* sel;      // [batch][n_sel]
-  float* y;
-  int N, K, G, gshift, r, batch, n_sel, segs;
-  int refine_row_words;  // N * r / 32
-  int staged;            // refine holds [batch][n_sel] staged rows
-  int rows_max;          // most rows a CTA owns
-  int plane_words;       // shared words of the activation planes
-  int area_words;        // shared words of the copy rings (reused by the slow correction path)
-  int fast;              // correction tables in their own shared region, filled before the base pass
-  int w_span;            // stride of the refinement-word table (words a CTA's rows can span)
-  int corr_rows;         // rows per lane in the correction (1, 2 or 4)
-  int corr_split;        // fast path: the warps' correction partials go to the free ring area
-  int pstride;           // row stride of the partial sums: segs base columns, then the correction
-  float* y_corr;         // non-null: the correction goes here ([batch][N]) and y gets the base only
+// Bounded waits that ran out (the host reads it with sf_device_wait_timeouts).
+__device__ unsigned int g_wait_timeouts;
+
+struct GemvArgs {
+  const uint8_t* base;      // codes; b = 3: plane L then plane H (hi_off bytes in)
+  const uint32_t* refine;   // channel-major rows [K][row_words], or staged rows [n_sel][row_words]
+  const uint32_t* sz;       // [N][gpr] words: fp16 (s, m)
+  const uint16_t* x;        // [K] fp16
+  const int32_t* sel;       // [n_sel]
+  float* y;                 // [N]
+  float* y_corr;            // non-null: the correction goes here, y gets the base product
+  size_t hi_off;
+  int N, K, gpr, gshift, r, n_sel;
+  int segs, R, W;           // segments, warps per segment, compute warps (segs * R)
+  int rc, stages;           // rows per stage (R * RPW), ring depth
+  int rowL, rowH;           // bytes per row of plane L (all codes for b = 2, 4) and of plane H
+  int stage_bytes;
+  int row_words, staged, rows_max;
+  int off_ring, off_sz, off_x, off_part, off_szt, off_jd, off_wt, off_cpart;  // shared memory offsets
+  int szt_pitch, wt_pitch, cparts;
 };
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+// ---- PTX helpers ------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
-__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
-  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for the phase of `bar` with this parity to complete, for at most
+// kWaitNs; false (and the timeout counted) if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitNs) {
+      atomicAdd(&g_wait_timeouts, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+// 1-D bulk copy global -> this CTA's shared memory, completion counted on bar.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
-  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sa), "l"(gmem) : "memory");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Named barrier over `count` threads (whole warps).
+__device__ __forceinline__ void bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
@@ -104,119 +160,160 @@ __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) 
   asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ int32_t dp4a_us(uint32_t a, uint32_t b, int32_t c) {
+__device__ __forceinline__ uint32_t dp4a_us(uint32_t a, uint32_t b, uint32_t c) {
   int32_t d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"((int32_t)c));
+  return (uint32_t)d;
 }
 
-// Per lane and row: CW words of codes (64 channels), U rows per task.
-template <int BITS>
-struct Lane {
-  static constexpr int CW = BITS == 2 ? 4 : BITS == 3 ? 6 : 8;
-  static constexpr int U = BITS == 4 ? 2 : 4;
-};
+// ---- activations -------------------------------------------------------------
 
-// Ring slot of one task (words): codes [U][C16][32 lanes][4] in 16-byte chunks,
-// for b = 3 then the high-bit words [U][32][2], then (s, m) [U][ZW][32].
-// Consecutive lanes read consecutive chunks, so reads are conflict-free.
-template <int BITS, int ZW>
-struct Ring {
-  static constexpr int CW = Lane<BITS>::CW, U = Lane<BITS>::U;
-  static constexpr int C16 = BITS == 3 ? 1 : CW / 4;
-  static constexpr int hi_off() { return U * C16 * 32 * 4; }
-  static constexpr int z_off = U * 32 * CW;
-  static constexpr int words = U * 32 * (CW + ZW);
-};
-
-// Copies of one row into ring slot position u: the lane's codes (lane_base:
-// the row-0 address of the lane's 16-byte chunks, row_bytes apart) and its
-// (s, m) word(s) (lane_z: row 0's, gpr words apart).
-template <int BITS, int ZW>
-__device__ __forceinline__ void issue_row(const uint8_t* lane_base, const uint8_t* lane_hi, size_t row_bytes,
-                                          const uint32_t* lane_z, int gpr, int row, uint32_t* slot, int u,
-                                          int lane) {
-  using R = Ring<BITS, ZW>;
-  const uint8_t* rb = lane_base + (size_t)row * row_bytes;
-#pragma unroll
-  for (int c = 0; c < R::C16; c++) cp_async16(slot + ((u * R::C16 + c) * 32 + lane) * 4, rb + 16 * c);
-  if constexpr (BITS == 3) cp_async8(slot + R::hi_off() + (u * 32 + lane) * 2, lane_hi + (size_t)row * (row_bytes / 2));
-  const uint32_t* zr = lane_z + (size_t)row * gpr;
-#pragma unroll
-  for (int h = 0; h < ZW; h++) cp_async4(slot + R::z_off + (u * ZW + h) * 32 + lane, zr + h);
-}
-
-// Code byte vector v (0..15) of a lane's 64 channels; byte L holds the code of
-// channel chan_of(v, L).
+// Byte L of code vector v of a lane's 64 channels holds the code of channel
+// chan_of(v, L) (local to the lane block).
 template <int BITS>
 __host__ __device__ __forceinline__ int chan_of(int v, int L) {
   if (BITS == 4) return 8 * (v >> 1) + (v & 1) + 2 * L;
   return 16 * (v >> 2) + (v & 3) + 4 * L;
 }
 
+// Lane block lg of x (64 channels) as fixed point: planes[kXP * v + p] = byte p
+// of x_fix for the four channels of code vector v; then sum of channels 0-31,
+// sum of 32-63 and the factor that turns the integer dot product back into
+// x units (2^e, divided by 4 where the byte vectors carry the factor 4).
 template <int BITS>
-__device__ __forceinline__ uint32_t code_vec(const uint32_t (&w)[Lane<BITS>::CW], int v) {
-  if constexpr (BITS == 4) {
-    return (w[v >> 1] >> (4 * (v & 1))) & 0x0F0F0F0Fu;
-  } else {
-    const int wi = v >> 2, j = v & 3;
-    uint32_t c = (w[wi] >> (2 * j)) & 0x03030303u;
-    if constexpr (BITS == 3) c |= ((w[4 + (wi >> 1)] >> (4 * (wi & 1) + j)) << 2) & 0x04040404u;
-    return c;
+__device__ void lane_planes(const uint16_t* __restrict__ xb, uint32_t* __restrict__ dst) {
+  uint32_t h[32];
+#pragma unroll
+  for (int v = 0; v < 8; v++) {
+    const uint4 q = reinterpret_cast<const uint4*>(xb)[v];
+    h[4 * v] = q.x, h[4 * v + 1] = q.y, h[4 * v + 2] = q.z, h[4 * v + 3] = q.w;
   }
+  uint32_t mx2 = 0;
+#pragma unroll
+  for (int i = 0; i < 32; i++) mx2 = __vmaxu2(mx2, h[i] & 0x7fff7fffu);
+  const uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i++) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    if (i < 16) s0 += f.x, s0 += f.y;
+    else s1 += f.x, s1 += f.y;
+  }
+  // x_fix = x * 2^(kXE - ilogb(max |x|)): the largest values are fp16
+  // mantissas times 2^(kXE - 10) (exact), smaller ones round to that step
+  const int eb = mx ? ((__float_as_int(h2f((uint16_t)mx)) >> 23) & 0xff) - 127 : 0;  // ilogb(max |x|)
+  const float scale = mx ? __int_as_float((127 + kXE - eb) << 23) : 0.f;
+  int q[64];
+#pragma unroll
+  for (int i = 0; i < 32; i++) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    // round to nearest even through the float mantissa: 1.5 * 2^23 + x_fix
+    q[2 * i] = __float_as_int(fmaf(f.x, scale, 12582912.0f)) - 0x4B400000;
+    q[2 * i + 1] = __float_as_int(fmaf(f.y, scale, 12582912.0f)) - 0x4B400000;
+  }
+#pragma unroll
+  for (int v = 0; v < 16; v++) {
+    const int a = q[chan_of<BITS>(v, 0)], b = q[chan_of<BITS>(v, 1)];
+    const int c = q[chan_of<BITS>(v, 2)], d = q[chan_of<BITS>(v, 3)];
+#pragma unroll
+    for (int p = 0; p < kXP; p++) {
+      const uint32_t sel = (uint32_t)p | ((uint32_t)(4 + p) << 4);
+      const uint32_t t01 = __byte_perm((uint32_t)a, (uint32_t)b, sel);
+      const uint32_t t23 = __byte_perm((uint32_t)c, (uint32_t)d, sel);
+      dst[kXP * v + p] = __byte_perm(t01, t23, 0x5410);
+    }
+  }
+  float* f = reinterpret_cast<float*>(dst + 16 * kXP);
+  f[0] = s0;
+  f[1] = s1;
+  f[2] = mx ? __int_as_float((127 + eb - kXE - (BITS == 4 ? 0 : 2)) << 23) : 1.0f;
+  f[3] = 0.f;
 }
 
-// sum_c code_c * x_fix_c over the lane's 64 channels (ZW = 1) or over each
-// 32-channel half (ZW = 2), exact in 32-bit integers: |x_fix| < 2^(8 kXP - 3)
-// and codes < 16 keep every partial below 2^31 (intermediate wrap-around
-// cancels).  Plane p of vector v is xr[kXP v + p]; the top plane is signed.
+// ---- the base pass of one row -------------------------------------------------
+
+// The lane's partial sum of one row: the integer dot products of its block
+// (per 32-channel half when ZW = 2), then s * 2^e * dot + m * sum(x).
+// cw: the row's codes of this lane (plane L), hw: plane H (b = 3),
+// zw: the row's (s, m) word(s) for the lane's group(s).
 template <int BITS, int ZW>
-__device__ __forceinline__ void lane_dot(const uint32_t (&w)[Lane<BITS>::CW], const uint32_t (&xr)[kXR],
-                                         int32_t (&d)[ZW]) {
-  auto mac = [&](uint32_t c, int v, uint32_t (&acc)[kXP]) {
+__device__ __forceinline__ float lane_row(const uint8_t* __restrict__ cw, const uint8_t* __restrict__ hw,
+                                          const uint32_t (&xr)[16 * kXP], float xs0, float xs1,
+                                          float xsc, uint32_t z0, uint32_t z1) {
+  uint32_t A[ZW][kXP], B[ZW][kXP];
 #pragma unroll
-    for (int q = 0; q < kXP; q++)
-      acc[q] = q == kXP - 1 ? (uint32_t)dp4a_us(c, xr[kXP * v + q], (int32_t)acc[q]) : dp4a_uu(c, xr[kXP * v + q], acc[q]);
+  for (int h = 0; h < ZW; h++)
+#pragma unroll
+    for (int p = 0; p < kXP; p++) A[h][p] = B[h][p] = 0u;
+  auto mac = [&](uint32_t c, int v, uint32_t(&acc)[kXP]) {
+#pragma unroll
+    for (int p = 0; p < kXP; p++)
+      acc[p] = p == kXP - 1 ? dp4a_us(c, xr[kXP * v + p], acc[p]) : dp4a_uu(c, xr[kXP * v + p], acc[p]);
   };
-  auto combine = [&](const uint32_t (&acc)[kXP]) {
-    uint32_t t = acc[0];
+  if constexpr (BITS == 4) {
+    const uint4 q0 = reinterpret_cast<const uint4*>(cw)[0], q1 = reinterpret_cast<const uint4*>(cw)[1];
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-    for (int q = 1; q < kXP; q++) t += acc[q] << (8 * q);
-    return (int32_t)t;
-  };
-  if constexpr (BITS == 2) {
-    // c0 = w & 0x03.. (channels 4L), c1 = w & 0x0C.. = 4 x (channels 4L+1),
-    // the same on w >> 4 for 4L+2 and 4L+3: set A has factor 1, set B factor 4
-    uint32_t A[ZW][kXP], B[ZW][kXP];
-#pragma unroll
-    for (int h = 0; h < ZW; h++)
-#pragma unroll
-      for (int q = 0; q < kXP; q++) A[h][q] = B[h][q] = 0;
-#pragma unroll
-    for (int wi = 0; wi < 4; wi++) {
-      const int h = ZW == 2 ? (wi >> 1) : 0;
-      const uint32_t w0 = w[wi], w4 = w0 >> 4;
-      mac(w0 & 0x03030303u, 4 * wi + 0, A[h]);
-      mac(w0 & 0x0C0C0C0Cu, 4 * wi + 1, B[h]);
-      mac(w4 & 0x03030303u, 4 * wi + 2, A[h]);
-      mac(w4 & 0x0C0C0C0Cu, 4 * wi + 3, B[h]);
+    for (int i = 0; i < 8; i++) {
+      const int h = ZW == 2 ? (i >> 2) : 0;
+      mac(w[i] & 0x0F0F0F0Fu, 2 * i, A[h]);
+      mac((w[i] >> 4) & 0x0F0F0F0Fu, 2 * i + 1, A[h]);
+    }
+  } else {
+    const uint4 q0 = *reinterpret_cast<const uint4*>(cw);
+    const uint32_t w[4] = {q0.x, q0.y, q0.z, q0.w};
+    uint32_t hi[2] = {0u, 0u};
+    if constexpr (BITS == 3) {
+      const uint2 t = *reinterpret_cast<const uint2*>(hw);
+      hi[0] = t.x, hi[1] = t.y;
     }
 #pragma unroll
-    for (int h = 0; h < ZW; h++) d[h] = combine(A[h]) + (combine(B[h]) >> 2);
+    for (int i = 0; i < 4; i++) {
+      const int h = ZW == 2 ? (i >> 1) : 0;
+      const uint32_t w0 = w[i], w4 = w0 >> 4;
+      uint32_t c0 = w0 & 0x03030303u, c1 = w0 & 0x0C0C0C0Cu;
+      uint32_t c2 = w4 & 0x03030303u, c3 = w4 & 0x0C0C0C0Cu;
+      if constexpr (BITS == 3) {
+        // the high bit of the codes of vector 4i + m sits at bit 4 (i & 1) + m of
+        // each byte of hi[i / 2]; it joins at bit 2 (factor-1 vectors) or 4
+        const uint32_t H = hi[i >> 1];
+        if ((i & 1) == 0) {
+          c0 |= (H << 2) & 0x04040404u;
+          c1 |= (H << 3) & 0x10101010u;
+          c2 |= H & 0x04040404u;
+          c3 |= (H << 1) & 0x10101010u;
+        } else {
+          c0 |= (H >> 2) & 0x04040404u;
+          c1 |= (H >> 1) & 0x10101010u;
+          c2 |= (H >> 4) & 0x04040404u;
+          c3 |= (H >> 3) & 0x10101010u;
+        }
+      }
+      mac(c0, 4 * i + 0, A[h]);
+      mac(c1, 4 * i + 1, B[h]);
+      mac(c2, 4 * i + 2, A[h]);
+      mac(c3, 4 * i + 3, B[h]);
+    }
+  }
+  // 4 x sum(code x_fix) (b = 2, 3: set B carries the factor 4) or sum(code x_fix) (b = 4)
+  int32_t J[ZW];
+#pragma unroll
+  for (int h = 0; h < ZW; h++) {
+    uint32_t a = A[h][0], bb = B[h][0];
+#pragma unroll
+    for (int p = 1; p < kXP; p++) a += A[h][p] << (8 * p), bb += B[h][p] << (8 * p);
+    J[h] = BITS == 4 ? (int32_t)a : (int32_t)((a << 2) + bb);
+  }
+  const float2 sm0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
+  if constexpr (ZW == 1) {
+    return fmaf(sm0.x * xsc, (float)J[0], sm0.y * (xs0 + xs1));
   } else {
-    uint32_t A[ZW][kXP];
-#pragma unroll
-    for (int h = 0; h < ZW; h++)
-#pragma unroll
-      for (int q = 0; q < kXP; q++) A[h][q] = 0;
-#pragma unroll
-    for (int v = 0; v < 16; v++) mac(code_vec<BITS>(w, v), v, A[ZW == 2 ? (chan_of<BITS>(v, 0) >= 32) : 0]);
-#pragma unroll
-    for (int h = 0; h < ZW; h++) d[h] = combine(A[h]);
+    const float2 sm1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
+    return fmaf(sm0.x * xsc, (float)J[0], fmaf(sm1.x * xsc, (float)J[1], fmaf(sm0.y, xs0, sm1.y * xs1)));
   }
 }
 
-// Sum each of U per-lane values over the warp.  Returns the full sum of row
+// Sum each of U per-lane values over the warp.  Returns the full sum of value
 // lane >> 3 (U = 4) or lane >> 4 (U = 2) in every lane.
 template <int U>
 __device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
@@ -245,404 +342,225 @@ __device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// correction table entries: (x_c, x_c (1 - off/2^r), group of c, word offset of
-// the refinement row of c), off = 1/2 - 2^(r-1)
+// ---- the kernel -----------------------------------------------------------------
 
-__device__ __forceinline__ uint4 make_jd(const GemvParams& p, int b, int j) {
-  const int c = __ldg(p.sel + (size_t)b * p.n_sel + j);
-  const float xc = h2f(__ldg(p.x + (size_t)b * p.K + c));
-  const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << p.r)) / (float)(1 << p.r);
-  const uint32_t off = p.staged ? (uint32_t)(((size_t)b * p.n_sel + j) * p.refine_row_words)
-                                : (uint32_t)((size_t)c * p.refine_row_words);
-  return make_uint4(__float_as_uint(xc), __float_as_uint(xc * cfac), (uint32_t)(c >> p.gshift), off);
-}
+// RPW: rows per compute warp per stage (2 or 4).  A CTA's warps are spread
+// over the SM's four schedulers, each with a quarter of the register file:
+// four warps of 120 registers a thread leave kSideRegs / 4 of every quarter
+// free for a staging CTA.
+static_assert(((kMaxWarps + 1 + 3) / 4) * 120 * 32 + kSideRegs / 4 <= 65536 / 4,
+              "GEMV registers leave no room for a staging CTA");
+template <int BITS, int ZW, int RPW>
+__global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int S = a.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* szbar = empty + kMaxStages;
+  uint8_t* ring = smem + a.off_ring;
+  uint32_t* szs = reinterpret_cast<uint32_t*>(smem + a.off_sz);
+  uint32_t* xpl = reinterpret_cast<uint32_t*>(smem + a.off_x);
+  float* part = reinterpret_cast<float*>(smem + a.off_part);
+  uint32_t* szt = reinterpret_cast<uint32_t*>(smem + a.off_szt);
+  uint2* jd = reinterpret_cast<uint2*>(smem + a.off_jd);
+  uint32_t* wt = reinterpret_cast<uint32_t*>(smem + a.off_wt);
+  float* cpart = reinterpret_cast<float*>(smem + a.off_cpart);
 
-// ---------------------------------------------------------------------------
-// activation prologue: every CTA turns batch row b of x into the fixed-point
-// byte planes of all K/64 lane groups in shared memory, one warp per group
-
-template <int BITS>
-__device__ void prep_planes(const GemvParams& p, int b, uint32_t* __restrict__ xs, int* __restrict__ scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int ngrp = p.K / kLaneCh;
-  // UNR groups per warp at a time (independent shuffle chains interleave); the
-  // warp's scratch holds their 64 fixed-point values each, by (vector, byte)
-  constexpr int UNR = 4;
-  int* sw = scratch + warp * UNR * kLaneCh;
-  auto slot_of = [](int c) {
-    const int v = BITS == 4 ? 2 * (c >> 3) + (c & 1) : 4 * (c >> 4) + (c & 3);
-    const int L = BITS == 4 ? (c >> 1) & 3 : (c >> 2) & 3;
-    return 4 * v + L;
-  };
-  for (int g0 = warp; g0 < ngrp; g0 += UNR * kWarps) {
-    uint32_t xw[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; u++) {
-      const int grp = g0 + u * kWarps;
-      xw[u] = grp < ngrp ? __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)b * p.K + (size_t)grp * kLaneCh) + lane)
-                         : 0u;
-    }
-    float2 xv[UNR];
-    float mx[UNR], sm[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; u++) {
-      xv[u] = __half22float2(*reinterpret_cast<const __half2*>(&xw[u]));
-      mx[u] = fmaxf(fabsf(xv[u].x), fabsf(xv[u].y));
-      sm[u] = xv[u].x + xv[u].y;  // channels 2 lane, 2 lane + 1: halves are lanes 0-15, 16-31
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int u = 0; u < UNR; u++) mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], o));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1)
-#pragma unroll
-      for (int u = 0; u < UNR; u++) sm[u] += __shfl_xor_sync(0xffffffffu, sm[u], o);
-    int eb[UNR];
-    float s1[UNR];
-#pragma unroll
-    for (int u = 0; u < UNR; u++) {
-      // x_fix = x 2^-e with e = ilogb(max |x|) - kXShift; every nonzero fp16 value
-      // is a normal float, so the exponent and 2^-e come from the float bits (exact)
-      eb[u] = (__float_as_int(mx[u]) >> 23) & 0xff;  // biased exponent; 0 only for max 0
-      const float scale = eb[u] ? __int_as_float((254 + kXShift - eb[u]) << 23) : 0.f;
-      sw[u * kLaneCh + slot_of(2 * lane)] = __float2int_rn(xv[u].x * scale);
-      sw[u * kLaneCh + slot_of(2 * lane + 1)] = __float2int_rn(xv[u].y * scale);
-      s1[u] = __shfl_sync(0xffffffffu, sm[u], 16);
-    }
-    __syncwarp();
-#pragma unroll
-    for (int u = 0; u < UNR; u++) {
-      const int grp = g0 + u * kWarps;
-      if (grp < ngrp) {
-        uint32_t* dst = xs + grp * kXWords;
-        if (lane < 16) {  // lane v: plane q of vector v = byte q of its four values
-          const int4 f = reinterpret_cast<const int4*>(sw + u * kLaneCh)[lane];
-#pragma unroll
-          for (int q = 0; q < kXP; q++) {
-            const uint32_t sel = (uint32_t)q | ((uint32_t)(4 + q) << 4);
-            const uint32_t t01 = __byte_perm((uint32_t)f.x, (uint32_t)f.y, sel);
-            const uint32_t t23 = __byte_perm((uint32_t)f.z, (uint32_t)f.w, sel);
-            dst[kXP * lane + q] = __byte_perm(t01, t23, 0x5410);
-          }
-        }
-        if (lane == 0) {  // lane 0 holds the first half's sum, s1 the second's
-          reinterpret_cast<float*>(dst)[kXR + 0] = sm[u];
-          reinterpret_cast<float*>(dst)[kXR + 1] = s1[u];
-          reinterpret_cast<float*>(dst)[kXR + 2] = eb[u] ? __int_as_float((eb[u] - kXShift) << 23) : 1.0f;
-          reinterpret_cast<float*>(dst)[kXR + 3] = sm[u] + s1[u];
-        }
-      }
-    }
-    __syncwarp();  // the scratch is rewritten by the next groups
-  }
-}
-
-// ---------------------------------------------------------------------------
-// correction
-
-// Table entries [j0, j0 + jn) of batch row b into jd, and the refinement words
-// [w_lo, w_lo + nwr) of each entry's row into wt (stride nwr), by cp.async.
-__device__ void corr_fill(const GemvParams& p, int b, int j0, int jn, int w_lo, int nwr, uint4* jd,
-                          uint32_t* wt) {
-  for (int i = threadIdx.x; i < jn; i += kThreads) {
-    if (p.staged) {  // the staged row of entry j is known without the selection: copy it first
-      const uint32_t off = (uint32_t)(((size_t)b * p.n_sel + j0 + i) * p.refine_row_words);
-      for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + off + w_lo + k);
-      jd[i] = make_jd(p, b, j0 + i);
-    } else {
-      const uint4 d = make_jd(p, b, j0 + i);
-      jd[i] = d;
-      for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)i * nwr + k, p.refine + d.w + w_lo + k);
-    }
-  }
-  cp_async_commit();
-}
-
-// Warp tasks of the correction: row blocks of 32 lanes x RL rows, times
-// splits of the table entries.
-__device__ __forceinline__ void corr_tasks(int rows, int RL, int& nblk, int& js_n) {
-  nblk = (rows / RL + 31) / 32;
-  js_n = nblk >= kWarps ? 1 : kWarps / nblk;
-}
-
-// The correction of table entries [0, jn): into cpart[js][row] (entry split
-// js, stride rows_max; every row of every split written), or added into
-// the correction column part[row][segs] when cpart is NULL.  Lanes own RL consecutive rows (inside one
-// refinement word); warps split the entries.
-// Entries come in ascending channel order, so channels of one scale group are
-// consecutive: each run is summed unscaled and multiplied by s once.  szt:
-// the CTA's (s, m) words group-major, [gpr][rows_max], so that the lanes of a
-// warp (consecutive rows) read consecutive words; or NULL (scales read from
-// global memory).
-template <int RL>
-__device__ void corr_process(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
-                             const uint4* __restrict__ jd, const uint32_t* __restrict__ wt,
-                             const uint32_t* __restrict__ szt, float* part, float* cpart) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gpr = p.K >> p.gshift;
-  const int units = rows / RL;
-  int nblk, js_n;
-  corr_tasks(rows, RL, nblk, js_n);
-  const int ntasks = nblk * js_n;
-  const int r = p.r;
-  const uint32_t fmask = ((1u << r) - 1u) << (23 - r);
-  for (int task = warp; task < ntasks; task += kWarps) {
-    const int blk = task % nblk, js = task / nblk;
-    const int qu = blk * 32 + lane;
-    const bool ok = qu < units;
-    const int rl0 = RL * qu;
-    const int bit0 = (n0 + rl0) * r;
-    const int wr = (bit0 >> 5) - w_lo;
-    int rot[RL];
-#pragma unroll
-    for (int t = 0; t < RL; t++) rot[t] = (23 - r - ((bit0 & 31) + r * t)) & 31;
-    const int ia = (int)((long)js * jn / js_n), ib = (int)((long)(js + 1) * jn / js_n);
-    float acc[RL], run[RL];
-#pragma unroll
-    for (int t = 0; t < RL; t++) acc[t] = run[t] = 0.f;
-    float C = 0.f;
-    int gcur = -1;
-    auto flush = [&]() {
-      if (gcur >= 0 && ok) {
-        // the lane's RL rows of group gcur are consecutive words of szt
-        uint32_t zt[RL];
-        if (szt) {
-          const uint32_t* zp = szt + gcur * p.rows_max + rl0;
-          if constexpr (RL == 4) {
-            const uint4 v = *reinterpret_cast<const uint4*>(zp);
-            zt[0] = v.x, zt[1] = v.y, zt[2] = v.z, zt[3] = v.w;
-          } else if constexpr (RL == 2) {
-            const uint2 v = *reinterpret_cast<const uint2*>(zp);
-            zt[0] = v.x, zt[1] = v.y;
-          } else {
-            zt[0] = zp[0];
-          }
-        }
-#pragma unroll
-        for (int t = 0; t < RL; t++) {
-          const uint32_t zw = szt ? zt[t]
-                                  : __ldg(reinterpret_cast<const uint32_t*>(p.sz) + (size_t)(n0 + rl0 + t) * gpr + gcur);
-          const float sc = __low2float(*reinterpret_cast<const __half2*>(&zw));
-          acc[t] = fmaf(sc, run[t] - C, acc[t]);
-        }
-      }
-    };
-    for (int i = ia; i < ib; i++) {
-      const uint4 d = jd[i];
-      if ((int)d.z != gcur) {
-        flush();
-        gcur = (int)d.z;
-        C = 0.f;
-#pragma unroll
-        for (int t = 0; t < RL; t++) run[t] = 0.f;
-      }
-      const uint32_t w = ok ? wt[(size_t)i * nwr + wr] : 0u;
-      const float xc = __uint_as_float(d.x);
-      // f = 1 + rho / 2^r; sum x f - sum x (1 - off/2^r) = sum x (rho + off) / 2^r
-#pragma unroll
-      for (int t = 0; t < RL; t++)
-        run[t] = fmaf(__uint_as_float(0x3F800000u | (__funnelshift_l(w, w, rot[t]) & fmask)), xc, run[t]);
-      C += __uint_as_float(d.y);
-    }
-    flush();
-    if (ok && cpart) {
-#pragma unroll
-      for (int t = 0; t < RL; t++) cpart[js * p.rows_max + rl0 + t] = acc[t];
-    } else if (ok && ib > ia) {
-#pragma unroll
-      for (int t = 0; t < RL; t++) atomicAdd(&part[(rl0 + t) * p.pstride + p.segs], acc[t]);
-    }
-  }
-}
-
-__device__ __forceinline__ void corr_dispatch(const GemvParams& p, int n0, int rows, int w_lo, int nwr, int jn,
-                                              const uint4* jd, const uint32_t* wt, const uint32_t* szt,
-                                              float* part, float* cpart) {
-  if (p.corr_rows == 4)
-    corr_process<4>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
-  else if (p.corr_rows == 2)
-    corr_process<2>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
-  else
-    corr_process<1>(p, n0, rows, w_lo, nwr, jn, jd, wt, szt, part, cpart);
-}
-
-// ---------------------------------------------------------------------------
-// the GEMV
-
-// 120 registers x 512 threads: kSideRegs of the SM's registers stay free
-static_assert(65536 - 120 * kThreads >= kSideRegs, "GEMV registers leave no room for a staging CTA");
-template <int BITS, int ZW, int PD>
-__global__ void __maxnreg__(120) gemv_kernel(GemvParams p) {
-  using R = Ring<BITS, ZW>;
-  constexpr int U = Lane<BITS>::U, CW = Lane<BITS>::CW;
-  extern __shared__ __align__(16) uint32_t smem[];
-  pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this grid
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int units = p.N / kRowUnit;
+  const int units = a.N / kRowUnit;
   const int n0 = (int)((long)blockIdx.x * units / gridDim.x) * kRowUnit;
   const int n1 = (int)((long)(blockIdx.x + 1) * units / gridDim.x) * kRowUnit;
   const int rows = n1 - n0;
-  const int ngrp = p.K / kLaneCh, gpr = p.K >> p.gshift;
-  // shared memory: partial sums [rows][segs] | rings | (fast) table, words, scales
-  float* part = reinterpret_cast<float*>(smem);
-  uint32_t* xs = smem + ((p.rows_max * p.pstride + 3) & ~3);  // activation planes [K/64][kXWords], prologue scratch
-  uint32_t* area = xs + p.plane_words;
-  uint4* jd_fast = reinterpret_cast<uint4*>(area + p.area_words);
-  uint32_t* wt_fast = reinterpret_cast<uint32_t*>(jd_fast + p.n_sel);
-  uint32_t* szt = wt_fast + (((size_t)p.n_sel * p.w_span + 3) & ~(size_t)3);
-  const int w_lo = (n0 * p.r) >> 5;
-  const int nwr = (((n1 * p.r) + 31) >> 5) - w_lo;
-  const int steps = (rows + U - 1) / U, ntask = p.segs * steps;
-  const int ta = (int)((long)warp * ntask / kWarps), tb = (int)((long)(warp + 1) * ntask / kWarps);
-  const size_t row_bytes = (size_t)p.K * (BITS == 3 ? 2 : BITS) / 8;
-  const bool fill_szt = p.fast && p.n_sel > 0;
-  // the fast correction's per-warp partials: in the ring area, free once the base pass is done
-  float* cpart = p.corr_split && p.fast && p.n_sel > 0 ? reinterpret_cast<float*>(area) : nullptr;
+  const int nst = (rows + a.rc - 1) / a.rc;
+  const int w_lo = (n0 * a.r) >> 5;
+  const int nwr = (((n1 * a.r) + 31) >> 5) - w_lo;
+  const bool corr = a.n_sel > 0;
 
-  for (int b = 0; b < p.batch; b++) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; s++) mbar_init(&full[s], 1), mbar_init(&empty[s], a.W);
+    mbar_init(szbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this grid
+
+  if (warp == a.W) {
+    // ---------------- producer warp
+    int issued = 0;
+    auto issue = [&](int i) {
+      const int slot = i % S;
+      const int r0 = i * a.rc, nr = min(a.rc, rows - r0);
+      const uint32_t bl = (uint32_t)(nr * a.rowL), bh = (uint32_t)(nr * a.rowH);
+      uint8_t* dst = ring + (size_t)slot * a.stage_bytes;
+      mbar_expect_tx(&full[slot], bl + bh);
+      bulk_g2s(dst, a.base + (size_t)(n0 + r0) * a.rowL, bl, &full[slot]);
+      if (BITS == 3) bulk_g2s(dst + (size_t)a.rc * a.rowL, a.base + a.hi_off + (size_t)(n0 + r0) * a.rowH, bh, &full[slot]);
+    };
+    if (lane == 0) {
+      const uint32_t zb = (uint32_t)(rows * a.gpr * 4);
+      mbar_expect_tx(szbar, zb);
+      bulk_g2s(szs, a.sz + (size_t)n0 * a.gpr, zb, szbar);
+      for (; issued < min(S, nst); issued++) issue(issued);
+    }
+    pdl_wait();  // x, the selection and the staged rows are complete
+    if (corr) {
+      // correction tables: (x_c, group of c) and the refinement words of the CTA's rows
+      for (int j = lane; j < a.n_sel; j += 32) {
+        // -1 - c: channel c selected but not refined now (no correction); a
+        // foreign index is clamped, so it never leaves the buffers
+        const int raw = __ldg(a.sel + j);
+        const int c = min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
+        const uint32_t xc = raw < 0 ? 0u : __float_as_uint(h2f(__ldg(a.x + c)));
+        jd[j] = make_uint2(xc, (uint32_t)(c >> a.gshift));
+        const uint32_t* src = a.refine + (size_t)(a.staged ? j : c) * a.row_words + w_lo;
+        for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)j * a.wt_pitch + k, src + k);
+      }
+      cp_async_commit();
+    }
+    if (lane == 0) {
+      for (; issued < nst; issued++) {
+        const int slot = issued % S;
+        if (!mbar_wait(&empty[slot], ((issued / S) - 1) & 1)) break;
+        issue(issued);
+      }
+      // nothing may still be landing in this CTA's shared memory when it exits
+      for (int i = max(0, issued - S); i < issued; i++) mbar_wait(&full[i % S], (i / S) & 1);
+      mbar_wait(szbar, 0);
+    }
+    cp_async_wait_all();
+    __syncwarp();
+  } else {
+    // ---------------- compute warps
+    const int seg = warp % a.segs, jw = warp / a.segs;
+    const int lg = seg * 32 + lane;  // lane block
+    const bool la = lg * kLaneCh < a.K;
+    pdl_wait();
+    // activation planes of segment `warp`, one warp per segment
+    if (warp < a.segs) {
+      uint32_t* dst = xpl + ((size_t)warp * 32 + lane) * kXW;
+      if (la) {
+        lane_planes<BITS>(a.x + (size_t)lg * kLaneCh, dst);
+      } else {
+#pragma unroll 4
+        for (int k = 0; k < kXW; k++) dst[k] = 0u;
+      }
+    }
+    bar_sync(1, a.W * 32);
+    uint32_t xr[16 * kXP];
+    float xs0, xs1, xsc;
     {
-      // ---- base pass of batch row b: every (row, segment) partial is written once
-      uint32_t* ring = area + warp * PD * R::words;
-      int iseg = ta / steps, ist = ta - iseg * steps, islot = 0, left = tb - ta;
-      auto issue = [&]() {
-        if (left > 0) {
-          const int lg = iseg * 32 + lane;
-          if (lg < ngrp) {
-            const uint8_t* lb = reinterpret_cast<const uint8_t*>(p.base) + 16 * R::C16 * lg;
-            const uint8_t* lh = reinterpret_cast<const uint8_t*>(p.base) + (size_t)p.N * p.K / 4 + 8 * lg;
-            const uint32_t* lz = reinterpret_cast<const uint32_t*>(p.sz) + ((lg * kLaneCh) >> p.gshift);
-            uint32_t* slot = ring + islot * R::words;
-            const int r0 = n0 + ist * U;
+      const uint4* src = reinterpret_cast<const uint4*>(xpl + ((size_t)seg * 32 + lane) * kXW);
 #pragma unroll
-            for (int u = 0; u < U; u++) issue_row<BITS, ZW>(lb, lh, row_bytes, lz, gpr, r0 + u, slot, u, lane);
+      for (int k = 0; k < 4 * kXP; k++) {
+        const uint4 q = src[k];
+        xr[4 * k] = q.x, xr[4 * k + 1] = q.y, xr[4 * k + 2] = q.z, xr[4 * k + 3] = q.w;
+      }
+      const float4 f = reinterpret_cast<const float4*>(src)[4 * kXP];
+      xs0 = f.x, xs1 = f.y, xsc = f.z;
+    }
+    const int g0 = (lg * kLaneCh) >> a.gshift;            // the lane's (first) group
+    const bool zown = corr && la && ((lg * kLaneCh) & ((1 << a.gshift) - 1)) == 0;
+    bool ok = mbar_wait(szbar, 0);
+    const size_t codeL = (size_t)lg * (BITS == 4 ? 32 : 16);
+    for (int i = 0; i < nst && ok; i++) {
+      const int slot = i % S;
+      if (!mbar_wait(&full[slot], (i / S) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* sl = ring + (size_t)slot * a.stage_bytes;
+      float pv[RPW];
+#pragma unroll
+      for (int t = 0; t < RPW; t++) {
+        const int rr = jw + a.R * t, lr = i * a.rc + rr;
+        pv[t] = 0.f;
+        if (la && lr < rows) {
+          const uint32_t* zr = szs + (size_t)lr * a.gpr + g0;
+          const uint32_t z0 = zr[0], z1 = ZW == 2 ? zr[1] : 0u;
+          if (zown) {
+            szt[(size_t)g0 * a.szt_pitch + lr] = z0;
+            if (ZW == 2) szt[(size_t)(g0 + 1) * a.szt_pitch + lr] = z1;
           }
-          if (++ist == steps) ist = 0, ++iseg;
-          --left;
+          pv[t] = lane_row<BITS, ZW>(sl + (size_t)rr * a.rowL + codeL,
+                                     sl + (size_t)a.rc * a.rowL + (size_t)rr * a.rowH + (size_t)lg * 8, xr, xs0,
+                                     xs1, xsc, z0, z1);
         }
-        islot = islot + 1 == PD ? 0 : islot + 1;
-        cp_async_commit();
+      }
+      const float tot = warp_sum_rows<RPW>(pv, lane);
+      const int t = RPW == 4 ? (lane >> 3) : (lane >> 4);
+      const int lr = i * a.rc + jw + a.R * t;
+      if ((lane & (32 / RPW - 1)) == 0 && lr < rows) part[(size_t)lr * a.segs + seg] = tot;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+  }
+  bar_sync(2, blockDim.x);  // base pass, tables and refinement words complete
+
+  // ---------------- correction of the selected channels (all threads)
+  if (corr) {
+    const int nb = rows / 4;
+    const int Q = a.cparts;
+    const int r = a.r;
+    const uint32_t fmask = ((1u << r) - 1u) << (23 - r);
+    const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << r)) / (float)(1 << r);
+    for (int task = threadIdx.x; task < nb * Q; task += blockDim.x) {
+      const int blk = task % nb, q = task / nb;
+      const int j0 = (int)((long)q * a.n_sel / Q), j1 = (int)((long)(q + 1) * a.n_sel / Q);
+      const int bit0 = (n0 + 4 * blk) * r;
+      const int wi = (bit0 >> 5) - w_lo;
+      int rot[4];
+#pragma unroll
+      for (int t = 0; t < 4; t++) rot[t] = (23 - r - ((bit0 & 31) + r * t)) & 31;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f}, run[4] = {0.f, 0.f, 0.f, 0.f};
+      float C = 0.f;
+      int gcur = -1;
+      auto flush = [&]() {
+        if (gcur >= 0) {
+          const uint4 z = *reinterpret_cast<const uint4*>(szt + (size_t)gcur * a.szt_pitch + 4 * blk);
+          const uint32_t zz[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+          for (int t = 0; t < 4; t++)
+            acc[t] = fmaf(__low2float(*reinterpret_cast<const __half2*>(&zz[t])), run[t] - C, acc[t]);
+        }
       };
+      for (int j = j0; j < j1; j++) {
+        const uint2 d = jd[j];
+        if ((int)d.y != gcur) {
+          flush();
+          gcur = (int)d.y, C = 0.f;
 #pragma unroll
-      for (int i = 0; i < PD - 1; i++) issue();
-      if (b == 0) pdl_wait();  // x, the selection and the staged rows are complete
-      for (int i = threadIdx.x; i < rows; i += kThreads) part[i * p.pstride + p.segs] = 0.f;  // correction column
-      prep_planes<BITS>(p, b, xs, reinterpret_cast<int*>(xs + ngrp * kXWords));
-      if (p.fast && p.n_sel > 0) corr_fill(p, b, 0, p.n_sel, w_lo, nwr, jd_fast, wt_fast);
-      __syncthreads();  // planes complete
-      uint32_t xr[kXR];
-      float xsum0 = 0.f, xsum1 = 0.f, xscale = 0.f;
-      int cseg = ta / steps, cst = ta - cseg * steps, cslot = 0, cur = -1;
-      for (int t = ta; t < tb; t++) {
-        issue();
-        const int lg = cseg * 32 + lane;
-        const bool la = lg < ngrp;
-        if (cseg != cur) {
-          cur = cseg;
-          if (la) {
-            const uint4* src = reinterpret_cast<const uint4*>(xs + lg * kXWords);
-#pragma unroll
-            for (int k = 0; k < kXR / 4; k++) {
-              const uint4 q = src[k];
-              xr[4 * k + 0] = q.x, xr[4 * k + 1] = q.y, xr[4 * k + 2] = q.z, xr[4 * k + 3] = q.w;
-            }
-            const float4 f = reinterpret_cast<const float4*>(src)[kXR / 4];
-            xsum0 = ZW == 2 ? f.x : f.w, xsum1 = f.y, xscale = f.z;
-          } else {
-#pragma unroll
-            for (int k = 0; k < kXR; k++) xr[k] = 0;
-            xsum0 = xsum1 = xscale = 0.f;
-          }
+          for (int t = 0; t < 4; t++) run[t] = 0.f;
         }
-        cp_async_wait<PD - 1>();
-        const uint32_t* slot = ring + cslot * R::words;
-        const int r0 = n0 + cst * U;
-        const int zg = (lg * kLaneCh) >> p.gshift;
-        const bool zown = fill_szt && la && ((lg * kLaneCh) & (p.G - 1)) == 0;
-        float acc[U];
+        const uint32_t w = wt[(size_t)j * a.wt_pitch + wi];
+        const float xc = __uint_as_float(d.x);
+        // f = 1 + rho / 2^r; sum x f - sum x (1 - off/2^r) = sum x (rho + off) / 2^r
 #pragma unroll
-        for (int u = 0; u < U; u++) {
-          acc[u] = 0.f;
-          if (la) {
-            uint32_t w[CW];
-#pragma unroll
-            for (int c = 0; c < R::C16; c++) {
-              const uint4 q = *reinterpret_cast<const uint4*>(slot + ((u * R::C16 + c) * 32 + lane) * 4);
-              w[4 * c + 0] = q.x, w[4 * c + 1] = q.y, w[4 * c + 2] = q.z, w[4 * c + 3] = q.w;
-            }
-            if constexpr (BITS == 3) {
-              const uint2 h = *reinterpret_cast<const uint2*>(slot + R::hi_off() + (u * 32 + lane) * 2);
-              w[4] = h.x, w[5] = h.y;
-            }
-            int32_t d[ZW];
-            lane_dot<BITS, ZW>(w, xr, d);
-            const uint32_t z0 = slot[R::z_off + (u * ZW) * 32 + lane];
-            const float2 sm0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
-            if constexpr (ZW == 1) {
-              acc[u] = fmaf(sm0.x * xscale, (float)d[0], sm0.y * xsum0);
-              if (zown) szt[zg * p.rows_max + (r0 + u - n0)] = z0;
-            } else {
-              const uint32_t z1 = slot[R::z_off + (u * ZW + 1) * 32 + lane];
-              const float2 sm1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
-              acc[u] = fmaf(sm0.x * xscale, (float)d[0],
-                            fmaf(sm1.x * xscale, (float)d[1], fmaf(sm0.y, xsum0, sm1.y * xsum1)));
-              if (fill_szt && la) szt[zg * p.rows_max + (r0 + u - n0)] = z0, szt[(zg + 1) * p.rows_max + (r0 + u - n0)] = z1;
-            }
-          }
-        }
-        const float tot = warp_sum_rows<U>(acc, lane);
-        const int u = U == 4 ? (lane >> 3) : (lane >> 4);
-        if ((lane & (32 / U - 1)) == 0) part[(r0 + u - n0) * p.pstride + cseg] = tot;
-        if (++cst == steps) cst = 0, ++cseg;
-        cslot = cslot + 1 == PD ? 0 : cslot + 1;
+        for (int t = 0; t < 4; t++)
+          run[t] = fmaf(__uint_as_float(0x3F800000u | (__funnelshift_l(w, w, rot[t]) & fmask)), xc, run[t]);
+        C = fmaf(xc, cfac, C);
       }
-      cp_async_wait<0>();
+      flush();
+      *reinterpret_cast<float4*>(cpart + (size_t)q * a.rows_max + 4 * blk) = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
-    __syncthreads();
+    bar_sync(2, blockDim.x);
+  }
 
-    // ---- correction of the selected channels of batch row b
-    if (p.n_sel > 0) {
-      if (p.fast) {
-        corr_dispatch(p, n0, rows, w_lo, nwr, p.n_sel, jd_fast, wt_fast, szt, part, cpart);
-      } else {
-        // tables in chunks in the ring area; scales from global memory
-        const int jcap = p.area_words / (4 + nwr);
-        uint4* jd = reinterpret_cast<uint4*>(area);
-        for (int j0 = 0; j0 < p.n_sel; j0 += jcap) {
-          const int jn = min(jcap, p.n_sel - j0);
-          uint32_t* wt = reinterpret_cast<uint32_t*>(jd + jn);
-          corr_fill(p, b, j0, jn, w_lo, nwr, jd, wt);
-          cp_async_wait<0>();
-          __syncthreads();
-          corr_dispatch(p, n0, rows, w_lo, nwr, jn, jd, wt, nullptr, part, nullptr);
-          __syncthreads();
-        }
-      }
+  // ---------------- output
+  for (int lr = threadIdx.x; lr < rows; lr += blockDim.x) {
+    float base = 0.f, c = 0.f;
+    for (int s = 0; s < a.segs; s++) base += part[(size_t)lr * a.segs + s];
+    if (corr)
+      for (int q = 0; q < a.cparts; q++) c += cpart[(size_t)q * a.rows_max + lr];
+    if (a.y_corr) {
+      a.y[n0 + lr] = base;
+      a.y_corr[n0 + lr] = c;
+    } else {
+      a.y[n0 + lr] = base + c;
     }
-    __syncthreads();
-
-    int cjs = 0;  // entry splits of the correction partials in cpart
-    if (cpart) {
-      int nblk;
-      corr_tasks(rows, p.corr_rows, nblk, cjs);
-    }
-    for (int row = n0 + threadIdx.x; row < n1; row += kThreads) {
-      const float* pr = part + (row - n0) * p.pstride;
-      float base = 0.f, corr = pr[p.segs];
-      for (int s = 0; s < p.segs; s++) base += pr[s];
-      for (int js = 0; js < cjs; js++) corr += cpart[js * p.rows_max + row - n0];
-      float* dst = p.y + (size_t)b * p.N + row;
-      if (p.y_corr) {
-        *dst = base;
-        p.y_corr[(size_t)b * p.N + row] = corr;
-      } else {
-        *dst = base + corr;
-      }
-    }
-    __syncthreads();
   }
 }
+
 
 // ---------------------------------------------------------------------------
 // the correction on its own (fetch lag), added into y
@@ -704,13 +622,19 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
     const size_t row = a.staged ? (size_t)b * a.n_sel + j : (size_t)c;
     return __ldg(a.refine + row * a.row_words + wi) >> sh;
   };
+  // entry j: channel and activation (-1 - c: selected, not refined now: x = 0)
+  auto chan = [&](int j) {
+    const int raw = __ldg(sel + j);
+    return min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
+  };
+  auto act = [&](int j, int c) { return __ldg(sel + j) < 0 ? 0.f : h2f(__ldg(xb + c)); };
   // channel j + 1's index, activation and word are loaded while j is summed
-  int c = a.n_sel > 0 ? __ldg(sel) : 0;
-  float xc = a.n_sel > 0 ? h2f(__ldg(xb + c)) : 0.f;
+  int c = a.n_sel > 0 ? chan(0) : 0;
+  float xc = a.n_sel > 0 ? act(0, c) : 0.f;
   uint32_t w = a.n_sel > 0 ? word_of(0, c) : 0u;
   for (int j = 0; j < a.n_sel; j++) {
-    const int cn = j + 1 < a.n_sel ? __ldg(sel + j + 1) : 0;
-    const float xn = j + 1 < a.n_sel ? h2f(__ldg(xb + cn)) : 0.f;
+    const int cn = j + 1 < a.n_sel ? chan(j + 1) : 0;
+    const float xn = j + 1 < a.n_sel ? act(j + 1, cn) : 0.f;
     const uint32_t wn = j + 1 < a.n_sel ? word_of(j + 1, cn) : 0u;
     const int g = c >> a.gshift;
     if (g != gcur) {
@@ -739,30 +663,86 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 
-size_t slot_words(int bits, int zw) {
-  if (bits == 2) return zw == 1 ? Ring<2, 1>::words : Ring<2, 2>::words;
-  if (bits == 3) return zw == 1 ? Ring<3, 1>::words : Ring<3, 2>::words;
-  return zw == 1 ? Ring<4, 1>::words : Ring<4, 2>::words;
+size_t align128(size_t v) { return (v + 127) & ~(size_t)127; }
+
+struct Plan {
+  GemvArgs a;  // shape and shared memory layout (pointers are set per launch)
+  int grid, threads, rpw, zw;
+  size_t smem;
+};
+
+// Work split and shared memory layout of one GEMV shape: segments of 2,048
+// channels, warps per segment (at most 16 compute warps), rows per stage (the
+// warps of a segment take RPW rows each), the ring depth that fits.
+sf_status make_plan(const sf_wq* w, int n_sel, Plan& P) {
+  GemvArgs& a = P.a;
+  a = GemvArgs{};
+  const int N = w->n, K = w->k;
+  a.N = N, a.K = K, a.r = w->r, a.n_sel = n_sel;
+  a.gpr = K / w->group;
+  a.gshift = 0;
+  while ((1 << a.gshift) < w->group) a.gshift++;
+  a.segs = (K + kSegCh - 1) / kSegCh;
+  SF_UNSUPPORTED(a.segs <= kMaxSegs, "k=%d above %d", K, kMaxSegs * kSegCh);
+  a.R = std::max(1, kMaxWarps / a.segs);
+  a.W = a.segs * a.R;
+  a.rowL = K * (w->b == 4 ? 4 : 2) / 8;
+  a.rowH = w->b == 3 ? K / 8 : 0;
+  a.hi_off = w->b == 3 ? (size_t)N * K / 4 : 0;
+  const size_t rowB = (size_t)a.rowL + a.rowH;
+  const int units = N / kRowUnit;
+  P.grid = std::min(num_sms(), units);
+  a.rows_max = ((units + P.grid - 1) / P.grid) * kRowUnit;
+  // four rows per warp per stage when a stage stays small and a CTA still gets
+  // two or more stages (compute starts as soon as the first one lands)
+  P.rpw = (size_t)a.R * 4 * rowB <= kStageTarget && a.rows_max >= 2 * a.R * 4 ? 4 : 2;
+  a.rc = a.R * P.rpw;
+  a.stage_bytes = (int)(a.rc * rowB);
+  a.row_words = N * w->r / 32;
+  a.wt_pitch = ((a.rows_max * w->r + 31) >> 5) + 1;
+  a.szt_pitch = (a.rows_max + 3) & ~3;
+  if (a.szt_pitch % 32 == 0) a.szt_pitch += 4;  // spread the group-major scale stores over banks
+  P.threads = (a.W + 1) * 32;
+  P.zw = w->group == 32 ? 2 : 1;
+  const int nb_max = a.rows_max / 4;
+  a.cparts = n_sel > 0 ? std::max(1, std::min(n_sel, P.threads / nb_max)) : 0;
+  size_t off = align128((2 * kMaxStages + 1) * sizeof(uint64_t));
+  a.off_sz = (int)off;
+  off += align128((size_t)a.rows_max * a.gpr * 4);
+  a.off_part = (int)off;
+  off += align128((size_t)a.rows_max * a.segs * 4);
+  // the activation planes are read once, before the correction partials are written
+  a.off_x = a.off_cpart = (int)off;
+  off += align128(std::max((size_t)a.segs * 32 * kXW * 4, (size_t)a.cparts * a.rows_max * 4));
+  if (n_sel > 0) {
+    a.off_szt = (int)off;
+    off += align128((size_t)a.gpr * a.szt_pitch * 4);
+    a.off_jd = (int)off;
+    off += align128((size_t)n_sel * 8);
+    a.off_wt = (int)off;
+    off += align128((size_t)n_sel * a.wt_pitch * 4);
+  }
+  a.off_ring = (int)off;
+  const int nst_max = (a.rows_max + a.rc - 1) / a.rc;
+  int S = std::min(kMaxStages, nst_max);
+  while (S > 1 && off + (size_t)S * a.stage_bytes > kSmemLimit) S--;
+  SF_UNSUPPORTED(off + (size_t)S * a.stage_bytes <= kSmemLimit,
+                 "n=%d, k=%d, %d selected channels: %zu bytes of shared memory needed", N, K, n_sel,
+                 off + (size_t)S * a.stage_bytes);
+  a.stages = S;
+  P.smem = off + (size_t)S * a.stage_bytes;
+  return SF_OK;
 }
 
 template <int BITS, int ZW>
-void* kernel_for(int pd) {
-  if (pd == 4) return (void*)gemv_kernel<BITS, ZW, 4>;
-  if (pd == 3) return (void*)gemv_kernel<BITS, ZW, 3>;
-  return (void*)gemv_kernel<BITS, ZW, 2>;
+void* kernel_for(int rpw) {
+  return rpw == 4 ? (void*)gemv_kernel<BITS, ZW, 4> : (void*)gemv_kernel<BITS, ZW, 2>;
 }
 
-// Rows per lane in the correction: the fewest warp steps, counting ~6 + 3 RL
-// instructions per step of RL rows.
-int pick_corr_rows(int rows) {
-  int best = 1;
-  long best_cost = -1;
-  for (int rl = 1; rl <= 4; rl *= 2) {
-    const long blocks = (rows / rl + 31) / 32;
-    const long cost = blocks * (6 + 3 * rl);
-    if (best_cost < 0 || cost < best_cost) best = rl, best_cost = cost;
-  }
-  return best;
+void* pick_kernel(int b, int zw, int rpw) {
+  if (b == 2) return zw == 1 ? kernel_for<2, 1>(rpw) : kernel_for<2, 2>(rpw);
+  if (b == 3) return zw == 1 ? kernel_for<3, 1>(rpw) : kernel_for<3, 2>(rpw);
+  return zw == 1 ? kernel_for<4, 1>(rpw) : kernel_for<4, 2>(rpw);
 }
 
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
@@ -787,85 +767,45 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
       SF_REQUIRE(sel_out && aligned16(sel_out), "sel_out is needed when sel_in is NULL");
     }
   }
-
-  GemvParams p = {};
-  p.base = (const uint32_t*)w->base;
-  p.refine = (const uint32_t*)(refine_rows ? refine_rows : w->refine);
-  p.sz = w->sz;
-  p.x = x;
-  p.y = y;
-  p.y_corr = y_corr;
-  p.N = w->n, p.K = w->k, p.G = w->group, p.r = w->r, p.batch = batch, p.n_sel = n_sel;
-  p.gshift = 0;
-  while ((1 << p.gshift) < w->group) p.gshift++;
-  p.segs = (w->k + kSegChannels - 1) / kSegChannels;
-  p.refine_row_words = w->n * w->r / 32;
-  p.staged = refine_rows != nullptr;
-
-  const int zw = w->group == 32 ? 2 : 1;
-  int grid = num_sms();
-  const int units = w->n / kRowUnit;
-  if (grid > units) grid = units;
-  p.rows_max = ((units + grid - 1) / grid) * kRowUnit;
-  p.w_span = p.rows_max * w->r / 32 + 2;
-  p.corr_rows = pick_corr_rows(p.rows_max);
-  p.plane_words = (w->k / kLaneCh) * kXWords + kWarps * 4 * kLaneCh;  // planes, then per-warp scratch
-  const size_t gpr = (size_t)(w->k / w->group);
-  p.pstride = p.segs + 1;
-  const size_t part_words = ((size_t)p.rows_max * p.pstride + 3) & ~(size_t)3;
-  const size_t table_words = (size_t)n_sel * 4 + (((size_t)n_sel * p.w_span + 3) & ~(size_t)3) +
-                             (size_t)p.rows_max * gpr;
-  const size_t limit_words = kSmemLimit / 4;
-  const size_t fixed = part_words + p.plane_words;
-  // ring depth: the deepest that leaves room for the correction tables, else
-  // the deepest that fits (the tables then go through the ring area in chunks)
-  int pd = 0;
-  size_t area = 0;
-  for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
-    const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
-    if (fixed + ring + (n_sel > 0 ? table_words : 0) <= limit_words) pd = d, area = ring, p.fast = n_sel > 0;
-  }
-  for (int d = (w->b == 3 ? 3 : 4); d >= 2 && !pd; d--) {
-    const size_t ring = (size_t)kWarps * d * slot_words(w->b, zw);
-    if (fixed + ring <= limit_words) pd = d, area = ring, p.fast = 0;
-  }
-  SF_UNSUPPORTED(pd > 0, "n=%d, k=%d does not fit in shared memory", w->n, w->k);
-  p.corr_split = p.fast && area >= (size_t)kWarps * p.rows_max;
-  if (!p.fast && n_sel > 0)
-    SF_UNSUPPORTED(area >= (size_t)(4 + p.w_span) * 16, "n=%d, k=%d: no room for the correction", w->n, w->k);
-  const size_t smem = (fixed + area + (p.fast ? table_words : 0)) * 4;
-  SF_UNSUPPORTED(smem <= kSmemLimit, "n=%d, k=%d needs %zu bytes of shared memory", w->n, w->k, smem);
-  p.area_words = (int)area;
+  Plan P;
+  st = make_plan(w, n_sel, P);
+  if (st != SF_OK) return st;
 
   // the selection (when not given), then the GEMV, which waits for it (and for
   // x) through programmatic dependent launch while its first code copies fly
+  const int32_t* sel = sel_in;
   if (kch > 0 && !sel_in) {
     st = launch_select(x, batch, w->k, chunk, kch, sel_out, s, true);
     if (st != SF_OK) return st;
-    p.sel = sel_out;
-  } else {
-    p.sel = sel_in;
+    sel = sel_out;
   }
+  void* kern = pick_kernel(w->b, P.zw, P.rpw);
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(P.grid);
+  cfg.blockDim = dim3(P.threads);
+  cfg.dynamicSmemBytes = P.smem;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  void* kern;
-  if (w->b == 2)
-    kern = zw == 1 ? kernel_for<2, 1>(pd) : kernel_for<2, 2>(pd);
-  else if (w->b == 3)
-    kern = zw == 1 ? kernel_for<3, 1>(pd) : kernel_for<3, 2>(pd);
-  else
-    kern = zw == 1 ? kernel_for<4, 1>(pd) : kernel_for<4, 2>(pd);
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit));
-  void* args[] = {&p};
-  SF_CUDA(cudaLaunchKernelExC(&cfg, kern, args));
+  // one launch per batch row: each streams the codes once for its row
+  for (int b = 0; b < batch; b++) {
+    GemvArgs a = P.a;
+    a.base = (const uint8_t*)w->base;
+    a.sz = (const uint32_t*)w->sz;
+    a.staged = refine_rows != nullptr;
+    a.refine = refine_rows ? (const uint32_t*)refine_rows + (size_t)b * n_sel * a.row_words
+                           : (const uint32_t*)w->refine;
+    a.x = x + (size_t)b * w->k;
+    a.sel = sel ? sel + (size_t)b * n_sel : nullptr;
+    a.y = y + (size_t)b * w->n;
+    a.y_corr = y_corr ? y_corr + (size_t)b * w->n : nullptr;
+    void* args[] = {&a};
+    SF_CUDA(cudaLaunchKernelExC(&cfg, kern, args));
+  }
   return SF_OK;
 }
 
@@ -932,4 +872,18 @@ extern "C" sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, in
   const char *a0 = (const char*)y_base, *b0 = (const char*)y_corr;
   SF_REQUIRE(!y_base || a0 + bytes <= b0 || b0 + bytes <= a0, "y_base and y_corr overlap");
   return gemv_launch(w, x, batch, chunk, kch, sel_in, nullptr, refine_rows, y_base, as_stream(stream), y_corr);
+}
+
+extern "C" sf_status sf_device_wait_timeouts(unsigned int* count, int reset) {
+  SF_REQUIRE(count, "count must be non-null");
+  SF_CUDA(cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned int)));
+  if (reset) {
+    const unsigned int zero = 0;
+    SF_CUDA(cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned int)));
+  }
+  if (*count) {
+    set_error("%u bounded device wait(s) ran out", *count);
+    return SF_ERR_TIMEOUT;
+  }
+  return SF_OK;
 }

@@ -21,16 +21,17 @@
 //                   integers in registers and contracted on the tensor cores
 //                   (mma.sync m16n8k16, fp32 accumulation); the per-token fp16
 //                   steps/offsets are applied in fp32.
-//   kv_post_kernel  one thread-block cluster per KV head: softmax statistics
-//                   from the partials, token scores, a cluster-wide radix
-//                   select of the top k_tok (histograms exchanged through
-//                   distributed shared memory), then the correction of the
-//                   selected tokens (each token's base contribution swapped
-//                   for its refined one, relative to the head's softmax
-//                   maximum) and the log-sum-exp merge of the partials.
+//   kv_select_kernel  scores every token (sum over the group's query heads of
+//                   the softmax probability, from the stored logits and the
+//                   statistics of the partials) and selects the top k_tok per
+//                   KV head: a histogram of the score bits, then, in the last
+//                   CTA of the head, the exact k_tok-th score and the selected
+//                   tokens in ascending order;
+//   kv_refine_kernel  swaps the selected tokens' base contributions for
+//                   their refined ones (relative to the head's softmax
+//                   maximum) and merges the partials by log-sum-exp.
 // The result equals softmax(q.k~) v~ with refined k~, v~ on the selected
 // tokens, up to fp32 rounding.
-#include <cooperative_groups.h>
 
 #include <algorithm>
 #include <cfloat>
@@ -46,16 +47,13 @@ constexpr int kD = kHeadDim;
 constexpr int kRec = kD + 2;     // partial record: acc[kD], m, l
 constexpr int kWarps = 4;        // warps per base-pass CTA (independent splits)
 constexpr int kStages = 4;       // cp.async ring depth per warp
+constexpr int kCtlWords = 2048 + 4;  // per head: selection histogram and two counters (kCtl below)
 
 // ---- small PTX helpers -------------------------------------------------------
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
-  uint32_t sa = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -128,6 +126,7 @@ struct BaseArgs {
   int h_q, gq;
   float* logits;  // [batch][h_q][T]
   float* part;    // [batch][h_q][nrec][rec]  (rec = kRec with values, 2 without)
+  int* ctl;       // [batch][h_kv][kCtl]: zeroed here for the kernels after the base pass
   int span, nsplit, nrec;
   float scale;
 };
@@ -162,6 +161,10 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int g = blockIdx.y, bat = blockIdx.z;
+  if (blockIdx.x == 0 && a.ctl) {  // the histogram and counters of the kernels after this one
+    int* c = a.ctl + ((long)bat * a.h_kv + g) * kCtlWords;
+    for (int i = threadIdx.x; i < kCtlWords; i += blockDim.x) c[i] = 0;
+  }
   const int split = blockIdx.x * kWarps + warp;
   uint8_t* wsm = smem + warp * WS::bytes;
   float* Zs = reinterpret_cast<float*>(wsm + WS::ring);        // [PV+1][16][4][2]
@@ -484,82 +487,345 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// after the base pass: one thread-block cluster per (batch, KV head)
+// after the base pass: scoring and selection, then refinement and merge
 //
-// The cluster's CTAs split the context: each scores its tokens (sum over the
-// group's query heads of the softmax probability, from the stored base
-// logits) into shared memory.  The k_tok-th largest score is found by a radix
-// select over the score bits (non-negative floats order like their bits),
-// 9 bits per pass from bit 30: every CTA histograms its keys, stores the
-// histogram into every peer's shared memory (distributed shared memory) and,
-// after the cluster barrier, all CTAs take the same decision from their local
-// copies.  Equal scores rank the lower token first; the selected tokens are
-// written in ascending order and also handed, by position, to the CTA that
-// refines them.  Each CTA then copies its share of the selected tokens' codes
-// and scales into shared memory with cp.async in one go and refines them, each
-// warp four tokens together (swapping each token's base contribution for its
-// refined one, relative to the head's softmax maximum; the refined logits of
-// the warp's (token, head) slots summed by one transposed butterfly, each
-// warp's sums kept in its own slot rather than added with shared-memory
-// atomics), sums an interleaved share of the base partial records, and CTA h
-// merges query head h.
+// kv_select_kernel -- CTAs of kSelThreads threads over slices of kSelTok
+// tokens of one (batch, KV head).  Each computes the softmax statistics of the
+// group's query heads from the base pass's split records, the scores of its
+// tokens from the stored logits (written out: the sum over the group's query
+// heads of each head's softmax probability), and the histogram of the score
+// keys' bits 30..20, added into the head's histogram in the workspace.  Scores
+// are non-negative, so their bit patterns order like their values; bits 30..20
+// are the exponent and the top three mantissa bits.  The last CTA of the head
+// to finish (an atomic counter: no CTA ever waits for another) selects: the
+// bucket that holds the k_tok-th largest key, from the histogram; one pass
+// over the scores marks every token of a higher bucket in a shared-memory
+// bitmap and collects the boundary bucket's keys and tokens; two 10-bit digits
+// over those pin the k_tok-th largest key K* exactly; the collected tokens
+// above K* are marked, and of the tokens equal to K* the lowest-indexed ones;
+// the marked tokens are written in ascending order.
+//
+// kv_refine_kernel -- kRefParts CTAs per (batch, KV head), each with a share
+// of the selected tokens and of the base pass's split records.  Per selected
+// token a warp reads its base and refinement codes and scales, swaps the
+// token's base contribution for its refined one (weights relative to the
+// head's softmax maximum: numerator v~ exp(l~ - M) - v^ exp(l^ - M), the
+// denominator likewise), and adds the CTA's records rescaled to M; the last
+// CTA of the head to finish divides the summed numerators by the summed
+// denominators.
 
-constexpr int kPostThreads = 512;
-constexpr int kPostMaxTok = 16640;  // tokens per CTA scored in shared memory (cluster of 8)
-constexpr int kPostCl = 8;
-constexpr int kPostStage = 64;      // selected tokens staged in shared memory at a time
-constexpr int kPostMaxSel = 512;    // selected tokens per CTA (k_tok <= 4096)
-constexpr int kMaxKTok = 4096;      // the largest k_tok every attention entry point accepts
-static_assert(kPostCl * kPostMaxSel == kMaxKTok, "the cluster's selection buffers must hold k_tok tokens");
-constexpr int kHistBins = 512;
-// a warp's share of one staging batch, times 8 query heads, fits its 32 lanes
-static_assert(kPostStage / (kPostThreads / 32) * 8 <= 32, "staging batch too large for the lane layout");
-// the per-warp partial numerators reuse the score keys' space
-static_assert((kPostThreads / 32) * 8 * kD <= kPostMaxTok, "key space too small for the partial numerators");
+constexpr int kSelThreads = 512;
+constexpr int kSelTok = 2048;        // tokens scored per CTA
+constexpr int kBins1 = 2048;         // first digit: key bits 30..20
+constexpr int kBins2 = 1024;         // then bits 19..10 and 9..0
+constexpr int kCandCap = 4096;       // boundary-bucket keys held in shared memory
+constexpr int kMaxT = 1 << 18;       // tokens a head's bitmap holds in shared memory
+constexpr int kCtl = kBins1 + 4;     // per head: histogram, selection counter, refinement counter
+static_assert(kCtl == kCtlWords, "the base pass zeroes exactly the control words");
+constexpr int kRefThreads = 256;
+constexpr int kRefWarps = kRefThreads / 32;
+constexpr int kRefTPW = 4;           // tokens a warp refines together
+constexpr int kRefPartsMax = 16;     // CTAs per head that refine
+constexpr int kMaxKTok = 4096;       // the largest k_tok every attention entry point accepts
+static_assert(kRefTPW * 8 <= 32, "a warp's (token, head) slots must fit its lanes");
 
-struct PostArgs {
+// Softmax statistics of query head h from the split records: M = max m,
+// Z = sum l exp(m - M).  One warp.
+__device__ __forceinline__ void head_stats(const float* __restrict__ pr, int nrec, int rec, int lane, float& M,
+                                           float& Z) {
+  float m = -INFINITY;
+  for (int s = lane; s < nrec; s += 32) m = fmaxf(m, pr[(long)s * rec + rec - 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float z = 0.f;
+  if (m > -INFINITY)
+    for (int s = lane; s < nrec; s += 32) {
+      const float ms = pr[(long)s * rec + rec - 2];
+      if (ms > -INFINITY) z += pr[(long)s * rec + rec - 1] * expf(ms - m);
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  M = m, Z = z;
+}
+
+// Exclusive prefix sum of v over the block's threads (in thread order), and the
+// total.  ws: 32 ints of shared memory.
+template <int NT>
+__device__ __forceinline__ int block_exclusive_sum(int v, int* ws, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  __syncthreads();  // ws may still be read by a previous call
+  if (lane == 31) ws[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int wv = lane < NT / 32 ? ws[lane] : 0;
+    int x = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += u;
+    }
+    if (lane < NT / 32) ws[lane] = x - wv;
+    if (lane == 31) ws[NT / 32] = x;
+  }
+  __syncthreads();
+  total = ws[NT / 32];
+  return ws[warp] + incl - v;
+}
+
+// The bucket of the kneed-th largest key: hist[0, nb) counts keys per digit;
+// bucket b is taken when the keys of higher buckets number fewer than kneed
+// and those at or above it kneed or more.  Returns b; *kleft = kneed minus the
+// keys above b.  Every thread gets the result.
+template <int NT>
+__device__ int find_bucket(const int* __restrict__ hist, int nb, int kneed, int* ws, int* res, int* kleft) {
+  const int per = nb / NT;  // 2 or 4 bins per thread, from the top
+  int c[4], tot = 0;
+#pragma unroll
+  for (int j = 0; j < 4; j++) {
+    c[j] = j < per ? hist[nb - 1 - per * (int)threadIdx.x - j] : 0;
+    tot += c[j];
+  }
+  int all;
+  const int above = block_exclusive_sum<NT>(tot, ws, all);
+  if (above < kneed && above + tot >= kneed) {
+    int run = above;
+    for (int j = 0; j < per; j++) {
+      if (run + c[j] >= kneed) {
+        res[0] = nb - 1 - per * (int)threadIdx.x - j;
+        res[1] = kneed - run;
+        break;
+      }
+      run += c[j];
+    }
+  }
+  __syncthreads();
+  *kleft = res[1];
+  return res[0];
+}
+
+struct SelArgs {
+  const float* logits;  // [batch][h_q][T] base logits (scaled)
+  const float* part;    // [batch][h_q][nrec][rec]
+  int nrec, rec;
+  int h_kv, h_q, gq, T, Tp, k_tok, nblk;
+  float* scores;        // [batch][h_kv][Tp] (Tp = T rounded up to 32: whole 16-byte rows)
+  float* scores_out;    // nullable [batch][h_kv][T]: the scores for the caller
+  int* ctl;             // [batch][h_kv][kCtl]
+  int32_t* sel;         // [batch][h_kv][k_tok]
+};
+
+struct SelShared {
+  int hist[kBins1];
+  int ws[40];
+  int res[2];
+  int ncand, last;
+  float M[8], iZ[8];
+};
+
+// Dynamic shared memory of a selection CTA: the bitmap of selected tokens,
+// the boundary bucket's keys and tokens, per-thread tie counts.
+constexpr size_t kSelDyn = (size_t)(kMaxT / 32) * 4 + (size_t)kCandCap * 8 + (size_t)kSelThreads * 4;
+
+template <int GQP>
+__global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
+  __shared__ SelShared sh;
+  extern __shared__ __align__(16) uint32_t dyn_sel[];
+  uint32_t* bits = dyn_sel;                                    // [kMaxT / 32]
+  uint32_t* ck = bits + kMaxT / 32;                            // [kCandCap] keys
+  int* ct = reinterpret_cast<int*>(ck + kCandCap);             // [kCandCap] tokens
+  int* tie = ct + kCandCap;                                    // [kSelThreads]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.y, bat = blockIdx.z, gq = a.gq;
+  const long hq0 = (long)bat * a.h_q + (long)g * gq;
+  const long head = (long)bat * a.h_kv + g;
+  pdl_trigger();
+  pdl_wait();  // the base pass (logits, records, zeroed histogram) is complete
+
+  if (warp < gq) {
+    float M, Z;
+    head_stats(a.part + (hq0 + warp) * a.nrec * a.rec, a.nrec, a.rec, lane, M, Z);
+    if (lane == 0) sh.M[warp] = M, sh.iZ[warp] = 1.0f / Z;
+  }
+  for (int i = tid; i < kBins1; i += kSelThreads) sh.hist[i] = 0;
+  __syncthreads();
+
+  // ---- scores of this CTA's tokens and their histogram
+  float* sc = a.scores + head * a.Tp;
+  float* sco = a.scores_out ? a.scores_out + head * a.T : nullptr;
+  {
+    const int t0 = blockIdx.x * kSelTok, t1 = min(a.T, t0 + kSelTok);
+    const float* lg = a.logits + hq0 * a.T;
+    constexpr int U = kSelTok / kSelThreads;
+    float l[GQP][U];
+#pragma unroll
+    for (int h = 0; h < GQP; h++)
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int t = t0 + tid + kSelThreads * u;
+        l[h][u] = (h < gq && t < t1) ? lg[(long)h * a.T + t] : -INFINITY;
+      }
+#pragma unroll
+    for (int u = 0; u < U; u++) {
+      const int t = t0 + tid + kSelThreads * u;
+      if (t < t1) {
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < GQP; h++)
+          if (h < gq) s += expf(l[h][u] - sh.M[h]) * sh.iZ[h];  // full-accuracy exp: the score decides
+        sc[t] = s;
+        if (sco) sco[t] = s;
+        atomicAdd(&sh.hist[__float_as_uint(s) >> 20], 1);
+      }
+    }
+  }
+  __syncthreads();
+  int* gh = a.ctl + head * kCtl;
+  for (int i = tid; i < kBins1; i += kSelThreads)
+    if (sh.hist[i]) atomicAdd(&gh[i], sh.hist[i]);
+  __threadfence();  // this CTA's scores and histogram before its count
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(&gh[kBins1], 1) == a.nblk - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();  // every other CTA's scores and histogram are visible
+
+  // ---- the last CTA of the head selects
+  const int T = a.T;
+  const int nw = (T + 31) / 32;                       // bitmap words
+  const int wper = (nw + kSelThreads - 1) / kSelThreads;
+  const int w0 = min(nw, tid * wper), w1 = min(nw, w0 + wper);
+  for (int i = tid; i < kBins1; i += kSelThreads) sh.hist[i] = __ldcg(gh + i);
+  if (tid == 0) sh.ncand = 0;
+  tie[tid] = 0;
+  __syncthreads();
+  int kneed;
+  const uint32_t b1 = (uint32_t)find_bucket<kSelThreads>(sh.hist, kBins1, a.k_tok, sh.ws, sh.res, &kneed);
+  // one pass: higher buckets marked, the boundary bucket collected
+  for (int w = w0; w < w1; w++) {
+    uint32_t key[32];
+    if (32 * w + 32 <= T) {  // a whole word of scores: eight 16-byte loads
+#pragma unroll
+      for (int v = 0; v < 8; v++) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + 32 * w) + v);
+        key[4 * v] = __float_as_uint(f.x), key[4 * v + 1] = __float_as_uint(f.y);
+        key[4 * v + 2] = __float_as_uint(f.z), key[4 * v + 3] = __float_as_uint(f.w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; i++) key[i] = 32 * w + i < T ? __float_as_uint(__ldcg(sc + 32 * w + i)) : 0u;
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+      const uint32_t d = key[i] >> 20;
+      if (32 * w + i < T && d > b1) m |= 1u << i;
+      if (32 * w + i < T && d == b1) {
+        const int slot = atomicAdd(&sh.ncand, 1);
+        if (slot < kCandCap) ck[slot] = key[i], ct[slot] = 32 * w + i;
+      }
+    }
+    bits[w] = m;
+  }
+  __syncthreads();
+  const int ncand = sh.ncand;
+  const bool in_smem = ncand <= kCandCap;
+  // the boundary bucket's keys: from shared memory, or (when too many) the scores again
+  auto for_cands = [&](auto&& f) {
+    if (in_smem) {
+      for (int j = tid; j < ncand; j += kSelThreads) f(ck[j], ct[j]);
+    } else {
+      for (int t = tid; t < T; t += kSelThreads) {
+        const uint32_t key = __float_as_uint(__ldcg(sc + t));
+        if ((key >> 20) == b1) f(key, t);
+      }
+    }
+  };
+  uint32_t prefix = b1 << 20, mask = 0xFFF00000u;
+#pragma unroll 1
+  for (int shift = 10; shift >= 0; shift -= 10) {
+    for (int i = tid; i < kBins2; i += kSelThreads) sh.hist[i] = 0;
+    __syncthreads();
+    for_cands([&](uint32_t key, int t) {
+      (void)t;
+      if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & (kBins2 - 1)], 1);
+    });
+    __syncthreads();
+    int kl;
+    const uint32_t d = (uint32_t)find_bucket<kSelThreads>(sh.hist, kBins2, kneed, sh.ws, sh.res, &kl);
+    kneed = kl;
+    prefix |= d << shift;
+    mask |= (uint32_t)(kBins2 - 1) << shift;
+  }
+  // prefix is the k_tok-th largest key K*; kneed of the keys equal to it are taken
+  const int tok_per = 32 * wper;
+  for_cands([&](uint32_t key, int t) {
+    if (key > prefix) atomicOr(&bits[t >> 5], 1u << (t & 31));
+    else if (key == prefix) atomicAdd(&tie[t / tok_per], 1);
+  });
+  __syncthreads();
+  int ties_all;
+  const int ties_before = block_exclusive_sum<kSelThreads>(tie[tid], sh.ws, ties_all);
+  const int take = max(0, min(tie[tid], kneed - ties_before));
+  if (take > 0) {  // the first `take` of this thread's tied tokens, in token order
+    int taken = 0;
+    for (int w = w0; w < w1 && taken < take; w++) {
+      uint32_t m = bits[w];
+      for (int i = 0; i < 32 && taken < take; i++) {
+        const int t = 32 * w + i;
+        if (t < T && __float_as_uint(__ldcg(sc + t)) == prefix) m |= 1u << i, taken++;
+      }
+      bits[w] = m;
+    }
+  }
+  __syncthreads();
+  int cnt = 0;
+  for (int w = w0; w < w1; w++) cnt += __popc(bits[w]);
+  int total;
+  int pos = block_exclusive_sum<kSelThreads>(cnt, sh.ws, total);
+  int32_t* out = a.sel + head * a.k_tok;
+  for (int w = w0; w < w1; w++) {
+    uint32_t m = bits[w];
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1;
+      if (pos < a.k_tok) out[pos] = 32 * w + i;
+      pos++;
+    }
+  }
+}
+
+struct RefArgs {
   const uint8_t *kb, *kr, *vb, *vr;
   const uint16_t *ksz, *vsz;
-  int h_kv, t_max, b, r, T;
+  int h_kv, t_max, T;
   const uint16_t* q;
   int h_q, gq;
-  const float* logits;  // base logits [batch][h_q][T]
-  const float* part;    // base partial records [batch][h_q][nrec][rec]
-  int nrec, rec;        // rec = kRec (with values) or 2 (scores only)
-  int k_tok;
-  int32_t* sel;         // [batch][h_kv][k_tok]: written when select, else read
-  int select;
-  float* scores;        // nullable [batch][h_kv][T]
+  const float* logits;  // base logits (scaled), [batch][h_q][T]
+  const float* part;    // [batch][h_q][nrec][kRec]
+  int nrec;
+  int k_tok, parts;
+  const int32_t* sel;   // [batch][h_kv][k_tok]
+  int* ctl;             // [batch][h_kv][kCtl]
+  float* rpart;         // [batch][h_kv][parts][gq][kD + 1]
   float* out;           // nullable [batch][h_q][kD]
-  uint16_t* out16;      // nullable [batch][h_q][kD], the same rounded to fp16
-  int chunk;            // tokens per CTA
+  uint16_t* out16;      // nullable [batch][h_q][kD]
   float scale;
 };
 
-struct PostShared {
-  int hist[kHistBins];  // this CTA's histogram of the current pass
-  int tot[kHistBins];
-  int warp_tot[32];
-  int cnt;
-  int digit, kleft, done;
+template <int GQP>
+struct RefShared {
   float M[8], Z[8];
-  float wden[kPostThreads / 32][8];      // per warp: its tokens' change of each head's denominator
-  float wtab[kPostThreads / 32][2 * 32];  // per warp: (w_refined, w_base) of its (token, head) slots
+  float num[kRefWarps][GQP][kD];
+  float den[kRefWarps][GQP];
+  float2 wtab[kRefWarps][kRefTPW * GQP];
+  int last;
 };
-
-// Filled by the peers (distributed shared memory stores, which do not stall the
-// writer); read locally after a cluster barrier.
-struct PostMail {
-  int hist[2][kPostCl][kHistBins];  // per pass (alternating): every CTA's histogram
-  int cnt[kPostCl];                 // every CTA's packed (above, equal) counts
-  int tok[kPostMaxSel];             // the selected tokens this CTA refines, by position
-  float num[kPostCl][kD];           // this CTA's query head: every CTA's partial numerator
-  float den[kPostCl];
-};
-
-// Words of one staged token: K codes (4b), K refinement (4r), K and V (s, m)
-// (4 + 4), the token's 8 value chunks of codes (8 x 2b) and refinement (8 x 2r).
-__host__ __device__ constexpr int tok_words(int b, int r) { return 20 * (b + r) + 8; }
 
 // Sums each of the N (16 or 32) per-lane values v over the warp; returns the
 // sum of value lane % N.  Each round keeps the half of the values that the
@@ -584,425 +850,192 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
 // GQP: query heads per KV head, padded to 4 or 8 (register arrays); B, R:
 // the cache's base and refinement bits.
 template <int GQP, int B, int R>
-__global__ void __launch_bounds__(kPostThreads, 1) kv_post_kernel(PostArgs a) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int cr = (int)cluster.block_rank(), CL = (int)cluster.num_blocks();
-  extern __shared__ __align__(16) uint8_t dyn[];
-  PostMail& mail = *reinterpret_cast<PostMail*>(dyn);
-  uint32_t* stage = reinterpret_cast<uint32_t*>(dyn + sizeof(PostMail));  // staged selected tokens
-  uint32_t* keys = stage + kPostStage * tok_words(B, R);               // this CTA's score keys
-  __shared__ PostShared sh;
+__global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
+  __shared__ RefShared<GQP> sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = kPostThreads / 32;
-  const int g = blockIdx.y, bat = blockIdx.z;
-  const int gq = a.gq;
+  const int part = blockIdx.x, g = blockIdx.y, bat = blockIdx.z, gq = a.gq;
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
+  const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
-  // every CTA of the cluster must have started before peers touch its shared
-  // memory: arrive now, wait right before the first distributed access
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  pdl_wait();  // the base pass is complete
-
-  // softmax statistics of the group's query heads: every record's (m, l)
-  // loaded in one batch per lane
+  pdl_wait();  // the base pass and the selection are complete
   if (warp < gq) {
-    const float* pr = a.part + (hq0 + warp) * a.nrec * a.rec;
-    constexpr int PER = 8;
-    float ms[PER], ls[PER];
-    float m = -INFINITY, z = 0.f;
-    for (int s0 = 0; s0 < a.nrec; s0 += 32 * PER) {
-#pragma unroll
-      for (int k = 0; k < PER; k++) {
-        const int s = s0 + lane + 32 * k;
-        ms[k] = s < a.nrec ? pr[(long)s * a.rec + a.rec - 2] : -INFINITY;
-        ls[k] = s < a.nrec ? pr[(long)s * a.rec + a.rec - 1] : 0.f;
-      }
-      float mb = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < PER; k++) mb = fmaxf(mb, ms[k]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      const float mn = fmaxf(m, mb);
-      float zb = 0.f;
-#pragma unroll
-      for (int k = 0; k < PER; k++)
-        if (ms[k] > -INFINITY) zb += ls[k] * expf(ms[k] - mn);
-      z = (m > -INFINITY ? z * expf(m - mn) : 0.f) + zb;
-      m = mn;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) sh.M[warp] = m, sh.Z[warp] = z;
+    float M, Z;
+    head_stats(a.part + (hq0 + warp) * a.nrec * kRec, a.nrec, kRec, lane, M, Z);
+    if (lane == 0) sh.M[warp] = M, sh.Z[warp] = Z;
   }
   __syncthreads();
 
-  const int ja = (int)((long)cr * a.k_tok / CL), jb = (int)((long)(cr + 1) * a.k_tok / CL);
-  if (a.select) {
-    const int t0 = cr * a.chunk, n = max(0, min(a.T, t0 + a.chunk) - t0);
-    const float* lg = a.logits + hq0 * a.T + t0;
-    float Mh[GQP], invZ[GQP];
+  // ---- the refined contribution of this CTA's share of the selected tokens
+  const int ja = (int)((long)part * a.k_tok / a.parts), jb = (int)((long)(part + 1) * a.k_tok / a.parts);
+  const float half = 0.5f * (float)(1 << R), inv = 1.0f / (float)(1 << R);
+  const uint32_t bmask = (1u << B) - 1u, rmask = (1u << R) - 1u;
+  const long slot0 = head * a.t_max;
+  int kw[4], kbit[4], krw[4], krbit[4];
+  float qv[GQP][4];
 #pragma unroll
-    for (int h = 0; h < GQP; h++) Mh[h] = h < gq ? sh.M[h] : 0.f, invZ[h] = h < gq ? 1.0f / sh.Z[h] : 0.f;
-    // eight tokens per thread per step (token tid + 512 e: coalesced), every load
-    // of the step issued first
-    constexpr int TPT = 8;
-    for (int i0 = tid; i0 < n; i0 += TPT * kPostThreads) {
-      float l[GQP][TPT];
+  for (int e = 0; e < 4; e++) {
+    key_pos(lane + 32 * e, B, kw[e], kbit[e]);
+    key_pos(lane + 32 * e, R, krw[e], krbit[e]);
 #pragma unroll
-      for (int h = 0; h < GQP; h++)
-#pragma unroll
-        for (int e = 0; e < TPT; e++) {
-          const int i = i0 + e * kPostThreads;
-          l[h][e] = (h < gq && i < n) ? lg[(long)h * a.T + i] : -INFINITY;
-        }
-#pragma unroll
-      for (int e = 0; e < TPT; e++) {
-        const int i = i0 + e * kPostThreads;
-        if (i < n) {
-          float sc = 0.f;
-#pragma unroll
-          for (int h = 0; h < GQP; h++)
-            if (h < gq) sc += expf(l[h][e] - Mh[h]) * invZ[h];  // full-accuracy exp: the score decides the selection
-          if (a.scores) a.scores[((long)bat * a.h_kv + g) * a.T + t0 + i] = sc;
-          keys[i] = __float_as_uint(sc);
-        }
-      }
-    }
-    // ---- radix select of the k_tok-th largest key over the cluster: digits of
-    // bits 30..22, 21..13, 12..4, 3..0 (bit 31 is 0 for non-negative scores)
-    uint32_t prefix = 0, mask = 0x80000000u;
-    int kleft = a.k_tok, buf = 0;
-    bool done = false;
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    for (int pass = 0; pass < 4 && !done; pass++) {
-      const int shift = pass < 3 ? 22 - 9 * pass : 0;
-      const int bits = pass < 3 ? 9 : 4, bins = 1 << bits;
-      for (int i = tid; i < bins; i += kPostThreads) sh.hist[i] = 0;
-      __syncthreads();
-      for (int i0 = warp * 32; i0 < n; i0 += kPostThreads) {  // whole warps: lanes with equal bins add once
-        const int i = i0 + lane;
-        const uint32_t key = i < n ? keys[i] : 0u;
-        const bool in = i < n && (key & mask) == prefix;
-        const int bn = in ? (int)((key >> shift) & (bins - 1)) : -1;
-        const unsigned same = __match_any_sync(0xffffffffu, bn);
-        if (in && (__ffs(same) - 1) == lane) atomicAdd(&sh.hist[bn], __popc(same));
-      }
-      __syncthreads();
-      for (int i = tid; i < bins * CL; i += kPostThreads)  // my histogram into every peer's mailbox
-        cluster.map_shared_rank(&mail.hist[buf][cr][0], i / bins)[i % bins] = sh.hist[i % bins];
-      cluster.sync();  // every CTA's histogram is in every mailbox
-      for (int bn = tid; bn < bins; bn += kPostThreads) {
-        int t = 0;
-        for (int rk = 0; rk < CL; rk++) t += mail.hist[buf][rk][bn];
-        sh.tot[bn] = t;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane covers the bins below bins - 1 - PL lane, from the top
-        const int PL = bins >= 32 ? bins / 32 : 1;
-        int c[16], tot = 0;
-#pragma unroll
-        for (int j = 0; j < 16; j++) {
-          const int bn = bins - 1 - PL * lane - j;
-          c[j] = (j < PL && bn >= 0) ? sh.tot[bn] : 0;
-          tot += c[j];
-        }
-        int incl = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        const int above = incl - tot;
-        if (above < kleft && incl >= kleft) {
-          int run = above;
-          for (int j = 0; j < PL; j++) {
-            if (run + c[j] >= kleft) {
-              sh.digit = bins - 1 - PL * lane - j;
-              sh.kleft = kleft - run;
-              sh.done = c[j] == kleft - run;  // the whole bucket is needed
-              break;
-            }
-            run += c[j];
-          }
-        }
-      }
-      __syncthreads();
-      prefix |= (uint32_t)sh.digit << shift;
-      mask |= (uint32_t)(bins - 1) << shift;
-      kleft = sh.kleft;
-      done = sh.done;
-      buf ^= 1;  // the next pass fills the other mailbox while this one may still be read
-    }
-    // keys above `prefix` (or, when the last bucket was taken whole, at or above
-    // it) are selected; of the keys equal to it, the first `kleft` in token order
-    const int per = (n + kPostThreads - 1) / kPostThreads;
-    const int i0 = min(n, tid * per), i1 = min(n, i0 + per);
-    int ngt = 0, neq = 0;
-    for (int i = i0; i < i1; i++) {
-      const uint32_t key = keys[i];
-      if (done ? key >= prefix : key > prefix) ngt++;
-      else if (!done && key == prefix) neq++;
-    }
-    // one block scan of the packed counts (above + equal << 16), in token order
-    const int v = ngt + (neq << 16);
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += u;
-    }
-    if (lane == 31) sh.warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int wv = lane < NW ? sh.warp_tot[lane] : 0;
-      int x = wv;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += u;
-      }
-      if (lane < NW) sh.warp_tot[lane] = x - wv;
-      if (lane == 31) sh.cnt = x;
-    }
-    __syncthreads();
-    const int ex = sh.warp_tot[warp] + incl - v;
-    const int gt_ex = ex & 0xFFFF, eq_ex = ex >> 16;
-    if (tid < CL) cluster.map_shared_rank(&mail.cnt[cr], tid)[0] = sh.cnt;
-    cluster.sync();  // every CTA's counts are in every mailbox
-    int sel_before = 0, eq_before = 0;
-    for (int rk = 0; rk < cr; rk++) {
-      const int c = mail.cnt[rk];
-      sel_before += (c & 0xFFFF) + max(0, min(c >> 16, kleft - eq_before));
-      eq_before += c >> 16;
-    }
-    // my selected tokens: above-threshold ones, and equal ones while the budget lasts
-    const int eq_mine = done ? 0 : max(0, min(neq, kleft - (eq_before + eq_ex)));
-    int pos = sel_before + gt_ex + max(0, min(eq_ex, kleft - eq_before));
-    int eq_seen = 0;
-    int32_t* selw = a.sel + ((long)bat * a.h_kv + g) * a.k_tok;
-    for (int i = i0; i < i1; i++) {
-      const uint32_t key = keys[i];
-      bool take = done ? key >= prefix : key > prefix;
-      if (!done && key == prefix) take = eq_seen++ < eq_mine;
-      if (take && pos < a.k_tok) {
-        selw[pos] = t0 + i;
-        if (a.out || a.out16) {  // hand the token to the CTA that refines position pos
-          const int dst = (int)(((long)(pos + 1) * CL + a.k_tok - 1) / a.k_tok) - 1;
-          const int dja = (int)((long)dst * a.k_tok / CL);
-          cluster.map_shared_rank(&mail.tok[0], dst)[pos - dja] = t0 + i;
-        }
-      }
-      if (take) pos++;
-    }
-    cluster.sync();  // every selected token is in its refining CTA's mailbox
-  } else {
-    const int32_t* selg = a.sel + ((long)bat * a.h_kv + g) * a.k_tok;
-    for (int j = ja + tid; j < jb; j += kPostThreads) mail.tok[j - ja] = selg[j];
-    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    __syncthreads();
+    for (int h = 0; h < GQP; h++) qv[h][e] = h < gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
   }
-  if (!a.out && !a.out16) return;  // no peer reads or writes this CTA's shared memory any more
-
-  // ---- refined attention on this CTA's share of the selected tokens
-  {
-    const int W = tok_words(B, R);
-    const int oK = 0, oKr = 4 * B, oZk = 4 * (B + R), oZv = oZk + 4, oV = oZv + 4, oVr = oV + 16 * B;
-    const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
-    const float half = 0.5f * (float)(1 << R), inv = 1.0f / (float)(1 << R);
-    const uint32_t bmask = (1u << B) - 1u, rmask = (1u << R) - 1u;
-    // lane owns head dims d_e = lane + 32 e (scale group e)
-    int kw[4], kbit[4], krw[4], krbit[4];
-    float qv[GQP][4];
+  float an[GQP][4], ad_own = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; e++) {
-      key_pos(lane + 32 * e, B, kw[e], kbit[e]);
-      key_pos(lane + 32 * e, R, krw[e], krbit[e]);
+  for (int h = 0; h < GQP; h++)
 #pragma unroll
-      for (int h = 0; h < GQP; h++) qv[h][e] = h < gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
+    for (int e = 0; e < 4; e++) an[h][e] = 0.f;
+  const int32_t* selg = a.sel + head * a.k_tok;
+  // lane L ends the transposed reduction holding slot u = L % (TPW GQP):
+  // token m_own = u / GQP of the warp's batch, head h_own = u % GQP
+  const int u_own = lane % (kRefTPW * GQP), m_own = u_own / GQP, h_own = u_own % GQP;
+  for (int j0 = ja + warp * kRefTPW; j0 < jb; j0 += kRefWarps * kRefTPW) {
+    int tok[kRefTPW];
+#pragma unroll
+    for (int m = 0; m < kRefTPW; m++) {
+      const int j = j0 + m;
+      int t = j < jb ? selg[j] : -1;
+      tok[m] = (t >= 0 && t < a.T) ? t : -1;  // a foreign index is skipped, never dereferenced
     }
-    constexpr int TPW = kPostStage / NW;  // tokens of a staging batch per warp
-    float an[GQP][4], ad_own = 0.f;
+    // every load of the warp's tokens first
+    uint32_t wk[kRefTPW][4], wkr[kRefTPW][4], wv[kRefTPW][4], wvr[kRefTPW][4], zk[kRefTPW][4], zv[kRefTPW][4];
 #pragma unroll
-    for (int h = 0; h < GQP; h++)
+    for (int m = 0; m < kRefTPW; m++) {
+      const int t = tok[m] < 0 ? 0 : tok[m];
+      const long slot = slot0 + t, tile = slot / 16;
+      const uint32_t* kp = reinterpret_cast<const uint32_t*>(a.kb + slot * 16 * B);
+      const uint32_t* krp = reinterpret_cast<const uint32_t*>(a.kr + slot * 16 * R);
+      const uint32_t* vp = reinterpret_cast<const uint32_t*>(a.vb + tile * 256 * B);
+      const uint32_t* vrp = reinterpret_cast<const uint32_t*>(a.vr + tile * 256 * R);
+      const uint32_t* zkp = reinterpret_cast<const uint32_t*>(a.ksz) + slot * 4;
+      const uint32_t* zvp = reinterpret_cast<const uint32_t*>(a.vsz) + slot * 4;
 #pragma unroll
-      for (int e = 0; e < 4; e++) an[h][e] = 0.f;
-    // pieces of one staged token: 16-byte copies (8-byte for 1-bit value refinement chunks)
-    const int pk = B, pkr = R, pv = 8 * (B >= 2 ? B / 2 : 1), pvr = 8 * (R >= 2 ? R / 2 : 1);
-    const int npiece = pk + pkr + 2 + pv + pvr;
-    for (int j0 = ja; j0 < jb; j0 += kPostStage) {
-      const int nt = min(kPostStage, jb - j0);
-      __syncthreads();  // the previous batch is consumed
-      for (int it = tid; it < nt * npiece; it += kPostThreads) {
-        const int i = it / npiece, pc = it % npiece;
-        int t = mail.tok[j0 - ja + i];
-        if (t < 0 || t >= a.T) t = 0;  // out-of-range indices are never produced by the selection
-        const long slot = slot0 + t, tile = slot / 16;
-        const int c = (t & 7) >> 1;  // the token's value chunk column
-        uint32_t* dst = stage + i * W;
-        if (pc < pk) {
-          cp_async16(dst + oK + 4 * pc, a.kb + slot * 16 * B + 16 * pc);
-        } else if (pc < pk + pkr) {
-          const int q4 = pc - pk;
-          cp_async16(dst + oKr + 4 * q4, a.kr + slot * 16 * R + 16 * q4);
-        } else if (pc == pk + pkr) {
-          cp_async16(dst + oZk, reinterpret_cast<const uint8_t*>(a.ksz) + slot * 16);
-        } else if (pc == pk + pkr + 1) {
-          cp_async16(dst + oZv, reinterpret_cast<const uint8_t*>(a.vsz) + slot * 16);
-        } else if (pc < pk + pkr + 2 + pv) {
-          // value codes: chunk l = 4 gg + c holds 2b words; b = 4 takes two 16-byte copies
-          const int q4 = pc - (pk + pkr + 2), gg = B >= 2 ? q4 / (B / 2) : q4, part = B >= 2 ? q4 % (B / 2) : 0;
-          cp_async16(dst + oV + gg * 2 * B + 4 * part,
-                     a.vb + tile * 256 * B + (size_t)(4 * gg + c) * 8 * B + 16 * part);
-        } else {
-          const int q4 = pc - (pk + pkr + 2 + pv);
-          if constexpr (R >= 2) {
-            const int gg = q4 / (R / 2), part = q4 % (R / 2);
-            cp_async16(dst + oVr + gg * 2 * R + 4 * part,
-                       a.vr + tile * 256 * R + (size_t)(4 * gg + c) * 8 * R + 16 * part);
-          } else {
-            cp_async8(dst + oVr + q4 * 2, a.vr + tile * 256 * R + (size_t)(4 * q4 + c) * 8 * R);
-          }
-        }
+      for (int e = 0; e < 4; e++) {
+        const int d = lane + 32 * e;
+        int vw, vbit, vrw, vrbit;
+        value_pos(t & 15, d, B, vw, vbit);
+        value_pos(t & 15, d, R, vrw, vrbit);
+        wk[m][e] = (kp[kw[e]] >> kbit[e]) & bmask;
+        wkr[m][e] = (krp[krw[e]] >> krbit[e]) & rmask;
+        wv[m][e] = (vp[vw] >> vbit) & bmask;
+        wvr[m][e] = (vrp[vrw] >> vrbit) & rmask;
+        zk[m][e] = zkp[e];
+        zv[m][e] = zvp[e];
       }
-      cp_async_commit();
-      // while the copies fly: the base weights exp(l_base - M) of the warp's
-      // tokens; lane L holds slot u = L % (TPW GQP), i.e. token i = warp + NW
-      // (u / GQP), head u % GQP (the slot the transposed reduction below
-      // leaves in lane L)
-      float wbl = 0.f;
-      const int u_own = lane % (TPW * GQP), m_own = u_own / GQP, h_own = u_own % GQP;
-      const bool own_ok = h_own < gq && warp + NW * m_own < nt;
-      if (own_ok)
-        wbl = __expf(a.logits[(hq0 + h_own) * a.T + mail.tok[j0 - ja + warp + NW * m_own]] - sh.M[h_own]);
-      cp_async_wait<0>();
-      __syncthreads();
-      // the warp's TPW tokens together: refined keys, base and refined values
-      float kf[TPW][4], vbs[TPW][4], vfs[TPW][4];
-#pragma unroll
-      for (int m = 0; m < TPW; m++) {
-        const int i = warp + NW * m;
-        const bool ok = i < nt;
-        const uint32_t* st = stage + (ok ? i : 0) * W;
-        const int tt = ok ? (mail.tok[j0 - ja + i] & 15) : 0;
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-          const int d = lane + 32 * e;
-          int vw, vbit, vrw, vrbit;
-          value_pos(tt, d, B, vw, vbit);
-          value_pos(tt, d, R, vrw, vrbit);
-          // staged chunk gg = d & 7 holds words [l 2w, l 2w + 2w) of the tile
-          const int vwl = vw - (4 * (d & 7) + ((tt & 7) >> 1)) * 2 * B + (d & 7) * 2 * B;
-          const int vrwl = vrw - (4 * (d & 7) + ((tt & 7) >> 1)) * 2 * R + (d & 7) * 2 * R;
-          const uint32_t zk = st[oZk + e], zv = st[oZv + e];
-          const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&zk));
-          const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv));
-          const uint32_t qk = (st[oK + kw[e]] >> kbit[e]) & bmask, rk = (st[oKr + krw[e]] >> krbit[e]) & rmask;
-          const uint32_t qq = (st[oV + vwl] >> vbit) & bmask, rv = (st[oVr + vrwl] >> vrbit) & rmask;
-          kf[m][e] = fmaf(k2.x, (float)qk + ((float)rk + 0.5f - half) * inv, k2.y);
-          vbs[m][e] = ok ? fmaf(v2.x, (float)qq, v2.y) : 0.f;
-          vfs[m][e] = ok ? fmaf(v2.x, (float)qq + ((float)rv + 0.5f - half) * inv, v2.y) : 0.f;
-        }
-      }
-      // refined logits of the TPW x GQP (token, head) slots: per-lane partial
-      // dot products, summed over the warp by a transposed butterfly that
-      // leaves slot lane % (TPW GQP) in each lane
-      float lg[TPW * GQP];
-#pragma unroll
-      for (int m = 0; m < TPW; m++)
-#pragma unroll
-        for (int h = 0; h < GQP; h++) {
-          float acc = 0.f;
-#pragma unroll
-          for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[m][e], acc);
-          lg[m * GQP + h] = acc;
-        }
-      const float lg_own = warp_transpose_sum<TPW * GQP>(lg, lane);
-      float wfl = 0.f;
-      if (own_ok) wfl = __expf(lg_own * a.scale - sh.M[h_own]);
-      // every lane needs every slot's (w_refined, w_base): through the warp's table
-      float2* wtab = reinterpret_cast<float2*>(&sh.wtab[warp][0]);
-      if (lane < TPW * GQP) wtab[lane] = make_float2(wfl, wbl);
-      ad_own += wfl - wbl;
-      __syncwarp();
-#pragma unroll
-      for (int m = 0; m < TPW; m++)
-#pragma unroll
-        for (int h = 0; h < GQP; h++) {
-          const float2 w = wtab[m * GQP + h];
-#pragma unroll
-          for (int e = 0; e < 4; e++) an[h][e] = fmaf(w.x, vfs[m][e], fmaf(-w.y, vbs[m][e], an[h][e]));
-        }
-      __syncwarp();
     }
-    // per-warp partial numerators and denominators (the score keys are no
-    // longer needed: their space holds them), summed in the merge below
-    float* wnum = reinterpret_cast<float*>(keys);
+    float wbl = 0.f;
+    const bool own_ok = h_own < gq && tok[m_own] >= 0;
+    if (own_ok) wbl = expf(a.logits[(hq0 + h_own) * a.T + tok[m_own]] - sh.M[h_own]);
+    float kf[kRefTPW][4], vbs[kRefTPW][4], vfs[kRefTPW][4];
 #pragma unroll
-    for (int h = 0; h < GQP; h++)
-      if (h < gq) {
+    for (int m = 0; m < kRefTPW; m++) {
+      const bool ok = tok[m] >= 0;
 #pragma unroll
-        for (int e = 0; e < 4; e++) wnum[(warp * GQP + h) * kD + lane + 32 * e] = an[h][e];
+      for (int e = 0; e < 4; e++) {
+        const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&zk[m][e]));
+        const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv[m][e]));
+        kf[m][e] = fmaf(k2.x, (float)wk[m][e] + ((float)wkr[m][e] + 0.5f - half) * inv, k2.y);
+        vbs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e], v2.y) : 0.f;
+        vfs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e] + ((float)wvr[m][e] + 0.5f - half) * inv, v2.y) : 0.f;
       }
-    // slot u's denominator change sits in lanes u, u + TPW GQP, ...; sum over
-    // the TPW tokens of each head
-    float dsum = lane < TPW * GQP ? ad_own : 0.f;
+    }
+    // refined logits of the TPW x GQP (token, head) slots
+    float lg[kRefTPW * GQP];
 #pragma unroll
-    for (int o = GQP; o < 32; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-    if (lane < gq) sh.wden[warp][lane] = dsum;
+    for (int m = 0; m < kRefTPW; m++)
+#pragma unroll
+      for (int h = 0; h < GQP; h++) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[m][e], acc);
+        lg[m * GQP + h] = acc;
+      }
+    const float lg_own = warp_transpose_sum<kRefTPW * GQP>(lg, lane);
+    float wfl = 0.f;
+    if (own_ok) wfl = expf(lg_own * a.scale - sh.M[h_own]);
+    if (lane < kRefTPW * GQP) sh.wtab[warp][lane] = make_float2(wfl, wbl);
+    ad_own += wfl - wbl;
+    __syncwarp();
+#pragma unroll
+    for (int m = 0; m < kRefTPW; m++)
+#pragma unroll
+      for (int h = 0; h < GQP; h++) {
+        const float2 w = sh.wtab[warp][m * GQP + h];
+#pragma unroll
+        for (int e = 0; e < 4; e++) an[h][e] = fmaf(w.x, vfs[m][e], fmaf(-w.y, vbs[m][e], an[h][e]));
+      }
+    __syncwarp();
   }
+#pragma unroll
+  for (int h = 0; h < GQP; h++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) sh.num[warp][h][lane + 32 * e] = an[h][e];
+  // slot u's denominator change sits in lanes u, u + TPW GQP, ...: sum each head's
+  float dsum = lane < kRefTPW * GQP ? ad_own : 0.f;
+#pragma unroll
+  for (int o = GQP; o < 32; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  if (lane < GQP) sh.den[warp][lane] = dsum;
   __syncthreads();
-  // this CTA's share of the base records: records s = cr, cr + CL, ... (loads batched)
-  for (int e = tid; e < gq * kD; e += kPostThreads) {
-    const int hh = e / kD, d = e % kD;
-    const float* pr = a.part + (hq0 + hh) * a.nrec * a.rec;
-    float num = 0.f;  // the correction: every warp's partial
-    for (int w = 0; w < NW; w++) num += reinterpret_cast<const float*>(keys)[(w * GQP + hh) * kD + d];
-    constexpr int PER = 8;
-    for (int s0 = cr; s0 < a.nrec; s0 += CL * PER) {
+
+  // ---- this CTA's share of the base records (s = part, part + parts, ...), rescaled to M
+  float* rp = a.rpart + (head * a.parts + part) * gq * (kD + 1);
+  for (int e = tid; e < gq * kD; e += kRefThreads) {
+    const int h = e / kD, d = e % kD;
+    const float* pr = a.part + (hq0 + h) * a.nrec * kRec;
+    float num = 0.f;
+    for (int w = 0; w < kRefWarps; w++) num += sh.num[w][h][d];
+    constexpr int PER = 4;
+    for (int s0 = part; s0 < a.nrec; s0 += a.parts * PER) {
       float mv[PER], av[PER];
 #pragma unroll
       for (int k = 0; k < PER; k++) {
-        const int s = s0 + CL * k;
-        mv[k] = s < a.nrec ? pr[(long)s * a.rec + kD] : -INFINITY;
-        av[k] = s < a.nrec ? pr[(long)s * a.rec + d] : 0.f;
+        const int s = s0 + a.parts * k;
+        mv[k] = s < a.nrec ? pr[(long)s * kRec + kD] : -INFINITY;
+        av[k] = s < a.nrec ? pr[(long)s * kRec + d] : 0.f;
       }
 #pragma unroll
       for (int k = 0; k < PER; k++)
-        if (mv[k] > -INFINITY) num = fmaf(__expf(mv[k] - sh.M[hh]), av[k], num);
+        if (mv[k] > -INFINITY) num = fmaf(expf(mv[k] - sh.M[h]), av[k], num);
     }
-    cluster.map_shared_rank(&mail.num[cr][0], hh)[d] = num;  // to the CTA that merges head hh
+    rp[h * (kD + 1) + d] = num;
   }
   if (tid < gq) {
     float den = 0.f;
-    for (int w = 0; w < NW; w++) den += sh.wden[w][tid];
-    cluster.map_shared_rank(&mail.den[cr], tid)[0] = den;
+    for (int w = 0; w < kRefWarps; w++) den += sh.den[w][tid];
+    rp[tid * (kD + 1) + kD] = den;
   }
-  cluster.sync();  // every partial numerator is in its head's mailbox
-  if (cr < gq) {
-    for (int d = tid; d < kD; d += kPostThreads) {
-      float num = 0.f, den = sh.Z[cr];
-      for (int rk = 0; rk < CL; rk++) num += mail.num[rk][d], den += mail.den[rk];
-      const float o = num / den;
-      if (a.out) a.out[(hq0 + cr) * kD + d] = o;
-      if (a.out16) a.out16[(hq0 + cr) * kD + d] = __half_as_ushort(__float2half_rn(o));
+  __threadfence();  // this CTA's partial before its count
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(a.ctl + head * kCtl + kBins1 + 1, 1) == a.parts - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();  // every other CTA's partial is visible
+  const float* rh = a.rpart + head * a.parts * gq * (kD + 1);
+  for (int e = tid; e < gq * kD; e += kRefThreads) {
+    const int h = e / kD, d = e % kD;
+    float num = 0.f, den = sh.Z[h];
+    for (int p = 0; p < a.parts; p++) {
+      num += __ldcg(rh + (p * gq + h) * (kD + 1) + d);
+      den += __ldcg(rh + (p * gq + h) * (kD + 1) + kD);
     }
+    const float o = num / den;
+    if (a.out) a.out[(hq0 + h) * kD + d] = o;
+    if (a.out16) a.out16[(hq0 + h) * kD + d] = __half_as_ushort(__float2half_rn(o));
   }
 }
+
 
 // ---------------------------------------------------------------------------
 // host side
 
 struct Plan {
   int nsplit, span, nrec;  // base pass (warp splits; one record per CTA of kWarps splits)
-  int cl, chunk;           // cluster size and tokens per CTA after the base pass
-  size_t off_logits, off_part, total;
+  int Tp, sel_blocks, parts;
+  size_t off_logits, off_part, off_scores, off_ctl, off_rpart, total;
 };
 
-Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, bool with_pv,
-               bool select, int n_splits) {
-  (void)k_tok, (void)select;
+// The workspace: [logits] [records] [scores, Tp-pitched] [control words] [refinement partials].
+Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, bool with_pv, bool select,
+               bool refine, int n_splits) {
   Plan P;
   const int sms = num_sms();
   const int heads = kv->batch * kv->h_kv;
@@ -1013,8 +1046,10 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   P.span = ((t + ns - 1) / ns + 15) / 16 * 16;
   P.nsplit = (t + P.span - 1) / P.span;
   P.nrec = (P.nsplit + kWarps - 1) / kWarps;
-  P.cl = kPostCl;
-  P.chunk = (t + P.cl - 1) / P.cl;
+  P.Tp = (t + 31) / 32 * 32;
+  P.sel_blocks = (t + kSelTok - 1) / kSelTok;
+  P.parts = std::max(1, std::min(kRefPartsMax, (k_tok + kRefWarps * kRefTPW - 1) / (kRefWarps * kRefTPW)));
+  const int gq = h_q / kv->h_kv;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -1024,18 +1059,11 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   const int rec = with_pv ? kRec : 2;
   P.off_logits = need_logits ? take((size_t)kv->batch * h_q * t * 4) : 0;
   P.off_part = take((size_t)kv->batch * h_q * P.nrec * rec * 4);
+  P.off_scores = select ? take((size_t)heads * P.Tp * 4) : 0;
+  P.off_ctl = take((size_t)heads * kCtl * 4);
+  P.off_rpart = refine ? take((size_t)heads * P.parts * gq * (kD + 1) * 4) : 0;
   P.total = off;
   return P;
-}
-
-// k_tok of every entry point: at most t, at most kMaxKTok (each of the kPostCl
-// CTAs of a head's cluster holds up to kPostMaxSel of the selected tokens), and
-// at least 1 unless a base-only call (allow_zero) is meant.
-sf_status check_ktok(int k_tok, int t, bool allow_zero) {
-  SF_REQUIRE(k_tok >= (allow_zero ? 0 : 1) && k_tok <= t, "k_tok=%d outside [%d, t=%d]", k_tok,
-             allow_zero ? 0 : 1, t);
-  SF_UNSUPPORTED(k_tok <= kMaxKTok, "k_tok=%d above %d", k_tok, kMaxKTok);
-  return SF_OK;
 }
 
 sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
@@ -1044,7 +1072,16 @@ sf_status check_q(const sf_kv* kv, int t, const uint16_t* q, int h_q) {
   SF_UNSUPPORTED(h_q > 0 && h_q % kv->h_kv == 0 && h_q / kv->h_kv <= 8,
                  "h_q=%d must be a multiple of h_kv=%d with at most 8 query heads per KV head", h_q,
                  kv->h_kv);
-  SF_UNSUPPORTED(t <= kPostCl * kPostMaxTok, "t=%d above %d", t, kPostCl * kPostMaxTok);
+  SF_UNSUPPORTED(t <= kMaxT, "t=%d above %d", t, kMaxT);
+  return SF_OK;
+}
+
+// k_tok of every entry point: at most t and kMaxKTok, at least 1 unless a
+// base-only call (allow_zero) is meant.
+sf_status check_ktok(int k_tok, int t, bool allow_zero) {
+  SF_REQUIRE(k_tok >= (allow_zero ? 0 : 1) && k_tok <= t, "k_tok=%d outside [%d, t=%d]", k_tok,
+             allow_zero ? 0 : 1, t);
+  SF_UNSUPPORTED(k_tok <= kMaxKTok, "k_tok=%d above %d", k_tok, kMaxKTok);
   return SF_OK;
 }
 
@@ -1053,17 +1090,7 @@ sf_status launch_base_t(const BaseArgs& a, int batch, cudaStream_t s) {
   const size_t smem = kWarps * WarpSmem<B, PV>::bytes;
   auto kern = kv_base_kernel<GQP, B, PV>;
   SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch);
-  cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;  // launch overlaps the previous kernel's tail
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  SF_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
+  SF_CUDA(launch_pdl(kern, dim3((a.nsplit + kWarps - 1) / kWarps, a.h_kv, batch), dim3(kWarps * 32), smem, s, a));
   return SF_OK;
 }
 
@@ -1077,61 +1104,57 @@ sf_status launch_base(const sf_kv* kv, const BaseArgs& a, bool pv, cudaStream_t 
   return pv ? launch_base_t<8, 4, true>(a, kv->batch, s) : launch_base_t<8, 4, false>(a, kv->batch, s);
 }
 
-BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* logits, float* part,
+BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* logits, float* part, int* ctl,
                    const Plan& P) {
   BaseArgs a;
   a.kb = (const uint8_t*)kv->kb, a.vb = (const uint8_t*)kv->vb;
   a.ksz = kv->ksz, a.vsz = kv->vsz;
   a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.T = t;
   a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
-  a.logits = logits, a.part = part;
+  a.logits = logits, a.part = part, a.ctl = ctl;
   a.span = P.span, a.nsplit = P.nsplit, a.nrec = P.nrec;
   a.scale = 1.0f / sqrtf((float)kD);
   return a;
 }
 
-// The cluster kernel after the base pass (launched with programmatic
-// serialization: its CTAs start while the base pass drains).
-sf_status launch_post(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
-                      const float* logits, const float* part, int rec, int32_t* sel, int select,
-                      float* scores, float* out, cudaStream_t s, uint16_t* out16 = nullptr) {
-  PostArgs a;
+// Scoring and selection after the base pass (programmatic serialization: its
+// CTAs start while the base pass drains).
+sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& P, const float* logits,
+                        const float* part, int rec, float* scores_ws, float* scores_out, int* ctl, int32_t* sel,
+                        cudaStream_t s) {
+  SelArgs a;
+  a.logits = logits, a.part = part, a.nrec = P.nrec, a.rec = rec;
+  a.h_kv = kv->h_kv, a.h_q = h_q, a.gq = h_q / kv->h_kv, a.T = t, a.Tp = P.Tp, a.k_tok = k_tok;
+  a.nblk = P.sel_blocks;
+  a.scores = scores_ws, a.scores_out = scores_out, a.ctl = ctl, a.sel = sel;
+  void (*kern)(SelArgs) = a.gq <= 4 ? kv_select_kernel<4> : kv_select_kernel<8>;
+  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDyn));
+  SF_CUDA(launch_pdl(kern, dim3(P.sel_blocks, kv->h_kv, kv->batch), dim3(kSelThreads), kSelDyn, s, a));
+  return SF_OK;
+}
+
+// Refinement of the selected tokens and the merge (programmatic serialization).
+sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
+                        const float* logits, const float* part, const int32_t* sel, int* ctl, float* rpart,
+                        float* out, uint16_t* out16, cudaStream_t s) {
+  RefArgs a;
   a.kb = (const uint8_t*)kv->kb, a.kr = (const uint8_t*)kv->kr;
   a.vb = (const uint8_t*)kv->vb, a.vr = (const uint8_t*)kv->vr;
   a.ksz = kv->ksz, a.vsz = kv->vsz;
-  a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.b = kv->b, a.r = kv->r, a.T = t;
+  a.h_kv = kv->h_kv, a.t_max = kv->t_max, a.T = t;
   a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
-  a.logits = logits, a.part = part, a.nrec = P.nrec, a.rec = rec;
-  a.k_tok = k_tok, a.sel = sel, a.select = select, a.scores = scores, a.out = out, a.out16 = out16;
-  a.chunk = P.chunk;
+  a.logits = logits, a.part = part, a.nrec = P.nrec;
+  a.k_tok = k_tok, a.parts = P.parts, a.sel = sel, a.ctl = ctl, a.rpart = rpart;
+  a.out = out, a.out16 = out16;
   a.scale = 1.0f / sqrtf((float)kD);
-  // the score keys' space, which later holds the per-warp partial numerators
-  // of the refined attention [warps][GQP][kD]
-  const size_t gqp = a.gq <= 4 ? 4 : 8;
-  const size_t key_words = (out || out16) ? std::max((size_t)P.chunk, (size_t)(kPostThreads / 32) * gqp * kD) : (size_t)P.chunk;
-  const size_t smem = sizeof(PostMail) + ((size_t)kPostStage * tok_words(kv->b, kv->r) + key_words) * 4;
-  void (*kern)(PostArgs);
+  void (*kern)(RefArgs);
   if (a.gq <= 4)
-    kern = kv->b == 2 ? (kv->r == 2 ? kv_post_kernel<4, 2, 2> : kv_post_kernel<4, 2, 1>)
-                      : (kv->r == 2 ? kv_post_kernel<4, 4, 2> : kv_post_kernel<4, 4, 1>);
+    kern = kv->b == 2 ? (kv->r == 2 ? kv_refine_kernel<4, 2, 2> : kv_refine_kernel<4, 2, 1>)
+                      : (kv->r == 2 ? kv_refine_kernel<4, 4, 2> : kv_refine_kernel<4, 4, 1>);
   else
-    kern = kv->b == 2 ? (kv->r == 2 ? kv_post_kernel<8, 2, 2> : kv_post_kernel<8, 2, 1>)
-                      : (kv->r == 2 ? kv_post_kernel<8, 4, 2> : kv_post_kernel<8, 4, 1>);
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)(sizeof(PostMail) + ((size_t)kPostStage * tok_words(4, 2) + kPostMaxTok) * 4)));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P.cl, kv->h_kv, kv->batch);
-  cfg.blockDim = dim3(kPostThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = P.cl, attr[0].val.clusterDim.y = 1, attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  SF_CUDA(cudaLaunchKernelEx(&cfg, kern, a));
+    kern = kv->b == 2 ? (kv->r == 2 ? kv_refine_kernel<8, 2, 2> : kv_refine_kernel<8, 2, 1>)
+                      : (kv->r == 2 ? kv_refine_kernel<8, 4, 2> : kv_refine_kernel<8, 4, 1>);
+  SF_CUDA(launch_pdl(kern, dim3(P.parts, kv->h_kv, kv->batch), dim3(kRefThreads), 0, s, a));
   return SF_OK;
 }
 
@@ -1152,7 +1175,7 @@ using namespace sf;
 extern "C" size_t sf_kv_score_select_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                                      int logits_given) {
   if (!kv || t <= 0 || h_q <= 0 || k_tok <= 0) return 0;
-  return make_plan(kv, t, h_q, k_tok, !logits_given, false, true, 0).total;
+  return make_plan(kv, t, h_q, k_tok, !logits_given, false, true, false, 0).total;
 }
 
 extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q,
@@ -1167,23 +1190,24 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(sel && aligned16(sel), "sel must be a non-null 16-byte aligned device pointer");
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE(!scores || aligned16(scores), "scores must be 16-byte aligned");
-  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, false, true, 0);
+  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, false, true, false, 0);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   float* lg = logits ? logits : (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
+  int* ctl = (int*)(w + P.off_ctl);
   cudaStream_t s = as_stream(stream);
-  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, false, s);
   if (st != SF_OK) return st;
-  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, 2, sel, 1, scores, nullptr, s);
+  return launch_select(kv, t, h_q, k_tok, P, lg, part, 2, (float*)(w + P.off_scores), scores, ctl, sel, s);
 }
 
 extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
                                              int n_splits) {
   if (!kv || t <= 0 || h_q <= 0) return 0;
-  return make_plan(kv, t, h_q, k_tok, true, true, false, n_splits).total;
+  return make_plan(kv, t, h_q, k_tok, true, true, false, true, n_splits).total;
 }
 
 extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* q, int h_q,
@@ -1198,24 +1222,24 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   SF_REQUIRE(k_tok == 0 || (sel && aligned16(sel)), "sel must be non-null and 16-byte aligned");
   SF_REQUIRE(n_splits >= 0, "n_splits=%d < 0", n_splits);
   SF_REQUIRE(out && aligned16(out), "out must be a non-null 16-byte aligned device pointer");
-  Plan P = make_plan(kv, t, h_q, k_tok, true, true, false, n_splits);
+  Plan P = make_plan(kv, t, h_q, k_tok, true, true, false, true, n_splits);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   cudaStream_t s = as_stream(stream);
   float* lg = (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
-  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
+  int* ctl = (int*)(w + P.off_ctl);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, const_cast<int32_t*>(sel), 0, nullptr,
-                     out, s);
+  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, nullptr, s);
 }
 
 extern "C" size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q,
                                                          int k_tok, int logits_given) {
   if (!kv || t <= 0 || h_q <= 0 || k_tok <= 0) return 0;
-  return make_plan(kv, t, h_q, k_tok, !logits_given, true, true, 0).total;
+  return make_plan(kv, t, h_q, k_tok, !logits_given, true, true, true, 0).total;
 }
 
 namespace sf {
@@ -1235,16 +1259,19 @@ sf_status attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q, i
   SF_REQUIRE(!logits || aligned16(logits), "logits must be 16-byte aligned");
   SF_REQUIRE((out || out16) && (!out || aligned16(out)) && (!out16 || aligned16(out16)),
              "out must be a non-null 16-byte aligned device pointer");
-  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0);
+  Plan P = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, true, 0);
   st = check_ws(ws, ws_bytes, P.total);
   if (st != SF_OK) return st;
   char* w = (char*)ws;
   float* lg = logits ? logits : (float*)(w + P.off_logits);
   float* part = (float*)(w + P.off_part);
-  BaseArgs a = base_args(kv, t, q, h_q, lg, part, P);
+  int* ctl = (int*)(w + P.off_ctl);
+  BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  return launch_post(kv, t, q, h_q, k_tok, P, lg, part, kRec, sel, 1, nullptr, out, s, out16);
+  st = launch_select(kv, t, h_q, k_tok, P, lg, part, kRec, (float*)(w + P.off_scores), nullptr, ctl, sel, s);
+  if (st != SF_OK) return st;
+  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, out16, s);
 }
 
 }  // namespace
@@ -1323,7 +1350,7 @@ extern "C" sf_status sf_kv_attend_selective_static(const sf_kv* kv, int t, const
   if (st != SF_OK) return st;
   st = check_ktok(k_tok, t, false);
   if (st != SF_OK) return st;
-  const size_t need = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, 0).total;
+  const size_t need = make_plan(kv, t, h_q, k_tok, logits == nullptr, true, true, true, 0).total;
   if (need > kStaticWsBytes) {
     set_error("workspace of %zu bytes needed (batch=%d, h_q=%d, t=%d, k_tok=%d, logits %s) is above "
               "the static scratch of %zu bytes; use sf_kv_attend_selective with a caller workspace",

@@ -56,6 +56,10 @@ class DecoderConfig:
     lead: int = 1
     lag: int = 1
     host_refine: bool = True  # refinement rows in pinned host memory, staged per layer
+    # refinement rows kept on the device across steps, per (layer, projection,
+    # batch row): capacity = cache_rows x the projection's selected channels (0: no cache)
+    cache_rows: float = 0.0
+    skip_missing: bool = False  # with the cache: a missing row leaves its channel at base precision this step
     eps: float = 1e-5
     theta: float = 500000.0
 
@@ -110,6 +114,11 @@ class Decoder:
                               for _ in range(2)] for n in PROJ}
         else:
             self.slots = None
+        # with the row cache: the selection each GEMV uses (channels whose rows
+        # did not arrive are marked -1 - c), per projection and slot
+        self.use_cache = bool(cfg.kch and cfg.host_refine and cfg.cache_rows > 0)
+        self.sel_eff = ({n: [i32(B, self.n_sel[n]) for _ in range(2)] for n in PROJ} if self.use_cache else None)
+        self.caches = []  # per layer: name -> (ctypes array of B sf_row_cache, tensors kept alive)
         # the GEMV's workspace (its size query returns 0 today; sized for the widest input)
         kmax = max(kk for _, _, kk in cfg.shapes())
         wq = abi.sf_wq(128, kmax, cfg.w_bits, cfg.w_refine, cfg.group, None, None, None)
@@ -122,11 +131,18 @@ class Decoder:
         self.stage_stream = {"qkv": self.side, "gate_up": self.side, "o": self.side2, "down": self.side2}
         self.ev_sel = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
         self.ev_stage = {n: [torch.cuda.Event() for _ in range(2)] for n in PROJ}
+        for evs in (self.ev_sel, self.ev_stage):  # create the events now: the library records them by handle
+            for pair in evs.values():
+                for ev in pair:
+                    ev.record(torch.cuda.current_stream(dev))
         # fetch lag: layer l's o correction, written by its projection and added
         # by the next layer's residual add
         self.delta = f32(B, cfg.hidden)
         self.lm_head = None
         self.ws = None
+        # when a list: every selection a projection or the attention uses is
+        # copied into it (on the step's stream), for checks against the oracle
+        self.trace = None
 
     # ---- model state -----------------------------------------------------
 
@@ -146,12 +162,47 @@ class Decoder:
                 qw.refine = None
                 qw.desc.refine = None
             L[n] = qw
+        if self.use_cache:
+            self.caches.append({n: self._make_caches(n) for n in PROJ})
         kv = KVCache(self.B, cfg.h_kv, self.t_max, cfg.kv_bits, cfg.kv_refine, cfg.d, device=self.dev)
         kv.pack_tokens(k_cache.contiguous(), v_cache.contiguous(), 0)
         L["kv"] = kv
         self.layers.append(L)
         self.host_rows.append(host)
         torch.cuda.synchronize(self.dev)
+
+    def _make_caches(self, name):
+        """One empty row cache per batch row for one projection of one layer."""
+        n_ch = self.shp[name][1]
+        cap = max(self.n_sel[name], int(round(self.cfg.cache_rows * self.n_sel[name])))
+        i32 = lambda n: torch.empty(n, dtype=torch.int32, device=self.dev)
+        arr = (abi.sf_row_cache * self.B)()
+        keep = []
+        for b in range(self.B):
+            t = dict(slot_of=i32(n_ch), channel_of=i32(cap), stamp=i32(cap), state=i32(4),
+                     work=i32(self.n_sel[name]),
+                     rows=torch.empty(cap * self.row_bytes[name], dtype=torch.uint8, device=self.dev))
+            keep.append(t)
+            arr[b] = abi.sf_row_cache(cap, n_ch, self.row_bytes[name], t["slot_of"].data_ptr(),
+                                      t["channel_of"].data_ptr(), t["stamp"].data_ptr(), t["state"].data_ptr(),
+                                      t["work"].data_ptr(), self.n_sel[name], t["rows"].data_ptr())
+            check(abi.sf_row_cache_reset(ctypes.byref(arr[b]), _s(torch.cuda.current_stream(self.dev))),
+                  "sf_row_cache_reset")
+        return arr, keep
+
+    def cache_stats(self):
+        """{projection: (hits, misses)} summed over the layers' and batch rows'
+        row caches since they were made (empty without caches)."""
+        out = {}
+        for L in self.caches:
+            for name, (arr, keep) in L.items():
+                h, m = out.get(name, (0, 0))
+                for t in keep:
+                    st = t["state"].cpu()
+                    h += int(st[2]) & 0xFFFFFFFF
+                    m += int(st[3]) & 0xFFFFFFFF
+                out[name] = (h, m)
+        return out
 
     def set_lm_head(self, lm_fp16: torch.Tensor):
         self.lm_head = lm_fp16.contiguous()
@@ -166,13 +217,25 @@ class Decoder:
         check(abi.sf_select_channels(_p(x), self.B, self.shp[name][1], cfg.chunk, cfg.kch,
                                      _p(self.sel[name][slot]), _s(stream)), "sf_select_channels")
 
-    def _stage(self, layer, name, slot):
+    def _stage(self, layer, name, slot, done):
         """Copy layer `layer`'s rows of the selection in `slot` into staging
-        slot `slot` on the projection's staging stream (after the selection)."""
+        slot `slot` on the projection's staging stream (after the selection);
+        `done` is recorded once the projection may use them."""
+        side = self.stage_stream[name]
+        if self.use_cache:
+            arr, _ = self.caches[layer][name]
+            check(abi.sf_stage_refinements_cached(_p(self.host_rows[layer][name]), self.row_bytes[name],
+                                                  self.shp[name][1], _p(self.sel[name][slot]), self.n_sel[name],
+                                                  self.B, arr, int(self.cfg.skip_missing), _p(self.slots[name][slot]),
+                                                  _p(self.sel_eff[name][slot]), _s(side),
+                                                  ctypes.c_void_p(done.cuda_event)),
+                  "sf_stage_refinements_cached")
+            return
         check(abi.sf_stage_refinements(_p(self.host_rows[layer][name]), self.row_bytes[name],
                                        self.shp[name][1], _p(self.sel[name][slot]), self.B * self.n_sel[name],
-                                       _p(self.slots[name][slot]), None, _s(self.stage_stream[name]), None),
+                                       _p(self.slots[name][slot]), None, _s(side), None),
               "sf_stage_refinements")
+        done.record(side)
 
     def _side_select_stage(self, layer, name, x, slot, main):
         """Selection from x and the row transfer, both on the projection's
@@ -183,8 +246,9 @@ class Decoder:
         side.wait_event(ev)
         self._select(name, x, slot, side)
         if self.slots is not None:
-            self._stage(layer, name, slot)
-        self.ev_stage[name][slot].record(side)
+            self._stage(layer, name, slot, self.ev_stage[name][slot])
+        else:
+            self.ev_stage[name][slot].record(side)
 
     def _ready(self, name, slot, main):
         """Wait (on the main stream) for the selection and rows in `slot`."""
@@ -201,13 +265,16 @@ class Decoder:
                                       _p(y), _p(self.gemv_ws), self.gemv_ws.numel(), _s(main)), "sf_gemv_refined")
             return
         rows = self._ready(name, slot, main)
+        sel = self.sel_eff[name][slot] if self.use_cache else self.sel[name][slot]
+        if self.trace is not None:
+            self.trace.append((("w", layer, name), sel.clone()))
         if y_corr is not None:
             check(abi.sf_gemv_refined_split(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
-                                            _p(self.sel[name][slot]), _p(rows), _p(y), _p(y_corr), _s(main)),
+                                            _p(sel), _p(rows), _p(y), _p(y_corr), _s(main)),
                   "sf_gemv_refined_split")
             return
         check(abi.sf_gemv_refined(ctypes.byref(qw.desc), _p(x), self.B, cfg.chunk, cfg.kch,
-                                  _p(self.sel[name][slot]), None, _p(rows), _p(y), _p(self.gemv_ws),
+                                  _p(sel), None, _p(rows), _p(y), _p(self.gemv_ws),
                                   self.gemv_ws.numel(), _s(main)),
               "sf_gemv_refined")
 
@@ -257,6 +324,8 @@ class Decoder:
             check(abi.sf_kv_attend_selective_f16(ctypes.byref(kv.desc), T + 1, _p(self.q), cfg.h_q, cfg.k_tok,
                                                  _p(self.tok_sel), None, _p(x_o), _p(self.ws), self.ws.numel(),
                                                  _s(main)), "sf_kv_attend_selective_f16")
+            if self.trace is not None:
+                self.trace.append((("tok", l), self.tok_sel.clone()))
             self._prepare(l, "o", x_o, main)
             self._lead(l, "o", x_o, main)
             self._proj(l, "o", x_o, self.o_out, slot, main, y_corr=self.delta if lagging else None)

@@ -169,3 +169,21 @@ def torch_normal(shape, std: float, seed: int, device="cuda", dtype=None):
     t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
     t.mul_(std)
     return t if dtype is None else t.to(dtype)
+
+
+def decoder_hidden_pool(seed: int, n: int, batch: int = 1, hidden: int = HIDDEN, outlier_frac: float = 0.01,
+                        outlier_scale: float = 20.0, device="cuda"):
+    """n decode-step inputs fp16 [n][batch][hidden], one per step of a
+    multi-step run: N(0, 1) per channel, with the same round(outlier_frac *
+    hidden) channels scaled by outlier_scale in every input (outlier channels
+    that persist from token to token, as the activation recipe's 1 % outliers
+    but fixed), drawn on the device with torch's seeded Philox generator."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    h = torch.randn((n, batch, hidden), generator=g, device=device, dtype=torch.float32)
+    gc = torch.Generator(device="cpu").manual_seed(seed)
+    ch = torch.randperm(hidden, generator=gc)[: int(round(outlier_frac * hidden))].to(device)
+    h[:, :, ch] *= outlier_scale
+    return h.to(torch.float16)

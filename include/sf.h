@@ -147,7 +147,10 @@ SF_API sf_status sf_select_channels(const uint16_t* x, int batch, int k, int chu
  *   kch = 0: base only (sel_in, sel_out, refine_rows ignored).
  *   sel_in (nullable): a selection made earlier ([batch][k/chunk][kch],
  *     ascending per chunk), e.g. from the previous layer's activation (fetch
- *     lead).  NULL: the call selects from x itself and writes sel_out.
+ *     lead).  NULL: the call selects from x itself and writes sel_out.  A
+ *     negative entry -1 - c names channel c as selected but not refined in
+ *     this call (its refinement did not arrive: base precision, no correction;
+ *     see sf_stage_refinements_cached).
  *   sel_out (nullable when sel_in is given): receives the selection used.
  *   refine_rows (nullable): staged refinement rows [batch][k/chunk*kch][n*r/8];
  *     row j of batch row b holds the refinement of channel sel[b][j]
@@ -185,6 +188,16 @@ SF_API sf_status sf_gemv_correction(const sf_wq* w, const uint16_t* x, int batch
 SF_API sf_status sf_gemv_refined_split(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
                                 const int32_t* sel_in, const void* refine_rows, float* y_base,
                                 float* y_corr, sf_stream_t stream);
+
+/* Number of bounded device-side waits that ran out on the current device
+ * (*count), optionally reset to 0 (reset != 0).  The refined GEMV waits on
+ * shared-memory barriers for its bulk copies; each such wait gives up after one
+ * second, counts itself here and lets the kernel finish without its result
+ * (the output is then undefined), so a fault in the memory system shows up as
+ * a count, not as a hung GPU.  A nonzero count makes this call return
+ * SF_ERR_TIMEOUT.  The call synchronises with the device (it reads the counter
+ * with cudaMemcpyFromSymbol). */
+SF_API sf_status sf_device_wait_timeouts(unsigned int* count, int reset);
 
 /* ======================================================================== */
 /* KV cache                                                                  */
@@ -246,10 +259,10 @@ SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* 
  *   q [batch][h_q][d] fp16;  sel [batch][h_kv][k_tok] int32.
  *   logits (nullable): receives the base logits [batch][h_q][t] fp32.
  *   scores (nullable): receives score [batch][h_kv][t] fp32.
- *   1 <= t <= min(t_max, 133120), 1 <= k_tok <= min(t, 4096),
+ *   1 <= t <= min(t_max, 262144), 1 <= k_tok <= min(t, 4096),
  *   h_q % h_kv == 0, h_q / h_kv <= 8 (SF_ERR_UNSUPPORTED above the caps: the
- *   per-head selection keeps every token's score, and the selected tokens, in
- *   the shared memory of one 8-CTA cluster). */
+ *   CTA that finishes a head's selection keeps a bitmap of the head's tokens
+ *   in shared memory). */
 SF_API sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok,
                              int32_t* sel, float* logits, float* scores, void* ws,
                              size_t ws_bytes, sf_stream_t stream);
@@ -347,6 +360,61 @@ SF_API sf_status sf_stage_refinements(const void* host_rows, size_t row_bytes, i
 SF_API sf_status sf_stage_refinements_host(const void* host_rows, size_t row_bytes, int n_rows,
                                            const int32_t* sel_host, int n_sel, void* dst,
                                            sf_stream_t stream, sf_event_t done);
+
+/* A device-resident cache of refinement rows, reused across decode steps
+ * ([EXPL] "the map app also loads tiles": fetched bits are kept and reused
+ * while the selections repeat from token to token; on a miss the runtime
+ * either waits for the transfer or runs the channel at its resident precision
+ * for the moment).  Every array is device memory owned by the caller.
+ *   capacity    rows held, n_sel <= capacity <= 8192;
+ *   n_channels  the channel index space (the rows of host_rows);
+ *   row_bytes   bytes per row (a multiple of 16);
+ *   slot_of     [n_channels] int32: slot holding the channel's row, -1 if none;
+ *   channel_of  [capacity] int32: channel held by the slot, -1 if free;
+ *   stamp       [capacity] uint32: step of the slot's last use;
+ *   state       [4] uint32: step counter, clock hand, cumulative hits,
+ *               cumulative misses (readable for statistics);
+ *   work        [max_sel] int32: scratch of one call;
+ *   max_sel     the most entries one call stages (<= 4096);
+ *   rows        [capacity][row_bytes].
+ * sf_row_cache_reset() empties it (enqueued on `stream`).  Calls that share a
+ * cache must not overlap on the GPU. */
+typedef struct {
+  int32_t capacity, n_channels, row_bytes;
+  int32_t* slot_of;
+  int32_t* channel_of;
+  uint32_t* stamp;
+  uint32_t* state;
+  int32_t* work;
+  int32_t max_sel;
+  void* rows;
+} sf_row_cache;
+
+SF_API sf_status sf_row_cache_reset(const sf_row_cache* cache, sf_stream_t stream);
+
+/* sf_stage_refinements through row caches, one per batch row.  The selected
+ * channels a cache holds are copied from its device rows (no host-link
+ * traffic); every other channel gets the cache's slot least recently used and
+ * not needed now, and its row is read from host_rows (mapped pinned memory, as
+ * for sf_stage_refinements) into that slot.
+ *   sel      [batch][n_sel] DEVICE, distinct channels per batch row;
+ *   caches   HOST array of `batch` caches (1 <= batch <= 8);
+ *   dst      [batch][n_sel][row_bytes] DEVICE;
+ *   sel_eff  [batch][n_sel] DEVICE, receives the selection the GEMV is to use:
+ *            sel[b][j], or -1 - sel[b][j] for a channel that stays at base
+ *            precision in this step (sf_gemv_refined adds no correction for a
+ *            negative entry);
+ *   skip_missing = 0: missing rows are read into dst too, and sel_eff == sel;
+ *   skip_missing = 1: missing channels are marked in sel_eff and their rows go
+ *            only to the cache, after `done`, on the same stream: a GEMV that
+ *            waits for `done` does not wait for the host link (skip on miss);
+ *   `done` (nullable) is recorded once dst and sel_eff are complete.
+ * An entry of sel outside [0, n_rows) is not staged (sel_eff marks it
+ * skipped). */
+SF_API sf_status sf_stage_refinements_cached(const void* host_rows, size_t row_bytes, int n_rows,
+                                             const int32_t* sel, int n_sel, int batch,
+                                             const sf_row_cache* caches, int skip_missing, void* dst,
+                                             int32_t* sel_eff, sf_stream_t stream, sf_event_t done);
 
 /* ======================================================================== */
 /* Decoder-step glue (standard Llama operations around the refined ones)     */

@@ -102,11 +102,15 @@ def test_ktok_cap_every_attention_entry_point(L):
 
 
 def test_context_cap(L):
-    """t above 133,120 tokens is refused (the per-head scores live in one cluster's shared memory)."""
+    """t above 262,144 tokens is refused (the selection keeps a bitmap of a
+    head's tokens in shared memory); 262,144 itself passes the check and stops
+    at the missing workspace."""
     p16 = ctypes.c_void_p(16)
-    kv = abi.sf_kv(1, 8, 128, 140000, 2, 2, 32, 16, 16, 16, 16, 16, 16)
-    assert abi.sf_kv_attend_selective(ctypes.byref(kv), 133121, p16, 32, 64, p16, None, p16, None, 0, None) \
+    kv = abi.sf_kv(1, 8, 128, 270000, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), 262145, p16, 32, 64, p16, None, p16, None, 0, None) \
         == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_attend_selective(ctypes.byref(kv), 262144, p16, 32, 64, p16, None, p16, None, 0, None) \
+        == abi.SF_ERR_WORKSPACE
 
 
 def test_stage_host_index_out_of_range(L):

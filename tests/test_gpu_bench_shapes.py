@@ -15,10 +15,10 @@ import pytest
 import torch
 
 import oracle
-from oracle.decoder import OracleDecoder
 from bit_decode_selective_b200 import inputs
-from bit_decode_selective_b200.decoder import Decoder, DecoderConfig
+from bit_decode_selective_b200.decoder import DecoderConfig
 from bit_decode_selective_b200.ops import QuantWeights
+from decoder_pair import run_step_pair
 
 pytestmark = pytest.mark.gpu
 
@@ -76,28 +76,6 @@ def test_gemv_step_shapes_b2r2(name, n, k):
     assert rel_l2(yb.cpu().numpy() + yc.cpu().numpy(), want) <= RTOL_L2
 
 
-def run_step_pair(cfg: DecoderConfig, T: int, batch: int, seed: int = 4):
-    h16, lm = inputs.decoder_io(seed, batch, cfg.hidden, cfg.vocab)
-    dec = Decoder(cfg, batch, T)
-    ref = OracleDecoder(h16, h_q=cfg.h_q, h_kv=cfg.h_kv, d=cfg.d, r=cfg.w_refine, G=cfg.group,
-                        chunk=cfg.chunk, kch=cfg.kch, kv_b=cfg.kv_bits, kv_r=cfg.kv_refine, k_tok=cfg.k_tok,
-                        lead=cfg.lead, lag=cfg.lag, eps=cfg.eps, theta=cfg.theta)
-    for l in range(cfg.n_layers):
-        W = inputs.decoder_layer_weights(seed, l, cfg.hidden, cfg.inter, cfg.h_q, cfg.h_kv, cfg.d)
-        k, v = inputs.decoder_layer_kv(seed, l, T, batch, cfg.h_kv, cfg.d)
-        dec.load_layer({n: cu(w) for n, w in W.items()}, cu(k.view(np.uint16)), cu(v.view(np.uint16)))
-        Q = {n: oracle.quant_weights(w, cfg.w_bits, cfg.w_refine, cfg.group) for n, w in W.items()}
-        del W
-        ref.layer(Q, k, v, T)
-        del Q, k, v
-    dec.set_lm_head(cu(lm.view(np.uint16)))
-    logits = dec.step(cu(h16.view(np.uint16)))
-    torch.cuda.synchronize()
-    got = logits.cpu().numpy()
-    want = ref.finish(lm)
-    return rel_l2(got, want)
-
-
 @pytest.mark.slow
 @pytest.mark.parametrize("batch", [1, 8])
 def test_decode_step_full_shape(batch):
@@ -105,5 +83,5 @@ def test_decode_step_full_shape(batch):
     14,336, vocab 128,256), T = 32,768, top-512 tokens, lead = lag = 1,
     refinement rows in pinned host memory staged per layer."""
     cfg = DecoderConfig(n_layers=2, lead=1, lag=1, host_refine=True)
-    err = run_step_pair(cfg, T=32768, batch=batch)
-    assert err <= RTOL_L2, err
+    err, wf, tf = run_step_pair(cfg, T=32768, batch=batch)
+    assert err <= RTOL_L2, (err, wf, tf)

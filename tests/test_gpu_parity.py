@@ -130,6 +130,24 @@ def gemv_check(w, x, b, r, G, chunk, kch, staged=False, give_sel=False):
     return err
 
 
+def fixed_point_bound(qb, rho, sz, r, G, x):
+    """Elementwise bound on |y_gpu - y| for the GEMV's arithmetic: the base
+    product takes x in fixed point per 64-channel block, x_fix =
+    round(x * 2^(19 - ilogb(max |x| of the block))), so each x_c moves by at most
+    half a step, 2^(ilogb - 20) (every x_c within 2^9 of the block's largest is
+    exact); the correction uses x_c as is.  Plus fp32 rounding of the partial
+    sums (a few ulps of the sum of |terms|)."""
+    f16 = lambda a: np.asarray(a, np.uint16).view(np.float16).astype(np.float64)
+    SQ = np.abs(np.repeat(f16(sz[:, :, 0]), G, axis=1) * qb)   # |s q|, the terms that take x_fix
+    M = np.abs(np.repeat(f16(sz[:, :, 1]), G, axis=1))
+    xb = x.astype(np.float64).reshape(x.shape[0], -1, 64)
+    mx = np.abs(xb).max(-1)
+    half = np.where(mx > 0, 2.0 ** (np.floor(np.log2(np.where(mx > 0, mx, 1))) - 20), 0.0)
+    h = np.repeat(half, 64, axis=-1)                        # [batch][k]
+    ax = np.abs(x.astype(np.float64))
+    return SQ @ h.T + 1e-5 * ((SQ + M) @ ax.T)              # [n][batch]
+
+
 @pytest.mark.parametrize("b,r", [(2, 2), (2, 1), (3, 1), (3, 2), (4, 2)])
 @pytest.mark.parametrize("kch", [0, 32, 1024])
 def test_gemv_parity(b, r, kch):
@@ -137,8 +155,16 @@ def test_gemv_parity(b, r, kch):
     # k = 3072: one full 2048-channel segment plus a half one (ragged lane tail)
     w = inputs.weight(rng, 384, 3072)
     x = inputs.activation(rng, 3072, batch=1)
-    err = gemv_check(w, x, b, r, 128, 1024, kch)
-    assert err < 1e-5  # fp32 accumulation of exact fixed-point partial sums
+    gemv_check(w, x, b, r, 128, 1024, kch)
+    # elementwise, within the bound the fixed-point activations allow
+    qb, rho, sz = oracle.quant_weights(w, b, r, 128)
+    qw = QuantWeights.pack(cu(w), b, r, 128)
+    y, _ = qw.gemv(cu(f16bits(x)), 1024, kch)
+    torch.cuda.synchronize()
+    sel_o = oracle.select_chunks(x, 1024, kch) if kch else None
+    yo = oracle.gemv_refined(qb, rho, sz, r, 128, x, sel_o, 1024, kch)
+    bound = fixed_point_bound(qb, rho, sz, r, 128, x).T
+    assert np.all(np.abs(host(y) - yo) <= bound)
 
 
 @pytest.mark.parametrize("batch", [2, 5])
@@ -458,3 +484,129 @@ def test_stage_refinements_out_of_range_index():
         else:
             assert int(got[j].sum()) == 0
     assert bad[0].item() == 3
+
+
+# ---------------------------------------------------------------------------
+# refinement rows cached across steps
+
+
+class CachePolicy:
+    """The row cache's replacement rule, restated: a selected channel the cache
+    holds is a hit (its slot is marked used in this step); each missing channel,
+    in entry order, takes the next slot not used in this step, in clock order
+    from the hand, and the hand moves past the last slot taken."""
+
+    def __init__(self, cap):
+        self.cap, self.slot_of, self.channel_of = cap, {}, [-1] * cap
+        self.stamp, self.now, self.hand = [0] * cap, 0, 0
+
+    def call(self, sel):
+        self.now += 1
+        hit = [c in self.slot_of for c in sel]
+        for c, h in zip(sel, hit):
+            if h:
+                self.stamp[self.slot_of[c]] = self.now
+        free = [(self.hand + i) % self.cap for i in range(self.cap)
+                if self.stamp[(self.hand + i) % self.cap] != self.now]
+        misses = [c for c, h in zip(sel, hit) if not h]
+        for c, v in zip(misses, free):
+            old = self.channel_of[v]
+            if old >= 0:
+                del self.slot_of[old]
+            self.channel_of[v], self.slot_of[c], self.stamp[v] = c, v, self.now
+        if misses:
+            self.hand = (free[len(misses) - 1] + 1) % self.cap
+        return hit
+
+
+def make_caches(batch, cap, n_ch, row_bytes, n_sel):
+    i32 = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    arr = (abi.sf_row_cache * batch)()
+    keep = []
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for b in range(batch):
+        t = dict(slot_of=i32(n_ch), channel_of=i32(cap), stamp=i32(cap), state=i32(4), work=i32(n_sel),
+                 rows=torch.empty(cap * row_bytes, dtype=torch.uint8, device="cuda"))
+        keep.append(t)
+        arr[b] = abi.sf_row_cache(cap, n_ch, row_bytes, t["slot_of"].data_ptr(), t["channel_of"].data_ptr(),
+                                  t["stamp"].data_ptr(), t["state"].data_ptr(), t["work"].data_ptr(), n_sel,
+                                  t["rows"].data_ptr())
+        abi.check(abi.sf_row_cache_reset(ctypes.byref(arr[b]), s), "sf_row_cache_reset")
+    return arr, keep
+
+
+@pytest.mark.parametrize("skip", [0, 1])
+def test_stage_refinements_cached(skip):
+    """Six steps of selections that partly repeat, two batch rows with a cache
+    each: staged rows equal the host rows of the entries the GEMV will refine;
+    hits and misses follow the replacement rule exactly; with skip, missing
+    channels are marked -1 - c in the effective selection and their rows are in
+    the cache (a hit) when the same channel comes again."""
+    n_ch, row_bytes, n_sel, cap, batch = 1000, 256, 64, 96, 2
+    rng = np.random.default_rng(80 + skip)
+    host_rows = torch.from_numpy(rng.integers(0, 256, n_ch * row_bytes, dtype=np.uint8)).pin_memory()
+    src = host_rows.view(n_ch, row_bytes)
+    arr, keep = make_caches(batch, cap, n_ch, row_bytes, n_sel)
+    models = [CachePolicy(cap) for _ in range(batch)]
+    prev = [rng.choice(n_ch, n_sel, replace=False) for _ in range(batch)]
+    dst = torch.empty(batch * n_sel * row_bytes, dtype=torch.uint8, device="cuda")
+    eff = torch.empty((batch, n_sel), dtype=torch.int32, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for step in range(6):
+        sels = []
+        for b in range(batch):
+            keepn = int(rng.integers(0, n_sel + 1))
+            old = rng.permutation(prev[b])[:keepn]
+            pool = np.setdiff1d(np.arange(n_ch), old)
+            sels.append(np.concatenate([old, rng.choice(pool, n_sel - keepn, replace=False)]).astype(np.int32))
+        prev = sels
+        sel_d = cu(np.stack(sels))
+        dst.fill_(0)
+        abi.check(abi.sf_stage_refinements_cached(ctypes.c_void_p(host_rows.data_ptr()), row_bytes, n_ch,
+                                                  _p(sel_d), n_sel, batch, arr, skip, _p(dst), _p(eff), s, None),
+                  "sf_stage_refinements_cached")
+        torch.cuda.synchronize()
+        got = dst.cpu().view(batch, n_sel, row_bytes)
+        e = host(eff)
+        for b in range(batch):
+            hit = models[b].call(sels[b].tolist())
+            for j, c in enumerate(sels[b]):
+                if skip and not hit[j]:
+                    assert e[b, j] == -1 - c
+                else:
+                    assert e[b, j] == c
+                    assert torch.equal(got[b, j], src[c]), (step, b, j)
+            st = host(keep[b]["state"]).view(np.uint32)
+            assert st[0] == step + 1
+    # every cached slot holds its channel's row
+    for b in range(batch):
+        ch = host(keep[b]["channel_of"])
+        rows = keep[b]["rows"].cpu().view(cap, row_bytes)
+        for slot in range(cap):
+            if ch[slot] >= 0:
+                assert torch.equal(rows[slot], src[ch[slot]])
+
+
+def test_gemv_skipped_entries_get_no_correction():
+    """An entry -1 - c of the selection leaves channel c at base precision: the
+    GEMV equals the base product plus the correction of the other entries."""
+    rng = np.random.default_rng(91)
+    w = inputs.weight(rng, 512, 4096)
+    x = inputs.activation(rng, 4096, batch=1)
+    qb, rho, sz = oracle.quant_weights(w, 2, 2, 128)
+    qw = QuantWeights.pack(cu(w), 2, 2, 128)
+    sel_o = oracle.select_chunks(x, 1024, 32)
+    flat = sel_o.reshape(-1).copy()
+    skip = rng.random(flat.size) < 0.4
+    eff = np.where(skip, -1 - flat, flat).astype(np.int32).reshape(sel_o.shape)
+    rows = qw.refine_rows()[cu(flat).long()].contiguous()
+    y, _ = qw.gemv(cu(f16bits(x)), 1024, 32, sel_in=cu(eff), refine_rows=rows)
+    yb, yc = qw.gemv_split(cu(f16bits(x)), cu(eff), 1024, 32, refine_rows=rows)
+    y2 = torch.zeros_like(y)
+    qw.correction(cu(f16bits(x)), cu(eff), y2, 1024, 32, refine_rows=rows)
+    torch.cuda.synchronize()
+    base = oracle.gemv_refined(qb, rho, sz, 2, 128, x, None, 1024, 0)
+    corr = oracle.gemv_correction(qb, rho, sz, 2, 128, x[0], flat[~skip])
+    assert rel_l2(host(y)[0], base[0] + corr) < 1e-5
+    assert rel_l2(host(yc)[0], corr) < 1e-5
+    assert rel_l2(host(y2)[0], corr) < 1e-5

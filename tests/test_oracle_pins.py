@@ -673,3 +673,49 @@ def test_oracle_decoder_down_lag_lands_with_down(orc):
     correction to hold back), lag 1 equals lag 0 up to the order of the sums."""
     outs = _lag_case(orc, 72, zero=("o",))
     assert np.allclose(outs[0], outs[1], rtol=1e-10, atol=1e-12)
+
+
+def test_oracle_decoder_forced_selections_are_its_own(orc):
+    """Teacher forcing (used by the decode-step parity tests) is plumbing only:
+    forcing the oracle to the selections it would make itself leaves every
+    output bit unchanged, and every recorded own choice equals the forced one;
+    forcing one channel swap changes the output."""
+    from oracle.decoder import OracleDecoder
+
+    rng = np.random.default_rng(73)
+    H, I, h_q, h_kv, d, T = 512, 1024, 4, 2, 128, 20
+    h16 = rng.normal(0, 1, (2, H)).astype(np.float16)
+    shapes = {"qkv": ((h_q + 2 * h_kv) * d, H), "o": (H, h_q * d), "gate_up": (2 * I, H), "down": (H, I)}
+    layers = []
+    for _ in range(2):
+        W = {n: orc.quant_weights(rng.normal(0, 0.05, s).astype(np.float32), 2, 2, 128) for n, s in shapes.items()}
+        layers.append((W, rng.normal(0, 1, (2, h_kv, T, d)).astype(np.float16),
+                       rng.normal(0, 1, (2, h_kv, T, d)).astype(np.float16)))
+    lm = rng.normal(0, 0.02, (50, H)).astype(np.float16)
+    kw = dict(h_q=h_q, h_kv=h_kv, d=d, chunk=256, kch=16, k_tok=5, lead=1, lag=1)
+
+    def run(force):
+        dec = OracleDecoder(h16, force=force, **kw)
+        for W, kc, vc in layers:
+            dec.layer(W, kc, vc, T)
+        return dec, dec.finish(lm)
+
+    free, out0 = run(None)
+    force = {}
+    for l, tr in enumerate(free.trace):
+        for name, per_b in tr["weights"].items():
+            force[("w", l, name)] = np.stack([np.asarray(s).reshape(-1) for s in per_b])
+        force[("tok", l)] = np.stack(tr["tokens"])
+    forced, out1 = run(force)
+    assert np.array_equal(out0, out1)
+    assert len(forced.checks) == 2 * 2 * 5
+    for kind, l, name, b, own, f, vals in forced.checks:
+        assert np.array_equal(np.asarray(own).reshape(-1), np.asarray(f).reshape(-1))
+    # swap one selected channel of layer 1's gate_up for an unselected one
+    f2 = {k: v.copy() for k, v in force.items()}
+    row = f2[("w", 1, "gate_up")][0]
+    chunk0 = set(row[:16].tolist())
+    row[0] = next(c for c in range(256) if c not in chunk0)
+    row[:16] = np.sort(row[:16])
+    _, out2 = run(f2)
+    assert not np.array_equal(out0, out2)
