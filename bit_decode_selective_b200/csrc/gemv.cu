@@ -23,11 +23,12 @@
 // memory stages with 1-D bulk copies (cp.async.bulk, completion counted on an
 // mbarrier per stage), and copies the rows' (s, m) words once.  The weights do
 // not depend on earlier kernels, so these copies start before the grid
-// dependency wait and overlap the previous kernel's tail.  After the wait the
-// warp builds the correction tables (selected channel, x_c, group) and copies
-// the refinement words of the CTA's rows with cp.async.
+// dependency wait and overlap the previous kernel's tail.
 //
-// Compute warps: warp w owns the 2,048-channel segment w % segs (lane L: 64
+// Compute warps: after the grid dependency wait they build the correction
+// tables (selected channel, x_c, group; the refinement words of the CTA's rows
+// copied with cp.async) and the activation planes (four threads per 64-channel
+// block) together.  Warp w owns the 2,048-channel segment w % segs (lane L: 64
 // consecutive channels) for every row whose index in its stage is congruent to
 // w / segs.  Its activations are turned once into fixed point
 // x = x_fix * 2^e per 64-channel lane block (e from the block's largest |x|,
@@ -176,45 +177,55 @@ __host__ __device__ __forceinline__ int chan_of(int v, int L) {
   return 16 * (v >> 2) + (v & 3) + 4 * L;
 }
 
-// Lane block lg of x (64 channels) as fixed point: planes[kXP * v + p] = byte p
-// of x_fix for the four channels of code vector v; then sum of channels 0-31,
-// sum of 32-63 and the factor that turns the integer dot product back into
-// x units (2^e, divided by 4 where the byte vectors carry the factor 4).
+// A quarter of lane block b of x (64 channels) as fixed point, by the four
+// consecutive lanes of a quad (quarter q = lane & 3: channels 16q .. 16q + 15,
+// which are exactly the channels of code vectors 4q .. 4q + 3).  The block's
+// exponent comes from the quad's largest |x|; dst = the block's shared words:
+// planes[kXP * v + p] = byte p of x_fix for the four channels of vector v,
+// then the sum of channels 0-31, of 32-63 and the factor that turns the
+// integer dot product back into x units (2^e, divided by 4 where the byte
+// vectors carry the factor 4).  Whole warps (valid = false: the lane computes
+// nothing but takes part in the shuffles).
 template <int BITS>
-__device__ void lane_planes(const uint16_t* __restrict__ xb, uint32_t* __restrict__ dst) {
-  uint32_t h[32];
-#pragma unroll
-  for (int v = 0; v < 8; v++) {
-    const uint4 q = reinterpret_cast<const uint4*>(xb)[v];
-    h[4 * v] = q.x, h[4 * v + 1] = q.y, h[4 * v + 2] = q.z, h[4 * v + 3] = q.w;
+__device__ __forceinline__ void quarter_planes(bool valid, const uint16_t* __restrict__ xq, int q,
+                                               uint32_t* __restrict__ dst) {
+  uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  if (valid) {
+    const uint4 a0 = reinterpret_cast<const uint4*>(xq)[0], a1 = reinterpret_cast<const uint4*>(xq)[1];
+    h[0] = a0.x, h[1] = a0.y, h[2] = a0.z, h[3] = a0.w, h[4] = a1.x, h[5] = a1.y, h[6] = a1.z, h[7] = a1.w;
   }
   uint32_t mx2 = 0;
 #pragma unroll
-  for (int i = 0; i < 32; i++) mx2 = __vmaxu2(mx2, h[i] & 0x7fff7fffu);
-  const uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
-  float s0 = 0.f, s1 = 0.f;
+  for (int i = 0; i < 8; i++) mx2 = __vmaxu2(mx2, h[i] & 0x7fff7fffu);
+  uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; i++) {
+  for (int i = 0; i < 8; i++) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    if (i < 16) s0 += f.x, s0 += f.y;
-    else s1 += f.x, s1 += f.y;
+    sq += f.x, sq += f.y;
   }
+  const float sh = sq + __shfl_xor_sync(0xffffffffu, sq, 1);  // quarters 0+1 or 2+3
+  const float so = __shfl_xor_sync(0xffffffffu, sh, 2);       // the other half
   // x_fix = x * 2^(kXE - ilogb(max |x|)): the largest values are fp16
   // mantissas times 2^(kXE - 10) (exact), smaller ones round to that step
   const int eb = mx ? ((__float_as_int(h2f((uint16_t)mx)) >> 23) & 0xff) - 127 : 0;  // ilogb(max |x|)
   const float scale = mx ? __int_as_float((127 + kXE - eb) << 23) : 0.f;
-  int q[64];
+  if (!valid) return;
+  int qv[16];
 #pragma unroll
-  for (int i = 0; i < 32; i++) {
+  for (int i = 0; i < 8; i++) {
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
     // round to nearest even through the float mantissa: 1.5 * 2^23 + x_fix
-    q[2 * i] = __float_as_int(fmaf(f.x, scale, 12582912.0f)) - 0x4B400000;
-    q[2 * i + 1] = __float_as_int(fmaf(f.y, scale, 12582912.0f)) - 0x4B400000;
+    qv[2 * i] = __float_as_int(fmaf(f.x, scale, 12582912.0f)) - 0x4B400000;
+    qv[2 * i + 1] = __float_as_int(fmaf(f.y, scale, 12582912.0f)) - 0x4B400000;
   }
 #pragma unroll
-  for (int v = 0; v < 16; v++) {
-    const int a = q[chan_of<BITS>(v, 0)], b = q[chan_of<BITS>(v, 1)];
-    const int c = q[chan_of<BITS>(v, 2)], d = q[chan_of<BITS>(v, 3)];
+  for (int vv = 0; vv < 4; vv++) {
+    const int v = 4 * q + vv;
+    const int a = qv[chan_of<BITS>(vv, 0) & 15], b = qv[chan_of<BITS>(vv, 1) & 15];
+    const int c = qv[chan_of<BITS>(vv, 2) & 15], d = qv[chan_of<BITS>(vv, 3) & 15];
 #pragma unroll
     for (int p = 0; p < kXP; p++) {
       const uint32_t sel = (uint32_t)p | ((uint32_t)(4 + p) << 4);
@@ -223,11 +234,13 @@ __device__ void lane_planes(const uint16_t* __restrict__ xb, uint32_t* __restric
       dst[kXP * v + p] = __byte_perm(t01, t23, 0x5410);
     }
   }
-  float* f = reinterpret_cast<float*>(dst + 16 * kXP);
-  f[0] = s0;
-  f[1] = s1;
-  f[2] = mx ? __int_as_float((127 + eb - kXE - (BITS == 4 ? 0 : 2)) << 23) : 1.0f;
-  f[3] = 0.f;
+  if (q == 0) {
+    float* f = reinterpret_cast<float*>(dst + 16 * kXP);
+    f[0] = sh;
+    f[1] = so;
+    f[2] = mx ? __int_as_float((127 + eb - kXE - (BITS == 4 ? 0 : 2)) << 23) : 1.0f;
+    f[3] = 0.f;
+  }
 }
 
 // ---- the base pass of one row -------------------------------------------------
@@ -403,21 +416,7 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
       bulk_g2s(szs, a.sz + (size_t)n0 * a.gpr, zb, szbar);
       for (; issued < min(S, nst); issued++) issue(issued);
     }
-    pdl_wait();  // x, the selection and the staged rows are complete
-    if (corr) {
-      // correction tables: (x_c, group of c) and the refinement words of the CTA's rows
-      for (int j = lane; j < a.n_sel; j += 32) {
-        // -1 - c: channel c selected but not refined now (no correction); a
-        // foreign index is clamped, so it never leaves the buffers
-        const int raw = __ldg(a.sel + j);
-        const int c = min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
-        const uint32_t xc = raw < 0 ? 0u : __float_as_uint(h2f(__ldg(a.x + c)));
-        jd[j] = make_uint2(xc, (uint32_t)(c >> a.gshift));
-        const uint32_t* src = a.refine + (size_t)(a.staged ? j : c) * a.row_words + w_lo;
-        for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)j * a.wt_pitch + k, src + k);
-      }
-      cp_async_commit();
-    }
+    pdl_wait();  // the previous kernel is complete (no data of it is read here)
     if (lane == 0) {
       for (; issued < nst; issued++) {
         const int slot = issued % S;
@@ -428,23 +427,47 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
       for (int i = max(0, issued - S); i < issued; i++) mbar_wait(&full[i % S], (i / S) & 1);
       mbar_wait(szbar, 0);
     }
-    cp_async_wait_all();
     __syncwarp();
   } else {
     // ---------------- compute warps
     const int seg = warp % a.segs, jw = warp / a.segs;
     const int lg = seg * 32 + lane;  // lane block
     const bool la = lg * kLaneCh < a.K;
-    pdl_wait();
-    // activation planes of segment `warp`, one warp per segment
-    if (warp < a.segs) {
-      uint32_t* dst = xpl + ((size_t)warp * 32 + lane) * kXW;
-      if (la) {
-        lane_planes<BITS>(a.x + (size_t)lg * kLaneCh, dst);
-      } else {
-#pragma unroll 4
-        for (int k = 0; k < kXW; k++) dst[k] = 0u;
+    const int tc = threadIdx.x, ntc = a.W * 32;
+    pdl_wait();  // x, the selection and the staged rows are complete
+    // correction tables, entries tc, tc + ntc, ...: the selection's loads are
+    // issued first, their activations after the planes (every load of a round
+    // in flight together)
+    constexpr int kJ = 2;
+    int rawj[kJ];
+    if (corr)
+#pragma unroll
+      for (int u = 0; u < kJ; u++) rawj[u] = tc + u * ntc < a.n_sel ? __ldg(a.sel + tc + u * ntc) : 0;
+    // activation planes: four threads per 64-channel lane block
+    {
+      const int nq = (a.K / kLaneCh) * 4;
+      for (int b0 = warp * 32; b0 < nq; b0 += ntc) {
+        const int idx = b0 + lane, b = idx >> 2, q = idx & 3;
+        quarter_planes<BITS>(idx < nq, a.x + (size_t)b * kLaneCh + 16 * q, q, xpl + (size_t)b * kXW);
       }
+    }
+    if (corr) {
+      // -1 - c: channel c selected but not refined now (no correction); a
+      // foreign index is clamped, so it never leaves the buffers
+      for (int j0 = 0; j0 < a.n_sel; j0 += kJ * ntc) {
+#pragma unroll
+        for (int u = 0; u < kJ; u++) {
+          const int j = j0 + tc + u * ntc;
+          if (j >= a.n_sel) continue;
+          const int raw = j0 == 0 ? rawj[u] : __ldg(a.sel + j);
+          const int c = min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
+          const uint32_t xc = raw < 0 ? 0u : __float_as_uint(h2f(__ldg(a.x + c)));
+          jd[j] = make_uint2(xc, (uint32_t)(c >> a.gshift));
+          const uint32_t* src = a.refine + (size_t)(a.staged ? j : c) * a.row_words + w_lo;
+          for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)j * a.wt_pitch + k, src + k);
+        }
+      }
+      cp_async_commit();
     }
     bar_sync(1, a.W * 32);
     uint32_t xr[16 * kXP];
@@ -494,6 +517,7 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
+    cp_async_wait_all();  // this thread's refinement words
   }
   bar_sync(2, blockDim.x);  // base pass, tables and refinement words complete
 
@@ -705,7 +729,9 @@ sf_status make_plan(const sf_wq* w, int n_sel, Plan& P) {
   P.threads = (a.W + 1) * 32;
   P.zw = w->group == 32 ? 2 : 1;
   const int nb_max = a.rows_max / 4;
-  a.cparts = n_sel > 0 ? std::max(1, std::min(n_sel, P.threads / nb_max)) : 0;
+  // channel shares of the correction: enough threads busy, and few partial
+  // sums per row for the output's serial add
+  a.cparts = n_sel > 0 ? std::max(1, std::min(std::min(n_sel, 16), P.threads / nb_max)) : 0;
   size_t off = align128((2 * kMaxStages + 1) * sizeof(uint64_t));
   a.off_sz = (int)off;
   off += align128((size_t)a.rows_max * a.gpr * 4);

@@ -21,12 +21,12 @@
 //                   integers in registers and contracted on the tensor cores
 //                   (mma.sync m16n8k16, fp32 accumulation); the per-token fp16
 //                   steps/offsets are applied in fp32.
-//   kv_select_kernel  scores every token (sum over the group's query heads of
-//                   the softmax probability, from the stored logits and the
-//                   statistics of the partials) and selects the top k_tok per
-//                   KV head: a histogram of the score bits, then, in the last
-//                   CTA of the head, the exact k_tok-th score and the selected
-//                   tokens in ascending order;
+//   kv_score_kernel, kv_pick_kernel  score every token (sum over the group's
+//                   query heads of the softmax probability, from the stored
+//                   logits and the statistics of the partials) and select the
+//                   top k_tok per KV head: a histogram of the score bits, the
+//                   boundary bucket, and in the head's last CTA the exact
+//                   k_tok-th score and the selected tokens in ascending order;
 //   kv_refine_kernel  swaps the selected tokens' base contributions for
 //                   their refined ones (relative to the head's softmax
 //                   maximum) and merges the partials by log-sum-exp.
@@ -47,7 +47,7 @@ constexpr int kD = kHeadDim;
 constexpr int kRec = kD + 2;     // partial record: acc[kD], m, l
 constexpr int kWarps = 4;        // warps per base-pass CTA (independent splits)
 constexpr int kStages = 4;       // cp.async ring depth per warp
-constexpr int kCtlWords = 2048 + 4;  // per head: selection histogram and two counters (kCtl below)
+constexpr int kCtlWords = 2048 + 32;  // per head: selection histogram, two counters, statistics (kCtl below)
 
 // ---- small PTX helpers -------------------------------------------------------
 
@@ -489,21 +489,23 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
 // ---------------------------------------------------------------------------
 // after the base pass: scoring and selection, then refinement and merge
 //
-// kv_select_kernel -- CTAs of kSelThreads threads over slices of kSelTok
+// kv_score_kernel -- CTAs of kSelThreads threads over slices of kSelTok
 // tokens of one (batch, KV head).  Each computes the softmax statistics of the
 // group's query heads from the base pass's split records, the scores of its
 // tokens from the stored logits (written out: the sum over the group's query
 // heads of each head's softmax probability), and the histogram of the score
 // keys' bits 30..20, added into the head's histogram in the workspace.  Scores
 // are non-negative, so their bit patterns order like their values; bits 30..20
-// are the exponent and the top three mantissa bits.  The last CTA of the head
-// to finish (an atomic counter: no CTA ever waits for another) selects: the
-// bucket that holds the k_tok-th largest key, from the histogram; one pass
-// over the scores marks every token of a higher bucket in a shared-memory
-// bitmap and collects the boundary bucket's keys and tokens; two 10-bit digits
-// over those pin the k_tok-th largest key K* exactly; the collected tokens
-// above K* are marked, and of the tokens equal to K* the lowest-indexed ones;
-// the marked tokens are written in ascending order.
+// are the exponent and the top three mantissa bits.
+//
+// kv_pick_kernel -- the same CTAs again: each finds, from the complete
+// histogram, the bucket that holds the k_tok-th largest key, writes the bitmap
+// words of its tokens in higher buckets and appends its boundary-bucket
+// (key, token) pairs to the head's list.  The last CTA of the head to finish
+// (an atomic counter: no CTA ever waits for another) loads the bitmap and the
+// list, pins the k_tok-th largest key K* with two 10-bit digits over the list,
+// marks the tokens above K* and the lowest-indexed ones equal to it, and
+// writes the marked tokens in ascending order.
 //
 // kv_refine_kernel -- kRefParts CTAs per (batch, KV head), each with a share
 // of the selected tokens and of the base pass's split records.  Per selected
@@ -519,8 +521,12 @@ constexpr int kSelTok = 2048;        // tokens scored per CTA
 constexpr int kBins1 = 2048;         // first digit: key bits 30..20
 constexpr int kBins2 = 1024;         // then bits 19..10 and 9..0
 constexpr int kCandCap = 4096;       // boundary-bucket keys held in shared memory
+constexpr int kTieCap = 2048;        // tokens equal to the k-th key ranked in shared memory
 constexpr int kMaxT = 1 << 18;       // tokens a head's bitmap holds in shared memory
-constexpr int kCtl = kBins1 + 4;     // per head: histogram, selection counter, refinement counter
+// per head: histogram, selection counter, refinement counter, a flag, then
+// (M, Z) of each of the group's query heads (up to 8), written by the selection
+constexpr int kCtl = kBins1 + 32;
+constexpr int kCtlStats = kBins1 + 4;
 static_assert(kCtl == kCtlWords, "the base pass zeroes exactly the control words");
 constexpr int kRefThreads = 256;
 constexpr int kRefWarps = kRefThreads / 32;
@@ -530,21 +536,25 @@ constexpr int kMaxKTok = 4096;       // the largest k_tok every attention entry 
 static_assert(kRefTPW * 8 <= 32, "a warp's (token, head) slots must fit its lanes");
 
 // Softmax statistics of query head h from the split records: M = max m,
-// Z = sum l exp(m - M).  One warp.
+// Z = sum l exp(m - M), in one pass (online rescaling).  One warp.
 __device__ __forceinline__ void head_stats(const float* __restrict__ pr, int nrec, int rec, int lane, float& M,
                                            float& Z) {
-  float m = -INFINITY;
-  for (int s = lane; s < nrec; s += 32) m = fmaxf(m, pr[(long)s * rec + rec - 2]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float z = 0.f;
-  if (m > -INFINITY)
-    for (int s = lane; s < nrec; s += 32) {
-      const float ms = pr[(long)s * rec + rec - 2];
-      if (ms > -INFINITY) z += pr[(long)s * rec + rec - 1] * expf(ms - m);
+  float m = -INFINITY, z = 0.f;
+  for (int s = lane; s < nrec; s += 32) {
+    const float ms = pr[(long)s * rec + rec - 2], ls = pr[(long)s * rec + rec - 1];
+    if (ms > -INFINITY) {
+      const float mn = fmaxf(m, ms);
+      z = z * expf(m - mn) + ls * expf(ms - mn);
+      m = mn;
     }
+  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o), zo = __shfl_xor_sync(0xffffffffu, z, o);
+    const float mn = fmaxf(m, mo);
+    z = (m > -INFINITY ? z * expf(m - mn) : 0.f) + (mo > -INFINITY ? zo * expf(mo - mn) : 0.f);
+    m = mn;
+  }
   M = m, Z = z;
 }
 
@@ -609,6 +619,14 @@ __device__ int find_bucket(const int* __restrict__ hist, int nb, int kneed, int*
   return res[0];
 }
 
+// Add 1 to hist[bin] for every lane with bin >= 0; lanes with equal bins add
+// once, by their count (scores often share a bucket: one same-address atomic
+// per lane would serialise).  Whole warps only.
+__device__ __forceinline__ void hist_add(int* hist, int bin) {
+  const unsigned same = __match_any_sync(0xffffffffu, bin);
+  if (bin >= 0 && (__ffs(same) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], __popc(same));
+}
+
 struct SelArgs {
   const float* logits;  // [batch][h_q][T] base logits (scaled)
   const float* part;    // [batch][h_q][nrec][rec]
@@ -617,6 +635,8 @@ struct SelArgs {
   float* scores;        // [batch][h_kv][Tp] (Tp = T rounded up to 32: whole 16-byte rows)
   float* scores_out;    // nullable [batch][h_kv][T]: the scores for the caller
   int* ctl;             // [batch][h_kv][kCtl]
+  uint32_t* bitmap;     // [batch][h_kv][Tp / 32]: tokens of the buckets above the boundary
+  uint2* cand;          // [batch][h_kv][kCandCap]: (key, token) of the boundary bucket
   int32_t* sel;         // [batch][h_kv][k_tok]
 };
 
@@ -626,36 +646,33 @@ struct SelShared {
   int res[2];
   int ncand, last;
   float M[8], iZ[8];
+  uint32_t words[kSelTok / 32];
 };
 
-// Dynamic shared memory of a selection CTA: the bitmap of selected tokens,
-// the boundary bucket's keys and tokens, per-thread tie counts.
-constexpr size_t kSelDyn = (size_t)(kMaxT / 32) * 4 + (size_t)kCandCap * 8 + (size_t)kSelThreads * 4;
-
+// kv_score_kernel: the statistics, the scores of the CTA's tokens and their
+// histogram, added into the head's histogram.
 template <int GQP>
-__global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads) kv_score_kernel(SelArgs a) {
   __shared__ SelShared sh;
-  extern __shared__ __align__(16) uint32_t dyn_sel[];
-  uint32_t* bits = dyn_sel;                                    // [kMaxT / 32]
-  uint32_t* ck = bits + kMaxT / 32;                            // [kCandCap] keys
-  int* ct = reinterpret_cast<int*>(ck + kCandCap);             // [kCandCap] tokens
-  int* tie = ct + kCandCap;                                    // [kSelThreads]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = blockIdx.y, bat = blockIdx.z, gq = a.gq;
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
   pdl_wait();  // the base pass (logits, records, zeroed histogram) is complete
-
   if (warp < gq) {
     float M, Z;
     head_stats(a.part + (hq0 + warp) * a.nrec * a.rec, a.nrec, a.rec, lane, M, Z);
-    if (lane == 0) sh.M[warp] = M, sh.iZ[warp] = 1.0f / Z;
+    if (lane == 0) {
+      sh.M[warp] = M, sh.iZ[warp] = 1.0f / Z;
+      if (blockIdx.x == 0) {  // for the refinement after it
+        float* st = reinterpret_cast<float*>(a.ctl + head * kCtl + kCtlStats);
+        st[2 * warp] = M, st[2 * warp + 1] = Z;
+      }
+    }
   }
   for (int i = tid; i < kBins1; i += kSelThreads) sh.hist[i] = 0;
   __syncthreads();
-
-  // ---- scores of this CTA's tokens and their histogram
   float* sc = a.scores + head * a.Tp;
   float* sco = a.scores_out ? a.scores_out + head * a.T : nullptr;
   {
@@ -673,6 +690,7 @@ __global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
 #pragma unroll
     for (int u = 0; u < U; u++) {
       const int t = t0 + tid + kSelThreads * u;
+      int bin = -1;
       if (t < t1) {
         float s = 0.f;
 #pragma unroll
@@ -680,69 +698,123 @@ __global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
           if (h < gq) s += expf(l[h][u] - sh.M[h]) * sh.iZ[h];  // full-accuracy exp: the score decides
         sc[t] = s;
         if (sco) sco[t] = s;
-        atomicAdd(&sh.hist[__float_as_uint(s) >> 20], 1);
+        bin = (int)(__float_as_uint(s) >> 20);
       }
+      hist_add(sh.hist, bin);
     }
   }
   __syncthreads();
   int* gh = a.ctl + head * kCtl;
   for (int i = tid; i < kBins1; i += kSelThreads)
     if (sh.hist[i]) atomicAdd(&gh[i], sh.hist[i]);
-  __threadfence();  // this CTA's scores and histogram before its count
-  __syncthreads();
-  if (tid == 0) sh.last = atomicAdd(&gh[kBins1], 1) == a.nblk - 1;
-  __syncthreads();
-  if (!sh.last) return;
-  __threadfence();  // every other CTA's scores and histogram are visible
+}
 
-  // ---- the last CTA of the head selects
-  const int T = a.T;
-  const int nw = (T + 31) / 32;                       // bitmap words
-  const int wper = (nw + kSelThreads - 1) / kSelThreads;
-  const int w0 = min(nw, tid * wper), w1 = min(nw, w0 + wper);
+// Dynamic shared memory of a pick CTA: the bitmap of selected tokens, the
+// boundary bucket's keys and tokens, the tied tokens.
+constexpr size_t kSelDyn = (size_t)(kMaxT / 32) * 4 + (size_t)kCandCap * 8 + (size_t)kTieCap * 4;
+
+// kv_pick_kernel: every CTA finds the bucket of the k_tok-th largest key from
+// the head's complete histogram, writes its tokens' bitmap words (tokens of
+// higher buckets) and appends its boundary-bucket tokens to the head's
+// candidate list; the head's last CTA pins the k_tok-th key among the
+// candidates, marks them and the lowest tied tokens, and writes the selection
+// in ascending order.
+__global__ void __launch_bounds__(kSelThreads) kv_pick_kernel(SelArgs a) {
+  __shared__ SelShared sh;
+  extern __shared__ __align__(16) uint32_t dyn_sel[];
+  uint32_t* bits = dyn_sel;                                    // [kMaxT / 32]
+  uint32_t* ck = bits + kMaxT / 32;                            // [kCandCap] keys
+  int* ct = reinterpret_cast<int*>(ck + kCandCap);             // [kCandCap] tokens
+  int* tie_t = ct + kCandCap;                                  // [kTieCap]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.y, bat = blockIdx.z;
+  const long head = (long)bat * a.h_kv + g;
+  pdl_trigger();
+  pdl_wait();  // every score and the complete histogram
+  int* gh = a.ctl + head * kCtl;
   for (int i = tid; i < kBins1; i += kSelThreads) sh.hist[i] = __ldcg(gh + i);
-  if (tid == 0) sh.ncand = 0;
-  tie[tid] = 0;
+  if (tid < kSelTok / 32) sh.words[tid] = 0u;
   __syncthreads();
   int kneed;
   const uint32_t b1 = (uint32_t)find_bucket<kSelThreads>(sh.hist, kBins1, a.k_tok, sh.ws, sh.res, &kneed);
-  // one pass: higher buckets marked, the boundary bucket collected
-  for (int w = w0; w < w1; w++) {
-    uint32_t key[32];
-    if (32 * w + 32 <= T) {  // a whole word of scores: eight 16-byte loads
-#pragma unroll
-      for (int v = 0; v < 8; v++) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + 32 * w) + v);
-        key[4 * v] = __float_as_uint(f.x), key[4 * v + 1] = __float_as_uint(f.y);
-        key[4 * v + 2] = __float_as_uint(f.z), key[4 * v + 3] = __float_as_uint(f.w);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; i++) key[i] = 32 * w + i < T ? __float_as_uint(__ldcg(sc + 32 * w + i)) : 0u;
+  const int T = a.T;
+  const float* sc = a.scores + head * a.Tp;
+  uint2* cl = a.cand + head * kCandCap;
+  int* ncand_g = gh + kBins1 + 3;
+  {
+    // four consecutive tokens per thread
+    const int t0 = blockIdx.x * kSelTok + 4 * tid;
+    uint32_t key[4] = {0u, 0u, 0u, 0u};
+    if (t0 + 4 <= a.Tp) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + t0));
+      key[0] = __float_as_uint(f.x), key[1] = __float_as_uint(f.y);
+      key[2] = __float_as_uint(f.z), key[3] = __float_as_uint(f.w);
     }
     uint32_t m = 0;
+    int nc = 0;
 #pragma unroll
-    for (int i = 0; i < 32; i++) {
+    for (int i = 0; i < 4; i++) {
+      const bool in = t0 + i < T;
       const uint32_t d = key[i] >> 20;
-      if (32 * w + i < T && d > b1) m |= 1u << i;
-      if (32 * w + i < T && d == b1) {
-        const int slot = atomicAdd(&sh.ncand, 1);
-        if (slot < kCandCap) ck[slot] = key[i], ct[slot] = 32 * w + i;
-      }
+      if (in && d > b1) m |= 1u << i;
+      nc += in && d == b1;
     }
-    bits[w] = m;
+    if (m) atomicOr(&sh.words[(4 * tid) >> 5], m << ((4 * tid) & 31));
+    // boundary-bucket tokens into the head's list: one atomic per warp
+    int incl = nc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    int base = 0;
+    if (lane == 31 && incl) base = atomicAdd(ncand_g, incl);
+    base = __shfl_sync(0xffffffffu, base, 31) + incl - nc;
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+      if (t0 + i < T && (key[i] >> 20) == b1) {
+        if (base < kCandCap) cl[base] = make_uint2(key[i], (uint32_t)(t0 + i));
+        base++;
+      }
   }
   __syncthreads();
-  const int ncand = sh.ncand;
+  {
+    const int w0 = blockIdx.x * (kSelTok / 32), nw = (T + 31) / 32;
+    if (tid < kSelTok / 32 && w0 + tid < nw) a.bitmap[head * (a.Tp / 32) + w0 + tid] = sh.words[tid];
+  }
+  __threadfence();  // this CTA's words and candidates before its count
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(gh + kBins1 + 2, 1) == a.nblk - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();  // every other CTA's words and candidates are visible
+
+  // ---- the head's last CTA
+  const int nw = (T + 31) / 32;
+  const int wper = (nw + kSelThreads - 1) / kSelThreads;
+  const int w0 = min(nw, tid * wper), w1 = min(nw, w0 + wper);
+  for (int w = tid; w < nw; w += kSelThreads) bits[w] = __ldcg(a.bitmap + head * (a.Tp / 32) + w);
+  const int ncand = __ldcg(ncand_g);
   const bool in_smem = ncand <= kCandCap;
-  // the boundary bucket's keys: from shared memory, or (when too many) the scores again
+  if (in_smem)
+    for (int j = tid; j < ncand; j += kSelThreads) {
+      const uint2 e = __ldcg(cl + j);
+      ck[j] = e.x, ct[j] = (int)e.y;
+    }
+  __syncthreads();
+  // f(valid, key, token) on whole warps (lanes past the end pass valid = false)
   auto for_cands = [&](auto&& f) {
     if (in_smem) {
-      for (int j = tid; j < ncand; j += kSelThreads) f(ck[j], ct[j]);
+      for (int j0 = tid - lane; j0 < ncand; j0 += kSelThreads) {
+        const int j = j0 + lane;
+        const bool v = j < ncand;
+        f(v, v ? ck[j] : 0u, v ? ct[j] : 0);
+      }
     } else {
-      for (int t = tid; t < T; t += kSelThreads) {
-        const uint32_t key = __float_as_uint(__ldcg(sc + t));
-        if ((key >> 20) == b1) f(key, t);
+      for (int t0 = tid - lane; t0 < T; t0 += kSelThreads) {
+        const int t = t0 + lane;
+        const uint32_t key = t < T ? __float_as_uint(__ldcg(sc + t)) : 0u;
+        f(t < T && (key >> 20) == b1, key, t);
       }
     }
   };
@@ -751,9 +823,9 @@ __global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
   for (int shift = 10; shift >= 0; shift -= 10) {
     for (int i = tid; i < kBins2; i += kSelThreads) sh.hist[i] = 0;
     __syncthreads();
-    for_cands([&](uint32_t key, int t) {
+    for_cands([&](bool v, uint32_t key, int t) {
       (void)t;
-      if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & (kBins2 - 1)], 1);
+      hist_add(sh.hist, v && (key & mask) == prefix ? (int)((key >> shift) & (kBins2 - 1)) : -1);
     });
     __syncthreads();
     int kl;
@@ -762,23 +834,46 @@ __global__ void __launch_bounds__(kSelThreads) kv_select_kernel(SelArgs a) {
     prefix |= d << shift;
     mask |= (uint32_t)(kBins2 - 1) << shift;
   }
-  // prefix is the k_tok-th largest key K*; kneed of the keys equal to it are taken
-  const int tok_per = 32 * wper;
-  for_cands([&](uint32_t key, int t) {
-    if (key > prefix) atomicOr(&bits[t >> 5], 1u << (t & 31));
-    else if (key == prefix) atomicAdd(&tie[t / tok_per], 1);
+  // prefix is the k_tok-th largest key K*; kneed of the keys equal to it are
+  // taken, the lowest tokens first
+  if (tid == 0) sh.res[0] = 0;
+  __syncthreads();
+  for_cands([&](bool v, uint32_t key, int t) {
+    if (v && key > prefix) atomicOr(&bits[t >> 5], 1u << (t & 31));
+    const bool eq = v && key == prefix;
+    const unsigned m = __ballot_sync(0xffffffffu, eq);
+    if (m) {  // one atomic per warp
+      int base = 0;
+      if (lane == __ffs(m) - 1) base = atomicAdd(&sh.res[0], __popc(m));
+      base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+      const int slot = base + __popc(m & ((1u << lane) - 1u));
+      if (eq && slot < kTieCap) tie_t[slot] = t;
+    }
   });
   __syncthreads();
-  int ties_all;
-  const int ties_before = block_exclusive_sum<kSelThreads>(tie[tid], sh.ws, ties_all);
-  const int take = max(0, min(tie[tid], kneed - ties_before));
-  if (take > 0) {  // the first `take` of this thread's tied tokens, in token order
-    int taken = 0;
-    for (int w = w0; w < w1 && taken < take; w++) {
+  const int nties = sh.res[0];
+  if (nties <= kTieCap) {
+    // a tie is taken when fewer than kneed tied tokens lie below it
+    for (int i = tid; i < nties; i += kSelThreads) {
+      const int t = tie_t[i];
+      int below = 0;
+      for (int k2 = 0; k2 < nties; k2++) below += tie_t[k2] < t;
+      if (below < kneed) atomicOr(&bits[t >> 5], 1u << (t & 31));
+    }
+  } else {
+    // many equal keys: per-thread counts of its own tied tokens, then each
+    // thread marks the first ones of its range that the budget still allows
+    int mine = 0;
+    for (int w = w0; w < w1; w++)
+      for (int i = 32 * w; i < min(T, 32 * w + 32); i++) mine += __float_as_uint(__ldcg(sc + i)) == prefix;
+    int ties_all;
+    const int ties_before = block_exclusive_sum<kSelThreads>(mine, sh.ws, ties_all);
+    int take = max(0, min(mine, kneed - ties_before));
+    for (int w = w0; w < w1 && take > 0; w++) {
       uint32_t m = bits[w];
-      for (int i = 0; i < 32 && taken < take; i++) {
+      for (int i = 0; i < 32 && take > 0; i++) {
         const int t = 32 * w + i;
-        if (t < T && __float_as_uint(__ldcg(sc + t)) == prefix) m |= 1u << i, taken++;
+        if (t < T && __float_as_uint(__ldcg(sc + t)) == prefix) m |= 1u << i, take--;
       }
       bits[w] = m;
     }
@@ -810,6 +905,7 @@ struct RefArgs {
   const float* part;    // [batch][h_q][nrec][kRec]
   int nrec;
   int k_tok, parts;
+  int stats_given;      // the selection left (M, Z) in the control words
   const int32_t* sel;   // [batch][h_kv][k_tok]
   int* ctl;             // [batch][h_kv][kCtl]
   float* rpart;         // [batch][h_kv][parts][gq][kD + 1]
@@ -847,8 +943,212 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
   return r;
 }
 
-// GQP: query heads per KV head, padded to 4 or 8 (register arrays); B, R:
-// the cache's base and refinement bits.
+// Per-lane constants of the refinement: the lane owns head dims lane + 32 e
+// (scale group e): their word and bit in a token's key codes and refinements,
+// and the query values of the group's heads there.
+template <int GQP, int B, int R>
+struct RefLane {
+  int kw[4], kbit[4], krw[4], krbit[4];
+  float qv[GQP][4];
+  __device__ __forceinline__ void init(const RefArgs& a, long hq0, int lane) {
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      key_pos(lane + 32 * e, B, kw[e], kbit[e]);
+      key_pos(lane + 32 * e, R, krw[e], krbit[e]);
+#pragma unroll
+      for (int h = 0; h < GQP; h++) qv[h][e] = h < a.gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
+    }
+  }
+};
+
+// One warp swaps the base contributions of up to kRefTPW tokens (tok[m] < 0:
+// none) for their refined ones: adds v~ exp(l~ - M) - v^ exp(l^ - M) into
+// an[h][e] (head h, dim lane + 32 e) and exp(l~ - M) - exp(l^ - M) of the
+// lane's (token, head) slot into ad_own.  wtab: the warp's kRefTPW * GQP
+// float2 of shared memory.
+template <int GQP, int B, int R>
+__device__ __forceinline__ void refine_batch(const RefArgs& a, const RefLane<GQP, B, R>& rl, const float* M,
+                                             long slot0, long hq0, const int (&tok)[kRefTPW], int lane,
+                                             float (&an)[GQP][4], float& ad_own, float2* wtab) {
+  const float half = 0.5f * (float)(1 << R), inv = 1.0f / (float)(1 << R);
+  const uint32_t bmask = (1u << B) - 1u, rmask = (1u << R) - 1u;
+  const int u_own = lane % (kRefTPW * GQP), m_own = u_own / GQP, h_own = u_own % GQP;
+  // every load of the warp's tokens first
+  uint32_t wk[kRefTPW][4], wkr[kRefTPW][4], wv[kRefTPW][4], wvr[kRefTPW][4], zk[kRefTPW][4], zv[kRefTPW][4];
+#pragma unroll
+  for (int m = 0; m < kRefTPW; m++) {
+    const int t = tok[m] < 0 ? 0 : tok[m];
+    const long slot = slot0 + t, tile = slot / 16;
+    const uint32_t* kp = reinterpret_cast<const uint32_t*>(a.kb + slot * 16 * B);
+    const uint32_t* krp = reinterpret_cast<const uint32_t*>(a.kr + slot * 16 * R);
+    const uint32_t* vp = reinterpret_cast<const uint32_t*>(a.vb + tile * 256 * B);
+    const uint32_t* vrp = reinterpret_cast<const uint32_t*>(a.vr + tile * 256 * R);
+    const uint32_t* zkp = reinterpret_cast<const uint32_t*>(a.ksz) + slot * 4;
+    const uint32_t* zvp = reinterpret_cast<const uint32_t*>(a.vsz) + slot * 4;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const int d = lane + 32 * e;
+      int vw, vbit, vrw, vrbit;
+      value_pos(t & 15, d, B, vw, vbit);
+      value_pos(t & 15, d, R, vrw, vrbit);
+      wk[m][e] = (kp[rl.kw[e]] >> rl.kbit[e]) & bmask;
+      wkr[m][e] = (krp[rl.krw[e]] >> rl.krbit[e]) & rmask;
+      wv[m][e] = (vp[vw] >> vbit) & bmask;
+      wvr[m][e] = (vrp[vrw] >> vrbit) & rmask;
+      zk[m][e] = zkp[e];
+      zv[m][e] = zvp[e];
+    }
+  }
+  int tok_own = tok[0];
+#pragma unroll
+  for (int m = 1; m < kRefTPW; m++)
+    if (m == m_own) tok_own = tok[m];
+  float wbl = 0.f;
+  const bool own_ok = h_own < a.gq && tok_own >= 0;
+  if (own_ok) wbl = expf(a.logits[(hq0 + h_own) * a.T + tok_own] - M[h_own]);
+  float kf[kRefTPW][4], vbs[kRefTPW][4], vfs[kRefTPW][4];
+#pragma unroll
+  for (int m = 0; m < kRefTPW; m++) {
+    const bool ok = tok[m] >= 0;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&zk[m][e]));
+      const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv[m][e]));
+      kf[m][e] = fmaf(k2.x, (float)wk[m][e] + ((float)wkr[m][e] + 0.5f - half) * inv, k2.y);
+      vbs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e], v2.y) : 0.f;
+      vfs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e] + ((float)wvr[m][e] + 0.5f - half) * inv, v2.y) : 0.f;
+    }
+  }
+  // refined logits of the TPW x GQP (token, head) slots
+  float lg[kRefTPW * GQP];
+#pragma unroll
+  for (int m = 0; m < kRefTPW; m++)
+#pragma unroll
+    for (int h = 0; h < GQP; h++) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; e++) acc = fmaf(rl.qv[h][e], kf[m][e], acc);
+      lg[m * GQP + h] = acc;
+    }
+  const float lg_own = warp_transpose_sum<kRefTPW * GQP>(lg, lane);
+  float wfl = 0.f;
+  if (own_ok) wfl = expf(lg_own * a.scale - M[h_own]);
+  if (lane < kRefTPW * GQP) wtab[lane] = make_float2(wfl, wbl);
+  ad_own += wfl - wbl;
+  __syncwarp();
+#pragma unroll
+  for (int m = 0; m < kRefTPW; m++)
+#pragma unroll
+    for (int h = 0; h < GQP; h++) {
+      const float2 w = wtab[m * GQP + h];
+#pragma unroll
+      for (int e = 0; e < 4; e++) an[h][e] = fmaf(w.x, vfs[m][e], fmaf(-w.y, vbs[m][e], an[h][e]));
+    }
+  __syncwarp();
+}
+
+// The share s = part, part + parts, ... of the base pass's split records of
+// the group's heads, rescaled to M: num[(h, d)] for the (h, d) pairs e =
+// tid, tid + nthreads, ... (at most 4 per thread), every load issued first.
+template <int GQP>
+__device__ __forceinline__ void record_share(const RefArgs& a, long hq0, const float* M, int part, int parts,
+                                             int tid, int nthreads, float (&num)[4]) {
+  constexpr int PER = 8;
+#pragma unroll
+  for (int i = 0; i < 4; i++) num[i] = 0.f;
+  for (int s0 = part; s0 < a.nrec; s0 += parts * PER) {
+    float mv[4][PER], av[4][PER];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const int e = tid + i * nthreads, h = e / kD, d = e % kD;
+      const float* pr = a.part + (hq0 + (h < a.gq ? h : 0)) * a.nrec * kRec;
+#pragma unroll
+      for (int k = 0; k < PER; k++) {
+        const int sidx = s0 + parts * k;
+        const bool ok = e < a.gq * kD && sidx < a.nrec;
+        mv[i][k] = ok ? pr[(long)sidx * kRec + kD] : -INFINITY;
+        av[i][k] = ok ? pr[(long)sidx * kRec + d] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const int e = tid + i * nthreads, h = (e / kD) < a.gq ? e / kD : 0;
+#pragma unroll
+      for (int k = 0; k < PER; k++)
+        if (mv[i][k] > -INFINITY) num[i] = fmaf(expf(mv[i][k] - M[h]), av[i][k], num[i]);
+    }
+  }
+}
+
+// The head's output from every CTA's partial: out[h] = sum of the parts'
+// numerators (+ extra) / (Z + sum of their denominators (+ extra_den)).
+template <int NT>
+__device__ __forceinline__ void merge_parts(const RefArgs& a, long hq0, long head, const float* Z, int parts,
+                                            const float* extra_num, const float* extra_den) {
+  const int gq = a.gq;
+  const float* rh = a.rpart + head * a.parts * gq * (kD + 1);
+  for (int e = threadIdx.x; e < gq * kD; e += NT) {
+    const int h = e / kD, d = e % kD;
+    float nv[kRefPartsMax], dv[kRefPartsMax];  // every part's load in flight together
+    float num = extra_num ? extra_num[e] : 0.f, den = Z[h] + (extra_den ? extra_den[h] : 0.f);
+    for (int p0 = 0; p0 < parts; p0 += kRefPartsMax) {
+#pragma unroll
+      for (int k = 0; k < kRefPartsMax; k++) {
+        const int p = p0 + k;
+        nv[k] = p < parts ? __ldcg(rh + (p * gq + h) * (kD + 1) + d) : 0.f;
+        dv[k] = p < parts ? __ldcg(rh + (p * gq + h) * (kD + 1) + kD) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kRefPartsMax; k++) num += nv[k], den += dv[k];
+    }
+    const float o = num / den;
+    if (a.out) a.out[(hq0 + h) * kD + d] = o;
+    if (a.out16) a.out16[(hq0 + h) * kD + d] = __half_as_ushort(__float2half_rn(o));
+  }
+}
+
+// The CTA's partial (its warps' numerators in num_w [warps][GQP][kD], their
+// denominators in den_w [warps][GQP], plus its record share rec[i] for pairs
+// tid + i NT) into the head's slot `part` of the workspace.
+template <int GQP, int NT>
+__device__ __forceinline__ void write_part(const RefArgs& a, long head, int part, const float* num_w,
+                                           const float* den_w, const float (&rec)[4]) {
+  constexpr int NW = NT / 32;
+  float* rp = a.rpart + (head * a.parts + part) * a.gq * (kD + 1);
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const int e = threadIdx.x + i * NT;
+    if (e < a.gq * kD) {
+      const int h = e / kD, d = e % kD;
+      float num = rec[i];
+      for (int w = 0; w < NW; w++) num += num_w[(w * GQP + h) * kD + d];
+      rp[h * (kD + 1) + d] = num;
+    }
+  }
+  if ((int)threadIdx.x < a.gq) {
+    float den = 0.f;
+    for (int w = 0; w < NW; w++) den += den_w[w * GQP + threadIdx.x];
+    rp[threadIdx.x * (kD + 1) + kD] = den;
+  }
+}
+
+// A warp's numerators and denominator changes into shared memory.
+template <int GQP>
+__device__ __forceinline__ void stash_warp(float (&an)[GQP][4], float ad_own, int warp, int lane, float* num_w,
+                                           float* den_w) {
+#pragma unroll
+  for (int h = 0; h < GQP; h++)
+#pragma unroll
+    for (int e = 0; e < 4; e++) num_w[(warp * GQP + h) * kD + lane + 32 * e] = an[h][e];
+  // slot u's denominator change sits in lanes u, u + TPW GQP, ...: sum each head's
+  float dsum = lane < kRefTPW * GQP ? ad_own : 0.f;
+#pragma unroll
+  for (int o = GQP; o < 32; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  if (lane < GQP) den_w[warp * GQP + lane] = dsum;
+}
+
+// kv_refine_kernel (a selection given): kRefParts CTAs per head, each a share
+// of the selected tokens and of the split records; the head's last CTA merges.
 template <int GQP, int B, int R>
 __global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
   __shared__ RefShared<GQP> sh;
@@ -857,172 +1157,46 @@ __global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
-  pdl_wait();  // the base pass and the selection are complete
+  pdl_wait();  // the base pass is complete
   if (warp < gq) {
     float M, Z;
     head_stats(a.part + (hq0 + warp) * a.nrec * kRec, a.nrec, kRec, lane, M, Z);
     if (lane == 0) sh.M[warp] = M, sh.Z[warp] = Z;
   }
   __syncthreads();
-
-  // ---- the refined contribution of this CTA's share of the selected tokens
   const int ja = (int)((long)part * a.k_tok / a.parts), jb = (int)((long)(part + 1) * a.k_tok / a.parts);
-  const float half = 0.5f * (float)(1 << R), inv = 1.0f / (float)(1 << R);
-  const uint32_t bmask = (1u << B) - 1u, rmask = (1u << R) - 1u;
   const long slot0 = head * a.t_max;
-  int kw[4], kbit[4], krw[4], krbit[4];
-  float qv[GQP][4];
-#pragma unroll
-  for (int e = 0; e < 4; e++) {
-    key_pos(lane + 32 * e, B, kw[e], kbit[e]);
-    key_pos(lane + 32 * e, R, krw[e], krbit[e]);
-#pragma unroll
-    for (int h = 0; h < GQP; h++) qv[h][e] = h < gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
-  }
+  RefLane<GQP, B, R> rl;
+  rl.init(a, hq0, lane);
+  float rec[4];
+  record_share<GQP>(a, hq0, sh.M, part, a.parts, tid, kRefThreads, rec);
   float an[GQP][4], ad_own = 0.f;
 #pragma unroll
   for (int h = 0; h < GQP; h++)
 #pragma unroll
     for (int e = 0; e < 4; e++) an[h][e] = 0.f;
   const int32_t* selg = a.sel + head * a.k_tok;
-  // lane L ends the transposed reduction holding slot u = L % (TPW GQP):
-  // token m_own = u / GQP of the warp's batch, head h_own = u % GQP
-  const int u_own = lane % (kRefTPW * GQP), m_own = u_own / GQP, h_own = u_own % GQP;
   for (int j0 = ja + warp * kRefTPW; j0 < jb; j0 += kRefWarps * kRefTPW) {
     int tok[kRefTPW];
 #pragma unroll
     for (int m = 0; m < kRefTPW; m++) {
       const int j = j0 + m;
-      int t = j < jb ? selg[j] : -1;
+      const int t = j < jb ? selg[j] : -1;
       tok[m] = (t >= 0 && t < a.T) ? t : -1;  // a foreign index is skipped, never dereferenced
     }
-    // every load of the warp's tokens first
-    uint32_t wk[kRefTPW][4], wkr[kRefTPW][4], wv[kRefTPW][4], wvr[kRefTPW][4], zk[kRefTPW][4], zv[kRefTPW][4];
-#pragma unroll
-    for (int m = 0; m < kRefTPW; m++) {
-      const int t = tok[m] < 0 ? 0 : tok[m];
-      const long slot = slot0 + t, tile = slot / 16;
-      const uint32_t* kp = reinterpret_cast<const uint32_t*>(a.kb + slot * 16 * B);
-      const uint32_t* krp = reinterpret_cast<const uint32_t*>(a.kr + slot * 16 * R);
-      const uint32_t* vp = reinterpret_cast<const uint32_t*>(a.vb + tile * 256 * B);
-      const uint32_t* vrp = reinterpret_cast<const uint32_t*>(a.vr + tile * 256 * R);
-      const uint32_t* zkp = reinterpret_cast<const uint32_t*>(a.ksz) + slot * 4;
-      const uint32_t* zvp = reinterpret_cast<const uint32_t*>(a.vsz) + slot * 4;
-#pragma unroll
-      for (int e = 0; e < 4; e++) {
-        const int d = lane + 32 * e;
-        int vw, vbit, vrw, vrbit;
-        value_pos(t & 15, d, B, vw, vbit);
-        value_pos(t & 15, d, R, vrw, vrbit);
-        wk[m][e] = (kp[kw[e]] >> kbit[e]) & bmask;
-        wkr[m][e] = (krp[krw[e]] >> krbit[e]) & rmask;
-        wv[m][e] = (vp[vw] >> vbit) & bmask;
-        wvr[m][e] = (vrp[vrw] >> vrbit) & rmask;
-        zk[m][e] = zkp[e];
-        zv[m][e] = zvp[e];
-      }
-    }
-    float wbl = 0.f;
-    const bool own_ok = h_own < gq && tok[m_own] >= 0;
-    if (own_ok) wbl = expf(a.logits[(hq0 + h_own) * a.T + tok[m_own]] - sh.M[h_own]);
-    float kf[kRefTPW][4], vbs[kRefTPW][4], vfs[kRefTPW][4];
-#pragma unroll
-    for (int m = 0; m < kRefTPW; m++) {
-      const bool ok = tok[m] >= 0;
-#pragma unroll
-      for (int e = 0; e < 4; e++) {
-        const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(&zk[m][e]));
-        const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(&zv[m][e]));
-        kf[m][e] = fmaf(k2.x, (float)wk[m][e] + ((float)wkr[m][e] + 0.5f - half) * inv, k2.y);
-        vbs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e], v2.y) : 0.f;
-        vfs[m][e] = ok ? fmaf(v2.x, (float)wv[m][e] + ((float)wvr[m][e] + 0.5f - half) * inv, v2.y) : 0.f;
-      }
-    }
-    // refined logits of the TPW x GQP (token, head) slots
-    float lg[kRefTPW * GQP];
-#pragma unroll
-    for (int m = 0; m < kRefTPW; m++)
-#pragma unroll
-      for (int h = 0; h < GQP; h++) {
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; e++) acc = fmaf(qv[h][e], kf[m][e], acc);
-        lg[m * GQP + h] = acc;
-      }
-    const float lg_own = warp_transpose_sum<kRefTPW * GQP>(lg, lane);
-    float wfl = 0.f;
-    if (own_ok) wfl = expf(lg_own * a.scale - sh.M[h_own]);
-    if (lane < kRefTPW * GQP) sh.wtab[warp][lane] = make_float2(wfl, wbl);
-    ad_own += wfl - wbl;
-    __syncwarp();
-#pragma unroll
-    for (int m = 0; m < kRefTPW; m++)
-#pragma unroll
-      for (int h = 0; h < GQP; h++) {
-        const float2 w = sh.wtab[warp][m * GQP + h];
-#pragma unroll
-        for (int e = 0; e < 4; e++) an[h][e] = fmaf(w.x, vfs[m][e], fmaf(-w.y, vbs[m][e], an[h][e]));
-      }
-    __syncwarp();
+    refine_batch<GQP, B, R>(a, rl, sh.M, slot0, hq0, tok, lane, an, ad_own, &sh.wtab[warp][0]);
   }
-#pragma unroll
-  for (int h = 0; h < GQP; h++)
-#pragma unroll
-    for (int e = 0; e < 4; e++) sh.num[warp][h][lane + 32 * e] = an[h][e];
-  // slot u's denominator change sits in lanes u, u + TPW GQP, ...: sum each head's
-  float dsum = lane < kRefTPW * GQP ? ad_own : 0.f;
-#pragma unroll
-  for (int o = GQP; o < 32; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-  if (lane < GQP) sh.den[warp][lane] = dsum;
+  stash_warp<GQP>(an, ad_own, warp, lane, &sh.num[0][0][0], &sh.den[0][0]);
   __syncthreads();
-
-  // ---- this CTA's share of the base records (s = part, part + parts, ...), rescaled to M
-  float* rp = a.rpart + (head * a.parts + part) * gq * (kD + 1);
-  for (int e = tid; e < gq * kD; e += kRefThreads) {
-    const int h = e / kD, d = e % kD;
-    const float* pr = a.part + (hq0 + h) * a.nrec * kRec;
-    float num = 0.f;
-    for (int w = 0; w < kRefWarps; w++) num += sh.num[w][h][d];
-    constexpr int PER = 4;
-    for (int s0 = part; s0 < a.nrec; s0 += a.parts * PER) {
-      float mv[PER], av[PER];
-#pragma unroll
-      for (int k = 0; k < PER; k++) {
-        const int s = s0 + a.parts * k;
-        mv[k] = s < a.nrec ? pr[(long)s * kRec + kD] : -INFINITY;
-        av[k] = s < a.nrec ? pr[(long)s * kRec + d] : 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < PER; k++)
-        if (mv[k] > -INFINITY) num = fmaf(expf(mv[k] - sh.M[h]), av[k], num);
-    }
-    rp[h * (kD + 1) + d] = num;
-  }
-  if (tid < gq) {
-    float den = 0.f;
-    for (int w = 0; w < kRefWarps; w++) den += sh.den[w][tid];
-    rp[tid * (kD + 1) + kD] = den;
-  }
+  write_part<GQP, kRefThreads>(a, head, part, &sh.num[0][0][0], &sh.den[0][0], rec);
   __threadfence();  // this CTA's partial before its count
   __syncthreads();
   if (tid == 0) sh.last = atomicAdd(a.ctl + head * kCtl + kBins1 + 1, 1) == a.parts - 1;
   __syncthreads();
   if (!sh.last) return;
   __threadfence();  // every other CTA's partial is visible
-  const float* rh = a.rpart + head * a.parts * gq * (kD + 1);
-  for (int e = tid; e < gq * kD; e += kRefThreads) {
-    const int h = e / kD, d = e % kD;
-    float num = 0.f, den = sh.Z[h];
-    for (int p = 0; p < a.parts; p++) {
-      num += __ldcg(rh + (p * gq + h) * (kD + 1) + d);
-      den += __ldcg(rh + (p * gq + h) * (kD + 1) + kD);
-    }
-    const float o = num / den;
-    if (a.out) a.out[(hq0 + h) * kD + d] = o;
-    if (a.out16) a.out16[(hq0 + h) * kD + d] = __half_as_ushort(__float2half_rn(o));
-  }
+  merge_parts<kRefThreads>(a, hq0, head, sh.Z, a.parts, nullptr, nullptr);
 }
-
 
 // ---------------------------------------------------------------------------
 // host side
@@ -1030,7 +1204,7 @@ __global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
 struct Plan {
   int nsplit, span, nrec;  // base pass (warp splits; one record per CTA of kWarps splits)
   int Tp, sel_blocks, parts;
-  size_t off_logits, off_part, off_scores, off_ctl, off_rpart, total;
+  size_t off_logits, off_part, off_scores, off_bitmap, off_cand, off_ctl, off_rpart, total;
 };
 
 // The workspace: [logits] [records] [scores, Tp-pitched] [control words] [refinement partials].
@@ -1048,7 +1222,10 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   P.nrec = (P.nsplit + kWarps - 1) / kWarps;
   P.Tp = (t + 31) / 32 * 32;
   P.sel_blocks = (t + kSelTok - 1) / kSelTok;
-  P.parts = std::max(1, std::min(kRefPartsMax, (k_tok + kRefWarps * kRefTPW - 1) / (kRefWarps * kRefTPW)));
+  // refinement CTAs per head: enough for the selected tokens and for the
+  // split records (a few per CTA: each CTA's record loads are in flight together)
+  P.parts = std::max(1, std::min(kRefPartsMax, std::max((k_tok + kRefWarps * kRefTPW - 1) / (kRefWarps * kRefTPW),
+                                                        (P.nrec + 7) / 8)));
   const int gq = h_q / kv->h_kv;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -1060,6 +1237,8 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   P.off_logits = need_logits ? take((size_t)kv->batch * h_q * t * 4) : 0;
   P.off_part = take((size_t)kv->batch * h_q * P.nrec * rec * 4);
   P.off_scores = select ? take((size_t)heads * P.Tp * 4) : 0;
+  P.off_bitmap = select ? take((size_t)heads * (P.Tp / 32) * 4) : 0;
+  P.off_cand = select ? take((size_t)heads * kCandCap * 8) : 0;
   P.off_ctl = take((size_t)heads * kCtl * 4);
   P.off_rpart = refine ? take((size_t)heads * P.parts * gq * (kD + 1) * 4) : 0;
   P.total = off;
@@ -1117,26 +1296,28 @@ BaseArgs base_args(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* lo
   return a;
 }
 
-// Scoring and selection after the base pass (programmatic serialization: its
-// CTAs start while the base pass drains).
+// Scoring, then selection, after the base pass (programmatic serialization:
+// the CTAs of each start while the kernel before it drains).
 sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& P, const float* logits,
-                        const float* part, int rec, float* scores_ws, float* scores_out, int* ctl, int32_t* sel,
+                        const float* part, int rec, char* ws, float* scores_out, int* ctl, int32_t* sel,
                         cudaStream_t s) {
   SelArgs a;
   a.logits = logits, a.part = part, a.nrec = P.nrec, a.rec = rec;
   a.h_kv = kv->h_kv, a.h_q = h_q, a.gq = h_q / kv->h_kv, a.T = t, a.Tp = P.Tp, a.k_tok = k_tok;
   a.nblk = P.sel_blocks;
-  a.scores = scores_ws, a.scores_out = scores_out, a.ctl = ctl, a.sel = sel;
-  void (*kern)(SelArgs) = a.gq <= 4 ? kv_select_kernel<4> : kv_select_kernel<8>;
-  SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDyn));
-  SF_CUDA(launch_pdl(kern, dim3(P.sel_blocks, kv->h_kv, kv->batch), dim3(kSelThreads), kSelDyn, s, a));
+  a.scores = (float*)(ws + P.off_scores), a.scores_out = scores_out, a.ctl = ctl, a.sel = sel;
+  a.bitmap = (uint32_t*)(ws + P.off_bitmap), a.cand = (uint2*)(ws + P.off_cand);
+  const dim3 grid(P.sel_blocks, kv->h_kv, kv->batch);
+  SF_CUDA(launch_pdl(a.gq <= 4 ? kv_score_kernel<4> : kv_score_kernel<8>, grid, dim3(kSelThreads), 0, s, a));
+  SF_CUDA(cudaFuncSetAttribute(kv_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDyn));
+  SF_CUDA(launch_pdl(kv_pick_kernel, grid, dim3(kSelThreads), kSelDyn, s, a));
   return SF_OK;
 }
 
 // Refinement of the selected tokens and the merge (programmatic serialization).
 sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
                         const float* logits, const float* part, const int32_t* sel, int* ctl, float* rpart,
-                        float* out, uint16_t* out16, cudaStream_t s) {
+                        float* out, uint16_t* out16, int stats_given, cudaStream_t s) {
   RefArgs a;
   a.kb = (const uint8_t*)kv->kb, a.kr = (const uint8_t*)kv->kr;
   a.vb = (const uint8_t*)kv->vb, a.vr = (const uint8_t*)kv->vr;
@@ -1145,6 +1326,7 @@ sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int 
   a.q = q, a.h_q = h_q, a.gq = h_q / kv->h_kv;
   a.logits = logits, a.part = part, a.nrec = P.nrec;
   a.k_tok = k_tok, a.parts = P.parts, a.sel = sel, a.ctl = ctl, a.rpart = rpart;
+  a.stats_given = stats_given;
   a.out = out, a.out16 = out16;
   a.scale = 1.0f / sqrtf((float)kD);
   void (*kern)(RefArgs);
@@ -1201,7 +1383,7 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, false, s);
   if (st != SF_OK) return st;
-  return launch_select(kv, t, h_q, k_tok, P, lg, part, 2, (float*)(w + P.off_scores), scores, ctl, sel, s);
+  return launch_select(kv, t, h_q, k_tok, P, lg, part, 2, w, scores, ctl, sel, s);
 }
 
 extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,
@@ -1233,7 +1415,7 @@ extern "C" sf_status sf_kv_attn_refined(const sf_kv* kv, int t, const uint16_t* 
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, nullptr, s);
+  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, nullptr, 0, s);
 }
 
 extern "C" size_t sf_kv_attend_selective_workspace_bytes(const sf_kv* kv, int t, int h_q,
@@ -1269,9 +1451,9 @@ sf_status attend_selective(const sf_kv* kv, int t, const uint16_t* q, int h_q, i
   BaseArgs a = base_args(kv, t, q, h_q, lg, part, ctl, P);
   st = launch_base(kv, a, true, s);
   if (st != SF_OK) return st;
-  st = launch_select(kv, t, h_q, k_tok, P, lg, part, kRec, (float*)(w + P.off_scores), nullptr, ctl, sel, s);
+  st = launch_select(kv, t, h_q, k_tok, P, lg, part, kRec, w, nullptr, ctl, sel, s);
   if (st != SF_OK) return st;
-  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, out16, s);
+  return launch_refine(kv, t, q, h_q, k_tok, P, lg, part, sel, ctl, (float*)(w + P.off_rpart), out, out16, 1, s);
 }
 
 }  // namespace
