@@ -19,59 +19,49 @@
 //
 // One CTA per SM owns a contiguous range of rows (a multiple of 4).
 //
-// Producer warp: one lane streams the CTA's codes through a ring of shared
-// memory stages with 1-D bulk copies (cp.async.bulk, completion counted on an
-// mbarrier per stage), and copies the rows' (s, m) words once.  The weights do
-// not depend on earlier kernels, so these copies start before the grid
-// dependency wait and overlap the previous kernel's tail.
+// Producer warp: streams the CTA's codes through a ring of shared memory
+// stages of 16-row blocks with 1-D bulk copies (cp.async.bulk; completion
+// counted on an mbarrier per stage; one copy per stage and plane), and copies
+// the rows' (s, m) words once.  The packed rows are stored with their 16-byte
+// units permuted by row mod 8 (wqlayout.cuh), so the eight rows a quad-lane
+// load touches fall in distinct banks.  The weights do not depend on earlier
+// kernels, so these copies start before the grid dependency wait and overlap
+// the previous kernel's tail.
 //
-// Compute warps: after the grid dependency wait they build the correction
-// tables (selected channel, x_c, group; the refinement words of the CTA's rows
-// copied with cp.async) and the activation planes (four threads per 64-channel
-// block) together.  Warp w owns the 2,048-channel segment w % segs (lane L: 64
-// consecutive channels) for every row whose index in its stage is congruent to
-// w / segs.  Its activations are turned once into fixed point
-// x = x_fix * 2^e per 64-channel lane block (e from the block's largest |x|,
-// |x_fix| < 2^20: every value within 2^9 of the block's largest is exact, the
-// rest round to 2^-20 of it) held as three byte planes in registers, in the
-// order of the code byte vectors: a 32-bit word of
-// 2-bit codes gives four byte vectors with one AND each (the codes at bit
-// offsets 2 and 6 of a byte carry a factor 4 that is folded into the scale),
-// dp4a takes four code x byte products per instruction, and the planes are
-// combined in 32-bit integers: the lane's partial dot product over its block is
-// exact for its fixed-point x.  Per row: s * 2^e * dot + m * sum(x), summed over
-// the warp with a transposed butterfly into a per-(row, segment) slot.
+// Compute warps: the inner sums run on the tensor cores as integer products,
+// mma.sync m16n8k32 with s8 operands and s32 accumulation: A = 16 rows x 32
+// channels of codes (byte vectors cut from the packed words with one AND,
+// or a shift and an AND), B = the activations of the same channels in fixed
+// point, one balanced byte digit per column (x_fix = d0 + 2^8 d1 + 2^16 d2,
+// x = x_fix * 2^(e - 19) per scale group, e from the group's largest |x|:
+// every value within 2^9 of the group's largest is exact, the rest round to
+// 2^-20 of it).  A k-step's 32 channels all lie in one scale group, so each
+// group's dot product per row and digit is exact in the s32 accumulator; the
+// digits are combined in fp32 and the group scaled once: s * 2^(e-19) * dot
+// + m * sum(x).  Work items are (16-row block, range of groups) of a stage;
+// their partial sums go to per-(row, range) slots.
 //
 // Correction (after the base pass, all threads): a thread owns 4 consecutive
 // rows (the r bits of 4 rows never straddle a 32-bit word) and a share of the
 // selected channels; per channel it reads one refinement word and adds
 // x_c * (1 + rho/2^r) to a per-row run, and every run of channels in one scale
 // group is scaled once, s * (run - sum x_c (1 - off/2^r)) with
-// off = 1/2 - 2^(r-1).  The base pass leaves the scales group-major for it.
-// Every partial has its own slot, so the sums are deterministic.
+// off = 1/2 - 2^(r-1).  Every partial has its own slot, so the sums are
+// deterministic.
 #include "common.cuh"
 #include "internal.cuh"
+#include "wqlayout.cuh"
 
 #include <algorithm>
 
 namespace sf {
 namespace {
 
-constexpr int kLaneCh = 64;                 // input channels per lane
-constexpr int kSegCh = 32 * kLaneCh;        // channels per warp segment
-constexpr int kMaxSegs = 16;                // k <= 32,768
-constexpr int kMaxWarps = 15;               // compute warps per CTA (plus the producer: 16 warps)
-#ifndef SF_GEMV_PLANES
-#define SF_GEMV_PLANES 3
-#endif
-constexpr int kXP = SF_GEMV_PLANES;         // byte planes of the fixed-point activations (2 or 3)
-constexpr int kXW = 16 * kXP + 4;           // shared words per lane block: planes, sum0, sum1, scale, pad
-// x_fix = x * 2^(kXE - ilogb(max |x| of the block)): |x_fix| < 2^(kXE + 1), so
-// 4 * sum code * x_fix over 64 channels fits an int32 for every base width
-constexpr int kXE = kXP == 2 ? 14 : 19;
+constexpr int kMaxWarps = 24;               // compute warps per CTA (plus the producer: 25 warps)
+constexpr int kXE = 19;                     // |x_fix| < 2^(kXE + 1): three byte digits
 constexpr int kRowUnit = 4;                 // CTA row ranges start at multiples of 4
 constexpr size_t kSmemLimit = 227 * 1024;   // dynamic shared memory of one CTA
-constexpr size_t kStageTarget = 36 * 1024;  // bytes of codes per ring stage, at most
+constexpr size_t kStageMax = 56 * 1024;     // bytes of codes per ring stage, at most (above: one row block)
 constexpr int kMaxStages = 6;
 constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
 
@@ -88,12 +78,12 @@ struct GemvArgs {
   float* y_corr;            // non-null: the correction goes here, y gets the base product
   size_t hi_off;
   int N, K, gpr, gshift, r, n_sel;
-  int segs, R, W;           // segments, warps per segment, compute warps (segs * R)
-  int rc, stages;           // rows per stage (R * RPW), ring depth
+  int nseg, nblk, rb, W;    // group ranges, blocks of max(G, 64) channels, row blocks per stage, compute warps
+  int rc, stages;           // rows per stage (16 rb), ring depth
   int rowL, rowH;           // bytes per row of plane L (all codes for b = 2, 4) and of plane H
   int stage_bytes;
   int row_words, staged, rows_max;
-  int off_ring, off_sz, off_x, off_part, off_szt, off_jd, off_wt, off_cpart;  // shared memory offsets
+  int off_ring, off_szt, off_xb, off_gt, off_part, off_jd, off_jrow, off_wt, off_cpart;  // shared memory offsets
   int szt_pitch, wt_pitch, cparts;
 };
 
@@ -156,227 +146,352 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t dp4a_us(uint32_t a, uint32_t b, uint32_t c) {
-  int32_t d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"((int32_t)c));
-  return (uint32_t)d;
-}
-
 // ---- activations -------------------------------------------------------------
 
-// Byte L of code vector v of a lane's 64 channels holds the code of channel
-// chan_of(v, L) (local to the lane block).
-template <int BITS>
-__host__ __device__ __forceinline__ int chan_of(int v, int L) {
-  if (BITS == 4) return 8 * (v >> 1) + (v & 1) + 2 * L;
-  return 16 * (v >> 2) + (v & 3) + 4 * L;
-}
-
-// A quarter of lane block b of x (64 channels) as fixed point, by the four
-// consecutive lanes of a quad (quarter q = lane & 3: channels 16q .. 16q + 15,
-// which are exactly the channels of code vectors 4q .. 4q + 3).  The block's
-// exponent comes from the quad's largest |x|; dst = the block's shared words:
-// planes[kXP * v + p] = byte p of x_fix for the four channels of vector v,
-// then the sum of channels 0-31, of 32-63 and the factor that turns the
-// integer dot product back into x units (2^e, divided by 4 where the byte
-// vectors carry the factor 4).  Whole warps (valid = false: the lane computes
-// nothing but takes part in the shuffles).
-template <int BITS>
-__device__ __forceinline__ void quarter_planes(bool valid, const uint16_t* __restrict__ xq, int q,
-                                               uint32_t* __restrict__ dst) {
-  uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-  if (valid) {
-    const uint4 a0 = reinterpret_cast<const uint4*>(xq)[0], a1 = reinterpret_cast<const uint4*>(xq)[1];
+// The activations of one batch row as the B operand of mma.m16n8k32 (s8).
+// Per scale group, x = x_fix * 2^(e - kXE) with e = ilogb(max |x| of the
+// group) and |x_fix| < 2^(kXE + 1); x_fix is split into balanced byte digits
+// x_fix = d0 + 2^8 d1 + 2^16 d2 (d0, d1 in [-128, 127], |d2| <= 16), one
+// digit plane per B column.  Unit u = 4 s + t (s: 64-channel block, t: quad
+// lane) holds 16 channels; for each plane one uint4 of byte vectors in the
+// order the main loop's A fragments take the codes:
+//   b = 2, 3: word k, byte L <- channel 64 s + 16 t + 4 L + {0, 2, 1, 3}[k]
+//             (the code byte vectors w & 0x03.., (w >> 4) & 0x03.. (set 0),
+//             w & 0x0C.., (w >> 4) & 0x0C.. (set 1, codes times 4) of the
+//             lane's 2-bit word 4 s + t);
+//   b = 4:    word k, byte L <- channel 64 s + 32 (k >> 1) + 8 t + 2 L + (k & 1)
+//             (the nibble vectors of the lane's words 8 s + t and 8 s + 4 + t).
+// Stored at xb[(s * 4 + p) * 4 + t] (p: plane; slot 3 is not used), so the
+// eight lanes of each quarter-warp read 128 consecutive bytes.  gt[g] =
+// (2^(e - kXE) / 4 (b = 2, 3) or 2^(e - kXE) (b = 4), sum of x over group g).
+// SPLIT (b = 4 with 32-channel groups): the unit's two halves lie in two
+// groups.  rw: units per group (SPLIT: 4, the units of one block).
+template <int BITS, bool SPLIT>
+__device__ __forceinline__ void build_unit(const uint16_t* __restrict__ x, int u, int rw, int gshift,
+                                           uint4* __restrict__ xb, float2* __restrict__ gt) {
+  const int s = u >> 2, t = u & 3;
+  uint32_t h[8];
+  {
+    const uint16_t* p0 = BITS == 4 ? x + 64 * s + 8 * t : x + 16 * u;
+    const uint16_t* p1 = BITS == 4 ? p0 + 32 : p0 + 8;
+    const uint4 a0 = *reinterpret_cast<const uint4*>(p0), a1 = *reinterpret_cast<const uint4*>(p1);
     h[0] = a0.x, h[1] = a0.y, h[2] = a0.z, h[3] = a0.w, h[4] = a1.x, h[5] = a1.y, h[6] = a1.z, h[7] = a1.w;
   }
-  uint32_t mx2 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; i++) mx2 = __vmaxu2(mx2, h[i] & 0x7fff7fffu);
-  uint32_t mx = max(mx2 & 0xffffu, mx2 >> 16);
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  float sq = 0.f;
+  // the largest |x| (fp16 bits order like magnitudes) and the sum, per half
+  uint32_t m2[2] = {0u, 0u};
+  float sm[2] = {0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 8; i++) {
+    m2[i >> 2] = __vmaxu2(m2[i >> 2], h[i] & 0x7fff7fffu);
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    sq += f.x, sq += f.y;
+    sm[i >> 2] += f.x + f.y;
   }
-  const float sh = sq + __shfl_xor_sync(0xffffffffu, sq, 1);  // quarters 0+1 or 2+3
-  const float so = __shfl_xor_sync(0xffffffffu, sh, 2);       // the other half
-  // x_fix = x * 2^(kXE - ilogb(max |x|)): the largest values are fp16
-  // mantissas times 2^(kXE - 10) (exact), smaller ones round to that step
-  const int eb = mx ? ((__float_as_int(h2f((uint16_t)mx)) >> 23) & 0xff) - 127 : 0;  // ilogb(max |x|)
-  const float scale = mx ? __int_as_float((127 + kXE - eb) << 23) : 0.f;
-  if (!valid) return;
-  int qv[16];
+  uint32_t mx[2] = {max(m2[0] & 0xffffu, m2[0] >> 16), max(m2[1] & 0xffffu, m2[1] >> 16)};
+  if (!SPLIT) mx[0] = mx[1] = max(mx[0], mx[1]), sm[0] += sm[1];
+  for (int o = 1; o < rw; o <<= 1) {
 #pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    // round to nearest even through the float mantissa: 1.5 * 2^23 + x_fix
-    qv[2 * i] = __float_as_int(fmaf(f.x, scale, 12582912.0f)) - 0x4B400000;
-    qv[2 * i + 1] = __float_as_int(fmaf(f.y, scale, 12582912.0f)) - 0x4B400000;
-  }
-#pragma unroll
-  for (int vv = 0; vv < 4; vv++) {
-    const int v = 4 * q + vv;
-    const int a = qv[chan_of<BITS>(vv, 0) & 15], b = qv[chan_of<BITS>(vv, 1) & 15];
-    const int c = qv[chan_of<BITS>(vv, 2) & 15], d = qv[chan_of<BITS>(vv, 3) & 15];
-#pragma unroll
-    for (int p = 0; p < kXP; p++) {
-      const uint32_t sel = (uint32_t)p | ((uint32_t)(4 + p) << 4);
-      const uint32_t t01 = __byte_perm((uint32_t)a, (uint32_t)b, sel);
-      const uint32_t t23 = __byte_perm((uint32_t)c, (uint32_t)d, sel);
-      dst[kXP * v + p] = __byte_perm(t01, t23, 0x5410);
+    for (int hh = 0; hh < 2; hh++) {
+      mx[hh] = max(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], o));
+      sm[hh] += __shfl_xor_sync(0xffffffffu, sm[hh], o);
     }
   }
-  if (q == 0) {
-    float* f = reinterpret_cast<float*>(dst + 16 * kXP);
-    f[0] = sh;
-    f[1] = so;
-    f[2] = mx ? __int_as_float((127 + eb - kXE - (BITS == 4 ? 0 : 2)) << 23) : 1.0f;
-    f[3] = 0.f;
+  float scale[2], fac[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; hh++) {
+    const int eb = mx[hh] ? ((__float_as_int(h2f((uint16_t)mx[hh])) >> 23) & 0xff) - 127 : 0;  // ilogb
+    scale[hh] = mx[hh] ? __int_as_float((127 + kXE - eb) << 23) : 0.f;
+    fac[hh] = mx[hh] ? __int_as_float((127 + eb - kXE - (BITS == 4 ? 0 : 2)) << 23) : 1.f;
+  }
+  // x_fix of the 16 channels in load order (c = 0..15; b = 4: halves of 8)
+  int q[16];
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    const float sc = scale[BITS == 4 ? (i >> 2) : 0];
+    // round to nearest even through the float mantissa: 1.5 * 2^23 + x_fix
+    q[2 * i] = __float_as_int(fmaf(f.x, sc, 12582912.0f)) - 0x4B400000;
+    q[2 * i + 1] = __float_as_int(fmaf(f.y, sc, 12582912.0f)) - 0x4B400000;
+  }
+  uint32_t wd[3][4];
+#pragma unroll
+  for (int k = 0; k < 4; k++) {
+    uint32_t acc[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int L = 0; L < 4; L++) {
+      constexpr int perm[4] = {0, 2, 1, 3};
+      const int c = BITS == 4 ? 8 * (k >> 1) + 2 * L + (k & 1) : 4 * L + perm[k];
+      const int v = q[c];
+      const int d0 = ((v + 128) & 255) - 128;
+      const int v1 = (v - d0) >> 8;
+      const int d1 = ((v1 + 128) & 255) - 128;
+      const int d2 = (v1 - d1) >> 8;
+      acc[0] |= (uint32_t)(d0 & 255) << (8 * L);
+      acc[1] |= (uint32_t)(d1 & 255) << (8 * L);
+      acc[2] |= (uint32_t)(d2 & 255) << (8 * L);
+    }
+#pragma unroll
+    for (int p = 0; p < 3; p++) wd[p][k] = acc[p];
+  }
+#pragma unroll
+  for (int p = 0; p < 3; p++) xb[(s * 4 + p) * 4 + t] = make_uint4(wd[p][0], wd[p][1], wd[p][2], wd[p][3]);
+  if (SPLIT) {
+    if (t == 0) gt[2 * s] = make_float2(fac[0], sm[0]), gt[2 * s + 1] = make_float2(fac[1], sm[1]);
+  } else if ((u & (rw - 1)) == 0) {
+    gt[(u * 16) >> gshift] = make_float2(fac[0], sm[0]);
   }
 }
 
-// ---- the base pass of one row -------------------------------------------------
+// ---- the tensor-core base pass ---------------------------------------------------
 
-// The lane's partial sum of one row: the integer dot products of its block
-// (per 32-channel half when ZW = 2), then s * 2^e * dot + m * sum(x).
-// cw: the row's codes of this lane (plane L), hw: plane H (b = 3),
-// zw: the row's (s, m) word(s) for the lane's group(s).
-template <int BITS, int ZW>
-__device__ __forceinline__ float lane_row(const uint8_t* __restrict__ cw, const uint8_t* __restrict__ hw,
-                                          const uint32_t (&xr)[16 * kXP], float xs0, float xs1,
-                                          float xsc, uint32_t z0, uint32_t z1) {
-  uint32_t A[ZW][kXP], B[ZW][kXP];
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+// The four code byte vectors of one 16-channel word of 2-bit codes (b = 3:
+// with the high bits of its 32-channel block word H merged in; par: which
+// half of the block the word is): c[0] = codes of channels 0, 4, 8, 12 of
+// the word, c[2] of 2, 6, 10, 14 (set 0), c[1] of 1, 5, 9, 13 and c[3] of
+// 3, 7, 11, 15, each times 4 (set 1).
+template <int BITS>
+__device__ __forceinline__ void code_vectors(uint32_t w, uint32_t H, int par, uint32_t (&c)[4]) {
+  const uint32_t w4 = w >> 4;
+  c[0] = w & 0x03030303u, c[1] = w & 0x0C0C0C0Cu, c[2] = w4 & 0x03030303u, c[3] = w4 & 0x0C0C0C0Cu;
+  if constexpr (BITS == 3) {
+    // the high bit of channel 4 L + m (+16 in the block's second half) sits at
+    // bit 8 L + m (+4) of H; it joins at bit 2 (set 0) or bit 4 (set 1)
+    if (par == 0) {
+      c[0] |= (H << 2) & 0x04040404u, c[1] |= (H << 3) & 0x10101010u;
+      c[2] |= H & 0x04040404u, c[3] |= (H << 1) & 0x10101010u;
+    } else {
+      c[0] |= (H >> 2) & 0x04040404u, c[1] |= (H >> 1) & 0x10101010u;
+      c[2] |= (H >> 4) & 0x04040404u, c[3] |= (H >> 3) & 0x10101010u;
+    }
+  }
+}
+
+// D = A B (the accumulator starts from zero).
+__device__ __forceinline__ void mma_s8_zero(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
+// Row sums per digit plane: acc[0], acc[1] (row gid, the lane's C columns 2t,
+// 2t + 1), acc[2], acc[3] (row gid + 8), and the offset terms am[0], am[1].
+struct RowAcc {
+  float acc[4], am[2];
+};
+
+// One group's integer dot products (J[i]: 4 sum code x_fix for b = 2, 3 or
+// sum code x_fix for b = 4, per digit plane = C column) into the rows' sums:
+// s * fac * dot per column, m * sum(x) once per row.
+__device__ __forceinline__ void group_epilogue(const int (&J)[4], float2 fx, uint32_t z0, uint32_t z1,
+                                               RowAcc& ra) {
+  const float2 s0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
+  const float2 s1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
+  const float f0 = s0.x * fx.x, f1 = s1.x * fx.x;
+  ra.acc[0] = fmaf(f0, (float)J[0], ra.acc[0]);
+  ra.acc[1] = fmaf(f0, (float)J[1], ra.acc[1]);
+  ra.acc[2] = fmaf(f1, (float)J[2], ra.acc[2]);
+  ra.acc[3] = fmaf(f1, (float)J[3], ra.acc[3]);
+  ra.am[0] = fmaf(s0.y, fx.y, ra.am[0]);
+  ra.am[1] = fmaf(s1.y, fx.y, ra.am[1]);
+}
+
+// The two rows' sums from the per-plane columns: plane 0 and 1 are the
+// columns of quad lane 0, plane 2 column 2 (quad lane 1).  Valid in quad lane 0.
+__device__ __forceinline__ void combine_planes(const RowAcc& ra, float& y0, float& y1) {
+  const float p2a = __shfl_down_sync(0xffffffffu, ra.acc[0], 1);
+  const float p2b = __shfl_down_sync(0xffffffffu, ra.acc[2], 1);
+  y0 = fmaf(65536.0f, p2a, fmaf(256.0f, ra.acc[1], ra.acc[0])) + ra.am[0];
+  y1 = fmaf(65536.0f, p2b, fmaf(256.0f, ra.acc[3], ra.acc[2])) + ra.am[1];
+}
+
+// The sums of the lane's rows of NB 16-row blocks (rows gid + 8 h, h < 2 NB)
+// over blocks [b0, b1) of max(G, 64) channels, per digit plane (acc[k]: row
+// block k).  rl: the item's first row (gid) of plane L in shared memory, rh:
+// of plane H (b = 3); sw: the rows' unit permutation (row mod 8, the same for
+// all of them).  xbl: the lane's column of the B operand (xb + 4 p + t).  z:
+// the rows' (s, m) words, group-major (row h, group j at z[h][j * zp]).
+// GM = G / 64 (0: G = 32).
+template <int BITS, int GM, int NB>
+__device__ __forceinline__ void row_blocks(const uint8_t* __restrict__ rl, int rowL, const uint8_t* __restrict__ rh,
+                                           int rowH, int sw, const uint4* __restrict__ xbl,
+                                           const float2* __restrict__ gt, const uint32_t* const (&z)[2 * NB], int zp,
+                                           int b0, int b1, int t, RowAcc (&acc)[NB]) {
+  constexpr int NR = 2 * NB;
+  const uint8_t* rp[NR];
+  const uint8_t* hp[NR];
 #pragma unroll
-  for (int h = 0; h < ZW; h++)
-#pragma unroll
-    for (int p = 0; p < kXP; p++) A[h][p] = B[h][p] = 0u;
-  auto mac = [&](uint32_t c, int v, uint32_t(&acc)[kXP]) {
-#pragma unroll
-    for (int p = 0; p < kXP; p++)
-      acc[p] = p == kXP - 1 ? dp4a_us(c, xr[kXP * v + p], acc[p]) : dp4a_uu(c, xr[kXP * v + p], acc[p]);
+  for (int h = 0; h < NR; h++) rp[h] = rl + h * 8 * rowL, hp[h] = rh + h * 8 * rowH;
+  const int swt = sw << 4, t4 = 4 * t;
+  // The raw words of 64-channel block s: the lane's plane-L word of each row
+  // (b = 4: its two words), its plane-H word (b = 3), its B fragments.  16-byte
+  // unit u of a row sits at unit u ^ sw.
+  struct Raw {
+    uint32_t w[NR], v[NR];
+    uint4 xv;
   };
-  if constexpr (BITS == 4) {
-    const uint4 q0 = reinterpret_cast<const uint4*>(cw)[0], q1 = reinterpret_cast<const uint4*>(cw)[1];
-    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  auto load = [&](int s, Raw& r) {
+    r.xv = xbl[s * 16];
+    if constexpr (BITS == 4) {
+      const int o1 = ((s << 5) ^ swt) | t4, o2 = o1 ^ 16;
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const int h = ZW == 2 ? (i >> 2) : 0;
-      mac(w[i] & 0x0F0F0F0Fu, 2 * i, A[h]);
-      mac((w[i] >> 4) & 0x0F0F0F0Fu, 2 * i + 1, A[h]);
-    }
-  } else {
-    const uint4 q0 = *reinterpret_cast<const uint4*>(cw);
-    const uint32_t w[4] = {q0.x, q0.y, q0.z, q0.w};
-    uint32_t hi[2] = {0u, 0u};
-    if constexpr (BITS == 3) {
-      const uint2 t = *reinterpret_cast<const uint2*>(hw);
-      hi[0] = t.x, hi[1] = t.y;
-    }
+      for (int h = 0; h < NR; h++) r.w[h] = lds32(rp[h] + o1), r.v[h] = lds32(rp[h] + o2);
+    } else {
+      // word 4 s + t of plane L; word 2 s + t / 2 of plane H (its block's high bits)
+      const int o = ((s << 4) ^ swt) | t4;
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const int h = ZW == 2 ? (i >> 1) : 0;
-      const uint32_t w0 = w[i], w4 = w0 >> 4;
-      uint32_t c0 = w0 & 0x03030303u, c1 = w0 & 0x0C0C0C0Cu;
-      uint32_t c2 = w4 & 0x03030303u, c3 = w4 & 0x0C0C0C0Cu;
+      for (int h = 0; h < NR; h++) r.w[h] = lds32(rp[h] + o);
       if constexpr (BITS == 3) {
-        // the high bit of the codes of vector 4i + m sits at bit 4 (i & 1) + m of
-        // each byte of hi[i / 2]; it joins at bit 2 (factor-1 vectors) or 4
-        const uint32_t H = hi[i >> 1];
-        if ((i & 1) == 0) {
-          c0 |= (H << 2) & 0x04040404u;
-          c1 |= (H << 3) & 0x10101010u;
-          c2 |= H & 0x04040404u;
-          c3 |= (H << 1) & 0x10101010u;
-        } else {
-          c0 |= (H >> 2) & 0x04040404u;
-          c1 |= (H >> 1) & 0x10101010u;
-          c2 |= (H >> 4) & 0x04040404u;
-          c3 |= (H >> 3) & 0x10101010u;
+        const int oh = (((s >> 1) << 4) ^ swt) | (4 * ((2 * s + (t >> 1)) & 3));
+#pragma unroll
+        for (int h = 0; h < NR; h++) r.v[h] = lds32(hp[h] + oh);
+      }
+    }
+  };
+  // the A fragments for row block k: set 0 (codes) and set 1 (codes times 4;
+  // b = 4: the block's second k-step)
+  auto decode = [&](const Raw& r, uint32_t (&f0)[NB][4], uint32_t (&f1)[NB][4]) {
+    if constexpr (BITS == 4) {
+#pragma unroll
+      for (int k = 0; k < NB; k++) {
+        const uint32_t wa = r.w[2 * k], wb = r.w[2 * k + 1], va = r.v[2 * k], vb = r.v[2 * k + 1];
+        f0[k][0] = wa & 0x0F0F0F0Fu, f0[k][1] = wb & 0x0F0F0F0Fu;
+        f0[k][2] = (wa >> 4) & 0x0F0F0F0Fu, f0[k][3] = (wb >> 4) & 0x0F0F0F0Fu;
+        f1[k][0] = va & 0x0F0F0F0Fu, f1[k][1] = vb & 0x0F0F0F0Fu;
+        f1[k][2] = (va >> 4) & 0x0F0F0F0Fu, f1[k][3] = (vb >> 4) & 0x0F0F0F0Fu;
+      }
+    } else {
+      uint32_t c[NR][4];
+#pragma unroll
+      for (int h = 0; h < NR; h++) code_vectors<BITS>(r.w[h], BITS == 3 ? r.v[h] : 0u, t & 1, c[h]);
+#pragma unroll
+      for (int k = 0; k < NB; k++) {
+        f0[k][0] = c[2 * k][0], f0[k][1] = c[2 * k + 1][0], f0[k][2] = c[2 * k][2], f0[k][3] = c[2 * k + 1][2];
+        f1[k][0] = c[2 * k][1], f1[k][1] = c[2 * k + 1][1], f1[k][2] = c[2 * k][3], f1[k][3] = c[2 * k + 1][3];
+      }
+    }
+  };
+  auto frags = [&](int s, uint32_t (&f0)[NB][4], uint32_t (&f1)[NB][4], uint4& xv) {
+    Raw r;
+    load(s, r);
+    decode(r, f0, f1);
+    xv = r.xv;
+  };
+  // a group's epilogue: its scale words and factor are loaded with its codes
+  struct Ep {
+    uint32_t z[NR];
+    float2 fx;
+  };
+  auto load_ep = [&](int g, Ep& e) {
+    e.fx = gt[g];
+    const int col = g * zp;
+#pragma unroll
+    for (int h = 0; h < NR; h++) e.z[h] = z[h][col];
+  };
+  auto finish = [&](const Ep& e, const int (&C0)[NB][4], const int (&C1)[NB][4]) {
+#pragma unroll
+    for (int k = 0; k < NB; k++) {
+      int J[4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) J[i] = BITS == 4 ? C0[k][i] + C1[k][i] : 4 * C0[k][i] + C1[k][i];
+      group_epilogue(J, e.fx, e.z[2 * k], e.z[2 * k + 1], acc[k]);
+    }
+  };
+  if constexpr (GM >= 1) {
+    for (int g = b0; g < b1; g++) {
+      int C0[NB][4], C1[NB][4];
+#pragma unroll
+      for (int m = 0; m < GM; m++) {
+        uint4 xv;
+        uint32_t f0[NB][4], f1[NB][4];
+        frags(g * GM + m, f0, f1, xv);
+#pragma unroll
+        for (int k = 0; k < NB; k++) {
+          if (m == 0) {
+            mma_s8_zero(C0[k], f0[k][0], f0[k][1], f0[k][2], f0[k][3], xv.x, xv.y);
+            mma_s8_zero(C1[k], f1[k][0], f1[k][1], f1[k][2], f1[k][3], xv.z, xv.w);
+          } else {
+            mma_s8(C0[k], f0[k][0], f0[k][1], f0[k][2], f0[k][3], xv.x, xv.y);
+            mma_s8(C1[k], f1[k][0], f1[k][1], f1[k][2], f1[k][3], xv.z, xv.w);
+          }
         }
       }
-      mac(c0, 4 * i + 0, A[h]);
-      mac(c1, 4 * i + 1, B[h]);
-      mac(c2, 4 * i + 2, A[h]);
-      mac(c3, 4 * i + 3, B[h]);
+      Ep e;
+      load_ep(g, e);
+      finish(e, C0, C1);
     }
-  }
-  // 4 x sum(code x_fix) (b = 2, 3: set B carries the factor 4) or sum(code x_fix) (b = 4)
-  int32_t J[ZW];
-#pragma unroll
-  for (int h = 0; h < ZW; h++) {
-    uint32_t a = A[h][0], bb = B[h][0];
-#pragma unroll
-    for (int p = 1; p < kXP; p++) a += A[h][p] << (8 * p), bb += B[h][p] << (8 * p);
-    J[h] = BITS == 4 ? (int32_t)a : (int32_t)((a << 2) + bb);
-  }
-  const float2 sm0 = __half22float2(*reinterpret_cast<const __half2*>(&z0));
-  if constexpr (ZW == 1) {
-    return fmaf(sm0.x * xsc, (float)J[0], sm0.y * (xs0 + xs1));
   } else {
-    const float2 sm1 = __half22float2(*reinterpret_cast<const __half2*>(&z1));
-    return fmaf(sm0.x * xsc, (float)J[0], fmaf(sm1.x * xsc, (float)J[1], fmaf(sm0.y, xs0, sm1.y * xs1)));
-  }
-}
-
-// Sum each of U per-lane values over the warp.  Returns the full sum of value
-// lane >> 3 (U = 4) or lane >> 4 (U = 2) in every lane.
-template <int U>
-__device__ __forceinline__ float warp_sum_rows(float (&a)[U], int lane) {
-  if constexpr (U == 4) {
-    const bool up = lane & 16;
-    float k0 = up ? a[2] : a[0], k1 = up ? a[3] : a[1];
-    float s0 = up ? a[0] : a[2], s1 = up ? a[1] : a[3];
-    k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-    k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    const bool up8 = lane & 8;
-    float k = up8 ? k1 : k0, s = up8 ? k0 : k1;
-    k += __shfl_xor_sync(0xffffffffu, s, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;
-  } else {
-    const bool up = lane & 16;
-    float k = up ? a[1] : a[0], s = up ? a[0] : a[1];
-    k += __shfl_xor_sync(0xffffffffu, s, 16);
-    k += __shfl_xor_sync(0xffffffffu, k, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;
+    // 32-channel groups: block s holds groups 2 s and 2 s + 1
+    for (int s = b0; s < b1; s++) {
+      uint4 xv;
+      uint32_t f0[NB][4], f1[NB][4];
+      frags(s, f0, f1, xv);
+      int Ca0[NB][4], Ca1[NB][4], Cb0[NB][4], Cb1[NB][4];  // group 2 s: Ca, group 2 s + 1: Cb
+#pragma unroll
+      for (int k = 0; k < NB; k++) {
+        if constexpr (BITS == 4) {
+          // the block's two k-steps are the two groups
+          mma_s8_zero(Ca0[k], f0[k][0], f0[k][1], f0[k][2], f0[k][3], xv.x, xv.y);
+          mma_s8_zero(Cb0[k], f1[k][0], f1[k][1], f1[k][2], f1[k][3], xv.z, xv.w);
+#pragma unroll
+          for (int i = 0; i < 4; i++) Ca1[k][i] = Cb1[k][i] = 0;
+        } else {
+          // quad lanes 0, 1 hold group 2 s, lanes 2, 3 group 2 s + 1: each
+          // group's products take the other lanes' activations as zero
+          const bool lo = t < 2;
+          mma_s8_zero(Ca0[k], f0[k][0], f0[k][1], f0[k][2], f0[k][3], lo ? xv.x : 0u, lo ? xv.y : 0u);
+          mma_s8_zero(Ca1[k], f1[k][0], f1[k][1], f1[k][2], f1[k][3], lo ? xv.z : 0u, lo ? xv.w : 0u);
+          mma_s8_zero(Cb0[k], f0[k][0], f0[k][1], f0[k][2], f0[k][3], lo ? 0u : xv.x, lo ? 0u : xv.y);
+          mma_s8_zero(Cb1[k], f1[k][0], f1[k][1], f1[k][2], f1[k][3], lo ? 0u : xv.z, lo ? 0u : xv.w);
+        }
+      }
+      Ep e0, e1;
+      load_ep(2 * s, e0);
+      load_ep(2 * s + 1, e1);
+      finish(e0, Ca0, Ca1);
+      finish(e1, Cb0, Cb1);
+    }
   }
 }
 
 // ---- the kernel -----------------------------------------------------------------
 
-// RPW: rows per compute warp per stage (2 or 4).  A CTA's warps are spread
-// over the SM's four schedulers, each with a quarter of the register file:
-// four warps of 120 registers a thread leave kSideRegs / 4 of every quarter
-// free for a staging CTA.
-static_assert(((kMaxWarps + 1 + 3) / 4) * 120 * 32 + kSideRegs / 4 <= 65536 / 4,
+// A CTA's warps are spread over the SM's four schedulers, each with a quarter
+// of the register file: seven warps of 64 registers a thread leave kSideRegs
+// / 4 of every quarter free for a staging CTA.
+constexpr int kGemvRegs = 64;
+static_assert(((kMaxWarps + 1 + 3) / 4) * kGemvRegs * 32 + kSideRegs / 4 <= 65536 / 4,
               "GEMV registers leave no room for a staging CTA");
-template <int BITS, int ZW, int RPW>
-__global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
+template <int BITS, int GM, int NB>
+__global__ void __maxnreg__(kGemvRegs) gemv_kernel(GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
   uint64_t* szbar = empty + kMaxStages;
   uint8_t* ring = smem + a.off_ring;
-  uint32_t* szs = reinterpret_cast<uint32_t*>(smem + a.off_sz);
-  uint32_t* xpl = reinterpret_cast<uint32_t*>(smem + a.off_x);
+  // the rows' (s, m) words: copied row-major into the region the correction
+  // partials take at the end, then transposed group-major (szt) for the
+  // epilogue and the correction, whose reads then take consecutive rows of
+  // one group
+  uint32_t* szs = reinterpret_cast<uint32_t*>(smem + a.off_cpart);  // [rows][gpr]
+  uint32_t* szt = reinterpret_cast<uint32_t*>(smem + a.off_szt);  // [gpr][szt_pitch]
+  uint4* xb = reinterpret_cast<uint4*>(smem + a.off_xb);
+  float2* gt = reinterpret_cast<float2*>(smem + a.off_gt);
   float* part = reinterpret_cast<float*>(smem + a.off_part);
-  uint32_t* szt = reinterpret_cast<uint32_t*>(smem + a.off_szt);
   uint2* jd = reinterpret_cast<uint2*>(smem + a.off_jd);
   uint32_t* wt = reinterpret_cast<uint32_t*>(smem + a.off_wt);
+  int* jrow = reinterpret_cast<int*>(smem + a.off_jrow);
   float* cpart = reinterpret_cast<float*>(smem + a.off_cpart);
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -399,8 +514,8 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
   pdl_trigger();  // the next kernel of the stream may be scheduled; it waits for this grid
 
   if (warp == a.W) {
-    // ---------------- producer warp
-    int issued = 0;
+    // ---------------- producer warp (lane 0): one bulk copy per stage and
+    // plane, the rows' (s, m) words in one copy
     auto issue = [&](int i) {
       const int slot = i % S;
       const int r0 = i * a.rc, nr = min(a.rc, rows - r0);
@@ -410,10 +525,16 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
       bulk_g2s(dst, a.base + (size_t)(n0 + r0) * a.rowL, bl, &full[slot]);
       if (BITS == 3) bulk_g2s(dst + (size_t)a.rc * a.rowL, a.base + a.hi_off + (size_t)(n0 + r0) * a.rowH, bh, &full[slot]);
     };
+    int issued = 0;
     if (lane == 0) {
-      const uint32_t zb = (uint32_t)(rows * a.gpr * 4);
-      mbar_expect_tx(szbar, zb);
-      bulk_g2s(szs, a.sz + (size_t)n0 * a.gpr, zb, szbar);
+      // the scale table and the first two stages are needed first: the other
+      // stages are requested once the table has landed, so that they do not
+      // compete with it for the memory system
+      const uint32_t zbytes = (uint32_t)(rows * a.gpr * 4);
+      mbar_expect_tx(szbar, zbytes);
+      bulk_g2s(szs, a.sz + (size_t)n0 * a.gpr, zbytes, szbar);
+      for (; issued < min(min(S, nst), 2); issued++) issue(issued);
+      mbar_wait(szbar, 0);
       for (; issued < min(S, nst); issued++) issue(issued);
     }
     pdl_wait();  // the previous kernel is complete (no data of it is read here)
@@ -430,25 +551,30 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
     __syncwarp();
   } else {
     // ---------------- compute warps
-    const int seg = warp % a.segs, jw = warp / a.segs;
-    const int lg = seg * 32 + lane;  // lane block
-    const bool la = lg * kLaneCh < a.K;
     const int tc = threadIdx.x, ntc = a.W * 32;
+    const int t = lane & 3, gid = lane >> 2, p = gid & 3;
+    // the scale table does not depend on earlier kernels: transposed before
+    // the grid dependency wait
+    bool ok = mbar_wait(szbar, 0);
+    for (int r = warp; r < rows; r += a.W)
+      for (int g = lane; g < a.gpr; g += 32) szt[g * a.szt_pitch + r] = szs[r * a.gpr + g];
     pdl_wait();  // x, the selection and the staged rows are complete
     // correction tables, entries tc, tc + ntc, ...: the selection's loads are
-    // issued first, their activations after the planes (every load of a round
-    // in flight together)
+    // issued first, their activations after the B operand (every load of a
+    // round in flight together)
     constexpr int kJ = 2;
     int rawj[kJ];
     if (corr)
 #pragma unroll
       for (int u = 0; u < kJ; u++) rawj[u] = tc + u * ntc < a.n_sel ? __ldg(a.sel + tc + u * ntc) : 0;
-    // activation planes: four threads per 64-channel lane block
     {
-      const int nq = (a.K / kLaneCh) * 4;
-      for (int b0 = warp * 32; b0 < nq; b0 += ntc) {
-        const int idx = b0 + lane, b = idx >> 2, q = idx & 3;
-        quarter_planes<BITS>(idx < nq, a.x + (size_t)b * kLaneCh + 16 * q, q, xpl + (size_t)b * kXW);
+      const int nu = a.K / 16;
+      const int rw = (BITS == 4 && GM == 0) ? 4 : (1 << (a.gshift - 4));
+      for (int u0 = warp * 32; u0 < nu; u0 += ntc) {
+        if (BITS == 4 && GM == 0)
+          build_unit<BITS, true>(a.x, u0 + lane, rw, a.gshift, xb, gt);
+        else
+          build_unit<BITS, false>(a.x, u0 + lane, rw, a.gshift, xb, gt);
       }
     }
     if (corr) {
@@ -463,29 +589,28 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
           const int c = min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
           const uint32_t xc = raw < 0 ? 0u : __float_as_uint(h2f(__ldg(a.x + c)));
           jd[j] = make_uint2(xc, (uint32_t)(c >> a.gshift));
-          const uint32_t* src = a.refine + (size_t)(a.staged ? j : c) * a.row_words + w_lo;
-          for (int k = 0; k < nwr; k++) cp_async4(wt + (size_t)j * a.wt_pitch + k, src + k);
+          jrow[j] = a.staged ? j : c;
         }
+      }
+    }
+    bar_sync(1, a.W * 32);  // B operand, group table, channel table and scale table complete
+    if (corr) {
+      // the refinement words of the CTA's rows, (entry, word) pairs spread
+      // over the threads; they land during the base pass
+      for (int e = tc; e < a.n_sel * nwr; e += ntc) {
+        const int j = e / nwr, k = e - j * nwr;
+        cp_async4(wt + (size_t)j * a.wt_pitch + k, a.refine + (size_t)jrow[j] * a.row_words + w_lo + k);
       }
       cp_async_commit();
     }
-    bar_sync(1, a.W * 32);
-    uint32_t xr[16 * kXP];
-    float xs0, xs1, xsc;
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(xpl + ((size_t)seg * 32 + lane) * kXW);
-#pragma unroll
-      for (int k = 0; k < 4 * kXP; k++) {
-        const uint4 q = src[k];
-        xr[4 * k] = q.x, xr[4 * k + 1] = q.y, xr[4 * k + 2] = q.z, xr[4 * k + 3] = q.w;
-      }
-      const float4 f = reinterpret_cast<const float4*>(src)[4 * kXP];
-      xs0 = f.x, xs1 = f.y, xsc = f.z;
-    }
-    const int g0 = (lg * kLaneCh) >> a.gshift;            // the lane's (first) group
-    const bool zown = corr && la && ((lg * kLaneCh) & ((1 << a.gshift) - 1)) == 0;
-    bool ok = mbar_wait(szbar, 0);
-    const size_t codeL = (size_t)lg * (BITS == 4 ? 32 : 16);
+    // the warp's item, the same in every stage ((rb / NB) nseg <= W): row
+    // blocks rbk .. rbk + NB - 1 of the stage, blocks [b0, b1) of the channels
+    const bool has_item = warp < (a.rb / NB) * a.nseg;
+    const int rbk = (warp / a.nseg) * NB, sg = warp % a.nseg;
+    const int b0 = sg * a.nblk / a.nseg, b1 = (sg + 1) * a.nblk / a.nseg;
+    const uint32_t rl_off = (uint32_t)(16 * rbk + gid) * a.rowL;
+    const uint32_t rh_off = (uint32_t)a.rc * a.rowL + (uint32_t)(16 * rbk + gid) * a.rowH;
+    const uint4* xbl = xb + 4 * p + t;
     for (int i = 0; i < nst && ok; i++) {
       const int slot = i % S;
       if (!mbar_wait(&full[slot], (i / S) & 1)) {
@@ -493,27 +618,29 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
         break;
       }
       const uint8_t* sl = ring + (size_t)slot * a.stage_bytes;
-      float pv[RPW];
+      const int lr0 = i * a.rc + 16 * rbk;
+      if (has_item && lr0 < rows) {
+        // the rows' (s, m) words; rows past the end read the last row's (their
+        // sums are not stored)
+        const uint32_t* z[2 * NB];
 #pragma unroll
-      for (int t = 0; t < RPW; t++) {
-        const int rr = jw + a.R * t, lr = i * a.rc + rr;
-        pv[t] = 0.f;
-        if (la && lr < rows) {
-          const uint32_t* zr = szs + (size_t)lr * a.gpr + g0;
-          const uint32_t z0 = zr[0], z1 = ZW == 2 ? zr[1] : 0u;
-          if (zown) {
-            szt[(size_t)g0 * a.szt_pitch + lr] = z0;
-            if (ZW == 2) szt[(size_t)(g0 + 1) * a.szt_pitch + lr] = z1;
+        for (int h = 0; h < 2 * NB; h++) z[h] = szt + min(lr0 + gid + 8 * h, rows - 1);
+        RowAcc acc[NB];
+#pragma unroll
+        for (int k = 0; k < NB; k++) acc[k] = RowAcc{{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f}};
+        row_blocks<BITS, GM, NB>(sl + rl_off, a.rowL, sl + rh_off, a.rowH, (n0 + lr0 + gid) & 7, xbl, gt, z,
+                                 a.szt_pitch, b0, b1, t, acc);
+#pragma unroll
+        for (int k = 0; k < NB; k++) {
+          float y0, y1;
+          combine_planes(acc[k], y0, y1);
+          const int r0 = lr0 + 16 * k + gid;
+          if (t == 0) {
+            if (r0 < rows) part[r0 * a.nseg + sg] = y0;
+            if (r0 + 8 < rows) part[(r0 + 8) * a.nseg + sg] = y1;
           }
-          pv[t] = lane_row<BITS, ZW>(sl + (size_t)rr * a.rowL + codeL,
-                                     sl + (size_t)a.rc * a.rowL + (size_t)rr * a.rowH + (size_t)lg * 8, xr, xs0,
-                                     xs1, xsc, z0, z1);
         }
       }
-      const float tot = warp_sum_rows<RPW>(pv, lane);
-      const int t = RPW == 4 ? (lane >> 3) : (lane >> 4);
-      const int lr = i * a.rc + jw + a.R * t;
-      if ((lane & (32 / RPW - 1)) == 0 && lr < rows) part[(size_t)lr * a.segs + seg] = tot;
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
@@ -530,7 +657,7 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
     const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << r)) / (float)(1 << r);
     for (int task = threadIdx.x; task < nb * Q; task += blockDim.x) {
       const int blk = task % nb, q = task / nb;
-      const int j0 = (int)((long)q * a.n_sel / Q), j1 = (int)((long)(q + 1) * a.n_sel / Q);
+      const int j0 = q * a.n_sel / Q, j1 = (q + 1) * a.n_sel / Q;
       const int bit0 = (n0 + 4 * blk) * r;
       const int wi = (bit0 >> 5) - w_lo;
       int rot[4];
@@ -541,28 +668,32 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
       int gcur = -1;
       auto flush = [&]() {
         if (gcur >= 0) {
-          const uint4 z = *reinterpret_cast<const uint4*>(szt + (size_t)gcur * a.szt_pitch + 4 * blk);
+          const uint4 z = *reinterpret_cast<const uint4*>(szt + gcur * a.szt_pitch + 4 * blk);
           const uint32_t zz[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
           for (int t = 0; t < 4; t++)
             acc[t] = fmaf(__low2float(*reinterpret_cast<const __half2*>(&zz[t])), run[t] - C, acc[t]);
         }
       };
+      // channel j + 1's table entry and refinement word are read while j is summed
+      uint2 d = j0 < j1 ? jd[j0] : make_uint2(0u, 0u);
+      uint32_t w = j0 < j1 ? wt[j0 * a.wt_pitch + wi] : 0u;
       for (int j = j0; j < j1; j++) {
-        const uint2 d = jd[j];
+        const uint2 dn = j + 1 < j1 ? jd[j + 1] : make_uint2(0u, 0u);
+        const uint32_t wn = j + 1 < j1 ? wt[(j + 1) * a.wt_pitch + wi] : 0u;
         if ((int)d.y != gcur) {
           flush();
           gcur = (int)d.y, C = 0.f;
 #pragma unroll
           for (int t = 0; t < 4; t++) run[t] = 0.f;
         }
-        const uint32_t w = wt[(size_t)j * a.wt_pitch + wi];
         const float xc = __uint_as_float(d.x);
         // f = 1 + rho / 2^r; sum x f - sum x (1 - off/2^r) = sum x (rho + off) / 2^r
 #pragma unroll
         for (int t = 0; t < 4; t++)
           run[t] = fmaf(__uint_as_float(0x3F800000u | (__funnelshift_l(w, w, rot[t]) & fmask)), xc, run[t]);
         C = fmaf(xc, cfac, C);
+        d = dn, w = wn;
       }
       flush();
       *reinterpret_cast<float4*>(cpart + (size_t)q * a.rows_max + 4 * blk) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -570,17 +701,34 @@ __global__ void __maxnreg__(120) gemv_kernel(GemvArgs a) {
     bar_sync(2, blockDim.x);
   }
 
-  // ---------------- output
-  for (int lr = threadIdx.x; lr < rows; lr += blockDim.x) {
-    float base = 0.f, c = 0.f;
-    for (int s = 0; s < a.segs; s++) base += part[(size_t)lr * a.segs + s];
-    if (corr)
-      for (int q = 0; q < a.cparts; q++) c += cpart[(size_t)q * a.rows_max + lr];
-    if (a.y_corr) {
-      a.y[n0 + lr] = base;
-      a.y_corr[n0 + lr] = c;
-    } else {
-      a.y[n0 + lr] = base + c;
+  // ---------------- output: T = 2^k threads per row (as many as the block
+  // has for its rows, at most 32) sum the row's partials (base pass ranges,
+  // correction shares), then combine over their lanes
+  {
+    int T = 1;
+    while (T < 32 && 2 * T * rows <= (int)blockDim.x) T *= 2;
+    const int sub = threadIdx.x & (T - 1);
+    for (int lr0 = 0; lr0 < rows; lr0 += (int)blockDim.x / T) {
+      const int lr = lr0 + (int)threadIdx.x / T;
+      const bool in = lr < rows;
+      float base = 0.f, c = 0.f;
+      if (in) {
+        for (int q = sub; q < a.nseg; q += T) base += part[lr * a.nseg + q];
+        if (corr)
+          for (int q = sub; q < a.cparts; q += T) c += cpart[(size_t)q * a.rows_max + lr];
+      }
+      for (int o = T / 2; o > 0; o >>= 1) {
+        base += __shfl_xor_sync(0xffffffffu, base, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+      }
+      if (in && sub == 0) {
+        if (a.y_corr) {
+          a.y[n0 + lr] = base;
+          a.y_corr[n0 + lr] = c;
+        } else {
+          a.y[n0 + lr] = base + c;
+        }
+      }
     }
   }
 }
@@ -619,12 +767,12 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
   const int per_b = a.N / kCorrRows;
   const int b = u / per_b, row0 = (u - b * per_b) * kCorrRows;
   const int bit0 = row0 * a.r, wi = bit0 >> 5;
-  const int gpr = a.K >> a.gshift;
   // the rows' bits start at bit sh of the word (a multiple of 8); the word is
   // shifted down first, so row t's field sits at bit R t
   const int sh = bit0 & 31;
   constexpr uint32_t fmask = ((1u << R) - 1u) << (23 - R);
   const float cfac = 1.0f - (0.5f - 0.5f * (float)(1 << R)) / (float)(1 << R);
+  const int gpr = a.K >> a.gshift;
   const uint32_t* zrow = reinterpret_cast<const uint32_t*>(a.sz) + (size_t)row0 * gpr;
   const int32_t* sel = a.sel + (size_t)b * a.n_sel;
   const uint16_t* xb = a.x + (size_t)b * a.K;
@@ -637,7 +785,7 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
     if (gcur >= 0) {
 #pragma unroll
       for (int t = 0; t < kCorrRows; t++) {
-        const uint32_t zw = __ldg(zrow + (size_t)t * gpr + gcur);
+        const uint32_t zw = __ldg(zrow + (t * gpr + gcur));
         acc[t] = fmaf(__low2float(*reinterpret_cast<const __half2*>(&zw)), run[t] - C, acc[t]);
       }
     }
@@ -691,25 +839,23 @@ size_t align128(size_t v) { return (v + 127) & ~(size_t)127; }
 
 struct Plan {
   GemvArgs a;  // shape and shared memory layout (pointers are set per launch)
-  int grid, threads, rpw, zw;
+  int grid, threads, gm;
   size_t smem;
 };
 
-// Work split and shared memory layout of one GEMV shape: segments of 2,048
-// channels, warps per segment (at most 16 compute warps), rows per stage (the
-// warps of a segment take RPW rows each), the ring depth that fits.
+// Work split and shared memory layout of one GEMV shape: 16-row blocks per
+// stage and group ranges per row block (each compute warp takes one (row
+// block, range) item per stage), the ring depth that fits.
 sf_status make_plan(const sf_wq* w, int n_sel, Plan& P) {
   GemvArgs& a = P.a;
   a = GemvArgs{};
-  const int N = w->n, K = w->k;
+  const int N = w->n, K = w->k, G = w->group;
   a.N = N, a.K = K, a.r = w->r, a.n_sel = n_sel;
-  a.gpr = K / w->group;
+  a.gpr = K / G;
   a.gshift = 0;
-  while ((1 << a.gshift) < w->group) a.gshift++;
-  a.segs = (K + kSegCh - 1) / kSegCh;
-  SF_UNSUPPORTED(a.segs <= kMaxSegs, "k=%d above %d", K, kMaxSegs * kSegCh);
-  a.R = std::max(1, kMaxWarps / a.segs);
-  a.W = a.segs * a.R;
+  while ((1 << a.gshift) < G) a.gshift++;
+  P.gm = G / 64;  // 0: 32-channel groups
+  a.nblk = K / std::max(G, 64);
   a.rowL = K * (w->b == 4 ? 4 : 2) / 8;
   a.rowH = w->b == 3 ? K / 8 : 0;
   a.hi_off = w->b == 3 ? (size_t)N * K / 4 : 0;
@@ -717,34 +863,49 @@ sf_status make_plan(const sf_wq* w, int n_sel, Plan& P) {
   const int units = N / kRowUnit;
   P.grid = std::min(num_sms(), units);
   a.rows_max = ((units + P.grid - 1) / P.grid) * kRowUnit;
-  // four rows per warp per stage when a stage stays small and a CTA still gets
-  // two or more stages (compute starts as soon as the first one lands)
-  P.rpw = (size_t)a.R * 4 * rowB <= kStageTarget && a.rows_max >= 2 * a.R * 4 ? 4 : 2;
-  a.rc = a.R * P.rpw;
+  a.W = kMaxWarps;
+  // row blocks per stage (rb) and group ranges (nseg = W / rb, one item per
+  // warp and stage): the split with the least work for the busiest warp,
+  // stages ceil(rows / 16 rb) x blocks ceil(nblk / nseg); among equal ones the
+  // smaller stage (a deeper ring)
+  {
+    const int blocks = (a.rows_max + 15) / 16;
+    long best = -1;
+    for (int rb = 1; rb <= std::min(blocks, 4); rb++) {
+      if (rb > 1 && (size_t)rb * 16 * rowB > kStageMax) break;
+      const int nseg = std::max(1, std::min(a.nblk, a.W / rb));
+      const long cost = (long)((blocks + rb - 1) / rb) * ((a.nblk + nseg - 1) / nseg);
+      if (best < 0 || cost < best) best = cost, a.rb = rb, a.nseg = nseg;
+    }
+  }
+  a.rc = 16 * a.rb;
   a.stage_bytes = (int)(a.rc * rowB);
   a.row_words = N * w->r / 32;
   a.wt_pitch = ((a.rows_max * w->r + 31) >> 5) + 1;
-  a.szt_pitch = (a.rows_max + 3) & ~3;
-  if (a.szt_pitch % 32 == 0) a.szt_pitch += 4;  // spread the group-major scale stores over banks
   P.threads = (a.W + 1) * 32;
-  P.zw = w->group == 32 ? 2 : 1;
   const int nb_max = a.rows_max / 4;
-  // channel shares of the correction: enough threads busy, and few partial
-  // sums per row for the output's serial add
-  a.cparts = n_sel > 0 ? std::max(1, std::min(std::min(n_sel, 16), P.threads / nb_max)) : 0;
+  // channel shares of the correction: every thread busy when the CTA has few
+  // rows (the output sums a row's shares on the lanes of a warp)
+  a.cparts = n_sel > 0 ? std::max(1, std::min(std::min(n_sel, 64), P.threads / nb_max)) : 0;
   size_t off = align128((2 * kMaxStages + 1) * sizeof(uint64_t));
-  a.off_sz = (int)off;
-  off += align128((size_t)a.rows_max * a.gpr * 4);
+  a.szt_pitch = (a.rows_max + 3) & ~3;
+  a.off_szt = (int)off;
+  off += align128((size_t)a.gpr * a.szt_pitch * 4);
+  a.off_gt = (int)off;
+  off += align128((size_t)a.gpr * 8);
   a.off_part = (int)off;
-  off += align128((size_t)a.rows_max * a.segs * 4);
-  // the activation planes are read once, before the correction partials are written
-  a.off_x = a.off_cpart = (int)off;
-  off += align128(std::max((size_t)a.segs * 32 * kXW * 4, (size_t)a.cparts * a.rows_max * 4));
+  off += align128((size_t)a.rows_max * a.nseg * 4);
+  a.off_xb = (int)off;
+  off += align128((size_t)K * 4);
+  // one region for the row-major scale copy (until it is transposed) and the
+  // correction partials (after the base pass)
+  a.off_cpart = (int)off;
+  off += align128(std::max((size_t)a.cparts * a.rows_max * 4, (size_t)a.rows_max * a.gpr * 4));
   if (n_sel > 0) {
-    a.off_szt = (int)off;
-    off += align128((size_t)a.gpr * a.szt_pitch * 4);
     a.off_jd = (int)off;
     off += align128((size_t)n_sel * 8);
+    a.off_jrow = (int)off;
+    off += align128((size_t)n_sel * 4);
     a.off_wt = (int)off;
     off += align128((size_t)n_sel * a.wt_pitch * 4);
   }
@@ -760,15 +921,20 @@ sf_status make_plan(const sf_wq* w, int n_sel, Plan& P) {
   return SF_OK;
 }
 
-template <int BITS, int ZW>
-void* kernel_for(int rpw) {
-  return rpw == 4 ? (void*)gemv_kernel<BITS, ZW, 4> : (void*)gemv_kernel<BITS, ZW, 2>;
+template <int BITS>
+void* kernel_for(int gm) {
+  switch (gm) {
+    case 0: return (void*)gemv_kernel<BITS, 0, 1>;
+    case 1: return (void*)gemv_kernel<BITS, 1, 1>;
+    case 2: return (void*)gemv_kernel<BITS, 2, 1>;
+    default: return (void*)gemv_kernel<BITS, 4, 1>;
+  }
 }
 
-void* pick_kernel(int b, int zw, int rpw) {
-  if (b == 2) return zw == 1 ? kernel_for<2, 1>(rpw) : kernel_for<2, 2>(rpw);
-  if (b == 3) return zw == 1 ? kernel_for<3, 1>(rpw) : kernel_for<3, 2>(rpw);
-  return zw == 1 ? kernel_for<4, 1>(rpw) : kernel_for<4, 2>(rpw);
+void* pick_kernel(int b, int gm) {
+  if (b == 2) return kernel_for<2>(gm);
+  if (b == 3) return kernel_for<3>(gm);
+  return kernel_for<4>(gm);
 }
 
 sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, int kch,
@@ -805,7 +971,7 @@ sf_status gemv_launch(const sf_wq* w, const uint16_t* x, int batch, int chunk, i
     if (st != SF_OK) return st;
     sel = sel_out;
   }
-  void* kern = pick_kernel(w->b, P.zw, P.rpw);
+  void* kern = pick_kernel(w->b, P.gm);
   SF_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

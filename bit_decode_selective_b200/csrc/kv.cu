@@ -726,7 +726,7 @@ __global__ void __launch_bounds__(kSelThreads) kv_pick_kernel(SelArgs a) {
   uint32_t* ck = bits + kMaxT / 32;                            // [kCandCap] keys
   int* ct = reinterpret_cast<int*>(ck + kCandCap);             // [kCandCap] tokens
   int* tie_t = ct + kCandCap;                                  // [kTieCap]
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int g = blockIdx.y, bat = blockIdx.z;
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();

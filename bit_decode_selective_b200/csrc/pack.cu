@@ -10,6 +10,7 @@
 // with the definition in sf.h.
 #include "common.cuh"
 #include "quant.cuh"
+#include "wqlayout.cuh"
 
 namespace sf {
 
@@ -41,7 +42,6 @@ __global__ void pack_weights_kernel(const float* __restrict__ w, int N, int K, i
   sz[idx * 2 + 0] = g.s16;
   sz[idx * 2 + 1] = g.m16;
   const int qmax = (1 << (b + r)) - 1;
-  const long c0 = (long)n * K + (long)j * G;  // first element of the group
   uint32_t* hiplane = base + (size_t)N * K / 16;  // b == 3: plane H after plane L
   for (int blk = 0; blk < G / 32; blk++) {
     uint32_t lw[4] = {0, 0, 0, 0};  // up to 128 bits of codes for 32 channels
@@ -59,15 +59,15 @@ __global__ void pack_weights_kernel(const float* __restrict__ w, int N, int K, i
       long rbit = ((long)ch * N + n) * r;
       atomicOr(&R[rbit >> 5], (uint32_t)rho << (rbit & 31));
     }
-    long e0 = c0 + blk * 32;  // element index of the block's first code
+    const int cb = j * G + blk * 32;  // the block's first channel
     if (b == 4) {
-      uint32_t* dst = base + e0 / 8;
-      for (int i = 0; i < 4; i++) dst[i] = lw[i];
+      uint32_t* row = base + (size_t)n * (K / 8);
+      for (int i = 0; i < 4; i++) row[wq_word(n, cb / 8 + i)] = lw[i];
     } else {
-      uint32_t* dst = base + e0 / 16;
-      dst[0] = lw[0];
-      dst[1] = lw[1];
-      if (b == 3) hiplane[e0 / 32] = hw;
+      uint32_t* row = base + (size_t)n * (K / 16);
+      row[wq_word(n, cb / 16)] = lw[0];
+      row[wq_word(n, cb / 16 + 1)] = lw[1];
+      if (b == 3) hiplane[(size_t)n * (K / 32) + wq_word(n, cb / 32)] = hw;
     }
   }
 }
@@ -80,12 +80,12 @@ __global__ void unpack_weights_kernel(const uint32_t* __restrict__ base,
   long n = idx / K, c = idx % K;
   int q;
   if (b == 4) {
-    q = (base[idx / 8] >> (4 * (idx & 7))) & 15;
+    q = (base[(size_t)n * (K / 8) + wq_word((int)n, (int)(c / 8))] >> (4 * (c & 7))) & 15;
   } else {
-    q = (base[idx / 16] >> (2 * (idx & 15))) & 3;
+    q = (base[(size_t)n * (K / 16) + wq_word((int)n, (int)(c / 16))] >> (2 * (c & 15))) & 3;
     if (b == 3) {
       const uint32_t* hp = base + (size_t)N * K / 16;
-      q |= ((hp[idx / 32] >> hi_plane_bit((int)(c & 31))) & 1) << 2;
+      q |= ((hp[(size_t)n * (K / 32) + wq_word((int)n, (int)(c / 32))] >> hi_plane_bit((int)(c & 31))) & 1) << 2;
     }
   }
   qb[idx] = (uint8_t)q;

@@ -103,6 +103,10 @@ SF_API const char* sf_last_error(void);
  *              32-bit word in which channel c (0..31 within the block) sits at
  *              bit 8*(c/4) + c%4 for c < 16 and at bit 8*((c-16)/4) + 4 +
  *              (c-16)%4 for c >= 16.
+ *   Each row of a plane is then cut into 16-byte units, and unit u of row i
+ *   is stored at unit u XOR (i mod 8) of the row (units move only inside
+ *   their aligned 128-byte block; rows of eight consecutive indices hold a
+ *   unit in eight different shared-memory bank groups).
  * refine (k*n*r/8 bytes): channel-major, one natural r-bit stream of the n
  *   refinement codes of each input channel ("one contiguous run per channel",
  *   so a selected channel's refinement is one row); may be NULL when

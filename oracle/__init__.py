@@ -152,6 +152,9 @@ def dequant_weights(qb, rho, sz, r: int, G: int, refined_mask=None) -> np.ndarra
 
 def pack_weights(qb, rho, b: int, r: int):
     N, K = qb.shape
+    # the format permutes 16-byte units inside 128-byte blocks of every row:
+    # rows of whole blocks only (the library's k % 1024 rule)
+    assert K % 1024 == 0, "k must be a multiple of 1024"
     qb = np.ascontiguousarray(qb, np.uint8)
     rho = np.ascontiguousarray(rho, np.uint8)
     base = np.empty(N * K * b // 8, np.uint8)

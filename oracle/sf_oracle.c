@@ -212,32 +212,51 @@ static int hi_plane_bit(int cp) {
 }
 
 /* Weight base codes, row n of N, channel c of K:
- *   b = 2, 4: one natural b-bit stream per row, rows consecutive (N*K*b/8 B);
- *   b = 3:    plane L (low 2 bits, natural 2-bit stream per row, N*K/4 B)
- *             followed by plane H (high bit, N*K/8 B): per row, per 32-channel
- *             block, one little-endian 32-bit word laid out by hi_plane_bit.
+ *   b = 2, 4: per row a natural b-bit stream (K*b/8 bytes), rows consecutive;
+ *   b = 3:    plane L (per row the natural 2-bit stream of the low 2 bits,
+ *             K/4 bytes) followed by plane H (per row K/8 bytes: per
+ *             32-channel block one little-endian 32-bit word laid out by
+ *             hi_plane_bit).
+ *   Every row of a plane is then cut into 16-byte units and unit u is stored
+ *   at unit (u XOR (n mod 8)) of the row (the units move only inside their
+ *   aligned 128-byte block).
  * Refinement codes: channel-major natural r-bit streams, R[c] holds rho[n][c]
  * for n = 0..N-1 (K rows of N*r/8 B). */
+static void store_row_units(uint8_t* dst_row, const uint8_t* natural, long bytes, long n) {
+  for (long u = 0; u < bytes / 16; u++) {
+    long to = u ^ (n % 8);
+    memcpy(dst_row + 16 * to, natural + 16 * u, 16);
+  }
+}
+
 OR_API void or_pack_weights(const uint8_t* qb, const uint8_t* rho, int N, int K, int b,
                             int r, uint8_t* base, uint8_t* refine) {
   size_t base_bytes = (size_t)N * K * b / 8;
   memset(base, 0, base_bytes);
   memset(refine, 0, (size_t)K * N * r / 8);
+  const long rowL = (long)K * (b == 3 ? 2 : b) / 8, rowH = K / 8;
+  uint8_t* lo = (uint8_t*)calloc((size_t)rowL, 1);
+  uint8_t* hi = (uint8_t*)calloc((size_t)rowH, 1);
   for (long n = 0; n < N; n++) {
+    memset(lo, 0, (size_t)rowL);
+    memset(hi, 0, (size_t)rowH);
     for (long c = 0; c < K; c++) {
       int q = qb[n * K + c];
       if (b == 2 || b == 4) {
-        put_bits(base, n * K + c, b, q);
+        put_bits(lo, c, b, q);
       } else { /* b == 3 */
-        put_bits(base, n * K + c, 2, q & 3);
-        uint8_t* hp = base + (size_t)N * K / 4 + (size_t)n * K / 8;
+        put_bits(lo, c, 2, q & 3);
         long blk = c / 32;
         int bit = hi_plane_bit((int)(c % 32));
-        hp[blk * 4 + bit / 8] |= (uint8_t)(((q >> 2) & 1) << (bit % 8));
+        hi[blk * 4 + bit / 8] |= (uint8_t)(((q >> 2) & 1) << (bit % 8));
       }
       put_bits(refine, c * N + n, r, rho[n * K + c]);
     }
+    store_row_units(base + (size_t)n * rowL, lo, rowL, n);
+    if (b == 3) store_row_units(base + (size_t)N * rowL + (size_t)n * rowH, hi, rowH, n);
   }
+  free(lo);
+  free(hi);
 }
 
 /* KV codes and refinements: pair-slot layout.  A little-endian 32-bit word

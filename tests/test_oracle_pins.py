@@ -194,22 +194,38 @@ def test_quant_kv_addressing(orc):
 
 
 def test_pack_weights_2bit_by_hand(orc):
-    qb = np.array([[0, 1, 2, 3, 3, 2, 1, 0] * 16], np.uint8)  # N=1, K=128
+    N, K = 64, 1024  # 256 bytes per row: 16 units of 16 bytes
+    qb = np.repeat(np.array([[0, 1, 2, 3, 3, 2, 1, 0] * 128], np.uint8), N, 0)
     rho = np.zeros_like(qb)
-    rho[0, 0] = 1
-    base, refine = orc.pack_weights(np.repeat(qb, 64, 0), np.repeat(rho, 64, 0), 2, 1)
+    rho[:, 0] = 1
+    base, refine = orc.pack_weights(qb, rho, 2, 1)
     # channel c at bits 2c: codes 0,1,2,3 -> 0b11_10_01_00 = 0xE4; 3,2,1,0 -> 0x1B
-    assert base[0] == 0xE4 and base[1] == 0x1B and base[32] == 0xE4
+    assert base[0] == 0xE4 and base[1] == 0x1B and base[256] == 0xE4
     # refinement: channel-major, row n at bit n (r=1): channel 0 has all 64 rows set
     assert (refine[:8] == 0xFF).all() and (refine[8:] == 0).all()
 
 
+def test_pack_weights_unit_permutation_by_hand(orc):
+    N, K = 16, 1024
+    qb = np.zeros((N, K), np.uint8)
+    qb[1, 0] = 1      # row 1, unit 0 -> unit 0 ^ 1 = 1: byte 16 of the row, bits 0-1
+    qb[9, 64] = 2     # row 9 (9 mod 8 = 1), channel 64 = bit 128 = unit 1 -> unit 0
+    qb[7, 1023] = 3   # row 7, bit 2046 = byte 255 (unit 15, bits 6-7) -> unit 8, byte 15
+    qb[12, 100] = 1   # row 12 (mod 8 = 4): bit 200 = byte 25 = unit 1, byte 9 -> unit 5
+    base, _ = orc.pack_weights(qb, np.zeros_like(qb), 2, 1)
+    rows = base.reshape(N, 256)
+    assert rows[1, 16] == 1 and rows[9, 0] == 2 << 0 and rows[7, 8 * 16 + 15] == 3 << 6
+    assert rows[12, 5 * 16 + 9] == 1 << 0
+    assert int(base.astype(np.int64).sum()) == 1 + 2 + (3 << 6) + 1
+
+
 def test_pack_weights_3bit_high_plane_by_hand(orc):
-    N, K = 64, 128
+    N, K = 64, 1024
     qb = np.zeros((N, K), np.uint8)
     qb[0, 5] = 4     # high bit only; channel 5 -> word 0 bit 8*1+1 = 9
     qb[0, 20] = 7    # channel 20 -> 16+4 -> bit 8*1+4+0 = 12; low bits 3
     qb[0, 32 + 31] = 4  # block 1, channel 31 -> 15 -> bit 8*3+4+3 = 31
+    qb[3, 5] = 4     # row 3: word 0 of its high plane is unit 0 -> unit 3
     base, _ = orc.pack_weights(qb, np.zeros_like(qb), 3, 1)
     lo, hi = base[:N * K // 4], base[N * K // 4:]
     word0 = int.from_bytes(hi[0:4].tobytes(), "little")
@@ -217,7 +233,9 @@ def test_pack_weights_3bit_high_plane_by_hand(orc):
     assert word0 == (1 << 9) | (1 << 12)
     assert word1 == (1 << 31)
     assert lo[20 // 4] == 3 << (2 * (20 % 4))
-    assert (hi[8:] == 0).all()
+    row3 = hi[3 * 128:4 * 128]
+    assert int.from_bytes(row3[48:52].tobytes(), "little") == 1 << 9
+    assert int(hi[8:].astype(np.int64).sum()) == (1 << 1)  # only row 3's bit 9 (byte 49, bit 1)
 
 
 def test_pack_kv_by_hand(orc):
