@@ -75,6 +75,11 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the timed region starts once the sampler reports (nvidia-smi takes
+            # a moment to start), so that its samples cover the region
+            t_end = time.time() + 3.0
+            while not self.rows and time.time() < t_end:
+                time.sleep(0.005)
         except Exception:
             self.proc = None
         return self
@@ -495,6 +500,9 @@ def run_ours(args, rank, world, local_rank):
     hbm_peak, peak_kind = peaks()
     dec, hidden = build_decoder(BATCH, T_CTX, device)
     cfg = dec.cfg
+    # the headline step stages every selected row over the host link each step
+    # (the faster schedule here); the row cache is measured as a variant
+    dec.use_cache = False
     # every step decodes a different input: a pool of hidden states whose
     # outlier channels persist from token to token
     pool = inputs.decoder_hidden_pool(SEED * 100000 + 97, POOL, BATCH, cfg.hidden, device=device)
@@ -516,7 +524,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
-        st0 = dec.cache_stats()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(local_rank) as clocks:
             e0.record(s)
@@ -525,7 +532,6 @@ def run_ours(args, rank, world, local_rank):
                 g.replay()
             e1.record(s)
             torch.cuda.synchronize()
-        st1 = dec.cache_stats()
         if world > 1:
             torch.distributed.barrier()
         ms = e0.elapsed_time(e1) / args.steps
@@ -549,23 +555,27 @@ def run_ours(args, rank, world, local_rank):
         roof = gemv_roofline(dec, max(3, args.steps // 5), max(3, args.warmup), hbm_peak)
         ms_base = base_only_ms(dec, hidden, s, max(3, args.steps // 2), args.warmup)
         ms_local = step_variant_ms(dec, hidden, s, sub, args.warmup, feed, lead=0, lag=0)
-        c0 = dec.cache_stats()
+        dec.use_cache = True
+        st0 = dec.cache_stats()
+        ms_cache = step_variant_ms(dec, hidden, s, sub, args.warmup, feed)
+        st1 = dec.cache_stats()
         ms_skip = step_variant_ms(dec, hidden, s, sub, args.warmup, feed, skip_missing=True)
         c1 = dec.cache_stats()
         dec.use_cache = False
-        ms_nocache = step_variant_ms(dec, hidden, s, sub, args.warmup, feed)
-        dec.use_cache = True
         kv_roof = kv_step_roofline(dec, sub, args.warmup, hbm_peak)
         lm_roof = lm_head_roofline(dec, sub, args.warmup, hbm_peak)
     delta = lambda a, b, i: sum(b[n][i] - a.get(n, (0, 0))[i] for n in b)
+    # the cached variant's steps: one eager step, the warm-up and the timed
+    # replays of its own graph (the hit rate includes the cold start)
+    cache_steps = 1 + args.warmup + sub
     hits, misses = delta(st0, st1, 0), delta(st0, st1, 1)
-    skip_hits, skip_misses = delta(c0, c1, 0), delta(c0, c1, 1)
+    skip_hits, skip_misses = delta(st1, c1, 0), delta(st1, c1, 1)
     miss_bytes = sum((st1[n][1] - st0.get(n, (0, 0))[1]) * dec.row_bytes[n] for n in st1)
     roof["peak_kind"] = kv_roof["peak_kind"] = lm_roof["peak_kind"] = peak_kind
-    ms, ms_e2e, ms_base, ms_local, ms_skip, ms_nocache = max_over_ranks(
-        [ms, ms_e2e, ms_base, ms_local, ms_skip, ms_nocache], world, device)
+    ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache = max_over_ranks(
+        [ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache], world, device)
     step_bytes = decode_step_bytes(cfg, BATCH, T_CTX)
-    pcie_per_step = miss_bytes / args.steps  # host-link bytes per step: the missing rows
+    pcie_per_step = staged_bytes(cfg, BATCH)  # host-link bytes per step: every selected row
     io_bytes = (hidden.numel() * 2, dec.logits.numel() * 4)
     del dec, hidden
     torch.cuda.empty_cache()
@@ -601,16 +611,18 @@ def run_ours(args, rank, world, local_rank):
         "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms / 1e3) / 1e9,
                 "frac_of_measured_copy": step_bytes / (ms / 1e3) / 1e9 / hbm_peak,
                 "frac_of_8tbs": step_bytes / (ms / 1e3) / 1e9 / 8000.0,
-                "pcie_bytes_per_step": pcie_per_step, "pcie_bytes_per_step_without_cache": staged_bytes(cfg, BATCH)},
-        "row_cache": {"capacity": f"{CACHE_ROWS} x the selected channels per (layer, projection)",
-                      "hit_rate": hits / max(1, hits + misses), "hits_per_step": hits / args.steps,
-                      "misses_per_step": misses / args.steps,
+                "pcie_bytes_per_step": pcie_per_step},
+        "row_cache": {"what": "the same step with selected rows cached on the device across steps "
+                              "(only missing rows cross the host link), its own graph",
+                      "capacity": f"{CACHE_ROWS} x the selected channels per (layer, projection)",
+                      "ms_per_step": ms_cache,
+                      "hit_rate": hits / max(1, hits + misses), "hits_per_step": hits / cache_steps,
+                      "misses_per_step": misses / cache_steps,
+                      "pcie_bytes_per_step": miss_bytes / cache_steps,
                       "inputs": f"{POOL} hidden states cycled, N(0,1) with 1% channels x20 fixed across them",
                       "skip_on_miss": {"ms_per_step": ms_skip, "hit_rate": skip_hits / max(1, skip_hits + skip_misses),
                                        "what": "misses stay at base precision this step; their rows land in "
-                                               "the cache for later steps"},
-                      "without_cache": {"ms_per_step": ms_nocache,
-                                        "what": "every selected row read over the host link every step"}},
+                                               "the cache for later steps"}},
         "roofline": {**roof, "traffic": roof["bytes_per_launch"] * GEMV_TRAFFIC_PER_BYTE},
         "e2e": {"value": job_us_per_token(ms_e2e, world), "unit": UNIT,
                 "h2d_bytes_per_step": io_bytes[0], "d2h_bytes_per_step": io_bytes[1]},
