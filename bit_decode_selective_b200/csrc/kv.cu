@@ -660,6 +660,20 @@ __global__ void __launch_bounds__(kSelThreads) kv_score_kernel(SelArgs a) {
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
   pdl_wait();  // the base pass (logits, records, zeroed histogram) is complete
+  // the CTA's logits are loaded first: their latency overlaps the statistics
+  const int t0 = blockIdx.x * kSelTok, t1 = min(a.T, t0 + kSelTok);
+  constexpr int U = kSelTok / kSelThreads;
+  float l[GQP][U];
+  {
+    const float* lg = a.logits + hq0 * a.T;
+#pragma unroll
+    for (int h = 0; h < GQP; h++)
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int t = t0 + tid + kSelThreads * u;
+        l[h][u] = (h < gq && t < t1) ? lg[(long)h * a.T + t] : -INFINITY;
+      }
+  }
   if (warp < gq) {
     float M, Z;
     head_stats(a.part + (hq0 + warp) * a.nrec * a.rec, a.nrec, a.rec, lane, M, Z);
@@ -676,17 +690,6 @@ __global__ void __launch_bounds__(kSelThreads) kv_score_kernel(SelArgs a) {
   float* sc = a.scores + head * a.Tp;
   float* sco = a.scores_out ? a.scores_out + head * a.T : nullptr;
   {
-    const int t0 = blockIdx.x * kSelTok, t1 = min(a.T, t0 + kSelTok);
-    const float* lg = a.logits + hq0 * a.T;
-    constexpr int U = kSelTok / kSelThreads;
-    float l[GQP][U];
-#pragma unroll
-    for (int h = 0; h < GQP; h++)
-#pragma unroll
-      for (int u = 0; u < U; u++) {
-        const int t = t0 + tid + kSelThreads * u;
-        l[h][u] = (h < gq && t < t1) ? lg[(long)h * a.T + t] : -INFINITY;
-      }
 #pragma unroll
     for (int u = 0; u < U; u++) {
       const int t = t0 + tid + kSelThreads * u;
@@ -733,25 +736,26 @@ __global__ void __launch_bounds__(kSelThreads) kv_pick_kernel(SelArgs a) {
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
   pdl_wait();  // every score and the complete histogram
+  const int T = a.T;
+  const float* sc = a.scores + head * a.Tp;
+  // the CTA's scores (four consecutive tokens per thread) are loaded first:
+  // their latency overlaps the histogram's load and the bucket search
+  const int t0 = blockIdx.x * kSelTok + 4 * tid;
+  uint32_t key[4] = {0u, 0u, 0u, 0u};
+  if (t0 + 4 <= a.Tp) {
+    const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + t0));
+    key[0] = __float_as_uint(f.x), key[1] = __float_as_uint(f.y);
+    key[2] = __float_as_uint(f.z), key[3] = __float_as_uint(f.w);
+  }
   int* gh = a.ctl + head * kCtl;
   for (int i = tid; i < kBins1; i += kSelThreads) sh.hist[i] = __ldcg(gh + i);
   if (tid < kSelTok / 32) sh.words[tid] = 0u;
   __syncthreads();
   int kneed;
   const uint32_t b1 = (uint32_t)find_bucket<kSelThreads>(sh.hist, kBins1, a.k_tok, sh.ws, sh.res, &kneed);
-  const int T = a.T;
-  const float* sc = a.scores + head * a.Tp;
   uint2* cl = a.cand + head * kCandCap;
   int* ncand_g = gh + kBins1 + 3;
   {
-    // four consecutive tokens per thread
-    const int t0 = blockIdx.x * kSelTok + 4 * tid;
-    uint32_t key[4] = {0u, 0u, 0u, 0u};
-    if (t0 + 4 <= a.Tp) {
-      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + t0));
-      key[0] = __float_as_uint(f.x), key[1] = __float_as_uint(f.y);
-      key[2] = __float_as_uint(f.z), key[3] = __float_as_uint(f.w);
-    }
     uint32_t m = 0;
     int nc = 0;
 #pragma unroll
