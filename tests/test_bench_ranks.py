@@ -33,7 +33,7 @@ def _rank_main(rank, world, port, out):
 @pytest.mark.timeout(120)
 def test_max_over_ranks_gloo_world_2():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
     assert out[0] == out[1] == [5.0, 7.0, 3.0]
 
