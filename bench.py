@@ -728,7 +728,8 @@ def run_case(name):
     """A few launches of one hot kernel on a small case, for profiler captures
     (no timing): `gemv` = the gate/up-shaped refined GEMV (28,672 x 4,096,
     2 + 2 bits, k = 32 per 1,024), base then refined with a given selection,
-    three times; `kv` = score-select-attend over 8 KV heads x 32,768 tokens,
+    three times; `gemv8` = the same at batch 8 (the tensor-core form), three
+    times; `kv` = score-select-attend over 8 KV heads x 32,768 tokens,
     top-512, three times; `step` = three eager decode steps of the benchmarked
     workload (for the launch list)."""
     import torch
@@ -741,6 +742,20 @@ def run_case(name):
         dec.use_cache = False  # the benchmarked schedule
         for _ in range(3):
             dec.step(hidden)
+        torch.cuda.synchronize()
+        print(json.dumps({"case": name, "ok": True}), flush=True)
+        return
+    if name == "gemv8":
+        # the batch-8 form: tensor-core base products (two launches of four
+        # rows) and the correction kernel, three times
+        w = inputs.torch_normal((28672, 4096), 0.02, 1)
+        qw = QuantWeights.pack(w, 2, 2, 128)
+        del w
+        x = inputs.torch_normal((8, 4096), 1.0, 2, dtype=torch.float16)
+        y = torch.empty(8, 28672, device="cuda")
+        sel = select_channels(x, 1024, 32)
+        for _ in range(3):
+            qw.gemv(x, 1024, 32, y=y, sel_in=sel)
         torch.cuda.synchronize()
         print(json.dumps({"case": name, "ok": True}), flush=True)
         return
@@ -776,7 +791,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["gemv", "kv", "step"], default=None,
+    ap.add_argument("--case", choices=["gemv", "gemv8", "kv", "step"], default=None,
                     help="run a few launches of one kernel for a profiler capture instead")
     args = ap.parse_args()
     if args.case:
