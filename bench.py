@@ -176,7 +176,7 @@ def count_kernels(graph) -> int | None:
 # (`bench.py --case gemv`: the 28,672 x 4,096 launch, 2 + 2 bits, k = 32 per
 # 1,024) over that launch's algorithmic bytes; traffic grows in proportion to the codes a launch streams,
 # so a launch's traffic is its bytes times this.
-GEMV_TRAFFIC_PER_BYTE = 33997568 / 34071040
+GEMV_TRAFFIC_PER_BYTE = 34000128 / 34071040
 
 
 def gemv_roofline(dec, steps, warmup, hbm_peak):
