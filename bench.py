@@ -448,7 +448,7 @@ def kv_step_roofline(dec, steps, warmup, hbm_peak):
     nbytes = bytemodel.kv_attention_bytes(dec.T + 1, cfg.h_kv, cfg.h_q, cfg.d, cfg.kv_bits, cfg.kv_refine, 32,
                                           cfg.k_tok, dec.B)
     ach = nbytes / (ms / 1e3) / 1e9
-    return {"kernel": "kv_base_kernel + kv_post_kernel (score, select, refined attention; 1 call per layer)",
+    return {"kernel": "kv_base_kernel + kv_score_kernel + kv_pick_kernel + kv_refine_kernel (base pass, scoring, selection, refined attention; 1 call per layer)",
             "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
             "bytes_per_launch": nbytes, "us_per_launch": ms * 1e3, "launches_per_step": cfg.n_layers}
 
