@@ -294,30 +294,50 @@ static void value_place(int tt, int d, int* l, int* p, int* second) {
   *p = 16 * h + 2 * m + e;
 }
 
-static void pack_keys(const uint8_t* x, int w, int B, int H, int T, int Tmax, int D, uint8_t* out) {
-  size_t tok_bytes = (size_t)16 * w;
-  memset(out, 0, (size_t)B * H * Tmax * tok_bytes);
+/* Bits [shift, shift + w) of every code go to a w-bit pair-slot plane that
+ * starts `off` bytes into each token's (keys) or tile's (values) `stride`
+ * bytes of the output. */
+static void pack_keys(const uint8_t* x, int w, int shift, size_t stride, size_t off, int B, int H, int T,
+                      int Tmax, int D, uint8_t* out) {
   for (long bh = 0; bh < (long)B * H; bh++)
     for (long t = 0; t < T; t++)
       for (int d = 0; d < D; d++) {
         int c, p, second;
         key_place(d, &c, &p, &second);
-        uint8_t* chunk = out + ((size_t)bh * Tmax + t) * tok_bytes + (size_t)c * 4 * w;
-        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d]);
+        uint8_t* chunk = out + ((size_t)bh * Tmax + t) * stride + off + (size_t)c * 4 * w;
+        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d] >> shift);
       }
 }
 
-static void pack_values(const uint8_t* x, int w, int B, int H, int T, int Tmax, int D, uint8_t* out) {
-  size_t tile_bytes = (size_t)256 * w;
-  memset(out, 0, (size_t)B * H * (Tmax / 16) * tile_bytes);
+static void pack_values(const uint8_t* x, int w, int shift, size_t stride, size_t off, int B, int H, int T,
+                        int Tmax, int D, uint8_t* out) {
   for (long bh = 0; bh < (long)B * H; bh++)
     for (long t = 0; t < T; t++)
       for (int d = 0; d < D; d++) {
         int l, p, second;
         value_place((int)(t % 16), d, &l, &p, &second);
-        uint8_t* chunk = out + ((size_t)bh * (Tmax / 16) + t / 16) * tile_bytes + (size_t)l * 8 * w;
-        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d]);
+        uint8_t* chunk = out + ((size_t)bh * (Tmax / 16) + t / 16) * stride + off + (size_t)l * 8 * w;
+        put_pair(chunk, w, p, second, x[((size_t)bh * T + t) * D + d] >> shift);
       }
+}
+
+/* One kind (keys or values) of w-bit codes.  w = 2 and 4 divide the 16 bits of
+ * a word half and use the pair-slot layout directly; 3-bit codes are stored as
+ * two planes of that layout, the low two bits of every code (w = 2) followed by
+ * the high bit (w = 1): 32 + 16 bytes per key token, 512 + 256 bytes per value
+ * tile. */
+static void pack_kind(const uint8_t* x, int which, int w, int B, int H, int T, int Tmax, int D,
+                      uint8_t* out) {
+  const size_t stride = (size_t)(which == 0 ? 16 : 256) * w;
+  memset(out, 0, (size_t)B * H * (which == 0 ? Tmax : Tmax / 16) * stride);
+  void (*pk)(const uint8_t*, int, int, size_t, size_t, int, int, int, int, int, uint8_t*) =
+      which == 0 ? pack_keys : pack_values;
+  if (w == 3) {
+    pk(x, 2, 0, stride, 0, B, H, T, Tmax, D, out);
+    pk(x, 1, 2, stride, (size_t)(which == 0 ? 32 : 512), B, H, T, Tmax, D, out);
+  } else {
+    pk(x, w, 0, stride, 0, B, H, T, Tmax, D, out);
+  }
 }
 
 /* which = 0: keys, 1: values.  Writes base (b bits) and refinement (r bits)
@@ -325,13 +345,8 @@ static void pack_values(const uint8_t* x, int w, int B, int H, int T, int Tmax, 
  * head are written, everything else is zero. */
 OR_API void or_pack_kv(const uint8_t* qb, const uint8_t* rho, int which, int B, int H, int T,
                        int Tmax, int D, int b, int r, uint8_t* base, uint8_t* refine) {
-  if (which == 0) {
-    pack_keys(qb, b, B, H, T, Tmax, D, base);
-    pack_keys(rho, r, B, H, T, Tmax, D, refine);
-  } else {
-    pack_values(qb, b, B, H, T, Tmax, D, base);
-    pack_values(rho, r, B, H, T, Tmax, D, refine);
-  }
+  pack_kind(qb, which, b, B, H, T, Tmax, D, base);
+  pack_kind(rho, which, r, B, H, T, Tmax, D, refine);
 }
 
 /* ------------------------------------------------------------------------- */

@@ -260,6 +260,33 @@ def test_pack_kv_by_hand(orc):
     assert vr1[28 * 8 + 2] == 1 << 3 and vr1.sum() == 1 << 3
 
 
+def test_pack_kv_3bit_planes_by_hand(orc):
+    # 3-bit codes: a plane of the low two bits (2-bit layout) followed by a
+    # plane of the high bits (1-bit layout); 48 bytes per key token, 768 per
+    # value tile.
+    qb = np.zeros((1, 2, 3, 128), np.uint8)
+    rho = np.zeros_like(qb)
+    qb[0, 1, 2, 3] = 6   # low bits 2, high bit 1
+    qb[0, 0, 1, 31] = 5  # low bits 1, high bit 1
+    kb, _ = orc.pack_kv(qb, rho, 0, 3, 2, t_max=16)
+    assert kb.size == 2 * 16 * 48
+    # token slot 18, dim 3: chunk 1, pair 0, second code.  Low plane: chunk at
+    # byte 8, bit 16; high plane: byte 32 + 4, bit 16.
+    assert kb[18 * 48 + 8 + 2] == 2 and kb[18 * 48 + 32 + 4 + 2] == 1
+    # token slot 1, dim 31: chunk 3, pair 3, second.  Low: byte 24, bit 16 + 6;
+    # high: byte 32 + 12, bit 16 + 3.
+    assert kb[48 + 24 + 2] == 1 << 6 and kb[48 + 44 + 2] == 1 << 3
+    assert int(kb.astype(np.int64).sum()) == 2 + 1 + 64 + 8
+    vb, _ = orc.pack_kv(qb, rho, 1, 3, 2, t_max=16)
+    assert vb.size == 2 * 768
+    # head 1 tile, token 2, dim 3: chunk 13, pair 0, first code.  Low plane:
+    # 16-byte chunks; high plane at byte 512, 8-byte chunks.
+    assert vb[768 + 13 * 16] == 2 and vb[768 + 512 + 13 * 8] == 1
+    # head 0 tile, token 1, dim 31: chunk 28, pair 3, second code
+    assert vb[28 * 16 + 2] == 1 << 6 and vb[512 + 28 * 8 + 2] == 1 << 3
+    assert int(vb.astype(np.int64).sum()) == 2 + 1 + 64 + 8
+
+
 # ---------------------------------------------------------------------------
 # chunked channel selection: brute force with forced ties
 
