@@ -369,17 +369,17 @@ def gemv_config(name, shapes, b, r, seed, steps, warmup, hbm_peak, device):
     return rec
 
 
-def kv_config(name, t, k_tok, seed, steps, warmup, hbm_peak, device):
-    """Configs 3 and 4: score + select + refined attention (sf_kv_attend_selective)
-    over t cached tokens, 8 KV / 32 query heads, 2 + 2 bits, top-k_tok per KV
-    head; base attention alone (k_tok = 0) beside it.  Rotating caches span
-    more than 3x L2."""
+def kv_config(name, t, k_tok, seed, steps, warmup, hbm_peak, device, b=2, r=2):
+    """Configs 3 and 4 (and the 3-bit base variant): score + select + refined
+    attention (sf_kv_attend_selective) over t cached tokens, 8 KV / 32 query
+    heads, b + r bits, top-k_tok per KV head; base attention alone (k_tok = 0)
+    beside it.  Rotating caches span more than 3x L2."""
     import torch
 
     from bit_decode_selective_b200 import bytemodel, inputs
     from bit_decode_selective_b200.ops import KVCache
 
-    per_copy = bytemodel.kv_attention_bytes(t, 8, 32, 128, 2, 2, 32, k_tok)
+    per_copy = bytemodel.kv_attention_bytes(t, 8, 32, 128, b, r, 32, k_tok)
     copies = max(2, -(-ROTATE_BYTES // per_copy))
     k = inputs.torch_normal((1, 8, t, 128), 1.0, seed * 10 + 1, device=device, dtype=torch.float16)
     v = inputs.torch_normal((1, 8, t, 128), 1.0, seed * 10 + 2, device=device, dtype=torch.float16)
@@ -387,12 +387,12 @@ def kv_config(name, t, k_tok, seed, steps, warmup, hbm_peak, device):
     for h in range(8):
         ch = torch.randperm(128, generator=g)[:4].to(device)
         k[:, h, :, ch] *= 10
-    c0 = KVCache(1, 8, t, 2, 2, device=device)
+    c0 = KVCache(1, 8, t, b, r, device=device)
     c0.pack_tokens(k, v, 0)
     del k, v
     caches = [c0]
     for _ in range(copies - 1):
-        c = KVCache(1, 8, t, 2, 2, device=device)
+        c = KVCache(1, 8, t, b, r, device=device)
         for nm in ("kb", "kr", "vb", "vr", "ksz", "vsz"):
             getattr(c, nm).copy_(getattr(c0, nm))
         caches.append(c)
@@ -591,6 +591,9 @@ def run_ours(args, rank, world, local_rank):
                              8192, 256, 2, sub, args.warmup, hbm_peak, device),
         "4_kv_128k": kv_config("refined KV attention, T=131072, 2+2 bits, top-1024 per KV head, split-K + LSE merge",
                                131072, 1024, 3, sub, args.warmup, hbm_peak, device),
+        "kv_32k_3bit": kv_config("refined KV attention, 32/8 heads x 128, T=32768, 3-bit base + 2 refinement bits, "
+                                 "top-512 per KV head (the pages' other KV base width)",
+                                 32768, 512, 6, sub, args.warmup, hbm_peak, device, b=3, r=2),
     }
     dec8, hidden8 = build_decoder(8, T_CTX, device)
     ms8 = graph_ms(lambda: dec8.step(hidden8), sub, args.warmup, torch.cuda.Stream(device=device))

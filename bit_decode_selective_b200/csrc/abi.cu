@@ -65,7 +65,7 @@ sf_status sf_kv_bytes(int batch, int h_kv, int d, int t_max, int b, int r, int g
                       size_t* code_bytes, size_t* refine_bytes, size_t* sz_bytes) {
   SF_REQUIRE(batch > 0 && h_kv > 0 && d > 0 && t_max > 0 && group > 0 && d % group == 0,
              "bad KV shape");
-  SF_REQUIRE((b == 2 || b == 4) && (r == 1 || r == 2), "bad KV bits b=%d r=%d", b, r);
+  SF_REQUIRE(b >= 2 && b <= 4 && (r == 1 || r == 2), "bad KV bits b=%d r=%d", b, r);
   size_t tok = (size_t)batch * h_kv * t_max;
   if (code_bytes) *code_bytes = tok * d * b / 8;
   if (refine_bytes) *refine_bytes = tok * d * r / 8;

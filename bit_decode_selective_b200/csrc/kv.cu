@@ -113,6 +113,80 @@ __device__ __forceinline__ uint32_t pair_of(const Words<W> (&ws)[N], int p) {
   return pair_at<W>(x.w, x.l2, x.r, p % per);
 }
 
+// 3-bit codes are two planes: the low two bits in a 2-bit pair-slot word, the
+// high bit in a 1-bit pair-slot word (16 slots; slot j at bits j and 16 + j).
+// The high-bit word is kept as given, shifted left by 3 and right by 6, so that
+// every slot's bit sits at an offset bh in [3, 9].
+struct HiWord {
+  uint32_t w, l3, r6;
+  __device__ __forceinline__ void set(uint32_t x) {
+    w = x;
+    l3 = x << 3;
+    r6 = x >> 6;
+  }
+};
+
+// Pair p of 3-bit codes as an exact half2 of centred codes c - 3.5: low bits
+// from slot p % 8 of lo[p / 8], high bit from slot p % 16 of hi[p / 16].
+// The low pair is placed at b2 as in pair_at<2> and rescaled with an offset
+// that also removes 4096 * 2^-bh; the second fused multiply-add adds the high
+// pair, 1024 + hi 2^bh, times 4 * 2^-bh.  Every intermediate is a multiple of
+// 0.5 below 1024 in magnitude, so both steps are exact in fp16.
+template <int NL, int NH>
+__device__ __forceinline__ uint32_t pair3_of(const Words<2> (&lo)[NL], const HiWord (&hi)[NH], int p) {
+  const Words<2>& x = lo[p / 8];
+  const int bit = 2 * (p % 8);
+  const bool left = bit < 2, right = !left && bit + 2 > 10;
+  const int b2 = left ? bit + 2 : right ? bit - 8 : bit;
+  const uint32_t src = left ? x.l2 : right ? x.r : x.w;
+  const uint32_t vl = (src & ((3u << b2) * 0x00010001u)) | 0x64006400u;  // 1024 + lo 2^b2 per half
+  const HiWord& y = hi[p / 16];
+  const int hb = p % 16;
+  const int bh = hb < 3 ? hb + 3 : hb < 10 ? hb : hb - 6;
+  const uint32_t hsrc = hb < 3 ? y.l3 : hb < 10 ? y.w : y.r6;
+  const uint32_t vh = (hsrc & ((1u << bh) * 0x00010001u)) | 0x64006400u;  // 1024 + hi 2^bh per half
+  // offset -(1024 2^-b2 + 4096 2^-bh + 3.5) = -n / 2 with n < 2048 an integer:
+  // fp16 exponent field e + 14 and mantissa (n - 2^e) 2^(10-e), e = floor(log2 n)
+  const uint32_t n = (2048u >> b2) + (8192u >> bh) + 7u;
+  const int e = 31 - __clz(n);
+  const uint32_t off = (0x8000u | ((uint32_t)(e + 14) << 10) | ((n - (1u << e)) << (10 - e))) * 0x00010001u;
+  const uint32_t sc = (uint32_t)((15 - b2) << 10) * 0x00010001u;  // 2^-b2
+  const uint32_t sh = (uint32_t)((17 - bh) << 10) * 0x00010001u;  // 4 * 2^-bh
+  __half2 c = __hfma2(*reinterpret_cast<const __half2*>(&vl), *reinterpret_cast<const __half2*>(&sc),
+                      *reinterpret_cast<const __half2*>(&off));
+  c = __hfma2(*reinterpret_cast<const __half2*>(&vh), *reinterpret_cast<const __half2*>(&sh), c);
+  return *reinterpret_cast<uint32_t*>(&c);
+}
+
+// The code words of one chunk of PAIRS pairs (a key token's chunk: 16; a value
+// tile's chunk: 32) in registers, B-bit codes.  load() takes the chunk's words
+// in the w = B layout (B = 3: its 2-bit plane words, and its 1-bit plane words
+// in hi).
+template <int B, int PAIRS>
+struct ChunkCodes {
+  static constexpr int NW = PAIRS * B / 16;
+  Words<B> w[NW];
+  __device__ __forceinline__ void load(const uint32_t* lo, const uint32_t*) {
+#pragma unroll
+    for (int i = 0; i < NW; i++) w[i].set(lo[i]);
+  }
+  __device__ __forceinline__ uint32_t pair(int p) const { return pair_of<B>(w, p); }
+};
+
+template <int PAIRS>
+struct ChunkCodes<3, PAIRS> {
+  static constexpr int NL = PAIRS / 8, NH = PAIRS / 16;
+  Words<2> lo[NL];
+  HiWord hi[NH];
+  __device__ __forceinline__ void load(const uint32_t* l, const uint32_t* h) {
+#pragma unroll
+    for (int i = 0; i < NL; i++) lo[i].set(l[i]);
+#pragma unroll
+    for (int i = 0; i < NH; i++) hi[i].set(h[i]);
+  }
+  __device__ __forceinline__ uint32_t pair(int p) const { return pair3_of(lo, hi, p); }
+};
+
 // ---------------------------------------------------------------------------
 // base pass
 
@@ -147,7 +221,7 @@ struct WarpSmem {
   static constexpr int bytes = ring + zf + ps;
 };
 
-// GQP: query heads per KV head padded to 4 or 8.  B: base bits (2 or 4).
+// GQP: query heads per KV head padded to 4 or 8.  B: base bits (2, 3 or 4).
 // four CTAs of 128 threads per SM at 120 registers (GQP = 4) leave kSideRegs
 // of the SM's registers free; GQP = 8 takes two CTAs of up to 255
 static_assert(65536 - 4 * 120 * kWarps * 32 >= kSideRegs, "base pass registers leave no room for a staging CTA");
@@ -221,10 +295,12 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
       uint8_t* st = wsm + (it % kStages) * St::bytes;
       const long slot = slot0 + tw0 + 16 * it;
 #pragma unroll
-      for (int c = 0; c < B / 2; c++) {
+      for (int c = 0; c < (B + 1) / 2; c++) {  // 16 B chunks of 16 tokens' keys (and the value tile)
         const int ci = lane + 32 * c;
-        cp_async16(st + 16 * ci, a.kb + slot * 16 * B + 16 * ci);
-        if (PV) cp_async16(st + St::kBytes + 16 * ci, a.vb + (slot / 16) * 256 * B + 16 * ci);
+        if (ci < 16 * B) {
+          cp_async16(st + 16 * ci, a.kb + slot * 16 * B + 16 * ci);
+          if (PV) cp_async16(st + St::kBytes + 16 * ci, a.vb + (slot / 16) * 256 * B + 16 * ci);
+        }
       }
       if (lane < 16)
         cp_async16(st + St::kBytes + St::vBytes + 16 * lane,
@@ -267,17 +343,17 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; i++) acc[j][i] = 0.f;
     {
+      // chunk tig of tokens gid and gid + 8 (3-bit codes: 2-bit plane words
+      // 2 tig, 2 tig + 1 and 1-bit plane word 8 + tig of the token)
       const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
-      Words<B> w0[B], w8[B];
-#pragma unroll
-      for (int i = 0; i < B; i++) {
-        w0[i].set(kc[gid * 4 * B + tig * B + i]);
-        w8[i].set(kc[(gid + 8) * 4 * B + tig * B + i]);
-      }
+      constexpr int LW = B == 3 ? 2 : B;
+      ChunkCodes<B, 16> w0, w8;
+      w0.load(kc + gid * 4 * B + tig * LW, kc + gid * 4 * B + 8 + tig);
+      w8.load(kc + (gid + 8) * 4 * B + tig * LW, kc + (gid + 8) * 4 * B + 8 + tig);
 #pragma unroll
       for (int s = 0; s < 8; s++) {
-        uint32_t a0 = pair_of<B>(w0, 2 * s), a1 = pair_of<B>(w8, 2 * s);
-        uint32_t a2 = pair_of<B>(w0, 2 * s + 1), a3 = pair_of<B>(w8, 2 * s + 1);
+        uint32_t a0 = w0.pair(2 * s), a1 = w8.pair(2 * s);
+        uint32_t a2 = w0.pair(2 * s + 1), a3 = w8.pair(2 * s + 1);
         mma16816(acc[s >> 1], a0, a1, a2, a3, qf[s][0], qf[s][1]);
       }
     }
@@ -391,17 +467,18 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
         }
         mt[2 * jj] = s0, mt[2 * jj + 1] = s1;
       }
+      // chunk `lane` of the value tile (3-bit codes: 2-bit plane words 4 lane ..
+      // 4 lane + 3, 1-bit plane words 128 + 2 lane, 128 + 2 lane + 1)
       const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + St::kBytes);
-      Words<B> vw[2 * B];
-#pragma unroll
-      for (int i = 0; i < 2 * B; i++) vw[i].set(vc[lane * 2 * B + i]);
+      ChunkCodes<B, 32> vw;
+      vw.load(vc + lane * 2 * (B == 3 ? 2 : B), vc + 128 + 2 * lane);
       // Each tile's product starts from zero and is folded into the running
       // sum with one fp32 FMA that also applies the softmax rescale: long
       // accumulation chains inside the tensor-core accumulator would drift.
 #pragma unroll
       for (int m = 0; m < 8; m++) {
-        uint32_t a0 = pair_of<B>(vw, 2 * m), a1 = pair_of<B>(vw, 2 * m + 1);
-        uint32_t a2 = pair_of<B>(vw, 16 + 2 * m), a3 = pair_of<B>(vw, 17 + 2 * m);
+        uint32_t a0 = vw.pair(2 * m), a1 = vw.pair(2 * m + 1);
+        uint32_t a2 = vw.pair(16 + 2 * m), a3 = vw.pair(17 + 2 * m);
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
           float t4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -954,12 +1031,15 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
 // and the query values of the group's heads there.
 template <int GQP, int B, int R>
 struct RefLane {
-  int kw[4], kbit[4], krw[4], krbit[4];
+  // 3-bit codes: (kw, kbit) in the 2-bit plane, (khw, khbit) in the 1-bit plane
+  int kw[4], kbit[4], khw[4], khbit[4], krw[4], krbit[4];
   float qv[GQP][4];
   __device__ __forceinline__ void init(const RefArgs& a, long hq0, int lane) {
 #pragma unroll
     for (int e = 0; e < 4; e++) {
-      key_pos(lane + 32 * e, B, kw[e], kbit[e]);
+      key_pos(lane + 32 * e, B == 3 ? 2 : B, kw[e], kbit[e]);
+      key_pos(lane + 32 * e, 1, khw[e], khbit[e]);
+      khw[e] += 8;
       key_pos(lane + 32 * e, R, krw[e], krbit[e]);
 #pragma unroll
       for (int h = 0; h < GQP; h++) qv[h][e] = h < a.gq ? h2f(a.q[(hq0 + h) * kD + lane + 32 * e]) : 0.f;
@@ -994,12 +1074,14 @@ __device__ __forceinline__ void refine_batch(const RefArgs& a, const RefLane<GQP
 #pragma unroll
     for (int e = 0; e < 4; e++) {
       const int d = lane + 32 * e;
-      int vw, vbit, vrw, vrbit;
-      value_pos(t & 15, d, B, vw, vbit);
+      int vrw, vrbit;
       value_pos(t & 15, d, R, vrw, vrbit);
-      wk[m][e] = (kp[rl.kw[e]] >> rl.kbit[e]) & bmask;
+      if constexpr (B == 3)
+        wk[m][e] = ((kp[rl.kw[e]] >> rl.kbit[e]) & 3u) | (((kp[rl.khw[e]] >> rl.khbit[e]) & 1u) << 2);
+      else
+        wk[m][e] = (kp[rl.kw[e]] >> rl.kbit[e]) & bmask;
       wkr[m][e] = (krp[rl.krw[e]] >> rl.krbit[e]) & rmask;
-      wv[m][e] = (vp[vw] >> vbit) & bmask;
+      wv[m][e] = value_code(vp, t & 15, d, B);
       wvr[m][e] = (vrp[vrw] >> vrbit) & rmask;
       zk[m][e] = zkp[e];
       zv[m][e] = zvp[e];
@@ -1285,6 +1367,10 @@ sf_status launch_base(const sf_kv* kv, const BaseArgs& a, bool pv, cudaStream_t 
     if (gqp == 4) return pv ? launch_base_t<4, 2, true>(a, kv->batch, s) : launch_base_t<4, 2, false>(a, kv->batch, s);
     return pv ? launch_base_t<8, 2, true>(a, kv->batch, s) : launch_base_t<8, 2, false>(a, kv->batch, s);
   }
+  if (kv->b == 3) {
+    if (gqp == 4) return pv ? launch_base_t<4, 3, true>(a, kv->batch, s) : launch_base_t<4, 3, false>(a, kv->batch, s);
+    return pv ? launch_base_t<8, 3, true>(a, kv->batch, s) : launch_base_t<8, 3, false>(a, kv->batch, s);
+  }
   if (gqp == 4) return pv ? launch_base_t<4, 4, true>(a, kv->batch, s) : launch_base_t<4, 4, false>(a, kv->batch, s);
   return pv ? launch_base_t<8, 4, true>(a, kv->batch, s) : launch_base_t<8, 4, false>(a, kv->batch, s);
 }
@@ -1320,6 +1406,13 @@ sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& 
   return SF_OK;
 }
 
+template <int GQP>
+void (*refine_kernel_for(int b, int r))(RefArgs) {
+  if (b == 2) return r == 2 ? kv_refine_kernel<GQP, 2, 2> : kv_refine_kernel<GQP, 2, 1>;
+  if (b == 3) return r == 2 ? kv_refine_kernel<GQP, 3, 2> : kv_refine_kernel<GQP, 3, 1>;
+  return r == 2 ? kv_refine_kernel<GQP, 4, 2> : kv_refine_kernel<GQP, 4, 1>;
+}
+
 // Refinement of the selected tokens and the merge (programmatic serialization).
 sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok, const Plan& P,
                         const float* logits, const float* part, const int32_t* sel, int* ctl, float* rpart,
@@ -1335,13 +1428,8 @@ sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int 
   a.stats_given = stats_given;
   a.out = out, a.out16 = out16;
   a.scale = 1.0f / sqrtf((float)kD);
-  void (*kern)(RefArgs);
-  if (a.gq <= 4)
-    kern = kv->b == 2 ? (kv->r == 2 ? kv_refine_kernel<4, 2, 2> : kv_refine_kernel<4, 2, 1>)
-                      : (kv->r == 2 ? kv_refine_kernel<4, 4, 2> : kv_refine_kernel<4, 4, 1>);
-  else
-    kern = kv->b == 2 ? (kv->r == 2 ? kv_refine_kernel<8, 2, 2> : kv_refine_kernel<8, 2, 1>)
-                      : (kv->r == 2 ? kv_refine_kernel<8, 4, 2> : kv_refine_kernel<8, 4, 1>);
+  void (*kern)(RefArgs) = refine_kernel_for<4>(kv->b, kv->r);
+  if (a.gq > 4) kern = refine_kernel_for<8>(kv->b, kv->r);
   SF_CUDA(launch_pdl(kern, dim3(P.parts, kv->h_kv, kv->batch), dim3(kRefThreads), 0, s, a));
   return SF_OK;
 }

@@ -153,15 +153,30 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
     const uint32_t q = (uint32_t)(Q >> R), rho = (uint32_t)(Q & ((1 << R) - 1));
     if (!is_value) {
       int word, bit;
-      key_pos(d, B, word, bit);
-      atomicOr(&a[word], q << bit);
+      if constexpr (B == 3) {  // low two bits: words 0..7; high bit: words 8..11
+        key_pos(d, 2, word, bit);
+        atomicOr(&a[word], (q & 3u) << bit);
+        key_pos(d, 1, word, bit);
+        atomicOr(&a[8 + word], (q >> 2) << bit);
+      } else {
+        key_pos(d, B, word, bit);
+        atomicOr(&a[word], q << bit);
+      }
       key_pos(d, R, word, bit);
       atomicOr(&a[4 * B + word], rho << bit);
     } else {
-      // half (gg, k) of the token's value words, slot `sl` of 16/w codes
+      // half (gg, k) of the token's value words, slot `sl` of 16/w codes; with
+      // 3-bit codes halves (gg, 0..1) of the low-bit plane and (gg, 2) of the
+      // high-bit plane
       const int m = d >> 4, within = d & 15, e = within >> 3, gg = within & 7;
-      atomicOr(&a[gg * B + (2 * m + e) / (16 / B)], q << (B * ((2 * m + e) % (16 / B))));
-      atomicOr(&a[8 * B + gg * R + (2 * m + e) / (16 / R)], rho << (R * ((2 * m + e) % (16 / R))));
+      const int pp = 2 * m + e;
+      if constexpr (B == 3) {
+        atomicOr(&a[gg * 3 + pp / 8], (q & 3u) << (2 * (pp % 8)));
+        atomicOr(&a[gg * 3 + 2], (q >> 2) << pp);
+      } else {
+        atomicOr(&a[gg * B + pp / (16 / B)], q << (B * (pp % (16 / B))));
+      }
+      atomicOr(&a[8 * B + gg * R + pp / (16 / R)], rho << (R * (pp % (16 / R))));
     }
   }
   __syncwarp();
@@ -176,7 +191,8 @@ __global__ void __launch_bounds__(kPackWarps * 32) pack_kv_kernel(PackArgs pa) {
       const bool base = i < 8 * B;
       const int W = base ? B : R, ii = base ? i : i - 8 * B;
       const int gg = ii / W, k = ii % W;
-      const int word = (4 * gg + c) * 2 * W + h * W + k;
+      int word = (4 * gg + c) * 2 * W + h * W + k;
+      if (B == 3 && base) word = k < 2 ? (4 * gg + c) * 4 + h * 2 + k : 128 + (4 * gg + c) * 2 + h;
       uint16_t* halves = reinterpret_cast<uint16_t*>((base ? codes + tile * 64 * B : refine + tile * 64 * R));
       halves[word * 2 + second] = (uint16_t)a[i];
     }
@@ -193,23 +209,14 @@ __global__ void unpack_kv_kernel(const uint32_t* __restrict__ codes,
   const long tok = idx / kHeadDim;
   const long bh = tok / t;
   const int tk = (int)(tok % t);
-  int word, bit;
   if (!is_value) {
     const long slot = bh * t_max + tk;
-    key_pos(d, b, word, bit);
-    qb[idx] = (uint8_t)((codes[slot * 4 * b + word] >> bit) & ((1u << b) - 1));
-    if (rho) {
-      key_pos(d, r, word, bit);
-      rho[idx] = (uint8_t)((refine[slot * 4 * r + word] >> bit) & ((1u << r) - 1));
-    }
+    qb[idx] = (uint8_t)key_code(codes + slot * 4 * b, d, b);
+    if (rho) rho[idx] = (uint8_t)key_code(refine + slot * 4 * r, d, r);
   } else {
     const long tile = bh * (t_max / 16) + tk / 16;
-    value_pos(tk & 15, d, b, word, bit);
-    qb[idx] = (uint8_t)((codes[tile * 64 * b + word] >> bit) & ((1u << b) - 1));
-    if (rho) {
-      value_pos(tk & 15, d, r, word, bit);
-      rho[idx] = (uint8_t)((refine[tile * 64 * r + word] >> bit) & ((1u << r) - 1));
-    }
+    qb[idx] = (uint8_t)value_code(codes + tile * 64 * b, tk & 15, d, b);
+    if (rho) rho[idx] = (uint8_t)value_code(refine + tile * 64 * r, tk & 15, d, r);
   }
 }
 
@@ -225,6 +232,8 @@ sf_status launch_pack(const PackArgs& pa, int kinds, cudaStream_t s) {
 sf_status launch_pack_any(const sf_kv* kv, const PackArgs& pa, int kinds, cudaStream_t s) {
   if (kv->b == 2 && kv->r == 2) return launch_pack<2, 2>(pa, kinds, s);
   if (kv->b == 2 && kv->r == 1) return launch_pack<2, 1>(pa, kinds, s);
+  if (kv->b == 3 && kv->r == 2) return launch_pack<3, 2>(pa, kinds, s);
+  if (kv->b == 3 && kv->r == 1) return launch_pack<3, 1>(pa, kinds, s);
   if (kv->b == 4 && kv->r == 2) return launch_pack<4, 2>(pa, kinds, s);
   return launch_pack<4, 1>(pa, kinds, s);
 }

@@ -10,6 +10,9 @@
 //   values -- per 16-token tile, 32 chunks l = 4g+c of 2w words; pair
 //             p = 16h+2m+e of chunk l: dim 16m+g+8e of tile tokens 2c+8h
 //             (first) and 2c+8h+1 (second).
+// 3-bit codes are two planes of this layout: the low two bits (w = 2), then the
+// high bit (w = 1) -- key words 0..7 and 8..11 of a token, value words 0..127
+// and 128..191 of a tile.
 #pragma once
 
 #include "common.cuh"
@@ -37,21 +40,31 @@ __host__ __device__ __forceinline__ void value_pos(int tt, int d, int w, int& wo
   bit = 16 * second + w * (p % per);
 }
 
-// Pair slot `slot` of word w as an exact half2 (first code in the low half).
-// Codes sitting at bit offsets that fit the fp16 mantissa are masked in
-// place; higher slots use the word shifted right by 8.
-template <int W, int SLOT>
-__device__ __forceinline__ uint32_t pair_h2(uint32_t w, uint32_t w_hi8) {
-  constexpr int BIT = W * SLOT;
-  constexpr bool SHIFT = BIT + W > 10;
-  constexpr int B2 = SHIFT ? BIT - 8 : BIT;
-  constexpr uint32_t MASK = (((1u << W) - 1u) << B2) * 0x00010001u;
-  uint32_t v = ((SHIFT ? w_hi8 : w) & MASK) | 0x64006400u;  // halves = 1024 + c * 2^B2
-  // c = v * 2^-B2 - 1024 * 2^-B2, exact in fp16
-  const __half2 sc = __float2half2_rn(1.0f / (float)(1 << B2));
-  const __half2 off = __float2half2_rn(-1024.0f / (float)(1 << B2));
-  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&v), sc, off);
-  return *reinterpret_cast<uint32_t*>(&r);
+// b-bit code of key element d of the token whose code words start at kp.
+__host__ __device__ __forceinline__ uint32_t key_code(const uint32_t* kp, int d, int b) {
+  int word, bit;
+  if (b != 3) {
+    key_pos(d, b, word, bit);
+    return (kp[word] >> bit) & ((1u << b) - 1u);
+  }
+  key_pos(d, 2, word, bit);
+  const uint32_t lo = (kp[word] >> bit) & 3u;
+  key_pos(d, 1, word, bit);
+  return lo | (((kp[8 + word] >> bit) & 1u) << 2);
+}
+
+// b-bit code of value element (tile token tt, dim d) of the tile whose code
+// words start at vp.
+__host__ __device__ __forceinline__ uint32_t value_code(const uint32_t* vp, int tt, int d, int b) {
+  int word, bit;
+  if (b != 3) {
+    value_pos(tt, d, b, word, bit);
+    return (vp[word] >> bit) & ((1u << b) - 1u);
+  }
+  value_pos(tt, d, 2, word, bit);
+  const uint32_t lo = (vp[word] >> bit) & 3u;
+  value_pos(tt, d, 1, word, bit);
+  return lo | (((vp[128 + word] >> bit) & 1u) << 2);
 }
 
 }  // namespace sf

@@ -120,7 +120,7 @@ sf_status check_kv(const sf_kv* kv) {
   SF_REQUIRE(kv->batch > 0 && kv->h_kv > 0 && kv->t_max > 0, "bad KV shape");
   SF_UNSUPPORTED(kv->d == 128 && kv->group == 32, "KV needs d=128, group=32 (got %d, %d)", kv->d,
                  kv->group);
-  SF_UNSUPPORTED(kv->b == 2 || kv->b == 4, "KV base bits %d not in {2,4}", kv->b);
+  SF_UNSUPPORTED(kv->b >= 2 && kv->b <= 4, "KV base bits %d not in {2,3,4}", kv->b);
   SF_UNSUPPORTED(kv->r == 1 || kv->r == 2, "KV refinement bits %d not in {1,2}", kv->r);
   SF_UNSUPPORTED(kv->t_max % 16 == 0, "t_max=%d must be a multiple of 16", kv->t_max);
   const void* ptrs[6] = {kv->kb, kv->kr, kv->vb, kv->vr, kv->ksz, kv->vsz};

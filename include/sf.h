@@ -209,7 +209,7 @@ SF_API sf_status sf_device_wait_timeouts(unsigned int* count, int reset);
 
 /* `batch` independent caches of h_kv heads with room for t_max tokens of d
  * elements, quantised per token in groups of `group` consecutive elements.
- *   d == 128, group == 32, b in {2,4}, r in {1,2}, t_max % 16 == 0.
+ *   d == 128, group == 32, b in {2,3,4}, r in {1,2}, t_max % 16 == 0.
  * Codes (w = b bits) and refinements (w = r bits) use a pair-slot layout laid
  * out for the tensor-core fragments that consume them: a little-endian 32-bit
  * word holds 16/w pairs of w-bit codes; pair slot j keeps its first code at
@@ -223,6 +223,11 @@ SF_API sf_status sf_device_wait_timeouts(unsigned int* count, int reset);
  *     p = 16*h + 2*m + e (h, e = 0..1, m = 0..7) of chunk l holds dim
  *     16*m + g + 8*e of tokens 16*u + 2*c + 8*h (first) and 16*u + 2*c + 8*h + 1
  *     (second).  [batch][h_kv][t_max/16][256*w bytes].
+ *   b = 3: 3 does not divide the 16 bits of a word half, so the codes are two
+ *     planes of this layout in the same 48 bytes per token (kb) or 768 bytes
+ *     per tile (vb): the low two bits of every code in the w = 2 layout (a key
+ *     token's words 0..7, a value tile's words 0..127), then the high bit in
+ *     the w = 1 layout (words 8..11, words 128..191).
  * ksz, vsz: [batch][h_kv][t_max][d/group][2] fp16 (s, m) per token and group. */
 typedef struct {
   int32_t batch, h_kv, d, t_max, b, r, group;

@@ -66,10 +66,13 @@ def test_validation_rejects_before_launch(L):
     # k_tok > t
     assert abi.sf_kv_score_select(ctypes.byref(kv), 10, ctypes.c_void_p(16), 32, 11, ctypes.c_void_p(16),
                                   None, None, None, 0, None) == abi.SF_ERR_INVALID_ARG
-    # 3-bit KV is not built
-    kv3 = abi.sf_kv(1, 8, 128, 8192, 3, 2, 32, 16, 16, 16, 16, 16, 16)
-    assert abi.sf_kv_pack_tokens(ctypes.byref(kv3), ctypes.c_void_p(16), None, 0, 1, None) \
+    # 5-bit KV bases are not built; 3-bit ones size as 48 bytes per key token
+    kv5 = abi.sf_kv(1, 8, 128, 8192, 5, 2, 32, 16, 16, 16, 16, 16, 16)
+    assert abi.sf_kv_pack_tokens(ctypes.byref(kv5), ctypes.c_void_p(16), None, 0, 1, None) \
         == abi.SF_ERR_UNSUPPORTED
+    s3 = [ctypes.c_size_t() for _ in range(3)]
+    assert abi.sf_kv_bytes(1, 8, 128, 16, 3, 2, 32, *[ctypes.byref(x) for x in s3]) == 0
+    assert s3[0].value == 8 * 16 * 48
     # too little workspace is reported, not overrun
     assert abi.sf_kv_attn_refined(ctypes.byref(kv), 100, ctypes.c_void_p(16), 32, None, 0, 4,
                                   ctypes.c_void_p(16), ctypes.c_void_p(16), 8, None) == abi.SF_ERR_WORKSPACE

@@ -273,7 +273,7 @@ def check_selection(sel, score, k_tok):
                 assert abs(score[bb, g, t] - kth) <= SEL_RTOL * kth, (bb, g, t, score[bb, g, t], kth)
 
 
-@pytest.mark.parametrize("b,r", [(2, 2), (2, 1), (4, 2), (4, 1)])
+@pytest.mark.parametrize("b,r", [(2, 2), (2, 1), (3, 2), (3, 1), (4, 2), (4, 1)])
 def test_kv_pack_bit_exact(b, r):
     cache, kc, vc, q = kv_setup(37, b, r, t_max=48, split_pack=True, batch=2, h_kv=2, h_q=8)
     torch.cuda.synchronize()
@@ -328,6 +328,15 @@ def test_kv_parity_batch_and_head_groups():
     kv_parity(300, 30, splits=(0, 5), h_kv=4, h_q=4, seed=12)            # 1 per KV head
 
 
+@pytest.mark.parametrize("T,k_tok,r,batch,h_kv,h_q,seed", [
+    (37, 5, 2, 1, 8, 32, 20),      # one partial tile, 4 query heads per KV head
+    (1000, 64, 2, 2, 4, 32, 21),   # 8 per KV head, two caches
+    (2049, 300, 1, 1, 2, 4, 22),   # ragged last tile, 2 per KV head, 1 refinement bit
+])
+def test_kv_parity_3bit_base(T, k_tok, r, batch, h_kv, h_q, seed):
+    kv_parity(T, k_tok, splits=(0, 3), b=3, r=r, batch=batch, h_kv=h_kv, h_q=h_q, seed=seed)
+
+
 def test_kv_base_only_and_all_selected():
     cache, kc, vc, q = kv_setup(300, batch=1, h_kv=8, h_q=32, seed=11)
     qd = cu(f16bits(q))
@@ -341,7 +350,7 @@ def test_kv_base_only_and_all_selected():
     assert np.abs(host(outT) - refT).max() <= ATTN_MAX_ABS and rel_l2(host(outT), refT) <= RTOL_L2
 
 
-@pytest.mark.parametrize("b,r,batch,t", [(2, 2, 1, 37), (4, 1, 2, 0), (2, 1, 3, 47)])
+@pytest.mark.parametrize("b,r,batch,t", [(2, 2, 1, 37), (4, 1, 2, 0), (2, 1, 3, 47), (3, 2, 2, 21)])
 def test_kv_append_rope_equals_rope_then_pack(b, r, batch, t):
     """The fused rotary embedding + append of the decode step's token stores
     the same codes, refinements and steps/offsets, and the same rotated q, as
