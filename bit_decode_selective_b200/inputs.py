@@ -55,6 +55,25 @@ def activation(rng: np.random.Generator, k: int, batch: int = 1, outlier_frac: f
     return out
 
 
+def calibration_activations(n: int, k: int, seed: int, structure_seed: int = 1000, rank: int = 16,
+                            noise: float = 0.5, outlier_frac: float = 0.01,
+                            outlier_scale: float = 20.0) -> np.ndarray:
+    """x[n][k] fp16 rows for fitting and checking refinement values: a rank-`rank`
+    factor part F L^T (F[n][rank] ~ N(0, 1), L[k][rank] ~ N(0, 1/rank), so each
+    channel's factor part has unit variance) plus N(0, noise) per element, with
+    the same round(outlier_frac * k) channels scaled by outlier_scale in every
+    row.  L and the outlier channels come from structure_seed, the rows from
+    seed: a calibration set and a held-out set share the structure and differ
+    in their rows."""
+    gs = np.random.default_rng(structure_seed)
+    L = gs.normal(0.0, 1.0, size=(k, rank)) / np.sqrt(rank)
+    out_ch = gs.choice(k, int(round(outlier_frac * k)), replace=False)
+    g = np.random.default_rng(seed)
+    x = g.normal(0.0, 1.0, size=(n, rank)) @ L.T + noise * g.normal(0.0, 1.0, size=(n, k))
+    x[:, out_ch] *= outlier_scale
+    return x.astype(np.float16)
+
+
 def kv_values(rng: np.random.Generator, h_kv: int, t: int, d: int, batch: int = 1,
               n_key_outliers: int = 4, key_scale: float = 10.0):
     """(k, v) each [batch][h_kv][t][d] fp16; per KV head n_key_outliers key channels scaled."""

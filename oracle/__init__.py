@@ -4,7 +4,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
 (and its ``--impl reference`` arm) may import this package.  The product path
 (``bit_decode_selective_b200``) never imports it, and the two share no code: the
 oracle is plain C in fp64 (``sf_oracle.c``), this module only marshals numpy
-arrays into it.
+arrays into it.  The one exception is ``fit.py``, the least-squares fit of
+weight refinement values, written in numpy fp64 with matrix products and a
+linear solve as its library steps.
 
 Each function cites the passage of the StrataFlux pages it follows; the C file
 states every reading taken where the pages are silent.
