@@ -50,6 +50,9 @@ _SIGNATURES = {
     "sf_pack_nested": ([c_void_p, POINTER(sf_wq), c_void_p], c_int),
     "sf_unpack_codes": ([POINTER(sf_wq), c_void_p, c_void_p, c_void_p], c_int),
     "sf_select_channels": ([c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p], c_int),
+    "sf_fit_refinements": ([c_void_p, POINTER(sf_wq), c_void_p, c_int, c_int, c_int, ctypes.c_double, c_void_p,
+                            c_void_p, c_size_t, c_void_p], c_int),
+    "sf_fit_refinements_workspace_bytes": ([c_int] * 5, c_size_t),
     "sf_gemv_refined": ([POINTER(sf_wq), c_void_p, c_int, c_int, c_int, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_gemv_workspace_bytes": ([POINTER(sf_wq), c_int, c_int, c_int], c_size_t),
@@ -137,6 +140,8 @@ sf_wq_bytes = _call("sf_wq_bytes")
 sf_pack_nested = _call("sf_pack_nested")
 sf_unpack_codes = _call("sf_unpack_codes")
 sf_select_channels = _call("sf_select_channels")
+sf_fit_refinements = _call("sf_fit_refinements")
+sf_fit_refinements_workspace_bytes = _call("sf_fit_refinements_workspace_bytes")
 sf_gemv_refined = _call("sf_gemv_refined")
 sf_gemv_workspace_bytes = _call("sf_gemv_workspace_bytes")
 sf_gemv_correction = _call("sf_gemv_correction")

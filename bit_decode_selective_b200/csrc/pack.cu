@@ -16,11 +16,6 @@ namespace sf {
 
 namespace {
 
-// Bit position of channel c (0..31) in the high-bit word of a 3-bit base block.
-__device__ __forceinline__ int hi_plane_bit(int c) {
-  return c < 16 ? 8 * (c >> 2) + (c & 3) : 8 * ((c - 16) >> 2) + 4 + ((c - 16) & 3);
-}
-
 // One thread per (row, group).  Refinement rows are channel-major, so several
 // threads share a 32-bit word of R: they OR their bits in atomically into a
 // zeroed buffer.
@@ -78,17 +73,7 @@ __global__ void unpack_weights_kernel(const uint32_t* __restrict__ base,
   long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;  // one element
   if (idx >= (long)N * K) return;
   long n = idx / K, c = idx % K;
-  int q;
-  if (b == 4) {
-    q = (base[(size_t)n * (K / 8) + wq_word((int)n, (int)(c / 8))] >> (4 * (c & 7))) & 15;
-  } else {
-    q = (base[(size_t)n * (K / 16) + wq_word((int)n, (int)(c / 16))] >> (2 * (c & 15))) & 3;
-    if (b == 3) {
-      const uint32_t* hp = base + (size_t)N * K / 16;
-      q |= ((hp[(size_t)n * (K / 32) + wq_word((int)n, (int)(c / 32))] >> hi_plane_bit((int)(c & 31))) & 1) << 2;
-    }
-  }
-  qb[idx] = (uint8_t)q;
+  qb[idx] = (uint8_t)packed_base_code(base, N, K, b, n, c);
   if (rho && R) {
     long rbit = (c * N + n) * r;
     rho[idx] = (uint8_t)((R[rbit >> 5] >> (rbit & 31)) & ((1u << r) - 1));

@@ -47,6 +47,21 @@ class QuantWeights:
         check(abi.sf_pack_nested(_p(w), ctypes.byref(q.desc), _stream()), "sf_pack_nested")
         return q
 
+    def fit_refinements(self, w: torch.Tensor, x_cal: torch.Tensor, chunk: int = 1024, kch: int = 32,
+                        alpha: float = 0.01, want_delta: bool = False, stream=None):
+        """Refit the refinement codes on calibration activations x_cal [n_cal][k]
+        (sf_fit_refinements); w is the fp32 matrix this one was packed from.
+        Returns the fitted corrections [n][k] fp64 when want_delta."""
+        assert w.dtype == torch.float32 and w.is_contiguous() and tuple(w.shape) == (self.n, self.k)
+        x_cal = _f16(x_cal)
+        n_cal = x_cal.shape[0]
+        nbytes = abi.sf_fit_refinements_workspace_bytes(self.n, self.k, n_cal, chunk, kch)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=w.device)
+        delta = torch.empty((self.n, self.k), dtype=torch.float64, device=w.device) if want_delta else None
+        check(abi.sf_fit_refinements(_p(w), ctypes.byref(self.desc), _p(x_cal), n_cal, chunk, kch, alpha, _p(delta),
+                                     _p(ws), nbytes, _stream(stream)), "sf_fit_refinements")
+        return delta
+
     def refine_rows(self) -> torch.Tensor:
         """The refinement buffer viewed as [k][n*r/8] rows (one per input channel)."""
         return self.refine.view(self.k, self.n * self.r // 8)

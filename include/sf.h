@@ -133,6 +133,33 @@ SF_API sf_status sf_pack_nested(const float* w, const sf_wq* out, sf_stream_t st
  * byte).  rho may be NULL (or out->refine NULL: rho is then not written). */
 SF_API sf_status sf_unpack_codes(const sf_wq* w, uint8_t* qb, uint8_t* rho, sf_stream_t stream);
 
+/* Fitted refinement values ([EXPL] "nested quantization": for weights the
+ * refinement values are fitted on a small calibration set, so that the
+ * channels a step refines partly make up for the error of the channels it
+ * leaves at base precision).  Rewrites w->refine of a matrix that
+ * sf_pack_nested(wf, w) packed; the base codes, steps and offsets stay.
+ *   wf    [n][k] fp32 device: the full-precision weights w was packed from;
+ *   x_cal [n_cal][k] fp16 device: calibration activations (16-byte aligned);
+ *   chunk, kch: the channel selection the decode step uses (as
+ *         sf_select_channels), applied to every calibration row;
+ *   alpha > 0: ridge weight;
+ *   delta (nullable) [n][k] fp64 device: receives the fitted corrections d.
+ * Per chunk J of input channels, with A = x_cal masked to each row's selected
+ * channels and e = wf minus the base value (m + s q):
+ *   G = A_J^T A_J,  lam = alpha * trace(G) / chunk  (1 where the trace is 0),
+ *   d_i[J] = (G + lam I)^-1 (A_J^T X_J + lam I) e_i[J],
+ * the minimiser of sum_n (X_nJ . e_iJ - A_nJ . d)^2 + lam |d - e_iJ|^2, and
+ *   rho = clamp(floor((d / s + 1/2) * 2^r), 0, 2^r - 1)  (0 where s = 0),
+ * the sub-bin of the base bin that holds base + d.  All arithmetic is fp64.
+ * ws: sf_fit_refinements_workspace_bytes(n, k, n_cal, chunk, kch) bytes,
+ * 16-byte aligned (about 16 (n + n_cal + chunk) k bytes).  A one-off
+ * preparation step: it synchronises with the stream before returning
+ * (SF_ERR_INVALID_ARG if G + lam I did not factor in fp64). */
+SF_API sf_status sf_fit_refinements(const float* wf, const sf_wq* w, const uint16_t* x_cal, int n_cal, int chunk,
+                                    int kch, double alpha, double* delta, void* ws, size_t ws_bytes,
+                                    sf_stream_t stream);
+SF_API size_t sf_fit_refinements_workspace_bytes(int n, int k, int n_cal, int chunk, int kch);
+
 /* Chunked channel selection ([EXPL] "which tiles count"): for every batch row
  * and every chunk of `chunk` input channels, the kch channels with the
  * largest fp16 magnitude |x| (bits & 0x7fff; +0 == -0), equal magnitudes to
