@@ -369,6 +369,53 @@ def gemv_config(name, shapes, b, r, seed, steps, warmup, hbm_peak, device):
     return rec
 
 
+def fit_config(device, n_cal=512, n_held=64, reps=3):
+    """Fitted refinement values (sf_fit_refinements) on the single-GEMV shape
+    (4096 x 4096, 2 + 2 bits, group 128, k = 32 per 1,024): the fit's own time
+    for n_cal calibration rows (a one-off preparation step, CUDA events around
+    the call), and the output error of the refined GEMV on n_held held-out rows
+    of the same distribution with the plain and with the fitted codes, relative
+    to the product of the unquantised weights in fp64 (the base-only error
+    beside them).  The decode kernels and their bytes do not change."""
+    import torch
+
+    from bit_decode_selective_b200 import inputs
+    from bit_decode_selective_b200.ops import QuantWeights
+
+    n = k = 4096
+    w = inputs.torch_normal((n, k), 0.02, 71, device=device)
+    xc = torch.from_numpy(inputs.calibration_activations(n_cal, k, 72).view(np.int16)).to(device)
+    xh = torch.from_numpy(inputs.calibration_activations(n_held, k, 73).view(np.int16)).to(device)
+    plain = QuantWeights.pack(w, 2, 2, 128)
+    fitted = QuantWeights.pack(w, 2, 2, 128)
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fitted.fit_refinements(w, xc, 1024, 32, 0.01)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    y_true = xh.view(torch.float16).double() @ w.double().t()
+
+    def rel_err(qw, kch):
+        ys = [qw.gemv(xh[i:i + 8], 1024, kch)[0] for i in range(0, n_held, 8)]
+        y = torch.cat(ys).double()
+        return float((y - y_true).norm() / y_true.norm())
+
+    rec = {"workload": "fitted refinement values, 4096x4096, 2-bit base + 2 refinement bits, k=32 per 1024, "
+                       f"{n_cal} calibration rows, ridge alpha 0.01",
+           "fit_ms": float(np.median(times)),
+           "rel_err_base_only": rel_err(plain, 0), "rel_err_plain_refined": rel_err(plain, 32),
+           "rel_err_fitted_refined": rel_err(fitted, 32),
+           "inputs": "calibration_activations: rank-16 factor part + N(0, 0.5) noise, 1% channels x20; "
+                     f"{n_held} held-out rows from another seed"}
+    rec["fitted_over_plain_error"] = rec["rel_err_fitted_refined"] / rec["rel_err_plain_refined"]
+    del plain, fitted, w
+    torch.cuda.empty_cache()
+    return rec
+
+
 def kv_config(name, t, k_tok, seed, steps, warmup, hbm_peak, device, b=2, r=2):
     """Configs 3 and 4 (and the 3-bit base variant): score + select + refined
     attention (sf_kv_attend_selective) over t cached tokens, 8 KV / 32 query
@@ -591,6 +638,7 @@ def run_ours(args, rank, world, local_rank):
                              8192, 256, 2, sub, args.warmup, hbm_peak, device),
         "4_kv_128k": kv_config("refined KV attention, T=131072, 2+2 bits, top-1024 per KV head, split-K + LSE merge",
                                131072, 1024, 3, sub, args.warmup, hbm_peak, device),
+        "fitted_refinements": fit_config(device),
         "kv_32k_3bit": kv_config("refined KV attention, 32/8 heads x 128, T=32768, 3-bit base + 2 refinement bits, "
                                  "top-512 per KV head (the pages' other KV base width)",
                                  32768, 512, 6, sub, args.warmup, hbm_peak, device, b=3, r=2),
