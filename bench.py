@@ -781,15 +781,15 @@ def run_case(name):
     2 + 2 bits, k = 32 per 1,024), base then refined with a given selection,
     three times; `gemv8` = the same at batch 8 (the tensor-core form), three
     times; `kv` = score-select-attend over 8 KV heads x 32,768 tokens,
-    top-512, three times; `step` = three eager decode steps of the benchmarked
-    workload (for the launch list)."""
+    top-512, three times (`kv3`: the same with a 3-bit base); `step` = three eager decode steps of the benchmarked
+    workload (for the launch list); `step8` = the same at batch 8."""
     import torch
 
     from bit_decode_selective_b200 import inputs
     from bit_decode_selective_b200.ops import KVCache, QuantWeights, select_channels
 
-    if name == "step":
-        dec, hidden = build_decoder(BATCH, T_CTX, torch.device("cuda"))
+    if name in ("step", "step8"):
+        dec, hidden = build_decoder(BATCH if name == "step" else 8, T_CTX, torch.device("cuda"))
         dec.use_cache = False  # the benchmarked schedule
         for _ in range(3):
             dec.step(hidden)
@@ -824,7 +824,7 @@ def run_case(name):
         t = 32768
         k = inputs.torch_normal((1, 8, t, 128), 1.0, 3, dtype=torch.float16)
         v = inputs.torch_normal((1, 8, t, 128), 1.0, 4, dtype=torch.float16)
-        c = KVCache(1, 8, t, 2, 2)
+        c = KVCache(1, 8, t, 3 if name == "kv3" else 2, 2)
         c.pack_tokens(k, v, 0)
         del k, v
         q = inputs.torch_normal((1, 32, 128), 1.0, 5, dtype=torch.float16)
@@ -842,7 +842,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["gemv", "gemv8", "kv", "step"], default=None,
+    ap.add_argument("--case", choices=["gemv", "gemv8", "kv", "kv3", "step", "step8"], default=None,
                     help="run a few launches of one kernel for a profiler capture instead")
     args = ap.parse_args()
     if args.case:

@@ -1245,8 +1245,15 @@ __global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
   const long hq0 = (long)bat * a.h_q + (long)g * gq;
   const long head = (long)bat * a.h_kv + g;
   pdl_trigger();
-  pdl_wait();  // the base pass is complete
-  if (warp < gq) {
+  pdl_wait();  // the base pass (and the selection, when it ran before) is complete
+  if (a.stats_given) {
+    // the statistics the scoring left in the control words (the same
+    // computation over the same records)
+    if (tid < gq) {
+      const float* st = reinterpret_cast<const float*>(a.ctl + head * kCtl + kCtlStats);
+      sh.M[tid] = __ldcg(st + 2 * tid), sh.Z[tid] = __ldcg(st + 2 * tid + 1);
+    }
+  } else if (warp < gq) {
     float M, Z;
     head_stats(a.part + (hq0 + warp) * a.nrec * kRec, a.nrec, kRec, lane, M, Z);
     if (lane == 0) sh.M[warp] = M, sh.Z[warp] = Z;
