@@ -602,6 +602,9 @@ def run_ours(args, rank, world, local_rank):
         roof = gemv_roofline(dec, max(3, args.steps // 5), max(3, args.warmup), hbm_peak)
         ms_base = base_only_ms(dec, hidden, s, max(3, args.steps // 2), args.warmup)
         ms_local = step_variant_ms(dec, hidden, s, sub, args.warmup, feed, lead=0, lag=0)
+        dec.set_rows_resident(True)
+        ms_dev = step_variant_ms(dec, hidden, s, sub, args.warmup, feed)
+        dec.set_rows_resident(False)
         dec.use_cache = True
         st0 = dec.cache_stats()
         ms_cache = step_variant_ms(dec, hidden, s, sub, args.warmup, feed)
@@ -619,8 +622,8 @@ def run_ours(args, rank, world, local_rank):
     skip_hits, skip_misses = delta(st1, c1, 0), delta(st1, c1, 1)
     miss_bytes = sum((st1[n][1] - st0.get(n, (0, 0))[1]) * dec.row_bytes[n] for n in st1)
     roof["peak_kind"] = kv_roof["peak_kind"] = lm_roof["peak_kind"] = peak_kind
-    ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache = max_over_ranks(
-        [ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache], world, device)
+    ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache, ms_dev = max_over_ranks(
+        [ms, ms_e2e, ms_base, ms_local, ms_skip, ms_cache, ms_dev], world, device)
     step_bytes = decode_step_bytes(cfg, BATCH, T_CTX)
     pcie_per_step = staged_bytes(cfg, BATCH)  # host-link bytes per step: every selected row
     io_bytes = (hidden.numel() * 2, dec.logits.numel() * 4)
@@ -681,6 +684,10 @@ def run_ours(args, rank, world, local_rank):
         "base_only": {"ms_per_step": ms_base, "refined_over_base_throughput": ms_base / ms,
                       "what": "the same step with no channel refinement (kch = 0: no selection, staging or "
                               "correction of the weights; the KV path unchanged), its own graph"},
+        "device_rows": {"ms_per_step": ms_dev, "refined_over_base_throughput": ms_base / ms_dev,
+                        "what": "the same step with the refinement rows resident on the device (each projection "
+                                "reads its selected rows from its own buffer, nothing crosses the host link; the "
+                                "selections still run a layer ahead), its own graph"},
         "projection_local": {"ms_per_step": ms_local, "lead_lag_1_vs_local": ms / ms_local - 1.0,
                              "what": "the same step with fetch lead = lag = 0 (each projection selects from its own "
                                      "input and waits for its rows): the schedule fetch lead/lag is compared with"},

@@ -204,6 +204,31 @@ class Decoder:
                 out[name] = (h, m)
         return out
 
+    def set_rows_resident(self, resident: bool):
+        """Keep the refinement rows on the device (True: every projection reads
+        its selected rows from its own refinement buffer and nothing crosses the
+        host link; the selections still run a layer ahead on the staging
+        streams) or stage them from pinned host memory again (False).  Only for
+        a decoder built with host_refine and run without the row cache."""
+        assert self.cfg.host_refine and self.cfg.kch and not self.use_cache
+        if resident and self.slots is not None:
+            self._host_slots = self.slots
+            self.slots = None
+            for L, host in zip(self.layers, self.host_rows):
+                for n in PROJ:
+                    qw = L[n]
+                    if getattr(qw, "_dev_refine", None) is None:
+                        qw._dev_refine = host[n].to(self.dev)
+                    qw.refine = qw._dev_refine
+                    qw.desc.refine = qw.refine.data_ptr()
+            torch.cuda.synchronize(self.dev)
+        elif not resident and self.slots is None:
+            self.slots = self._host_slots
+            for L in self.layers:
+                for n in PROJ:
+                    L[n].refine = None
+                    L[n].desc.refine = None
+
     def set_lm_head(self, lm_fp16: torch.Tensor):
         self.lm_head = lm_fp16.contiguous()
         kv = self.layers[0]["kv"]
