@@ -15,7 +15,7 @@ import torch
 import oracle
 from oracle import fit as ofit
 from bit_decode_selective_b200 import inputs
-from bit_decode_selective_b200.ops import QuantWeights, select_channels
+from bit_decode_selective_b200.ops import QuantWeights
 
 pytestmark = pytest.mark.gpu
 
@@ -100,3 +100,12 @@ def test_refined_gemv_with_fitted_codes():
     torch.cuda.synchronize()
     y_true = Xh.astype(np.float64) @ w.astype(np.float64).T
     assert np.linalg.norm(yg - y_true) < 0.95 * np.linalg.norm(yp.cpu().numpy() - y_true)
+
+
+def test_fit_benchmarked_shape():
+    # the benchmarked fit: 4096 x 4096, 2+2 bits, group 128, 512 calibration
+    # rows, k = 32 per 1,024 -- every correction and every code
+    w, qb, rho, sz, qw, rho_o, D_o, D_g, rho_g = fit_both(4096, 4096, 2, 2, 128, 512, 1024, 32, 70)
+    E = w.astype(np.float64) - oracle.dequant_weights(qb, np.zeros_like(qb), sz, 2, 128)
+    assert np.abs(D_g - D_o).max() <= D_TOL * np.abs(E).max()
+    check_codes(rho_o, rho_g, D_o, sz, 2, 128)

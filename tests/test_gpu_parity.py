@@ -407,6 +407,11 @@ def test_kv_attention_128k_workload():
     kv_parity(131072, 1024, splits=(0,), seed=3)
 
 
+def test_kv_attention_3bit_32k_workload():
+    """The benchmarked 3-bit base: T = 32,768, 3+2 bits, top-512 tokens per KV head."""
+    kv_parity(32768, 512, splits=(0,), b=3, r=2, seed=6)
+
+
 # ---------------------------------------------------------------------------
 # decoder glue
 
