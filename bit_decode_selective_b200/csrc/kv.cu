@@ -1237,8 +1237,11 @@ __device__ __forceinline__ void stash_warp(float (&an)[GQP][4], float ad_own, in
 
 // kv_refine_kernel (a selection given): kRefParts CTAs per head, each a share
 // of the selected tokens and of the split records; the head's last CTA merges.
-template <int GQP, int B, int R>
-__global__ void __launch_bounds__(kRefThreads) kv_refine_kernel(RefArgs a) {
+// MINB = 2 holds the registers to two CTAs per SM (for grids of more than one
+// wave, e.g. 8 caches at once; a few spills), MINB = 1 lets one CTA take what it
+// needs (no spills).
+template <int GQP, int B, int R, int MINB>
+__global__ void __launch_bounds__(kRefThreads, MINB) kv_refine_kernel(RefArgs a) {
   __shared__ RefShared<GQP> sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int part = blockIdx.x, g = blockIdx.y, bat = blockIdx.z, gq = a.gq;
@@ -1413,11 +1416,11 @@ sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& 
   return SF_OK;
 }
 
-template <int GQP>
+template <int GQP, int MINB>
 void (*refine_kernel_for(int b, int r))(RefArgs) {
-  if (b == 2) return r == 2 ? kv_refine_kernel<GQP, 2, 2> : kv_refine_kernel<GQP, 2, 1>;
-  if (b == 3) return r == 2 ? kv_refine_kernel<GQP, 3, 2> : kv_refine_kernel<GQP, 3, 1>;
-  return r == 2 ? kv_refine_kernel<GQP, 4, 2> : kv_refine_kernel<GQP, 4, 1>;
+  if (b == 2) return r == 2 ? kv_refine_kernel<GQP, 2, 2, MINB> : kv_refine_kernel<GQP, 2, 1, MINB>;
+  if (b == 3) return r == 2 ? kv_refine_kernel<GQP, 3, 2, MINB> : kv_refine_kernel<GQP, 3, 1, MINB>;
+  return r == 2 ? kv_refine_kernel<GQP, 4, 2, MINB> : kv_refine_kernel<GQP, 4, 1, MINB>;
 }
 
 // Refinement of the selected tokens and the merge (programmatic serialization).
@@ -1435,8 +1438,11 @@ sf_status launch_refine(const sf_kv* kv, int t, const uint16_t* q, int h_q, int 
   a.stats_given = stats_given;
   a.out = out, a.out16 = out16;
   a.scale = 1.0f / sqrtf((float)kD);
-  void (*kern)(RefArgs) = refine_kernel_for<4>(kv->b, kv->r);
-  if (a.gq > 4) kern = refine_kernel_for<8>(kv->b, kv->r);
+  // two CTAs per SM when the grid is more than one wave of one CTA per SM
+  const bool two = (long)P.parts * kv->h_kv * kv->batch > num_sms();
+  void (*kern)(RefArgs);
+  if (a.gq <= 4) kern = two ? refine_kernel_for<4, 2>(kv->b, kv->r) : refine_kernel_for<4, 1>(kv->b, kv->r);
+  else kern = two ? refine_kernel_for<8, 2>(kv->b, kv->r) : refine_kernel_for<8, 1>(kv->b, kv->r);
   SF_CUDA(launch_pdl(kern, dim3(P.parts, kv->h_kv, kv->batch), dim3(kRefThreads), 0, s, a));
   return SF_OK;
 }

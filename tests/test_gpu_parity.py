@@ -326,6 +326,8 @@ def test_kv_parity_batch_and_head_groups():
     kv_parity(777, 50, splits=(0, 3), batch=2, h_kv=4, h_q=32, seed=9)   # 8 query heads per KV head
     kv_parity(500, 20, splits=(0,), b=4, r=1, h_kv=2, h_q=4, seed=10)    # 2 per KV head, 4-bit base
     kv_parity(300, 30, splits=(0, 5), h_kv=4, h_q=4, seed=12)            # 1 per KV head
+    # 3 caches x 8 heads x 16 refinement CTAs: more than one wave, two CTAs per SM
+    kv_parity(2000, 512, splits=(0,), batch=3, h_kv=8, h_q=32, seed=13)
 
 
 @pytest.mark.parametrize("T,k_tok,r,batch,h_kv,h_q,seed", [
