@@ -1311,7 +1311,9 @@ Plan make_plan(const sf_kv* kv, int t, int h_q, int k_tok, bool need_logits, boo
   Plan P;
   const int sms = num_sms();
   const int heads = kv->batch * kv->h_kv;
-  int ns = n_splits > 0 ? n_splits : (16 * sms + heads - 1) / heads;
+  // splits per head: whole CTAs of kWarps splits, all (batch, head) CTAs in one
+  // wave of 4 CTAs per SM (e.g. 296 for 8 heads, 36 for 64)
+  int ns = n_splits > 0 ? n_splits : kWarps * std::max(1, 4 * sms / heads);
   int maxs = (t + 15) / 16;
   if (ns > maxs) ns = maxs;
   if (ns < 1) ns = 1;
