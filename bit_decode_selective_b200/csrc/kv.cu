@@ -594,6 +594,7 @@ __global__ void __maxnreg__(GQP == 4 ? 120 : 255) kv_base_kernel(BaseArgs a) {
 // denominators.
 
 constexpr int kSelThreads = 512;
+constexpr size_t kSpreadSmem = 120 * 1024;  // more than half an SM's shared memory
 constexpr int kSelTok = 2048;        // tokens scored per CTA
 constexpr int kBins1 = 2048;         // first digit: key bits 30..20
 constexpr int kBins2 = 1024;         // then bits 19..10 and 9..0
@@ -1412,7 +1413,13 @@ sf_status launch_select(const sf_kv* kv, int t, int h_q, int k_tok, const Plan& 
   a.scores = (float*)(ws + P.off_scores), a.scores_out = scores_out, a.ctl = ctl, a.sel = sel;
   a.bitmap = (uint32_t*)(ws + P.off_bitmap), a.cand = (uint2*)(ws + P.off_cand);
   const dim3 grid(P.sel_blocks, kv->h_kv, kv->batch);
-  SF_CUDA(launch_pdl(a.gq <= 4 ? kv_score_kernel<4> : kv_score_kernel<8>, grid, dim3(kSelThreads), 0, s, a));
+  // a grid of at most one CTA per SM is spread over the SMs: the CTA reserves
+  // shared memory enough that no second one fits beside it (the scoring of a
+  // head's tokens is latency-bound; two CTAs on one SM would share its load path)
+  auto score = a.gq <= 4 ? kv_score_kernel<4> : kv_score_kernel<8>;
+  const size_t spread = (long)grid.x * grid.y * grid.z <= num_sms() ? kSpreadSmem : 0;
+  if (spread) SF_CUDA(cudaFuncSetAttribute(score, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)spread));
+  SF_CUDA(launch_pdl(score, grid, dim3(kSelThreads), spread, s, a));
   SF_CUDA(cudaFuncSetAttribute(kv_pick_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDyn));
   SF_CUDA(launch_pdl(kv_pick_kernel, grid, dim3(kSelThreads), kSelDyn, s, a));
   return SF_OK;
