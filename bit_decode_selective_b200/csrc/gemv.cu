@@ -1124,26 +1124,27 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
       }
     }
   };
-  auto word_of = [&](int j, int c) {
-    const size_t row = a.staged ? (size_t)b * a.n_sel + j : (size_t)c;
-    return __ldg(a.refine + row * a.row_words + wi) >> sh;
-  };
-  // entry j: channel and activation (-1 - c: selected, not refined now: x = 0)
-  auto chan = [&](int j) {
+  // entry j: channel, activation (-1 - c: selected, not refined now: x = 0)
+  // and the rows' refinement word, from one load of the selection
+  auto entry = [&](int j, int& c, float& xc, uint32_t& w) {
     const int raw = __ldg(sel + j);
-    return min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
+    c = min(max(raw < 0 ? -1 - raw : raw, 0), a.K - 1);
+    xc = raw < 0 ? 0.f : h2f(__ldg(xb + c));
+    const size_t row = a.staged ? (size_t)b * a.n_sel + j : (size_t)c;
+    w = __ldg(a.refine + row * a.row_words + wi) >> sh;
   };
-  auto act = [&](int j, int c) { return __ldg(sel + j) < 0 ? 0.f : h2f(__ldg(xb + c)); };
   // the lane's share [j0, j1); channel j + 1's index, activation and word are
   // loaded while j is summed
   const int j0 = lane * a.n_sel / 32, j1 = (lane + 1) * a.n_sel / 32;
-  int c = j0 < j1 ? chan(j0) : 0;
-  float xc = j0 < j1 ? act(j0, c) : 0.f;
-  uint32_t w = j0 < j1 ? word_of(j0, c) : 0u;
+  int c = 0;
+  float xc = 0.f;
+  uint32_t w = 0u;
+  if (j0 < j1) entry(j0, c, xc, w);
   for (int j = j0; j < j1; j++) {
-    const int cn = j + 1 < j1 ? chan(j + 1) : 0;
-    const float xn = j + 1 < j1 ? act(j + 1, cn) : 0.f;
-    const uint32_t wn = j + 1 < j1 ? word_of(j + 1, cn) : 0u;
+    int cn = 0;
+    float xn = 0.f;
+    uint32_t wn = 0u;
+    if (j + 1 < j1) entry(j + 1, cn, xn, wn);
     const int g = c >> a.gshift;
     if (g != gcur) {
       flush();
@@ -1159,18 +1160,25 @@ __global__ void __maxnreg__(64) corr_only_kernel(CorrArgs a) {
     c = cn, xc = xn, w = wn;
   }
   flush();
+  // the 8 rows' sums over the warp, reduced and scattered at once: each round
+  // keeps the half of the rows that the lane's bit selects and adds the
+  // partner's copy; lane l ends with row (l >> 2) & 7 (a fixed order)
+  static_assert(kCorrRows == 8, "the reduction below is written for 8 rows");
 #pragma unroll
-  for (int t = 0; t < kCorrRows; t++)
+  for (int n = 8, o = 16; n > 1; n >>= 1, o >>= 1) {
+    const bool up = lane & o;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-  if (lane != 0) return;
-  float4* yv = reinterpret_cast<float4*>(a.y + (size_t)b * a.N + row0);
-#pragma unroll
-  for (int q = 0; q < kCorrRows / 4; q++) {
-    float4 v = a.overwrite ? make_float4(0.f, 0.f, 0.f, 0.f) : yv[q];
-    v.x += acc[4 * q], v.y += acc[4 * q + 1], v.z += acc[4 * q + 2], v.w += acc[4 * q + 3];
-    yv[q] = v;
+    for (int t = 0; t < n / 2; t++) {
+      const float keep = up ? acc[t + n / 2] : acc[t], send = up ? acc[t] : acc[t + n / 2];
+      acc[t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
   }
+  float v = acc[0];
+  v += __shfl_xor_sync(0xffffffffu, v, 2);
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  if ((lane & 3) != 0) return;
+  float* yr = a.y + (size_t)b * a.N + row0 + ((lane >> 2) & 7);
+  *yr = a.overwrite ? v : *yr + v;
 }
 
 // ---------------------------------------------------------------------------
