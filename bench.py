@@ -788,7 +788,9 @@ def run_case(name):
     2 + 2 bits, k = 32 per 1,024), base then refined with a given selection,
     three times; `gemv8` = the same at batch 8 (the tensor-core form), three
     times; `kv` = score-select-attend over 8 KV heads x 32,768 tokens,
-    top-512, three times (`kv3`: the same with a 3-bit base); `step` = three eager decode steps of the benchmarked
+    top-512, three times (`kv3`: the same with a 3-bit base); `kvfma` = the
+    base logits there in the tensor-core and the CUDA-core form, timed, then
+    three launches of each; `step` = three eager decode steps of the benchmarked
     workload (for the launch list); `step8` = the same at batch 8."""
     import torch
 
@@ -802,6 +804,47 @@ def run_case(name):
             dec.step(hidden)
         torch.cuda.synchronize()
         print(json.dumps({"case": name, "ok": True}), flush=True)
+        return
+    if name == "kvfma":
+        # the base logits of 8 KV heads x 32,768 tokens, 32 query heads: the
+        # tensor-core form (kv_base_kernel without values, inside
+        # sf_kv_score_select, top-1) and the CUDA-core form (sf_kv_logits_fma),
+        # each timed with CUDA events over 32 rotating caches (keys 400 MB), then
+        # three more launches of each for a profiler
+        t, copies = 32768, 32
+        k = inputs.torch_normal((1, 8, t, 128), 1.0, 3, dtype=torch.float16)
+        v = inputs.torch_normal((1, 8, t, 128), 1.0, 4, dtype=torch.float16)
+        caches = []
+        for _ in range(copies):
+            c = KVCache(1, 8, t, 2, 2)
+            c.pack_tokens(k, v, 0)
+            caches.append(c)
+        del k, v
+        q = inputs.torch_normal((1, 32, 128), 1.0, 5, dtype=torch.float16)
+        lg = torch.empty(1, 32, t, device="cuda")
+        sel = torch.empty(1, 8, 1, dtype=torch.int32, device="cuda")
+        ws = torch.empty(max(caches[0].score_select_workspace(t, 32, 1, True), 16), dtype=torch.uint8,
+                         device="cuda")
+        forms = {"tensor_cores": lambda c: c.score_select(q, t, 1, logits=lg, sel=sel, ws=ws),
+                 "cuda_cores": lambda c: c.logits_fma(q, t, logits=lg, ws=ws)}
+        res = {"case": name, "ok": True}
+        for fname, fn in forms.items():
+            for c in caches[:4]:
+                fn(c)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(3):
+                for c in caches:
+                    fn(c)
+            e1.record()
+            torch.cuda.synchronize()
+            res[fname + "_us_per_call"] = e0.elapsed_time(e1) * 1e3 / (3 * copies)
+        for _ in range(3):
+            for fn in forms.values():
+                fn(caches[0])
+        torch.cuda.synchronize()
+        print(json.dumps(res), flush=True)
         return
     if name == "gemv8":
         # the batch-8 form: tensor-core base products (two launches of four
@@ -849,7 +892,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["gemv", "gemv8", "kv", "kv3", "step", "step8"], default=None,
+    ap.add_argument("--case", choices=["gemv", "gemv8", "kv", "kv3", "kvfma", "step", "step8"], default=None,
                     help="run a few launches of one kernel for a profiler capture instead")
     args = ap.parse_args()
     if args.case:

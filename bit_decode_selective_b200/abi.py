@@ -69,6 +69,8 @@ _SIGNATURES = {
     "sf_kv_score_select": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_int, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_kv_score_select_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
+    "sf_kv_logits_fma": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p], c_int),
+    "sf_kv_logits_fma_workspace_bytes": ([POINTER(sf_kv), c_int, c_int], c_size_t),
     "sf_kv_attn_refined": ([POINTER(sf_kv), c_int, c_void_p, c_int, c_void_p, c_int, c_int,
                             c_void_p, c_void_p, c_size_t, c_void_p], c_int),
     "sf_kv_attn_workspace_bytes": ([POINTER(sf_kv), c_int, c_int, c_int, c_int], c_size_t),
@@ -153,6 +155,8 @@ sf_kv_unpack_codes = _call("sf_kv_unpack_codes")
 sf_kv_append_rope = _call("sf_kv_append_rope")
 sf_kv_score_select = _call("sf_kv_score_select")
 sf_kv_score_select_workspace_bytes = _call("sf_kv_score_select_workspace_bytes")
+sf_kv_logits_fma = _call("sf_kv_logits_fma")
+sf_kv_logits_fma_workspace_bytes = _call("sf_kv_logits_fma_workspace_bytes")
 sf_kv_attn_refined = _call("sf_kv_attn_refined")
 sf_kv_attn_workspace_bytes = _call("sf_kv_attn_workspace_bytes")
 sf_kv_attend_selective = _call("sf_kv_attend_selective")

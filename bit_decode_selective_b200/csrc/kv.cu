@@ -1365,6 +1365,121 @@ sf_status check_ktok(int k_tok, int t, bool allow_zero) {
   return SF_OK;
 }
 
+// kv_logits_fma_kernel -- the base pass without values on the CUDA cores: the
+// same logits and per-CTA (max, sum) records as kv_base_kernel<4, 2, false>,
+// with the key contraction done by fp32 FMAs (a lane per token, up to 4 query
+// heads) instead of mma.sync.  Kept to measure the two against each other
+// (2-bit keys).  The query heads sit in shared memory in the order of the code
+// stream (qs[code][head]: one 16-byte load gives a code's 4 heads); code k of
+// a token's key word w (bit 2k) is dim 16 s + 2 c + 8 e + (k >= 8) with
+// c = w / 2, pair p = 8 (w % 2) + k % 8 = 2 s + e, in scale group s / 2.
+__global__ void __launch_bounds__(kWarps * 32) kv_logits_fma_kernel(BaseArgs a) {
+  __shared__ __align__(16) float qs[kD][4];
+  __shared__ float Qg[4][4];              // [head][group]: sum of q over the group
+  __shared__ float wr[kWarps][4][2];      // warp records: (max, sum) per head
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.y, bat = blockIdx.z, gq = a.gq;
+  const uint16_t* qg = a.q + ((long)bat * a.h_q + (long)g * gq) * kD;
+  for (int e = threadIdx.x; e < 4 * kD; e += blockDim.x) {
+    const int h = e / kD, d = e % kD;
+    int word, bit;
+    key_pos(d, 2, word, bit);
+    qs[word * 16 + bit / 2][h] = h < gq ? h2f(qg[h * kD + d]) : 0.f;
+  }
+  if (threadIdx.x < 16) {
+    const int h = threadIdx.x >> 2, j = threadIdx.x & 3;
+    float v = 0.f;
+    for (int d = 32 * j; d < 32 * j + 32; d++) v += h < gq ? h2f(qg[h * kD + d]) : 0.f;
+    Qg[h][j] = v;
+  }
+  __syncthreads();
+  const int split = blockIdx.x * kWarps + warp;
+  const int tw0 = split * a.span, tw1 = split < a.nsplit ? min(a.T, tw0 + a.span) : tw0;
+  const long slot0 = ((long)bat * a.h_kv + g) * a.t_max;
+  float mrun[4], lsum[4];
+#pragma unroll
+  for (int h = 0; h < 4; h++) mrun[h] = -INFINITY, lsum[h] = 0.f;
+  float* lg = a.logits + ((long)bat * a.h_q + (long)g * gq) * a.T;
+  for (int tb = tw0; tb < tw1; tb += 32) {
+    const int t = tb + lane;
+    const bool ok = t < tw1;
+    uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0, zz = c0;
+    if (ok) {
+      const uint4* kp = reinterpret_cast<const uint4*>(a.kb + (slot0 + t) * 32);
+      c0 = __ldg(kp), c1 = __ldg(kp + 1);
+      zz = __ldg(reinterpret_cast<const uint4*>(a.ksz) + (slot0 + t));
+    }
+    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float acc[4][4];  // [head][group]
+#pragma unroll
+    for (int h = 0; h < 4; h++)
+#pragma unroll
+      for (int j = 0; j < 4; j++) acc[h][j] = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < 8; wi++)
+#pragma unroll
+      for (int k = 0; k < 16; k++) {
+        const int grp = (wi & 1) * 2 + (k & 7) / 4;
+        const float c = (float)((w[wi] >> (2 * k)) & 3u);
+        const float4 qv = *reinterpret_cast<const float4*>(&qs[wi * 16 + k][0]);
+        acc[0][grp] = fmaf(qv.x, c, acc[0][grp]);
+        acc[1][grp] = fmaf(qv.y, c, acc[1][grp]);
+        acc[2][grp] = fmaf(qv.z, c, acc[2][grp]);
+        acc[3][grp] = fmaf(qv.w, c, acc[3][grp]);
+      }
+    // (s, m') per group, m' = m + 1.5 s: the codes enter uncentred, so the
+    // offset term is m, not m'
+    const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+    float l[4];
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+      float x = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(&zw[j]));
+        x = fmaf(sm.x, acc[h][j], fmaf(sm.y, Qg[h][j], x));
+      }
+      l[h] = ok && h < gq ? x * a.scale : -INFINITY;
+      if (ok && h < gq) lg[(long)h * a.T + t] = l[h];
+    }
+    // online softmax over the warp's tokens, one warp-wide max per chunk
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+      float mx = l[h];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (mx > -INFINITY) {
+        const float mn = fmaxf(mrun[h], mx);
+        lsum[h] = lsum[h] * __expf(mrun[h] - mn) + (l[h] > -INFINITY ? __expf(l[h] - mn) : 0.f);
+        mrun[h] = mn;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 4; h++) {
+    float v = lsum[h];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) wr[warp][h][0] = mrun[h], wr[warp][h][1] = v;
+  }
+  __syncthreads();
+  const long hq0 = (long)bat * a.h_q + (long)g * gq;
+  if (threadIdx.x < gq) {
+    const int h = threadIdx.x;
+    float M = -INFINITY, L = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < kWarps; w2++) M = fmaxf(M, wr[w2][h][0]);
+    if (M > -INFINITY)
+#pragma unroll
+      for (int w2 = 0; w2 < kWarps; w2++)
+        if (wr[w2][h][0] > -INFINITY) L = fmaf(__expf(wr[w2][h][0] - M), wr[w2][h][1], L);
+    a.part[((hq0 + h) * a.nrec + blockIdx.x) * 2 + 0] = M;
+    a.part[((hq0 + h) * a.nrec + blockIdx.x) * 2 + 1] = L;
+  }
+}
+
 template <int GQP, int B, bool PV>
 sf_status launch_base_t(const BaseArgs& a, int batch, cudaStream_t s) {
   const size_t smem = kWarps * WarpSmem<B, PV>::bytes;
@@ -1500,6 +1615,29 @@ extern "C" sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* 
   st = launch_base(kv, a, false, s);
   if (st != SF_OK) return st;
   return launch_select(kv, t, h_q, k_tok, P, lg, part, 2, w, scores, ctl, sel, s);
+}
+
+extern "C" size_t sf_kv_logits_fma_workspace_bytes(const sf_kv* kv, int t, int h_q) {
+  if (!kv || t <= 0 || h_q <= 0) return 0;
+  return make_plan(kv, t, h_q, 0, false, false, false, false, 0).total;
+}
+
+extern "C" sf_status sf_kv_logits_fma(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* logits,
+                                      void* ws, size_t ws_bytes, sf_stream_t stream) {
+  sf_status st = check_kv(kv);
+  if (st != SF_OK) return st;
+  st = check_q(kv, t, q, h_q);
+  if (st != SF_OK) return st;
+  SF_UNSUPPORTED(kv->b == 2 && h_q / kv->h_kv <= 4, "the CUDA-core form takes 2-bit keys and <= 4 query heads per KV head");
+  SF_REQUIRE(logits && aligned16(logits), "logits must be a non-null 16-byte aligned device pointer");
+  Plan P = make_plan(kv, t, h_q, 0, false, false, false, false, 0);
+  st = check_ws(ws, ws_bytes, P.total);
+  if (st != SF_OK) return st;
+  char* w = (char*)ws;
+  BaseArgs a = base_args(kv, t, q, h_q, logits, (float*)(w + P.off_part), nullptr, P);
+  SF_CUDA(launch_pdl(kv_logits_fma_kernel, dim3((a.nsplit + kWarps - 1) / kWarps, a.h_kv, kv->batch),
+                     dim3(kWarps * 32), 0, as_stream(stream), a));
+  return SF_OK;
 }
 
 extern "C" size_t sf_kv_attn_workspace_bytes(const sf_kv* kv, int t, int h_q, int k_tok,

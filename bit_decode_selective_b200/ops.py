@@ -179,6 +179,19 @@ class KVCache:
               "sf_kv_score_select")
         return sel, logits, scores
 
+    def logits_fma(self, q: torch.Tensor, t: int, logits=None, ws=None, stream=None):
+        """The base logits on the CUDA cores (sf_kv_logits_fma): [batch][h_q][t] fp32."""
+        q = _f16(q)
+        h_q = q.shape[1]
+        if logits is None:
+            logits = torch.empty((self.batch, h_q, t), dtype=torch.float32, device=q.device)
+        need = abi.sf_kv_logits_fma_workspace_bytes(ctypes.byref(self.desc), t, h_q)
+        if ws is None:
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        check(abi.sf_kv_logits_fma(ctypes.byref(self.desc), t, _p(q), h_q, _p(logits), _p(ws), ws.numel(),
+                                   _stream(stream)), "sf_kv_logits_fma")
+        return logits
+
     def attn_workspace(self, t: int, h_q: int, k_tok: int, n_splits: int = 0) -> int:
         return abi.sf_kv_attn_workspace_bytes(ctypes.byref(self.desc), t, h_q, k_tok, n_splits)
 

@@ -299,6 +299,17 @@ SF_API sf_status sf_kv_unpack_codes(const sf_kv* kv, int which, int t, uint8_t* 
  *   h_q % h_kv == 0, h_q / h_kv <= 8 (SF_ERR_UNSUPPORTED above the caps: the
  *   CTA that finishes a head's selection keeps a bitmap of the head's tokens
  *   in shared memory). */
+/* The base logits of sf_kv_score_select computed on the CUDA cores (fp32 FMAs,
+ * a thread per token) instead of the tensor cores, kept to compare the two
+ * forms of the key contraction ([EXPL] "which tiles count": the scores come
+ * from the resident low-bit keys).  logits [batch][h_q][t] fp32, as
+ * sf_kv_score_select writes them; 2-bit keys and h_q / h_kv <= 4 only
+ * (SF_ERR_UNSUPPORTED otherwise).  ws: sf_kv_logits_fma_workspace_bytes(kv, t,
+ * h_q) bytes, 16-byte aligned (the per-split softmax records). */
+SF_API sf_status sf_kv_logits_fma(const sf_kv* kv, int t, const uint16_t* q, int h_q, float* logits, void* ws,
+                                  size_t ws_bytes, sf_stream_t stream);
+SF_API size_t sf_kv_logits_fma_workspace_bytes(const sf_kv* kv, int t, int h_q);
+
 SF_API sf_status sf_kv_score_select(const sf_kv* kv, int t, const uint16_t* q, int h_q, int k_tok,
                              int32_t* sel, float* logits, float* scores, void* ws,
                              size_t ws_bytes, sf_stream_t stream);

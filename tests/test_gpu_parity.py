@@ -339,6 +339,20 @@ def test_kv_parity_3bit_base(T, k_tok, r, batch, h_kv, h_q, seed):
     kv_parity(T, k_tok, splits=(0, 3), b=3, r=r, batch=batch, h_kv=h_kv, h_q=h_q, seed=seed)
 
 
+@pytest.mark.parametrize("T,batch,h_kv,h_q", [(37, 1, 8, 32), (2049, 2, 4, 16), (32768, 1, 8, 32)])
+def test_kv_logits_cuda_core_form(T, batch, h_kv, h_q):
+    # the CUDA-core form of the key contraction: the oracle's logits, and the
+    # tensor-core form's within fp32 summation order
+    cache, kc, vc, q = kv_setup(T, 2, 2, batch=batch, h_kv=h_kv, h_q=h_q, seed=14)
+    qd = cu(f16bits(q))
+    lf = cache.logits_fma(qd, T)
+    _, lt, _ = cache.score_select(qd, T, 1)
+    torch.cuda.synchronize()
+    lo = oracle.kv_logits(kc[0], kc[2], q)
+    assert rel_l2(host(lf), lo) < 1e-5
+    assert np.abs(host(lf) - host(lt)).max() <= 1e-4 * np.abs(lo).max()
+
+
 def test_kv_base_only_and_all_selected():
     cache, kc, vc, q = kv_setup(300, batch=1, h_kv=8, h_q=32, seed=11)
     qd = cu(f16bits(q))
