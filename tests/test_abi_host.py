@@ -162,3 +162,37 @@ def test_decode_step_forms_reject_before_launch(L):
         == abi.SF_ERR_INVALID_ARG
     assert abi.sf_gemv_correction(ctypes.byref(wq), p16, 1, 1024, 32, p16, None, None, None) \
         == abi.SF_ERR_INVALID_ARG
+
+
+def test_fit_refinements_checks(L):
+    # every refusal happens on the host, before any launch
+    p16 = ctypes.c_void_p(16)
+    wq = abi.sf_wq(4096, 4096, 2, 2, 128, 16, 16, 16)
+    need = abi.sf_fit_refinements_workspace_bytes(4096, 4096, 512, 1024, 32)
+    assert need > 2 * 4096 * 4096 * 8  # the base errors and the fitted corrections, fp64
+    assert abi.sf_fit_refinements_workspace_bytes(4096, 4096, 0, 1024, 32) == 0
+    fit = lambda **kw: abi.sf_fit_refinements(
+        kw.get("wf", p16), ctypes.byref(kw.get("wq", wq)), kw.get("x", p16), kw.get("n_cal", 512),
+        kw.get("chunk", 1024), kw.get("kch", 32), ctypes.c_double(kw.get("alpha", 0.01)), None,
+        kw.get("ws", p16), kw.get("ws_bytes", need), None)
+    assert fit(alpha=0.0) == abi.SF_ERR_INVALID_ARG
+    assert fit(alpha=float("nan")) == abi.SF_ERR_INVALID_ARG
+    assert fit(n_cal=0) == abi.SF_ERR_INVALID_ARG
+    assert fit(wf=None) == abi.SF_ERR_INVALID_ARG
+    assert fit(chunk=1000) == abi.SF_ERR_UNSUPPORTED
+    assert fit(kch=0) == abi.SF_ERR_INVALID_ARG
+    assert fit(ws_bytes=need - 1) == abi.SF_ERR_WORKSPACE
+    assert fit(wq=abi.sf_wq(4096, 4096, 2, 2, 128, 16, None, 16)) == abi.SF_ERR_INVALID_ARG  # no refine buffer
+
+
+def test_logits_cuda_core_form_refusals(L):
+    p16 = ctypes.c_void_p(16)
+    kv2 = abi.sf_kv(1, 8, 128, 8192, 2, 2, 32, 16, 16, 16, 16, 16, 16)
+    kv3 = abi.sf_kv(1, 8, 128, 8192, 3, 2, 32, 16, 16, 16, 16, 16, 16)
+    need = abi.sf_kv_logits_fma_workspace_bytes(ctypes.byref(kv2), 4096, 32)
+    assert need > 0
+    # 3-bit keys and groups of 8 query heads are outside the comparison form
+    assert abi.sf_kv_logits_fma(ctypes.byref(kv3), 4096, p16, 32, p16, p16, need, None) == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_logits_fma(ctypes.byref(kv2), 4096, p16, 64, p16, p16, need, None) == abi.SF_ERR_UNSUPPORTED
+    assert abi.sf_kv_logits_fma(ctypes.byref(kv2), 4096, p16, 32, None, p16, need, None) == abi.SF_ERR_INVALID_ARG
+    assert abi.sf_kv_logits_fma(ctypes.byref(kv2), 4096, p16, 32, p16, p16, need - 1, None) == abi.SF_ERR_WORKSPACE
